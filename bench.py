@@ -1,0 +1,465 @@
+#!/usr/bin/env python
+"""INT2 KV-cache decode benchmark at 100K context on B200.
+
+Workload (default): 4 sequences, 32 query heads / 8 KV heads, head_dim 128,
+context 100000 tokens in 16-token blocks with a shuffled block table, 128-token
+fp16 window, INT2 groups of 128.  One step appends one new K/V token per
+sequence through the rotate-quantise kernel and runs decode attention (query
+rotation, split-K attention, split combine with the value un-rotation).
+
+Timed region: a CUDA graph replaying K steps, bracketed by CUDA events with a
+synchronize (and a barrier under torchrun) on both sides.  The cache read each
+step (232 MB) is larger than L2 (126 MB), so L2 is not flushed.  value =
+tokens decoded per second over all ranks (B * K * N / max-over-ranks time).
+
+`--impl reference` times the CPU oracle on a bounded sample of the same
+workload instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "INT2-KV decode attn achieved HBM GB/s & tokens/s at 100K ctx; append Mtok/s"
+PROFILES = os.path.join(ROOT, "profiles")
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=64)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+# ----------------------------------------------------------------- plumbing
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+class Clocks:
+    """nvidia-smi sampler for the timed region."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.file = None
+
+    def start(self):
+        try:
+            self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.QUERY}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.file, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.file.flush()
+        self.file.seek(0)
+        rows = [r.split(",") for r in self.file.read().strip().splitlines() if r.strip()]
+        os.unlink(self.file.name)
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            try:
+                sm.append(float(r[1]))
+                mx = max(mx, float(r[2]))
+                for n, v in zip(names, r[5:9]):
+                    if v.strip().lower() == "active":
+                        reasons.add(n)
+            except (ValueError, IndexError):
+                continue
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def measured_peak_hbm():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for name in ("decode.cu", "okv_common.cuh"):
+        with open(os.path.join(ROOT, "int2_kv_cache_rotate_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic():
+    """DRAM bytes per decode launch from the last ncu capture, if the kernel is unchanged."""
+    try:
+        with open(os.path.join(PROFILES, "decode_traffic.json")) as f:
+            rec = json.load(f)
+        if rec.get("source_hash") == kernel_source_hash():
+            return rec
+    except Exception:
+        pass
+    return None
+
+
+# ------------------------------------------------------------------ workload
+
+def workload_config():
+    from int2_kv_cache_rotate_b200 import workloads as WL
+    return WL.config(2)
+
+
+def algorithmic_bytes(lens, hkv):
+    """Cache bytes decode must read: 72 B per INT2 token-head (K and V codes,
+    scales, mins), 512 B per fp16 window token-head (K and V)."""
+    tot = 0
+    for L in lens:
+        n_int2 = max(0, L - 128)
+        n_win = min(L, 128)
+        tot += hkv * (n_int2 * 72 + n_win * 512)
+    return tot
+
+
+def build_gpu_workload(seed, rank, total_steps, torch, okv, WL):
+    wl = workload_config()
+    B, hq, hkv = wl.batch, wl.hq, wl.hkv
+    L0 = wl.ctx[0]
+    cfg = 2
+    qc, kc, vc = WL.calibration_set(seed, cfg, 0, hq, hkv, n=1024)
+    rot = okv.calibrate_rotations(qc, kc, vc, hq, hkv)
+    table, num_blocks = WL.block_table(seed + rank, cfg, [L0] * B, extra_tokens=total_steps + 16)
+    cache = okv.Cache(hq, hkv, num_blocks, B, table.shape[1], rot["U_K"], rot["U_V"])
+    dev = torch.device("cuda")
+    table_d = torch.from_numpy(table).to(dev)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(1000003 * (seed + 1) + rank)
+    outl = torch.from_numpy(WL.outlier_channels(seed, cfg, 0).astype(np.int64)).to(dev)
+
+    def kv(n):
+        k = torch.randn((n, hkv, 128), generator=gen, device=dev)
+        k[:, :, outl] *= 16.0
+        v = torch.randn((n, hkv, 128), generator=gen, device=dev)
+        return k.to(torch.bfloat16), v.to(torch.bfloat16)
+
+    chunk = 8192
+    lens_d = torch.full((B,), L0, dtype=torch.int32, device=dev)
+    for b in range(B):
+        for p0 in range(0, L0, chunk):
+            n = min(chunk, L0 - p0)
+            k, v = kv(n)
+            okv.append_quantize(cache, k, v, torch.full((n,), b, dtype=torch.int32, device=dev),
+                                torch.arange(p0, p0 + n, dtype=torch.int32, device=dev), table_d, lens_d)
+    torch.cuda.synchronize()
+    assert cache.device_status() == 0, cache.device_status()
+    # per-step inputs
+    S = total_steps
+    knew = torch.empty((S, B, hkv, 128), dtype=torch.bfloat16, device=dev)
+    vnew = torch.empty_like(knew)
+    for i in range(S):
+        knew[i], vnew[i] = kv(B)
+    qs = (torch.randn((S, B, hq, 128), generator=gen, device=dev)).to(torch.bfloat16)
+    pos = (L0 + torch.arange(S, dtype=torch.int32, device=dev))[:, None].repeat(1, B).contiguous()
+    lens = (pos + 1).contiguous()
+    return dict(wl=wl, cache=cache, table=table_d, knew=knew, vnew=vnew, q=qs, pos=pos, lens=lens, L0=L0,
+                seq=torch.arange(B, dtype=torch.int32, device=dev), B=B, hq=hq, hkv=hkv, gen=gen, kv=kv)
+
+
+def step(w, i, okv, out, ws, ev=None):
+    c = w["cache"]
+    okv.append_quantize(c, w["knew"][i], w["vnew"][i], w["seq"], w["pos"][i], w["table"], w["lens"][i])
+    if ev is not None:
+        okv.time_next_decode_kernel(*ev)
+    okv.decode_attention(c, w["q"][i], w["seq"], w["table"], w["lens"][i], out=out, ws=ws)
+
+
+def prefill_append_rate(torch, okv, WL, seed):
+    """Mtok/s of an 8192-token bf16 append (all 8 KV heads, K and V)."""
+    n, hkv, hq = 8192, 8, 32
+    table, nb = WL.block_table(seed, 4, [n])
+    r = np.random.default_rng(seed)
+    uk = np.stack([WL.haar_orthogonal(r) for _ in range(hkv)]).astype(np.float32)
+    cache = okv.Cache(hq, hkv, nb, 1, table.shape[1], uk, uk)
+    dev = torch.device("cuda")
+    k = torch.randn((n, hkv, 128), device=dev).to(torch.bfloat16)
+    v = torch.randn((n, hkv, 128), device=dev).to(torch.bfloat16)
+    seq = torch.zeros(n, dtype=torch.int32, device=dev)
+    pos = torch.arange(n, dtype=torch.int32, device=dev)
+    lens = torch.tensor([n], dtype=torch.int32, device=dev)
+    td = torch.from_numpy(table).to(dev)
+    for _ in range(2):
+        okv.append_quantize(cache, k, v, seq, pos, td, lens)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    reps = 5
+    e0.record()
+    for _ in range(reps):
+        okv.append_quantize(cache, k, v, seq, pos, td, lens)
+    e1.record()
+    torch.cuda.synchronize()
+    us = e0.elapsed_time(e1) * 1e3 / reps
+    bytes_moved = n * hkv * (2 * 128 * 2 + 72)
+    return {"tokens": n, "us": round(us, 2), "mtok_s": round(n / us, 3), "gbs": round(bytes_moved / us / 1e3, 1)}
+
+
+# ---------------------------------------------------------------- oracle arm
+
+def oracle_sample_setup(seed):
+    """Oracle cache for one (sequence, KV head) unit of the workload at 100K."""
+    from int2_kv_cache_rotate_b200 import workloads as WL
+    from oracle import okv_oracle as O
+    wl = workload_config()
+    L0, cfg = wl.ctx[0], 2
+    r = np.random.default_rng(np.random.SeedSequence([seed, 77]))
+    cache = O.Cache(1, WL.haar_orthogonal(r)[None], WL.haar_orthogonal(r)[None])
+    k = WL.sample_keys(seed, cfg, 0, 0, L0, extra=0)[:, None, :]
+    v = WL.sample_values(seed, cfg, 0, 0, L0, extra=0)[:, None, :]
+    cache.append(0, 0, k, v)
+    return cache, wl
+
+
+def oracle_sample_step(cache, wl, i, seed):
+    """One decode step of the sampled unit: append one token, attend with its G query heads."""
+    from int2_kv_cache_rotate_b200 import workloads as WL
+    from oracle import okv_oracle as O
+    g, L0 = wl.hq // wl.hkv, wl.ctx[0]
+    pos = L0 + i
+    kn = WL.sample_keys(seed, 2, 0, 0, 1, extra=100 + i)[:, None, :]
+    vn = WL.sample_values(seed, 2, 0, 0, 1, extra=100 + i)[:, None, :]
+    q = WL.sample_queries(seed, 2, 0, 0, 1, g, extra=100 + i)
+    t0 = time.perf_counter()
+    cache.append(0, pos, kn, vn)
+    O.decode(cache, q, [0], [pos + 1], g)
+    return time.perf_counter() - t0
+
+
+def oracle_units(wl):
+    return wl.batch * wl.hkv
+
+
+def cpu_baseline(seed, steps=3):
+    cores = len(os.sched_getaffinity(0))
+    cache, wl = oracle_sample_setup(seed)
+    ts = [oracle_sample_step(cache, wl, i, seed) for i in range(steps)]
+    step_s = statistics.median(ts) * oracle_units(wl)
+    return {"value": round(wl.batch / step_s, 5), "unit": "tok/s", "cores": cores, "kind": "oracle",
+            "sample": (f"one decode step (1-token append + attention of its {wl.hq // wl.hkv} query heads) of "
+                       f"1 of the {oracle_units(wl)} (sequence, KV head) units at {wl.ctx[0]} tokens, NumPy fp64, "
+                       f"median of {steps}; scaled x{oracle_units(wl)} to the full step")}
+
+
+def run_reference(args):
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return 0
+    wl = workload_config()
+    cores = len(os.sched_getaffinity(0))
+    cache, _ = oracle_sample_setup(args.seed)
+    for i in range(args.warmup):
+        oracle_sample_step(cache, wl, i, args.seed)
+    ts = [oracle_sample_step(cache, wl, args.warmup + i, args.seed) for i in range(args.steps)]
+    per_step = sum(ts) / len(ts) * oracle_units(wl)
+    value = wl.batch / per_step
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 5), "unit": "tok/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(per_step * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_block(wl),
+        "cpu_baseline": {"value": round(value, 5), "unit": "tok/s", "cores": cores, "kind": "oracle",
+                         "sample": (f"each step: 1 of the {oracle_units(wl)} (sequence, KV head) units, "
+                                    f"scaled x{oracle_units(wl)}")},
+        "e2e": {"value": round(value, 5), "unit": "tok/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def config_block(wl):
+    return {"workload": wl.name, "batch": wl.batch, "hq": wl.hq, "hkv": wl.hkv, "head_dim": 128,
+            "context_start": wl.ctx[0], "block_tokens": 16, "window": 128, "group": 128,
+            "step": "append 1 bf16 K/V token per sequence + decode attention",
+            "l2": "not flushed: each step reads the 232 MB cache, larger than the 126 MB L2",
+            "timed_as": "CUDA graph of K steps"}
+
+
+# ------------------------------------------------------------------ our arm
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+    from int2_kv_cache_rotate_b200 import okv
+    from int2_kv_cache_rotate_b200 import workloads as WL
+
+    world, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    K, W = args.steps, args.warmup
+    e2e_steps = 0 if args.no_e2e else K
+    total = W + K + e2e_steps + 1
+    w = build_gpu_workload(args.seed, rank, total, torch, okv, WL)
+    B, hq = w["B"], w["hq"]
+    out = torch.empty((B, hq, 128), dtype=torch.float32, device="cuda")
+    ws = okv.workspace(w["cache"], B)
+    # eager pre-warm (idempotent with graph step 0: same token, same position)
+    step(w, 0, okv, out, ws)
+    torch.cuda.synchronize()
+
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    for a, b in evs:
+        a.record()
+        b.record()
+    torch.cuda.synchronize()
+    cap = torch.cuda.Stream()
+    g_warm, g_time = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_warm, stream=cap):
+        for i in range(W):
+            step(w, i, okv, out, ws)
+    with torch.cuda.graph(g_time, stream=cap):
+        for i in range(K):
+            step(w, W + i, okv, out, ws, ev=evs[i])
+    g_warm.replay()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = Clocks(local)
+    clocks.start()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    t0.record()
+    g_time.replay()
+    t1.record()
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    ms = t0.elapsed_time(t1)
+    dec_us = [a.elapsed_time(b) * 1e3 for a, b in evs]
+    if world > 1:
+        t = torch.tensor([ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+        dist.barrier()
+    assert w["cache"].device_status() == 0, w["cache"].device_status()
+
+    # end to end through the public calls, inputs from pinned host memory
+    e2e = None
+    if e2e_steps:
+        hk = w["knew"].cpu().pin_memory()
+        hv = w["vnew"].cpu().pin_memory()
+        hqv = w["q"].cpu().pin_memory()
+        hpos = w["pos"].cpu().pin_memory()
+        hlen = w["lens"].cpu().pin_memory()
+        hout = torch.empty((B, hq, 128), dtype=torch.float32).pin_memory()
+        dk, dv = torch.empty_like(w["knew"][0]), torch.empty_like(w["vnew"][0])
+        dq = torch.empty_like(w["q"][0])
+        dpos, dlen = torch.empty_like(w["pos"][0]), torch.empty_like(w["lens"][0])
+        c = w["cache"]
+        base = W + K
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for i in range(base, base + e2e_steps):
+            dk.copy_(hk[i], non_blocking=True)
+            dv.copy_(hv[i], non_blocking=True)
+            dq.copy_(hqv[i], non_blocking=True)
+            dpos.copy_(hpos[i], non_blocking=True)
+            dlen.copy_(hlen[i], non_blocking=True)
+            okv.append_quantize(c, dk, dv, w["seq"], dpos, w["table"], dlen)
+            okv.decode_attention(c, dq, w["seq"], w["table"], dlen, out=out, ws=ws)
+            hout.copy_(out, non_blocking=True)
+        e1.record()
+        torch.cuda.synchronize()
+        e_ms = e0.elapsed_time(e1)
+        if world > 1:
+            t = torch.tensor([e_ms], device="cuda")
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e_ms = float(t.item())
+        h2d = sum(x[0].numel() * x.element_size() for x in (hk, hv, hqv, hpos, hlen))
+        e2e = {"value": round(world * B * e2e_steps / (e_ms * 1e-3), 2), "unit": "tok/s",
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(hout.numel() * 4),
+               "ms_per_step": round(e_ms / e2e_steps, 4), "timed_as": "eager calls, one per step"}
+
+    append_rate = prefill_append_rate(torch, okv, WL, args.seed) if rank == 0 else None
+
+    if rank == 0:
+        lens_timed = [[w["L0"] + W + i + 1] * B for i in range(K)]
+        alg = statistics.mean(algorithmic_bytes(l, w["hkv"]) for l in lens_timed)
+        dec_mean = statistics.mean(dec_us)
+        achieved = alg / (dec_mean * 1e-6) / 1e9
+        peak, peak_src = measured_peak_hbm()
+        tr = recorded_traffic()
+        line = {
+            "metric": METRIC,
+            "value": round(world * B * K / (ms * 1e-3), 2),
+            "unit": "tok/s",
+            "n_gpus": world, "steps": K, "warmup": W, "ms_per_step": round(ms / K, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f32", "data": "synthetic",
+            "config": config_block(w["wl"]),
+            "hbm_gbs": round(achieved, 1),
+            "decode_kernel_us": round(dec_mean, 3),
+            "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                         "frac": round(achieved / peak, 4), "peak_source": peak_src,
+                         "traffic": (tr["bytes_per_launch"] if tr else None),
+                         "kernel": "split-K INT2 decode attention",
+                         "algorithmic_bytes_per_launch": int(alg)},
+            "append_prefill": append_rate,
+            "e2e": e2e,
+            "gpu_launches": 4 * K,
+            "clocks": clk,
+        }
+        if not args.no_cpu_baseline and world == 1:
+            line["cpu_baseline"] = cpu_baseline(args.seed)
+        print(json.dumps(line), flush=True)
+    del g_warm, g_time
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

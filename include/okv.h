@@ -1,0 +1,189 @@
+/*
+ * okv.h -- C ABI of the B200 INT2 KV-cache library (OSCAR-style rotations).
+ *
+ * What the library computes, as the pages describe it:
+ *   - keys are rotated by R_K = U_K H P_br, with U_K the eigenbasis of the
+ *     calibration query covariance; values by R_V = U_V H P_br, with U_V the
+ *     eigenbasis of the attention-score-weighted value covariance; H is a
+ *     normalised Hadamard and P_br the bit-reversal permutation, applied in
+ *     that order (gen-hub.ru, "Together AI открывает OSCAR…", section
+ *     "Что придумали в Together AI"; aiforradalom.hu, "Az Apple, a Google és
+ *     a NYU új technikái…", section "OSCAR: figyelem-tudatos és bevetésre kész");
+ *   - the rotated vectors are stored as 2-bit codes with a per-group scale
+ *     and minimum (bigsaas.top, "Revolução no Serviço de LLMs…", section
+ *     "Resultados e Métricas de Desempenho": INT2 at about 2.28 bits);
+ *   - recent tokens are also kept in 16-bit, older ones only in INT2, in a
+ *     paged cache (encorp.ai, "KV cache compression е инфраструктурно
+ *     решение…", section "OSCAR има значение…");
+ *   - decode attention reads that cache; decode is bound by reading the cache
+ *     from HBM (aiforradalom.hu intro).
+ *
+ * Conventions
+ *   - Row vectors: x_rot = x R.  Matrices are row-major fp32.
+ *   - d (head_dim) = 128, quantisation group = 128 (one group per token-head),
+ *     16 tokens per block, fp16 window W = 128 tokens.  Other values return
+ *     OKV_ERR_UNSUPPORTED.
+ *   - "device" pointers point to memory of the current CUDA device; "host"
+ *     pointers to ordinary host memory.  The caller owns every buffer; the
+ *     library allocates nothing on the hot path and never synchronises the
+ *     stream.  `stream` is a cudaStream_t (NULL = legacy default stream).
+ *   - Every call validates its arguments on the host before launching and
+ *     returns a status.  Launch failures return OKV_ERR_CUDA.  Conditions
+ *     only the device can see (a block id outside [0, num_blocks), a position
+ *     beyond the block table, a decode length beyond the table) are skipped by
+ *     the kernels and recorded in `desc->status_word` (if not NULL) as a
+ *     bitwise OR of OKV_DEV_* flags; the caller reads it when it chooses.
+ *   - okv_last_error_string() describes the last non-OK status of the
+ *     calling thread.
+ *
+ * Physical layout of one block (16 tokens) of one KV head: 1152 bytes
+ *   [   0,  512) K codes, token-major: 16 rows of 32 bytes; byte b of row t
+ *                holds channels 4b..4b+3 of token t at bits 0-1, 2-3, 4-5, 6-7
+ *                (channel = index after the rotation, i.e. after P_br).
+ *   [ 512, 1024) V codes, the same bytes regrouped: 32 chunks of 16 bytes;
+ *                byte b of token t sits at 512 + ((b>>2)*4 + (t>>2))*16
+ *                + (b&3)*4 + (t&3).
+ *   [1024, 1088) K scale and min: token t at 1024 + 4t, fp16 scale then fp16 min.
+ *   [1088, 1152) V scale and min, the same.
+ * Block `blk`, head `h` starts at pages + (blk * num_kv_heads + h) * 1152.
+ * Window ring: fp16 [num_seq_slots][num_kv_heads][2 (K,V)][W][d]; position p
+ * of a sequence lives in row p % W; values are the rotated vector in fp16.
+ */
+#ifndef OKV_H
+#define OKV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  OKV_OK = 0,
+  OKV_ERR_INVALID_ARG = 1,  /* bad pointer, size, alignment or shape      */
+  OKV_ERR_UNSUPPORTED = 2,  /* valid but not implemented (d != 128, ...)  */
+  OKV_ERR_CUDA = 3,         /* a CUDA runtime call or a launch failed     */
+  OKV_ERR_NUMERIC = 4,      /* the eigensolver did not converge           */
+} okv_status;
+
+/* bits of *status_word written by the kernels */
+#define OKV_DEV_BAD_BLOCK 1u     /* block id outside [0, num_blocks)       */
+#define OKV_DEV_BAD_POS 2u       /* position or length beyond the table    */
+#define OKV_DEV_BAD_SLOT 4u      /* sequence slot outside [0, num_seq_slots) */
+
+/* okv_append_quantize flags */
+#define OKV_PRE_ROTATED 1u  /* k, v are fp32 values already in the rotated basis */
+
+#define OKV_HEAD_DIM 128
+#define OKV_BLOCK_TOKENS 16
+#define OKV_WINDOW 128
+#define OKV_BLOCK_HEAD_BYTES 1152
+
+typedef struct {
+  int32_t num_q_heads;        /* Hq; a multiple of num_kv_heads            */
+  int32_t num_kv_heads;       /* Hkv                                        */
+  int32_t head_dim;           /* must be 128                                */
+  int32_t group;              /* must be 128                                */
+  int32_t block_tokens;       /* must be 16                                 */
+  int32_t window;             /* must be 128                                */
+  int32_t num_blocks;         /* physical blocks in `pages`                 */
+  int32_t num_seq_slots;      /* sequences the window ring holds            */
+  int32_t max_blocks_per_seq; /* row length of every block table            */
+  int32_t reserved;
+  void* pages;                /* device, num_blocks*Hkv*1152 B, 16-B aligned */
+  void* window_ring;          /* device fp16, layout above, 16-B aligned     */
+  const float* u_k;           /* device fp32 [Hkv][d][d]: U_K of each KV head */
+  const float* u_v;           /* device fp32 [Hkv][d][d]: U_V of each KV head */
+  uint32_t* status_word;      /* device, nullable: OKV_DEV_* flags (OR-ed)   */
+} okv_cache_desc;
+
+/* Offline calibration of the rotations, on the host in fp64 (once per layer).
+ * q: host fp32 [nq][hq][d] calibration queries; k, v: host fp32 [nk][hkv][d]
+ * calibration keys and values.  Query head j belongs to KV head j/(hq/hkv).
+ *   C_Q = mean of q q^T over the nq*G queries of the group (uncentred),
+ *   C_S = sum_ij p_ij v_j v_j^T / sum_ij p_ij, p_ij = softmax_j(q_i.k_j/sqrt(d)),
+ *   U = eigenvectors by descending eigenvalue, each column signed so that its
+ *   largest-magnitude entry is positive; R = U H P_br.
+ * Outputs (host fp32 [hkv][d][d], each nullable): r_k, r_v, u_k, u_v.
+ * Errors: INVALID_ARG (null inputs, nq/nk < 1, hq % hkv), UNSUPPORTED
+ * (d != 128), NUMERIC (Jacobi sweeps did not converge).
+ * Pages: gen-hub.ru "Что придумали в Together AI" (both covariances and the
+ * three-step transform) and "Открытый код — это серьёзно" (offline, once). */
+okv_status okv_calibrate_rotations(const float* q, int64_t nq, const float* k, const float* v,
+                                   int64_t nk, int32_t hq, int32_t hkv, int32_t d, float* r_k,
+                                   float* r_v, float* u_k, float* u_v);
+
+/* Bytes the caller allocates for `pages` and for `window_ring`. */
+size_t okv_pages_bytes(int32_t num_blocks, int32_t num_kv_heads);
+size_t okv_window_bytes(int32_t num_seq_slots, int32_t num_kv_heads);
+
+/* Append T tokens: rotate each K and V vector of every KV head by its R,
+ * quantise it to 2-bit codes with fp16 scale and min (fp32 round-to-nearest
+ * steps: s = fp16((max-min)/3), m = fp16(min), c = clamp(rint((z-m)/s),0,3),
+ * c = 0 when s = 0; fp16 conversions saturate at +-65504), write codes and
+ * (s, m) into slot pos%16 of block block_table[slot][pos/16], and, when
+ * pos >= slot_lens[slot] - W, also write the fp16 rotated vector into the
+ * window ring row pos % W.
+ *   k, v: device [T][Hkv][d], bf16 (or fp32 already rotated with OKV_PRE_ROTATED);
+ *   seq_slot, pos: device int32 [T]; block_table: device int32
+ *   [num_seq_slots][max_blocks_per_seq]; slot_lens: device int32
+ *   [num_seq_slots], each sequence's length after this append;
+ *   rotated_out: device fp32 [T][2][Hkv][d] (nullable), the rotated fp32
+ *   vectors the quantiser saw.
+ * Tokens with equal (slot, pos) in one call race; T = 0 is a no-op.
+ * Pages: gen-hub.ru "Что придумали в Together AI" (U, then H, then P_br);
+ * bigsaas.top "Resultados e Métricas de Desempenho" (INT2). */
+okv_status okv_append_quantize(const okv_cache_desc* desc, const void* k, const void* v, int32_t T,
+                               const int32_t* seq_slot, const int32_t* pos,
+                               const int32_t* block_table, const int32_t* slot_lens,
+                               uint32_t flags, float* rotated_out, void* stream);
+
+/* Workspace bytes okv_decode_attention needs for batch B on the current device. */
+size_t okv_decode_workspace_bytes(const okv_cache_desc* desc, int32_t B);
+
+/* Decode attention for one new query per sequence.
+ *   q: device bf16 [B][Hq][d]; seq_slot: device int32 [B] (row of block table
+ *   and window ring); block_table as above; context_lens: device int32 [B],
+ *   tokens in the cache for each sequence (the caller appends the step's own
+ *   token first); out: device fp32 [B][Hq][d]; workspace: device, at least
+ *   okv_decode_workspace_bytes(desc, B) bytes, 256-B aligned.
+ * Query head j reads KV head j/(Hq/Hkv).  With L = context_lens[b], positions
+ * [0, L-W) are read from the INT2 blocks and [max(0,L-W), L) from the fp16
+ * window; q~ = q R_K, softmax(q~ x^T / sqrt(d)) over those, then o = o~ R_V^T.
+ * L = 0 gives zeros.  Launches three kernels on `stream` (query rotation,
+ * split-K attention, split combine with the value un-rotation).
+ * Pages: aiforradalom.hu intro (decode streams the cache from HBM);
+ * gen-hub.ru "Что придумали в Together AI" (rotations of Q and of SV). */
+okv_status okv_decode_attention(const okv_cache_desc* desc, const void* q, int32_t B,
+                                const int32_t* seq_slot, const int32_t* block_table,
+                                const int32_t* context_lens, float* out, void* workspace,
+                                size_t workspace_bytes, void* stream);
+
+/* Gather and dequantise the cache into dense fp32.
+ *   which: 0 keys, 1 values.  basis: 0 rotated (as stored), 1 original
+ *   (multiplied back by R^T).  source: 0 INT2 for every position, 1 as decode
+ *   reads it (fp16 window for the last W positions).  out: device fp32
+ *   [B][Hkv][max_ctx][d]; rows at positions >= context_lens[b] are zero.
+ * INT2 values are s*c + m computed with one fused multiply-add. */
+okv_status okv_dequantize(const okv_cache_desc* desc, int32_t B, const int32_t* seq_slot,
+                          const int32_t* block_table, const int32_t* context_lens,
+                          int32_t max_ctx, int32_t which, int32_t basis, int32_t source,
+                          float* out, void* stream);
+
+/* Measurement hook: the next okv_decode_attention call made by this thread
+ * records `start_event` just before its split-K attention kernel and
+ * `stop_event` just after it (both cudaEvent_t, recorded on the call's
+ * stream), then forgets them.  Passing two NULLs clears a pending request.
+ * Lets a caller time the dominant kernel inside a running decode step.
+ * Errors: INVALID_ARG if exactly one event is NULL. */
+okv_status okv_time_next_decode_kernel(void* start_event, void* stop_event);
+
+const char* okv_status_string(okv_status s);
+const char* okv_last_error_string(void);
+int32_t okv_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* OKV_H */

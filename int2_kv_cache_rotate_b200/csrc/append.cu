@@ -1,0 +1,122 @@
+// Append kernel: rotate (U, Hadamard butterfly, bit-reversal remap), quantise
+// to INT2 with fp16 scale/min, pack, and write the paged cache and fp16 window.
+#include "okv_common.cuh"
+#include "okv_internal.h"
+
+namespace okv {
+namespace {
+
+struct AppendArgs {
+  const void* k;
+  const void* v;
+  const int32_t* seq_slot;
+  const int32_t* pos;
+  const int32_t* block_table;
+  const int32_t* slot_lens;
+  const float* u_k;
+  const float* u_v;
+  uint8_t* pages;
+  __half* ring;
+  float* rotated_out;
+  uint32_t* status;
+  int hkv, num_blocks, num_slots, mbps;
+};
+
+// One CTA per (token, KV head, K|V).  Lane l of warp 0 ends up owning the
+// pre-permutation channels l + 32a, which after P_br are rotated channels
+// 4*rev5(l) + rev2(a): exactly the four codes of packed byte rev5(l).  So the
+// permutation costs nothing: it is the choice of which byte a lane writes.
+template <bool kPre>
+__global__ void __launch_bounds__(128) append_kernel(AppendArgs a) {
+  __shared__ float red[4][kD];
+  const int t = blockIdx.x, h = blockIdx.y, kind = blockIdx.z;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const size_t vec = ((size_t)t * a.hkv + h) * kD;
+  float y[4];
+  if constexpr (!kPre) {
+    const __nv_bfloat16* src = (const __nv_bfloat16*)(kind ? a.v : a.k) + vec;
+    rotate_cta(src, (kind ? a.u_v : a.u_k) + (size_t)h * kD * kD, red, y);
+    if (warp != 0) return;
+  } else {
+    const float* src = (const float*)(kind ? a.v : a.k) + vec;
+    const float4 z4 = *reinterpret_cast<const float4*>(src + 4 * rev5(lane));
+    y[0] = z4.x;  // rotated channel 4r+0 <- pre-permutation index l
+    y[1] = z4.z;  // 4r+2 <- l+32
+    y[2] = z4.y;  // 4r+1 <- l+64
+    y[3] = z4.w;  // 4r+3 <- l+96
+  }
+
+  const int slot = a.seq_slot[t];
+  const int p = a.pos[t];
+  if (slot < 0 || slot >= a.num_slots) {
+    if (lane == 0) raise_flag(a.status, OKV_DEV_BAD_SLOT);
+    return;
+  }
+  const int len = a.slot_lens[slot];
+  if (p < 0 || (p >> 4) >= a.mbps || p >= len) {
+    if (lane == 0) raise_flag(a.status, OKV_DEV_BAD_POS);
+    return;
+  }
+  const int blk = a.block_table[(size_t)slot * a.mbps + (p >> 4)];
+  if (blk < 0 || blk >= a.num_blocks) {
+    if (lane == 0) raise_flag(a.status, OKV_DEV_BAD_BLOCK);
+    return;
+  }
+  const int r = rev5(lane);
+  if (a.rotated_out != nullptr) {
+    float4 o = make_float4(y[0], y[2], y[1], y[3]);
+    *reinterpret_cast<float4*>(a.rotated_out + (((size_t)t * 2 + kind) * a.hkv + h) * kD + 4 * r) = o;
+  }
+  const Quantized q = quantize_warp(y);
+  uint8_t* base = a.pages + ((size_t)blk * a.hkv + h) * kBlockHeadBytes;
+  const int s16 = p & 15;
+  if (kind == 0) {
+    base[kKcOff + s16 * 32 + r] = (uint8_t)q.byte;
+  } else {
+    base[v_code_offset(s16, r)] = (uint8_t)q.byte;
+  }
+  if (lane == 0) *reinterpret_cast<uint32_t*>(base + (kind ? kVsmOff : kKsmOff) + 4 * s16) = q.sm;
+  if (p >= len - kWin) {
+    __half* row = a.ring + ((((size_t)slot * a.hkv + h) * 2 + kind) * kWin + (p % kWin)) * kD + 4 * r;
+    __half2 lo = __halves2half2(fp16_sat(y[0]), fp16_sat(y[2]));
+    __half2 hi = __halves2half2(fp16_sat(y[1]), fp16_sat(y[3]));
+    uint2 w;
+    w.x = *reinterpret_cast<uint32_t*>(&lo);
+    w.y = *reinterpret_cast<uint32_t*>(&hi);
+    *reinterpret_cast<uint2*>(row) = w;
+  }
+}
+
+}  // namespace
+
+okv_status launch_append(const okv_cache_desc* d, const void* k, const void* v, int T,
+                         const int32_t* seq_slot, const int32_t* pos, const int32_t* block_table,
+                         const int32_t* slot_lens, uint32_t flags, float* rotated_out,
+                         cudaStream_t s) {
+  AppendArgs a;
+  a.k = k;
+  a.v = v;
+  a.seq_slot = seq_slot;
+  a.pos = pos;
+  a.block_table = block_table;
+  a.slot_lens = slot_lens;
+  a.u_k = d->u_k;
+  a.u_v = d->u_v;
+  a.pages = (uint8_t*)d->pages;
+  a.ring = (__half*)d->window_ring;
+  a.rotated_out = rotated_out;
+  a.status = d->status_word;
+  a.hkv = d->num_kv_heads;
+  a.num_blocks = d->num_blocks;
+  a.num_slots = d->num_seq_slots;
+  a.mbps = d->max_blocks_per_seq;
+  dim3 grid(T, d->num_kv_heads, 2);
+  if (flags & OKV_PRE_ROTATED) {
+    append_kernel<true><<<grid, 32, 0, s>>>(a);
+  } else {
+    append_kernel<false><<<grid, 128, 0, s>>>(a);
+  }
+  return check_launch("append");
+}
+
+}  // namespace okv

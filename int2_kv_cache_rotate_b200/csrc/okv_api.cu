@@ -1,0 +1,204 @@
+// C ABI entry points: argument validation, workspace planning, launches.
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include "okv_common.cuh"
+#include "okv_internal.h"
+
+namespace okv {
+
+static thread_local char g_last_error[512] = "";
+static thread_local cudaEvent_t g_ev_start = nullptr, g_ev_stop = nullptr;
+
+void take_decode_events(cudaEvent_t* start, cudaEvent_t* stop) {
+  *start = g_ev_start;
+  *stop = g_ev_stop;
+  g_ev_start = g_ev_stop = nullptr;
+}
+
+void set_last_error(const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
+  va_end(ap);
+}
+
+okv_status fail(okv_status s, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
+  va_end(ap);
+  return s;
+}
+
+okv_status check_launch(const char* what) {
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(OKV_ERR_CUDA, "%s launch failed: %s", what, cudaGetErrorString(e));
+  return OKV_OK;
+}
+
+int device_sm_count() {
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  return sms;
+}
+
+static bool aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
+
+okv_status validate_desc(const okv_cache_desc* d) {
+  if (d == nullptr) return fail(OKV_ERR_INVALID_ARG, "desc is NULL");
+  if (d->head_dim != kD || d->group != kD || d->block_tokens != kBlock || d->window != kWin)
+    return fail(OKV_ERR_UNSUPPORTED, "only head_dim=128, group=128, block_tokens=16, window=128 are built "
+                "(got %d, %d, %d, %d)", d->head_dim, d->group, d->block_tokens, d->window);
+  if (d->num_kv_heads < 1 || d->num_q_heads < 1 || d->num_q_heads % d->num_kv_heads != 0)
+    return fail(OKV_ERR_INVALID_ARG, "num_q_heads (%d) must be a positive multiple of num_kv_heads (%d)",
+                d->num_q_heads, d->num_kv_heads);
+  if (d->num_kv_heads > 65535 || d->num_q_heads > 65535)
+    return fail(OKV_ERR_INVALID_ARG, "too many heads");
+  if (d->num_blocks < 0 || d->num_seq_slots < 1 || d->max_blocks_per_seq < 1)
+    return fail(OKV_ERR_INVALID_ARG, "num_blocks >= 0, num_seq_slots >= 1, max_blocks_per_seq >= 1 required");
+  if (d->pages == nullptr && d->num_blocks > 0) return fail(OKV_ERR_INVALID_ARG, "pages is NULL");
+  if (d->window_ring == nullptr) return fail(OKV_ERR_INVALID_ARG, "window_ring is NULL");
+  if (d->u_k == nullptr || d->u_v == nullptr) return fail(OKV_ERR_INVALID_ARG, "u_k/u_v is NULL");
+  if (!aligned(d->pages, 16) || !aligned(d->window_ring, 16) || !aligned(d->u_k, 16) || !aligned(d->u_v, 16))
+    return fail(OKV_ERR_INVALID_ARG, "pages, window_ring, u_k and u_v must be 16-byte aligned");
+  if ((long long)d->max_blocks_per_seq * kBlock > 0x3fffffffLL)
+    return fail(OKV_ERR_INVALID_ARG, "max_blocks_per_seq too large");
+  return OKV_OK;
+}
+
+static size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+DecodePlan make_decode_plan(int batch, int hq, int hkv) {
+  DecodePlan p;
+  p.batch = batch;
+  p.hq = hq;
+  p.hkv = hkv;
+  p.g = hq / hkv;
+  const int sms = device_sm_count();
+  p.num_ctas = (sms > 0 ? sms : 148) * 4;
+  p.num_units = batch * hkv;
+  size_t off = 0;
+  p.qrot_off = off;
+  off = align_up(off + (size_t)batch * hq * kD * sizeof(float), 256);
+  p.qlimb_off = off;
+  off = align_up(off + (size_t)batch * hq * 2 * kD, 256);
+  p.qscale_off = off;
+  off = align_up(off + (size_t)batch * hq * 4 * sizeof(float), 256);
+  p.prefix_off = off;
+  off = align_up(off + (size_t)(batch + 1) * sizeof(int32_t), 256);
+  p.part_off = off;
+  off = align_up(off + (size_t)(p.num_ctas + p.num_units) * p.g * kPartStride * sizeof(float), 256);
+  p.total = off;
+  return p;
+}
+
+}  // namespace okv
+
+using namespace okv;
+
+extern "C" {
+
+int32_t okv_version(void) { return 1; }
+
+okv_status okv_time_next_decode_kernel(void* start_event, void* stop_event) {
+  if ((start_event == nullptr) != (stop_event == nullptr))
+    return fail(OKV_ERR_INVALID_ARG, "pass two events or two NULLs");
+  g_ev_start = (cudaEvent_t)start_event;
+  g_ev_stop = (cudaEvent_t)stop_event;
+  return OKV_OK;
+}
+
+const char* okv_last_error_string(void) { return g_last_error; }
+
+const char* okv_status_string(okv_status s) {
+  switch (s) {
+    case OKV_OK: return "OKV_OK";
+    case OKV_ERR_INVALID_ARG: return "OKV_ERR_INVALID_ARG";
+    case OKV_ERR_UNSUPPORTED: return "OKV_ERR_UNSUPPORTED";
+    case OKV_ERR_CUDA: return "OKV_ERR_CUDA";
+    case OKV_ERR_NUMERIC: return "OKV_ERR_NUMERIC";
+  }
+  return "unknown okv_status";
+}
+
+size_t okv_pages_bytes(int32_t num_blocks, int32_t num_kv_heads) {
+  if (num_blocks < 0 || num_kv_heads < 0) return 0;
+  return (size_t)num_blocks * (size_t)num_kv_heads * kBlockHeadBytes;
+}
+
+size_t okv_window_bytes(int32_t num_seq_slots, int32_t num_kv_heads) {
+  if (num_seq_slots < 0 || num_kv_heads < 0) return 0;
+  return (size_t)num_seq_slots * num_kv_heads * 2 * kWin * kD * sizeof(__half);
+}
+
+okv_status okv_append_quantize(const okv_cache_desc* desc, const void* k, const void* v, int32_t T,
+                               const int32_t* seq_slot, const int32_t* pos,
+                               const int32_t* block_table, const int32_t* slot_lens,
+                               uint32_t flags, float* rotated_out, void* stream) {
+  okv_status st = validate_desc(desc);
+  if (st != OKV_OK) return st;
+  if (T < 0) return fail(OKV_ERR_INVALID_ARG, "T must be >= 0");
+  if (flags & ~OKV_PRE_ROTATED) return fail(OKV_ERR_INVALID_ARG, "unknown flags 0x%x", flags);
+  if (T == 0) return OKV_OK;
+  if (!k || !v || !seq_slot || !pos || !block_table || !slot_lens)
+    return fail(OKV_ERR_INVALID_ARG, "k, v, seq_slot, pos, block_table and slot_lens must be non-NULL");
+  if (desc->num_blocks == 0) return fail(OKV_ERR_INVALID_ARG, "cache has no blocks");
+  const size_t al = (flags & OKV_PRE_ROTATED) ? 16 : 2;
+  if ((uintptr_t)k % al || (uintptr_t)v % al)
+    return fail(OKV_ERR_INVALID_ARG, "k and v must be %zu-byte aligned", al);
+  if (rotated_out && (uintptr_t)rotated_out % 16)
+    return fail(OKV_ERR_INVALID_ARG, "rotated_out must be 16-byte aligned");
+  return launch_append(desc, k, v, T, seq_slot, pos, block_table, slot_lens, flags, rotated_out,
+                       (cudaStream_t)stream);
+}
+
+size_t okv_decode_workspace_bytes(const okv_cache_desc* desc, int32_t B) {
+  if (validate_desc(desc) != OKV_OK || B < 0) return 0;
+  return make_decode_plan(B, desc->num_q_heads, desc->num_kv_heads).total;
+}
+
+okv_status okv_decode_attention(const okv_cache_desc* desc, const void* q, int32_t B,
+                                const int32_t* seq_slot, const int32_t* block_table,
+                                const int32_t* context_lens, float* out, void* workspace,
+                                size_t workspace_bytes, void* stream) {
+  okv_status st = validate_desc(desc);
+  if (st != OKV_OK) return st;
+  if (B < 0) return fail(OKV_ERR_INVALID_ARG, "B must be >= 0");
+  if (B == 0) return OKV_OK;
+  if (!q || !seq_slot || !block_table || !context_lens || !out || !workspace)
+    return fail(OKV_ERR_INVALID_ARG, "q, seq_slot, block_table, context_lens, out and workspace must be non-NULL");
+  const int g = desc->num_q_heads / desc->num_kv_heads;
+  if (g != 1 && g != 2 && g != 4 && g != 8 && g != 16)
+    return fail(OKV_ERR_UNSUPPORTED, "Hq/Hkv = %d not in {1,2,4,8,16}", g);
+  if ((long long)B * desc->num_kv_heads * ((long long)desc->max_blocks_per_seq + kWinCost) >= 0x7fffffffLL)
+    return fail(OKV_ERR_INVALID_ARG, "B * Hkv * max_blocks_per_seq too large");
+  if ((uintptr_t)workspace % 256) return fail(OKV_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  const DecodePlan plan = make_decode_plan(B, desc->num_q_heads, desc->num_kv_heads);
+  if (workspace_bytes < plan.total)
+    return fail(OKV_ERR_INVALID_ARG, "workspace too small: %zu < %zu bytes", workspace_bytes, plan.total);
+  return launch_decode(desc, q, B, seq_slot, block_table, context_lens, out, workspace, plan,
+                       (cudaStream_t)stream);
+}
+
+okv_status okv_dequantize(const okv_cache_desc* desc, int32_t B, const int32_t* seq_slot,
+                          const int32_t* block_table, const int32_t* context_lens,
+                          int32_t max_ctx, int32_t which, int32_t basis, int32_t source,
+                          float* out, void* stream) {
+  okv_status st = validate_desc(desc);
+  if (st != OKV_OK) return st;
+  if (B < 0 || max_ctx < 0) return fail(OKV_ERR_INVALID_ARG, "B and max_ctx must be >= 0");
+  if ((which != 0 && which != 1) || (basis != 0 && basis != 1) || (source != 0 && source != 1))
+    return fail(OKV_ERR_INVALID_ARG, "which, basis and source must each be 0 or 1");
+  if (B == 0 || max_ctx == 0) return OKV_OK;
+  if (!seq_slot || !block_table || !context_lens || !out)
+    return fail(OKV_ERR_INVALID_ARG, "seq_slot, block_table, context_lens and out must be non-NULL");
+  if ((uintptr_t)out % 16) return fail(OKV_ERR_INVALID_ARG, "out must be 16-byte aligned");
+  if (B > 65535) return fail(OKV_ERR_INVALID_ARG, "B > 65535");
+  return launch_dequant(desc, B, seq_slot, block_table, context_lens, max_ctx, which, basis, source, out,
+                        (cudaStream_t)stream);
+}
+
+}  // extern "C"

@@ -1,0 +1,160 @@
+// Shared device-side definitions of the INT2 KV-cache library.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "okv.h"
+
+namespace okv {
+
+constexpr int kD = 128;           // head dimension = quantisation group
+constexpr int kBlock = 16;        // tokens per block
+constexpr int kWin = 128;         // fp16 window length
+constexpr int kBlockHeadBytes = 1152;
+constexpr int kKcOff = 0;         // K codes, token-major 16 x 32 B
+constexpr int kVcOff = 512;       // V codes, 4-token-interleaved chunks
+constexpr int kKsmOff = 1024;     // K (fp16 scale, fp16 min) per token
+constexpr int kVsmOff = 1088;     // V (fp16 scale, fp16 min) per token
+constexpr float kInvSqrtD = 0.088388347648318440550f;  // 1/sqrt(128)
+constexpr float kLog2e = 1.4426950408889634074f;
+
+// Byte offset, inside one block-head, of canonical code byte b (channels
+// 4b..4b+3) of token t in the V region.  Chunk (b>>2, t>>2) of 16 bytes holds
+// bytes 4*(b>>2)..+3 of the four tokens 4*(t>>2)..+3, one 4-byte word per
+// code byte, one byte per token inside the word.
+__host__ __device__ __forceinline__ int v_code_offset(int t, int b) {
+  return kVcOff + (((b >> 2) * 4 + (t >> 2)) << 4) + ((b & 3) << 2) + (t & 3);
+}
+
+__host__ __device__ __forceinline__ int rev5(int x) {
+  return ((x & 1) << 4) | ((x & 2) << 2) | (x & 4) | ((x & 8) >> 2) | ((x & 16) >> 4);
+}
+// position of pre-permutation index (lane l, register a), i = l + 32a, after P_br:
+// br7(32a + l) = 4*rev5(l) + rev2(a), rev2 = {0, 2, 1, 3}.
+__host__ __device__ __forceinline__ int rev2(int a) { return ((a & 1) << 1) | (a >> 1); }
+
+__device__ __forceinline__ void raise_flag(uint32_t* w, uint32_t bits) {
+  if (w != nullptr) atomicOr(w, bits);
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+__device__ __forceinline__ float warp_min(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fminf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+// Walsh-Hadamard butterfly over 128 values held as y[a] = v[l + 32a] in lane l
+// of a warp (natural/Sylvester order, unnormalised).  Lane bits use shuffles,
+// register bits stay in registers.
+__device__ __forceinline__ void wht128_warp(float y[4], int lane) {
+#pragma unroll
+  for (int b = 1; b < 32; b <<= 1) {
+    const bool hi = (lane & b) != 0;
+#pragma unroll
+    for (int a = 0; a < 4; ++a) {
+      const float p = __shfl_xor_sync(0xffffffffu, y[a], b);
+      y[a] = hi ? __fsub_rn(p, y[a]) : __fadd_rn(y[a], p);
+    }
+  }
+  float t0 = __fadd_rn(y[0], y[1]), t1 = __fsub_rn(y[0], y[1]);
+  float t2 = __fadd_rn(y[2], y[3]), t3 = __fsub_rn(y[2], y[3]);
+  y[0] = __fadd_rn(t0, t2);
+  y[2] = __fsub_rn(t0, t2);
+  y[1] = __fadd_rn(t1, t3);
+  y[3] = __fsub_rn(t1, t3);
+}
+
+__device__ __forceinline__ __half fp16_sat(float x) {
+  return __float2half_rn(fminf(fmaxf(x, -65504.0f), 65504.0f));
+}
+
+// INT2 group quantiser over the 128 values of a warp (y[a] = value at
+// pre-permutation index l + 32a, i.e. rotated channel 4*rev5(l) + rev2(a)).
+// All steps are IEEE fp32 round-to-nearest; returns this lane's packed code
+// byte (canonical byte rev5(l)) and the fp16 scale/min bits.
+struct Quantized {
+  uint32_t byte;
+  uint32_t sm;  // fp16 scale in bits 0-15, fp16 min in bits 16-31
+};
+
+__device__ __forceinline__ Quantized quantize_warp(const float y[4]) {
+  float mn = fminf(fminf(y[0], y[1]), fminf(y[2], y[3]));
+  float mx = fmaxf(fmaxf(y[0], y[1]), fmaxf(y[2], y[3]));
+  mn = warp_min(mn);
+  mx = warp_max(mx);
+  const float s32 = __fdiv_rn(__fsub_rn(mx, mn), 3.0f);
+  const __half s16 = fp16_sat(s32);
+  const __half m16 = fp16_sat(mn);
+  const float s = __half2float(s16);
+  const float m = __half2float(m16);
+  uint32_t byte = 0;
+#pragma unroll
+  for (int a = 0; a < 4; ++a) {
+    uint32_t c = 0;
+    if (s != 0.0f) {
+      const float r = rintf(__fdiv_rn(__fsub_rn(y[a], m), s));
+      c = (uint32_t)fminf(fmaxf(r, 0.0f), 3.0f);
+    }
+    byte |= c << (2 * rev2(a));
+  }
+  Quantized q;
+  q.byte = byte;
+  q.sm = (uint32_t)__half_as_ushort(s16) | ((uint32_t)__half_as_ushort(m16) << 16);
+  return q;
+}
+
+}  // namespace okv
+
+namespace okv {
+
+// x = in . U (fp32 accumulate), then the normalised Hadamard, on a CTA of 128
+// threads.  Warp w sums input channels 32w..32w+31; the four partials meet in
+// shared memory; warp 0 finishes and returns y[a] = (x H)[l + 32a].
+// `in` holds 128 consecutive bf16 values; U is row-major [128][128].
+template <typename InT>
+__device__ __forceinline__ void rotate_cta(const InT* __restrict__ in, const float* __restrict__ u,
+                                           float (*red)[kD], float y[4]) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  float xin;
+  if constexpr (sizeof(InT) == 2) {
+    xin = __bfloat162float(in[32 * warp + lane]);
+  } else {
+    xin = in[32 * warp + lane];
+  }
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  const float* urow = u + (size_t)(32 * warp) * kD + lane;
+#pragma unroll 8
+  for (int cc = 0; cc < 32; ++cc) {
+    const float xc = __shfl_sync(0xffffffffu, xin, cc);
+#pragma unroll
+    for (int a = 0; a < 4; ++a) acc[a] = fmaf(xc, __ldg(urow + cc * kD + 32 * a), acc[a]);
+  }
+#pragma unroll
+  for (int a = 0; a < 4; ++a) red[warp][lane + 32 * a] = acc[a];
+  __syncthreads();
+  if (warp == 0) {
+#pragma unroll
+    for (int a = 0; a < 4; ++a) {
+      const int i = lane + 32 * a;
+      y[a] = ((red[0][i] + red[1][i]) + red[2][i]) + red[3][i];
+    }
+    wht128_warp(y, lane);
+#pragma unroll
+    for (int a = 0; a < 4; ++a) y[a] *= kInvSqrtD;
+  }
+}
+
+}  // namespace okv

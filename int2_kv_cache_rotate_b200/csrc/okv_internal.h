@@ -1,0 +1,50 @@
+// Host-side declarations shared by the library's translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "okv.h"
+
+namespace okv {
+
+void set_last_error(const char* fmt, ...);
+okv_status fail(okv_status s, const char* fmt, ...);
+okv_status check_launch(const char* what);
+okv_status validate_desc(const okv_cache_desc* d);
+int device_sm_count();
+// events set by okv_time_next_decode_kernel (consumed by the next decode launch)
+void take_decode_events(cudaEvent_t* start, cudaEvent_t* stop);
+
+// decode workspace layout (bytes, from the workspace base)
+struct DecodePlan {
+  int batch = 0;
+  int hq = 0, hkv = 0, g = 0;
+  int num_ctas = 0;         // split-K CTAs
+  int num_units = 0;        // batch * hkv
+  size_t qrot_off = 0;      // fp32 [B][Hq][128] rotated queries
+  size_t qlimb_off = 0;     // int8 [B][Hq][2][128] query limbs (MMA order)
+  size_t qscale_off = 0;    // fp32 [B][Hq][4] (sigma, sum, -, -)
+  size_t prefix_off = 0;    // int32 [B+1] cost prefix over batch entries
+  size_t part_off = 0;      // fp32 [(num_ctas + num_units)][G][kPartStride]
+  size_t total = 0;
+};
+constexpr int kPartStride = 132;  // o'[128], m, l, 2 spare
+constexpr int kWinCost = 8;       // cost of a unit's window in block units
+
+DecodePlan make_decode_plan(int batch, int hq, int hkv);
+
+// launchers (return cudaGetLastError-mapped status)
+okv_status launch_append(const okv_cache_desc* d, const void* k, const void* v, int T,
+                         const int32_t* seq_slot, const int32_t* pos, const int32_t* block_table,
+                         const int32_t* slot_lens, uint32_t flags, float* rotated_out,
+                         cudaStream_t s);
+okv_status launch_decode(const okv_cache_desc* d, const void* q, int B, const int32_t* seq_slot,
+                         const int32_t* block_table, const int32_t* context_lens, float* out,
+                         void* ws, const DecodePlan& plan, cudaStream_t s);
+okv_status launch_dequant(const okv_cache_desc* d, int B, const int32_t* seq_slot,
+                          const int32_t* block_table, const int32_t* context_lens, int max_ctx,
+                          int which, int basis, int source, float* out, cudaStream_t s);
+
+}  // namespace okv

@@ -1,0 +1,231 @@
+"""Thin ctypes binding over ``libokv.so`` (argument marshalling only).
+
+Every step of the hot path runs in the library's CUDA kernels; this module
+checks dtypes/devices/shapes of torch tensors, passes raw pointers and the
+current CUDA stream, and turns non-OK statuses into ``OkvError``.  Nothing
+here computes any part of the method.  If the library is missing the first
+call raises: there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libokv.so")
+HEADER = os.path.join(os.path.dirname(_HERE), "include", "okv.h")
+
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_NUMERIC = range(5)
+DEV_BAD_BLOCK, DEV_BAD_POS, DEV_BAD_SLOT = 1, 2, 4
+PRE_ROTATED = 1
+HEAD_DIM, BLOCK_TOKENS, WINDOW, BLOCK_HEAD_BYTES = 128, 16, 128, 1152
+
+
+class OkvError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"{status}: {msg}")
+        self.status = status
+
+
+class CacheDesc(ctypes.Structure):
+    _fields_ = [
+        ("num_q_heads", ctypes.c_int32),
+        ("num_kv_heads", ctypes.c_int32),
+        ("head_dim", ctypes.c_int32),
+        ("group", ctypes.c_int32),
+        ("block_tokens", ctypes.c_int32),
+        ("window", ctypes.c_int32),
+        ("num_blocks", ctypes.c_int32),
+        ("num_seq_slots", ctypes.c_int32),
+        ("max_blocks_per_seq", ctypes.c_int32),
+        ("reserved", ctypes.c_int32),
+        ("pages", ctypes.c_void_p),
+        ("window_ring", ctypes.c_void_p),
+        ("u_k", ctypes.c_void_p),
+        ("u_v", ctypes.c_void_p),
+        ("status_word", ctypes.c_void_p),
+    ]
+
+
+_lib = None
+_P = ctypes.c_void_p
+_I32 = ctypes.c_int32
+_I64 = ctypes.c_int64
+_U32 = ctypes.c_uint32
+_SZ = ctypes.c_size_t
+_DESC = ctypes.POINTER(CacheDesc)
+
+_SIGNATURES = {
+    "okv_calibrate_rotations": (_I32, [_P, _I64, _P, _P, _I64, _I32, _I32, _I32, _P, _P, _P, _P]),
+    "okv_pages_bytes": (_SZ, [_I32, _I32]),
+    "okv_window_bytes": (_SZ, [_I32, _I32]),
+    "okv_append_quantize": (_I32, [_DESC, _P, _P, _I32, _P, _P, _P, _P, _U32, _P, _P]),
+    "okv_decode_workspace_bytes": (_SZ, [_DESC, _I32]),
+    "okv_decode_attention": (_I32, [_DESC, _P, _I32, _P, _P, _P, _P, _P, _SZ, _P]),
+    "okv_dequantize": (_I32, [_DESC, _I32, _P, _P, _P, _I32, _I32, _I32, _I32, _P, _P]),
+    "okv_status_string": (ctypes.c_char_p, [_I32]),
+    "okv_last_error_string": (ctypes.c_char_p, []),
+    "okv_version": (_I32, []),
+    "okv_time_next_decode_kernel": (_I32, [_P, _P]),
+}
+
+
+def lib() -> ctypes.CDLL:
+    """Load ``libokv.so`` (built in-tree); raise if it is missing."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise OkvError(-1, f"{LIB_PATH} is missing: run `python -m int2_kv_cache_rotate_b200.build`")
+        handle = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGNATURES.items():
+            fn = getattr(handle, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = handle
+    return _lib
+
+
+def header_functions() -> list:
+    """Names of the functions ``include/okv.h`` declares."""
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(okv_[a-z0-9_]+)\s*\(", text)))
+
+
+def _check(status: int):
+    if status != OK:
+        msg = lib().okv_last_error_string().decode()
+        raise OkvError(status, msg)
+
+
+def _ptr(t) -> int:
+    return 0 if t is None else t.data_ptr()
+
+
+def _stream(stream) -> int:
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream
+
+
+def _need(t, dtype, name, device=True):
+    import torch
+    if t is None:
+        raise ValueError(f"{name} is required")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if device and not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t
+
+
+# ---------------------------------------------------------------- calibration
+
+def calibrate_rotations(q: np.ndarray, k: np.ndarray, v: np.ndarray, hq: int, hkv: int) -> dict:
+    """Host fp64 calibration.  q [nq, hq, 128], k/v [nk, hkv, 128] (float32)."""
+    q = np.ascontiguousarray(q, dtype=np.float32)
+    k = np.ascontiguousarray(k, dtype=np.float32)
+    v = np.ascontiguousarray(v, dtype=np.float32)
+    out = {n: np.zeros((hkv, HEAD_DIM, HEAD_DIM), np.float32) for n in ("R_K", "R_V", "U_K", "U_V")}
+    p = lambda a: a.ctypes.data_as(ctypes.c_void_p)
+    _check(lib().okv_calibrate_rotations(p(q), q.shape[0], p(k), p(v), k.shape[0], hq, hkv, q.shape[-1],
+                                         p(out["R_K"]), p(out["R_V"]), p(out["U_K"]), p(out["U_V"])))
+    return out
+
+
+# ---------------------------------------------------------------------- cache
+
+class Cache:
+    """Device buffers of one layer's INT2 cache plus its C descriptor.
+
+    Memory comes from torch (the caller's allocator); the library only
+    receives pointers."""
+
+    def __init__(self, hq: int, hkv: int, num_blocks: int, num_seq_slots: int, max_blocks_per_seq: int,
+                 u_k, u_v, device="cuda"):
+        import torch
+        self.hq, self.hkv = hq, hkv
+        self.num_blocks, self.num_seq_slots, self.max_blocks_per_seq = num_blocks, num_seq_slots, max_blocks_per_seq
+        nbytes = lib().okv_pages_bytes(num_blocks, hkv)
+        self.pages = torch.zeros(max(nbytes, 16), dtype=torch.uint8, device=device)
+        self.ring = torch.zeros((num_seq_slots, hkv, 2, WINDOW, HEAD_DIM), dtype=torch.float16, device=device)
+        self.u_k = torch.as_tensor(np.asarray(u_k, dtype=np.float32)).to(device).contiguous()
+        self.u_v = torch.as_tensor(np.asarray(u_v, dtype=np.float32)).to(device).contiguous()
+        self.status = torch.zeros(4, dtype=torch.int32, device=device)
+        self.desc = CacheDesc(hq, hkv, HEAD_DIM, HEAD_DIM, BLOCK_TOKENS, WINDOW, num_blocks, num_seq_slots,
+                              max_blocks_per_seq, 0, self.pages.data_ptr(), self.ring.data_ptr(),
+                              self.u_k.data_ptr(), self.u_v.data_ptr(), self.status.data_ptr())
+
+    def device_status(self) -> int:
+        return int(self.status[0].item())
+
+    def clear_status(self):
+        self.status.zero_()
+
+
+def append_quantize(cache: Cache, k, v, seq_slot, pos, block_table, slot_lens, pre_rotated=False,
+                    rotated_out=None, stream=None):
+    import torch
+    dt = torch.float32 if pre_rotated else torch.bfloat16
+    _need(k, dt, "k"), _need(v, dt, "v")
+    for name, t in (("seq_slot", seq_slot), ("pos", pos), ("block_table", block_table), ("slot_lens", slot_lens)):
+        _need(t, torch.int32, name)
+    if rotated_out is not None:
+        _need(rotated_out, torch.float32, "rotated_out")
+    T = k.shape[0] if k.dim() > 0 else 0
+    _check(lib().okv_append_quantize(ctypes.byref(cache.desc), _ptr(k), _ptr(v), T, _ptr(seq_slot), _ptr(pos),
+                                     _ptr(block_table), _ptr(slot_lens), PRE_ROTATED if pre_rotated else 0,
+                                     _ptr(rotated_out), _stream(stream)))
+
+
+def decode_workspace_bytes(cache: Cache, batch: int) -> int:
+    return int(lib().okv_decode_workspace_bytes(ctypes.byref(cache.desc), batch))
+
+
+def workspace(cache: Cache, batch: int):
+    import torch
+    return torch.empty(max(decode_workspace_bytes(cache, batch), 256), dtype=torch.uint8, device="cuda")
+
+
+def decode_attention(cache: Cache, q, seq_slot, block_table, context_lens, out=None, ws=None, stream=None):
+    import torch
+    _need(q, torch.bfloat16, "q")
+    for name, t in (("seq_slot", seq_slot), ("block_table", block_table), ("context_lens", context_lens)):
+        _need(t, torch.int32, name)
+    batch = q.shape[0]
+    if out is None:
+        out = torch.empty((batch, cache.hq, HEAD_DIM), dtype=torch.float32, device=q.device)
+    _need(out, torch.float32, "out")
+    if ws is None:
+        ws = workspace(cache, batch)
+    _check(lib().okv_decode_attention(ctypes.byref(cache.desc), _ptr(q), batch, _ptr(seq_slot), _ptr(block_table),
+                                      _ptr(context_lens), _ptr(out), _ptr(ws), ws.numel(), _stream(stream)))
+    return out
+
+
+def time_next_decode_kernel(start_event, stop_event):
+    """Record two torch.cuda.Event objects around the next decode call's split-K kernel."""
+    for e in (start_event, stop_event):
+        if not e.cuda_event:  # torch creates the CUDA event lazily, on first record
+            e.record()
+    _check(lib().okv_time_next_decode_kernel(start_event.cuda_event, stop_event.cuda_event))
+
+
+def dequantize(cache: Cache, seq_slot, block_table, context_lens, max_ctx: int, which: int, basis: int = 0,
+               source: int = 0, out=None, stream=None):
+    import torch
+    for name, t in (("seq_slot", seq_slot), ("block_table", block_table), ("context_lens", context_lens)):
+        _need(t, torch.int32, name)
+    batch = seq_slot.shape[0]
+    if out is None:
+        out = torch.empty((batch, cache.hkv, max_ctx, HEAD_DIM), dtype=torch.float32, device="cuda")
+    _need(out, torch.float32, "out")
+    _check(lib().okv_dequantize(ctypes.byref(cache.desc), batch, _ptr(seq_slot), _ptr(block_table),
+                                _ptr(context_lens), max_ctx, which, basis, source, _ptr(out), _stream(stream)))
+    return out
