@@ -160,6 +160,29 @@ okv_status okv_decode_attention(const okv_cache_desc* desc, const void* q, int32
                                 const int32_t* context_lens, float* out, void* workspace,
                                 size_t workspace_bytes, void* stream);
 
+/* Size of the device array behind okv_decode_attention_noalloc (8 MiB). */
+#define OKV_NOALLOC_SCRATCH_BYTES (8u << 20)
+
+/* Decode attention that allocates nothing and takes no workspace.  The pages
+ * have no counterpart to this call: it exists for callers that cannot
+ * allocate device memory -- a plugin handed only its tensors by an engine
+ * that owns all device memory, or code that must not call cudaMalloc because
+ * it can synchronise the device and stall other streams.
+ *   Same arguments, results and kernels as okv_decode_attention, minus the
+ *   workspace.  Scratch is a static device array of OKV_NOALLOC_SCRATCH_BYTES
+ *   that every GPU which loads the library holds until process exit; a batch
+ *   whose scratch (okv_decode_workspace_bytes) exceeds it is rejected with
+ *   OKV_ERR_INVALID_ARG before anything runs.
+ *   The first call on each device looks up the array's device address with
+ *   that device current; make that first call before any stream capture.
+ *   All calls share the one array (it keeps the last call's contents, none of
+ *   which a later call relies on): calls that overlap on the GPU -- on
+ *   different streams, or from different threads -- race and must be
+ *   serialised by the caller. */
+okv_status okv_decode_attention_noalloc(const okv_cache_desc* desc, const void* q, int32_t B,
+                                        const int32_t* seq_slot, const int32_t* block_table,
+                                        const int32_t* context_lens, float* out, void* stream);
+
 /* Gather and dequantise the cache into dense fp32.
  *   which: 0 keys, 1 values.  basis: 0 rotated (as stored), 1 original
  *   (multiplied back by R^T).  source: 0 INT2 for every position, 1 as decode

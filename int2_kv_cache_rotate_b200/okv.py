@@ -70,6 +70,7 @@ _SIGNATURES = {
     "okv_last_error_string": (ctypes.c_char_p, []),
     "okv_version": (_I32, []),
     "okv_time_next_decode_kernel": (_I32, [_P, _P]),
+    "okv_decode_attention_noalloc": (_I32, [_DESC, _P, _I32, _P, _P, _P, _P, _P]),
 }
 
 
@@ -206,6 +207,21 @@ def decode_attention(cache: Cache, q, seq_slot, block_table, context_lens, out=N
         ws = workspace(cache, batch)
     _check(lib().okv_decode_attention(ctypes.byref(cache.desc), _ptr(q), batch, _ptr(seq_slot), _ptr(block_table),
                                       _ptr(context_lens), _ptr(out), _ptr(ws), ws.numel(), _stream(stream)))
+    return out
+
+
+def decode_attention_noalloc(cache: Cache, q, seq_slot, block_table, context_lens, out=None, stream=None):
+    """Decode attention with the library's static scratch (no workspace, no allocation in the library)."""
+    import torch
+    _need(q, torch.bfloat16, "q")
+    for name, t in (("seq_slot", seq_slot), ("block_table", block_table), ("context_lens", context_lens)):
+        _need(t, torch.int32, name)
+    batch = q.shape[0]
+    if out is None:
+        out = torch.empty((batch, cache.hq, HEAD_DIM), dtype=torch.float32, device=q.device)
+    _need(out, torch.float32, "out")
+    _check(lib().okv_decode_attention_noalloc(ctypes.byref(cache.desc), _ptr(q), batch, _ptr(seq_slot),
+                                              _ptr(block_table), _ptr(context_lens), _ptr(out), _stream(stream)))
     return out
 
 
