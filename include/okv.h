@@ -71,6 +71,7 @@ typedef enum {
 #define OKV_DEV_BAD_BLOCK 1u     /* block id outside [0, num_blocks)       */
 #define OKV_DEV_BAD_POS 2u       /* position or length beyond the table    */
 #define OKV_DEV_BAD_SLOT 4u      /* sequence slot outside [0, num_seq_slots) */
+#define OKV_DEV_TIMEOUT 8u       /* a bulk copy did not land within ~1 s; the kernel gave up */
 
 /* okv_append_quantize flags */
 #define OKV_PRE_ROTATED 1u  /* k, v are fp32 values already in the rotated basis */

@@ -65,7 +65,8 @@ struct DecodeArgs {
   uint32_t* status;
   float* qrot;       // [B][Hq][128]
   int8_t* qlimb;     // [B][Hq][2][128]
-  float* qscale;     // [B][Hq][4]
+  float* qscale;     // [B][Hq][4]: score scale, min-term scale, sigma, sum
+  __half* qwin;      // [B][Hq][2][128]: q~/sigma as fp16 hi, lo (natural channel order)
   int32_t* prefix;   // [B+1] cost prefix over batch entries (units of b are consecutive)
   float* part;       // [(NC + NU)][G][kPartStride]
   int batch, hq, hkv, g, nc, num_blocks, num_slots, mbps;
@@ -110,8 +111,40 @@ __global__ void __launch_bounds__(128) qrot_kernel(DecodeArgs a) {
   rotate_cta(src, a.u_k + (size_t)(h / a.g) * kD * kD, red, y);
   if (warp != 0) return;
   const int r = rev5(lane);
-  float* dst = a.qrot + ((size_t)b * a.hq + h) * kD + 4 * r;
+  const size_t bh = (size_t)b * a.hq + h;
+  float* dst = a.qrot + bh * kD + 4 * r;
   *reinterpret_cast<float4*>(dst) = make_float4(y[0], y[2], y[1], y[3]);
+
+  // Integer limbs for the tensor-core score tiles: Q = rint(q~/sigma) in
+  // [-32000, 32000] = 256*hi + lo with hi, lo signed 8-bit.  Bytes are stored
+  // in MMA-fragment order: channel c = 32t + 16h + 4i + s goes to position
+  // 32t + 8s + 4h + i, so a lane of quad t reads its 32 bytes in one go.
+  const float zc[4] = {y[0], y[2], y[1], y[3]};  // rotated channels 4r + e
+  float amax = fmaxf(fmaxf(fabsf(y[0]), fabsf(y[1])), fmaxf(fabsf(y[2]), fabsf(y[3])));
+  amax = warp_max(amax);
+  const float sum = warp_sum((y[0] + y[1]) + (y[2] + y[3]));
+  const float sigma = amax > 0.f ? amax / 32000.f : 1.f;
+  const float inv = amax > 0.f ? 32000.f / amax : 0.f;
+  int8_t* lim = a.qlimb + bh * 2 * kD;
+  __half* qw = a.qwin + bh * 2 * kD;
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const int c = 4 * r + e;
+    const float x = zc[e] * inv;
+    const int q = max(-32000, min(32000, __float2int_rn(x)));
+    const int hi = ((q + 32896) >> 8) - 128;
+    const int lo = q - 256 * hi;
+    const int pos = (c >> 5) * 32 + (c & 3) * 8 + ((c >> 4) & 1) * 4 + ((c >> 2) & 3);
+    lim[pos] = (int8_t)hi;
+    lim[kD + pos] = (int8_t)lo;
+    const __half hx = __float2half_rn(x);
+    qw[c] = hx;
+    qw[kD + c] = __float2half_rn(x - __half2float(hx));
+  }
+  if (lane == 0) {
+    float4 qs4 = make_float4(sigma * (kInvSqrtD * kLog2e), sum * (kInvSqrtD * kLog2e), sigma, sum);
+    *reinterpret_cast<float4*>(a.qscale + bh * 4) = qs4;
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -330,6 +363,509 @@ __global__ void __launch_bounds__(kDecWarps * 32) decode_simt_kernel(DecodeArgs 
 }
 
 // ---------------------------------------------------------------------------
+// Kernel 2 (tensor cores): split-K attention for G = Hq/Hkv in {1, 2, 4, 8}.
+//
+// Each warp streams its own 2-block steps (32 tokens, 2 x 1152 B) through a
+// 4-stage ring of bulk copies into shared memory and computes, per step:
+//   scores  S[32 tok x 4NT heads] = C_K (u8 codes) . Q (two s8 limbs) on
+//           mma.m16n8k32, then s_t * sigma * raw + m_t * sum(q~);
+//   values  O[128 ch x heads] += C_V^T (u8 codes) . P' (two u8 limbs of
+//           round(p * s_t * 65535 / s_cap)), exact in int32, flushed to fp32
+//           only when the running max or the scale cap moves;
+//   plus sum(p * m_t) for the value minimum term.
+// Fragment facts (PTX m16n8k32, 8-bit): lane (g = lane/4, t = lane%4) holds
+// A rows g and g+8, K-columns 4t..4t+3 and 16+4t..16+4t+3; B K-rows 4t..+3 and
+// 16+4t..+3 of column g; D rows g, g+8, columns 2t, 2t+1.  Every contraction
+// index permutation is absorbed by the query-limb and P' layouts.
+// The window (the last <= 128 tokens, fp16) is attended by one warp in ring
+// order (softmax attention does not depend on token order): scores on
+// mma.m16n8k16 f16 with the query as two fp16 halves, P.V on CUDA cores.
+// ---------------------------------------------------------------------------
+constexpr int kMmaWarps = 4;
+constexpr int kStages = 4;
+constexpr int kStageBytes = 2 * kBlockHeadBytes;
+constexpr int kPStride = 40;  // u16 per head row of the P' staging tile
+constexpr uint32_t kM2 = 0x03030303u;
+
+template <int G>
+struct MmaCfg {
+  static constexpr int NT = G <= 4 ? 1 : G / 4;  // n-tiles of 8 columns = 4 heads x 2 limbs
+  static constexpr int HP = 4 * NT;              // heads incl. padding
+  static constexpr size_t smem_bytes() {
+    return (size_t)kMmaWarps * kStages * kStageBytes          // stage ring
+           + (size_t)kMmaWarps * kStages * 8                   // mbarriers
+           + (size_t)kMmaWarps * HP * kPStride * 2             // P' tiles
+           + (size_t)G * 16 * 4                                // window p tile [16 tok][G]
+           + (size_t)(kMmaWarps + 1) * G * kD * 4              // merge o'
+           + (size_t)(kMmaWarps + 1) * G * 2 * 4;              // merge (m, l)
+  }
+};
+
+__device__ __forceinline__ float lo_half(uint32_t w) {
+  return __half2float(__ushort_as_half((unsigned short)(w & 0xffffu)));
+}
+__device__ __forceinline__ float hi_half(uint32_t w) {
+  return __half2float(__ushort_as_half((unsigned short)(w >> 16)));
+}
+
+__device__ __forceinline__ void mma_f16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};\n"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+template <int G>
+struct MmaWarpState {
+  static constexpr int NT = MmaCfg<G>::NT;
+  float m[NT], l[NT], msum[NT];
+  float acc[NT][16];   // fp32 partial o' for channels 16g + 0..15 of head 4nt + t
+  int acci[NT][8][4];  // exact int32 o' contributions since the last flush
+};
+
+template <int G>
+__device__ __forceinline__ void mma_flush(MmaWarpState<G>& st, int nt, float inv) {
+  const float hi_w = 256.f * inv;
+#pragma unroll
+  for (int mt = 0; mt < 8; ++mt) {
+    st.acc[nt][2 * mt] += fmaf((float)st.acci[nt][mt][0], hi_w, (float)st.acci[nt][mt][1] * inv);
+    st.acc[nt][2 * mt + 1] += fmaf((float)st.acci[nt][mt][2], hi_w, (float)st.acci[nt][mt][3] * inv);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) st.acci[nt][mt][j] = 0;
+  }
+}
+
+template <int G>
+__global__ void __launch_bounds__(kMmaWarps * 32, kCtasPerSm) decode_mma_kernel(DecodeArgs a) {
+  constexpr int NT = MmaCfg<G>::NT, HP = MmaCfg<G>::HP;
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  unsigned char* stages = smem_raw;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(stages + kMmaWarps * kStages * kStageBytes);
+  uint16_t* pst = reinterpret_cast<uint16_t*>(bars + kMmaWarps * kStages);
+  float* pw = reinterpret_cast<float*>(pst + kMmaWarps * HP * kPStride);  // [16][G]
+  float* mo = pw + 16 * G;                                                // [NW+1][G][128]
+  float* ml = mo + (kMmaWarps + 1) * G * kD;                              // [NW+1][G][2]
+
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int g = lane >> 2, t = lane & 3;
+  const long long total = a.prefix[a.batch];
+  if (total == 0) return;
+  const int nc = (int)min((long long)a.nc, total);
+  const int c = blockIdx.x;
+  if (c >= nc) return;
+  const long long start = (long long)c * total / nc;
+  const long long end = (long long)(c + 1) * total / nc;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kMmaWarps * kStages; ++i) mbar_init(&bars[i], 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  uint64_t* mybar = bars + warp * kStages;
+  unsigned char* myst = stages + warp * kStages * kStageBytes;
+  uint16_t* myp = pst + warp * HP * kPStride;
+  uint32_t it = 0;      // steps this warp has issued and consumed so far (ring position)
+  bool alive = true;    // cleared if a bulk copy never lands
+
+  int lo = 0, hi = a.batch - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (a.prefix[mid] <= start) lo = mid; else hi = mid - 1;
+  }
+  for (int b = lo; b < a.batch && a.prefix[b] < end; ++b) {
+    const UnitShape us = unit_shape(clamp_len(a.context_lens, b, a.mbps, a.status, false));
+    if (us.cost == 0) continue;
+    const int slot = a.seq_slot[b];
+    const bool slot_ok = slot >= 0 && slot < a.num_slots;
+    for (int hk = 0; hk < a.hkv; ++hk) {
+      const long long pu = a.prefix[b] + (long long)hk * us.cost;
+      if (pu + us.cost <= start) continue;
+      if (pu >= end) break;
+      const int u = b * a.hkv + hk;
+      const int l0 = (int)(max(start, pu) - pu), l1 = (int)(min(end, pu + us.cost) - pu);
+      const size_t bh0 = (size_t)b * a.hq + (size_t)hk * G;  // first query head of the unit
+      __syncthreads();  // the previous unit's merge buffers are free again
+
+      // ---------------- INT2 blocks ----------------
+      MmaWarpState<G> st;
+      uint32_t qb[NT][8];
+      float ah[NT], bh[NT];
+      bool hv[NT];
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        st.m[nt] = -INFINITY;
+        st.l[nt] = 0.f;
+        st.msum[nt] = 0.f;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) st.acc[nt][i] = 0.f;
+#pragma unroll
+        for (int mt = 0; mt < 8; ++mt)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) st.acci[nt][mt][j] = 0;
+        const int hcol = 4 * nt + (g >> 1);  // head of this lane's B column
+        if (hcol < G) {
+          const uint4* src = reinterpret_cast<const uint4*>(a.qlimb + ((bh0 + hcol) * 2 + (g & 1)) * kD + 32 * t);
+          const uint4 x0 = src[0], x1 = src[1];
+          qb[nt][0] = x0.x; qb[nt][1] = x0.y; qb[nt][2] = x0.z; qb[nt][3] = x0.w;
+          qb[nt][4] = x1.x; qb[nt][5] = x1.y; qb[nt][6] = x1.z; qb[nt][7] = x1.w;
+        } else {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) qb[nt][i] = 0u;
+        }
+        const int hs = 4 * nt + t;  // head of this lane's score columns
+        hv[nt] = hs < G;
+        ah[nt] = hv[nt] ? a.qscale[(bh0 + hs) * 4 + 0] : 0.f;
+        bh[nt] = hv[nt] ? a.qscale[(bh0 + hs) * 4 + 1] : 0.f;
+      }
+      float s_cap = 0.f, lam = 0.f, inv = 0.f;
+      int since_flush = 0;
+
+      const int p0 = max(l0, us.win_cost) - us.win_cost;
+      const int p1 = l1 - us.win_cost;
+      const int nsteps = p1 > p0 ? (p1 - p0 + 1) >> 1 : 0;
+      const int nmy = (slot_ok && alive && nsteps > warp) ? (nsteps - warp + kMmaWarps - 1) / kMmaWarps : 0;
+      const int32_t* trow = a.block_table + (size_t)(slot_ok ? slot : 0) * a.mbps;
+
+      // issue local step j into ring position it + j (lane 0 only)
+      auto issue = [&](int j) {
+        const int k = warp + kMmaWarps * j;
+        const int pa = p0 + 2 * k;
+        const uint32_t stg = (it + j) % kStages;
+        int blk[2];
+        uint32_t bytes = 0;
+#pragma unroll
+        for (int bb = 0; bb < 2; ++bb) {
+          const int pi = pa + bb;
+          blk[bb] = pi < p1 ? trow[pi] : -1;
+          if (blk[bb] >= a.num_blocks) blk[bb] = -1;
+          if (blk[bb] >= 0) bytes += kBlockHeadBytes;
+        }
+        mbar_arrive_expect_tx(&mybar[stg], bytes);
+#pragma unroll
+        for (int bb = 0; bb < 2; ++bb)
+          if (blk[bb] >= 0)
+            bulk_g2s(myst + stg * kStageBytes + bb * kBlockHeadBytes,
+                     a.pages + ((size_t)blk[bb] * a.hkv + hk) * kBlockHeadBytes, kBlockHeadBytes, &mybar[stg]);
+      };
+      if (lane == 0)
+        for (int j = 0; j < min(kStages, nmy); ++j) issue(j);
+
+      int done = 0;
+      for (int j = 0; j < nmy; ++j) {
+        const uint32_t stg = (it + j) % kStages;
+        const uint32_t par = ((it + j) / kStages) & 1u;
+        const bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(&mybar[stg], par));
+        if (!ok) {
+          if (lane == 0) raise_flag(a.status, OKV_DEV_TIMEOUT);
+          alive = false;
+          break;
+        }
+        const int k = warp + kMmaWarps * j;
+        const int pa = p0 + 2 * k;
+        int ntok[2];
+#pragma unroll
+        for (int bb = 0; bb < 2; ++bb) {
+          const int pi = pa + bb;
+          int bid = pi < p1 ? trow[pi] : -1;
+          if (pi < p1 && (bid < 0 || bid >= a.num_blocks)) {
+            if (lane == 0) raise_flag(a.status, OKV_DEV_BAD_BLOCK);
+            bid = -1;
+          }
+          ntok[bb] = bid >= 0 ? min(kBlock, us.n_int2 - kBlock * pi) : 0;
+        }
+        const unsigned char* s0 = myst + stg * kStageBytes;
+
+        // scores
+        int dq[2][NT][4];
+        uint32_t smk[4], smv[4];
+#pragma unroll
+        for (int bb = 0; bb < 2; ++bb) {
+          const unsigned char* sb = s0 + bb * kBlockHeadBytes;
+          const uint2 wa = *reinterpret_cast<const uint2*>(sb + kKcOff + 32 * g + 8 * t);
+          const uint2 wb = *reinterpret_cast<const uint2*>(sb + kKcOff + 32 * (g + 8) + 8 * t);
+          smk[2 * bb] = *reinterpret_cast<const uint32_t*>(sb + kKsmOff + 4 * g);
+          smk[2 * bb + 1] = *reinterpret_cast<const uint32_t*>(sb + kKsmOff + 4 * (g + 8));
+          smv[2 * bb] = *reinterpret_cast<const uint32_t*>(sb + kVsmOff + 4 * g);
+          smv[2 * bb + 1] = *reinterpret_cast<const uint32_t*>(sb + kVsmOff + 4 * (g + 8));
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) dq[bb][nt][jj] = 0;
+#pragma unroll
+          for (int s = 0; s < 4; ++s) {
+            uint32_t af[4];
+            af[0] = (wa.x >> (2 * s)) & kM2;
+            af[1] = (wb.x >> (2 * s)) & kM2;
+            af[2] = (wa.y >> (2 * s)) & kM2;
+            af[3] = (wb.y >> (2 * s)) & kM2;
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) mma_u8s8(dq[bb][nt], af, qb[nt][2 * s], qb[nt][2 * s + 1]);
+          }
+        }
+        // token e of this lane: block e>>1, row g + 8*(e&1)
+        bool tv[4];
+        float sv[4], mv[4];
+        float smax = 0.f;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          tv[e] = (g + 8 * (e & 1)) < ntok[e >> 1];
+          sv[e] = lo_half(smv[e]);
+          mv[e] = hi_half(smv[e]);
+          if (tv[e]) smax = fmaxf(smax, sv[e]);
+        }
+        smax = fmaxf(smax, __shfl_xor_sync(0xffffffffu, smax, 4));
+        smax = fmaxf(smax, __shfl_xor_sync(0xffffffffu, smax, 8));
+        smax = fmaxf(smax, __shfl_xor_sync(0xffffffffu, smax, 16));
+        if (smax > s_cap) {  // raise the scale cap: flush every head at the old cap first
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) mma_flush(st, nt, inv);
+          since_flush = 0;
+          s_cap = smax;
+          lam = 65535.f / s_cap;
+          inv = s_cap / 65535.f;
+        }
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          float sc[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int bb = e >> 1, r = 2 * (e & 1);
+            const int raw = dq[bb][nt][r] * 256 + dq[bb][nt][r + 1];
+            sc[e] = (tv[e] && hv[nt]) ? fmaf(lo_half(smk[e]) * ah[nt], (float)raw, hi_half(smk[e]) * bh[nt])
+                                       : -INFINITY;
+          }
+          float bm = fmaxf(fmaxf(sc[0], sc[1]), fmaxf(sc[2], sc[3]));
+          bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 4));
+          bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 8));
+          bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 16));
+          if (bm > st.m[nt]) {
+            mma_flush(st, nt, inv);
+            const float alpha = exp2f(st.m[nt] - bm);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) st.acc[nt][i] *= alpha;
+            st.l[nt] *= alpha;
+            st.msum[nt] *= alpha;
+            st.m[nt] = bm;
+          }
+          uint16_t* prow = myp + (4 * nt + t) * kPStride;
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float p = (sc[e] == -INFINITY) ? 0.f : exp2f(sc[e] - st.m[nt]);
+            st.l[nt] += p;
+            st.msum[nt] = fmaf(p, mv[e], st.msum[nt]);
+            const uint32_t pi = (p > 0.f) ? min(__float2uint_rn(p * sv[e] * lam), 65535u) : 0u;
+            prow[16 * (e >> 1) + g + 8 * (e & 1)] = (uint16_t)pi;
+          }
+        }
+        __syncwarp();
+        // values
+        const uint4 v0 = *reinterpret_cast<const uint4*>(s0 + kVcOff + 16 * lane);
+        const uint4 v1 = *reinterpret_cast<const uint4*>(s0 + kBlockHeadBytes + kVcOff + 16 * lane);
+        const uint32_t va[4] = {v0.x, v0.y, v0.z, v0.w};
+        const uint32_t vb[4] = {v1.x, v1.y, v1.z, v1.w};
+        uint32_t pb0[NT], pb1[NT];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          const uint16_t* prow = myp + (4 * nt + (g >> 1)) * kPStride;
+          const uint2 x0 = *reinterpret_cast<const uint2*>(prow + 4 * t);
+          const uint2 x1 = *reinterpret_cast<const uint2*>(prow + 16 + 4 * t);
+          const uint32_t sel = (g & 1) ? 0x6420u : 0x7531u;  // lo limb = low byte, hi limb = high byte
+          pb0[nt] = prmt(x0.x, x0.y, sel);
+          pb1[nt] = prmt(x1.x, x1.y, sel);
+        }
+#pragma unroll
+        for (int mt = 0; mt < 8; ++mt) {
+          const int jw = mt >> 1, f0 = 4 * (mt & 1);
+          uint32_t af[4];
+          af[0] = (va[jw] >> f0) & kM2;
+          af[1] = (va[jw] >> (f0 + 2)) & kM2;
+          af[2] = (vb[jw] >> f0) & kM2;
+          af[3] = (vb[jw] >> (f0 + 2)) & kM2;
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) mma_u8u8(st.acci[nt][mt], af, pb0[nt], pb1[nt]);
+        }
+        if (++since_flush >= 128) {
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) mma_flush(st, nt, inv);
+          since_flush = 0;
+        }
+        __syncwarp();
+        ++done;
+        if (lane == 0 && j + kStages < nmy) issue(j + kStages);
+      }
+      if (!alive) {  // drain what is still in flight, with the same bound, then stop streaming
+        for (int j = done + 1; j < min(nmy, done + kStages); ++j)
+          (void)mbar_wait_bounded(&mybar[(it + j) % kStages], ((it + j) / kStages) & 1u);
+      }
+      it += (uint32_t)nmy;
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        mma_flush(st, nt, inv);
+        float l = st.l[nt], ms = st.msum[nt];
+#pragma unroll
+        for (int o = 4; o < 32; o <<= 1) {
+          l += __shfl_xor_sync(0xffffffffu, l, o);
+          ms += __shfl_xor_sync(0xffffffffu, ms, o);
+        }
+        const int hs = 4 * nt + t;
+        if (hs < G) {
+          float* dst = mo + ((size_t)warp * G + hs) * kD + 16 * g;
+#pragma unroll
+          for (int i = 0; i < 16; ++i) dst[i] = st.acc[nt][i] + ms;
+          if (g == 0) {
+            ml[(warp * G + hs) * 2 + 0] = st.m[nt];
+            ml[(warp * G + hs) * 2 + 1] = l;
+          }
+        }
+      }
+
+      // ---------------- fp16 window (warp 0, if this CTA owns it) ----------------
+      if (warp == 0) {
+        float wm[NT], wl[NT], wo[G][4];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) { wm[nt] = -INFINITY; wl[nt] = 0.f; }
+#pragma unroll
+        for (int hh = 0; hh < G; ++hh)
+#pragma unroll
+          for (int i = 0; i < 4; ++i) wo[hh][i] = 0.f;
+        if (l0 == 0 && us.win_cost > 0 && slot_ok) {
+          const __half* kr = a.ring + (((size_t)slot * a.hkv + hk) * 2 + 0) * kWin * kD;
+          const __half* vr = a.ring + (((size_t)slot * a.hkv + hk) * 2 + 1) * kWin * kD;
+          // query halves of this lane's B column, channels 32t .. 32t+31
+          uint32_t qh[NT][16];
+          float wsc[NT];
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) {
+            const int hcol = 4 * nt + (g >> 1);
+            if (hcol < G) {
+              const uint4* src = reinterpret_cast<const uint4*>(a.qwin + ((bh0 + hcol) * 2 + (g & 1)) * kD + 32 * t);
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                const uint4 x = src[i];
+                qh[nt][4 * i] = x.x; qh[nt][4 * i + 1] = x.y; qh[nt][4 * i + 2] = x.z; qh[nt][4 * i + 3] = x.w;
+              }
+            } else {
+#pragma unroll
+              for (int i = 0; i < 16; ++i) qh[nt][i] = 0u;
+            }
+            const int hs = 4 * nt + t;
+            wsc[nt] = hs < G ? a.qscale[(bh0 + hs) * 4 + 0] : 0.f;
+          }
+          for (int r0 = 0; r0 < us.n_win; r0 += 16) {
+            // scores of ring rows r0 + g and r0 + g + 8
+            uint32_t ka[16], kb[16];
+            const bool va_ = r0 + g < us.n_win, vb_ = r0 + g + 8 < us.n_win;
+            const uint4* ra = reinterpret_cast<const uint4*>(kr + (size_t)(r0 + g) * kD + 32 * t);
+            const uint4* rb = reinterpret_cast<const uint4*>(kr + (size_t)(r0 + g + 8) * kD + 32 * t);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const uint4 x = va_ ? ra[i] : make_uint4(0, 0, 0, 0);
+              const uint4 y = vb_ ? rb[i] : make_uint4(0, 0, 0, 0);
+              ka[4 * i] = x.x; ka[4 * i + 1] = x.y; ka[4 * i + 2] = x.z; ka[4 * i + 3] = x.w;
+              kb[4 * i] = y.x; kb[4 * i + 1] = y.y; kb[4 * i + 2] = y.z; kb[4 * i + 3] = y.w;
+            }
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+              float d[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+              for (int ks = 0; ks < 8; ++ks) {
+                const uint32_t af[4] = {ka[2 * ks], kb[2 * ks], ka[2 * ks + 1], kb[2 * ks + 1]};
+                mma_f16(d, af, qh[nt][2 * ks], qh[nt][2 * ks + 1]);
+              }
+              const int hs = 4 * nt + t;
+              const float s_a = (va_ && hs < G) ? (d[0] + d[1]) * wsc[nt] : -INFINITY;
+              const float s_b = (vb_ && hs < G) ? (d[2] + d[3]) * wsc[nt] : -INFINITY;
+              float bm = fmaxf(s_a, s_b);
+              bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 4));
+              bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 8));
+              bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 16));
+              const float mnew = fmaxf(wm[nt], bm);
+              const float alpha = (mnew == -INFINITY) ? 1.f : exp2f(wm[nt] - mnew);
+              const float pa_ = (s_a == -INFINITY) ? 0.f : exp2f(s_a - mnew);
+              const float pb_ = (s_b == -INFINITY) ? 0.f : exp2f(s_b - mnew);
+              wl[nt] = wl[nt] * alpha + pa_ + pb_;
+              wm[nt] = mnew;
+              if (hs < G) {
+                pw[g * G + hs] = pa_;
+                pw[(g + 8) * G + hs] = pb_;
+              }
+              // rescale this n-tile's heads in the P.V accumulators (lane owns 4 channels of every head)
+#pragma unroll
+              for (int q4 = 0; q4 < 4; ++q4) {
+                const float al = __shfl_sync(0xffffffffu, alpha, q4);  // lane q4 holds head 4nt + q4
+                const int hh = 4 * nt + q4;
+                if (hh < G) {
+#pragma unroll
+                  for (int i = 0; i < 4; ++i) wo[hh][i] *= al;
+                }
+              }
+            }
+            __syncwarp();
+            const int nrow = min(16, us.n_win - r0);
+            for (int rr = 0; rr < nrow; ++rr) {
+              const uint2 w2 = *reinterpret_cast<const uint2*>(vr + (size_t)(r0 + rr) * kD + 4 * lane);
+              const float2 f0 = __half22float2(*reinterpret_cast<const __half2*>(&w2.x));
+              const float2 f1 = __half22float2(*reinterpret_cast<const __half2*>(&w2.y));
+#pragma unroll
+              for (int hh = 0; hh < G; ++hh) {
+                const float p = pw[rr * G + hh];
+                wo[hh][0] = fmaf(p, f0.x, wo[hh][0]);
+                wo[hh][1] = fmaf(p, f0.y, wo[hh][1]);
+                wo[hh][2] = fmaf(p, f1.x, wo[hh][2]);
+                wo[hh][3] = fmaf(p, f1.y, wo[hh][3]);
+              }
+            }
+            __syncwarp();
+          }
+        }
+        // the window's state fills merge slot kMmaWarps (lane owns channels 4*lane .. +3)
+#pragma unroll
+        for (int hh = 0; hh < G; ++hh) {
+          float* dst = mo + ((size_t)kMmaWarps * G + hh) * kD + 4 * lane;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) dst[i] = wo[hh][i];
+        }
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          float l = wl[nt];
+#pragma unroll
+          for (int o = 4; o < 32; o <<= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+          const int hs = 4 * nt + t;
+          if (hs < G && g == 0) {
+            ml[(kMmaWarps * G + hs) * 2 + 0] = wm[nt];
+            ml[(kMmaWarps * G + hs) * 2 + 1] = l;
+          }
+        }
+      }
+      __syncthreads();
+      // merge the warps (and the window) into this CTA's partial for unit u
+      float* dstp = a.part + ((size_t)(c + u) * G) * kPartStride;
+      for (int i = threadIdx.x; i < G * kD; i += blockDim.x) {
+        const int hh = i / kD, ch = i % kD;
+        float mx = -INFINITY;
+        for (int w = 0; w <= kMmaWarps; ++w) mx = fmaxf(mx, ml[(w * G + hh) * 2]);
+        float o = 0.f, l = 0.f;
+        if (mx != -INFINITY) {
+          for (int w = 0; w <= kMmaWarps; ++w) {
+            const float mw = ml[(w * G + hh) * 2];
+            if (mw == -INFINITY) continue;
+            const float sc = exp2f(mw - mx);
+            o = fmaf(mo[(w * G + hh) * kD + ch], sc, o);
+            l = fmaf(ml[(w * G + hh) * 2 + 1], sc, l);
+          }
+        }
+        dstp[hh * kPartStride + ch] = o;
+        if (ch == 0) {
+          dstp[hh * kPartStride + 128] = mx;
+          dstp[hh * kPartStride + 129] = l;
+        }
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
 // Kernel 3: merge the splits of each unit, normalise, undo the value rotation
 // (un-permute, Hadamard, U_V^T) and write fp32 outputs.  One CTA per unit.
 // ---------------------------------------------------------------------------
@@ -400,12 +936,26 @@ __global__ void __launch_bounds__(128) combine_kernel(DecodeArgs a) {
 }
 
 template <int G>
-static okv_status launch_decode_g(const DecodeArgs& a, cudaStream_t s) {
+static okv_status launch_decode_simt(const DecodeArgs& a, cudaStream_t s) {
   const size_t smem = (size_t)(G * kD + kDecWarps * G * kD + kDecWarps * G * 2) * sizeof(float);
   cudaError_t e = cudaFuncSetAttribute(decode_simt_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
   if (e != cudaSuccess) return fail(OKV_ERR_CUDA, "decode smem attribute: %s", cudaGetErrorString(e));
   decode_simt_kernel<G><<<a.nc, kDecWarps * 32, smem, s>>>(a);
+  return check_launch("decode");
+}
+
+template <int G>
+static okv_status launch_decode_mma(const DecodeArgs& a, cudaStream_t s) {
+  const size_t smem = MmaCfg<G>::smem_bytes();
+  static bool configured = false;  // the attribute is per function; set it once
+  if (!configured) {
+    cudaError_t e = cudaFuncSetAttribute(decode_mma_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return fail(OKV_ERR_CUDA, "decode smem attribute: %s", cudaGetErrorString(e));
+    configured = true;
+  }
+  decode_mma_kernel<G><<<a.nc, kMmaWarps * 32, smem, s>>>(a);
   return check_launch("decode");
 }
 
@@ -427,6 +977,7 @@ okv_status launch_decode(const okv_cache_desc* d, const void* q, int B, const in
   a.qrot = (float*)(w + plan.qrot_off);
   a.qlimb = (int8_t*)(w + plan.qlimb_off);
   a.qscale = (float*)(w + plan.qscale_off);
+  a.qwin = (__half*)(w + plan.qwin_off);
   a.prefix = (int32_t*)(w + plan.prefix_off);
   a.part = (float*)(w + plan.part_off);
   a.batch = B;
@@ -446,11 +997,11 @@ okv_status launch_decode(const okv_cache_desc* d, const void* q, int B, const in
   if (ev0 != nullptr && cudaEventRecordWithFlags(ev0, s, cudaEventRecordExternal) != cudaSuccess)
     return fail(OKV_ERR_CUDA, "cudaEventRecord failed");
   switch (a.g) {
-    case 1: st = launch_decode_g<1>(a, s); break;
-    case 2: st = launch_decode_g<2>(a, s); break;
-    case 4: st = launch_decode_g<4>(a, s); break;
-    case 8: st = launch_decode_g<8>(a, s); break;
-    case 16: st = launch_decode_g<16>(a, s); break;
+    case 1: st = launch_decode_mma<1>(a, s); break;
+    case 2: st = launch_decode_mma<2>(a, s); break;
+    case 4: st = launch_decode_mma<4>(a, s); break;
+    case 8: st = launch_decode_mma<8>(a, s); break;
+    case 16: st = launch_decode_simt<16>(a, s); break;
     default: return fail(OKV_ERR_UNSUPPORTED, "group size %d (Hq/Hkv) not in {1,2,4,8,16}", a.g);
   }
   if (st != OKV_OK) return st;

@@ -78,7 +78,7 @@ DecodePlan make_decode_plan(int batch, int hq, int hkv) {
   p.hkv = hkv;
   p.g = hq / hkv;
   const int sms = device_sm_count();
-  p.num_ctas = (sms > 0 ? sms : 148) * 4;
+  p.num_ctas = (sms > 0 ? sms : 148) * kCtasPerSm;
   p.num_units = batch * hkv;
   size_t off = 0;
   p.qrot_off = off;
@@ -87,6 +87,8 @@ DecodePlan make_decode_plan(int batch, int hq, int hkv) {
   off = align_up(off + (size_t)batch * hq * 2 * kD, 256);
   p.qscale_off = off;
   off = align_up(off + (size_t)batch * hq * 4 * sizeof(float), 256);
+  p.qwin_off = off;
+  off = align_up(off + (size_t)batch * hq * 2 * kD * 2, 256);
   p.prefix_off = off;
   off = align_up(off + (size_t)(batch + 1) * sizeof(int32_t), 256);
   p.part_off = off;

@@ -25,13 +25,15 @@ struct DecodePlan {
   int num_units = 0;        // batch * hkv
   size_t qrot_off = 0;      // fp32 [B][Hq][128] rotated queries
   size_t qlimb_off = 0;     // int8 [B][Hq][2][128] query limbs (MMA order)
-  size_t qscale_off = 0;    // fp32 [B][Hq][4] (sigma, sum, -, -)
+  size_t qscale_off = 0;    // fp32 [B][Hq][4] (score scale, min term, sigma, sum)
+  size_t qwin_off = 0;      // fp16 [B][Hq][2][128] scaled query hi/lo halves (window MMA)
   size_t prefix_off = 0;    // int32 [B+1] cost prefix over batch entries
   size_t part_off = 0;      // fp32 [(num_ctas + num_units)][G][kPartStride]
   size_t total = 0;
 };
 constexpr int kPartStride = 132;  // o'[128], m, l, 2 spare
-constexpr int kWinCost = 8;       // cost of a unit's window in block units
+constexpr int kWinCost = 16;      // cost of a unit's window in block units
+constexpr int kCtasPerSm = 3;     // resident split-K CTAs per SM
 
 DecodePlan make_decode_plan(int batch, int hq, int hkv);
 
