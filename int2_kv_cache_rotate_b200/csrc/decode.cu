@@ -366,20 +366,28 @@ __global__ void __launch_bounds__(kDecWarps * 32) decode_simt_kernel(DecodeArgs 
 // Kernel 2 (tensor cores): split-K attention for G = Hq/Hkv in {1, 2, 4, 8}.
 //
 // Each warp streams its own 2-block steps (32 tokens, 2 x 1152 B) through a
-// 4-stage ring of bulk copies into shared memory and computes, per step:
+// ring of bulk copies into shared memory and computes, per step:
 //   scores  S[32 tok x 4NT heads] = C_K (u8 codes) . Q (two s8 limbs) on
 //           mma.m16n8k32, then s_t * sigma * raw + m_t * sum(q~);
-//   values  O[128 ch x heads] += C_V^T (u8 codes) . P' (two u8 limbs of
-//           round(p * s_t * 65535 / s_cap)), exact in int32, flushed to fp32
-//           only when the running max or the scale cap moves;
+//   values  O[128 ch x heads] += C_V^T . P', P' = round(p * s_t * 65535 / s_cap)
+//           as two u8 limbs, exact in int32, flushed to fp32 only when the
+//           running max or the scale cap moves (or every 128 steps);
 //   plus sum(p * m_t) for the value minimum term.
 // Fragment facts (PTX m16n8k32, 8-bit): lane (g = lane/4, t = lane%4) holds
-// A rows g and g+8, K-columns 4t..4t+3 and 16+4t..16+4t+3; B K-rows 4t..+3 and
-// 16+4t..+3 of column g; D rows g, g+8, columns 2t, 2t+1.  Every contraction
-// index permutation is absorbed by the query-limb and P' layouts.
-// The window (the last <= 128 tokens, fp16) is attended by one warp in ring
-// order (softmax attention does not depend on token order): scores on
-// mma.m16n8k16 f16 with the query as two fp16 halves, P.V on CUDA cores.
+// A rows g and g+8 with K-columns 4t..4t+3 and 16+4t..16+4t+3; B K-rows
+// 4t..4t+3 and 16+4t..+3 of column g; D rows g, g+8, columns 2t, 2t+1.
+//   K side: the 32 code bytes of a token row are the contraction; a lane
+//   reads 8 of them and (w >> 2s) & 0x03030303 is one A register.  Which
+//   channel sits in which K-column is absorbed by the query-limb layout.
+//   V side: one 16-byte chunk per lane holds 4 tokens x 16 channels; field f
+//   of word j is channel 16g + 4j + f, which is an output row, so the codes
+//   are only masked (w & (3 << 2f)), leaving a known 4^f factor per output
+//   row that the flush removes.
+// The fp16 window (at most 128 tokens) is attended in ring order (softmax
+// attention does not depend on token order), 16 rows per warp-chunk, all
+// warps sharing the chunks: scores and P.V on mma.m16n8k16 (f16 in, f32
+// accumulate; query and probabilities as fp16 hi+lo pairs); the window state
+// is folded into the warp's own state in registers.
 // ---------------------------------------------------------------------------
 constexpr int kMmaWarps = 4;
 constexpr int kStages = 4;
@@ -391,15 +399,16 @@ template <int G>
 struct MmaCfg {
   static constexpr int NT = G <= 4 ? 1 : G / 4;  // n-tiles of 8 columns = 4 heads x 2 limbs
   static constexpr int HP = 4 * NT;              // heads incl. padding
+  static constexpr size_t ring_bytes = (size_t)kMmaWarps * kStages * kStageBytes;
   static constexpr size_t smem_bytes() {
-    return (size_t)kMmaWarps * kStages * kStageBytes          // stage ring
-           + (size_t)kMmaWarps * kStages * 8                   // mbarriers
-           + (size_t)kMmaWarps * HP * kPStride * 2             // P' tiles
-           + (size_t)G * 16 * 4                                // window p tile [16 tok][G]
-           + (size_t)(kMmaWarps + 1) * G * kD * 4              // merge o'
-           + (size_t)(kMmaWarps + 1) * G * 2 * 4;              // merge (m, l)
+    return ring_bytes                                  // stage rings (reused for merge buffers)
+           + (size_t)kMmaWarps * kStages * 8           // mbarriers
+           + (size_t)kMmaWarps * kStages * 4           // per-stage token counts
+           + (size_t)kMmaWarps * HP * kPStride * 2     // P' tiles
+           + (size_t)kMmaWarps * G * 2 * 4;            // merge (m, l)
   }
 };
+static_assert(kMmaWarps * 8 * kD * 4 <= kMmaWarps * kStages * kStageBytes, "merge buffer must fit the rings");
 
 __device__ __forceinline__ float lo_half(uint32_t w) {
   return __half2float(__ushort_as_half((unsigned short)(w & 0xffffu)));
@@ -416,36 +425,67 @@ __device__ __forceinline__ void mma_f16(float (&d)[4], const uint32_t (&a)[4], u
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
+// D = A . B with a zero accumulator
+__device__ __forceinline__ void mma_u8s8_z(int (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%10,%10,%10,%10};\n"
+      : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "r"(0));
+}
+
+__device__ __forceinline__ void ldmatrix_x4_trans(uint32_t (&r)[4], const void* p) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(smem_u32(p)));
+}
+
+__device__ __forceinline__ float fast_ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ uint32_t cvt_u16_sat(float x) {
+  uint16_t r;
+  asm("cvt.rni.sat.u16.f32 %0, %1;\n" : "=h"(r) : "f"(x));
+  return r;
+}
+
 template <int G>
 struct MmaWarpState {
   static constexpr int NT = MmaCfg<G>::NT;
   float m[NT], l[NT], msum[NT];
-  float acc[NT][16];   // fp32 partial o' for channels 16g + 0..15 of head 4nt + t
-  int acci[NT][8][4];  // exact int32 o' contributions since the last flush
+  float acc[NT][16];   // fp32 o' for channels 16g + 0..15 of head 4nt + t
+  int acci[NT][8][4];  // exact int32 o' contributions since the last flush (row scale 4^f)
 };
 
+// acci[mt] holds channel 16g + 2mt (regs 0,1 = hi, lo limb) and 16g + 2mt + 1
+// (regs 2,3); those channels come from code field f = 2(mt&1) and f + 1,
+// which the unshifted masks scaled by 4^f.
 template <int G>
 __device__ __forceinline__ void mma_flush(MmaWarpState<G>& st, int nt, float inv) {
-  const float hi_w = 256.f * inv;
 #pragma unroll
   for (int mt = 0; mt < 8; ++mt) {
-    st.acc[nt][2 * mt] += fmaf((float)st.acci[nt][mt][0], hi_w, (float)st.acci[nt][mt][1] * inv);
-    st.acc[nt][2 * mt + 1] += fmaf((float)st.acci[nt][mt][2], hi_w, (float)st.acci[nt][mt][3] * inv);
+    const float s0 = (mt & 1) ? inv * (1.f / 16.f) : inv;  // field 0 or 2
+    const float s1 = s0 * 0.25f;                            // field 1 or 3
+    st.acc[nt][2 * mt] += fmaf((float)st.acci[nt][mt][0], 256.f * s0, (float)st.acci[nt][mt][1] * s0);
+    st.acc[nt][2 * mt + 1] += fmaf((float)st.acci[nt][mt][2], 256.f * s1, (float)st.acci[nt][mt][3] * s1);
 #pragma unroll
     for (int j = 0; j < 4; ++j) st.acci[nt][mt][j] = 0;
   }
 }
 
 template <int G>
-__global__ void __launch_bounds__(kMmaWarps * 32, kCtasPerSm) decode_mma_kernel(DecodeArgs a) {
+__global__ void __launch_bounds__(kMmaWarps * 32, (G <= 4) ? 4 : 3) decode_mma_kernel(DecodeArgs a) {
   constexpr int NT = MmaCfg<G>::NT, HP = MmaCfg<G>::HP;
   extern __shared__ __align__(16) unsigned char smem_raw[];
-  unsigned char* stages = smem_raw;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(stages + kMmaWarps * kStages * kStageBytes);
-  uint16_t* pst = reinterpret_cast<uint16_t*>(bars + kMmaWarps * kStages);
-  float* pw = reinterpret_cast<float*>(pst + kMmaWarps * HP * kPStride);  // [16][G]
-  float* mo = pw + 16 * G;                                                // [NW+1][G][128]
-  float* ml = mo + (kMmaWarps + 1) * G * kD;                              // [NW+1][G][2]
+  unsigned char* rings = smem_raw;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(rings + MmaCfg<G>::ring_bytes);
+  uint32_t* stinfo = reinterpret_cast<uint32_t*>(bars + kMmaWarps * kStages);
+  uint16_t* pst = reinterpret_cast<uint16_t*>(stinfo + kMmaWarps * kStages);
+  float* ml = reinterpret_cast<float*>(pst + kMmaWarps * HP * kPStride);  // [NW][G][2]
+  float* mo = reinterpret_cast<float*>(rings);  // [NW][G][128], only while the rings are idle
 
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int g = lane >> 2, t = lane & 3;
@@ -463,10 +503,11 @@ __global__ void __launch_bounds__(kMmaWarps * 32, kCtasPerSm) decode_mma_kernel(
   }
   __syncthreads();
   uint64_t* mybar = bars + warp * kStages;
-  unsigned char* myst = stages + warp * kStages * kStageBytes;
+  uint32_t* myinfo = stinfo + warp * kStages;
+  unsigned char* myst = rings + warp * kStages * kStageBytes;
   uint16_t* myp = pst + warp * HP * kPStride;
-  uint32_t it = 0;      // steps this warp has issued and consumed so far (ring position)
-  bool alive = true;    // cleared if a bulk copy never lands
+  uint32_t it = 0;    // ring position of this warp (continues across units)
+  bool alive = true;  // cleared if a bulk copy never lands
 
   int lo = 0, hi = a.batch - 1;
   while (lo < hi) {
@@ -485,13 +526,12 @@ __global__ void __launch_bounds__(kMmaWarps * 32, kCtasPerSm) decode_mma_kernel(
       const int u = b * a.hkv + hk;
       const int l0 = (int)(max(start, pu) - pu), l1 = (int)(min(end, pu + us.cost) - pu);
       const size_t bh0 = (size_t)b * a.hq + (size_t)hk * G;  // first query head of the unit
-      __syncthreads();  // the previous unit's merge buffers are free again
+      __syncthreads();  // the previous unit's merge buffers (on the rings) are free again
 
       // ---------------- INT2 blocks ----------------
       MmaWarpState<G> st;
       uint32_t qb[NT][8];
-      float ah[NT], bh[NT];
-      bool hv[NT];
+      float ah[NT], bh[NT], hbias[NT];
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
         st.m[nt] = -INFINITY;
@@ -514,9 +554,10 @@ __global__ void __launch_bounds__(kMmaWarps * 32, kCtasPerSm) decode_mma_kernel(
           for (int i = 0; i < 8; ++i) qb[nt][i] = 0u;
         }
         const int hs = 4 * nt + t;  // head of this lane's score columns
-        hv[nt] = hs < G;
-        ah[nt] = hv[nt] ? a.qscale[(bh0 + hs) * 4 + 0] : 0.f;
-        bh[nt] = hv[nt] ? a.qscale[(bh0 + hs) * 4 + 1] : 0.f;
+        const bool ok = hs < G;
+        ah[nt] = ok ? a.qscale[(bh0 + hs) * 4 + 0] : 0.f;
+        bh[nt] = ok ? a.qscale[(bh0 + hs) * 4 + 1] : 0.f;
+        hbias[nt] = ok ? 0.f : -INFINITY;
       }
       float s_cap = 0.f, lam = 0.f, inv = 0.f;
       int since_flush = 0;
@@ -527,20 +568,30 @@ __global__ void __launch_bounds__(kMmaWarps * 32, kCtasPerSm) decode_mma_kernel(
       const int nmy = (slot_ok && alive && nsteps > warp) ? (nsteps - warp + kMmaWarps - 1) / kMmaWarps : 0;
       const int32_t* trow = a.block_table + (size_t)(slot_ok ? slot : 0) * a.mbps;
 
-      // issue local step j into ring position it + j (lane 0 only)
+      // lane 0: issue local step j into ring position it + j, recording how
+      // many valid tokens each of its two blocks holds
       auto issue = [&](int j) {
-        const int k = warp + kMmaWarps * j;
-        const int pa = p0 + 2 * k;
+        const int pa = p0 + 2 * (warp + kMmaWarps * j);
         const uint32_t stg = (it + j) % kStages;
         int blk[2];
-        uint32_t bytes = 0;
+        uint32_t bytes = 0, info = 0;
 #pragma unroll
         for (int bb = 0; bb < 2; ++bb) {
           const int pi = pa + bb;
-          blk[bb] = pi < p1 ? trow[pi] : -1;
-          if (blk[bb] >= a.num_blocks) blk[bb] = -1;
-          if (blk[bb] >= 0) bytes += kBlockHeadBytes;
+          blk[bb] = -1;
+          if (pi < p1) {
+            blk[bb] = trow[pi];
+            if (blk[bb] < 0 || blk[bb] >= a.num_blocks) {
+              raise_flag(a.status, OKV_DEV_BAD_BLOCK);
+              blk[bb] = -1;
+            }
+          }
+          if (blk[bb] >= 0) {
+            bytes += kBlockHeadBytes;
+            info |= (uint32_t)min(kBlock, us.n_int2 - kBlock * pi) << (8 * bb);
+          }
         }
+        myinfo[stg] = info;
         mbar_arrive_expect_tx(&mybar[stg], bytes);
 #pragma unroll
         for (int bb = 0; bb < 2; ++bb)
@@ -550,48 +601,35 @@ __global__ void __launch_bounds__(kMmaWarps * 32, kCtasPerSm) decode_mma_kernel(
       };
       if (lane == 0)
         for (int j = 0; j < min(kStages, nmy); ++j) issue(j);
+      __syncwarp();
 
       int done = 0;
       for (int j = 0; j < nmy; ++j) {
         const uint32_t stg = (it + j) % kStages;
         const uint32_t par = ((it + j) / kStages) & 1u;
-        const bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(&mybar[stg], par));
-        if (!ok) {
+        if (!__all_sync(0xffffffffu, mbar_wait_bounded(&mybar[stg], par))) {
           if (lane == 0) raise_flag(a.status, OKV_DEV_TIMEOUT);
           alive = false;
           break;
         }
-        const int k = warp + kMmaWarps * j;
-        const int pa = p0 + 2 * k;
-        int ntok[2];
-#pragma unroll
-        for (int bb = 0; bb < 2; ++bb) {
-          const int pi = pa + bb;
-          int bid = pi < p1 ? trow[pi] : -1;
-          if (pi < p1 && (bid < 0 || bid >= a.num_blocks)) {
-            if (lane == 0) raise_flag(a.status, OKV_DEV_BAD_BLOCK);
-            bid = -1;
-          }
-          ntok[bb] = bid >= 0 ? min(kBlock, us.n_int2 - kBlock * pi) : 0;
-        }
+        const uint32_t info = myinfo[stg];
+        const int n0 = (int)(info & 0xffu), n1 = (int)(info >> 8);
+        const bool full = (n0 == kBlock) && (n1 == kBlock);
         const unsigned char* s0 = myst + stg * kStageBytes;
+        const unsigned char* s1 = s0 + kBlockHeadBytes;
 
-        // scores
+        // ---- scores: D[tok][col] for both blocks
         int dq[2][NT][4];
         uint32_t smk[4], smv[4];
 #pragma unroll
         for (int bb = 0; bb < 2; ++bb) {
-          const unsigned char* sb = s0 + bb * kBlockHeadBytes;
+          const unsigned char* sb = bb ? s1 : s0;
           const uint2 wa = *reinterpret_cast<const uint2*>(sb + kKcOff + 32 * g + 8 * t);
           const uint2 wb = *reinterpret_cast<const uint2*>(sb + kKcOff + 32 * (g + 8) + 8 * t);
           smk[2 * bb] = *reinterpret_cast<const uint32_t*>(sb + kKsmOff + 4 * g);
           smk[2 * bb + 1] = *reinterpret_cast<const uint32_t*>(sb + kKsmOff + 4 * (g + 8));
           smv[2 * bb] = *reinterpret_cast<const uint32_t*>(sb + kVsmOff + 4 * g);
           smv[2 * bb + 1] = *reinterpret_cast<const uint32_t*>(sb + kVsmOff + 4 * (g + 8));
-#pragma unroll
-          for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-            for (int jj = 0; jj < 4; ++jj) dq[bb][nt][jj] = 0;
 #pragma unroll
           for (int s = 0; s < 4; ++s) {
             uint32_t af[4];
@@ -600,20 +638,24 @@ __global__ void __launch_bounds__(kMmaWarps * 32, kCtasPerSm) decode_mma_kernel(
             af[2] = (wa.y >> (2 * s)) & kM2;
             af[3] = (wb.y >> (2 * s)) & kM2;
 #pragma unroll
-            for (int nt = 0; nt < NT; ++nt) mma_u8s8(dq[bb][nt], af, qb[nt][2 * s], qb[nt][2 * s + 1]);
+            for (int nt = 0; nt < NT; ++nt) {
+              if (s == 0) mma_u8s8_z(dq[bb][nt], af, qb[nt][0], qb[nt][1]);
+              else mma_u8s8(dq[bb][nt], af, qb[nt][2 * s], qb[nt][2 * s + 1]);
+            }
           }
         }
         // token e of this lane: block e>>1, row g + 8*(e&1)
+        float sk[4], mk[4], sv[4], mv[4];
         bool tv[4];
-        float sv[4], mv[4];
-        float smax = 0.f;
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          tv[e] = (g + 8 * (e & 1)) < ntok[e >> 1];
-          sv[e] = lo_half(smv[e]);
-          mv[e] = hi_half(smv[e]);
-          if (tv[e]) smax = fmaxf(smax, sv[e]);
+          const float2 k2 = __half22float2(*reinterpret_cast<const __half2*>(&smk[e]));
+          const float2 v2 = __half22float2(*reinterpret_cast<const __half2*>(&smv[e]));
+          sk[e] = k2.x; mk[e] = k2.y; sv[e] = v2.x; mv[e] = v2.y;
+          tv[e] = full || ((g + 8 * (e & 1)) < ((e >> 1) ? n1 : n0));
         }
+        float smax = fmaxf(fmaxf(tv[0] ? sv[0] : 0.f, tv[1] ? sv[1] : 0.f),
+                           fmaxf(tv[2] ? sv[2] : 0.f, tv[3] ? sv[3] : 0.f));
         smax = fmaxf(smax, __shfl_xor_sync(0xffffffffu, smax, 4));
         smax = fmaxf(smax, __shfl_xor_sync(0xffffffffu, smax, 8));
         smax = fmaxf(smax, __shfl_xor_sync(0xffffffffu, smax, 16));
@@ -625,6 +667,9 @@ __global__ void __launch_bounds__(kMmaWarps * 32, kCtasPerSm) decode_mma_kernel(
           lam = 65535.f / s_cap;
           inv = s_cap / 65535.f;
         }
+        float svl[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) svl[e] = tv[e] ? sv[e] * lam : 0.f;
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
           float sc[4];
@@ -632,8 +677,9 @@ __global__ void __launch_bounds__(kMmaWarps * 32, kCtasPerSm) decode_mma_kernel(
           for (int e = 0; e < 4; ++e) {
             const int bb = e >> 1, r = 2 * (e & 1);
             const int raw = dq[bb][nt][r] * 256 + dq[bb][nt][r + 1];
-            sc[e] = (tv[e] && hv[nt]) ? fmaf(lo_half(smk[e]) * ah[nt], (float)raw, hi_half(smk[e]) * bh[nt])
-                                       : -INFINITY;
+            float x = fmaf(sk[e] * ah[nt], (float)raw, mk[e] * bh[nt]);
+            if constexpr (G < 4) x += hbias[nt];
+            sc[e] = tv[e] ? x : -INFINITY;
           }
           float bm = fmaxf(fmaxf(sc[0], sc[1]), fmaxf(sc[2], sc[3]));
           bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 4));
@@ -641,27 +687,27 @@ __global__ void __launch_bounds__(kMmaWarps * 32, kCtasPerSm) decode_mma_kernel(
           bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 16));
           if (bm > st.m[nt]) {
             mma_flush(st, nt, inv);
-            const float alpha = exp2f(st.m[nt] - bm);
+            const float alpha = fast_ex2(st.m[nt] - bm);  // ex2(-inf) = 0 on the first step
 #pragma unroll
             for (int i = 0; i < 16; ++i) st.acc[nt][i] *= alpha;
             st.l[nt] *= alpha;
             st.msum[nt] *= alpha;
             st.m[nt] = bm;
           }
+          const float mref = st.m[nt] == -INFINITY ? 0.f : st.m[nt];
           uint16_t* prow = myp + (4 * nt + t) * kPStride;
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const float p = (sc[e] == -INFINITY) ? 0.f : exp2f(sc[e] - st.m[nt]);
+            const float p = fast_ex2(sc[e] - mref);  // 0 for masked tokens
             st.l[nt] += p;
             st.msum[nt] = fmaf(p, mv[e], st.msum[nt]);
-            const uint32_t pi = (p > 0.f) ? min(__float2uint_rn(p * sv[e] * lam), 65535u) : 0u;
-            prow[16 * (e >> 1) + g + 8 * (e & 1)] = (uint16_t)pi;
+            prow[16 * (e >> 1) + g + 8 * (e & 1)] = (uint16_t)cvt_u16_sat(p * svl[e]);
           }
         }
         __syncwarp();
-        // values
+        // ---- values: acci[mt] += C_V (masked, row scale 4^f) . P'
         const uint4 v0 = *reinterpret_cast<const uint4*>(s0 + kVcOff + 16 * lane);
-        const uint4 v1 = *reinterpret_cast<const uint4*>(s0 + kBlockHeadBytes + kVcOff + 16 * lane);
+        const uint4 v1 = *reinterpret_cast<const uint4*>(s1 + kVcOff + 16 * lane);
         const uint32_t va[4] = {v0.x, v0.y, v0.z, v0.w};
         const uint32_t vb[4] = {v1.x, v1.y, v1.z, v1.w};
         uint32_t pb0[NT], pb1[NT];
@@ -670,22 +716,19 @@ __global__ void __launch_bounds__(kMmaWarps * 32, kCtasPerSm) decode_mma_kernel(
           const uint16_t* prow = myp + (4 * nt + (g >> 1)) * kPStride;
           const uint2 x0 = *reinterpret_cast<const uint2*>(prow + 4 * t);
           const uint2 x1 = *reinterpret_cast<const uint2*>(prow + 16 + 4 * t);
-          const uint32_t sel = (g & 1) ? 0x6420u : 0x7531u;  // lo limb = low byte, hi limb = high byte
+          const uint32_t sel = (g & 1) ? 0x6420u : 0x7531u;  // odd column: low byte (lo limb)
           pb0[nt] = prmt(x0.x, x0.y, sel);
           pb1[nt] = prmt(x1.x, x1.y, sel);
         }
 #pragma unroll
         for (int mt = 0; mt < 8; ++mt) {
-          const int jw = mt >> 1, f0 = 4 * (mt & 1);
-          uint32_t af[4];
-          af[0] = (va[jw] >> f0) & kM2;
-          af[1] = (va[jw] >> (f0 + 2)) & kM2;
-          af[2] = (vb[jw] >> f0) & kM2;
-          af[3] = (vb[jw] >> (f0 + 2)) & kM2;
+          const int jw = mt >> 1;
+          const uint32_t m0 = kM2 << (4 * (mt & 1)), m1 = m0 << 2;
+          const uint32_t af[4] = {va[jw] & m0, va[jw] & m1, vb[jw] & m0, vb[jw] & m1};
 #pragma unroll
           for (int nt = 0; nt < NT; ++nt) mma_u8u8(st.acci[nt][mt], af, pb0[nt], pb1[nt]);
         }
-        if (++since_flush >= 128) {
+        if (++since_flush >= 96) {
 #pragma unroll
           for (int nt = 0; nt < NT; ++nt) mma_flush(st, nt, inv);
           since_flush = 0;
@@ -700,8 +743,157 @@ __global__ void __launch_bounds__(kMmaWarps * 32, kCtasPerSm) decode_mma_kernel(
       }
       it += (uint32_t)nmy;
 #pragma unroll
+      for (int nt = 0; nt < NT; ++nt) mma_flush(st, nt, inv);
+
+      // ---------------- fp16 window: chunks ci = warp, warp + NW, ... ----------------
+      const int nchunk = (l0 == 0 && us.win_cost > 0 && slot_ok) ? (us.n_win + 15) / 16 : 0;
+      if (warp < nchunk) {
+        const __half* kr = a.ring + (((size_t)slot * a.hkv + hk) * 2 + 0) * kWin * kD;
+        const __half* vr = a.ring + (((size_t)slot * a.hkv + hk) * 2 + 1) * kWin * kD;
+        unsigned char* tile = myst;                                   // 16 rows x 256 B, swizzled
+        float* pw = reinterpret_cast<float*>(myst + 4096);            // [HP][16]
+        float* wo = reinterpret_cast<float*>(myst + 4096 + HP * 64);  // [G][128]
+        uint32_t qh[NT][16];
+        float wsc[NT], wm[NT], wl[NT];
+        float wacc[NT][8][4];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          const int hcol = 4 * nt + (g >> 1);
+          if (hcol < G) {
+            const uint4* src = reinterpret_cast<const uint4*>(a.qwin + ((bh0 + hcol) * 2 + (g & 1)) * kD + 32 * t);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const uint4 x = src[i];
+              qh[nt][4 * i] = x.x; qh[nt][4 * i + 1] = x.y; qh[nt][4 * i + 2] = x.z; qh[nt][4 * i + 3] = x.w;
+            }
+          } else {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) qh[nt][i] = 0u;
+          }
+          const int hs = 4 * nt + t;
+          wsc[nt] = hs < G ? a.qscale[(bh0 + hs) * 4 + 2] * (kInvSqrtD * kLog2e) : 0.f;
+          wm[nt] = -INFINITY;
+          wl[nt] = 0.f;
+#pragma unroll
+          for (int mt = 0; mt < 8; ++mt)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) wacc[nt][mt][i] = 0.f;
+        }
+        for (int ci = warp; ci < nchunk; ci += kMmaWarps) {
+          const int r0 = 16 * ci;
+          // stage the V rows (swizzled 16-byte chunks) for the transposing loads
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const int q = lane + 32 * k, row = q >> 4, col = q & 15;
+            uint4 x = make_uint4(0, 0, 0, 0);
+            if (r0 + row < us.n_win) x = *reinterpret_cast<const uint4*>(vr + (size_t)(r0 + row) * kD + 8 * col);
+            *reinterpret_cast<uint4*>(tile + row * 256 + ((col ^ (row & 7)) << 4)) = x;
+          }
+          // scores of ring rows r0 + g and r0 + g + 8
+          uint32_t ka[16], kb[16];
+          const bool va_ = r0 + g < us.n_win, vb_ = r0 + g + 8 < us.n_win;
+          const uint4* ra = reinterpret_cast<const uint4*>(kr + (size_t)(r0 + g) * kD + 32 * t);
+          const uint4* rb = reinterpret_cast<const uint4*>(kr + (size_t)(r0 + g + 8) * kD + 32 * t);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const uint4 x = va_ ? ra[i] : make_uint4(0, 0, 0, 0);
+            const uint4 y = vb_ ? rb[i] : make_uint4(0, 0, 0, 0);
+            ka[4 * i] = x.x; ka[4 * i + 1] = x.y; ka[4 * i + 2] = x.z; ka[4 * i + 3] = x.w;
+            kb[4 * i] = y.x; kb[4 * i + 1] = y.y; kb[4 * i + 2] = y.z; kb[4 * i + 3] = y.w;
+          }
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) {
+            float d[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks) {
+              const uint32_t af[4] = {ka[2 * ks], kb[2 * ks], ka[2 * ks + 1], kb[2 * ks + 1]};
+              mma_f16(d, af, qh[nt][2 * ks], qh[nt][2 * ks + 1]);
+            }
+            const int hs = 4 * nt + t;
+            const float s_a = (va_ && hs < G) ? (d[0] + d[1]) * wsc[nt] : -INFINITY;
+            const float s_b = (vb_ && hs < G) ? (d[2] + d[3]) * wsc[nt] : -INFINITY;
+            float bm = fmaxf(s_a, s_b);
+            bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 4));
+            bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 8));
+            bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 16));
+            const float mnew = fmaxf(wm[nt], bm);
+            const float mref = mnew == -INFINITY ? 0.f : mnew;
+            const float alpha = fast_ex2(wm[nt] - mref);
+            const float pa_ = fast_ex2(s_a - mref), pb_ = fast_ex2(s_b - mref);
+            wl[nt] = wl[nt] * alpha + pa_ + pb_;
+            wm[nt] = mnew;
+            pw[(4 * nt + t) * 16 + g] = pa_;
+            pw[(4 * nt + t) * 16 + g + 8] = pb_;
+            // D rows of this lane hold heads 4nt + t: rescale them
+#pragma unroll
+            for (int mt = 0; mt < 8; ++mt)
+#pragma unroll
+              for (int i = 0; i < 4; ++i) wacc[nt][mt][i] *= alpha;
+          }
+          __syncwarp();
+          // P.V: A = V^T (channels x tokens) by transposing loads, B = p as fp16 hi/lo
+          uint32_t b0[NT], b1[NT];
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) {
+            const float* prw = pw + (4 * nt + (g >> 1)) * 16;
+            const float2 pa2 = *reinterpret_cast<const float2*>(prw + 2 * t);
+            const float2 pb2 = *reinterpret_cast<const float2*>(prw + 2 * t + 8);
+            const __half2 ha = __floats2half2_rn(pa2.x, pa2.y), hb = __floats2half2_rn(pb2.x, pb2.y);
+            __half2 ra2 = ha, rb2 = hb;
+            if (g & 1) {
+              const float2 fa = __half22float2(ha), fb = __half22float2(hb);
+              ra2 = __floats2half2_rn(pa2.x - fa.x, pa2.y - fa.y);
+              rb2 = __floats2half2_rn(pb2.x - fb.x, pb2.y - fb.y);
+            }
+            b0[nt] = *reinterpret_cast<uint32_t*>(&ra2);
+            b1[nt] = *reinterpret_cast<uint32_t*>(&rb2);
+          }
+          {
+            const int mi = lane >> 3, ri = lane & 7;
+            const int tok = ri + 8 * (mi >> 1);
+#pragma unroll
+            for (int mt = 0; mt < 8; ++mt) {
+              const int col = 2 * mt + (mi & 1);
+              uint32_t af[4];
+              ldmatrix_x4_trans(af, tile + tok * 256 + ((col ^ (tok & 7)) << 4));
+#pragma unroll
+              for (int nt = 0; nt < NT; ++nt) mma_f16(wacc[nt][mt], af, b0[nt], b1[nt]);
+            }
+          }
+          __syncwarp();
+        }
+        // window o' per (head, channel) through shared memory, then fold into the block state
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          const int hs = 4 * nt + t;
+          if (hs < G) {
+#pragma unroll
+            for (int mt = 0; mt < 8; ++mt) {
+              wo[hs * kD + 16 * mt + g] = wacc[nt][mt][0] + wacc[nt][mt][1];
+              wo[hs * kD + 16 * mt + g + 8] = wacc[nt][mt][2] + wacc[nt][mt][3];
+            }
+          }
+        }
+        __syncwarp();
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          const int hs = 4 * nt + t;
+          if (hs < G) {
+            const float M = fmaxf(st.m[nt], wm[nt]);
+            const float mref = M == -INFINITY ? 0.f : M;
+            const float ab = fast_ex2(st.m[nt] - mref), aw = fast_ex2(wm[nt] - mref);
+            const float* src = wo + hs * kD + 16 * g;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) st.acc[nt][i] = fmaf(st.acc[nt][i], ab, src[i] * aw);
+            st.l[nt] = fmaf(st.l[nt], ab, wl[nt] * aw);
+            st.msum[nt] *= ab;
+            st.m[nt] = M;
+          }
+        }
+      }
+      __syncthreads();  // every warp is done with its ring: the rings become merge buffers
+#pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
-        mma_flush(st, nt, inv);
         float l = st.l[nt], ms = st.msum[nt];
 #pragma unroll
         for (int o = 4; o < 32; o <<= 1) {
@@ -712,142 +904,27 @@ __global__ void __launch_bounds__(kMmaWarps * 32, kCtasPerSm) decode_mma_kernel(
         if (hs < G) {
           float* dst = mo + ((size_t)warp * G + hs) * kD + 16 * g;
 #pragma unroll
-          for (int i = 0; i < 16; ++i) dst[i] = st.acc[nt][i] + ms;
+          for (int i = 0; i < 16; i += 4)
+            *reinterpret_cast<float4*>(dst + i) =
+                make_float4(st.acc[nt][i] + ms, st.acc[nt][i + 1] + ms, st.acc[nt][i + 2] + ms, st.acc[nt][i + 3] + ms);
           if (g == 0) {
             ml[(warp * G + hs) * 2 + 0] = st.m[nt];
             ml[(warp * G + hs) * 2 + 1] = l;
           }
         }
       }
-
-      // ---------------- fp16 window (warp 0, if this CTA owns it) ----------------
-      if (warp == 0) {
-        float wm[NT], wl[NT], wo[G][4];
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) { wm[nt] = -INFINITY; wl[nt] = 0.f; }
-#pragma unroll
-        for (int hh = 0; hh < G; ++hh)
-#pragma unroll
-          for (int i = 0; i < 4; ++i) wo[hh][i] = 0.f;
-        if (l0 == 0 && us.win_cost > 0 && slot_ok) {
-          const __half* kr = a.ring + (((size_t)slot * a.hkv + hk) * 2 + 0) * kWin * kD;
-          const __half* vr = a.ring + (((size_t)slot * a.hkv + hk) * 2 + 1) * kWin * kD;
-          // query halves of this lane's B column, channels 32t .. 32t+31
-          uint32_t qh[NT][16];
-          float wsc[NT];
-#pragma unroll
-          for (int nt = 0; nt < NT; ++nt) {
-            const int hcol = 4 * nt + (g >> 1);
-            if (hcol < G) {
-              const uint4* src = reinterpret_cast<const uint4*>(a.qwin + ((bh0 + hcol) * 2 + (g & 1)) * kD + 32 * t);
-#pragma unroll
-              for (int i = 0; i < 4; ++i) {
-                const uint4 x = src[i];
-                qh[nt][4 * i] = x.x; qh[nt][4 * i + 1] = x.y; qh[nt][4 * i + 2] = x.z; qh[nt][4 * i + 3] = x.w;
-              }
-            } else {
-#pragma unroll
-              for (int i = 0; i < 16; ++i) qh[nt][i] = 0u;
-            }
-            const int hs = 4 * nt + t;
-            wsc[nt] = hs < G ? a.qscale[(bh0 + hs) * 4 + 0] : 0.f;
-          }
-          for (int r0 = 0; r0 < us.n_win; r0 += 16) {
-            // scores of ring rows r0 + g and r0 + g + 8
-            uint32_t ka[16], kb[16];
-            const bool va_ = r0 + g < us.n_win, vb_ = r0 + g + 8 < us.n_win;
-            const uint4* ra = reinterpret_cast<const uint4*>(kr + (size_t)(r0 + g) * kD + 32 * t);
-            const uint4* rb = reinterpret_cast<const uint4*>(kr + (size_t)(r0 + g + 8) * kD + 32 * t);
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              const uint4 x = va_ ? ra[i] : make_uint4(0, 0, 0, 0);
-              const uint4 y = vb_ ? rb[i] : make_uint4(0, 0, 0, 0);
-              ka[4 * i] = x.x; ka[4 * i + 1] = x.y; ka[4 * i + 2] = x.z; ka[4 * i + 3] = x.w;
-              kb[4 * i] = y.x; kb[4 * i + 1] = y.y; kb[4 * i + 2] = y.z; kb[4 * i + 3] = y.w;
-            }
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt) {
-              float d[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-              for (int ks = 0; ks < 8; ++ks) {
-                const uint32_t af[4] = {ka[2 * ks], kb[2 * ks], ka[2 * ks + 1], kb[2 * ks + 1]};
-                mma_f16(d, af, qh[nt][2 * ks], qh[nt][2 * ks + 1]);
-              }
-              const int hs = 4 * nt + t;
-              const float s_a = (va_ && hs < G) ? (d[0] + d[1]) * wsc[nt] : -INFINITY;
-              const float s_b = (vb_ && hs < G) ? (d[2] + d[3]) * wsc[nt] : -INFINITY;
-              float bm = fmaxf(s_a, s_b);
-              bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 4));
-              bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 8));
-              bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 16));
-              const float mnew = fmaxf(wm[nt], bm);
-              const float alpha = (mnew == -INFINITY) ? 1.f : exp2f(wm[nt] - mnew);
-              const float pa_ = (s_a == -INFINITY) ? 0.f : exp2f(s_a - mnew);
-              const float pb_ = (s_b == -INFINITY) ? 0.f : exp2f(s_b - mnew);
-              wl[nt] = wl[nt] * alpha + pa_ + pb_;
-              wm[nt] = mnew;
-              if (hs < G) {
-                pw[g * G + hs] = pa_;
-                pw[(g + 8) * G + hs] = pb_;
-              }
-              // rescale this n-tile's heads in the P.V accumulators (lane owns 4 channels of every head)
-#pragma unroll
-              for (int q4 = 0; q4 < 4; ++q4) {
-                const float al = __shfl_sync(0xffffffffu, alpha, q4);  // lane q4 holds head 4nt + q4
-                const int hh = 4 * nt + q4;
-                if (hh < G) {
-#pragma unroll
-                  for (int i = 0; i < 4; ++i) wo[hh][i] *= al;
-                }
-              }
-            }
-            __syncwarp();
-            const int nrow = min(16, us.n_win - r0);
-            for (int rr = 0; rr < nrow; ++rr) {
-              const uint2 w2 = *reinterpret_cast<const uint2*>(vr + (size_t)(r0 + rr) * kD + 4 * lane);
-              const float2 f0 = __half22float2(*reinterpret_cast<const __half2*>(&w2.x));
-              const float2 f1 = __half22float2(*reinterpret_cast<const __half2*>(&w2.y));
-#pragma unroll
-              for (int hh = 0; hh < G; ++hh) {
-                const float p = pw[rr * G + hh];
-                wo[hh][0] = fmaf(p, f0.x, wo[hh][0]);
-                wo[hh][1] = fmaf(p, f0.y, wo[hh][1]);
-                wo[hh][2] = fmaf(p, f1.x, wo[hh][2]);
-                wo[hh][3] = fmaf(p, f1.y, wo[hh][3]);
-              }
-            }
-            __syncwarp();
-          }
-        }
-        // the window's state fills merge slot kMmaWarps (lane owns channels 4*lane .. +3)
-#pragma unroll
-        for (int hh = 0; hh < G; ++hh) {
-          float* dst = mo + ((size_t)kMmaWarps * G + hh) * kD + 4 * lane;
-#pragma unroll
-          for (int i = 0; i < 4; ++i) dst[i] = wo[hh][i];
-        }
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-          float l = wl[nt];
-#pragma unroll
-          for (int o = 4; o < 32; o <<= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
-          const int hs = 4 * nt + t;
-          if (hs < G && g == 0) {
-            ml[(kMmaWarps * G + hs) * 2 + 0] = wm[nt];
-            ml[(kMmaWarps * G + hs) * 2 + 1] = l;
-          }
-        }
-      }
       __syncthreads();
-      // merge the warps (and the window) into this CTA's partial for unit u
+      // merge the warps into this CTA's partial for unit u
       float* dstp = a.part + ((size_t)(c + u) * G) * kPartStride;
       for (int i = threadIdx.x; i < G * kD; i += blockDim.x) {
         const int hh = i / kD, ch = i % kD;
         float mx = -INFINITY;
-        for (int w = 0; w <= kMmaWarps; ++w) mx = fmaxf(mx, ml[(w * G + hh) * 2]);
+#pragma unroll
+        for (int w = 0; w < kMmaWarps; ++w) mx = fmaxf(mx, ml[(w * G + hh) * 2]);
         float o = 0.f, l = 0.f;
         if (mx != -INFINITY) {
-          for (int w = 0; w <= kMmaWarps; ++w) {
+#pragma unroll
+          for (int w = 0; w < kMmaWarps; ++w) {
             const float mw = ml[(w * G + hh) * 2];
             if (mw == -INFINITY) continue;
             const float sc = exp2f(mw - mx);

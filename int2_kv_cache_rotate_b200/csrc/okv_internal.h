@@ -33,7 +33,7 @@ struct DecodePlan {
 };
 constexpr int kPartStride = 132;  // o'[128], m, l, 2 spare
 constexpr int kWinCost = 16;      // cost of a unit's window in block units
-constexpr int kCtasPerSm = 3;     // resident split-K CTAs per SM
+constexpr int kCtasPerSm = 4;     // resident split-K CTAs per SM
 
 DecodePlan make_decode_plan(int batch, int hq, int hkv);
 
