@@ -7,13 +7,14 @@
 namespace okv {
 
 // ---------------------------------------------------------------------------
-// Work partition.  Unit u = (batch entry b, KV head hk).  With L tokens in the
-// cache, the unit costs ceil(max(L-W,0)/16) INT2 blocks plus kWinCost for its
-// fp16 window (if L > 0).  Units are laid end to end in "cost space"; split-K
-// CTA c takes the contiguous range [c*total/NC, (c+1)*total/NC).  Inside a
-// unit, cost positions [0, kWinCost) stand for the window and the rest for the
-// blocks in order.  A (unit, CTA) pair writes partial slot c + u: distinct
-// for distinct pairs because CTAs and units are both contiguous.
+// Work partition.  Batch entry b with L tokens costs ceil(max(L-W,0)/16)
+// blocks (every KV head of a block is one contiguous run) plus kWinCost for
+// its fp16 window (if L > 0).  Entries are laid end to end in "cost space";
+// split-K CTA c takes the contiguous range [c*total/NC, (c+1)*total/NC).
+// Inside an entry, cost positions [0, kWinCost) stand for the window and the
+// rest for the blocks in order.  A (entry, CTA) pair writes partial slot
+// c + b (all query heads): distinct for distinct pairs because CTAs and
+// entries are both contiguous.
 // ---------------------------------------------------------------------------
 struct UnitShape {
   int len;      // tokens in the cache
@@ -35,7 +36,7 @@ __device__ __forceinline__ UnitShape unit_shape(int len) {
   return s;
 }
 
-// first CTA whose range contains cost position x (x < total)
+// CTA whose range contains cost position x (x < total)
 __device__ __forceinline__ int cta_of(long long x, long long total, int nc) {
   const long long num = (x + 1) * (long long)nc;
   return (int)((num + total - 1) / total) - 1;
@@ -67,31 +68,42 @@ struct DecodeArgs {
   int8_t* qlimb;     // [B][Hq][2][128]
   float* qscale;     // [B][Hq][4]: score scale, min-term scale, sigma, sum
   __half* qwin;      // [B][Hq][2][128]: q~/sigma as fp16 hi, lo (natural channel order)
-  int32_t* prefix;   // [B+1] cost prefix over batch entries (units of b are consecutive)
-  float* part;       // [(NC + NU)][G][kPartStride]
+  int32_t* prefix;   // [B+1] cost prefix over batch entries
+  float* part;       // [(NC + B)][Hq][kPartStride]
   int batch, hq, hkv, g, nc, num_blocks, num_slots, mbps;
 };
 
+// split-K CTA count actually used: with fewer cost units than CTAs only the
+// first `total` take work, so every working CTA owns a non-empty range
+__device__ __forceinline__ int working_ctas(const DecodeArgs& a, long long total) {
+  return (int)min((long long)a.nc, total);
+}
+
 // ---------------------------------------------------------------------------
-// Kernel 1: q~ = q R_K for every (b, query head), plus the cost prefix.
+// Kernel 1: q~ = q R_K for every query head, in CTAs of one (b, KV head) that
+// load U_K once (warp w holds rows 16w..16w+15, lane l columns 4l..4l+3, all
+// loads in flight together), plus the cost prefix (CTA (0,0)).
+// Also emits the query in the two forms the split-K kernel consumes:
+// signed 8-bit limbs in MMA-fragment order and fp16 hi/lo halves.
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(128) qrot_kernel(DecodeArgs a) {
-  __shared__ float red[4][kD];
-  const int b = blockIdx.x, h = blockIdx.y;
+constexpr int kPrepThreads = 256;
+
+__global__ void __launch_bounds__(kPrepThreads) qrot_kernel(DecodeArgs a) {
+  extern __shared__ float red[];  // [G][8][128]
+  const int b = blockIdx.x, hk = blockIdx.y;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  if (b == 0 && h == 0) {
-    // cost prefix over batch entries: thread-serial chunks + one pass over chunk sums
-    __shared__ int chunk_sum[128];
-    const int per = (a.batch + 127) / 128;
+  const int G = a.g;
+  if (b == 0 && hk == 0) {
+    __shared__ int chunk_sum[kPrepThreads];
+    const int per = (a.batch + kPrepThreads - 1) / kPrepThreads;
     const int lo = threadIdx.x * per, hi = min(a.batch, lo + per);
     int s = 0;
-    for (int i = lo; i < hi; ++i)
-      s += a.hkv * unit_shape(clamp_len(a.context_lens, i, a.mbps, a.status, true)).cost;
+    for (int i = lo; i < hi; ++i) s += unit_shape(clamp_len(a.context_lens, i, a.mbps, a.status, true)).cost;
     chunk_sum[threadIdx.x] = s;
     __syncthreads();
     if (threadIdx.x == 0) {
       int run = 0;
-      for (int i = 0; i < 128; ++i) {
+      for (int i = 0; i < kPrepThreads; ++i) {
         const int c = chunk_sum[i];
         chunk_sum[i] = run;
         run += c;
@@ -102,57 +114,82 @@ __global__ void __launch_bounds__(128) qrot_kernel(DecodeArgs a) {
     int run = chunk_sum[threadIdx.x];
     for (int i = lo; i < hi; ++i) {
       a.prefix[i] = run;
-      run += a.hkv * unit_shape(clamp_len(a.context_lens, i, a.mbps, a.status, false)).cost;
+      run += unit_shape(clamp_len(a.context_lens, i, a.mbps, a.status, false)).cost;
     }
-    __syncthreads();
   }
-  float y[4];
-  const __nv_bfloat16* src = a.q + ((size_t)b * a.hq + h) * kD;
-  rotate_cta(src, a.u_k + (size_t)(h / a.g) * kD * kD, red, y);
-  if (warp != 0) return;
-  const int r = rev5(lane);
-  const size_t bh = (size_t)b * a.hq + h;
-  float* dst = a.qrot + bh * kD + 4 * r;
-  *reinterpret_cast<float4*>(dst) = make_float4(y[0], y[2], y[1], y[3]);
-
-  // Integer limbs for the tensor-core score tiles: Q = rint(q~/sigma) in
-  // [-32000, 32000] = 256*hi + lo with hi, lo signed 8-bit.  Bytes are stored
-  // in MMA-fragment order: channel c = 32t + 16h + 4i + s goes to position
-  // 32t + 8s + 4h + i, so a lane of quad t reads its 32 bytes in one go.
-  const float zc[4] = {y[0], y[2], y[1], y[3]};  // rotated channels 4r + e
-  float amax = fmaxf(fmaxf(fabsf(y[0]), fabsf(y[1])), fmaxf(fabsf(y[2]), fabsf(y[3])));
-  amax = warp_max(amax);
-  const float sum = warp_sum((y[0] + y[1]) + (y[2] + y[3]));
-  const float sigma = amax > 0.f ? amax / 32000.f : 1.f;
-  const float inv = amax > 0.f ? 32000.f / amax : 0.f;
-  int8_t* lim = a.qlimb + bh * 2 * kD;
-  __half* qw = a.qwin + bh * 2 * kD;
+  const float* U = a.u_k + (size_t)hk * kD * kD;
+  float4 u[16];
 #pragma unroll
-  for (int e = 0; e < 4; ++e) {
-    const int c = 4 * r + e;
-    const float x = zc[e] * inv;
-    const int q = max(-32000, min(32000, __float2int_rn(x)));
-    const int hi = ((q + 32896) >> 8) - 128;
-    const int lo = q - 256 * hi;
-    const int pos = (c >> 5) * 32 + (c & 3) * 8 + ((c >> 4) & 1) * 4 + ((c >> 2) & 3);
-    lim[pos] = (int8_t)hi;
-    lim[kD + pos] = (int8_t)lo;
-    const __half hx = __float2half_rn(x);
-    qw[c] = hx;
-    qw[kD + c] = __float2half_rn(x - __half2float(hx));
+  for (int r = 0; r < 16; ++r) u[r] = __ldg(reinterpret_cast<const float4*>(U + (size_t)(16 * warp + r) * kD) + lane);
+  for (int gg = 0; gg < G; ++gg) {
+    const __nv_bfloat16* qv = a.q + ((size_t)b * a.hq + (size_t)hk * G + gg) * kD;
+    const float xv = __bfloat162float(qv[16 * warp + (lane & 15)]);
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int r = 0; r < 16; ++r) {
+      const float x = __shfl_sync(0xffffffffu, xv, r);
+      acc.x = fmaf(x, u[r].x, acc.x);
+      acc.y = fmaf(x, u[r].y, acc.y);
+      acc.z = fmaf(x, u[r].z, acc.z);
+      acc.w = fmaf(x, u[r].w, acc.w);
+    }
+    *reinterpret_cast<float4*>(red + ((size_t)gg * 8 + warp) * kD + 4 * lane) = acc;
   }
-  if (lane == 0) {
-    float4 qs4 = make_float4(sigma * (kInvSqrtD * kLog2e), sum * (kInvSqrtD * kLog2e), sigma, sum);
-    *reinterpret_cast<float4*>(a.qscale + bh * 4) = qs4;
+  __syncthreads();
+  for (int gg = warp; gg < G; gg += 8) {
+    float y[4];
+#pragma unroll
+    for (int aa = 0; aa < 4; ++aa) {
+      float s = 0.f;
+#pragma unroll
+      for (int w = 0; w < 8; ++w) s += red[((size_t)gg * 8 + w) * kD + lane + 32 * aa];
+      y[aa] = s;
+    }
+    wht128_warp(y, lane);
+#pragma unroll
+    for (int aa = 0; aa < 4; ++aa) y[aa] *= kInvSqrtD;
+    const int r = rev5(lane);
+    const size_t bh = (size_t)b * a.hq + (size_t)hk * G + gg;
+    *reinterpret_cast<float4*>(a.qrot + bh * kD + 4 * r) = make_float4(y[0], y[2], y[1], y[3]);
+    // Integer limbs for the tensor-core score tiles: Q = rint(q~/sigma) in
+    // [-32000, 32000] = 256*hi + lo with hi, lo signed 8-bit.  Bytes are stored
+    // in MMA-fragment order: channel c = 32t + 16h + 4i + s goes to position
+    // 32t + 8s + 4h + i, so a lane of quad t reads its 32 bytes in one go.
+    const float zc[4] = {y[0], y[2], y[1], y[3]};  // rotated channels 4r + e
+    float amax = fmaxf(fmaxf(fabsf(y[0]), fabsf(y[1])), fmaxf(fabsf(y[2]), fabsf(y[3])));
+    amax = warp_max(amax);
+    const float sum = warp_sum((y[0] + y[1]) + (y[2] + y[3]));
+    const float sigma = amax > 0.f ? amax / 32000.f : 1.f;
+    const float inv = amax > 0.f ? 32000.f / amax : 0.f;
+    int8_t* lim = a.qlimb + bh * 2 * kD;
+    __half* qw = a.qwin + bh * 2 * kD;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int c = 4 * r + e;
+      const float x = zc[e] * inv;
+      const int q = max(-32000, min(32000, __float2int_rn(x)));
+      const int hi = ((q + 32896) >> 8) - 128;
+      const int lo = q - 256 * hi;
+      const int pos = (c >> 5) * 32 + (c & 3) * 8 + ((c >> 4) & 1) * 4 + ((c >> 2) & 3);
+      lim[pos] = (int8_t)hi;
+      lim[kD + pos] = (int8_t)lo;
+      const __half hx = __float2half_rn(x);
+      qw[c] = hx;
+      qw[kD + c] = __float2half_rn(x - __half2float(hx));
+    }
+    if (lane == 0) {
+      float4 qs4 = make_float4(sigma * (kInvSqrtD * kLog2e), sum * (kInvSqrtD * kLog2e), sigma, sum);
+      *reinterpret_cast<float4*>(a.qscale + bh * 4) = qs4;
+    }
   }
 }
 
 // ---------------------------------------------------------------------------
-// Kernel 2 (SIMT): split-K attention.  4 warps per CTA; a warp takes whole
-// 16-token chunks (an INT2 block, or 16 window rows) and keeps its own
-// online-softmax state; warps merge through shared memory at unit end.
-// Lane l scores token l/2 over channels 64*(l&1)..+63 and accumulates the
-// output channels 4l..4l+3 (canonical code byte l).
+// Kernel 2 (SIMT fallback, for head groupings the tensor-core kernel does not
+// cover): 4 warps per CTA; a warp takes whole 16-token chunks (an INT2 block,
+// or 16 window rows) of one KV head and keeps its own online-softmax state;
+// warps merge through shared memory.  Lane l scores token l/2 over channels
+// 64*(l&1)..+63 and accumulates output channels 4l..4l+3.
 // ---------------------------------------------------------------------------
 constexpr int kDecWarps = 4;
 
@@ -261,46 +298,37 @@ __global__ void __launch_bounds__(kDecWarps * 32) decode_simt_kernel(DecodeArgs 
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const long long total = a.prefix[a.batch];
   if (total == 0) return;
-  // with fewer cost units than CTAs, only the first `total` CTAs take work, so
-  // that every working CTA owns a non-empty range
-  const int nc = (int)min((long long)a.nc, total);
+  const int nc = working_ctas(a, total);
   const int c = blockIdx.x;
   if (c >= nc) return;
   const long long start = (long long)c * total / nc;
   const long long end = (long long)(c + 1) * total / nc;
-  // first batch entry whose units reach past `start`
   int lo = 0, hi = a.batch - 1;
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
     if (a.prefix[mid] <= start) lo = mid; else hi = mid - 1;
   }
-  int b = lo;
-  for (; b < a.batch && a.prefix[b] < end; ++b) {
+  for (int b = lo; b < a.batch && a.prefix[b] < end; ++b) {
     const UnitShape us = unit_shape(clamp_len(a.context_lens, b, a.mbps, a.status, false));
     if (us.cost == 0) continue;
     const int slot = a.seq_slot[b];
     const bool slot_ok = slot >= 0 && slot < a.num_slots;
+    const long long pu = a.prefix[b];
+    const int l0 = (int)(max(start, pu) - pu), l1 = (int)(min(end, pu + us.cost) - pu);
     for (int hk = 0; hk < a.hkv; ++hk) {
-      const long long pu = a.prefix[b] + (long long)hk * us.cost;
-      if (pu + us.cost <= start) continue;
-      if (pu >= end) break;
-      const int u = b * a.hkv + hk;
-      const int l0 = (int)(max(start, pu) - pu), l1 = (int)(min(end, pu + us.cost) - pu);
-      // rotated queries of this unit into shared memory
       __syncthreads();
       for (int i = threadIdx.x; i < G * kD; i += blockDim.x)
         qs[i] = a.qrot[((size_t)b * a.hq + hk * G) * kD + i];
       __syncthreads();
       WarpState<G> st;
 #pragma unroll
-      for (int g = 0; g < G; ++g) {
-        st.m[g] = -INFINITY;
-        st.l[g] = 0.f;
+      for (int gg = 0; gg < G; ++gg) {
+        st.m[gg] = -INFINITY;
+        st.l[gg] = 0.f;
 #pragma unroll
-        for (int j = 0; j < 4; ++j) st.o[g][j] = 0.f;
+        for (int j = 0; j < 4; ++j) st.o[gg][j] = 0.f;
       }
       if (slot_ok) {
-        // window part
         if (l0 == 0 && us.win_cost > 0) {
           const __half* kbase = a.ring + (((size_t)slot * a.hkv + hk) * 2 + 0) * kWin * kD;
           const __half* vbase = a.ring + (((size_t)slot * a.hkv + hk) * 2 + 1) * kWin * kD;
@@ -311,11 +339,10 @@ __global__ void __launch_bounds__(kDecWarps * 32) decode_simt_kernel(DecodeArgs 
             simt_chunk<G, true>(a, qs, nullptr, kbase, vbase, first + ci * kBlock, ntok, st, lane);
           }
         }
-        // INT2 blocks
         const int p0 = max(l0, us.win_cost) - us.win_cost;
         const int p1 = l1 - us.win_cost;
         for (int pi = p0 + warp; pi < p1; pi += kDecWarps) {
-          int blk = a.block_table[(size_t)slot * a.mbps + pi];
+          const int blk = a.block_table[(size_t)slot * a.mbps + pi];
           if (blk < 0 || blk >= a.num_blocks) {
             if (lane == 0) raise_flag(a.status, OKV_DEV_BAD_BLOCK);
             continue;
@@ -327,35 +354,34 @@ __global__ void __launch_bounds__(kDecWarps * 32) decode_simt_kernel(DecodeArgs 
       } else if (lane == 0 && warp == 0) {
         raise_flag(a.status, OKV_DEV_BAD_SLOT);
       }
-      // merge the warps' states
 #pragma unroll
-      for (int g = 0; g < G; ++g) {
+      for (int gg = 0; gg < G; ++gg) {
 #pragma unroll
-        for (int j = 0; j < 4; ++j) mo[(warp * G + g) * kD + 4 * lane + j] = st.o[g][j];
+        for (int j = 0; j < 4; ++j) mo[(warp * G + gg) * kD + 4 * lane + j] = st.o[gg][j];
         if (lane == 0) {
-          ml[(warp * G + g) * 2 + 0] = st.m[g];
-          ml[(warp * G + g) * 2 + 1] = st.l[g];
+          ml[(warp * G + gg) * 2 + 0] = st.m[gg];
+          ml[(warp * G + gg) * 2 + 1] = st.l[gg];
         }
       }
       __syncthreads();
-      float* dst = a.part + ((size_t)(c + u) * G) * kPartStride;
+      float* dst = a.part + ((size_t)(c + b) * a.hq + (size_t)hk * G) * kPartStride;
       for (int i = threadIdx.x; i < G * kD; i += blockDim.x) {
-        const int g = i / kD, ch = i % kD;
+        const int gg = i / kD, ch = i % kD;
         float mx = -INFINITY;
-        for (int w = 0; w < kDecWarps; ++w) mx = fmaxf(mx, ml[(w * G + g) * 2]);
+        for (int w = 0; w < kDecWarps; ++w) mx = fmaxf(mx, ml[(w * G + gg) * 2]);
         float o = 0.f, l = 0.f;
         if (mx != -INFINITY) {
           for (int w = 0; w < kDecWarps; ++w) {
-            const float mw = ml[(w * G + g) * 2];
+            const float mw = ml[(w * G + gg) * 2];
             const float sc = (mw == -INFINITY) ? 0.f : exp2f(mw - mx);
-            o = fmaf(mo[(w * G + g) * kD + ch], sc, o);
-            l = fmaf(ml[(w * G + g) * 2 + 1], sc, l);
+            o = fmaf(mo[(w * G + gg) * kD + ch], sc, o);
+            l = fmaf(ml[(w * G + gg) * 2 + 1], sc, l);
           }
         }
-        dst[g * kPartStride + ch] = o;
+        dst[gg * kPartStride + ch] = o;
         if (ch == 0) {
-          dst[g * kPartStride + 128] = mx;
-          dst[g * kPartStride + 129] = l;
+          dst[gg * kPartStride + 128] = mx;
+          dst[gg * kPartStride + 129] = l;
         }
       }
     }
@@ -363,15 +389,20 @@ __global__ void __launch_bounds__(kDecWarps * 32) decode_simt_kernel(DecodeArgs 
 }
 
 // ---------------------------------------------------------------------------
-// Kernel 2 (tensor cores): split-K attention for G = Hq/Hkv in {1, 2, 4, 8}.
+// Kernel 2 (tensor cores): split-K attention for G = Hq/Hkv in {1, 2, 4, 8}
+// and Hkv in {1, 2, 4, 8}.
 //
-// Each warp streams its own 2-block steps (32 tokens, 2 x 1152 B) through a
-// ring of bulk copies into shared memory and computes, per step:
+// A CTA of 8 warps streams a range of blocks of one sequence for every KV
+// head at once: every block is one contiguous run of Hkv x 1152 bytes, fetched
+// by a single bulk copy into a 4-stage CTA ring (16 block-heads per stage,
+// full/empty mbarriers, the copies issued by lane 0 of warp 0 two stages
+// ahead).  Warp w serves KV head w % Hkv and, per stage, two of its blocks.
+// Per 2-block step a warp computes:
 //   scores  S[32 tok x 4NT heads] = C_K (u8 codes) . Q (two s8 limbs) on
 //           mma.m16n8k32, then s_t * sigma * raw + m_t * sum(q~);
-//   values  O[128 ch x heads] += C_V^T . P', P' = round(p * s_t * 65535 / s_cap)
+//   values  O[128 ch x heads] += C_V . P', P' = round(p * s_t * 65535 / s_cap)
 //           as two u8 limbs, exact in int32, flushed to fp32 only when the
-//           running max or the scale cap moves (or every 128 steps);
+//           running max or the scale cap moves (or every 96 steps);
 //   plus sum(p * m_t) for the value minimum term.
 // Fragment facts (PTX m16n8k32, 8-bit): lane (g = lane/4, t = lane%4) holds
 // A rows g and g+8 with K-columns 4t..4t+3 and 16+4t..16+4t+3; B K-rows
@@ -384,31 +415,33 @@ __global__ void __launch_bounds__(kDecWarps * 32) decode_simt_kernel(DecodeArgs 
 //   are only masked (w & (3 << 2f)), leaving a known 4^f factor per output
 //   row that the flush removes.
 // The fp16 window (at most 128 tokens) is attended in ring order (softmax
-// attention does not depend on token order), 16 rows per warp-chunk, all
-// warps sharing the chunks: scores and P.V on mma.m16n8k16 (f16 in, f32
-// accumulate; query and probabilities as fp16 hi+lo pairs); the window state
-// is folded into the warp's own state in registers.
+// attention does not depend on token order), 16 rows per chunk: scores and
+// P.V on mma.m16n8k16 (f16 in, f32 accumulate; query and probabilities as
+// fp16 hi+lo pairs), folded into the warp's state in registers.
 // ---------------------------------------------------------------------------
-constexpr int kMmaWarps = 4;
-constexpr int kStages = 4;
-constexpr int kStageBytes = 2 * kBlockHeadBytes;
-constexpr int kPStride = 40;  // u16 per head row of the P' staging tile
+constexpr int kHW = 8;                             // warps per CTA
+constexpr int kHStages = 4;                        // ring stages
+constexpr int kSlotsPerStage = 16;                 // block-heads per stage
+constexpr int kHStageBytes = kSlotsPerStage * kBlockHeadBytes;  // 18432
+constexpr int kPStride = 40;                       // u16 per head row of the P' tile
+constexpr int kWarpScratch = kHStages * kHStageBytes / kHW;     // 9216 B of ring per warp
 constexpr uint32_t kM2 = 0x03030303u;
 
 template <int G>
-struct MmaCfg {
+struct HCfg {
   static constexpr int NT = G <= 4 ? 1 : G / 4;  // n-tiles of 8 columns = 4 heads x 2 limbs
   static constexpr int HP = 4 * NT;              // heads incl. padding
-  static constexpr size_t ring_bytes = (size_t)kMmaWarps * kStages * kStageBytes;
+  static constexpr size_t ring_bytes = (size_t)kHStages * kHStageBytes;
   static constexpr size_t smem_bytes() {
-    return ring_bytes                                  // stage rings (reused for merge buffers)
-           + (size_t)kMmaWarps * kStages * 8           // mbarriers
-           + (size_t)kMmaWarps * kStages * 4           // per-stage token counts
-           + (size_t)kMmaWarps * HP * kPStride * 2     // P' tiles
-           + (size_t)kMmaWarps * G * 2 * 4;            // merge (m, l)
+    return ring_bytes                            // ring (reused for window scratch and merging)
+           + (size_t)2 * kHStages * 8            // full / empty mbarriers
+           + (size_t)kHStages * kSlotsPerStage   // tokens per block slot
+           + (size_t)kHW * HP * kPStride * 2     // P' tiles
+           + (size_t)kHW * G * 2 * 4;            // merge (m, l)
   }
 };
-static_assert(kMmaWarps * 8 * kD * 4 <= kMmaWarps * kStages * kStageBytes, "merge buffer must fit the rings");
+static_assert(kHW * 8 * kD * 4 <= kHStages * kHStageBytes, "merge buffer must fit the ring");
+static_assert(4096 + 8 * 64 + 8 * kD * 4 <= kWarpScratch, "window scratch must fit a warp's share of the ring");
 
 __device__ __forceinline__ float lo_half(uint32_t w) {
   return __half2float(__ushort_as_half((unsigned short)(w & 0xffffu)));
@@ -454,7 +487,7 @@ __device__ __forceinline__ uint32_t cvt_u16_sat(float x) {
 
 template <int G>
 struct MmaWarpState {
-  static constexpr int NT = MmaCfg<G>::NT;
+  static constexpr int NT = HCfg<G>::NT;
   float m[NT], l[NT], msum[NT];
   float acc[NT][16];   // fp32 o' for channels 16g + 0..15 of head 4nt + t
   int acci[NT][8][4];  // exact int32 o' contributions since the last flush (row scale 4^f)
@@ -477,37 +510,43 @@ __device__ __forceinline__ void mma_flush(MmaWarpState<G>& st, int nt, float inv
 }
 
 template <int G>
-__global__ void __launch_bounds__(kMmaWarps * 32, (G <= 4) ? 4 : 3) decode_mma_kernel(DecodeArgs a) {
-  constexpr int NT = MmaCfg<G>::NT, HP = MmaCfg<G>::HP;
+__global__ void __launch_bounds__(kHW * 32, (G <= 4) ? 2 : 1) decode_heads_kernel(DecodeArgs a) {
+  constexpr int NT = HCfg<G>::NT, HP = HCfg<G>::HP;
   extern __shared__ __align__(16) unsigned char smem_raw[];
-  unsigned char* rings = smem_raw;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(rings + MmaCfg<G>::ring_bytes);
-  uint32_t* stinfo = reinterpret_cast<uint32_t*>(bars + kMmaWarps * kStages);
-  uint16_t* pst = reinterpret_cast<uint16_t*>(stinfo + kMmaWarps * kStages);
-  float* ml = reinterpret_cast<float*>(pst + kMmaWarps * HP * kPStride);  // [NW][G][2]
-  float* mo = reinterpret_cast<float*>(rings);  // [NW][G][128], only while the rings are idle
+  unsigned char* ring = smem_raw;
+  uint64_t* full = reinterpret_cast<uint64_t*>(ring + HCfg<G>::ring_bytes);
+  uint64_t* empty = full + kHStages;
+  uint8_t* ntok = reinterpret_cast<uint8_t*>(empty + kHStages);                 // [S][16]
+  uint16_t* pst = reinterpret_cast<uint16_t*>(ntok + kHStages * kSlotsPerStage);  // [8][HP][40]
+  float* ml = reinterpret_cast<float*>(pst + kHW * HP * kPStride);              // [8][G][2]
+  float* mo = reinterpret_cast<float*>(ring);  // [8][G][128], only while the ring is idle
 
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int g = lane >> 2, t = lane & 3;
+  const int hkv = a.hkv;                 // 1, 2, 4 or 8
+  const int wph = kHW / hkv;             // warps per KV head
+  const int head = warp % hkv, grp = warp / hkv;
+  const int nb = 2 * wph;                // blocks per stage
+  const uint32_t copy_bytes = (uint32_t)hkv * kBlockHeadBytes;
   const long long total = a.prefix[a.batch];
   if (total == 0) return;
-  const int nc = (int)min((long long)a.nc, total);
+  const int nc = working_ctas(a, total);
   const int c = blockIdx.x;
   if (c >= nc) return;
   const long long start = (long long)c * total / nc;
   const long long end = (long long)(c + 1) * total / nc;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kMmaWarps * kStages; ++i) mbar_init(&bars[i], 1);
+    for (int i = 0; i < kHStages; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], kHW);
+    }
     fence_mbar_init();
   }
   __syncthreads();
-  uint64_t* mybar = bars + warp * kStages;
-  uint32_t* myinfo = stinfo + warp * kStages;
-  unsigned char* myst = rings + warp * kStages * kStageBytes;
   uint16_t* myp = pst + warp * HP * kPStride;
-  uint32_t it = 0;    // ring position of this warp (continues across units)
-  bool alive = true;  // cleared if a bulk copy never lands
+  uint32_t it = 0;    // CTA ring position (continues across batch entries)
+  bool alive = true;  // cleared if a wait never completes
 
   int lo = 0, hi = a.batch - 1;
   while (lo < hi) {
@@ -519,104 +558,104 @@ __global__ void __launch_bounds__(kMmaWarps * 32, (G <= 4) ? 4 : 3) decode_mma_k
     if (us.cost == 0) continue;
     const int slot = a.seq_slot[b];
     const bool slot_ok = slot >= 0 && slot < a.num_slots;
-    for (int hk = 0; hk < a.hkv; ++hk) {
-      const long long pu = a.prefix[b] + (long long)hk * us.cost;
-      if (pu + us.cost <= start) continue;
-      if (pu >= end) break;
-      const int u = b * a.hkv + hk;
-      const int l0 = (int)(max(start, pu) - pu), l1 = (int)(min(end, pu + us.cost) - pu);
-      const size_t bh0 = (size_t)b * a.hq + (size_t)hk * G;  // first query head of the unit
-      __syncthreads();  // the previous unit's merge buffers (on the rings) are free again
+    const long long pu = a.prefix[b];
+    const int l0 = (int)(max(start, pu) - pu), l1 = (int)(min(end, pu + us.cost) - pu);
+    const size_t bh0 = (size_t)b * a.hq + (size_t)head * G;  // first query head of this warp's KV head
+    __syncthreads();  // the previous entry's window scratch / merge buffers (on the ring) are free again
+    if (!slot_ok && threadIdx.x == 0) raise_flag(a.status, OKV_DEV_BAD_SLOT);
 
-      // ---------------- INT2 blocks ----------------
-      MmaWarpState<G> st;
-      uint32_t qb[NT][8];
-      float ah[NT], bh[NT], hbias[NT];
+    // ---------------- per-warp state for (b, head) ----------------
+    MmaWarpState<G> st;
+    uint32_t qb[NT][8];
+    float ah[NT], bh[NT], hbias[NT];
 #pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
-        st.m[nt] = -INFINITY;
-        st.l[nt] = 0.f;
-        st.msum[nt] = 0.f;
+    for (int nt = 0; nt < NT; ++nt) {
+      st.m[nt] = -INFINITY;
+      st.l[nt] = 0.f;
+      st.msum[nt] = 0.f;
 #pragma unroll
-        for (int i = 0; i < 16; ++i) st.acc[nt][i] = 0.f;
+      for (int i = 0; i < 16; ++i) st.acc[nt][i] = 0.f;
 #pragma unroll
-        for (int mt = 0; mt < 8; ++mt)
+      for (int mt = 0; mt < 8; ++mt)
 #pragma unroll
-          for (int j = 0; j < 4; ++j) st.acci[nt][mt][j] = 0;
-        const int hcol = 4 * nt + (g >> 1);  // head of this lane's B column
-        if (hcol < G) {
-          const uint4* src = reinterpret_cast<const uint4*>(a.qlimb + ((bh0 + hcol) * 2 + (g & 1)) * kD + 32 * t);
-          const uint4 x0 = src[0], x1 = src[1];
-          qb[nt][0] = x0.x; qb[nt][1] = x0.y; qb[nt][2] = x0.z; qb[nt][3] = x0.w;
-          qb[nt][4] = x1.x; qb[nt][5] = x1.y; qb[nt][6] = x1.z; qb[nt][7] = x1.w;
-        } else {
+        for (int j = 0; j < 4; ++j) st.acci[nt][mt][j] = 0;
+      const int hcol = 4 * nt + (g >> 1);  // head of this lane's B column
+      if (hcol < G) {
+        const uint4* src = reinterpret_cast<const uint4*>(a.qlimb + ((bh0 + hcol) * 2 + (g & 1)) * kD + 32 * t);
+        const uint4 x0 = src[0], x1 = src[1];
+        qb[nt][0] = x0.x; qb[nt][1] = x0.y; qb[nt][2] = x0.z; qb[nt][3] = x0.w;
+        qb[nt][4] = x1.x; qb[nt][5] = x1.y; qb[nt][6] = x1.z; qb[nt][7] = x1.w;
+      } else {
 #pragma unroll
-          for (int i = 0; i < 8; ++i) qb[nt][i] = 0u;
-        }
-        const int hs = 4 * nt + t;  // head of this lane's score columns
-        const bool ok = hs < G;
-        ah[nt] = ok ? a.qscale[(bh0 + hs) * 4 + 0] : 0.f;
-        bh[nt] = ok ? a.qscale[(bh0 + hs) * 4 + 1] : 0.f;
-        hbias[nt] = ok ? 0.f : -INFINITY;
+        for (int i = 0; i < 8; ++i) qb[nt][i] = 0u;
       }
-      float s_cap = 0.f, lam = 0.f, inv = 0.f;
-      int since_flush = 0;
+      const int hs = 4 * nt + t;  // head of this lane's score columns
+      const bool ok = hs < G;
+      ah[nt] = ok ? a.qscale[(bh0 + hs) * 4 + 0] : 0.f;
+      bh[nt] = ok ? a.qscale[(bh0 + hs) * 4 + 1] : 0.f;
+      hbias[nt] = ok ? 0.f : -INFINITY;
+    }
+    float s_cap = 0.f, lam = 0.f, inv = 0.f;
+    int since_flush = 0;
 
-      const int p0 = max(l0, us.win_cost) - us.win_cost;
-      const int p1 = l1 - us.win_cost;
-      const int nsteps = p1 > p0 ? (p1 - p0 + 1) >> 1 : 0;
-      const int nmy = (slot_ok && alive && nsteps > warp) ? (nsteps - warp + kMmaWarps - 1) / kMmaWarps : 0;
-      const int32_t* trow = a.block_table + (size_t)(slot_ok ? slot : 0) * a.mbps;
+    // ---------------- INT2 blocks through the ring ----------------
+    const int p0 = max(l0, us.win_cost) - us.win_cost;
+    const int p1 = l1 - us.win_cost;
+    const int nst = (slot_ok && alive && p1 > p0) ? (p1 - p0 + nb - 1) / nb : 0;
+    const int32_t* trow = a.block_table + (size_t)(slot_ok ? slot : 0) * a.mbps;
 
-      // lane 0: issue local step j into ring position it + j, recording how
-      // many valid tokens each of its two blocks holds
-      auto issue = [&](int j) {
-        const int pa = p0 + 2 * (warp + kMmaWarps * j);
-        const uint32_t stg = (it + j) % kStages;
-        int blk[2];
-        uint32_t bytes = 0, info = 0;
-#pragma unroll
-        for (int bb = 0; bb < 2; ++bb) {
-          const int pi = pa + bb;
-          blk[bb] = -1;
-          if (pi < p1) {
-            blk[bb] = trow[pi];
-            if (blk[bb] < 0 || blk[bb] >= a.num_blocks) {
-              raise_flag(a.status, OKV_DEV_BAD_BLOCK);
-              blk[bb] = -1;
-            }
-          }
-          if (blk[bb] >= 0) {
-            bytes += kBlockHeadBytes;
-            info |= (uint32_t)min(kBlock, us.n_int2 - kBlock * pi) << (8 * bb);
-          }
+    // warp 0 lane 0: put stage j of this entry in ring position it + j
+    auto issue = [&](int j) -> bool {
+      const uint32_t pos = it + (uint32_t)j;
+      const uint32_t s = pos % kHStages;
+      if (pos >= (uint32_t)kHStages && !mbar_wait_bounded(&empty[s], ((pos / kHStages) - 1) & 1u)) return false;
+      uint32_t bytes = 0;
+      for (int q = 0; q < nb; ++q) {  // token counts first: the barrier must expect every byte
+        const int pi = p0 + j * nb + q;
+        int bid = pi < p1 ? trow[pi] : -1;
+        if (pi < p1 && (bid < 0 || bid >= a.num_blocks)) {
+          raise_flag(a.status, OKV_DEV_BAD_BLOCK);
+          bid = -1;
         }
-        myinfo[stg] = info;
-        mbar_arrive_expect_tx(&mybar[stg], bytes);
-#pragma unroll
-        for (int bb = 0; bb < 2; ++bb)
-          if (blk[bb] >= 0)
-            bulk_g2s(myst + stg * kStageBytes + bb * kBlockHeadBytes,
-                     a.pages + ((size_t)blk[bb] * a.hkv + hk) * kBlockHeadBytes, kBlockHeadBytes, &mybar[stg]);
-      };
-      if (lane == 0)
-        for (int j = 0; j < min(kStages, nmy); ++j) issue(j);
-      __syncwarp();
+        ntok[s * kSlotsPerStage + q] = bid >= 0 ? (uint8_t)min(kBlock, us.n_int2 - kBlock * pi) : 0;
+        if (bid >= 0) bytes += copy_bytes;
+      }
+      mbar_arrive_expect_tx(&full[s], bytes);
+      for (int q = 0; q < nb; ++q) {
+        const int pi = p0 + j * nb + q;
+        const int bid = pi < p1 ? trow[pi] : -1;
+        if (bid >= 0 && bid < a.num_blocks)
+          bulk_g2s(ring + s * kHStageBytes + q * copy_bytes, a.pages + (size_t)bid * copy_bytes, copy_bytes,
+                   &full[s]);
+      }
+      return true;
+    };
+    bool prod_ok = true;
+    if (warp == 0 && lane == 0)
+      for (int j = 0; j < min(kHStages - 2, nst) && prod_ok; ++j) prod_ok = issue(j);
 
-      int done = 0;
-      for (int j = 0; j < nmy; ++j) {
-        const uint32_t stg = (it + j) % kStages;
-        const uint32_t par = ((it + j) / kStages) & 1u;
-        if (!__all_sync(0xffffffffu, mbar_wait_bounded(&mybar[stg], par))) {
+    int done = 0;
+    for (int j = 0; j < nst; ++j) {
+      if (warp == 0) {
+        if (lane == 0 && prod_ok && j + kHStages - 2 < nst) prod_ok = issue(j + kHStages - 2);
+        if (!__shfl_sync(0xffffffffu, prod_ok, 0)) {
           if (lane == 0) raise_flag(a.status, OKV_DEV_TIMEOUT);
           alive = false;
-          break;
         }
-        const uint32_t info = myinfo[stg];
-        const int n0 = (int)(info & 0xffu), n1 = (int)(info >> 8);
-        const bool full = (n0 == kBlock) && (n1 == kBlock);
-        const unsigned char* s0 = myst + stg * kStageBytes;
-        const unsigned char* s1 = s0 + kBlockHeadBytes;
+      }
+      const uint32_t pos = it + (uint32_t)j;
+      const uint32_t s = pos % kHStages;
+      if (!__all_sync(0xffffffffu, alive && mbar_wait_bounded(&full[s], (pos / kHStages) & 1u))) {
+        if (lane == 0) raise_flag(a.status, OKV_DEV_TIMEOUT);
+        alive = false;
+        break;
+      }
+      const int q0 = 2 * grp;
+      const int n0 = ntok[s * kSlotsPerStage + q0], n1 = ntok[s * kSlotsPerStage + q0 + 1];
+      if (n0 + n1 > 0) {
+        const bool fullstep = (n0 == kBlock) && (n1 == kBlock);
+        const unsigned char* s0 = ring + s * kHStageBytes + q0 * copy_bytes + head * kBlockHeadBytes;
+        const unsigned char* s1 = s0 + copy_bytes;
 
         // ---- scores: D[tok][col] for both blocks
         int dq[2][NT][4];
@@ -631,16 +670,16 @@ __global__ void __launch_bounds__(kMmaWarps * 32, (G <= 4) ? 4 : 3) decode_mma_k
           smv[2 * bb] = *reinterpret_cast<const uint32_t*>(sb + kVsmOff + 4 * g);
           smv[2 * bb + 1] = *reinterpret_cast<const uint32_t*>(sb + kVsmOff + 4 * (g + 8));
 #pragma unroll
-          for (int s = 0; s < 4; ++s) {
+          for (int sf = 0; sf < 4; ++sf) {
             uint32_t af[4];
-            af[0] = (wa.x >> (2 * s)) & kM2;
-            af[1] = (wb.x >> (2 * s)) & kM2;
-            af[2] = (wa.y >> (2 * s)) & kM2;
-            af[3] = (wb.y >> (2 * s)) & kM2;
+            af[0] = (wa.x >> (2 * sf)) & kM2;
+            af[1] = (wb.x >> (2 * sf)) & kM2;
+            af[2] = (wa.y >> (2 * sf)) & kM2;
+            af[3] = (wb.y >> (2 * sf)) & kM2;
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
-              if (s == 0) mma_u8s8_z(dq[bb][nt], af, qb[nt][0], qb[nt][1]);
-              else mma_u8s8(dq[bb][nt], af, qb[nt][2 * s], qb[nt][2 * s + 1]);
+              if (sf == 0) mma_u8s8_z(dq[bb][nt], af, qb[nt][0], qb[nt][1]);
+              else mma_u8s8(dq[bb][nt], af, qb[nt][2 * sf], qb[nt][2 * sf + 1]);
             }
           }
         }
@@ -651,8 +690,11 @@ __global__ void __launch_bounds__(kMmaWarps * 32, (G <= 4) ? 4 : 3) decode_mma_k
         for (int e = 0; e < 4; ++e) {
           const float2 k2 = __half22float2(*reinterpret_cast<const __half2*>(&smk[e]));
           const float2 v2 = __half22float2(*reinterpret_cast<const __half2*>(&smv[e]));
-          sk[e] = k2.x; mk[e] = k2.y; sv[e] = v2.x; mv[e] = v2.y;
-          tv[e] = full || ((g + 8 * (e & 1)) < ((e >> 1) ? n1 : n0));
+          tv[e] = fullstep || ((g + 8 * (e & 1)) < ((e >> 1) ? n1 : n0));
+          // masked slots may hold any bits (a slot whose block was not fetched
+          // keeps stale shared memory): select, never multiply, them away
+          sk[e] = k2.x; mk[e] = k2.y; sv[e] = v2.x;
+          mv[e] = tv[e] ? v2.y : 0.f;
         }
         float smax = fmaxf(fmaxf(tv[0] ? sv[0] : 0.f, tv[1] ? sv[1] : 0.f),
                            fmaxf(tv[2] ? sv[2] : 0.f, tv[3] ? sv[3] : 0.f));
@@ -733,165 +775,189 @@ __global__ void __launch_bounds__(kMmaWarps * 32, (G <= 4) ? 4 : 3) decode_mma_k
           for (int nt = 0; nt < NT; ++nt) mma_flush(st, nt, inv);
           since_flush = 0;
         }
-        __syncwarp();
-        ++done;
-        if (lane == 0 && j + kStages < nmy) issue(j + kStages);
       }
-      if (!alive) {  // drain what is still in flight, with the same bound, then stop streaming
-        for (int j = done + 1; j < min(nmy, done + kStages); ++j)
-          (void)mbar_wait_bounded(&mybar[(it + j) % kStages], ((it + j) / kStages) & 1u);
-      }
-      it += (uint32_t)nmy;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[s]);
+      ++done;
+    }
+    it += (uint32_t)nst;
 #pragma unroll
-      for (int nt = 0; nt < NT; ++nt) mma_flush(st, nt, inv);
+    for (int nt = 0; nt < NT; ++nt) mma_flush(st, nt, inv);
+    __syncthreads();  // every warp is done with the ring: it becomes window scratch, then merge buffers
 
-      // ---------------- fp16 window: chunks ci = warp, warp + NW, ... ----------------
-      const int nchunk = (l0 == 0 && us.win_cost > 0 && slot_ok) ? (us.n_win + 15) / 16 : 0;
-      if (warp < nchunk) {
-        const __half* kr = a.ring + (((size_t)slot * a.hkv + hk) * 2 + 0) * kWin * kD;
-        const __half* vr = a.ring + (((size_t)slot * a.hkv + hk) * 2 + 1) * kWin * kD;
-        unsigned char* tile = myst;                                   // 16 rows x 256 B, swizzled
-        float* pw = reinterpret_cast<float*>(myst + 4096);            // [HP][16]
-        float* wo = reinterpret_cast<float*>(myst + 4096 + HP * 64);  // [G][128]
-        uint32_t qh[NT][16];
-        float wsc[NT], wm[NT], wl[NT];
-        float wacc[NT][8][4];
+    // ---------------- fp16 window: chunks ci = grp, grp + wph, ... of this warp's head ----------------
+    const int nchunk = (l0 == 0 && us.win_cost > 0 && slot_ok) ? (us.n_win + 15) / 16 : 0;
+    if (grp < nchunk) {
+      const __half* kr = a.ring + (((size_t)slot * hkv + head) * 2 + 0) * kWin * kD;
+      const __half* vr = a.ring + (((size_t)slot * hkv + head) * 2 + 1) * kWin * kD;
+      unsigned char* scratch = ring + warp * kWarpScratch;
+      unsigned char* tile = scratch;                                   // 16 rows x 256 B, swizzled
+      float* pw = reinterpret_cast<float*>(scratch + 4096);            // [HP][16]
+      float* wo = reinterpret_cast<float*>(scratch + 4096 + HP * 64);  // [G][128]
+      uint32_t qh[NT][16];
+      float wsc[NT], wm[NT], wl[NT];
+      float wacc[NT][8][4];
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        const int hcol = 4 * nt + (g >> 1);
+        if (hcol < G) {
+          const uint4* src = reinterpret_cast<const uint4*>(a.qwin + ((bh0 + hcol) * 2 + (g & 1)) * kD + 32 * t);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const uint4 x = src[i];
+            qh[nt][4 * i] = x.x; qh[nt][4 * i + 1] = x.y; qh[nt][4 * i + 2] = x.z; qh[nt][4 * i + 3] = x.w;
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) qh[nt][i] = 0u;
+        }
+        const int hs = 4 * nt + t;
+        wsc[nt] = hs < G ? a.qscale[(bh0 + hs) * 4 + 2] * (kInvSqrtD * kLog2e) : 0.f;
+        wm[nt] = -INFINITY;
+        wl[nt] = 0.f;
+#pragma unroll
+        for (int mt = 0; mt < 8; ++mt)
+#pragma unroll
+          for (int i = 0; i < 4; ++i) wacc[nt][mt][i] = 0.f;
+      }
+      for (int ci = grp; ci < nchunk; ci += wph) {
+        const int r0 = 16 * ci;
+        // stage the V rows (swizzled 16-byte chunks) for the transposing loads
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const int q = lane + 32 * k, row = q >> 4, col = q & 15;
+          uint4 x = make_uint4(0, 0, 0, 0);
+          if (r0 + row < us.n_win) x = *reinterpret_cast<const uint4*>(vr + (size_t)(r0 + row) * kD + 8 * col);
+          *reinterpret_cast<uint4*>(tile + row * 256 + ((col ^ (row & 7)) << 4)) = x;
+        }
+        // scores of ring rows r0 + g and r0 + g + 8
+        uint32_t ka[16], kb[16];
+        const bool va_ = r0 + g < us.n_win, vb_ = r0 + g + 8 < us.n_win;
+        const uint4* ra = reinterpret_cast<const uint4*>(kr + (size_t)(r0 + g) * kD + 32 * t);
+        const uint4* rb = reinterpret_cast<const uint4*>(kr + (size_t)(r0 + g + 8) * kD + 32 * t);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const uint4 x = va_ ? ra[i] : make_uint4(0, 0, 0, 0);
+          const uint4 y = vb_ ? rb[i] : make_uint4(0, 0, 0, 0);
+          ka[4 * i] = x.x; ka[4 * i + 1] = x.y; ka[4 * i + 2] = x.z; ka[4 * i + 3] = x.w;
+          kb[4 * i] = y.x; kb[4 * i + 1] = y.y; kb[4 * i + 2] = y.z; kb[4 * i + 3] = y.w;
+        }
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
-          const int hcol = 4 * nt + (g >> 1);
-          if (hcol < G) {
-            const uint4* src = reinterpret_cast<const uint4*>(a.qwin + ((bh0 + hcol) * 2 + (g & 1)) * kD + 32 * t);
+          float d[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              const uint4 x = src[i];
-              qh[nt][4 * i] = x.x; qh[nt][4 * i + 1] = x.y; qh[nt][4 * i + 2] = x.z; qh[nt][4 * i + 3] = x.w;
-            }
-          } else {
-#pragma unroll
-            for (int i = 0; i < 16; ++i) qh[nt][i] = 0u;
+          for (int ks = 0; ks < 8; ++ks) {
+            const uint32_t af[4] = {ka[2 * ks], kb[2 * ks], ka[2 * ks + 1], kb[2 * ks + 1]};
+            mma_f16(d, af, qh[nt][2 * ks], qh[nt][2 * ks + 1]);
           }
           const int hs = 4 * nt + t;
-          wsc[nt] = hs < G ? a.qscale[(bh0 + hs) * 4 + 2] * (kInvSqrtD * kLog2e) : 0.f;
-          wm[nt] = -INFINITY;
-          wl[nt] = 0.f;
+          const float s_a = (va_ && hs < G) ? (d[0] + d[1]) * wsc[nt] : -INFINITY;
+          const float s_b = (vb_ && hs < G) ? (d[2] + d[3]) * wsc[nt] : -INFINITY;
+          float bm = fmaxf(s_a, s_b);
+          bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 4));
+          bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 8));
+          bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 16));
+          const float mnew = fmaxf(wm[nt], bm);
+          const float mref = mnew == -INFINITY ? 0.f : mnew;
+          const float alpha = fast_ex2(wm[nt] - mref);
+          const float pa_ = fast_ex2(s_a - mref), pb_ = fast_ex2(s_b - mref);
+          wl[nt] = wl[nt] * alpha + pa_ + pb_;
+          wm[nt] = mnew;
+          pw[(4 * nt + t) * 16 + g] = pa_;
+          pw[(4 * nt + t) * 16 + g + 8] = pb_;
 #pragma unroll
           for (int mt = 0; mt < 8; ++mt)
 #pragma unroll
-            for (int i = 0; i < 4; ++i) wacc[nt][mt][i] = 0.f;
+            for (int i = 0; i < 4; ++i) wacc[nt][mt][i] *= alpha;
         }
-        for (int ci = warp; ci < nchunk; ci += kMmaWarps) {
-          const int r0 = 16 * ci;
-          // stage the V rows (swizzled 16-byte chunks) for the transposing loads
-#pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            const int q = lane + 32 * k, row = q >> 4, col = q & 15;
-            uint4 x = make_uint4(0, 0, 0, 0);
-            if (r0 + row < us.n_win) x = *reinterpret_cast<const uint4*>(vr + (size_t)(r0 + row) * kD + 8 * col);
-            *reinterpret_cast<uint4*>(tile + row * 256 + ((col ^ (row & 7)) << 4)) = x;
-          }
-          // scores of ring rows r0 + g and r0 + g + 8
-          uint32_t ka[16], kb[16];
-          const bool va_ = r0 + g < us.n_win, vb_ = r0 + g + 8 < us.n_win;
-          const uint4* ra = reinterpret_cast<const uint4*>(kr + (size_t)(r0 + g) * kD + 32 * t);
-          const uint4* rb = reinterpret_cast<const uint4*>(kr + (size_t)(r0 + g + 8) * kD + 32 * t);
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const uint4 x = va_ ? ra[i] : make_uint4(0, 0, 0, 0);
-            const uint4 y = vb_ ? rb[i] : make_uint4(0, 0, 0, 0);
-            ka[4 * i] = x.x; ka[4 * i + 1] = x.y; ka[4 * i + 2] = x.z; ka[4 * i + 3] = x.w;
-            kb[4 * i] = y.x; kb[4 * i + 1] = y.y; kb[4 * i + 2] = y.z; kb[4 * i + 3] = y.w;
-          }
-#pragma unroll
-          for (int nt = 0; nt < NT; ++nt) {
-            float d[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int ks = 0; ks < 8; ++ks) {
-              const uint32_t af[4] = {ka[2 * ks], kb[2 * ks], ka[2 * ks + 1], kb[2 * ks + 1]};
-              mma_f16(d, af, qh[nt][2 * ks], qh[nt][2 * ks + 1]);
-            }
-            const int hs = 4 * nt + t;
-            const float s_a = (va_ && hs < G) ? (d[0] + d[1]) * wsc[nt] : -INFINITY;
-            const float s_b = (vb_ && hs < G) ? (d[2] + d[3]) * wsc[nt] : -INFINITY;
-            float bm = fmaxf(s_a, s_b);
-            bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 4));
-            bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 8));
-            bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 16));
-            const float mnew = fmaxf(wm[nt], bm);
-            const float mref = mnew == -INFINITY ? 0.f : mnew;
-            const float alpha = fast_ex2(wm[nt] - mref);
-            const float pa_ = fast_ex2(s_a - mref), pb_ = fast_ex2(s_b - mref);
-            wl[nt] = wl[nt] * alpha + pa_ + pb_;
-            wm[nt] = mnew;
-            pw[(4 * nt + t) * 16 + g] = pa_;
-            pw[(4 * nt + t) * 16 + g + 8] = pb_;
-            // D rows of this lane hold heads 4nt + t: rescale them
-#pragma unroll
-            for (int mt = 0; mt < 8; ++mt)
-#pragma unroll
-              for (int i = 0; i < 4; ++i) wacc[nt][mt][i] *= alpha;
-          }
-          __syncwarp();
-          // P.V: A = V^T (channels x tokens) by transposing loads, B = p as fp16 hi/lo
-          uint32_t b0[NT], b1[NT];
-#pragma unroll
-          for (int nt = 0; nt < NT; ++nt) {
-            const float* prw = pw + (4 * nt + (g >> 1)) * 16;
-            const float2 pa2 = *reinterpret_cast<const float2*>(prw + 2 * t);
-            const float2 pb2 = *reinterpret_cast<const float2*>(prw + 2 * t + 8);
-            const __half2 ha = __floats2half2_rn(pa2.x, pa2.y), hb = __floats2half2_rn(pb2.x, pb2.y);
-            __half2 ra2 = ha, rb2 = hb;
-            if (g & 1) {
-              const float2 fa = __half22float2(ha), fb = __half22float2(hb);
-              ra2 = __floats2half2_rn(pa2.x - fa.x, pa2.y - fa.y);
-              rb2 = __floats2half2_rn(pb2.x - fb.x, pb2.y - fb.y);
-            }
-            b0[nt] = *reinterpret_cast<uint32_t*>(&ra2);
-            b1[nt] = *reinterpret_cast<uint32_t*>(&rb2);
-          }
-          {
-            const int mi = lane >> 3, ri = lane & 7;
-            const int tok = ri + 8 * (mi >> 1);
-#pragma unroll
-            for (int mt = 0; mt < 8; ++mt) {
-              const int col = 2 * mt + (mi & 1);
-              uint32_t af[4];
-              ldmatrix_x4_trans(af, tile + tok * 256 + ((col ^ (tok & 7)) << 4));
-#pragma unroll
-              for (int nt = 0; nt < NT; ++nt) mma_f16(wacc[nt][mt], af, b0[nt], b1[nt]);
-            }
-          }
-          __syncwarp();
-        }
-        // window o' per (head, channel) through shared memory, then fold into the block state
+        __syncwarp();
+        // P.V: A = V^T (channels x tokens) by transposing loads, B = p as fp16 hi/lo
+        uint32_t b0[NT], b1[NT];
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
-          const int hs = 4 * nt + t;
-          if (hs < G) {
+          const float* prw = pw + (4 * nt + (g >> 1)) * 16;
+          const float2 pa2 = *reinterpret_cast<const float2*>(prw + 2 * t);
+          const float2 pb2 = *reinterpret_cast<const float2*>(prw + 2 * t + 8);
+          const __half2 ha = __floats2half2_rn(pa2.x, pa2.y), hb = __floats2half2_rn(pb2.x, pb2.y);
+          __half2 ra2 = ha, rb2 = hb;
+          if (g & 1) {
+            const float2 fa = __half22float2(ha), fb = __half22float2(hb);
+            ra2 = __floats2half2_rn(pa2.x - fa.x, pa2.y - fa.y);
+            rb2 = __floats2half2_rn(pb2.x - fb.x, pb2.y - fb.y);
+          }
+          b0[nt] = *reinterpret_cast<uint32_t*>(&ra2);
+          b1[nt] = *reinterpret_cast<uint32_t*>(&rb2);
+        }
+        {
+          const int mi = lane >> 3, ri = lane & 7;
+          const int tok = ri + 8 * (mi >> 1);
 #pragma unroll
-            for (int mt = 0; mt < 8; ++mt) {
-              wo[hs * kD + 16 * mt + g] = wacc[nt][mt][0] + wacc[nt][mt][1];
-              wo[hs * kD + 16 * mt + g + 8] = wacc[nt][mt][2] + wacc[nt][mt][3];
-            }
+          for (int mt = 0; mt < 8; ++mt) {
+            const int col = 2 * mt + (mi & 1);
+            uint32_t af[4];
+            ldmatrix_x4_trans(af, tile + tok * 256 + ((col ^ (tok & 7)) << 4));
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) mma_f16(wacc[nt][mt], af, b0[nt], b1[nt]);
           }
         }
         __syncwarp();
+      }
+      // window o' per (head, channel) through shared memory, then fold into the block state
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-          const int hs = 4 * nt + t;
-          if (hs < G) {
-            const float M = fmaxf(st.m[nt], wm[nt]);
-            const float mref = M == -INFINITY ? 0.f : M;
-            const float ab = fast_ex2(st.m[nt] - mref), aw = fast_ex2(wm[nt] - mref);
-            const float* src = wo + hs * kD + 16 * g;
+      for (int nt = 0; nt < NT; ++nt) {
+        const int hs = 4 * nt + t;
+        if (hs < G) {
 #pragma unroll
-            for (int i = 0; i < 16; ++i) st.acc[nt][i] = fmaf(st.acc[nt][i], ab, src[i] * aw);
-            st.l[nt] = fmaf(st.l[nt], ab, wl[nt] * aw);
-            st.msum[nt] *= ab;
-            st.m[nt] = M;
+          for (int mt = 0; mt < 8; ++mt) {
+            wo[hs * kD + 16 * mt + g] = wacc[nt][mt][0] + wacc[nt][mt][1];
+            wo[hs * kD + 16 * mt + g + 8] = wacc[nt][mt][2] + wacc[nt][mt][3];
           }
         }
       }
-      __syncthreads();  // every warp is done with its ring: the rings become merge buffers
+      __syncwarp();
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        const int hs = 4 * nt + t;
+        if (hs < G) {
+          const float M = fmaxf(st.m[nt], wm[nt]);
+          const float mref = M == -INFINITY ? 0.f : M;
+          const float ab = fast_ex2(st.m[nt] - mref), aw = fast_ex2(wm[nt] - mref);
+          const float* src = wo + hs * kD + 16 * g;
+#pragma unroll
+          for (int i = 0; i < 16; ++i) st.acc[nt][i] = fmaf(st.acc[nt][i], ab, src[i] * aw);
+          st.l[nt] = fmaf(st.l[nt], ab, wl[nt] * aw);
+          st.msum[nt] *= ab;
+          st.m[nt] = M;
+        }
+      }
+    }
+
+    // ---------------- partial for (c, b): one warp per KV head, or merged across its warps ----------------
+    float* part_b = a.part + ((size_t)(c + b) * a.hq + (size_t)head * G) * kPartStride;
+    if (wph == 1) {
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        float l = st.l[nt], ms = st.msum[nt];
+#pragma unroll
+        for (int o = 4; o < 32; o <<= 1) {
+          l += __shfl_xor_sync(0xffffffffu, l, o);
+          ms += __shfl_xor_sync(0xffffffffu, ms, o);
+        }
+        const int hs = 4 * nt + t;
+        if (hs < G) {
+          float* dst = part_b + (size_t)hs * kPartStride + 16 * g;
+#pragma unroll
+          for (int i = 0; i < 16; i += 4)
+            *reinterpret_cast<float4*>(dst + i) = make_float4(st.acc[nt][i] + ms, st.acc[nt][i + 1] + ms,
+                                                              st.acc[nt][i + 2] + ms, st.acc[nt][i + 3] + ms);
+          if (g == 0) {
+            part_b[(size_t)hs * kPartStride + 128] = st.m[nt];
+            part_b[(size_t)hs * kPartStride + 129] = l;
+          }
+        }
+      }
+    } else {
+      __syncthreads();  // window scratch no longer in use: the ring becomes merge buffers
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
         float l = st.l[nt], ms = st.msum[nt];
@@ -904,9 +970,7 @@ __global__ void __launch_bounds__(kMmaWarps * 32, (G <= 4) ? 4 : 3) decode_mma_k
         if (hs < G) {
           float* dst = mo + ((size_t)warp * G + hs) * kD + 16 * g;
 #pragma unroll
-          for (int i = 0; i < 16; i += 4)
-            *reinterpret_cast<float4*>(dst + i) =
-                make_float4(st.acc[nt][i] + ms, st.acc[nt][i + 1] + ms, st.acc[nt][i + 2] + ms, st.acc[nt][i + 3] + ms);
+          for (int i = 0; i < 16; ++i) dst[i] = st.acc[nt][i] + ms;
           if (g == 0) {
             ml[(warp * G + hs) * 2 + 0] = st.m[nt];
             ml[(warp * G + hs) * 2 + 1] = l;
@@ -914,28 +978,27 @@ __global__ void __launch_bounds__(kMmaWarps * 32, (G <= 4) ? 4 : 3) decode_mma_k
         }
       }
       __syncthreads();
-      // merge the warps into this CTA's partial for unit u
-      float* dstp = a.part + ((size_t)(c + u) * G) * kPartStride;
-      for (int i = threadIdx.x; i < G * kD; i += blockDim.x) {
-        const int hh = i / kD, ch = i % kD;
+      // thread -> (KV head, query head, channel); warps hh, hh + hkv, ... share KV head hh
+      for (int i = threadIdx.x; i < hkv * G * kD; i += blockDim.x) {
+        const int hh = i / (G * kD), gg = (i / kD) % G, ch = i % kD;
         float mx = -INFINITY;
-#pragma unroll
-        for (int w = 0; w < kMmaWarps; ++w) mx = fmaxf(mx, ml[(w * G + hh) * 2]);
+        for (int k = 0; k < wph; ++k) mx = fmaxf(mx, ml[((hh + k * hkv) * G + gg) * 2]);
         float o = 0.f, l = 0.f;
         if (mx != -INFINITY) {
-#pragma unroll
-          for (int w = 0; w < kMmaWarps; ++w) {
-            const float mw = ml[(w * G + hh) * 2];
+          for (int k = 0; k < wph; ++k) {
+            const int w = hh + k * hkv;
+            const float mw = ml[(w * G + gg) * 2];
             if (mw == -INFINITY) continue;
             const float sc = exp2f(mw - mx);
-            o = fmaf(mo[(w * G + hh) * kD + ch], sc, o);
-            l = fmaf(ml[(w * G + hh) * 2 + 1], sc, l);
+            o = fmaf(mo[((size_t)w * G + gg) * kD + ch], sc, o);
+            l = fmaf(ml[(w * G + gg) * 2 + 1], sc, l);
           }
         }
-        dstp[hh * kPartStride + ch] = o;
+        float* dst = a.part + ((size_t)(c + b) * a.hq + (size_t)hh * G + gg) * kPartStride;
+        dst[ch] = o;
         if (ch == 0) {
-          dstp[hh * kPartStride + 128] = mx;
-          dstp[hh * kPartStride + 129] = l;
+          dst[128] = mx;
+          dst[129] = l;
         }
       }
     }
@@ -943,12 +1006,16 @@ __global__ void __launch_bounds__(kMmaWarps * 32, (G <= 4) ? 4 : 3) decode_mma_k
 }
 
 // ---------------------------------------------------------------------------
-// Kernel 3: merge the splits of each unit, normalise, undo the value rotation
-// (un-permute, Hadamard, U_V^T) and write fp32 outputs.  One CTA per unit.
+// Kernel 3: merge the splits of each (b, KV head), normalise, undo the value
+// rotation (un-permute, Hadamard, U_V^T) and write fp32 outputs.  U_V is
+// staged in shared memory with all loads in flight together (warp w rows
+// 16w..16w+15, lane l columns 4l..4l+3), padded to 129 columns so that each
+// thread can walk its own output row without bank conflicts.
 // ---------------------------------------------------------------------------
 constexpr int kUPad = 129;
+constexpr int kCombThreads = 256;
 
-__global__ void __launch_bounds__(128) combine_kernel(DecodeArgs a) {
+__global__ void __launch_bounds__(kCombThreads) combine_kernel(DecodeArgs a) {
   extern __shared__ float smem[];
   float* us_ = smem;                 // U_V [128][129]
   float* xs = us_ + kD * kUPad;      // [G][128]
@@ -956,59 +1023,74 @@ __global__ void __launch_bounds__(128) combine_kernel(DecodeArgs a) {
   const int b = u / a.hkv, hk = u % a.hkv;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int G = a.g;
-  const float* uv = a.u_v + (size_t)hk * kD * kD;
-  for (int i = tid; i < kD * kD; i += blockDim.x) us_[(i / kD) * kUPad + (i % kD)] = uv[i];
+  {
+    const float* uv = a.u_v + (size_t)hk * kD * kD;
+    float4 r[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) r[i] = __ldg(reinterpret_cast<const float4*>(uv + (size_t)(16 * warp + i) * kD) + lane);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      float* row = us_ + (16 * warp + i) * kUPad + 4 * lane;
+      row[0] = r[i].x;
+      row[1] = r[i].y;
+      row[2] = r[i].z;
+      row[3] = r[i].w;
+    }
+  }
   const UnitShape sh = unit_shape(clamp_len(a.context_lens, b, a.mbps, a.status, false));
   const long long total = a.prefix[a.batch];
-  float* outp = a.out + ((size_t)b * a.hq + hk * G) * kD;
+  float* outp = a.out + ((size_t)b * a.hq + (size_t)hk * G) * kD;
   if (sh.cost == 0 || total == 0) {
     for (int i = tid; i < G * kD; i += blockDim.x) outp[i] = 0.f;
     return;
   }
-  const long long pu = a.prefix[b] + (long long)hk * sh.cost;
-  const int nc = (int)min((long long)a.nc, total);
+  const long long pu = a.prefix[b];
+  const int nc = working_ctas(a, total);
   const int c0 = cta_of(pu, total, nc);
   const int c1 = cta_of(pu + sh.cost - 1, total, nc);
-  // merge splits: thread = channel
-  for (int g = 0; g < G; ++g) {
+  for (int i = tid; i < G * kD; i += blockDim.x) {
+    const int gg = i / kD, ch = i % kD;
+    const size_t head = (size_t)hk * G + gg;
     float mx = -INFINITY;
-    for (int c = c0; c <= c1; ++c) mx = fmaxf(mx, a.part[((size_t)(c + u) * G + g) * kPartStride + 128]);
+    for (int c = c0; c <= c1; ++c) mx = fmaxf(mx, a.part[((size_t)(c + b) * a.hq + head) * kPartStride + 128]);
     float o = 0.f, l = 0.f;
     if (mx != -INFINITY) {
       for (int c = c0; c <= c1; ++c) {
-        const float* src = a.part + ((size_t)(c + u) * G + g) * kPartStride;
+        const float* src = a.part + ((size_t)(c + b) * a.hq + head) * kPartStride;
         const float mw = src[128];
         if (mw == -INFINITY) continue;
         const float sc = exp2f(mw - mx);
-        o = fmaf(src[tid], sc, o);
+        o = fmaf(src[ch], sc, o);
         l = fmaf(src[129], sc, l);
       }
     }
-    xs[g * kD + tid] = (l > 0.f) ? o / l : 0.f;
+    xs[gg * kD + ch] = (l > 0.f) ? o / l : 0.f;
   }
   __syncthreads();
   // un-permute + Hadamard, one warp per head: lane holds pre-permutation
   // channels l + 32a = rotated channels 4*rev5(l) + rev2(a)
-  for (int g = warp; g < G; g += 4) {
+  for (int gg = warp; gg < G; gg += kCombThreads / 32) {
     const int r = rev5(lane);
     float y[4];
-    y[0] = xs[g * kD + 4 * r + 0];
-    y[1] = xs[g * kD + 4 * r + 2];
-    y[2] = xs[g * kD + 4 * r + 1];
-    y[3] = xs[g * kD + 4 * r + 3];
+    y[0] = xs[gg * kD + 4 * r + 0];
+    y[1] = xs[gg * kD + 4 * r + 2];
+    y[2] = xs[gg * kD + 4 * r + 1];
+    y[3] = xs[gg * kD + 4 * r + 3];
     __syncwarp();
     wht128_warp(y, lane);
 #pragma unroll
-    for (int j = 0; j < 4; ++j) xs[g * kD + lane + 32 * j] = y[j] * kInvSqrtD;
+    for (int j = 0; j < 4; ++j) xs[gg * kD + lane + 32 * j] = y[j] * kInvSqrtD;
   }
   __syncthreads();
-  // o_c = sum_i x_i U_V[c][i]: thread = output channel c
-  for (int g = 0; g < G; ++g) {
+  // o_c = sum_i x_i U_V[c][i]: thread = (output channel, half of the heads)
+  const int ch = tid & (kD - 1), half = tid >> 7;
+  for (int gg = half; gg < G; gg += 2) {
     float acc = 0.f;
-    const float* xr = xs + g * kD;
-#pragma unroll 8
-    for (int i = 0; i < kD; ++i) acc = fmaf(xr[i], us_[tid * kUPad + i], acc);
-    outp[g * kD + tid] = acc;
+    const float* xr = xs + gg * kD;
+    const float* ur = us_ + ch * kUPad;
+#pragma unroll 16
+    for (int i = 0; i < kD; ++i) acc = fmaf(xr[i], ur[i], acc);
+    outp[gg * kD + ch] = acc;
   }
 }
 
@@ -1023,17 +1105,22 @@ static okv_status launch_decode_simt(const DecodeArgs& a, cudaStream_t s) {
 }
 
 template <int G>
-static okv_status launch_decode_mma(const DecodeArgs& a, cudaStream_t s) {
-  const size_t smem = MmaCfg<G>::smem_bytes();
-  static bool configured = false;  // the attribute is per function; set it once
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(decode_mma_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
-    if (e != cudaSuccess) return fail(OKV_ERR_CUDA, "decode smem attribute: %s", cudaGetErrorString(e));
-    configured = true;
-  }
-  decode_mma_kernel<G><<<a.nc, kMmaWarps * 32, smem, s>>>(a);
+static okv_status launch_decode_heads(const DecodeArgs& a, cudaStream_t s) {
+  const size_t smem = HCfg<G>::smem_bytes();
+  cudaError_t e = cudaFuncSetAttribute(decode_heads_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem);
+  if (e != cudaSuccess) return fail(OKV_ERR_CUDA, "decode smem attribute: %s", cudaGetErrorString(e));
+  decode_heads_kernel<G><<<a.nc, kHW * 32, smem, s>>>(a);
   return check_launch("decode");
+}
+
+bool decode_uses_tensor_cores(int g, int hkv) {
+  return (g == 1 || g == 2 || g == 4 || g == 8) && (hkv == 1 || hkv == 2 || hkv == 4 || hkv == 8);
+}
+
+int decode_ctas_per_sm(int g, int hkv) {
+  if (decode_uses_tensor_cores(g, hkv)) return g <= 4 ? 2 : 1;
+  return 4;
 }
 
 okv_status launch_decode(const okv_cache_desc* d, const void* q, int B, const int32_t* seq_slot,
@@ -1066,28 +1153,40 @@ okv_status launch_decode(const okv_cache_desc* d, const void* q, int B, const in
   a.num_slots = d->num_seq_slots;
   a.mbps = d->max_blocks_per_seq;
 
-  qrot_kernel<<<dim3(B, a.hq), 128, 0, s>>>(a);
+  const size_t qsmem = (size_t)a.g * 8 * kD * sizeof(float);
+  cudaError_t e = cudaFuncSetAttribute(qrot_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)qsmem);
+  if (e != cudaSuccess) return fail(OKV_ERR_CUDA, "query rotation smem attribute: %s", cudaGetErrorString(e));
+  qrot_kernel<<<dim3(B, a.hkv), kPrepThreads, qsmem, s>>>(a);
   okv_status st = check_launch("query rotation");
   if (st != OKV_OK) return st;
   cudaEvent_t ev0, ev1;
   take_decode_events(&ev0, &ev1);
   if (ev0 != nullptr && cudaEventRecordWithFlags(ev0, s, cudaEventRecordExternal) != cudaSuccess)
     return fail(OKV_ERR_CUDA, "cudaEventRecord failed");
-  switch (a.g) {
-    case 1: st = launch_decode_mma<1>(a, s); break;
-    case 2: st = launch_decode_mma<2>(a, s); break;
-    case 4: st = launch_decode_mma<4>(a, s); break;
-    case 8: st = launch_decode_mma<8>(a, s); break;
-    case 16: st = launch_decode_simt<16>(a, s); break;
-    default: return fail(OKV_ERR_UNSUPPORTED, "group size %d (Hq/Hkv) not in {1,2,4,8,16}", a.g);
+  if (decode_uses_tensor_cores(a.g, a.hkv)) {
+    switch (a.g) {
+      case 1: st = launch_decode_heads<1>(a, s); break;
+      case 2: st = launch_decode_heads<2>(a, s); break;
+      case 4: st = launch_decode_heads<4>(a, s); break;
+      default: st = launch_decode_heads<8>(a, s); break;
+    }
+  } else {
+    switch (a.g) {
+      case 1: st = launch_decode_simt<1>(a, s); break;
+      case 2: st = launch_decode_simt<2>(a, s); break;
+      case 4: st = launch_decode_simt<4>(a, s); break;
+      case 8: st = launch_decode_simt<8>(a, s); break;
+      case 16: st = launch_decode_simt<16>(a, s); break;
+      default: return fail(OKV_ERR_UNSUPPORTED, "group size %d (Hq/Hkv) not in {1,2,4,8,16}", a.g);
+    }
   }
   if (st != OKV_OK) return st;
   if (ev1 != nullptr && cudaEventRecordWithFlags(ev1, s, cudaEventRecordExternal) != cudaSuccess)
     return fail(OKV_ERR_CUDA, "cudaEventRecord failed");
   const size_t csmem = (size_t)(kD * kUPad + a.g * kD) * sizeof(float);
-  cudaError_t e = cudaFuncSetAttribute(combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)csmem);
+  e = cudaFuncSetAttribute(combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)csmem);
   if (e != cudaSuccess) return fail(OKV_ERR_CUDA, "combine smem attribute: %s", cudaGetErrorString(e));
-  combine_kernel<<<plan.num_units, 128, csmem, s>>>(a);
+  combine_kernel<<<B * a.hkv, kCombThreads, csmem, s>>>(a);
   return check_launch("combine");
 }
 

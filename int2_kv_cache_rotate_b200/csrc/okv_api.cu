@@ -78,7 +78,7 @@ DecodePlan make_decode_plan(int batch, int hq, int hkv) {
   p.hkv = hkv;
   p.g = hq / hkv;
   const int sms = device_sm_count();
-  p.num_ctas = (sms > 0 ? sms : 148) * kCtasPerSm;
+  p.num_ctas = (sms > 0 ? sms : 148) * decode_ctas_per_sm(p.g, hkv);
   p.num_units = batch * hkv;
   size_t off = 0;
   p.qrot_off = off;
@@ -92,7 +92,7 @@ DecodePlan make_decode_plan(int batch, int hq, int hkv) {
   p.prefix_off = off;
   off = align_up(off + (size_t)(batch + 1) * sizeof(int32_t), 256);
   p.part_off = off;
-  off = align_up(off + (size_t)(p.num_ctas + p.num_units) * p.g * kPartStride * sizeof(float), 256);
+  off = align_up(off + (size_t)(p.num_ctas + batch) * hq * kPartStride * sizeof(float), 256);
   p.total = off;
   return p;
 }

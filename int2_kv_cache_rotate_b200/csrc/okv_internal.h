@@ -28,12 +28,14 @@ struct DecodePlan {
   size_t qscale_off = 0;    // fp32 [B][Hq][4] (score scale, min term, sigma, sum)
   size_t qwin_off = 0;      // fp16 [B][Hq][2][128] scaled query hi/lo halves (window MMA)
   size_t prefix_off = 0;    // int32 [B+1] cost prefix over batch entries
-  size_t part_off = 0;      // fp32 [(num_ctas + num_units)][G][kPartStride]
+  size_t part_off = 0;      // fp32 [(num_ctas + batch)][Hq][kPartStride]
   size_t total = 0;
 };
 constexpr int kPartStride = 132;  // o'[128], m, l, 2 spare
-constexpr int kWinCost = 16;      // cost of a unit's window in block units
-constexpr int kCtasPerSm = 4;     // resident split-K CTAs per SM
+constexpr int kWinCost = 8;       // cost of an entry's window in block units (all heads)
+// split-K kernel choice and residency (decode.cu)
+bool decode_uses_tensor_cores(int g, int hkv);
+int decode_ctas_per_sm(int g, int hkv);
 
 DecodePlan make_decode_plan(int batch, int hq, int hkv);
 

@@ -246,3 +246,23 @@ def test_end_to_end_calibrated_fused_path():
     den = np.abs(want).max(axis=-1)
     diff = np.abs(got - want).max(axis=-1)
     assert np.all(diff <= TOL * den + bound), (diff / den, bound / den)
+
+
+def test_decode_partial_last_block_with_live_tail():
+    """The last INT2 block is only partly inside the context while its other
+    slots hold real tokens (the cache was filled further than the decode
+    length), and entries so short that a split streams a single block."""
+    okv = _okv()
+    fill = [3000, 129, 1, 777]
+    dec = [2900, 129, 1, 770]
+    gc, oc, lay, zs = _fill_pre_rotated(21, 32, 8, fill)
+    q = np.stack([WL.sample_queries(21, 0, 0, h, len(fill), 4, extra=3) for h in range(8)], 1).reshape(len(fill), 32, 128)
+    seq = np.arange(len(fill), dtype=np.int32)
+    for _ in range(3):
+        got = okv.decode_attention(gc, _t(q, torch.bfloat16), _t(seq), _t(lay.table),
+                                   _t(np.array(dec, np.int32))).cpu().numpy()
+        assert np.isfinite(got).all()
+    # the oracle sees the same cache as the kernels: positions < decode length,
+    # the window ring rows holding whatever was appended last
+    for b in range(len(fill)):
+        assert oc.seqs[(b, 0, 0)]["set"][:dec[b]].all()
