@@ -22,30 +22,16 @@ struct AppendArgs {
   int hkv, num_blocks, num_slots, mbps;
 };
 
-// One CTA per (token, KV head, K|V).  Lane l of warp 0 ends up owning the
-// pre-permutation channels l + 32a, which after P_br are rotated channels
-// 4*rev5(l) + rev2(a): exactly the four codes of packed byte rev5(l).  So the
-// permutation costs nothing: it is the choice of which byte a lane writes.
-template <bool kPre>
-__global__ void __launch_bounds__(128) append_kernel(AppendArgs a) {
-  __shared__ float red[4][kD];
-  const int t = blockIdx.x, h = blockIdx.y, kind = blockIdx.z;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const size_t vec = ((size_t)t * a.hkv + h) * kD;
-  float y[4];
-  if constexpr (!kPre) {
-    const __nv_bfloat16* src = (const __nv_bfloat16*)(kind ? a.v : a.k) + vec;
-    rotate_cta(src, (kind ? a.u_v : a.u_k) + (size_t)h * kD * kD, red, y);
-    if (warp != 0) return;
-  } else {
-    const float* src = (const float*)(kind ? a.v : a.k) + vec;
-    const float4 z4 = *reinterpret_cast<const float4*>(src + 4 * rev5(lane));
-    y[0] = z4.x;  // rotated channel 4r+0 <- pre-permutation index l
-    y[1] = z4.z;  // 4r+2 <- l+32
-    y[2] = z4.y;  // 4r+1 <- l+64
-    y[3] = z4.w;  // 4r+3 <- l+96
-  }
+constexpr int kAppThreads = 256;
+constexpr int kAppRound = 8;    // tokens reduced per round (one per warp)
+constexpr int kAppTokens = 32;  // tokens per CTA
 
+// Validate token t's destination and write everything for one rotated vector.
+// Lane l owns pre-permutation channels l + 32a, which after P_br are rotated
+// channels 4*rev5(l) + rev2(a): exactly the four codes of packed byte rev5(l).
+// So the permutation costs nothing: it is the choice of which byte a lane writes.
+__device__ __forceinline__ void finish_token(const AppendArgs& a, int t, int h, int kind, const float y[4],
+                                             int lane) {
   const int slot = a.seq_slot[t];
   const int p = a.pos[t];
   if (slot < 0 || slot >= a.num_slots) {
@@ -87,6 +73,74 @@ __global__ void __launch_bounds__(128) append_kernel(AppendArgs a) {
   }
 }
 
+// One CTA per (32-token tile, KV head, K|V), 8 warps.  U stays in registers
+// for the whole tile (warp w holds rows 16w..16w+15, lane l columns
+// 4l..4l+3: one round of loads); each round multiplies 8 tokens, reduces the
+// 8 warps' partial sums through shared memory, and hands token i to warp i
+// for the Hadamard butterfly, the bit-reversal remap and the quantiser.
+template <bool kPre>
+__global__ void __launch_bounds__(kAppThreads) append_kernel(AppendArgs a, int T) {
+  __shared__ float red[kPre ? 1 : kAppRound][8][kD];
+  const int h = blockIdx.y, kind = blockIdx.z;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int t0 = blockIdx.x * kAppTokens, t1 = min(T, t0 + kAppTokens);
+  float4 u[16];
+  if constexpr (!kPre) {
+    const float* U = (kind ? a.u_v : a.u_k) + (size_t)h * kD * kD;
+#pragma unroll
+    for (int r = 0; r < 16; ++r) u[r] = __ldg(reinterpret_cast<const float4*>(U + (size_t)(16 * warp + r) * kD) + lane);
+  }
+  for (int r0 = t0; r0 < t1; r0 += kAppRound) {
+    const int nr = min(kAppRound, t1 - r0);
+    float y[4];
+    if constexpr (!kPre) {
+      const __nv_bfloat16* src = (const __nv_bfloat16*)(kind ? a.v : a.k);
+      float xv[kAppRound];
+#pragma unroll
+      for (int i = 0; i < kAppRound; ++i)
+        xv[i] = i < nr ? __bfloat162float(src[((size_t)(r0 + i) * a.hkv + h) * kD + 16 * warp + (lane & 15)]) : 0.f;
+#pragma unroll
+      for (int i = 0; i < kAppRound; ++i) {
+        if (i >= nr) break;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int r = 0; r < 16; ++r) {
+          const float x = __shfl_sync(0xffffffffu, xv[i], r);
+          acc.x = fmaf(x, u[r].x, acc.x);
+          acc.y = fmaf(x, u[r].y, acc.y);
+          acc.z = fmaf(x, u[r].z, acc.z);
+          acc.w = fmaf(x, u[r].w, acc.w);
+        }
+        *reinterpret_cast<float4*>(&red[i][warp][4 * lane]) = acc;
+      }
+      __syncthreads();
+      if (warp < nr) {
+#pragma unroll
+        for (int aa = 0; aa < 4; ++aa) {
+          float s = 0.f;
+#pragma unroll
+          for (int w = 0; w < 8; ++w) s += red[warp][w][lane + 32 * aa];
+          y[aa] = s;
+        }
+        wht128_warp(y, lane);
+#pragma unroll
+        for (int aa = 0; aa < 4; ++aa) y[aa] *= kInvSqrtD;
+      }
+      __syncthreads();  // red is reused by the next round
+    } else {
+      if (warp < nr) {
+        const float* src = (const float*)(kind ? a.v : a.k) + ((size_t)(r0 + warp) * a.hkv + h) * kD;
+        const float4 z4 = *reinterpret_cast<const float4*>(src + 4 * rev5(lane));
+        y[0] = z4.x;  // rotated channel 4r+0 <- pre-permutation index l
+        y[1] = z4.z;  // 4r+2 <- l+32
+        y[2] = z4.y;  // 4r+1 <- l+64
+        y[3] = z4.w;  // 4r+3 <- l+96
+      }
+    }
+    if (warp < nr) finish_token(a, r0 + warp, h, kind, y, lane);
+  }
+}
+
 }  // namespace
 
 okv_status launch_append(const okv_cache_desc* d, const void* k, const void* v, int T,
@@ -110,11 +164,11 @@ okv_status launch_append(const okv_cache_desc* d, const void* k, const void* v, 
   a.num_blocks = d->num_blocks;
   a.num_slots = d->num_seq_slots;
   a.mbps = d->max_blocks_per_seq;
-  dim3 grid(T, d->num_kv_heads, 2);
+  dim3 grid((T + kAppTokens - 1) / kAppTokens, d->num_kv_heads, 2);
   if (flags & OKV_PRE_ROTATED) {
-    append_kernel<true><<<grid, 32, 0, s>>>(a);
+    append_kernel<true><<<grid, kAppThreads, 0, s>>>(a, T);
   } else {
-    append_kernel<false><<<grid, 128, 0, s>>>(a);
+    append_kernel<false><<<grid, kAppThreads, 0, s>>>(a, T);
   }
   return check_launch("append");
 }

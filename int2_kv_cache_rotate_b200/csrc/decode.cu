@@ -8,11 +8,12 @@ namespace okv {
 
 // ---------------------------------------------------------------------------
 // Work partition.  Batch entry b with L tokens costs ceil(max(L-W,0)/16)
-// blocks (every KV head of a block is one contiguous run) plus kWinCost for
-// its fp16 window (if L > 0).  Entries are laid end to end in "cost space";
-// split-K CTA c takes the contiguous range [c*total/NC, (c+1)*total/NC).
-// Inside an entry, cost positions [0, kWinCost) stand for the window and the
-// rest for the blocks in order.  A (entry, CTA) pair writes partial slot
+// blocks (every KV head of a block is one contiguous run) plus kWinCost per
+// 16-row chunk of its fp16 window.  Entries are laid end to end in "cost
+// space"; split-K CTA c takes the contiguous range [c*total/NC, (c+1)*total/NC).
+// Inside an entry, cost positions [0, n_chunks * kWinCost) stand for the
+// window chunks (chunk i belongs to the CTA holding position i * kWinCost) and
+// the rest for the blocks in order.  A (entry, CTA) pair writes partial slot
 // c + b (all query heads): distinct for distinct pairs because CTAs and
 // entries are both contiguous.
 // ---------------------------------------------------------------------------
@@ -21,6 +22,7 @@ struct UnitShape {
   int n_int2;   // tokens read from INT2 blocks
   int n_pages;  // INT2 blocks touched
   int n_win;    // tokens read from the fp16 window
+  int n_wchunk; // 16-row chunks of the window
   int win_cost;
   int cost;
 };
@@ -31,7 +33,8 @@ __device__ __forceinline__ UnitShape unit_shape(int len) {
   s.n_int2 = len > kWin ? len - kWin : 0;
   s.n_pages = (s.n_int2 + kBlock - 1) / kBlock;
   s.n_win = len < kWin ? len : kWin;
-  s.win_cost = len > 0 ? kWinCost : 0;
+  s.n_wchunk = (s.n_win + kBlock - 1) / kBlock;
+  s.win_cost = s.n_wchunk * kWinCost;
   s.cost = s.n_pages + s.win_cost;
   return s;
 }
@@ -121,9 +124,16 @@ __global__ void __launch_bounds__(kPrepThreads) qrot_kernel(DecodeArgs a) {
   float4 u[16];
 #pragma unroll
   for (int r = 0; r < 16; ++r) u[r] = __ldg(reinterpret_cast<const float4*>(U + (size_t)(16 * warp + r) * kD) + lane);
-  for (int gg = 0; gg < G; ++gg) {
-    const __nv_bfloat16* qv = a.q + ((size_t)b * a.hq + (size_t)hk * G + gg) * kD;
-    const float xv = __bfloat162float(qv[16 * warp + (lane & 15)]);
+  float xq[16];  // this lane's input channel 16*warp + (lane & 15), every head of the group
+  {
+    const __nv_bfloat16* qv = a.q + ((size_t)b * a.hq + (size_t)hk * G) * kD + 16 * warp + (lane & 15);
+#pragma unroll
+    for (int gg = 0; gg < 16; ++gg) xq[gg] = gg < G ? __bfloat162float(qv[(size_t)gg * kD]) : 0.f;
+  }
+#pragma unroll
+  for (int gg = 0; gg < 16; ++gg) {
+    if (gg >= G) break;
+    const float xv = xq[gg];
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
     for (int r = 0; r < 16; ++r) {
@@ -329,12 +339,13 @@ __global__ void __launch_bounds__(kDecWarps * 32) decode_simt_kernel(DecodeArgs 
         for (int j = 0; j < 4; ++j) st.o[gg][j] = 0.f;
       }
       if (slot_ok) {
-        if (l0 == 0 && us.win_cost > 0) {
+        {
           const __half* kbase = a.ring + (((size_t)slot * a.hkv + hk) * 2 + 0) * kWin * kD;
           const __half* vbase = a.ring + (((size_t)slot * a.hkv + hk) * 2 + 1) * kWin * kD;
           const int first = us.len - us.n_win;
-          const int nchunk = (us.n_win + kBlock - 1) / kBlock;
-          for (int ci = warp; ci < nchunk; ci += kDecWarps) {
+          const int ci0 = (l0 + kWinCost - 1) / kWinCost;
+          const int ci1 = min(us.n_wchunk, (l1 + kWinCost - 1) / kWinCost);
+          for (int ci = ci0 + warp; ci < ci1; ci += kDecWarps) {
             const int ntok = min(kBlock, us.n_win - ci * kBlock);
             simt_chunk<G, true>(a, qs, nullptr, kbase, vbase, first + ci * kBlock, ntok, st, lane);
           }
@@ -786,8 +797,10 @@ __global__ void __launch_bounds__(kHW * 32, (G <= 4) ? 2 : 1) decode_heads_kerne
     __syncthreads();  // every warp is done with the ring: it becomes window scratch, then merge buffers
 
     // ---------------- fp16 window: chunks ci = grp, grp + wph, ... of this warp's head ----------------
-    const int nchunk = (l0 == 0 && us.win_cost > 0 && slot_ok) ? (us.n_win + 15) / 16 : 0;
-    if (grp < nchunk) {
+    // window chunks owned by this CTA: chunk ci where l0 <= ci * kWinCost < l1
+    const int ci0 = (l0 + kWinCost - 1) / kWinCost;
+    const int ci1 = slot_ok ? min(us.n_wchunk, (l1 + kWinCost - 1) / kWinCost) : ci0;
+    if (ci0 + grp < ci1) {
       const __half* kr = a.ring + (((size_t)slot * hkv + head) * 2 + 0) * kWin * kD;
       const __half* vr = a.ring + (((size_t)slot * hkv + head) * 2 + 1) * kWin * kD;
       unsigned char* scratch = ring + warp * kWarpScratch;
@@ -820,7 +833,7 @@ __global__ void __launch_bounds__(kHW * 32, (G <= 4) ? 2 : 1) decode_heads_kerne
 #pragma unroll
           for (int i = 0; i < 4; ++i) wacc[nt][mt][i] = 0.f;
       }
-      for (int ci = grp; ci < nchunk; ci += wph) {
+      for (int ci = ci0 + grp; ci < ci1; ci += wph) {
         const int r0 = 16 * ci;
         // stage the V rows (swizzled 16-byte chunks) for the transposing loads
 #pragma unroll
@@ -1014,6 +1027,7 @@ __global__ void __launch_bounds__(kHW * 32, (G <= 4) ? 2 : 1) decode_heads_kerne
 // ---------------------------------------------------------------------------
 constexpr int kUPad = 129;
 constexpr int kCombThreads = 256;
+constexpr int kMaxSplits = 1024;  // >= split-K CTAs (at most 4 per SM)
 
 __global__ void __launch_bounds__(kCombThreads) combine_kernel(DecodeArgs a) {
   extern __shared__ float smem[];
@@ -1047,24 +1061,67 @@ __global__ void __launch_bounds__(kCombThreads) combine_kernel(DecodeArgs a) {
   const long long pu = a.prefix[b];
   const int nc = working_ctas(a, total);
   const int c0 = cta_of(pu, total, nc);
-  const int c1 = cta_of(pu + sh.cost - 1, total, nc);
-  for (int i = tid; i < G * kD; i += blockDim.x) {
-    const int gg = i / kD, ch = i % kD;
-    const size_t head = (size_t)hk * G + gg;
+  const int ns = cta_of(pu + sh.cost - 1, total, nc) - c0 + 1;  // splits of this entry
+  float* wts = xs + G * kD;                 // [G][kMaxSplits] split weights 2^(m_c - M)
+  float* red = wts + G * kMaxSplits;        // [G] 1/l
+  float* wpart = red + ((G + 3) & ~3);      // [8 warps][G][128] partial sums (16-B aligned)
+  const float* base = a.part + ((size_t)(c0 + b) * a.hq + (size_t)hk * G) * kPartStride;
+  const size_t split_stride = (size_t)a.hq * kPartStride;
+  // 1) per head (one warp each): max of the split maxima, weights, 1/l
+  for (int gg = warp; gg < G; gg += kCombThreads / 32) {
     float mx = -INFINITY;
-    for (int c = c0; c <= c1; ++c) mx = fmaxf(mx, a.part[((size_t)(c + b) * a.hq + head) * kPartStride + 128]);
-    float o = 0.f, l = 0.f;
-    if (mx != -INFINITY) {
-      for (int c = c0; c <= c1; ++c) {
-        const float* src = a.part + ((size_t)(c + b) * a.hq + head) * kPartStride;
-        const float mw = src[128];
-        if (mw == -INFINITY) continue;
-        const float sc = exp2f(mw - mx);
-        o = fmaf(src[ch], sc, o);
-        l = fmaf(src[129], sc, l);
+    for (int c = lane; c < ns; c += 32) mx = fmaxf(mx, base[c * split_stride + (size_t)gg * kPartStride + 128]);
+    mx = warp_max(mx);
+    float l = 0.f;
+    for (int c = lane; c < ns; c += 32) {
+      const float* src = base + c * split_stride + (size_t)gg * kPartStride;
+      const float w = (mx == -INFINITY || src[128] == -INFINITY) ? 0.f : exp2f(src[128] - mx);
+      wts[gg * kMaxSplits + c] = w;
+      l = fmaf(src[129], w, l);
+    }
+    l = warp_sum(l);
+    if (lane == 0) red[gg] = l > 0.f ? 1.f / l : 0.f;
+  }
+  __syncthreads();
+  // 2) weighted sum of the splits: warp w takes splits w, w+8, ...; lane l
+  //    channels 4l..4l+3; four splits in flight per iteration
+  for (int gg = 0; gg < G; ++gg) {
+    const float* hb = base + (size_t)gg * kPartStride + 4 * lane;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    int c = warp;
+    for (; c + 24 < ns; c += 32) {
+      float4 x[4];
+      float w[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        x[k] = *reinterpret_cast<const float4*>(hb + (size_t)(c + 8 * k) * split_stride);
+        w[k] = wts[gg * kMaxSplits + c + 8 * k];
+      }
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        acc.x = fmaf(x[k].x, w[k], acc.x);
+        acc.y = fmaf(x[k].y, w[k], acc.y);
+        acc.z = fmaf(x[k].z, w[k], acc.z);
+        acc.w = fmaf(x[k].w, w[k], acc.w);
       }
     }
-    xs[gg * kD + ch] = (l > 0.f) ? o / l : 0.f;
+    for (; c < ns; c += 8) {
+      const float4 x = *reinterpret_cast<const float4*>(hb + (size_t)c * split_stride);
+      const float w = wts[gg * kMaxSplits + c];
+      acc.x = fmaf(x.x, w, acc.x);
+      acc.y = fmaf(x.y, w, acc.y);
+      acc.z = fmaf(x.z, w, acc.z);
+      acc.w = fmaf(x.w, w, acc.w);
+    }
+    *reinterpret_cast<float4*>(wpart + ((size_t)warp * G + gg) * kD + 4 * lane) = acc;
+  }
+  __syncthreads();
+  for (int i = tid; i < G * kD; i += blockDim.x) {
+    const int gg = i / kD, ch = i % kD;
+    float o = 0.f;
+#pragma unroll
+    for (int w = 0; w < kCombThreads / 32; ++w) o += wpart[((size_t)w * G + gg) * kD + ch];
+    xs[i] = o * red[gg];
   }
   __syncthreads();
   // un-permute + Hadamard, one warp per head: lane holds pre-permutation
@@ -1183,7 +1240,7 @@ okv_status launch_decode(const okv_cache_desc* d, const void* q, int B, const in
   if (st != OKV_OK) return st;
   if (ev1 != nullptr && cudaEventRecordWithFlags(ev1, s, cudaEventRecordExternal) != cudaSuccess)
     return fail(OKV_ERR_CUDA, "cudaEventRecord failed");
-  const size_t csmem = (size_t)(kD * kUPad + a.g * kD) * sizeof(float);
+  const size_t csmem = (size_t)(kD * kUPad + a.g * kD + a.g * kMaxSplits + ((a.g + 3) & ~3) + 8 * a.g * kD) * sizeof(float);
   e = cudaFuncSetAttribute(combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)csmem);
   if (e != cudaSuccess) return fail(OKV_ERR_CUDA, "combine smem attribute: %s", cudaGetErrorString(e));
   combine_kernel<<<B * a.hkv, kCombThreads, csmem, s>>>(a);

@@ -79,6 +79,7 @@ DecodePlan make_decode_plan(int batch, int hq, int hkv) {
   p.g = hq / hkv;
   const int sms = device_sm_count();
   p.num_ctas = (sms > 0 ? sms : 148) * decode_ctas_per_sm(p.g, hkv);
+  if (p.num_ctas > 1024) p.num_ctas = 1024;  // the combine caches one weight per split
   p.num_units = batch * hkv;
   size_t off = 0;
   p.qrot_off = off;

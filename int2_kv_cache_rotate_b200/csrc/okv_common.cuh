@@ -118,46 +118,6 @@ __device__ __forceinline__ Quantized quantize_warp(const float y[4]) {
 
 }  // namespace okv
 
-namespace okv {
-
-// x = in . U (fp32 accumulate), then the normalised Hadamard, on a CTA of 128
-// threads.  Warp w sums input channels 32w..32w+31; the four partials meet in
-// shared memory; warp 0 finishes and returns y[a] = (x H)[l + 32a].
-// `in` holds 128 consecutive bf16 values; U is row-major [128][128].
-template <typename InT>
-__device__ __forceinline__ void rotate_cta(const InT* __restrict__ in, const float* __restrict__ u,
-                                           float (*red)[kD], float y[4]) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  float xin;
-  if constexpr (sizeof(InT) == 2) {
-    xin = __bfloat162float(in[32 * warp + lane]);
-  } else {
-    xin = in[32 * warp + lane];
-  }
-  float acc[4] = {0.f, 0.f, 0.f, 0.f};
-  const float* urow = u + (size_t)(32 * warp) * kD + lane;
-#pragma unroll 8
-  for (int cc = 0; cc < 32; ++cc) {
-    const float xc = __shfl_sync(0xffffffffu, xin, cc);
-#pragma unroll
-    for (int a = 0; a < 4; ++a) acc[a] = fmaf(xc, __ldg(urow + cc * kD + 32 * a), acc[a]);
-  }
-#pragma unroll
-  for (int a = 0; a < 4; ++a) red[warp][lane + 32 * a] = acc[a];
-  __syncthreads();
-  if (warp == 0) {
-#pragma unroll
-    for (int a = 0; a < 4; ++a) {
-      const int i = lane + 32 * a;
-      y[a] = ((red[0][i] + red[1][i]) + red[2][i]) + red[3][i];
-    }
-    wht128_warp(y, lane);
-#pragma unroll
-    for (int a = 0; a < 4; ++a) y[a] *= kInvSqrtD;
-  }
-}
-
-}  // namespace okv
 
 namespace okv {
 
