@@ -1,6 +1,8 @@
 // Decode attention over the INT2 paged cache: query rotation, split-K
 // attention with online softmax, and the split combine with the value
 // un-rotation.
+#include <type_traits>
+
 #include "okv_common.cuh"
 #include "okv_internal.h"
 
@@ -431,11 +433,11 @@ __global__ void __launch_bounds__(kDecWarps * 32) decode_simt_kernel(DecodeArgs 
 // fp16 hi+lo pairs), folded into the warp's state in registers.
 // ---------------------------------------------------------------------------
 constexpr int kHW = 8;                             // warps per CTA
-constexpr int kHStages = 4;                        // ring stages
+constexpr int kHStages = 5;                        // ring stages (3 in flight ahead of the consumers)
 constexpr int kSlotsPerStage = 16;                 // block-heads per stage
 constexpr int kHStageBytes = kSlotsPerStage * kBlockHeadBytes;  // 18432
 constexpr int kPStride = 40;                       // u16 per head row of the P' tile
-constexpr int kWarpScratch = kHStages * kHStageBytes / kHW;     // 9216 B of ring per warp
+constexpr int kWarpScratch = 9216;                 // ring bytes each warp may use as window scratch
 constexpr uint32_t kM2 = 0x03030303u;
 
 template <int G>
@@ -443,8 +445,11 @@ struct HCfg {
   static constexpr int NT = G <= 4 ? 1 : G / 4;  // n-tiles of 8 columns = 4 heads x 2 limbs
   static constexpr int HP = 4 * NT;              // heads incl. padding
   static constexpr size_t ring_bytes = (size_t)kHStages * kHStageBytes;
+  static constexpr int acc_stride = NT * 16 + 1;   // per-thread fp32 accumulator row (padded)
+  static constexpr size_t acc_bytes = (size_t)kHW * 32 * acc_stride * 4;
   static constexpr size_t smem_bytes() {
     return ring_bytes                            // ring (reused for window scratch and merging)
+           + acc_bytes                           // fp32 o' accumulators, touched only on flushes
            + (size_t)2 * kHStages * 8            // full / empty mbarriers
            + (size_t)kHStages * kSlotsPerStage   // tokens per block slot
            + (size_t)kHW * HP * kPStride * 2     // P' tiles
@@ -452,6 +457,7 @@ struct HCfg {
   }
 };
 static_assert(kHW * 8 * kD * 4 <= kHStages * kHStageBytes, "merge buffer must fit the ring");
+static_assert(kHStages * kHStageBytes / kHW >= 9216, "window scratch per warp");
 static_assert(4096 + 8 * 64 + 8 * kD * 4 <= kWarpScratch, "window scratch must fit a warp's share of the ring");
 
 __device__ __forceinline__ float lo_half(uint32_t w) {
@@ -500,23 +506,23 @@ template <int G>
 struct MmaWarpState {
   static constexpr int NT = HCfg<G>::NT;
   float m[NT], l[NT], msum[NT];
-  float acc[NT][16];   // fp32 o' for channels 16g + 0..15 of head 4nt + t
-  int acci[NT][8][4];  // exact int32 o' contributions since the last flush (row scale 4^f)
+  float* acc;          // shared row: fp32 o' for channels 16g + 0..15 of head 4nt + t at [16 nt + i]
 };
 
 // acci[mt] holds channel 16g + 2mt (regs 0,1 = hi, lo limb) and 16g + 2mt + 1
 // (regs 2,3); those channels come from code field f = 2(mt&1) and f + 1,
 // which the unshifted masks scaled by 4^f.
+// acci: exact int32 o' contributions since the last flush (row scale 4^f)
 template <int G>
-__device__ __forceinline__ void mma_flush(MmaWarpState<G>& st, int nt, float inv) {
+__device__ __forceinline__ void mma_flush(MmaWarpState<G>& st, int (&acci)[HCfg<G>::NT][8][4], int nt, float inv) {
 #pragma unroll
   for (int mt = 0; mt < 8; ++mt) {
     const float s0 = (mt & 1) ? inv * (1.f / 16.f) : inv;  // field 0 or 2
     const float s1 = s0 * 0.25f;                            // field 1 or 3
-    st.acc[nt][2 * mt] += fmaf((float)st.acci[nt][mt][0], 256.f * s0, (float)st.acci[nt][mt][1] * s0);
-    st.acc[nt][2 * mt + 1] += fmaf((float)st.acci[nt][mt][2], 256.f * s1, (float)st.acci[nt][mt][3] * s1);
+    st.acc[16 * nt + 2 * mt] += fmaf((float)acci[nt][mt][0], 256.f * s0, (float)acci[nt][mt][1] * s0);
+    st.acc[16 * nt + 2 * mt + 1] += fmaf((float)acci[nt][mt][2], 256.f * s1, (float)acci[nt][mt][3] * s1);
 #pragma unroll
-    for (int j = 0; j < 4; ++j) st.acci[nt][mt][j] = 0;
+    for (int j = 0; j < 4; ++j) acci[nt][mt][j] = 0;
   }
 }
 
@@ -525,7 +531,8 @@ __global__ void __launch_bounds__(kHW * 32, (G <= 4) ? 2 : 1) decode_heads_kerne
   constexpr int NT = HCfg<G>::NT, HP = HCfg<G>::HP;
   extern __shared__ __align__(16) unsigned char smem_raw[];
   unsigned char* ring = smem_raw;
-  uint64_t* full = reinterpret_cast<uint64_t*>(ring + HCfg<G>::ring_bytes);
+  float* accs = reinterpret_cast<float*>(ring + HCfg<G>::ring_bytes);
+  uint64_t* full = reinterpret_cast<uint64_t*>(reinterpret_cast<unsigned char*>(accs) + HCfg<G>::acc_bytes);
   uint64_t* empty = full + kHStages;
   uint8_t* ntok = reinterpret_cast<uint8_t*>(empty + kHStages);                 // [S][16]
   uint16_t* pst = reinterpret_cast<uint16_t*>(ntok + kHStages * kSlotsPerStage);  // [8][HP][40]
@@ -577,6 +584,8 @@ __global__ void __launch_bounds__(kHW * 32, (G <= 4) ? 2 : 1) decode_heads_kerne
 
     // ---------------- per-warp state for (b, head) ----------------
     MmaWarpState<G> st;
+    int acci[NT][8][4];
+    st.acc = accs + threadIdx.x * HCfg<G>::acc_stride;
     uint32_t qb[NT][8];
     float ah[NT], bh[NT], hbias[NT];
 #pragma unroll
@@ -585,11 +594,11 @@ __global__ void __launch_bounds__(kHW * 32, (G <= 4) ? 2 : 1) decode_heads_kerne
       st.l[nt] = 0.f;
       st.msum[nt] = 0.f;
 #pragma unroll
-      for (int i = 0; i < 16; ++i) st.acc[nt][i] = 0.f;
+      for (int i = 0; i < 16; ++i) st.acc[16 * nt + i] = 0.f;
 #pragma unroll
       for (int mt = 0; mt < 8; ++mt)
 #pragma unroll
-        for (int j = 0; j < 4; ++j) st.acci[nt][mt][j] = 0;
+        for (int j = 0; j < 4; ++j) acci[nt][mt][j] = 0;
       const int hcol = 4 * nt + (g >> 1);  // head of this lane's B column
       if (hcol < G) {
         const uint4* src = reinterpret_cast<const uint4*>(a.qlimb + ((bh0 + hcol) * 2 + (g & 1)) * kD + 32 * t);
@@ -615,11 +624,16 @@ __global__ void __launch_bounds__(kHW * 32, (G <= 4) ? 2 : 1) decode_heads_kerne
     const int nst = (slot_ok && alive && p1 > p0) ? (p1 - p0 + nb - 1) / nb : 0;
     const int32_t* trow = a.block_table + (size_t)(slot_ok ? slot : 0) * a.mbps;
 
-    // warp 0 lane 0: put stage j of this entry in ring position it + j
+    // warp 0 lane 0: put stage j of this entry in the next ring position
+    // (ps = its stage, puse = how often that stage was filled before)
+    uint32_t ps = it % kHStages, puse = it / kHStages;
     auto issue = [&](int j) -> bool {
-      const uint32_t pos = it + (uint32_t)j;
-      const uint32_t s = pos % kHStages;
-      if (pos >= (uint32_t)kHStages && !mbar_wait_bounded(&empty[s], ((pos / kHStages) - 1) & 1u)) return false;
+      const uint32_t s = ps;
+      if (puse > 0 && !mbar_wait_bounded(&empty[s], (puse - 1) & 1u)) return false;
+      if (++ps == (uint32_t)kHStages) {
+        ps = 0;
+        ++puse;
+      }
       uint32_t bytes = 0;
       for (int q = 0; q < nb; ++q) {  // token counts first: the barrier must expect every byte
         const int pi = p0 + j * nb + q;
@@ -646,6 +660,7 @@ __global__ void __launch_bounds__(kHW * 32, (G <= 4) ? 2 : 1) decode_heads_kerne
       for (int j = 0; j < min(kHStages - 2, nst) && prod_ok; ++j) prod_ok = issue(j);
 
     int done = 0;
+    uint32_t cs = it % kHStages, cph = (it / kHStages) & 1u;  // consumer stage and phase parity
     for (int j = 0; j < nst; ++j) {
       if (warp == 0) {
         if (lane == 0 && prod_ok && j + kHStages - 2 < nst) prod_ok = issue(j + kHStages - 2);
@@ -654,17 +669,20 @@ __global__ void __launch_bounds__(kHW * 32, (G <= 4) ? 2 : 1) decode_heads_kerne
           alive = false;
         }
       }
-      const uint32_t pos = it + (uint32_t)j;
-      const uint32_t s = pos % kHStages;
-      if (!__all_sync(0xffffffffu, alive && mbar_wait_bounded(&full[s], (pos / kHStages) & 1u))) {
+      const uint32_t s = cs, par = cph;
+      if (++cs == (uint32_t)kHStages) {
+        cs = 0;
+        cph ^= 1u;
+      }
+      if (!__all_sync(0xffffffffu, alive && mbar_wait_bounded(&full[s], par))) {
         if (lane == 0) raise_flag(a.status, OKV_DEV_TIMEOUT);
         alive = false;
         break;
       }
       const int q0 = 2 * grp;
       const int n0 = ntok[s * kSlotsPerStage + q0], n1 = ntok[s * kSlotsPerStage + q0 + 1];
-      if (n0 + n1 > 0) {
-        const bool fullstep = (n0 == kBlock) && (n1 == kBlock);
+      auto step = [&](auto full_tag) {
+        constexpr bool fullstep = decltype(full_tag)::value;
         const unsigned char* s0 = ring + s * kHStageBytes + q0 * copy_bytes + head * kBlockHeadBytes;
         const unsigned char* s1 = s0 + copy_bytes;
 
@@ -709,12 +727,12 @@ __global__ void __launch_bounds__(kHW * 32, (G <= 4) ? 2 : 1) decode_heads_kerne
         }
         float smax = fmaxf(fmaxf(tv[0] ? sv[0] : 0.f, tv[1] ? sv[1] : 0.f),
                            fmaxf(tv[2] ? sv[2] : 0.f, tv[3] ? sv[3] : 0.f));
-        smax = fmaxf(smax, __shfl_xor_sync(0xffffffffu, smax, 4));
-        smax = fmaxf(smax, __shfl_xor_sync(0xffffffffu, smax, 8));
-        smax = fmaxf(smax, __shfl_xor_sync(0xffffffffu, smax, 16));
-        if (smax > s_cap) {  // raise the scale cap: flush every head at the old cap first
+        if (__any_sync(0xffffffffu, smax > s_cap)) {  // rare: raise the scale cap, flushing every head first
+          smax = fmaxf(smax, __shfl_xor_sync(0xffffffffu, smax, 4));
+          smax = fmaxf(smax, __shfl_xor_sync(0xffffffffu, smax, 8));
+          smax = fmaxf(smax, __shfl_xor_sync(0xffffffffu, smax, 16));
 #pragma unroll
-          for (int nt = 0; nt < NT; ++nt) mma_flush(st, nt, inv);
+          for (int nt = 0; nt < NT; ++nt) mma_flush(st, acci, nt, inv);
           since_flush = 0;
           s_cap = smax;
           lam = 65535.f / s_cap;
@@ -735,14 +753,16 @@ __global__ void __launch_bounds__(kHW * 32, (G <= 4) ? 2 : 1) decode_heads_kerne
             sc[e] = tv[e] ? x : -INFINITY;
           }
           float bm = fmaxf(fmaxf(sc[0], sc[1]), fmaxf(sc[2], sc[3]));
-          bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 4));
-          bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 8));
-          bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 16));
+          if (__any_sync(0xffffffffu, bm > st.m[nt])) {  // rare after the first steps: a new running max
+            bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 4));
+            bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 8));
+            bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 16));
+          }
           if (bm > st.m[nt]) {
-            mma_flush(st, nt, inv);
+            mma_flush(st, acci, nt, inv);
             const float alpha = fast_ex2(st.m[nt] - bm);  // ex2(-inf) = 0 on the first step
 #pragma unroll
-            for (int i = 0; i < 16; ++i) st.acc[nt][i] *= alpha;
+            for (int i = 0; i < 16; ++i) st.acc[16 * nt + i] *= alpha;
             st.l[nt] *= alpha;
             st.msum[nt] *= alpha;
             st.m[nt] = bm;
@@ -754,7 +774,9 @@ __global__ void __launch_bounds__(kHW * 32, (G <= 4) ? 2 : 1) decode_heads_kerne
             const float p = fast_ex2(sc[e] - mref);  // 0 for masked tokens
             st.l[nt] += p;
             st.msum[nt] = fmaf(p, mv[e], st.msum[nt]);
-            prow[16 * (e >> 1) + g + 8 * (e & 1)] = (uint16_t)cvt_u16_sat(p * svl[e]);
+            // round(p * s * lam) <= 65535 via the 1.5 * 2^23 magic add (one FFMA, no conversion unit)
+            prow[16 * (e >> 1) + g + 8 * (e & 1)] =
+                (uint16_t)(__float_as_uint(fmaf(p, svl[e], 12582912.f)) - 0x4B400000u);
           }
         }
         __syncwarp();
@@ -779,21 +801,23 @@ __global__ void __launch_bounds__(kHW * 32, (G <= 4) ? 2 : 1) decode_heads_kerne
           const uint32_t m0 = kM2 << (4 * (mt & 1)), m1 = m0 << 2;
           const uint32_t af[4] = {va[jw] & m0, va[jw] & m1, vb[jw] & m0, vb[jw] & m1};
 #pragma unroll
-          for (int nt = 0; nt < NT; ++nt) mma_u8u8(st.acci[nt][mt], af, pb0[nt], pb1[nt]);
+          for (int nt = 0; nt < NT; ++nt) mma_u8u8(acci[nt][mt], af, pb0[nt], pb1[nt]);
         }
         if (++since_flush >= 96) {
 #pragma unroll
-          for (int nt = 0; nt < NT; ++nt) mma_flush(st, nt, inv);
+          for (int nt = 0; nt < NT; ++nt) mma_flush(st, acci, nt, inv);
           since_flush = 0;
         }
-      }
+      };
+      if (n0 == kBlock && n1 == kBlock) step(std::true_type{});
+      else if (n0 + n1 > 0) step(std::false_type{});
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[s]);
       ++done;
     }
     it += (uint32_t)nst;
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) mma_flush(st, nt, inv);
+    for (int nt = 0; nt < NT; ++nt) mma_flush(st, acci, nt, inv);
     __syncthreads();  // every warp is done with the ring: it becomes window scratch, then merge buffers
 
     // ---------------- fp16 window: chunks ci = grp, grp + wph, ... of this warp's head ----------------
@@ -937,7 +961,7 @@ __global__ void __launch_bounds__(kHW * 32, (G <= 4) ? 2 : 1) decode_heads_kerne
           const float ab = fast_ex2(st.m[nt] - mref), aw = fast_ex2(wm[nt] - mref);
           const float* src = wo + hs * kD + 16 * g;
 #pragma unroll
-          for (int i = 0; i < 16; ++i) st.acc[nt][i] = fmaf(st.acc[nt][i], ab, src[i] * aw);
+          for (int i = 0; i < 16; ++i) st.acc[16 * nt + i] = fmaf(st.acc[16 * nt + i], ab, src[i] * aw);
           st.l[nt] = fmaf(st.l[nt], ab, wl[nt] * aw);
           st.msum[nt] *= ab;
           st.m[nt] = M;
@@ -961,8 +985,9 @@ __global__ void __launch_bounds__(kHW * 32, (G <= 4) ? 2 : 1) decode_heads_kerne
           float* dst = part_b + (size_t)hs * kPartStride + 16 * g;
 #pragma unroll
           for (int i = 0; i < 16; i += 4)
-            *reinterpret_cast<float4*>(dst + i) = make_float4(st.acc[nt][i] + ms, st.acc[nt][i + 1] + ms,
-                                                              st.acc[nt][i + 2] + ms, st.acc[nt][i + 3] + ms);
+            *reinterpret_cast<float4*>(dst + i) =
+                make_float4(st.acc[16 * nt + i] + ms, st.acc[16 * nt + i + 1] + ms, st.acc[16 * nt + i + 2] + ms,
+                            st.acc[16 * nt + i + 3] + ms);
           if (g == 0) {
             part_b[(size_t)hs * kPartStride + 128] = st.m[nt];
             part_b[(size_t)hs * kPartStride + 129] = l;
@@ -983,7 +1008,7 @@ __global__ void __launch_bounds__(kHW * 32, (G <= 4) ? 2 : 1) decode_heads_kerne
         if (hs < G) {
           float* dst = mo + ((size_t)warp * G + hs) * kD + 16 * g;
 #pragma unroll
-          for (int i = 0; i < 16; ++i) dst[i] = st.acc[nt][i] + ms;
+          for (int i = 0; i < 16; ++i) dst[i] = st.acc[16 * nt + i] + ms;
           if (g == 0) {
             ml[(warp * G + hs) * 2 + 0] = st.m[nt];
             ml[(warp * G + hs) * 2 + 1] = l;
