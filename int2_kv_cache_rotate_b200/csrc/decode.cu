@@ -407,9 +407,11 @@ __global__ void __launch_bounds__(kDecWarps * 32) decode_simt_kernel(DecodeArgs 
 //
 // A CTA of 8 warps streams a range of blocks of one sequence for every KV
 // head at once: every block is one contiguous run of Hkv x 1152 bytes, fetched
-// by a single bulk copy into a 4-stage CTA ring (16 block-heads per stage,
-// full/empty mbarriers, the copies issued by lane 0 of warp 0 two stages
-// ahead).  Warp w serves KV head w % Hkv and, per stage, two of its blocks.
+// by a single bulk copy into a 5-stage CTA ring (16 block-heads per stage,
+// full/empty mbarriers; lane 0 of warp 0 keeps four stages in flight, and
+// every warp copies its share of a stage to registers and releases the stage
+// before computing on it).  Warp w serves KV head w % Hkv and, per stage, two
+// of its blocks.
 // Per 2-block step a warp computes:
 //   scores  S[32 tok x 4NT heads] = C_K (u8 codes) . Q (two s8 limbs) on
 //           mma.m16n8k32, then s_t * sigma * raw + m_t * sum(q~);
@@ -433,12 +435,14 @@ __global__ void __launch_bounds__(kDecWarps * 32) decode_simt_kernel(DecodeArgs 
 // fp16 hi+lo pairs), folded into the warp's state in registers.
 // ---------------------------------------------------------------------------
 constexpr int kHW = 8;                             // warps per CTA
-constexpr int kHStages = 5;                        // ring stages (3 in flight ahead of the consumers)
+constexpr int kHStages = 5;                        // ring stages (4 in flight ahead of the consumers)
 constexpr int kSlotsPerStage = 16;                 // block-heads per stage
 constexpr int kHStageBytes = kSlotsPerStage * kBlockHeadBytes;  // 18432
 constexpr int kPStride = 40;                       // u16 per head row of the P' tile
 constexpr int kWarpScratch = 9216;                 // ring bytes each warp may use as window scratch
 constexpr uint32_t kM2 = 0x03030303u;
+constexpr float kMaxSlack = 2.f;  // log2 units a score may exceed the reference max without a rescale
+constexpr float kPSlack = 4.f;    // = 2^kMaxSlack
 
 template <int G>
 struct HCfg {
@@ -657,13 +661,13 @@ __global__ void __launch_bounds__(kHW * 32, (G <= 4) ? 2 : 1) decode_heads_kerne
     };
     bool prod_ok = true;
     if (warp == 0 && lane == 0)
-      for (int j = 0; j < min(kHStages - 2, nst) && prod_ok; ++j) prod_ok = issue(j);
+      for (int j = 0; j < min(kHStages - 1, nst) && prod_ok; ++j) prod_ok = issue(j);
 
     int done = 0;
     uint32_t cs = it % kHStages, cph = (it / kHStages) & 1u;  // consumer stage and phase parity
     for (int j = 0; j < nst; ++j) {
       if (warp == 0) {
-        if (lane == 0 && prod_ok && j + kHStages - 2 < nst) prod_ok = issue(j + kHStages - 2);
+        if (lane == 0 && prod_ok && j + kHStages - 1 < nst) prod_ok = issue(j + kHStages - 1);
         if (!__shfl_sync(0xffffffffu, prod_ok, 0)) {
           if (lane == 0) raise_flag(a.status, OKV_DEV_TIMEOUT);
           alive = false;
@@ -686,18 +690,30 @@ __global__ void __launch_bounds__(kHW * 32, (G <= 4) ? 2 : 1) decode_heads_kerne
         const unsigned char* s0 = ring + s * kHStageBytes + q0 * copy_bytes + head * kBlockHeadBytes;
         const unsigned char* s1 = s0 + copy_bytes;
 
-        // ---- scores: D[tok][col] for both blocks
-        int dq[2][NT][4];
+        // ---- everything this lane needs from the stage goes to registers, then
+        //      the stage is released so the producer can refill it while we compute
+        uint2 kw[2][2];
         uint32_t smk[4], smv[4];
+        uint4 vw[2];
 #pragma unroll
         for (int bb = 0; bb < 2; ++bb) {
           const unsigned char* sb = bb ? s1 : s0;
-          const uint2 wa = *reinterpret_cast<const uint2*>(sb + kKcOff + 32 * g + 8 * t);
-          const uint2 wb = *reinterpret_cast<const uint2*>(sb + kKcOff + 32 * (g + 8) + 8 * t);
+          kw[bb][0] = *reinterpret_cast<const uint2*>(sb + kKcOff + 32 * g + 8 * t);
+          kw[bb][1] = *reinterpret_cast<const uint2*>(sb + kKcOff + 32 * (g + 8) + 8 * t);
           smk[2 * bb] = *reinterpret_cast<const uint32_t*>(sb + kKsmOff + 4 * g);
           smk[2 * bb + 1] = *reinterpret_cast<const uint32_t*>(sb + kKsmOff + 4 * (g + 8));
           smv[2 * bb] = *reinterpret_cast<const uint32_t*>(sb + kVsmOff + 4 * g);
           smv[2 * bb + 1] = *reinterpret_cast<const uint32_t*>(sb + kVsmOff + 4 * (g + 8));
+          vw[bb] = *reinterpret_cast<const uint4*>(sb + kVcOff + 16 * lane);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[s]);
+
+        // ---- scores: D[tok][col] for both blocks
+        int dq[2][NT][4];
+#pragma unroll
+        for (int bb = 0; bb < 2; ++bb) {
+          const uint2 wa = kw[bb][0], wb = kw[bb][1];
 #pragma unroll
           for (int sf = 0; sf < 4; ++sf) {
             uint32_t af[4];
@@ -734,9 +750,11 @@ __global__ void __launch_bounds__(kHW * 32, (G <= 4) ? 2 : 1) decode_heads_kerne
 #pragma unroll
           for (int nt = 0; nt < NT; ++nt) mma_flush(st, acci, nt, inv);
           since_flush = 0;
-          s_cap = smax;
-          lam = 65535.f / s_cap;
-          inv = s_cap / 65535.f;
+          // headroom: the cap jumps to twice the new maximum, and P' leaves room
+          // for p up to 2^kMaxSlack, so later small increases cost nothing
+          s_cap = 2.f * smax;
+          lam = 65535.f / (s_cap * kPSlack);
+          inv = (s_cap * kPSlack) / 65535.f;
         }
         float svl[4];
 #pragma unroll
@@ -752,13 +770,15 @@ __global__ void __launch_bounds__(kHW * 32, (G <= 4) ? 2 : 1) decode_heads_kerne
             if constexpr (G < 4) x += hbias[nt];
             sc[e] = tv[e] ? x : -INFINITY;
           }
+          // The reference max moves only when a score passes it by more than
+          // kMaxSlack (log2 units): p <= 2^kMaxSlack, which P' has room for.
           float bm = fmaxf(fmaxf(sc[0], sc[1]), fmaxf(sc[2], sc[3]));
-          if (__any_sync(0xffffffffu, bm > st.m[nt])) {  // rare after the first steps: a new running max
+          if (__any_sync(0xffffffffu, bm > st.m[nt] + kMaxSlack)) {
             bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 4));
             bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 8));
             bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 16));
           }
-          if (bm > st.m[nt]) {
+          if (bm > st.m[nt] + kMaxSlack) {
             mma_flush(st, acci, nt, inv);
             const float alpha = fast_ex2(st.m[nt] - bm);  // ex2(-inf) = 0 on the first step
 #pragma unroll
@@ -781,8 +801,7 @@ __global__ void __launch_bounds__(kHW * 32, (G <= 4) ? 2 : 1) decode_heads_kerne
         }
         __syncwarp();
         // ---- values: acci[mt] += C_V (masked, row scale 4^f) . P'
-        const uint4 v0 = *reinterpret_cast<const uint4*>(s0 + kVcOff + 16 * lane);
-        const uint4 v1 = *reinterpret_cast<const uint4*>(s1 + kVcOff + 16 * lane);
+        const uint4 v0 = vw[0], v1 = vw[1];
         const uint32_t va[4] = {v0.x, v0.y, v0.z, v0.w};
         const uint32_t vb[4] = {v1.x, v1.y, v1.z, v1.w};
         uint32_t pb0[NT], pb1[NT];
@@ -809,10 +828,15 @@ __global__ void __launch_bounds__(kHW * 32, (G <= 4) ? 2 : 1) decode_heads_kerne
           since_flush = 0;
         }
       };
-      if (n0 == kBlock && n1 == kBlock) step(std::true_type{});
-      else if (n0 + n1 > 0) step(std::false_type{});
+      if (n0 == kBlock && n1 == kBlock) {
+        step(std::true_type{});
+      } else if (n0 + n1 > 0) {
+        step(std::false_type{});
+      } else {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[s]);
+      }
       __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[s]);
       ++done;
     }
     it += (uint32_t)nst;
