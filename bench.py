@@ -58,6 +58,26 @@ def dist_env():
     return world, rank, local
 
 
+def job_time_ms(ms, world, dist=None, device="cpu"):
+    """The job's time is its slowest rank's: the max over ranks (every rank calls this)."""
+    if world == 1:
+        return float(ms)
+    import torch
+    t = torch.tensor([float(ms)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_units(units, world, dist=None, device="cpu"):
+    """Units (decoded tokens) processed by all ranks together (every rank calls this)."""
+    if world == 1:
+        return int(units)
+    import torch
+    t = torch.tensor([int(units)], dtype=torch.int64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return int(t.item())
+
+
 class Clocks:
     """nvidia-smi sampler for the timed region."""
 
@@ -368,10 +388,9 @@ def run_ours(args):
     clk = clocks.stop()
     ms = t0.elapsed_time(t1)
     dec_us = [a.elapsed_time(b) * 1e3 for a, b in evs]
+    ms = job_time_ms(ms, world, dist, "cuda")
+    units = job_units(B * K, world, dist, "cuda")
     if world > 1:
-        t = torch.tensor([ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
         dist.barrier()
     assert w["cache"].device_status() == 0, w["cache"].device_status()
 
@@ -405,13 +424,10 @@ def run_ours(args):
             hout.copy_(out, non_blocking=True)
         e1.record()
         torch.cuda.synchronize()
-        e_ms = e0.elapsed_time(e1)
-        if world > 1:
-            t = torch.tensor([e_ms], device="cuda")
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e_ms = float(t.item())
+        e_ms = job_time_ms(e0.elapsed_time(e1), world, dist, "cuda")
+        e_units = job_units(B * e2e_steps, world, dist, "cuda")
         h2d = sum(x[0].numel() * x.element_size() for x in (hk, hv, hqv, hpos, hlen))
-        e2e = {"value": round(world * B * e2e_steps / (e_ms * 1e-3), 2), "unit": "tok/s",
+        e2e = {"value": round(e_units / (e_ms * 1e-3), 2), "unit": "tok/s",
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(hout.numel() * 4),
                "ms_per_step": round(e_ms / e2e_steps, 4), "timed_as": "eager calls, one per step"}
 
@@ -426,7 +442,7 @@ def run_ours(args):
         tr = recorded_traffic()
         line = {
             "metric": METRIC,
-            "value": round(world * B * K / (ms * 1e-3), 2),
+            "value": round(units / (ms * 1e-3), 2),
             "unit": "tok/s",
             "n_gpus": world, "steps": K, "warmup": W, "ms_per_step": round(ms / K, 4),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,

@@ -119,10 +119,14 @@ def test_dequantize_bit_exact_and_original_basis():
                 assert np.abs(orig[b, h, :n] - back).max() <= 1e-5 * np.abs(back).max()
 
 
-def test_append_fused_rotation_and_codes():
+@pytest.mark.parametrize("lens", [
+    [700, 45],   # 745 tokens: tensor-core kernel, 3 CTAs, ragged last round
+    [60, 45],    # 105 tokens: CUDA-core kernel
+    [128],       # exactly the tensor-core threshold
+])
+def test_append_fused_rotation_and_codes(lens):
     okv = _okv()
     seed, hq, hkv = 3, 8, 2
-    lens = [700, 45]
     lay = H.Layout(seed, lens)
     uk, uv = H.rotations(seed, hkv)
     gc = _gpu_cache(hq, hkv, lay, uk, uv)
