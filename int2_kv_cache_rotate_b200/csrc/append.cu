@@ -2,6 +2,8 @@
 // to INT2 with fp16 scale/min, pack, and write the paged cache and fp16 window.
 // Decode steps (a few tokens) run the CUDA-core kernel; prefill chunks of 128
 // tokens or more run the tensor-core kernel.
+#include <algorithm>
+
 #include "okv_common.cuh"
 #include "okv_internal.h"
 
@@ -146,24 +148,30 @@ __global__ void __launch_bounds__(kAppThreads) append_kernel(AppendArgs a, int T
 // ---------------------------------------------------------------------------
 // Tensor-core append for long token runs (prefill chunks).
 //
-// x = k U is a dense [T x 128] x [128 x 128] contraction, so it runs on
-// mma.m16n8k16 (bf16 in, fp32 accumulate): k is exact in bf16 and U is split
-// into three bf16 parts (hi + mid + lo carry 24 mantissa bits), so every
-// product is exact and the sum is an fp32 sum, like the CUDA-core path.
-// A CTA stages U^T (three parts, rows padded to 136 elements so the fragment
-// loads do not collide in banks) once and runs 4 warps x 16 tokens per round.
-// In the accumulator layout lane (g, t) holds, for tokens g and g+8, outputs
-// i = 8 nt + 2t + e (nt = 0..15, e = 0..1): Hadamard index bits 0 and 3..6 are
-// in registers, bits 1..2 across the four lanes of a quad (two shuffle
-// stages).  Bits 5..6 are register bits too, so after the bit reversal each
-// lane owns whole packed bytes: byte b collects outputs rev5(b) + 32a.
+// z = k R with R = U H P_br / sqrt(128) is a dense [T x 128] x [128 x 128]
+// contraction, so it runs on mma.m16n8k16 (bf16 in, fp32 accumulate).  k is
+// exact in bf16; R is split into three bf16 parts (hi + mid + lo carry 24
+// mantissa bits), so every product is exact and the sums are fp32 sums.
+// Each CTA builds R for its (KV head, K|V) once in shared memory: a warp
+// takes a row c of U, runs the Hadamard butterfly across the warp and writes
+// the row of R, already split, to columns in the order below.  Folding H and
+// P_br into the staged matrix removes the per-token butterfly; the column
+// order makes every lane own whole code bytes.
+//
+// Column order: in the accumulator of n-tile nt, lane (g, t) holds columns
+// 8 nt + 2t + e (e = 0, 1) for tokens g and g + 8.  Physical column
+// p = 8 (2k + (f >> 1)) + 2t + (f & 1) carries rotated channel 4 (8t + k) + f,
+// so lane t holds packed bytes 8t .. 8t + 7 (channels 32t .. 32t + 31) of its
+// two tokens: byte k field f is d[2k + (f >> 1)][2 half + (f & 1)].
+// B fragments come from the [c][p] row-major R with ldmatrix.trans; rows
+// are padded to 136 elements so the eight rows of a matrix fall in distinct
+// bank groups.
 // ---------------------------------------------------------------------------
-constexpr int kTcMinTokens = 128;  // below this the CUDA-core kernel wins (U staging dominates)
-constexpr int kTcWarps = 4;
-constexpr int kTcRound = 16 * kTcWarps;   // tokens per round
-constexpr int kTcCtaTokens = 256;         // tokens per CTA (U staged once)
-constexpr int kUtStride = 136;            // bf16 per U^T row in shared memory
-constexpr size_t kTcSmem = (size_t)3 * kD * kUtStride * 2;
+constexpr int kTcMinTokens = 128;  // below this the CUDA-core kernel wins (R staging dominates)
+constexpr int kTcWarps = 8;
+constexpr int kTcRound = 16 * kTcWarps;  // tokens per CTA round
+constexpr int kRStride = 136;            // bf16 per staged row of R
+constexpr size_t kTcSmem = (size_t)3 * kD * kRStride * 2;
 
 __device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
   asm volatile(
@@ -173,19 +181,29 @@ __device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], 
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-// One token's rotated vector, spread over the four lanes of a quad:
-// zb[q][a] = y at pre-permutation index r_q + 32a, r_q = 8 (q >> 1) + 2t + (q & 1).
-// The min/max reduction runs on every lane (the quad shuffles need all of
-// them); `live` then gates validation and the stores.
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+
+// physical column of rotated channel j = 4b + f
+__device__ __forceinline__ int tc_column(int b, int f) {
+  return 8 * (2 * (b & 7) + (f >> 1)) + 2 * (b >> 3) + (f & 1);
+}
+
+// One token held by the four lanes of a quad: v[k][f] = rotated channel
+// 4 (8t + k) + f.  The min/max reduction runs on every lane (the quad
+// shuffles need all of them); `live` then gates validation and the stores.
 __device__ __forceinline__ void finish_token_tc(const AppendArgs& a, int tok, bool live, int h, int kind,
-                                                const float (&zb)[8][4], int t) {
-  float mn = zb[0][0], mx = zb[0][0];
+                                                const float (&v)[8][4], int t) {
+  float mn = v[0][0], mx = v[0][0];
 #pragma unroll
-  for (int q = 0; q < 8; ++q)
+  for (int k = 0; k < 8; ++k)
 #pragma unroll
-    for (int aa = 0; aa < 4; ++aa) {
-      mn = fminf(mn, zb[q][aa]);
-      mx = fmaxf(mx, zb[q][aa]);
+    for (int f = 0; f < 4; ++f) {
+      mn = fminf(mn, v[k][f]);
+      mx = fmaxf(mx, v[k][f]);
     }
   mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, 1));
   mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
@@ -214,66 +232,96 @@ __device__ __forceinline__ void finish_token_tc(const AppendArgs& a, int tok, bo
   const __half m16 = fp16_sat(mn);
   const float s = __half2float(s16);
   const float m = __half2float(m16);
+  uint32_t w[2] = {0u, 0u};
+  if (s != 0.0f) {
+    const CodeThresholds th = code_thresholds(s);
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+#pragma unroll
+      for (int f = 0; f < 4; ++f) w[k >> 2] |= int2_code(__fsub_rn(v[k][f], m), th) << (8 * (k & 3) + 2 * f);
+  }
   uint8_t* base = a.pages + ((size_t)blk * a.hkv + h) * kBlockHeadBytes;
   const int sl = p & 15;
-  const bool in_win = p >= len - kWin;
-  __half* wrow = a.ring + ((((size_t)slot * a.hkv + h) * 2 + kind) * kWin + (p % kWin)) * kD;
-  float* rrow = a.rotated_out ? a.rotated_out + (((size_t)tok * 2 + kind) * a.hkv + h) * kD : nullptr;
+  if (kind == 0) {
+    *reinterpret_cast<uint2*>(base + kKcOff + sl * 32 + 8 * t) = make_uint2(w[0], w[1]);
+  } else {
 #pragma unroll
-  for (int q = 0; q < 8; ++q) {
-    const int b = rev5(8 * (q >> 1) + 2 * t + (q & 1));  // packed byte = canonical channels 4b..4b+3
-    uint32_t byte = 0;
-#pragma unroll
-    for (int aa = 0; aa < 4; ++aa) {
-      uint32_t c = 0;
-      if (s != 0.0f) {
-        const float rr = rintf(__fdiv_rn(__fsub_rn(zb[q][aa], m), s));
-        c = (uint32_t)fminf(fmaxf(rr, 0.0f), 3.0f);
-      }
-      byte |= c << (2 * rev2(aa));
-    }
-    if (kind == 0) base[kKcOff + sl * 32 + b] = (uint8_t)byte;
-    else base[v_code_offset(sl, b)] = (uint8_t)byte;
-    // channel 4b + e holds the value at a = rev2(e): e = 0..3 <- a = 0, 2, 1, 3
-    if (in_win) {
-      __half2 lo = __halves2half2(fp16_sat(zb[q][0]), fp16_sat(zb[q][2]));
-      __half2 hi = __halves2half2(fp16_sat(zb[q][1]), fp16_sat(zb[q][3]));
-      uint2 w;
-      w.x = *reinterpret_cast<uint32_t*>(&lo);
-      w.y = *reinterpret_cast<uint32_t*>(&hi);
-      *reinterpret_cast<uint2*>(wrow + 4 * b) = w;
-    }
-    if (rrow) *reinterpret_cast<float4*>(rrow + 4 * b) = make_float4(zb[q][0], zb[q][2], zb[q][1], zb[q][3]);
+    for (int k = 0; k < 8; ++k) base[v_code_offset(sl, 8 * t + k)] = (uint8_t)(w[k >> 2] >> (8 * (k & 3)));
   }
   if (t == 0)
     *reinterpret_cast<uint32_t*>(base + (kind ? kVsmOff : kKsmOff) + 4 * sl) =
         (uint32_t)__half_as_ushort(s16) | ((uint32_t)__half_as_ushort(m16) << 16);
+  if (p >= len - kWin) {
+    __half* row = a.ring + ((((size_t)slot * a.hkv + h) * 2 + kind) * kWin + (p % kWin)) * kD + 32 * t;
+#pragma unroll
+    for (int k = 0; k < 8; k += 2) {
+      __half2 h0 = __halves2half2(fp16_sat(v[k][0]), fp16_sat(v[k][1]));
+      __half2 h1 = __halves2half2(fp16_sat(v[k][2]), fp16_sat(v[k][3]));
+      __half2 h2 = __halves2half2(fp16_sat(v[k + 1][0]), fp16_sat(v[k + 1][1]));
+      __half2 h3 = __halves2half2(fp16_sat(v[k + 1][2]), fp16_sat(v[k + 1][3]));
+      uint4 q4;
+      q4.x = *reinterpret_cast<uint32_t*>(&h0);
+      q4.y = *reinterpret_cast<uint32_t*>(&h1);
+      q4.z = *reinterpret_cast<uint32_t*>(&h2);
+      q4.w = *reinterpret_cast<uint32_t*>(&h3);
+      *reinterpret_cast<uint4*>(row + 4 * k) = q4;
+    }
+  }
+  if (a.rotated_out != nullptr) {
+    float* row = a.rotated_out + (((size_t)tok * 2 + kind) * a.hkv + h) * kD + 32 * t;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) *reinterpret_cast<float4*>(row + 4 * k) = make_float4(v[k][0], v[k][1], v[k][2], v[k][3]);
+  }
 }
 
-__global__ void __launch_bounds__(kTcWarps * 32) append_tc_kernel(AppendArgs a, int T) {
+// Grid (ceil(T / tokens_per_cta), Hkv, 2); a CTA stages R once and runs
+// rounds of 128 tokens (16 per warp) over its token range.
+__global__ void __launch_bounds__(kTcWarps * 32, 2) append_tc_kernel(AppendArgs a, int T, int tokens_per_cta) {
   extern __shared__ __align__(16) unsigned char tc_smem[];
-  __nv_bfloat16* ut = reinterpret_cast<__nv_bfloat16*>(tc_smem);  // [3][128][136]: U^T split in three
+  __nv_bfloat16* rs = reinterpret_cast<__nv_bfloat16*>(tc_smem);  // [3][128 c][136]: R split in three
   const int h = blockIdx.y, kind = blockIdx.z;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int g = lane >> 2, t = lane & 3;
-  const int t0 = blockIdx.x * kTcCtaTokens, t1 = min(T, t0 + kTcCtaTokens);
+  const int t0 = blockIdx.x * tokens_per_cta, t1 = min(T, t0 + tokens_per_cta);
   {
-    // U^T[i][c] = U[c][i], split as U = p0 + p1 + p2 (each bf16, residuals exact in fp32);
-    // a thread takes column i of two consecutive rows c, c+1 and stores bf16 pairs.
+    // row c of R = (row c of U) H P_br / sqrt(128): butterfly across the warp;
+    // lane l's value a is rotated channel 4 rev5(l) + rev2(a)
     const float* U = (kind ? a.u_v : a.u_k) + (size_t)h * kD * kD;
-    for (int idx = threadIdx.x; idx < kD * kD / 2; idx += blockDim.x) {
-      const int i = idx & (kD - 1), c = 2 * (idx >> 7);
-      const float u0 = __ldg(U + (size_t)c * kD + i), u1 = __ldg(U + (size_t)(c + 1) * kD + i);
-      const __nv_bfloat162 p0 = __floats2bfloat162_rn(u0, u1);
-      const float r0 = u0 - __low2float(p0), r1 = u1 - __high2float(p0);
-      const __nv_bfloat162 p1 = __floats2bfloat162_rn(r0, r1);
-      const __nv_bfloat162 p2 = __floats2bfloat162_rn(r0 - __low2float(p1), r1 - __high2float(p1));
-      *reinterpret_cast<__nv_bfloat162*>(ut + (0 * kD + i) * kUtStride + c) = p0;
-      *reinterpret_cast<__nv_bfloat162*>(ut + (1 * kD + i) * kUtStride + c) = p1;
-      *reinterpret_cast<__nv_bfloat162*>(ut + (2 * kD + i) * kUtStride + c) = p2;
+    const int b = rev5(lane);
+    int col[4];
+#pragma unroll
+    for (int aa = 0; aa < 4; ++aa) col[aa] = tc_column(b, rev2(aa));
+    for (int c0 = warp; c0 < kD; c0 += 4 * kTcWarps) {  // rows c0 + {0, 1, 2, 3} * kTcWarps
+      float y[4][4];
+#pragma unroll
+      for (int r = 0; r < 4; ++r)
+#pragma unroll
+        for (int aa = 0; aa < 4; ++aa) y[r][aa] = __ldg(U + (size_t)(c0 + r * kTcWarps) * kD + lane + 32 * aa);
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        wht128_warp(y[r], lane);
+        const int c = c0 + r * kTcWarps;
+#pragma unroll
+        for (int aa = 0; aa < 4; ++aa) {
+          const float u = y[r][aa] * kInvSqrtD;
+          const __nv_bfloat16 p0 = __float2bfloat16_rn(u);
+          const float r1 = u - __bfloat162float(p0);
+          const __nv_bfloat16 p1 = __float2bfloat16_rn(r1);
+          const __nv_bfloat16 p2 = __float2bfloat16_rn(r1 - __bfloat162float(p1));
+          rs[(0 * kD + c) * kRStride + col[aa]] = p0;
+          rs[(1 * kD + c) * kRStride + col[aa]] = p1;
+          rs[(2 * kD + c) * kRStride + col[aa]] = p2;
+        }
+      }
     }
   }
   __syncthreads();
+  // ldmatrix.trans row addresses: lanes 8j..8j+7 give the rows of matrix j;
+  // matrices 0, 1 = k rows 0-7 / 8-15 of an n-tile (b0, b1), 2, 3 = the same
+  // for the next n-tile.
+  const int mrow = (lane & 7) + 8 * ((lane >> 3) & 1);
+  const int mcol = 8 * (lane >> 4);
+  const uint32_t rs_base = smem_u32(rs) + (uint32_t)(mrow * kRStride + mcol) * 2u;
   const __nv_bfloat16* src = (const __nv_bfloat16*)(kind ? a.v : a.k);
   for (int r0 = t0 + 16 * warp; r0 < t1; r0 += kTcRound) {
     const int ta = r0 + g, tb = r0 + g + 8;
@@ -283,69 +331,35 @@ __global__ void __launch_bounds__(kTcWarps * 32) append_tc_kernel(AppendArgs a, 
     uint32_t af[8][4];
 #pragma unroll
     for (int ks = 0; ks < 8; ++ks) {
-      af[ks][0] = va ? ra[8 * ks + t] : 0u;
-      af[ks][1] = vb ? rb[8 * ks + t] : 0u;
-      af[ks][2] = va ? ra[8 * ks + 4 + t] : 0u;
-      af[ks][3] = vb ? rb[8 * ks + 4 + t] : 0u;
+      af[ks][0] = va ? __ldg(ra + 8 * ks + t) : 0u;
+      af[ks][1] = vb ? __ldg(rb + 8 * ks + t) : 0u;
+      af[ks][2] = va ? __ldg(ra + 8 * ks + 4 + t) : 0u;
+      af[ks][3] = vb ? __ldg(rb + 8 * ks + 4 + t) : 0u;
     }
     float d[16][4];
 #pragma unroll
-    for (int nt = 0; nt < 16; ++nt) {
+    for (int nt = 0; nt < 16; ++nt)
 #pragma unroll
       for (int j = 0; j < 4; ++j) d[nt][j] = 0.f;
 #pragma unroll
-      for (int part = 0; part < 3; ++part) {
-        const __nv_bfloat16* urow = ut + ((size_t)part * kD + 8 * nt + g) * kUtStride + 2 * t;
+    for (int ks = 0; ks < 8; ++ks)
 #pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
-          const uint32_t b0 = *reinterpret_cast<const uint32_t*>(urow + 16 * ks);
-          const uint32_t b1 = *reinterpret_cast<const uint32_t*>(urow + 16 * ks + 8);
-          mma_bf16(d[nt], af[ks], b0, b1);
+      for (int part = 0; part < 3; ++part)
+#pragma unroll
+        for (int nt = 0; nt < 16; nt += 2) {
+          uint32_t bf[4];
+          ldsm_x4_trans(bf, rs_base + (uint32_t)((part * kD + 16 * ks) * kRStride + 8 * nt) * 2u);
+          mma_bf16(d[nt], af[ks], bf[0], bf[1]);
+          mma_bf16(d[nt + 1], af[ks], bf[2], bf[3]);
         }
-      }
-    }
-    // Walsh-Hadamard over i = 8 nt + 2t + e, for token g (regs 0,1) and g+8 (regs 2,3)
-#pragma unroll
-    for (int nt = 0; nt < 16; ++nt) {  // bit 0 (e)
-      const float x0 = d[nt][0], x1 = d[nt][1], x2 = d[nt][2], x3 = d[nt][3];
-      d[nt][0] = __fadd_rn(x0, x1);
-      d[nt][1] = __fsub_rn(x0, x1);
-      d[nt][2] = __fadd_rn(x2, x3);
-      d[nt][3] = __fsub_rn(x2, x3);
-    }
-#pragma unroll
-    for (int bit = 1; bit <= 2; bit <<= 1) {  // bits 1, 2 (t): across the quad
-      const bool up = (t & bit) != 0;
-#pragma unroll
-      for (int nt = 0; nt < 16; ++nt)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const float pv = __shfl_xor_sync(0xffffffffu, d[nt][j], bit);
-          d[nt][j] = up ? __fsub_rn(pv, d[nt][j]) : __fadd_rn(d[nt][j], pv);
-        }
-    }
-#pragma unroll
-    for (int bit = 1; bit < 16; bit <<= 1) {  // bits 3..6 (nt)
-#pragma unroll
-      for (int nt = 0; nt < 16; ++nt) {
-        if (nt & bit) continue;
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const float x0 = d[nt][j], x1 = d[nt | bit][j];
-          d[nt][j] = __fadd_rn(x0, x1);
-          d[nt | bit][j] = __fsub_rn(x0, x1);
-        }
-      }
-    }
-    // per token: zb[q][a] = y at r_q + 32a, r_q = 8 (q >> 1) + 2t + (q & 1): nt = (q >> 1) + 4a, e = q & 1
 #pragma unroll
     for (int half = 0; half < 2; ++half) {
-      float zb[8][4];
+      float v[8][4];
 #pragma unroll
-      for (int q = 0; q < 8; ++q)
+      for (int k = 0; k < 8; ++k)
 #pragma unroll
-        for (int aa = 0; aa < 4; ++aa) zb[q][aa] = d[(q >> 1) + 4 * aa][2 * half + (q & 1)] * kInvSqrtD;
-      finish_token_tc(a, half ? tb : ta, half ? vb : va, h, kind, zb, t);
+        for (int f = 0; f < 4; ++f) v[k][f] = d[2 * k + (f >> 1)][2 * half + (f & 1)];
+      finish_token_tc(a, half ? tb : ta, half ? vb : va, h, kind, v, t);
     }
   }
 }
@@ -377,8 +391,13 @@ okv_status launch_append(const okv_cache_desc* d, const void* k, const void* v, 
     // set on every call: the attribute belongs to the current device's context
     cudaError_t e = cudaFuncSetAttribute(append_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kTcSmem);
     if (e != cudaSuccess) return fail(OKV_ERR_CUDA, "append smem attribute: %s", cudaGetErrorString(e));
-    dim3 grid((T + kTcCtaTokens - 1) / kTcCtaTokens, d->num_kv_heads, 2);
-    append_tc_kernel<<<grid, kTcWarps * 32, kTcSmem, s>>>(a, T);
+    // about two CTAs per SM over all (KV head, K|V) pairs; each CTA takes whole rounds
+    const int pairs = 2 * d->num_kv_heads;
+    const int per_pair = std::max(1, 2 * device_sm_count() / pairs);
+    const int rounds = (T + kTcRound - 1) / kTcRound;
+    const int tokens_per_cta = ((rounds + per_pair - 1) / per_pair) * kTcRound;
+    dim3 grid((T + tokens_per_cta - 1) / tokens_per_cta, d->num_kv_heads, 2);
+    append_tc_kernel<<<grid, kTcWarps * 32, kTcSmem, s>>>(a, T, tokens_per_cta);
     return check_launch("append (tensor cores)");
   }
   dim3 grid((T + kAppTokens - 1) / kAppTokens, d->num_kv_heads, 2);

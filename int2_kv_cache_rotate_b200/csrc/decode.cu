@@ -85,57 +85,55 @@ __device__ __forceinline__ int working_ctas(const DecodeArgs& a, long long total
 }
 
 // ---------------------------------------------------------------------------
-// Kernel 1: q~ = q R_K for every query head, in CTAs of one (b, KV head) that
-// load U_K once (warp w holds rows 16w..16w+15, lane l columns 4l..4l+3, all
-// loads in flight together), plus the cost prefix (CTA (0,0)).
+// Kernel 1: q~ = q R_K for one (b, query head) per CTA: warp w holds rows
+// 16w..16w+15 of U_K (lane l columns 4l..4l+3, all loads in flight
+// together), the eight warps' partial sums meet in shared memory and warp 0
+// runs the butterfly.  CTA 0 also writes the cost prefix.
 // Also emits the query in the two forms the split-K kernel consumes:
 // signed 8-bit limbs in MMA-fragment order and fp16 hi/lo halves.
 // ---------------------------------------------------------------------------
 constexpr int kPrepThreads = 256;
 
 __global__ void __launch_bounds__(kPrepThreads) qrot_kernel(DecodeArgs a) {
-  extern __shared__ float red[];  // [G][8][128]
-  const int b = blockIdx.x, hk = blockIdx.y;
+  __shared__ float red[8][kD];
+  const int b = blockIdx.x / a.hq, head = blockIdx.x % a.hq;
+  const int hk = head / a.g;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int G = a.g;
-  if (b == 0 && hk == 0) {
-    __shared__ int chunk_sum[kPrepThreads];
-    const int per = (a.batch + kPrepThreads - 1) / kPrepThreads;
-    const int lo = threadIdx.x * per, hi = min(a.batch, lo + per);
-    int s = 0;
-    for (int i = lo; i < hi; ++i) s += unit_shape(clamp_len(a.context_lens, i, a.mbps, a.status, true)).cost;
-    chunk_sum[threadIdx.x] = s;
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      int run = 0;
-      for (int i = 0; i < kPrepThreads; ++i) {
-        const int c = chunk_sum[i];
-        chunk_sum[i] = run;
-        run += c;
-      }
-      a.prefix[a.batch] = run;
-    }
-    __syncthreads();
-    int run = chunk_sum[threadIdx.x];
-    for (int i = lo; i < hi; ++i) {
-      a.prefix[i] = run;
-      run += unit_shape(clamp_len(a.context_lens, i, a.mbps, a.status, false)).cost;
-    }
-  }
   const float* U = a.u_k + (size_t)hk * kD * kD;
   float4 u[16];
 #pragma unroll
   for (int r = 0; r < 16; ++r) u[r] = __ldg(reinterpret_cast<const float4*>(U + (size_t)(16 * warp + r) * kD) + lane);
-  float xq[16];  // this lane's input channel 16*warp + (lane & 15), every head of the group
-  {
-    const __nv_bfloat16* qv = a.q + ((size_t)b * a.hq + (size_t)hk * G) * kD + 16 * warp + (lane & 15);
+  const float xv = __bfloat162float(a.q[((size_t)b * a.hq + head) * kD + 16 * warp + (lane & 15)]);
+  if (blockIdx.x == 0) {
+    // cost prefix: thread i sums its chunk of consecutive entries, then a
+    // block-wide exclusive scan (warp shuffles, then the eight warp totals)
+    __shared__ int warp_tot[kPrepThreads / 32];
+    const int per = (a.batch + kPrepThreads - 1) / kPrepThreads;
+    const int lo = threadIdx.x * per, hi = min(a.batch, lo + per);
+    int own = 0;
+    for (int i = lo; i < hi; ++i) own += unit_shape(clamp_len(a.context_lens, i, a.mbps, a.status, true)).cost;
+    int inc = own;
 #pragma unroll
-    for (int gg = 0; gg < 16; ++gg) xq[gg] = gg < G ? __bfloat162float(qv[(size_t)gg * kD]) : 0.f;
+    for (int d = 1; d < 32; d <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, inc, d);
+      if (lane >= d) inc += v;
+    }
+    if (lane == 31) warp_tot[warp] = inc;
+    __syncthreads();
+    int before = 0, total = 0;
+#pragma unroll
+    for (int w = 0; w < kPrepThreads / 32; ++w) {
+      before += w < warp ? warp_tot[w] : 0;
+      total += warp_tot[w];
+    }
+    int run = before + inc - own;
+    for (int i = lo; i < hi; ++i) {
+      a.prefix[i] = run;
+      run += unit_shape(clamp_len(a.context_lens, i, a.mbps, a.status, false)).cost;
+    }
+    if (threadIdx.x == 0) a.prefix[a.batch] = total;
   }
-#pragma unroll
-  for (int gg = 0; gg < 16; ++gg) {
-    if (gg >= G) break;
-    const float xv = xq[gg];
+  {
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
     for (int r = 0; r < 16; ++r) {
@@ -145,23 +143,23 @@ __global__ void __launch_bounds__(kPrepThreads) qrot_kernel(DecodeArgs a) {
       acc.z = fmaf(x, u[r].z, acc.z);
       acc.w = fmaf(x, u[r].w, acc.w);
     }
-    *reinterpret_cast<float4*>(red + ((size_t)gg * 8 + warp) * kD + 4 * lane) = acc;
+    *reinterpret_cast<float4*>(&red[warp][4 * lane]) = acc;
   }
   __syncthreads();
-  for (int gg = warp; gg < G; gg += 8) {
+  if (warp == 0) {
     float y[4];
 #pragma unroll
     for (int aa = 0; aa < 4; ++aa) {
       float s = 0.f;
 #pragma unroll
-      for (int w = 0; w < 8; ++w) s += red[((size_t)gg * 8 + w) * kD + lane + 32 * aa];
+      for (int w = 0; w < 8; ++w) s += red[w][lane + 32 * aa];
       y[aa] = s;
     }
     wht128_warp(y, lane);
 #pragma unroll
     for (int aa = 0; aa < 4; ++aa) y[aa] *= kInvSqrtD;
     const int r = rev5(lane);
-    const size_t bh = (size_t)b * a.hq + (size_t)hk * G + gg;
+    const size_t bh = (size_t)b * a.hq + head;
     *reinterpret_cast<float4*>(a.qrot + bh * kD + 4 * r) = make_float4(y[0], y[2], y[1], y[3]);
     // Integer limbs for the tensor-core score tiles: Q = rint(q~/sigma) in
     // [-32000, 32000] = 256*hi + lo with hi, lo signed 8-bit.  Bytes are stored
@@ -534,6 +532,7 @@ template <int G>
 __global__ void __launch_bounds__(kHW * 32, (G <= 4) ? 2 : 1) decode_heads_kernel(DecodeArgs a) {
   constexpr int NT = HCfg<G>::NT, HP = HCfg<G>::HP;
   extern __shared__ __align__(16) unsigned char smem_raw[];
+  __shared__ int btq[2][32];  // producer's block ids, two 32-block windows
   unsigned char* ring = smem_raw;
   float* accs = reinterpret_cast<float*>(ring + HCfg<G>::ring_bytes);
   uint64_t* full = reinterpret_cast<uint64_t*>(reinterpret_cast<unsigned char*>(accs) + HCfg<G>::acc_bytes);
@@ -628,47 +627,73 @@ __global__ void __launch_bounds__(kHW * 32, (G <= 4) ? 2 : 1) decode_heads_kerne
     const int nst = (slot_ok && alive && p1 > p0) ? (p1 - p0 + nb - 1) / nb : 0;
     const int32_t* trow = a.block_table + (size_t)(slot_ok ? slot : 0) * a.mbps;
 
-    // warp 0 lane 0: put stage j of this entry in the next ring position
-    // (ps = its stage, puse = how often that stage was filled before)
+    // Warp 0 puts stage j of this entry in the next ring position (ps = its
+    // stage, puse = how often that stage was filled before).  Block ids come
+    // from a two-window shared buffer that async copies fill one 32-block
+    // window ahead (btq[bt_buf] holds blocks bt_base .. bt_base + 31), so no
+    // block-table load sits between a released stage and its refill.  Lane
+    // q < nb handles block q of the stage.
     uint32_t ps = it % kHStages, puse = it / kHStages;
-    auto issue = [&](int j) -> bool {
+    int bt_base = p0, bt_buf = 0;
+    auto bt_fill = [&](int wbase, int buf) {  // all lanes of warp 0
+      const int pi = wbase + lane;
+      if (pi < p1) cp_async4(&btq[buf][lane], trow + pi);
+      else btq[buf][lane] = -1;
+      cp_async_commit();
+    };
+    if (warp == 0 && nst > 0) {
+      cp_async_wait_all();  // the previous entry's prefetch
+      __syncwarp();
+      bt_fill(p0, 0);
+      cp_async_wait_all();
+      __syncwarp();
+      bt_fill(p0 + 32, 1);
+    }
+    auto issue = [&](int j) -> bool {  // all lanes of warp 0
       const uint32_t s = ps;
-      if (puse > 0 && !mbar_wait_bounded(&empty[s], (puse - 1) & 1u)) return false;
+      bool ok = true;
+      if (lane == 0 && puse > 0) ok = mbar_wait_bounded(&empty[s], (puse - 1) & 1u);
+      if (!__shfl_sync(0xffffffffu, ok, 0)) return false;
       if (++ps == (uint32_t)kHStages) {
         ps = 0;
         ++puse;
       }
-      uint32_t bytes = 0;
-      for (int q = 0; q < nb; ++q) {  // token counts first: the barrier must expect every byte
-        const int pi = p0 + j * nb + q;
-        int bid = pi < p1 ? trow[pi] : -1;
-        if (pi < p1 && (bid < 0 || bid >= a.num_blocks)) {
-          raise_flag(a.status, OKV_DEV_BAD_BLOCK);
-          bid = -1;
-        }
-        ntok[s * kSlotsPerStage + q] = bid >= 0 ? (uint8_t)min(kBlock, us.n_int2 - kBlock * pi) : 0;
-        if (bid >= 0) bytes += copy_bytes;
+      const int pj = p0 + j * nb;  // nb divides 32, so a stage never straddles two windows
+      while (pj >= bt_base + 32) {
+        bt_base += 32;
+        bt_buf ^= 1;
+        cp_async_wait_all();
+        __syncwarp();
+        bt_fill(bt_base + 32, bt_buf ^ 1);  // the window just retired takes the one after next
       }
-      mbar_arrive_expect_tx(&full[s], bytes);
-      for (int q = 0; q < nb; ++q) {
-        const int pi = p0 + j * nb + q;
-        const int bid = pi < p1 ? trow[pi] : -1;
-        if (bid >= 0 && bid < a.num_blocks)
-          bulk_g2s(ring + s * kHStageBytes + q * copy_bytes, a.pages + (size_t)bid * copy_bytes, copy_bytes,
-                   &full[s]);
+      const int pi = pj + lane;
+      const bool mine = lane < nb && pi < p1;
+      int bid = mine ? btq[bt_buf][pj - bt_base + lane] : -1;
+      if (mine && (bid < 0 || bid >= a.num_blocks)) {
+        raise_flag(a.status, OKV_DEV_BAD_BLOCK);
+        bid = -1;
       }
+      if (lane < nb) ntok[s * kSlotsPerStage + lane] = bid >= 0 ? (uint8_t)min(kBlock, us.n_int2 - kBlock * pi) : 0;
+      const uint32_t nvalid = __popc(__ballot_sync(0xffffffffu, bid >= 0));
+      __syncwarp();
+      // the barrier must expect every byte before any copy can complete on it
+      if (lane == 0) mbar_arrive_expect_tx(&full[s], nvalid * copy_bytes);
+      __syncwarp();
+      if (bid >= 0)
+        bulk_g2s(ring + s * kHStageBytes + lane * copy_bytes, a.pages + (size_t)bid * copy_bytes, copy_bytes,
+                 &full[s]);
       return true;
     };
     bool prod_ok = true;
-    if (warp == 0 && lane == 0)
+    if (warp == 0)
       for (int j = 0; j < min(kHStages - 1, nst) && prod_ok; ++j) prod_ok = issue(j);
 
     int done = 0;
     uint32_t cs = it % kHStages, cph = (it / kHStages) & 1u;  // consumer stage and phase parity
     for (int j = 0; j < nst; ++j) {
       if (warp == 0) {
-        if (lane == 0 && prod_ok && j + kHStages - 1 < nst) prod_ok = issue(j + kHStages - 1);
-        if (!__shfl_sync(0xffffffffu, prod_ok, 0)) {
+        if (prod_ok && j + kHStages - 1 < nst) prod_ok = issue(j + kHStages - 1);
+        if (!prod_ok) {
           if (lane == 0) raise_flag(a.status, OKV_DEV_TIMEOUT);
           alive = false;
         }
@@ -1065,139 +1090,169 @@ __global__ void __launch_bounds__(kHW * 32, (G <= 4) ? 2 : 1) decode_heads_kerne
       }
     }
   }
+  if (warp == 0) cp_async_wait_all();  // no block-id prefetch may outlive the CTA
 }
 
 // ---------------------------------------------------------------------------
-// Kernel 3: merge the splits of each (b, KV head), normalise, undo the value
-// rotation (un-permute, Hadamard, U_V^T) and write fp32 outputs.  U_V is
-// staged in shared memory with all loads in flight together (warp w rows
-// 16w..16w+15, lane l columns 4l..4l+3), padded to 129 columns so that each
-// thread can walk its own output row without bank conflicts.
+// Kernel 3: merge the splits of one (b, query head), normalise, undo the
+// value rotation (un-permute, Hadamard, U_V^T) and write the fp32 output.
+// One CTA per (b, query head) so that enough loads are in flight: before any
+// reduction a CTA starts async copies of U_V into shared memory and loads the
+// o' rows of the first 128 splits into registers (warp w: splits w, w+8, ...;
+// lane l: channels 4l..4l+3).
 // ---------------------------------------------------------------------------
-constexpr int kUPad = 129;
 constexpr int kCombThreads = 256;
+constexpr int kCombWarps = kCombThreads / 32;
+constexpr int kCombPre = 16;      // o' rows per warp loaded ahead of the weights
 constexpr int kMaxSplits = 1024;  // >= split-K CTAs (at most 4 per SM)
+constexpr size_t kCombSmem = (size_t)(kD * kD + kMaxSplits + kCombWarps * kD + kD + 2 * kCombWarps) * sizeof(float);
+
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(smem_u32(smem_dst)), "l"(gsrc) : "memory");
+}
 
 __global__ void __launch_bounds__(kCombThreads) combine_kernel(DecodeArgs a) {
-  extern __shared__ float smem[];
-  float* us_ = smem;                 // U_V [128][129]
-  float* xs = us_ + kD * kUPad;      // [G][128]
-  const int u = blockIdx.x;
-  const int b = u / a.hkv, hk = u % a.hkv;
+  extern __shared__ __align__(16) float csm[];
+  float* us_ = csm;                        // U_V [128][128]
+  float* ml = us_ + kD * kD;               // [kMaxSplits] split maxima, then weights 2^(m_c - M)
+  float* wsum = ml + kMaxSplits;           // [warps][128] per-warp partial sums
+  float* xs = wsum + kCombWarps * kD;      // [128] merged, normalised, un-rotated o
+  float* redm = xs + kD;                   // [warps]
+  float* redl = redm + kCombWarps;         // [warps]
+  const int b = blockIdx.x / a.hq, head = blockIdx.x % a.hq;
+  const int hk = head / a.g;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int G = a.g;
   {
-    const float* uv = a.u_v + (size_t)hk * kD * kD;
-    float4 r[16];
+    const float* U = a.u_v + (size_t)hk * kD * kD;
 #pragma unroll
-    for (int i = 0; i < 16; ++i) r[i] = __ldg(reinterpret_cast<const float4*>(uv + (size_t)(16 * warp + i) * kD) + lane);
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      float* row = us_ + (16 * warp + i) * kUPad + 4 * lane;
-      row[0] = r[i].x;
-      row[1] = r[i].y;
-      row[2] = r[i].z;
-      row[3] = r[i].w;
+    for (int k = 0; k < kD * kD / 4 / kCombThreads; ++k) {
+      const int i = tid + kCombThreads * k;
+      cp_async16(us_ + 4 * i, U + 4 * i);
     }
+    cp_async_commit();
   }
   const UnitShape sh = unit_shape(clamp_len(a.context_lens, b, a.mbps, a.status, false));
   const long long total = a.prefix[a.batch];
-  float* outp = a.out + ((size_t)b * a.hq + (size_t)hk * G) * kD;
+  float* outp = a.out + ((size_t)b * a.hq + head) * kD;
   if (sh.cost == 0 || total == 0) {
-    for (int i = tid; i < G * kD; i += blockDim.x) outp[i] = 0.f;
+    if (tid < kD) outp[tid] = 0.f;
+    cp_async_wait_all();
     return;
   }
   const long long pu = a.prefix[b];
   const int nc = working_ctas(a, total);
   const int c0 = cta_of(pu, total, nc);
   const int ns = cta_of(pu + sh.cost - 1, total, nc) - c0 + 1;  // splits of this entry
-  float* wts = xs + G * kD;                 // [G][kMaxSplits] split weights 2^(m_c - M)
-  float* red = wts + G * kMaxSplits;        // [G] 1/l
-  float* wpart = red + ((G + 3) & ~3);      // [8 warps][G][128] partial sums (16-B aligned)
-  const float* base = a.part + ((size_t)(c0 + b) * a.hq + (size_t)hk * G) * kPartStride;
   const size_t split_stride = (size_t)a.hq * kPartStride;
-  // 1) per head (one warp each): max of the split maxima, weights, 1/l
-  for (int gg = warp; gg < G; gg += kCombThreads / 32) {
-    float mx = -INFINITY;
-    for (int c = lane; c < ns; c += 32) mx = fmaxf(mx, base[c * split_stride + (size_t)gg * kPartStride + 128]);
-    mx = warp_max(mx);
-    float l = 0.f;
-    for (int c = lane; c < ns; c += 32) {
-      const float* src = base + c * split_stride + (size_t)gg * kPartStride;
-      const float w = (mx == -INFINITY || src[128] == -INFINITY) ? 0.f : exp2f(src[128] - mx);
-      wts[gg * kMaxSplits + c] = w;
-      l = fmaf(src[129], w, l);
-    }
-    l = warp_sum(l);
-    if (lane == 0) red[gg] = l > 0.f ? 1.f / l : 0.f;
-  }
-  __syncthreads();
-  // 2) weighted sum of the splits: warp w takes splits w, w+8, ...; lane l
-  //    channels 4l..4l+3; four splits in flight per iteration
-  for (int gg = 0; gg < G; ++gg) {
-    const float* hb = base + (size_t)gg * kPartStride + 4 * lane;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    int c = warp;
-    for (; c + 24 < ns; c += 32) {
-      float4 x[4];
-      float w[4];
+  const float* base = a.part + ((size_t)(c0 + b) * a.hq + head) * kPartStride;
+  // o' rows of the first kCombPre splits of this warp
+  float4 pre[kCombPre];
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        x[k] = *reinterpret_cast<const float4*>(hb + (size_t)(c + 8 * k) * split_stride);
-        w[k] = wts[gg * kMaxSplits + c + 8 * k];
-      }
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        acc.x = fmaf(x[k].x, w[k], acc.x);
-        acc.y = fmaf(x[k].y, w[k], acc.y);
-        acc.z = fmaf(x[k].z, w[k], acc.z);
-        acc.w = fmaf(x[k].w, w[k], acc.w);
-      }
-    }
-    for (; c < ns; c += 8) {
-      const float4 x = *reinterpret_cast<const float4*>(hb + (size_t)c * split_stride);
-      const float w = wts[gg * kMaxSplits + c];
-      acc.x = fmaf(x.x, w, acc.x);
-      acc.y = fmaf(x.y, w, acc.y);
-      acc.z = fmaf(x.z, w, acc.z);
-      acc.w = fmaf(x.w, w, acc.w);
-    }
-    *reinterpret_cast<float4*>(wpart + ((size_t)warp * G + gg) * kD + 4 * lane) = acc;
+  for (int j = 0; j < kCombPre; ++j) {
+    const int c = warp + kCombWarps * j;
+    pre[j] = c < ns ? *reinterpret_cast<const float4*>(base + (size_t)c * split_stride + 4 * lane)
+                    : make_float4(0.f, 0.f, 0.f, 0.f);
   }
-  __syncthreads();
-  for (int i = tid; i < G * kD; i += blockDim.x) {
-    const int gg = i / kD, ch = i % kD;
-    float o = 0.f;
-#pragma unroll
-    for (int w = 0; w < kCombThreads / 32; ++w) o += wpart[((size_t)w * G + gg) * kD + ch];
-    xs[i] = o * red[gg];
+  // split maxima and sums, and the global maximum
+  float mx = -INFINITY;
+  for (int c = tid; c < ns; c += kCombThreads) {
+    const float2 m2 = *reinterpret_cast<const float2*>(base + (size_t)c * split_stride + 128);
+    ml[c] = m2.x;
+    wsum[c] = m2.y;  // the sums borrow the partial-sum buffer until the weights are known
+    mx = fmaxf(mx, m2.x);
   }
+  mx = warp_max(mx);
+  if (lane == 0) redm[warp] = mx;
   __syncthreads();
-  // un-permute + Hadamard, one warp per head: lane holds pre-permutation
-  // channels l + 32a = rotated channels 4*rev5(l) + rev2(a)
-  for (int gg = warp; gg < G; gg += kCombThreads / 32) {
+  mx = redm[0];
+#pragma unroll
+  for (int w = 1; w < kCombWarps; ++w) mx = fmaxf(mx, redm[w]);
+  float l = 0.f;
+  for (int c = tid; c < ns; c += kCombThreads) {
+    const float m = ml[c];
+    const float w = (mx == -INFINITY || m == -INFINITY) ? 0.f : exp2f(m - mx);
+    ml[c] = w;
+    l = fmaf(wsum[c], w, l);
+  }
+  l = warp_sum(l);
+  if (lane == 0) redl[warp] = l;
+  __syncthreads();
+  l = 0.f;
+#pragma unroll
+  for (int w = 0; w < kCombWarps; ++w) l += redl[w];
+  const float inv_l = l > 0.f ? 1.f / l : 0.f;
+  // weighted sum of the splits
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+  for (int j = 0; j < kCombPre; ++j) {
+    const int c = warp + kCombWarps * j;
+    const float w = c < ns ? ml[c] : 0.f;
+    acc.x = fmaf(pre[j].x, w, acc.x);
+    acc.y = fmaf(pre[j].y, w, acc.y);
+    acc.z = fmaf(pre[j].z, w, acc.z);
+    acc.w = fmaf(pre[j].w, w, acc.w);
+  }
+  for (int c0w = warp + kCombWarps * kCombPre; c0w < ns; c0w += kCombWarps * kCombPre) {
+#pragma unroll
+    for (int j = 0; j < kCombPre; ++j) {
+      const int c = c0w + kCombWarps * j;
+      pre[j] = c < ns ? *reinterpret_cast<const float4*>(base + (size_t)c * split_stride + 4 * lane)
+                      : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int j = 0; j < kCombPre; ++j) {
+      const int c = c0w + kCombWarps * j;
+      const float w = c < ns ? ml[c] : 0.f;
+      acc.x = fmaf(pre[j].x, w, acc.x);
+      acc.y = fmaf(pre[j].y, w, acc.y);
+      acc.z = fmaf(pre[j].z, w, acc.z);
+      acc.w = fmaf(pre[j].w, w, acc.w);
+    }
+  }
+  __syncthreads();  // every thread is done with the sums borrowed in wsum
+  *reinterpret_cast<float4*>(&wsum[warp * kD + 4 * lane]) = acc;
+  cp_async_wait_all();
+  __syncthreads();
+  // un-permute + Hadamard in warp 0: lane holds pre-permutation channels
+  // l + 32a = rotated channels 4*rev5(l) + rev2(a)
+  if (warp == 0) {
     const int r = rev5(lane);
     float y[4];
-    y[0] = xs[gg * kD + 4 * r + 0];
-    y[1] = xs[gg * kD + 4 * r + 2];
-    y[2] = xs[gg * kD + 4 * r + 1];
-    y[3] = xs[gg * kD + 4 * r + 3];
-    __syncwarp();
+#pragma unroll
+    for (int aa = 0; aa < 4; ++aa) {
+      const int ch = 4 * r + rev2(aa);
+      float o = 0.f;
+#pragma unroll
+      for (int w = 0; w < kCombWarps; ++w) o += wsum[w * kD + ch];
+      y[aa] = o * inv_l;
+    }
     wht128_warp(y, lane);
 #pragma unroll
-    for (int j = 0; j < 4; ++j) xs[gg * kD + lane + 32 * j] = y[j] * kInvSqrtD;
+    for (int aa = 0; aa < 4; ++aa) xs[lane + 32 * aa] = y[aa] * kInvSqrtD;
   }
   __syncthreads();
-  // o_c = sum_i x_i U_V[c][i]: thread = (output channel, half of the heads)
-  const int ch = tid & (kD - 1), half = tid >> 7;
-  for (int gg = half; gg < G; gg += 2) {
-    float acc = 0.f;
-    const float* xr = xs + gg * kD;
-    const float* ur = us_ + ch * kUPad;
-#pragma unroll 16
-    for (int i = 0; i < kD; ++i) acc = fmaf(xr[i], ur[i], acc);
-    outp[gg * kD + ch] = acc;
+  // o_c = sum_i x_i U_V[c][i]: warp w, channels 16w..16w+15; lane l inputs 4l..4l+3
+  const float4 xv = *reinterpret_cast<const float4*>(&xs[4 * lane]);
+  float part[16];
+#pragma unroll
+  for (int r = 0; r < 16; ++r) {
+    const float4 u = *reinterpret_cast<const float4*>(us_ + (16 * warp + r) * kD + 4 * lane);
+    part[r] = fmaf(xv.x, u.x, fmaf(xv.y, u.y, fmaf(xv.z, u.z, xv.w * u.w)));
   }
+  // transpose-reduce: after the four halving steps lane l holds the partial of
+  // channel 16w + (l & 15) summed over 16 lanes; one more step finishes it
+#pragma unroll
+  for (int step = 8; step >= 1; step >>= 1) {
+    const bool upper = (lane & step) != 0;
+#pragma unroll
+    for (int r = 0; r < step; ++r) {
+      const float send = upper ? part[r] : part[r + step];
+      const float keep = upper ? part[r + step] : part[r];
+      part[r] = keep + __shfl_xor_sync(0xffffffffu, send, step);
+    }
+  }
+  const float o = part[0] + __shfl_xor_sync(0xffffffffu, part[0], 16);
+  if (lane < 16) outp[16 * warp + lane] = o;
 }
 
 template <int G>
@@ -1259,10 +1314,8 @@ okv_status launch_decode(const okv_cache_desc* d, const void* q, int B, const in
   a.num_slots = d->num_seq_slots;
   a.mbps = d->max_blocks_per_seq;
 
-  const size_t qsmem = (size_t)a.g * 8 * kD * sizeof(float);
-  cudaError_t e = cudaFuncSetAttribute(qrot_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)qsmem);
-  if (e != cudaSuccess) return fail(OKV_ERR_CUDA, "query rotation smem attribute: %s", cudaGetErrorString(e));
-  qrot_kernel<<<dim3(B, a.hkv), kPrepThreads, qsmem, s>>>(a);
+  cudaError_t e = cudaSuccess;
+  qrot_kernel<<<B * a.hq, kPrepThreads, 0, s>>>(a);
   okv_status st = check_launch("query rotation");
   if (st != OKV_OK) return st;
   cudaEvent_t ev0, ev1;
@@ -1289,10 +1342,9 @@ okv_status launch_decode(const okv_cache_desc* d, const void* q, int B, const in
   if (st != OKV_OK) return st;
   if (ev1 != nullptr && cudaEventRecordWithFlags(ev1, s, cudaEventRecordExternal) != cudaSuccess)
     return fail(OKV_ERR_CUDA, "cudaEventRecord failed");
-  const size_t csmem = (size_t)(kD * kUPad + a.g * kD + a.g * kMaxSplits + ((a.g + 3) & ~3) + 8 * a.g * kD) * sizeof(float);
-  e = cudaFuncSetAttribute(combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)csmem);
+  e = cudaFuncSetAttribute(combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kCombSmem);
   if (e != cudaSuccess) return fail(OKV_ERR_CUDA, "combine smem attribute: %s", cudaGetErrorString(e));
-  combine_kernel<<<B * a.hkv, kCombThreads, csmem, s>>>(a);
+  combine_kernel<<<B * a.hq, kCombThreads, kCombSmem, s>>>(a);
   return check_launch("combine");
 }
 

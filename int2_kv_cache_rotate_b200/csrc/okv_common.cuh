@@ -81,6 +81,42 @@ __device__ __forceinline__ __half fp16_sat(float x) {
   return __float2half_rn(fminf(fmaxf(x, -65504.0f), 65504.0f));
 }
 
+// The quantiser's code decision without a division.  With x = fl(z - m)
+// and s > 0, the code clamp(rint_even(fl(x / s)), 0, 3) is the number of
+// thresholds x passes, because round-to-nearest-even puts the decision points
+// exactly at
+//   c >= 1  <=>  fl(x / s) > 0.5  <=>  x / s > 0.5 + 2^-25   (0.5 is the even neighbour)
+//   c >= 2  <=>  fl(x / s) >= 1.5 <=>  x / s >= 1.5 - 2^-24  (1.5 is the even neighbour)
+//   c >= 3  <=>  fl(x / s) > 2.5  <=>  x / s > 2.5 + 2^-23  (2.5 is the even neighbour)
+// (the half-ulp of fp32 in [0.5, 1), [1, 2) and [2, 4)).  Multiplied through
+// by s: x - 0.5s > s 2^-25, x - 1.5s >= -s 2^-24, x - 2.5s > s 2^-23.  k s is
+// exact for k in {0.5, 1.5, 2.5} (s has 11 significant bits), s 2^-n is
+// exact (s >= 2^-24), and each difference x - k s is exact whenever x lies
+// within a factor of two of k s (Sterbenz); when it does not, |x - k s| >=
+// k s / 2, far from the tiny threshold, so the rounded difference has the
+// same side.  Every code therefore equals the division's, bit for bit.
+struct CodeThresholds {
+  float h1, h2, h3;  // 0.5 s, 1.5 s, 2.5 s
+  float e1, e2, e3;  // s 2^-25, -s 2^-24, s 2^-23
+};
+
+__device__ __forceinline__ CodeThresholds code_thresholds(float s) {
+  CodeThresholds t;
+  t.h1 = 0.5f * s;
+  t.h2 = 1.5f * s;
+  t.h3 = 2.5f * s;
+  t.e1 = s * 0x1p-25f;
+  t.e2 = -s * 0x1p-24f;
+  t.e3 = s * 0x1p-23f;
+  return t;
+}
+
+// code of x = fl(z - m); only for s > 0 (s = 0 gives code 0 by definition)
+__device__ __forceinline__ uint32_t int2_code(float x, const CodeThresholds& t) {
+  return (uint32_t)(__fsub_rn(x, t.h1) > t.e1) + (uint32_t)(__fsub_rn(x, t.h2) >= t.e2) +
+         (uint32_t)(__fsub_rn(x, t.h3) > t.e3);
+}
+
 // INT2 group quantiser over the 128 values of a warp (y[a] = value at
 // pre-permutation index l + 32a, i.e. rotated channel 4*rev5(l) + rev2(a)).
 // All steps are IEEE fp32 round-to-nearest; returns this lane's packed code
@@ -101,14 +137,10 @@ __device__ __forceinline__ Quantized quantize_warp(const float y[4]) {
   const float s = __half2float(s16);
   const float m = __half2float(m16);
   uint32_t byte = 0;
+  if (s != 0.0f) {
+    const CodeThresholds th = code_thresholds(s);
 #pragma unroll
-  for (int a = 0; a < 4; ++a) {
-    uint32_t c = 0;
-    if (s != 0.0f) {
-      const float r = rintf(__fdiv_rn(__fsub_rn(y[a], m), s));
-      c = (uint32_t)fminf(fmaxf(r, 0.0f), 3.0f);
-    }
-    byte |= c << (2 * rev2(a));
+    for (int a = 0; a < 4; ++a) byte |= int2_code(__fsub_rn(y[a], m), th) << (2 * rev2(a));
   }
   Quantized q;
   q.byte = byte;
@@ -151,6 +183,16 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
       "l"(src), "r"(bytes), "r"(smem_u32(bar))
       : "memory");
 }
+
+// 4-byte asynchronous global -> shared copy (no register round trip), grouped
+// per thread; cp_async_wait_all waits for this thread's groups.
+__device__ __forceinline__ void cp_async4(void* smem_dst, const void* gsrc) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;\n" ::"r"(smem_u32(smem_dst)), "l"(gsrc) : "memory");
+}
+
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;\n" ::: "memory"); }
 
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(smem_u32(bar)) : "memory");

@@ -66,6 +66,40 @@ def special_vectors() -> np.ndarray:
     return np.stack(rows)
 
 
+def rounding_boundary_vectors(seed: int, n: int) -> np.ndarray:
+    """[n, 128] fp32 groups whose values sit within 8 fp32 ulps of each
+    rounding midpoint m + (k + 1/2) s of their own quantiser, so that the
+    code decision turns on the last bit of fl(fl(z - m) / s) and on ties to
+    even.  s spans fp16 normals and subnormals, m sits up to 2^7 s away from
+    zero on either side (so fl(z - m) rounds too).  The oracle's quantiser
+    only locates s and m; the rows are then quantised afresh by both sides."""
+    r = np.random.default_rng(np.random.SeedSequence([seed, 4242]))
+    rows = np.empty((n, D), np.float32)
+    for i in range(n):
+        s_t = np.float64(np.float16(r.uniform(1.0, 2.0) * 2.0 ** int(r.integers(-24, 11))))
+        if s_t == 0:
+            s_t = 2.0 ** -24
+        m_t = np.float32(np.float16(np.clip(r.uniform(-1.0, 1.0) * s_t * 2.0 ** int(r.integers(0, 8)),
+                                            -60000.0, 60000.0)))
+        row = np.full(D, m_t, np.float32)
+        row[1] = np.float32(np.float64(m_t) + 3.0 * s_t)
+        _, s16, m16 = O.quantize(row[None])
+        s, m = np.float64(s16[0]), np.float64(m16[0])
+        vals = []
+        for k in range(3):
+            c = np.float32(m + (k + 0.5) * s)
+            up = dn = c
+            vals.append(c)
+            for _ in range(8):
+                up = np.nextafter(up, np.float32(np.inf))
+                dn = np.nextafter(dn, np.float32(-np.inf))
+                vals += [up, dn]
+        vals = np.array(vals, np.float32)
+        row[2:2 + len(vals)] = np.clip(vals, row[0], row[1])
+        rows[i] = row[r.permutation(D)]
+    return rows
+
+
 def rotations(seed: int, hkv: int):
     """Seeded orthogonal U_K, U_V per KV head (fp32-exact values, as float64)."""
     r = np.random.default_rng(np.random.SeedSequence([seed, 999]))

@@ -94,6 +94,31 @@ def test_append_pre_rotated_bit_exact(lens):
                     assert np.array_equal(row.view(np.uint16), st["z16"][p].view(np.uint16)), (b, h, kind, p)
 
 
+def test_quantizer_rounding_midpoints_bit_exact():
+    """Groups built so that codes are decided by the last bit of the fp32
+    division and by ties to even: the kernels' code decisions must match the
+    oracle's division-based quantiser exactly."""
+    okv = _okv()
+    n = 3000
+    rows = H.rounding_boundary_vectors(31, n)
+    lay = H.Layout(31, [n])
+    uk, uv = H.rotations(31, 1)
+    gc = _gpu_cache(4, 1, lay, uk, uv)
+    k, v = rows[:, None, :], rows[::-1].copy()[:, None, :]
+    slots, pos = lay.flat()
+    okv.append_quantize(gc, _t(k), _t(v), _t(slots), _t(pos), _t(lay.table), _t(np.array([n], np.int32)),
+                        pre_rotated=True)
+    pages = gc.pages.cpu().numpy()
+    for kind, z in ((0, k[:, 0]), (1, v[:, 0])):
+        c_ref, s_ref, m_ref = O.quantize(z)
+        packed, s16, m16 = H.gather_codes(pages, lay.table, 0, 0, 1, n, kind)
+        assert np.array_equal(s16.view(np.uint16), s_ref.view(np.uint16))
+        assert np.array_equal(m16.view(np.uint16), m_ref.view(np.uint16))
+        bad = np.argwhere(O.unpack(packed) != c_ref)
+        assert len(bad) == 0, (kind, bad[:5])
+    assert gc.device_status() == 0
+
+
 def test_dequantize_bit_exact_and_original_basis():
     okv = _okv()
     lens = [300, 17, 0, 144]
