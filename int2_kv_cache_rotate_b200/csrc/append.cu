@@ -364,6 +364,335 @@ __global__ void __launch_bounds__(kTcWarps * 32, 2) append_tc_kernel(AppendArgs 
   }
 }
 
+// ---------------------------------------------------------------------------
+// tcgen05 append (prefill chunks): the same z = k R contraction on the
+// 5th-generation tensor cores, accumulators in tensor memory.
+//
+// B = R^T (128 output channels x K = 384: R's three bf16 parts stacked along
+// K, so one accumulation gives k R0 + k R1 + k R2) lives in shared memory in
+// the K-major 128-byte-swizzled layout the MMA descriptors describe: part pt,
+// K-block kb (64 channels) is a 16 KB region of 128 rows x 128 B; element
+// (n, c) sits in row n, 16-byte chunk ((c % 64) / 8) ^ (n % 8).  A is one
+// 128-token tile of k for this KV head, two K-blocks of the same layout,
+// loaded by zero-filling async copies (rows past T read as zeros).
+// One thread issues 24 MMAs (M = N = 128, K = 16 each) per tile into a
+// 128-column TMEM buffer; two buffers let the MMAs of tile i+1 run during the
+// epilogue of tile i.  Epilogue: warp w reads TMEM lanes 32 (w % 4) .. +31
+// (tokens) and columns 64 (w / 4) .. +63, so each thread holds half a token's
+// rotated vector; the two halves meet in shared memory for min/max.
+// Every mbarrier wait is bounded; TMEM is freed on every path.
+// ---------------------------------------------------------------------------
+constexpr int kUmWarps = 8;
+constexpr int kUmThreads = 32 * kUmWarps;
+constexpr int kUmTile = 128;
+constexpr uint32_t kUmRegion = 16384;                 // 128 rows x 128 B
+constexpr uint32_t kUmBBytes = 6 * kUmRegion;         // 3 parts x 2 K-blocks
+constexpr uint32_t kUmABytes = 2 * kUmRegion;         // one tile, 2 K-blocks
+constexpr uint32_t kUmCtlBytes = 64 + 2 * kUmTile * 2 * 4;  // barriers, TMEM base, min/max exchange
+constexpr size_t kUmSmem = 1024 + kUmBBytes + 2 * kUmABytes + kUmCtlBytes;
+constexpr uint32_t kUmTmemCols = 256;
+// instruction descriptor: D f32, A and B bf16, both K-major, N = 128, M = 128
+constexpr uint32_t kUmIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((128u >> 3) << 17) | ((128u >> 4) << 24);
+
+__device__ __forceinline__ uint32_t um_swz(uint32_t row, uint32_t byte_in_row) {
+  return row * 128u + ((((byte_in_row >> 4) ^ (row & 7u)) << 4) | (byte_in_row & 15u));
+}
+
+// shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row groups 1024 B apart
+__device__ __forceinline__ uint64_t um_desc(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);   // start address
+  d |= (uint64_t)1u << 16;                   // leading byte offset (unused for swizzled K-major), 16 B
+  d |= (uint64_t)(1024u >> 4) << 32;         // stride byte offset
+  d |= (uint64_t)1u << 46;                   // descriptor version for tcgen05
+  d |= (uint64_t)2u << 61;                   // 128-byte swizzle
+  return d;
+}
+
+__device__ __forceinline__ void um_cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+
+__device__ __forceinline__ void um_fence_proxy_async() {
+  asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+}
+__device__ __forceinline__ void um_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
+}
+__device__ __forceinline__ void um_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
+}
+
+__device__ __forceinline__ void um_mma(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(tmem_d),
+      "l"(adesc), "l"(bdesc), "r"(kUmIdesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void um_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(smem_u32(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ void um_ld32(uint32_t taddr, float (&v)[32]) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ void um_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory"); }
+
+__global__ void __launch_bounds__(kUmThreads, 1) append_umma_kernel(AppendArgs a, int T) {
+  extern __shared__ unsigned char um_raw[];
+  const uint32_t raw_u32 = smem_u32(um_raw);
+  const uint32_t base = (raw_u32 + 1023u) & ~1023u;  // swizzle atoms need 1024-byte alignment
+  unsigned char* gbase = um_raw + (base - raw_u32);
+  const uint32_t sB = base, sA = base + kUmBBytes;
+  unsigned char* ctl = gbase + kUmBBytes + 2 * kUmABytes;
+  uint64_t* mbar = reinterpret_cast<uint64_t*>(ctl);             // [2]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ctl + 16);
+  float* xch = reinterpret_cast<float*>(ctl + 64);               // [2 halves][128 tokens][min, max]
+
+  const int h = blockIdx.y, kind = blockIdx.z;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int n_tiles_all = (T + kUmTile - 1) / kUmTile;
+  const int my_tiles = n_tiles_all > (int)blockIdx.x ? (n_tiles_all - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+  if (my_tiles == 0) return;  // before any TMEM allocation
+  const __nv_bfloat16* src = (const __nv_bfloat16*)(kind ? a.v : a.k);
+
+  auto load_tile = [&](int tile, uint32_t abuf) {  // all threads: 2048 chunks of 16 B
+    const int t0 = tile * kUmTile;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int id = tid + kUmThreads * i;
+      const int r = id >> 4, j = id & 15;
+      const int tok = t0 + r;
+      const bool ok = tok < T;
+      const __nv_bfloat16* g = src + ((size_t)(ok ? tok : 0) * a.hkv + h) * kD + 8 * j;
+      um_cp_async16(abuf + (uint32_t)(j >> 3) * kUmRegion + um_swz((uint32_t)r, (uint32_t)(j & 7) * 16u), g,
+                    ok ? 16u : 0u);
+    }
+    cp_async_commit();
+  };
+
+  // first tile's loads go out before the R staging
+  load_tile(blockIdx.x, sA);
+
+  // R = U H P_br / sqrt(128), split in three bf16 parts, into B (row n = output channel, K = input channel).
+  // A warp takes rows c = warp + 8 i; the loads of eight rows go out together.
+  {
+    const float* U = (kind ? a.u_v : a.u_k) + (size_t)h * kD * kD;
+    const int b = rev5(lane);
+#pragma unroll 1
+    for (int c0 = warp; c0 < kD; c0 += 8 * kUmWarps) {
+      float y[8][4];
+#pragma unroll
+      for (int r = 0; r < 8; ++r)
+#pragma unroll
+        for (int aa = 0; aa < 4; ++aa) y[r][aa] = __ldg(U + (size_t)(c0 + r * kUmWarps) * kD + lane + 32 * aa);
+#pragma unroll
+      for (int r = 0; r < 8; ++r) {
+        const int c = c0 + r * kUmWarps;
+        wht128_warp(y[r], lane);
+        const uint32_t kb = (uint32_t)c >> 6, cb = ((uint32_t)c & 63u) * 2u;
+#pragma unroll
+        for (int aa = 0; aa < 4; ++aa) {
+          const uint32_t n = (uint32_t)(4 * b + rev2(aa));  // rotated channel of this value
+          const float u = y[r][aa] * kInvSqrtD;
+          const __nv_bfloat16 p0 = __float2bfloat16_rn(u);
+          const float r1 = u - __bfloat162float(p0);
+          const __nv_bfloat16 p1 = __float2bfloat16_rn(r1);
+          const __nv_bfloat16 p2 = __float2bfloat16_rn(r1 - __bfloat162float(p1));
+          const uint32_t off = kb * kUmRegion + um_swz(n, cb);
+          *reinterpret_cast<__nv_bfloat16*>(gbase + 0 * 2 * kUmRegion + off) = p0;
+          *reinterpret_cast<__nv_bfloat16*>(gbase + 1 * 2 * kUmRegion + off) = p1;
+          *reinterpret_cast<__nv_bfloat16*>(gbase + 2 * 2 * kUmRegion + off) = p2;
+        }
+      }
+    }
+  }
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(smem_u32(tmem_slot)),
+                 "r"(kUmTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::: "memory");
+  }
+  if (tid == 0) {
+    mbar_init(&mbar[0], 1);
+    mbar_init(&mbar[1], 1);
+    fence_mbar_init();
+  }
+  um_fence_proxy_async();  // R was written by ordinary stores; the MMA reads it through the async proxy
+  um_fence_before();
+  __syncthreads();
+  um_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  bool alive = true;
+
+  auto issue_mma = [&](int i) {  // tile i of this CTA, from A buffer i & 1 into TMEM buffer i & 1
+    const uint32_t u = (uint32_t)i & 1u;
+    const uint32_t abuf = sA + u * kUmABytes;
+    const uint32_t dcol = tmem + u * 128u;
+    int step = 0;
+#pragma unroll
+    for (int pt = 0; pt < 3; ++pt)
+#pragma unroll
+      for (int kb = 0; kb < 2; ++kb)
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks) {
+          const uint64_t ad = um_desc(abuf + (uint32_t)kb * kUmRegion + (uint32_t)ks * 32u);
+          const uint64_t bd = um_desc(sB + (uint32_t)(2 * pt + kb) * kUmRegion + (uint32_t)ks * 32u);
+          um_mma(dcol, ad, bd, step > 0 ? 1u : 0u);
+          ++step;
+        }
+    um_commit(&mbar[u]);
+  };
+
+  // tile 0: wait for its loads, then the MMAs
+  cp_async_wait_all();
+  um_fence_proxy_async();
+  __syncthreads();
+  if (tid == 0) {
+    um_fence_after();
+    issue_mma(0);
+  }
+  if (my_tiles > 1) load_tile(blockIdx.x + gridDim.x, sA + kUmABytes);
+
+  const int q = warp & 3, half = warp >> 2;
+  for (int i = 0; i < my_tiles; ++i) {
+    const uint32_t u = (uint32_t)i & 1u;
+    // this thread's token and its destination, fetched before the accumulator wait
+    const int tile = blockIdx.x + i * gridDim.x;
+    const int tok = tile * kUmTile + 32 * q + lane;
+    int slot = -1, p = -1;
+    if (tok < T) {
+      slot = a.seq_slot[tok];
+      p = a.pos[tok];
+    }
+    const bool slot_ok = slot >= 0 && slot < a.num_slots;
+    const int len = slot_ok ? a.slot_lens[slot] : 0;
+    const bool pos_ok = slot_ok && p >= 0 && (p >> 4) < a.mbps && p < len;
+    const int blk = pos_ok ? a.block_table[(size_t)slot * a.mbps + (p >> 4)] : -1;
+    // MMAs of tile i+1 (its A buffer is loaded; its TMEM buffer was drained by the epilogue of tile i-1)
+    if (i + 1 < my_tiles) {
+      cp_async_wait_all();
+      um_fence_proxy_async();
+      um_fence_before();
+      __syncthreads();
+      if (tid == 0 && alive) {
+        um_fence_after();
+        issue_mma(i + 1);
+      }
+    }
+    // tile i: wait for its accumulators (after a timeout nothing more is waited for)
+    if (alive && !mbar_wait_bounded(&mbar[u], ((uint32_t)i >> 1) & 1u)) {
+      if (lane == 0) raise_flag(a.status, OKV_DEV_TIMEOUT);
+      alive = false;
+    }
+    alive = __syncthreads_and(alive);
+    um_fence_after();
+    // A buffer u is free again (every thread passed the wait above): tile i+2's loads
+    if (i + 2 < my_tiles) load_tile(blockIdx.x + (i + 2) * gridDim.x, sA + u * kUmABytes);
+    float v[64];
+    {
+      float w32[32];
+      const uint32_t taddr = tmem + ((uint32_t)(32 * q) << 16) + u * 128u + (uint32_t)(64 * half);
+      um_ld32(taddr, w32);
+#pragma unroll
+      for (int j = 0; j < 32; ++j) v[j] = w32[j];
+      um_ld32(taddr + 32u, w32);
+#pragma unroll
+      for (int j = 0; j < 32; ++j) v[32 + j] = w32[j];
+      um_wait_ld();
+    }
+    float mn = v[0], mx = v[0];
+#pragma unroll
+    for (int j = 1; j < 64; ++j) {
+      mn = fminf(mn, v[j]);
+      mx = fmaxf(mx, v[j]);
+    }
+    const int row = 32 * q + lane;
+    xch[(half * kUmTile + row) * 2 + 0] = mn;
+    xch[(half * kUmTile + row) * 2 + 1] = mx;
+    um_fence_before();
+    __syncthreads();
+    mn = fminf(mn, xch[((half ^ 1) * kUmTile + row) * 2 + 0]);
+    mx = fmaxf(mx, xch[((half ^ 1) * kUmTile + row) * 2 + 1]);
+    const bool live = alive && tok < T;
+    if (live) {
+      if (half == 0) {
+        if (!slot_ok) raise_flag(a.status, OKV_DEV_BAD_SLOT);
+        else if (!pos_ok) raise_flag(a.status, OKV_DEV_BAD_POS);
+        else if (blk < 0 || blk >= a.num_blocks) raise_flag(a.status, OKV_DEV_BAD_BLOCK);
+      }
+      if (blk >= 0 && blk < a.num_blocks) {
+        const float s32 = __fdiv_rn(__fsub_rn(mx, mn), 3.0f);
+        const __half s16 = fp16_sat(s32);
+        const __half m16 = fp16_sat(mn);
+        const float sc = __half2float(s16);
+        const float m = __half2float(m16);
+        uint32_t w[4] = {0u, 0u, 0u, 0u};  // 16 code bytes: channels 64 half .. 64 half + 63
+        if (sc != 0.0f) {
+          const CodeThresholds th = code_thresholds(sc);
+#pragma unroll
+          for (int j = 0; j < 64; ++j) w[j >> 4] |= int2_code(__fsub_rn(v[j], m), th) << (2 * (j & 15));
+        }
+        uint8_t* bp = a.pages + ((size_t)blk * a.hkv + h) * kBlockHeadBytes;
+        const int sl = p & 15;
+        if (kind == 0) {
+          *reinterpret_cast<uint4*>(bp + kKcOff + sl * 32 + 16 * half) = make_uint4(w[0], w[1], w[2], w[3]);
+        } else {
+#pragma unroll
+          for (int bb = 0; bb < 16; ++bb) bp[v_code_offset(sl, 16 * half + bb)] = (uint8_t)(w[bb >> 2] >> (8 * (bb & 3)));
+        }
+        if (half == 0)
+          *reinterpret_cast<uint32_t*>(bp + (kind ? kVsmOff : kKsmOff) + 4 * sl) =
+              (uint32_t)__half_as_ushort(s16) | ((uint32_t)__half_as_ushort(m16) << 16);
+        if (p >= len - kWin) {
+          __half* wr = a.ring + ((((size_t)slot * a.hkv + h) * 2 + kind) * kWin + (p % kWin)) * kD + 64 * half;
+#pragma unroll
+          for (int j = 0; j < 64; j += 8) {
+            __half2 h0 = __floats2half2_rn(0.f, 0.f), h1 = h0, h2 = h0, h3 = h0;
+            h0 = __halves2half2(fp16_sat(v[j + 0]), fp16_sat(v[j + 1]));
+            h1 = __halves2half2(fp16_sat(v[j + 2]), fp16_sat(v[j + 3]));
+            h2 = __halves2half2(fp16_sat(v[j + 4]), fp16_sat(v[j + 5]));
+            h3 = __halves2half2(fp16_sat(v[j + 6]), fp16_sat(v[j + 7]));
+            uint4 q4;
+            q4.x = *reinterpret_cast<uint32_t*>(&h0);
+            q4.y = *reinterpret_cast<uint32_t*>(&h1);
+            q4.z = *reinterpret_cast<uint32_t*>(&h2);
+            q4.w = *reinterpret_cast<uint32_t*>(&h3);
+            *reinterpret_cast<uint4*>(wr + j) = q4;
+          }
+        }
+        if (a.rotated_out != nullptr) {
+          float* ro = a.rotated_out + (((size_t)tok * 2 + kind) * a.hkv + h) * kD + 64 * half;
+#pragma unroll
+          for (int j = 0; j < 64; j += 4) *reinterpret_cast<float4*>(ro + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+        }
+      }
+    }
+    __syncthreads();  // the exchange slots are reused by the next tile
+  }
+  // free TMEM: every thread's loads completed (wait::ld) before the barrier above
+  um_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    um_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tmem), "r"(kUmTmemCols) : "memory");
+  }
+}
+
 }  // namespace
 
 okv_status launch_append(const okv_cache_desc* d, const void* k, const void* v, int T,
@@ -387,6 +716,17 @@ okv_status launch_append(const okv_cache_desc* d, const void* k, const void* v, 
   a.num_blocks = d->num_blocks;
   a.num_slots = d->num_seq_slots;
   a.mbps = d->max_blocks_per_seq;
+  const bool rows16 = (((uintptr_t)k | (uintptr_t)v) & 15u) == 0;  // the tile loads copy 16-byte chunks
+  if (!(flags & OKV_PRE_ROTATED) && T >= kTcMinTokens && rows16) {
+    cudaError_t e = cudaFuncSetAttribute(append_umma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kUmSmem);
+    if (e != cudaSuccess) return fail(OKV_ERR_CUDA, "append smem attribute: %s", cudaGetErrorString(e));
+    const int pairs = 2 * d->num_kv_heads;
+    const int tiles = (T + kUmTile - 1) / kUmTile;
+    const int per_pair = std::max(1, std::min(tiles, device_sm_count() / pairs));
+    dim3 grid(per_pair, d->num_kv_heads, 2);
+    append_umma_kernel<<<grid, kUmThreads, kUmSmem, s>>>(a, T);
+    return check_launch("append (tcgen05)");
+  }
   if (!(flags & OKV_PRE_ROTATED) && T >= kTcMinTokens) {
     // set on every call: the attribute belongs to the current device's context
     cudaError_t e = cudaFuncSetAttribute(append_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kTcSmem);

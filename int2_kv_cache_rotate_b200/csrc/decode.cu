@@ -585,42 +585,6 @@ __global__ void __launch_bounds__(kHW * 32, (G <= 4) ? 2 : 1) decode_heads_kerne
     __syncthreads();  // the previous entry's window scratch / merge buffers (on the ring) are free again
     if (!slot_ok && threadIdx.x == 0) raise_flag(a.status, OKV_DEV_BAD_SLOT);
 
-    // ---------------- per-warp state for (b, head) ----------------
-    MmaWarpState<G> st;
-    int acci[NT][8][4];
-    st.acc = accs + threadIdx.x * HCfg<G>::acc_stride;
-    uint32_t qb[NT][8];
-    float ah[NT], bh[NT], hbias[NT];
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-      st.m[nt] = -INFINITY;
-      st.l[nt] = 0.f;
-      st.msum[nt] = 0.f;
-#pragma unroll
-      for (int i = 0; i < 16; ++i) st.acc[16 * nt + i] = 0.f;
-#pragma unroll
-      for (int mt = 0; mt < 8; ++mt)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) acci[nt][mt][j] = 0;
-      const int hcol = 4 * nt + (g >> 1);  // head of this lane's B column
-      if (hcol < G) {
-        const uint4* src = reinterpret_cast<const uint4*>(a.qlimb + ((bh0 + hcol) * 2 + (g & 1)) * kD + 32 * t);
-        const uint4 x0 = src[0], x1 = src[1];
-        qb[nt][0] = x0.x; qb[nt][1] = x0.y; qb[nt][2] = x0.z; qb[nt][3] = x0.w;
-        qb[nt][4] = x1.x; qb[nt][5] = x1.y; qb[nt][6] = x1.z; qb[nt][7] = x1.w;
-      } else {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) qb[nt][i] = 0u;
-      }
-      const int hs = 4 * nt + t;  // head of this lane's score columns
-      const bool ok = hs < G;
-      ah[nt] = ok ? a.qscale[(bh0 + hs) * 4 + 0] : 0.f;
-      bh[nt] = ok ? a.qscale[(bh0 + hs) * 4 + 1] : 0.f;
-      hbias[nt] = ok ? 0.f : -INFINITY;
-    }
-    float s_cap = 0.f, lam = 0.f, inv = 0.f;
-    int since_flush = 0;
-
     // ---------------- INT2 blocks through the ring ----------------
     const int p0 = max(l0, us.win_cost) - us.win_cost;
     const int p1 = l1 - us.win_cost;
@@ -687,6 +651,43 @@ __global__ void __launch_bounds__(kHW * 32, (G <= 4) ? 2 : 1) decode_heads_kerne
     bool prod_ok = true;
     if (warp == 0)
       for (int j = 0; j < min(kHStages - 1, nst) && prod_ok; ++j) prod_ok = issue(j);
+
+    // ---------------- per-warp state for (b, head), loaded while the first stages are in flight ----------------
+    MmaWarpState<G> st;
+    int acci[NT][8][4];
+    st.acc = accs + threadIdx.x * HCfg<G>::acc_stride;
+    uint32_t qb[NT][8];
+    float ah[NT], bh[NT], hbias[NT];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      st.m[nt] = -INFINITY;
+      st.l[nt] = 0.f;
+      st.msum[nt] = 0.f;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) st.acc[16 * nt + i] = 0.f;
+#pragma unroll
+      for (int mt = 0; mt < 8; ++mt)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acci[nt][mt][j] = 0;
+      const int hcol = 4 * nt + (g >> 1);  // head of this lane's B column
+      if (hcol < G) {
+        const uint4* src = reinterpret_cast<const uint4*>(a.qlimb + ((bh0 + hcol) * 2 + (g & 1)) * kD + 32 * t);
+        const uint4 x0 = src[0], x1 = src[1];
+        qb[nt][0] = x0.x; qb[nt][1] = x0.y; qb[nt][2] = x0.z; qb[nt][3] = x0.w;
+        qb[nt][4] = x1.x; qb[nt][5] = x1.y; qb[nt][6] = x1.z; qb[nt][7] = x1.w;
+      } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) qb[nt][i] = 0u;
+      }
+      const int hs = 4 * nt + t;  // head of this lane's score columns
+      const bool ok = hs < G;
+      ah[nt] = ok ? a.qscale[(bh0 + hs) * 4 + 0] : 0.f;
+      bh[nt] = ok ? a.qscale[(bh0 + hs) * 4 + 1] : 0.f;
+      hbias[nt] = ok ? 0.f : -INFINITY;
+    }
+    float s_cap = 0.f, lam = 0.f, inv = 0.f;
+    int since_flush = 0;
+
 
     int done = 0;
     uint32_t cs = it % kHStages, cph = (it / kHStages) & 1u;  // consumer stage and phase parity

@@ -82,22 +82,21 @@ __device__ __forceinline__ __half fp16_sat(float x) {
 }
 
 // The quantiser's code decision without a division.  With x = fl(z - m)
-// and s > 0, the code clamp(rint_even(fl(x / s)), 0, 3) is the number of
-// thresholds x passes, because round-to-nearest-even puts the decision points
-// exactly at
-//   c >= 1  <=>  fl(x / s) > 0.5  <=>  x / s > 0.5 + 2^-25   (0.5 is the even neighbour)
-//   c >= 2  <=>  fl(x / s) >= 1.5 <=>  x / s >= 1.5 - 2^-24  (1.5 is the even neighbour)
-//   c >= 3  <=>  fl(x / s) > 2.5  <=>  x / s > 2.5 + 2^-23  (2.5 is the even neighbour)
-// (the half-ulp of fp32 in [0.5, 1), [1, 2) and [2, 4)).  Multiplied through
-// by s: x - 0.5s > s 2^-25, x - 1.5s >= -s 2^-24, x - 2.5s > s 2^-23.  k s is
-// exact for k in {0.5, 1.5, 2.5} (s has 11 significant bits), s 2^-n is
-// exact (s >= 2^-24), and each difference x - k s is exact whenever x lies
-// within a factor of two of k s (Sterbenz); when it does not, |x - k s| >=
-// k s / 2, far from the tiny threshold, so the rounded difference has the
-// same side.  Every code therefore equals the division's, bit for bit.
+// and s > 0 an fp16 value, the code clamp(rint_even(fl(x / s)), 0, 3) is
+//   [x > s/2] + [x >= 3s/2] + [x > 5s/2]
+// exactly.  Round-to-nearest-even puts the decision points of fl(x / s) at
+//   c >= 1  <=>  x / s > 1/2 + 2^-25   (a tie at 1/2 goes to the even 1/2, rint 0)
+//   c >= 2  <=>  x / s >= 3/2 - 2^-24  (a tie goes to the even 3/2, rint 2)
+//   c >= 3  <=>  x / s > 5/2 + 2^-23   (a tie goes to the even 5/2, rint 2)
+// (half-ulps of fp32 in [1/2, 1), [1, 2), [2, 4)).  Times s, each bound is
+// k s (exact: s has 11 significant bits) moved by less than one ulp of k s
+// and by at least a third of one: s 2^-25 = (s/2) 2^-24, s 2^-24 =
+// (3s/2) (2/3) 2^-24, s 2^-23 = (5s/2) (4/5) 2^-24.  So no fp32 number lies
+// between k s and the bound, and comparing x with k s itself decides the
+// same way (3s/2 is never a power of two, so its predecessor is a full ulp
+// below).  Every code therefore equals the division's, bit for bit.
 struct CodeThresholds {
-  float h1, h2, h3;  // 0.5 s, 1.5 s, 2.5 s
-  float e1, e2, e3;  // s 2^-25, -s 2^-24, s 2^-23
+  float h1, h2, h3;  // s/2, 3s/2, 5s/2 (exact)
 };
 
 __device__ __forceinline__ CodeThresholds code_thresholds(float s) {
@@ -105,16 +104,12 @@ __device__ __forceinline__ CodeThresholds code_thresholds(float s) {
   t.h1 = 0.5f * s;
   t.h2 = 1.5f * s;
   t.h3 = 2.5f * s;
-  t.e1 = s * 0x1p-25f;
-  t.e2 = -s * 0x1p-24f;
-  t.e3 = s * 0x1p-23f;
   return t;
 }
 
 // code of x = fl(z - m); only for s > 0 (s = 0 gives code 0 by definition)
 __device__ __forceinline__ uint32_t int2_code(float x, const CodeThresholds& t) {
-  return (uint32_t)(__fsub_rn(x, t.h1) > t.e1) + (uint32_t)(__fsub_rn(x, t.h2) >= t.e2) +
-         (uint32_t)(__fsub_rn(x, t.h3) > t.e3);
+  return (uint32_t)(x > t.h1) + (uint32_t)(x >= t.h2) + (uint32_t)(x > t.h3);
 }
 
 // INT2 group quantiser over the 128 values of a warp (y[a] = value at

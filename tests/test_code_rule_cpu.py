@@ -1,5 +1,6 @@
-"""The kernels decide INT2 codes by three threshold comparisons instead of
-the fp32 division of the quantiser's definition.  This checks, in numpy fp32,
+"""The kernels decide INT2 codes by three comparisons with the exact
+midpoints s/2, 3s/2, 5s/2 instead of the fp32 division of the quantiser's
+definition.  This checks, in numpy fp32,
 that the comparison rule gives exactly the oracle's codes, on groups built to
 sit on the rounding midpoints (ties to even included) and on ordinary data.
 The GPU-side counterpart runs the same groups through the kernels."""
@@ -11,14 +12,14 @@ from tests import gpu_helpers as H
 
 
 def _rule(z, s16, m16):
-    """x = fl(z - m); c = [x - s/2 > s 2^-25] + [x - 3s/2 >= -s 2^-24] + [x - 5s/2 > s 2^-23]."""
+    """x = fl(z - m); c = [x > s/2] + [x >= 3s/2] + [x > 5s/2] (all products exact)."""
     s = s16.astype(np.float32)[:, None]
     m = m16.astype(np.float32)[:, None]
     x = (z - m).astype(np.float32)
     f = np.float32
-    c = ((x - f(0.5) * s) > s * f(2.0 ** -25)).astype(np.uint8)
-    c += ((x - f(1.5) * s) >= -s * f(2.0 ** -24)).astype(np.uint8)
-    c += ((x - f(2.5) * s) > s * f(2.0 ** -23)).astype(np.uint8)
+    c = (x > f(0.5) * s).astype(np.uint8)
+    c += (x >= f(1.5) * s).astype(np.uint8)
+    c += (x > f(2.5) * s).astype(np.uint8)
     return np.where(s == 0, 0, c).astype(np.uint8)
 
 

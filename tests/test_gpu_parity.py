@@ -144,12 +144,13 @@ def test_dequantize_bit_exact_and_original_basis():
                 assert np.abs(orig[b, h, :n] - back).max() <= 1e-5 * np.abs(back).max()
 
 
-@pytest.mark.parametrize("lens", [
-    [700, 45],   # 745 tokens: tensor-core kernel, 3 CTAs, ragged last round
-    [60, 45],    # 105 tokens: CUDA-core kernel
-    [128],       # exactly the tensor-core threshold
+@pytest.mark.parametrize("lens,misalign", [
+    ([700, 45], False),   # 745 tokens: tcgen05 kernel, 6 tiles, ragged last tile
+    ([60, 45], False),    # 105 tokens: CUDA-core kernel
+    ([128], False),       # exactly the tensor-core threshold: one tile
+    ([700, 45], True),    # K/V not 16-byte aligned: the mma.sync tensor-core kernel
 ])
-def test_append_fused_rotation_and_codes(lens):
+def test_append_fused_rotation_and_codes(lens, misalign):
     okv = _okv()
     seed, hq, hkv = 3, 8, 2
     lay = H.Layout(seed, lens)
@@ -161,8 +162,12 @@ def test_append_fused_rotation_and_codes(lens):
     slots, pos = lay.flat()
     kk, vv = np.concatenate(k), np.concatenate(v)
     rot = torch.zeros((len(slots), 2, hkv, 128), dtype=torch.float32, device="cuda")
-    okv.append_quantize(gc, _t(kk, torch.bfloat16), _t(vv, torch.bfloat16), _t(slots), _t(pos), _t(lay.table),
-                        _t(np.array(lens, np.int32)), rotated_out=rot)
+    kd, vd = _t(kk, torch.bfloat16), _t(vv, torch.bfloat16)
+    if misalign:  # same values at an address 4 bytes past a 16-byte boundary
+        kd = torch.cat([torch.zeros(2, dtype=torch.bfloat16, device="cuda"), kd.flatten()])[2:].view(kd.shape)
+        vd = torch.cat([torch.zeros(2, dtype=torch.bfloat16, device="cuda"), vd.flatten()])[2:].view(vd.shape)
+        assert kd.data_ptr() % 16 == 4 and vd.data_ptr() % 16 == 4
+    okv.append_quantize(gc, kd, vd, _t(slots), _t(pos), _t(lay.table), _t(np.array(lens, np.int32)), rotated_out=rot)
     rot = rot.cpu().numpy()
     pages = gc.pages.cpu().numpy()
     off = 0
