@@ -373,23 +373,30 @@ __global__ void __launch_bounds__(kTcWarps * 32, 2) append_tc_kernel(AppendArgs 
 // the K-major 128-byte-swizzled layout the MMA descriptors describe: part pt,
 // K-block kb (64 channels) is a 16 KB region of 128 rows x 128 B; element
 // (n, c) sits in row n, 16-byte chunk ((c % 64) / 8) ^ (n % 8).  A is one
-// 128-token tile of k for this KV head, two K-blocks of the same layout,
-// loaded by zero-filling async copies (rows past T read as zeros).
-// One thread issues 24 MMAs (M = N = 128, K = 16 each) per tile into a
-// 128-column TMEM buffer; two buffers let the MMAs of tile i+1 run during the
-// epilogue of tile i.  Epilogue: warp w reads TMEM lanes 32 (w % 4) .. +31
-// (tokens) and columns 64 (w / 4) .. +63, so each thread holds half a token's
-// rotated vector; the two halves meet in shared memory for min/max.
+// 128-token tile of k for this KV head in the same layout (two K-blocks).
+//
+// Roles (warp-specialised):
+//   warp 8      producer: zero-filling async copies of A tiles into a 3-stage
+//               ring (one copy group per tile); once a tile's group is in,
+//               every lane fences it for the async proxy and one lane issues
+//               the 24 MMAs (M = N = 128, K = 16) into TMEM buffer i & 1,
+//               committed to mma_done[i & 1];
+//   warps 0-3   epilogue of even tiles, warps 4-7 of odd tiles: warp w reads
+//               TMEM lanes 32 (w % 4) .. +31, one token per thread, all 128
+//               columns; it frees the TMEM buffer (tmem_free) as soon as the
+//               values are in registers, then quantises and stores.
 // Every mbarrier wait is bounded; TMEM is freed on every path.
 // ---------------------------------------------------------------------------
-constexpr int kUmWarps = 8;
-constexpr int kUmThreads = 32 * kUmWarps;
+constexpr int kUmEpiWarps = 8;
+constexpr int kUmProducer = kUmEpiWarps;             // warp index of the producer
+constexpr int kUmThreads = 32 * (kUmEpiWarps + 1);
 constexpr int kUmTile = 128;
+constexpr int kUmStages = 3;
 constexpr uint32_t kUmRegion = 16384;                 // 128 rows x 128 B
 constexpr uint32_t kUmBBytes = 6 * kUmRegion;         // 3 parts x 2 K-blocks
 constexpr uint32_t kUmABytes = 2 * kUmRegion;         // one tile, 2 K-blocks
-constexpr uint32_t kUmCtlBytes = 64 + 2 * kUmTile * 2 * 4;  // barriers, TMEM base, min/max exchange
-constexpr size_t kUmSmem = 1024 + kUmBBytes + 2 * kUmABytes + kUmCtlBytes;
+constexpr uint32_t kUmCtlBytes = 64;                  // barriers and the TMEM base
+constexpr size_t kUmSmem = 1024 + kUmBBytes + kUmStages * kUmABytes + kUmCtlBytes;
 constexpr uint32_t kUmTmemCols = 256;
 // instruction descriptor: D f32, A and B bf16, both K-major, N = 128, M = 128
 constexpr uint32_t kUmIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((128u >> 3) << 17) | ((128u >> 4) << 24);
@@ -412,7 +419,6 @@ __device__ __forceinline__ uint64_t um_desc(uint32_t saddr) {
 __device__ __forceinline__ void um_cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
 }
-
 __device__ __forceinline__ void um_fence_proxy_async() {
   asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
 }
@@ -436,7 +442,7 @@ __device__ __forceinline__ void um_commit(uint64_t* bar) {
                : "memory");
 }
 
-__device__ __forceinline__ void um_ld32(uint32_t taddr, float (&v)[32]) {
+__device__ __forceinline__ void um_ld32(uint32_t taddr, float* v) {
   uint32_t r[32];
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
@@ -458,23 +464,26 @@ __global__ void __launch_bounds__(kUmThreads, 1) append_umma_kernel(AppendArgs a
   const uint32_t base = (raw_u32 + 1023u) & ~1023u;  // swizzle atoms need 1024-byte alignment
   unsigned char* gbase = um_raw + (base - raw_u32);
   const uint32_t sB = base, sA = base + kUmBBytes;
-  unsigned char* ctl = gbase + kUmBBytes + 2 * kUmABytes;
-  uint64_t* mbar = reinterpret_cast<uint64_t*>(ctl);             // [2]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ctl + 16);
-  float* xch = reinterpret_cast<float*>(ctl + 64);               // [2 halves][128 tokens][min, max]
+  unsigned char* ctl = gbase + kUmBBytes + kUmStages * kUmABytes;
+  uint64_t* mma_done = reinterpret_cast<uint64_t*>(ctl);  // [2], one commit
+  uint64_t* tmem_free = mma_done + 2;                    // [2], 128 arrivals (an epilogue warpgroup)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tmem_free + 2);
 
   const int h = blockIdx.y, kind = blockIdx.z;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int n_tiles_all = (T + kUmTile - 1) / kUmTile;
-  const int my_tiles = n_tiles_all > (int)blockIdx.x ? (n_tiles_all - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
-  if (my_tiles == 0) return;  // before any TMEM allocation
+  const int n = n_tiles_all > (int)blockIdx.x ? (n_tiles_all - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+  if (n == 0) return;  // before any TMEM allocation
   const __nv_bfloat16* src = (const __nv_bfloat16*)(kind ? a.v : a.k);
+  auto tile_of = [&](int i) { return (int)blockIdx.x + i * (int)gridDim.x; };
 
-  auto load_tile = [&](int tile, uint32_t abuf) {  // all threads: 2048 chunks of 16 B
-    const int t0 = tile * kUmTile;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int id = tid + kUmThreads * i;
+  // producer lane: its 64 chunks of tile i into stage i % 3, as one copy group
+  auto load_tile = [&](int i) {
+    const int t0 = tile_of(i) * kUmTile;
+    const uint32_t abuf = sA + (uint32_t)(i % kUmStages) * kUmABytes;
+#pragma unroll 8
+    for (int k = 0; k < 64; ++k) {
+      const int id = lane + 32 * k;
       const int r = id >> 4, j = id & 15;
       const int tok = t0 + r;
       const bool ok = tok < T;
@@ -485,41 +494,62 @@ __global__ void __launch_bounds__(kUmThreads, 1) append_umma_kernel(AppendArgs a
     cp_async_commit();
   };
 
-  // first tile's loads go out before the R staging
-  load_tile(blockIdx.x, sA);
-
-  // R = U H P_br / sqrt(128), split in three bf16 parts, into B (row n = output channel, K = input channel).
-  // A warp takes rows c = warp + 8 i; the loads of eight rows go out together.
-  {
+  if (tid == 0) {
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&mma_done[i], 1);
+      mbar_init(&tmem_free[i], 128);
+    }
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (warp == kUmProducer) {
+    // the first tiles' loads go out while the other warps stage R
+    load_tile(0);
+    if (n > 1) load_tile(1);
+  } else {
+    // R = U H P_br / sqrt(128), split in three bf16 parts, into B (row n = output channel,
+    // K = input channel).  Warp w takes input channels 16w .. 16w + 15 in two batches of eight:
+    // after the butterflies a lane holds its four output channels for all eight input
+    // channels, which is one 16-byte chunk of each of those four B rows.
     const float* U = (kind ? a.u_v : a.u_k) + (size_t)h * kD * kD;
     const int b = rev5(lane);
 #pragma unroll 1
-    for (int c0 = warp; c0 < kD; c0 += 8 * kUmWarps) {
+    for (int c0 = 16 * warp; c0 < 16 * warp + 16; c0 += 8) {
       float y[8][4];
 #pragma unroll
       for (int r = 0; r < 8; ++r)
 #pragma unroll
-        for (int aa = 0; aa < 4; ++aa) y[r][aa] = __ldg(U + (size_t)(c0 + r * kUmWarps) * kD + lane + 32 * aa);
+        for (int aa = 0; aa < 4; ++aa) y[r][aa] = __ldg(U + (size_t)(c0 + r) * kD + lane + 32 * aa);
 #pragma unroll
       for (int r = 0; r < 8; ++r) {
-        const int c = c0 + r * kUmWarps;
         wht128_warp(y[r], lane);
-        const uint32_t kb = (uint32_t)c >> 6, cb = ((uint32_t)c & 63u) * 2u;
 #pragma unroll
-        for (int aa = 0; aa < 4; ++aa) {
-          const uint32_t n = (uint32_t)(4 * b + rev2(aa));  // rotated channel of this value
-          const float u = y[r][aa] * kInvSqrtD;
-          const __nv_bfloat16 p0 = __float2bfloat16_rn(u);
-          const float r1 = u - __bfloat162float(p0);
-          const __nv_bfloat16 p1 = __float2bfloat16_rn(r1);
-          const __nv_bfloat16 p2 = __float2bfloat16_rn(r1 - __bfloat162float(p1));
-          const uint32_t off = kb * kUmRegion + um_swz(n, cb);
-          *reinterpret_cast<__nv_bfloat16*>(gbase + 0 * 2 * kUmRegion + off) = p0;
-          *reinterpret_cast<__nv_bfloat16*>(gbase + 1 * 2 * kUmRegion + off) = p1;
-          *reinterpret_cast<__nv_bfloat16*>(gbase + 2 * 2 * kUmRegion + off) = p2;
+        for (int aa = 0; aa < 4; ++aa) y[r][aa] *= kInvSqrtD;
+      }
+      const uint32_t kb = (uint32_t)c0 >> 6, cb = ((uint32_t)c0 & 63u) * 2u;
+#pragma unroll
+      for (int aa = 0; aa < 4; ++aa) {
+        const uint32_t nn = (uint32_t)(4 * b + rev2(aa));  // rotated channel of these values
+        uint32_t pk[3][4];
+#pragma unroll
+        for (int r = 0; r < 8; r += 2) {
+          float u0 = y[r][aa], u1 = y[r + 1][aa];
+#pragma unroll
+          for (int pt = 0; pt < 3; ++pt) {
+            const __nv_bfloat162 pp = __floats2bfloat162_rn(u0, u1);
+            pk[pt][r >> 1] = *reinterpret_cast<const uint32_t*>(&pp);
+            u0 -= __low2float(pp);
+            u1 -= __high2float(pp);
+          }
         }
+        const uint32_t off = kb * kUmRegion + um_swz(nn, cb);
+#pragma unroll
+        for (int pt = 0; pt < 3; ++pt)
+          *reinterpret_cast<uint4*>(gbase + (uint32_t)pt * 2 * kUmRegion + off) =
+              make_uint4(pk[pt][0], pk[pt][1], pk[pt][2], pk[pt][3]);
       }
     }
+    um_fence_proxy_async();  // R was written by ordinary stores; the MMA reads it through the async proxy
   }
   if (warp == 0) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(smem_u32(tmem_slot)),
@@ -527,164 +557,157 @@ __global__ void __launch_bounds__(kUmThreads, 1) append_umma_kernel(AppendArgs a
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::: "memory");
   }
-  if (tid == 0) {
-    mbar_init(&mbar[0], 1);
-    mbar_init(&mbar[1], 1);
-    fence_mbar_init();
-  }
-  um_fence_proxy_async();  // R was written by ordinary stores; the MMA reads it through the async proxy
   um_fence_before();
   __syncthreads();
   um_fence_after();
   const uint32_t tmem = *tmem_slot;
   bool alive = true;
 
-  auto issue_mma = [&](int i) {  // tile i of this CTA, from A buffer i & 1 into TMEM buffer i & 1
-    const uint32_t u = (uint32_t)i & 1u;
-    const uint32_t abuf = sA + u * kUmABytes;
-    const uint32_t dcol = tmem + u * 128u;
-    int step = 0;
+  if (warp == kUmProducer) {
+    for (int i = 0; i < n; ++i) {
+      // MMAs of tile i: its copy group is in (only tile i + 1's group can be younger), and the
+      // epilogue of tile i - 2 has drained TMEM buffer i & 1
+      if (i + 1 < n) cp_async_wait_group<1>();
+      else cp_async_wait_group<0>();
+      um_fence_proxy_async();  // this lane's copies, made visible to the async proxy
+      __syncwarp();
+      if (lane == 0 && alive) {
+        const bool ok = i < 2 || mbar_wait_bounded(&tmem_free[i & 1], ((uint32_t)(i - 2) >> 1) & 1u);
+        if (ok) {
+          um_fence_after();
+          const uint32_t abuf = sA + (uint32_t)(i % kUmStages) * kUmABytes;
+          const uint32_t dcol = tmem + ((uint32_t)i & 1u) * 128u;
+          int step = 0;
 #pragma unroll
-    for (int pt = 0; pt < 3; ++pt)
+          for (int pt = 0; pt < 3; ++pt)
 #pragma unroll
-      for (int kb = 0; kb < 2; ++kb)
+            for (int kb = 0; kb < 2; ++kb)
 #pragma unroll
-        for (int ks = 0; ks < 4; ++ks) {
-          const uint64_t ad = um_desc(abuf + (uint32_t)kb * kUmRegion + (uint32_t)ks * 32u);
-          const uint64_t bd = um_desc(sB + (uint32_t)(2 * pt + kb) * kUmRegion + (uint32_t)ks * 32u);
-          um_mma(dcol, ad, bd, step > 0 ? 1u : 0u);
-          ++step;
-        }
-    um_commit(&mbar[u]);
-  };
-
-  // tile 0: wait for its loads, then the MMAs
-  cp_async_wait_all();
-  um_fence_proxy_async();
-  __syncthreads();
-  if (tid == 0) {
-    um_fence_after();
-    issue_mma(0);
-  }
-  if (my_tiles > 1) load_tile(blockIdx.x + gridDim.x, sA + kUmABytes);
-
-  const int q = warp & 3, half = warp >> 2;
-  for (int i = 0; i < my_tiles; ++i) {
-    const uint32_t u = (uint32_t)i & 1u;
-    // this thread's token and its destination, fetched before the accumulator wait
-    const int tile = blockIdx.x + i * gridDim.x;
-    const int tok = tile * kUmTile + 32 * q + lane;
-    int slot = -1, p = -1;
-    if (tok < T) {
-      slot = a.seq_slot[tok];
-      p = a.pos[tok];
-    }
-    const bool slot_ok = slot >= 0 && slot < a.num_slots;
-    const int len = slot_ok ? a.slot_lens[slot] : 0;
-    const bool pos_ok = slot_ok && p >= 0 && (p >> 4) < a.mbps && p < len;
-    const int blk = pos_ok ? a.block_table[(size_t)slot * a.mbps + (p >> 4)] : -1;
-    // MMAs of tile i+1 (its A buffer is loaded; its TMEM buffer was drained by the epilogue of tile i-1)
-    if (i + 1 < my_tiles) {
-      cp_async_wait_all();
-      um_fence_proxy_async();
-      um_fence_before();
-      __syncthreads();
-      if (tid == 0 && alive) {
-        um_fence_after();
-        issue_mma(i + 1);
-      }
-    }
-    // tile i: wait for its accumulators (after a timeout nothing more is waited for)
-    if (alive && !mbar_wait_bounded(&mbar[u], ((uint32_t)i >> 1) & 1u)) {
-      if (lane == 0) raise_flag(a.status, OKV_DEV_TIMEOUT);
-      alive = false;
-    }
-    alive = __syncthreads_and(alive);
-    um_fence_after();
-    // A buffer u is free again (every thread passed the wait above): tile i+2's loads
-    if (i + 2 < my_tiles) load_tile(blockIdx.x + (i + 2) * gridDim.x, sA + u * kUmABytes);
-    float v[64];
-    {
-      float w32[32];
-      const uint32_t taddr = tmem + ((uint32_t)(32 * q) << 16) + u * 128u + (uint32_t)(64 * half);
-      um_ld32(taddr, w32);
-#pragma unroll
-      for (int j = 0; j < 32; ++j) v[j] = w32[j];
-      um_ld32(taddr + 32u, w32);
-#pragma unroll
-      for (int j = 0; j < 32; ++j) v[32 + j] = w32[j];
-      um_wait_ld();
-    }
-    float mn = v[0], mx = v[0];
-#pragma unroll
-    for (int j = 1; j < 64; ++j) {
-      mn = fminf(mn, v[j]);
-      mx = fmaxf(mx, v[j]);
-    }
-    const int row = 32 * q + lane;
-    xch[(half * kUmTile + row) * 2 + 0] = mn;
-    xch[(half * kUmTile + row) * 2 + 1] = mx;
-    um_fence_before();
-    __syncthreads();
-    mn = fminf(mn, xch[((half ^ 1) * kUmTile + row) * 2 + 0]);
-    mx = fmaxf(mx, xch[((half ^ 1) * kUmTile + row) * 2 + 1]);
-    const bool live = alive && tok < T;
-    if (live) {
-      if (half == 0) {
-        if (!slot_ok) raise_flag(a.status, OKV_DEV_BAD_SLOT);
-        else if (!pos_ok) raise_flag(a.status, OKV_DEV_BAD_POS);
-        else if (blk < 0 || blk >= a.num_blocks) raise_flag(a.status, OKV_DEV_BAD_BLOCK);
-      }
-      if (blk >= 0 && blk < a.num_blocks) {
-        const float s32 = __fdiv_rn(__fsub_rn(mx, mn), 3.0f);
-        const __half s16 = fp16_sat(s32);
-        const __half m16 = fp16_sat(mn);
-        const float sc = __half2float(s16);
-        const float m = __half2float(m16);
-        uint32_t w[4] = {0u, 0u, 0u, 0u};  // 16 code bytes: channels 64 half .. 64 half + 63
-        if (sc != 0.0f) {
-          const CodeThresholds th = code_thresholds(sc);
-#pragma unroll
-          for (int j = 0; j < 64; ++j) w[j >> 4] |= int2_code(__fsub_rn(v[j], m), th) << (2 * (j & 15));
-        }
-        uint8_t* bp = a.pages + ((size_t)blk * a.hkv + h) * kBlockHeadBytes;
-        const int sl = p & 15;
-        if (kind == 0) {
-          *reinterpret_cast<uint4*>(bp + kKcOff + sl * 32 + 16 * half) = make_uint4(w[0], w[1], w[2], w[3]);
+              for (int ks = 0; ks < 4; ++ks) {
+                const uint64_t ad = um_desc(abuf + (uint32_t)kb * kUmRegion + (uint32_t)ks * 32u);
+                const uint64_t bd = um_desc(sB + (uint32_t)(2 * pt + kb) * kUmRegion + (uint32_t)ks * 32u);
+                um_mma(dcol, ad, bd, step > 0 ? 1u : 0u);
+                ++step;
+              }
+          um_commit(&mma_done[i & 1]);
         } else {
-#pragma unroll
-          for (int bb = 0; bb < 16; ++bb) bp[v_code_offset(sl, 16 * half + bb)] = (uint8_t)(w[bb >> 2] >> (8 * (bb & 3)));
-        }
-        if (half == 0)
-          *reinterpret_cast<uint32_t*>(bp + (kind ? kVsmOff : kKsmOff) + 4 * sl) =
-              (uint32_t)__half_as_ushort(s16) | ((uint32_t)__half_as_ushort(m16) << 16);
-        if (p >= len - kWin) {
-          __half* wr = a.ring + ((((size_t)slot * a.hkv + h) * 2 + kind) * kWin + (p % kWin)) * kD + 64 * half;
-#pragma unroll
-          for (int j = 0; j < 64; j += 8) {
-            __half2 h0 = __floats2half2_rn(0.f, 0.f), h1 = h0, h2 = h0, h3 = h0;
-            h0 = __halves2half2(fp16_sat(v[j + 0]), fp16_sat(v[j + 1]));
-            h1 = __halves2half2(fp16_sat(v[j + 2]), fp16_sat(v[j + 3]));
-            h2 = __halves2half2(fp16_sat(v[j + 4]), fp16_sat(v[j + 5]));
-            h3 = __halves2half2(fp16_sat(v[j + 6]), fp16_sat(v[j + 7]));
-            uint4 q4;
-            q4.x = *reinterpret_cast<uint32_t*>(&h0);
-            q4.y = *reinterpret_cast<uint32_t*>(&h1);
-            q4.z = *reinterpret_cast<uint32_t*>(&h2);
-            q4.w = *reinterpret_cast<uint32_t*>(&h3);
-            *reinterpret_cast<uint4*>(wr + j) = q4;
-          }
-        }
-        if (a.rotated_out != nullptr) {
-          float* ro = a.rotated_out + (((size_t)tok * 2 + kind) * a.hkv + h) * kD + 64 * half;
-#pragma unroll
-          for (int j = 0; j < 64; j += 4) *reinterpret_cast<float4*>(ro + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+          alive = false;
         }
       }
+      alive = __shfl_sync(0xffffffffu, alive, 0);
+      // tile i + 2 goes to the stage that held tile i - 1: wait until its MMAs are done
+      if (alive && i + 2 < n) {
+        if (i >= 1 && !mbar_wait_bounded(&mma_done[(i - 1) & 1], ((uint32_t)(i - 1) >> 1) & 1u)) alive = false;
+        alive = __all_sync(0xffffffffu, alive);
+        if (alive) load_tile(i + 2);
+      }
+      if (!alive) {
+        if (lane == 0) raise_flag(a.status, OKV_DEV_TIMEOUT);
+        break;
+      }
     }
-    __syncthreads();  // the exchange slots are reused by the next tile
+    cp_async_wait_all();  // no copy may outlive the CTA
+  } else {
+    const int wg = warp >> 2, q = warp & 3;
+    // destination of this thread's token in tile i, fetched one tile (of this warpgroup) ahead
+    auto token_of = [&](int i) { return tile_of(i) * kUmTile + 32 * q + lane; };
+    int n_slot = -1, n_pos = -1;
+    if (wg < n && token_of(wg) < T) {
+      n_slot = a.seq_slot[token_of(wg)];
+      n_pos = a.pos[token_of(wg)];
+    }
+    for (int i = wg; i < n; i += 2) {
+      const int tok = token_of(i);
+      const int slot = n_slot, p = n_pos;
+      const bool slot_ok = slot >= 0 && slot < a.num_slots;
+      const int len = slot_ok ? a.slot_lens[slot] : 0;
+      const bool pos_ok = slot_ok && p >= 0 && (p >> 4) < a.mbps && p < len;
+      const int blk = pos_ok ? a.block_table[(size_t)slot * a.mbps + (p >> 4)] : -1;
+      n_slot = n_pos = -1;
+      if (i + 2 < n && token_of(i + 2) < T) {
+        n_slot = a.seq_slot[token_of(i + 2)];
+        n_pos = a.pos[token_of(i + 2)];
+      }
+      if (alive && !mbar_wait_bounded(&mma_done[i & 1], ((uint32_t)i >> 1) & 1u)) alive = false;
+      alive = __all_sync(0xffffffffu, alive);
+      if (!alive) {
+        if (lane == 0) raise_flag(a.status, OKV_DEV_TIMEOUT);
+        break;
+      }
+      um_fence_after();
+      float v[128];
+      const uint32_t taddr = tmem + ((uint32_t)(32 * q) << 16) + ((uint32_t)i & 1u) * 128u;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) um_ld32(taddr + 32u * c, v + 32 * c);
+      um_wait_ld();
+      um_fence_before();
+      mbar_arrive(&tmem_free[i & 1]);  // the buffer may take tile i + 2's MMAs
+      if (tok >= T) continue;
+      if (!slot_ok) {
+        raise_flag(a.status, OKV_DEV_BAD_SLOT);
+        continue;
+      }
+      if (!pos_ok) {
+        raise_flag(a.status, OKV_DEV_BAD_POS);
+        continue;
+      }
+      if (blk < 0 || blk >= a.num_blocks) {
+        raise_flag(a.status, OKV_DEV_BAD_BLOCK);
+        continue;
+      }
+      float mn = v[0], mx = v[0];
+#pragma unroll
+      for (int j = 1; j < 128; ++j) {
+        mn = fminf(mn, v[j]);
+        mx = fmaxf(mx, v[j]);
+      }
+      const float s32 = __fdiv_rn(__fsub_rn(mx, mn), 3.0f);
+      const __half s16 = fp16_sat(s32);
+      const __half m16 = fp16_sat(mn);
+      const float sc = __half2float(s16);
+      const float m = __half2float(m16);
+      uint32_t w[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};  // the 32 code bytes of the token
+      if (sc != 0.0f) {
+        const CodeThresholds th = code_thresholds(sc);
+#pragma unroll
+        for (int j = 0; j < 128; ++j) w[j >> 4] |= int2_code(__fsub_rn(v[j], m), th) << (2 * (j & 15));
+      }
+      uint8_t* bp = a.pages + ((size_t)blk * a.hkv + h) * kBlockHeadBytes;
+      const int sl = p & 15;
+      if (kind == 0) {
+        uint4* kp = reinterpret_cast<uint4*>(bp + kKcOff + sl * 32);
+        kp[0] = make_uint4(w[0], w[1], w[2], w[3]);
+        kp[1] = make_uint4(w[4], w[5], w[6], w[7]);
+      } else {
+#pragma unroll
+        for (int bb = 0; bb < 32; ++bb) bp[v_code_offset(sl, bb)] = (uint8_t)(w[bb >> 2] >> (8 * (bb & 3)));
+      }
+      *reinterpret_cast<uint32_t*>(bp + (kind ? kVsmOff : kKsmOff) + 4 * sl) =
+          (uint32_t)__half_as_ushort(s16) | ((uint32_t)__half_as_ushort(m16) << 16);
+      if (p >= len - kWin) {
+        __half* wr = a.ring + ((((size_t)slot * a.hkv + h) * 2 + kind) * kWin + (p % kWin)) * kD;
+#pragma unroll
+        for (int j = 0; j < 128; j += 8) {
+          const __half2 h0 = __halves2half2(fp16_sat(v[j + 0]), fp16_sat(v[j + 1]));
+          const __half2 h1 = __halves2half2(fp16_sat(v[j + 2]), fp16_sat(v[j + 3]));
+          const __half2 h2 = __halves2half2(fp16_sat(v[j + 4]), fp16_sat(v[j + 5]));
+          const __half2 h3 = __halves2half2(fp16_sat(v[j + 6]), fp16_sat(v[j + 7]));
+          uint4 q4;
+          q4.x = *reinterpret_cast<const uint32_t*>(&h0);
+          q4.y = *reinterpret_cast<const uint32_t*>(&h1);
+          q4.z = *reinterpret_cast<const uint32_t*>(&h2);
+          q4.w = *reinterpret_cast<const uint32_t*>(&h3);
+          *reinterpret_cast<uint4*>(wr + j) = q4;
+        }
+      }
+      if (a.rotated_out != nullptr) {
+        float* ro = a.rotated_out + (((size_t)tok * 2 + kind) * a.hkv + h) * kD;
+#pragma unroll
+        for (int j = 0; j < 128; j += 4) *reinterpret_cast<float4*>(ro + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+      }
+    }
   }
-  // free TMEM: every thread's loads completed (wait::ld) before the barrier above
+  // free TMEM: every epilogue read completed (wait::ld) before this barrier
   um_fence_before();
   __syncthreads();
   if (warp == 0) {

@@ -644,8 +644,8 @@ __global__ void __launch_bounds__(kHW * 32, (G <= 4) ? 2 : 1) decode_heads_kerne
       if (lane == 0) mbar_arrive_expect_tx(&full[s], nvalid * copy_bytes);
       __syncwarp();
       if (bid >= 0)
-        bulk_g2s(ring + s * kHStageBytes + lane * copy_bytes, a.pages + (size_t)bid * copy_bytes, copy_bytes,
-                 &full[s]);
+        bulk_g2s_hint(ring + s * kHStageBytes + lane * copy_bytes, a.pages + (size_t)bid * copy_bytes, copy_bytes,
+                      &full[s], l2_evict_first_policy());  // each block is read once
       return true;
     };
     bool prod_ok = true;
