@@ -58,6 +58,15 @@ __device__ __forceinline__ int clamp_len(const int32_t* context_lens, int b, int
   return len;
 }
 
+// the same clamp, reading the length with a load that bypasses L1 (used before
+// grid_dep_wait(), when the kernel may start ahead of its predecessor)
+__device__ __forceinline__ int clamp_len_cg(const int32_t* context_lens, int b, int mbps) {
+  int len = __ldcg(context_lens + b);
+  const int cap = mbps * kBlock;
+  if (len < 0 || len > cap) len = len < 0 ? 0 : cap;
+  return len;
+}
+
 struct DecodeArgs {
   const __nv_bfloat16* q;
   const int32_t* seq_slot;
@@ -96,6 +105,7 @@ constexpr int kPrepThreads = 256;
 
 __global__ void __launch_bounds__(kPrepThreads) qrot_kernel(DecodeArgs a) {
   __shared__ float red[8][kD];
+  grid_dep_launch();  // the split-K kernel may start its partition and first copies now
   const int b = blockIdx.x / a.hq, head = blockIdx.x % a.hq;
   const int hk = head / a.g;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -549,11 +559,60 @@ __global__ void __launch_bounds__(kHW * 32, (G <= 4) ? 2 : 1) decode_heads_kerne
   const int head = warp % hkv, grp = warp / hkv;
   const int nb = 2 * wph;                // blocks per stage
   const uint32_t copy_bytes = (uint32_t)hkv * kBlockHeadBytes;
-  const long long total = a.prefix[a.batch];
-  if (total == 0) return;
-  const int nc = working_ctas(a, total);
+  grid_dep_launch();  // the combine kernel may take SMs as split-K CTAs finish
+
+  // The work partition, computed here from the context lengths with loads that
+  // bypass L1, so that this kernel can start (and put its first copies in
+  // flight) while the query rotation is still running.  Thread i sums the costs
+  // of a chunk of consecutive entries; a block-wide scan gives the total and
+  // the entry holding this CTA's first cost position.
+  __shared__ int part_tot[kHW], part_first[2];
+  int total;
+  {
+    const int per = (a.batch + blockDim.x - 1) / blockDim.x;
+    const int i0 = threadIdx.x * per, i1 = min(a.batch, i0 + per);
+    int own = 0;
+    for (int i = i0; i < i1; ++i) own += unit_shape(clamp_len_cg(a.context_lens, i, a.mbps)).cost;
+    int inc = own;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, inc, d);
+      if (lane >= d) inc += v;
+    }
+    if (lane == 31) part_tot[warp] = inc;
+    __syncthreads();
+    int before = 0;
+    total = 0;
+#pragma unroll
+    for (int w = 0; w < kHW; ++w) {
+      before += w < warp ? part_tot[w] : 0;
+      total += part_tot[w];
+    }
+    before += inc - own;
+    if (total > 0) {
+      const int ncw = (int)min((long long)a.nc, (long long)total);
+      const long long st0 = (long long)blockIdx.x * total / ncw;
+      if ((int)blockIdx.x < ncw && st0 >= before && st0 < before + own) {
+        int pu = before;
+        for (int i = i0; i < i1; ++i) {
+          const int cst = unit_shape(clamp_len_cg(a.context_lens, i, a.mbps)).cost;
+          if (st0 < pu + cst) {
+            part_first[0] = i;
+            part_first[1] = pu;
+            break;
+          }
+          pu += cst;
+        }
+      }
+    }
+    __syncthreads();
+  }
+  const int nc = (int)min((long long)a.nc, (long long)total);
   const int c = blockIdx.x;
-  if (c >= nc) return;
+  if (total == 0 || c >= nc) {
+    grid_dep_wait();  // no CTA finishes before the query rotation has
+    return;
+  }
   const long long start = (long long)c * total / nc;
   const long long end = (long long)(c + 1) * total / nc;
 
@@ -569,17 +628,15 @@ __global__ void __launch_bounds__(kHW * 32, (G <= 4) ? 2 : 1) decode_heads_kerne
   uint32_t it = 0;    // CTA ring position (continues across batch entries)
   bool alive = true;  // cleared if a wait never completes
 
-  int lo = 0, hi = a.batch - 1;
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (a.prefix[mid] <= start) lo = mid; else hi = mid - 1;
-  }
-  for (int b = lo; b < a.batch && a.prefix[b] < end; ++b) {
-    const UnitShape us = unit_shape(clamp_len(a.context_lens, b, a.mbps, a.status, false));
+  bool waited = false;  // grid_dep_wait() done (the query rotation's outputs are readable)
+  long long pnext = part_first[1];
+  for (int b = part_first[0]; b < a.batch && pnext < end; ++b) {
+    const UnitShape us = unit_shape(clamp_len_cg(a.context_lens, b, a.mbps));
+    const long long pu = pnext;
+    pnext += us.cost;
     if (us.cost == 0) continue;
-    const int slot = a.seq_slot[b];
+    const int slot = __ldcg(a.seq_slot + b);
     const bool slot_ok = slot >= 0 && slot < a.num_slots;
-    const long long pu = a.prefix[b];
     const int l0 = (int)(max(start, pu) - pu), l1 = (int)(min(end, pu + us.cost) - pu);
     const size_t bh0 = (size_t)b * a.hq + (size_t)head * G;  // first query head of this warp's KV head
     __syncthreads();  // the previous entry's window scratch / merge buffers (on the ring) are free again
@@ -608,8 +665,7 @@ __global__ void __launch_bounds__(kHW * 32, (G <= 4) ? 2 : 1) decode_heads_kerne
     if (warp == 0 && nst > 0) {
       cp_async_wait_all();  // the previous entry's prefetch
       __syncwarp();
-      bt_fill(p0, 0);
-      cp_async_wait_all();
+      btq[0][lane] = p0 + lane < p1 ? __ldcg(trow + p0 + lane) : -1;  // first window: loads that bypass L1
       __syncwarp();
       bt_fill(p0 + 32, 1);
     }
@@ -652,6 +708,10 @@ __global__ void __launch_bounds__(kHW * 32, (G <= 4) ? 2 : 1) decode_heads_kerne
     if (warp == 0)
       for (int j = 0; j < min(kHStages - 1, nst) && prod_ok; ++j) prod_ok = issue(j);
 
+    if (!waited) {  // from here on the query rotation's outputs are read
+      grid_dep_wait();
+      waited = true;
+    }
     // ---------------- per-warp state for (b, head), loaded while the first stages are in flight ----------------
     MmaWarpState<G> st;
     int acci[NT][8][4];
@@ -1091,6 +1151,7 @@ __global__ void __launch_bounds__(kHW * 32, (G <= 4) ? 2 : 1) decode_heads_kerne
       }
     }
   }
+  if (!waited) grid_dep_wait();
   if (warp == 0) cp_async_wait_all();  // no block-id prefetch may outlive the CTA
 }
 
@@ -1132,6 +1193,7 @@ __global__ void __launch_bounds__(kCombThreads) combine_kernel(DecodeArgs a) {
     }
     cp_async_commit();
   }
+  grid_dep_wait();  // the split partials (and the cost prefix) are read from here on
   const UnitShape sh = unit_shape(clamp_len(a.context_lens, b, a.mbps, a.status, false));
   const long long total = a.prefix[a.batch];
   float* outp = a.out + ((size_t)b * a.hq + head) * kD;
@@ -1266,13 +1328,33 @@ static okv_status launch_decode_simt(const DecodeArgs& a, cudaStream_t s) {
   return check_launch("decode");
 }
 
+// Launch with programmatic stream serialisation when `early` is set: the
+// kernel may begin while its predecessor on the stream is still running (it
+// calls grid_dep_wait() before reading the predecessor's outputs).
+template <typename... Args>
+static cudaError_t launch_pdl(void (*kernel)(Args...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                              bool early, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = early ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 template <int G>
-static okv_status launch_decode_heads(const DecodeArgs& a, cudaStream_t s) {
+static okv_status launch_decode_heads(const DecodeArgs& a, cudaStream_t s, bool early) {
   const size_t smem = HCfg<G>::smem_bytes();
   cudaError_t e = cudaFuncSetAttribute(decode_heads_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
   if (e != cudaSuccess) return fail(OKV_ERR_CUDA, "decode smem attribute: %s", cudaGetErrorString(e));
-  decode_heads_kernel<G><<<a.nc, kHW * 32, smem, s>>>(a);
+  e = launch_pdl(decode_heads_kernel<G>, dim3(a.nc), dim3(kHW * 32), smem, s, early, a);
+  if (e != cudaSuccess) return fail(OKV_ERR_CUDA, "decode launch: %s", cudaGetErrorString(e));
   return check_launch("decode");
 }
 
@@ -1323,12 +1405,17 @@ okv_status launch_decode(const okv_cache_desc* d, const void* q, int B, const in
   take_decode_events(&ev0, &ev1);
   if (ev0 != nullptr && cudaEventRecordWithFlags(ev0, s, cudaEventRecordExternal) != cudaSuccess)
     return fail(OKV_ERR_CUDA, "cudaEventRecord failed");
-  if (decode_uses_tensor_cores(a.g, a.hkv)) {
+  // Early (programmatic) launches overlap each kernel's start with its
+  // predecessor; they are left out when the split-K kernel is being timed, so
+  // that the events bracket it alone.
+  const bool early = ev0 == nullptr;
+  const bool tc = decode_uses_tensor_cores(a.g, a.hkv);
+  if (tc) {
     switch (a.g) {
-      case 1: st = launch_decode_heads<1>(a, s); break;
-      case 2: st = launch_decode_heads<2>(a, s); break;
-      case 4: st = launch_decode_heads<4>(a, s); break;
-      default: st = launch_decode_heads<8>(a, s); break;
+      case 1: st = launch_decode_heads<1>(a, s, early); break;
+      case 2: st = launch_decode_heads<2>(a, s, early); break;
+      case 4: st = launch_decode_heads<4>(a, s, early); break;
+      default: st = launch_decode_heads<8>(a, s, early); break;
     }
   } else {
     switch (a.g) {
@@ -1345,7 +1432,8 @@ okv_status launch_decode(const okv_cache_desc* d, const void* q, int B, const in
     return fail(OKV_ERR_CUDA, "cudaEventRecord failed");
   e = cudaFuncSetAttribute(combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kCombSmem);
   if (e != cudaSuccess) return fail(OKV_ERR_CUDA, "combine smem attribute: %s", cudaGetErrorString(e));
-  combine_kernel<<<B * a.hq, kCombThreads, kCombSmem, s>>>(a);
+  e = launch_pdl(combine_kernel, dim3(B * a.hq), dim3(kCombThreads), kCombSmem, s, early && tc, a);
+  if (e != cudaSuccess) return fail(OKV_ERR_CUDA, "combine launch: %s", cudaGetErrorString(e));
   return check_launch("combine");
 }
 

@@ -179,6 +179,14 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
       : "memory");
 }
 
+// Programmatic dependent launch: a kernel launched with programmatic stream
+// serialisation may start before its predecessor finishes; it must call
+// grid_dep_wait() before reading anything the predecessor writes.
+// grid_dep_launch() lets the successor be scheduled early.  Both are no-ops
+// for ordinary launches.
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory"); }
+
 // 4-byte asynchronous global -> shared copy (no register round trip), grouped
 // per thread; cp_async_wait_all waits for this thread's groups.
 __device__ __forceinline__ void cp_async4(void* smem_dst, const void* gsrc) {

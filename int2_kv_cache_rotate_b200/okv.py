@@ -19,7 +19,7 @@ LIB_PATH = os.path.join(_HERE, "libokv.so")
 HEADER = os.path.join(os.path.dirname(_HERE), "include", "okv.h")
 
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_NUMERIC = range(5)
-DEV_BAD_BLOCK, DEV_BAD_POS, DEV_BAD_SLOT = 1, 2, 4
+DEV_BAD_BLOCK, DEV_BAD_POS, DEV_BAD_SLOT, DEV_TIMEOUT = 1, 2, 4, 8
 PRE_ROTATED = 1
 HEAD_DIM, BLOCK_TOKENS, WINDOW, BLOCK_HEAD_BYTES = 128, 16, 128, 1152
 
