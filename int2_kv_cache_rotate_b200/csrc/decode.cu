@@ -443,7 +443,7 @@ __global__ void __launch_bounds__(kDecWarps * 32) decode_simt_kernel(DecodeArgs 
 // fp16 hi+lo pairs), folded into the warp's state in registers.
 // ---------------------------------------------------------------------------
 constexpr int kHW = 8;                             // warps per CTA
-constexpr int kHStages = 5;                        // ring stages (4 in flight ahead of the consumers)
+constexpr int kHStages = 6;                        // ring stages (5 in flight ahead of the consumers)
 constexpr int kSlotsPerStage = 16;                 // block-heads per stage
 constexpr int kHStageBytes = kSlotsPerStage * kBlockHeadBytes;  // 18432
 constexpr int kPStride = 40;                       // u16 per head row of the P' tile
@@ -457,12 +457,13 @@ struct HCfg {
   static constexpr int NT = G <= 4 ? 1 : G / 4;  // n-tiles of 8 columns = 4 heads x 2 limbs
   static constexpr int HP = 4 * NT;              // heads incl. padding
   static constexpr size_t ring_bytes = (size_t)kHStages * kHStageBytes;
-  static constexpr int acc_stride = NT * 16 + 1;   // per-thread fp32 accumulator row (padded)
-  static constexpr size_t acc_bytes = (size_t)kHW * 32 * acc_stride * 4;
+  // fp32 o' accumulators live in tensor memory: thread (warp w, lane l) owns
+  // TMEM lane 32 (w % 4) + l, columns 16 NT (w / 4) .. +16 NT
+  static constexpr uint32_t tmem_cols = 32u * NT;
   static constexpr size_t smem_bytes() {
     return ring_bytes                            // ring (reused for window scratch and merging)
-           + acc_bytes                           // fp32 o' accumulators, touched only on flushes
            + (size_t)2 * kHStages * 8            // full / empty mbarriers
+           + 16                                  // TMEM base address
            + (size_t)kHStages * kSlotsPerStage   // tokens per block slot
            + (size_t)kHW * HP * kPStride * 2     // P' tiles
            + (size_t)kHW * G * 2 * 4;            // merge (m, l)
@@ -518,23 +519,62 @@ template <int G>
 struct MmaWarpState {
   static constexpr int NT = HCfg<G>::NT;
   float m[NT], l[NT], msum[NT];
-  float* acc;          // shared row: fp32 o' for channels 16g + 0..15 of head 4nt + t at [16 nt + i]
+  uint32_t tacc;  // TMEM address of fp32 o' for channels 16g + 0..15 of head 4nt + t at column 16 nt + i
 };
+
+// warp-collective: 8 fp32 accumulators of every lane from / to tensor memory
+__device__ __forceinline__ void tacc_load8(uint32_t taddr, float* v) {
+  uint32_t r[8];
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];\n"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+               : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ void tacc_store8(uint32_t taddr, const float* v) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};\n" ::"r"(taddr),
+               "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
+               "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
+               "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7]))
+               : "memory");
+  asm volatile("tcgen05.wait::st.sync.aligned;\n" ::: "memory");
+}
+
+__device__ __forceinline__ void tacc_load(uint32_t taddr, float (&v)[16]) {
+  tacc_load8(taddr, v);
+  tacc_load8(taddr + 8u, v + 8);
+}
+
+__device__ __forceinline__ void tacc_store(uint32_t taddr, const float (&v)[16]) {
+  tacc_store8(taddr, v);
+  tacc_store8(taddr + 8u, v + 8);
+}
 
 // acci[mt] holds channel 16g + 2mt (regs 0,1 = hi, lo limb) and 16g + 2mt + 1
 // (regs 2,3); those channels come from code field f = 2(mt&1) and f + 1,
 // which the unshifted masks scaled by 4^f.
-// acci: exact int32 o' contributions since the last flush (row scale 4^f)
+// acci: exact int32 o' contributions since the last flush (row scale 4^f).
+// Flush: o' = (o' + acci / scale) * rescale, in tensor memory (warp-collective).
 template <int G>
-__device__ __forceinline__ void mma_flush(MmaWarpState<G>& st, int (&acci)[HCfg<G>::NT][8][4], int nt, float inv) {
+__device__ __forceinline__ void mma_flush(MmaWarpState<G>& st, int (&acci)[HCfg<G>::NT][8][4], int nt, float inv,
+                                          float rescale = 1.f) {
 #pragma unroll
-  for (int mt = 0; mt < 8; ++mt) {
-    const float s0 = (mt & 1) ? inv * (1.f / 16.f) : inv;  // field 0 or 2
-    const float s1 = s0 * 0.25f;                            // field 1 or 3
-    st.acc[16 * nt + 2 * mt] += fmaf((float)acci[nt][mt][0], 256.f * s0, (float)acci[nt][mt][1] * s0);
-    st.acc[16 * nt + 2 * mt + 1] += fmaf((float)acci[nt][mt][2], 256.f * s1, (float)acci[nt][mt][3] * s1);
+  for (int hh = 0; hh < 2; ++hh) {  // two halves of 8 channels: fewer live registers
+    float v[8];
+    tacc_load8(st.tacc + 16u * nt + 8u * hh, v);
 #pragma unroll
-    for (int j = 0; j < 4; ++j) acci[nt][mt][j] = 0;
+    for (int mq = 0; mq < 4; ++mq) {
+      const int mt = 4 * hh + mq;
+      const float s0 = (mt & 1) ? inv * (1.f / 16.f) : inv;  // field 0 or 2
+      const float s1 = s0 * 0.25f;                            // field 1 or 3
+      v[2 * mq] = (v[2 * mq] + fmaf((float)acci[nt][mt][0], 256.f * s0, (float)acci[nt][mt][1] * s0)) * rescale;
+      v[2 * mq + 1] = (v[2 * mq + 1] + fmaf((float)acci[nt][mt][2], 256.f * s1, (float)acci[nt][mt][3] * s1)) * rescale;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) acci[nt][mt][j] = 0;
+    }
+    tacc_store8(st.tacc + 16u * nt + 8u * hh, v);
   }
 }
 
@@ -544,10 +584,10 @@ __global__ void __launch_bounds__(kHW * 32, (G <= 4) ? 2 : 1) decode_heads_kerne
   extern __shared__ __align__(16) unsigned char smem_raw[];
   __shared__ int btq[2][32];  // producer's block ids, two 32-block windows
   unsigned char* ring = smem_raw;
-  float* accs = reinterpret_cast<float*>(ring + HCfg<G>::ring_bytes);
-  uint64_t* full = reinterpret_cast<uint64_t*>(reinterpret_cast<unsigned char*>(accs) + HCfg<G>::acc_bytes);
+  uint64_t* full = reinterpret_cast<uint64_t*>(ring + HCfg<G>::ring_bytes);
   uint64_t* empty = full + kHStages;
-  uint8_t* ntok = reinterpret_cast<uint8_t*>(empty + kHStages);                 // [S][16]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(empty + kHStages);          // TMEM base (16 B)
+  uint8_t* ntok = reinterpret_cast<uint8_t*>(tmem_slot + 4);                    // [S][16]
   uint16_t* pst = reinterpret_cast<uint16_t*>(ntok + kHStages * kSlotsPerStage);  // [8][HP][40]
   float* ml = reinterpret_cast<float*>(pst + kHW * HP * kPStride);              // [8][G][2]
   float* mo = reinterpret_cast<float*>(ring);  // [8][G][128], only while the ring is idle
@@ -623,7 +663,15 @@ __global__ void __launch_bounds__(kHW * 32, (G <= 4) ? 2 : 1) decode_heads_kerne
     }
     fence_mbar_init();
   }
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(smem_u32(tmem_slot)),
+                 "r"(HCfg<G>::tmem_cols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::: "memory");
+  }
+  asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
   __syncthreads();
+  asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
   uint16_t* myp = pst + warp * HP * kPStride;
   uint32_t it = 0;    // CTA ring position (continues across batch entries)
   bool alive = true;  // cleared if a wait never completes
@@ -715,7 +763,7 @@ __global__ void __launch_bounds__(kHW * 32, (G <= 4) ? 2 : 1) decode_heads_kerne
     // ---------------- per-warp state for (b, head), loaded while the first stages are in flight ----------------
     MmaWarpState<G> st;
     int acci[NT][8][4];
-    st.acc = accs + threadIdx.x * HCfg<G>::acc_stride;
+    st.tacc = *tmem_slot + ((uint32_t)(32 * (warp & 3)) << 16) + (uint32_t)(16 * NT * (warp >> 2));
     uint32_t qb[NT][8];
     float ah[NT], bh[NT], hbias[NT];
 #pragma unroll
@@ -723,8 +771,6 @@ __global__ void __launch_bounds__(kHW * 32, (G <= 4) ? 2 : 1) decode_heads_kerne
       st.m[nt] = -INFINITY;
       st.l[nt] = 0.f;
       st.msum[nt] = 0.f;
-#pragma unroll
-      for (int i = 0; i < 16; ++i) st.acc[16 * nt + i] = 0.f;
 #pragma unroll
       for (int mt = 0; mt < 8; ++mt)
 #pragma unroll
@@ -744,6 +790,13 @@ __global__ void __launch_bounds__(kHW * 32, (G <= 4) ? 2 : 1) decode_heads_kerne
       ah[nt] = ok ? a.qscale[(bh0 + hs) * 4 + 0] : 0.f;
       bh[nt] = ok ? a.qscale[(bh0 + hs) * 4 + 1] : 0.f;
       hbias[nt] = ok ? 0.f : -INFINITY;
+    }
+    {
+      float zero[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) zero[i] = 0.f;
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) tacc_store(st.tacc + 16u * nt, zero);
     }
     float s_cap = 0.f, lam = 0.f, inv = 0.f;
     int since_flush = 0;
@@ -863,15 +916,16 @@ __global__ void __launch_bounds__(kHW * 32, (G <= 4) ? 2 : 1) decode_heads_kerne
             bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 4));
             bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 8));
             bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 16));
-          }
-          if (bm > st.m[nt] + kMaxSlack) {
-            mma_flush(st, acci, nt, inv);
-            const float alpha = fast_ex2(st.m[nt] - bm);  // ex2(-inf) = 0 on the first step
-#pragma unroll
-            for (int i = 0; i < 16; ++i) st.acc[16 * nt + i] *= alpha;
-            st.l[nt] *= alpha;
-            st.msum[nt] *= alpha;
-            st.m[nt] = bm;
+            // the whole warp flushes (the accumulators are read and written
+            // warp-collectively); heads whose max did not move keep scale 1
+            const bool need = bm > st.m[nt] + kMaxSlack;
+            const float alpha = need ? fast_ex2(st.m[nt] - bm) : 1.f;  // ex2(-inf) = 0 on the first step
+            mma_flush(st, acci, nt, inv, alpha);
+            if (need) {
+              st.l[nt] *= alpha;
+              st.msum[nt] *= alpha;
+              st.m[nt] = bm;
+            }
           }
           const float mref = st.m[nt] == -INFINITY ? 0.f : st.m[nt];
           uint16_t* prow = myp + (4 * nt + t) * kPStride;
@@ -1065,17 +1119,20 @@ __global__ void __launch_bounds__(kHW * 32, (G <= 4) ? 2 : 1) decode_heads_kerne
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
         const int hs = 4 * nt + t;
+        float v[16];
+        tacc_load(st.tacc + 16u * nt, v);
         if (hs < G) {
           const float M = fmaxf(st.m[nt], wm[nt]);
           const float mref = M == -INFINITY ? 0.f : M;
           const float ab = fast_ex2(st.m[nt] - mref), aw = fast_ex2(wm[nt] - mref);
           const float* src = wo + hs * kD + 16 * g;
 #pragma unroll
-          for (int i = 0; i < 16; ++i) st.acc[16 * nt + i] = fmaf(st.acc[16 * nt + i], ab, src[i] * aw);
+          for (int i = 0; i < 16; ++i) v[i] = fmaf(v[i], ab, src[i] * aw);
           st.l[nt] = fmaf(st.l[nt], ab, wl[nt] * aw);
           st.msum[nt] *= ab;
           st.m[nt] = M;
         }
+        tacc_store(st.tacc + 16u * nt, v);
       }
     }
 
@@ -1091,13 +1148,13 @@ __global__ void __launch_bounds__(kHW * 32, (G <= 4) ? 2 : 1) decode_heads_kerne
           ms += __shfl_xor_sync(0xffffffffu, ms, o);
         }
         const int hs = 4 * nt + t;
+        float v[16];
+        tacc_load(st.tacc + 16u * nt, v);
         if (hs < G) {
           float* dst = part_b + (size_t)hs * kPartStride + 16 * g;
 #pragma unroll
           for (int i = 0; i < 16; i += 4)
-            *reinterpret_cast<float4*>(dst + i) =
-                make_float4(st.acc[16 * nt + i] + ms, st.acc[16 * nt + i + 1] + ms, st.acc[16 * nt + i + 2] + ms,
-                            st.acc[16 * nt + i + 3] + ms);
+            *reinterpret_cast<float4*>(dst + i) = make_float4(v[i] + ms, v[i + 1] + ms, v[i + 2] + ms, v[i + 3] + ms);
           if (g == 0) {
             part_b[(size_t)hs * kPartStride + 128] = st.m[nt];
             part_b[(size_t)hs * kPartStride + 129] = l;
@@ -1115,10 +1172,12 @@ __global__ void __launch_bounds__(kHW * 32, (G <= 4) ? 2 : 1) decode_heads_kerne
           ms += __shfl_xor_sync(0xffffffffu, ms, o);
         }
         const int hs = 4 * nt + t;
+        float v[16];
+        tacc_load(st.tacc + 16u * nt, v);
         if (hs < G) {
           float* dst = mo + ((size_t)warp * G + hs) * kD + 16 * g;
 #pragma unroll
-          for (int i = 0; i < 16; ++i) dst[i] = st.acc[16 * nt + i] + ms;
+          for (int i = 0; i < 16; ++i) dst[i] = v[i] + ms;
           if (g == 0) {
             ml[(warp * G + hs) * 2 + 0] = st.m[nt];
             ml[(warp * G + hs) * 2 + 1] = l;
@@ -1153,6 +1212,13 @@ __global__ void __launch_bounds__(kHW * 32, (G <= 4) ? 2 : 1) decode_heads_kerne
   }
   if (!waited) grid_dep_wait();
   if (warp == 0) cp_async_wait_all();  // no block-id prefetch may outlive the CTA
+  asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
+  __syncthreads();
+  if (warp == 0) {
+    asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(*tmem_slot), "r"(HCfg<G>::tmem_cols)
+                 : "memory");
+  }
 }
 
 // ---------------------------------------------------------------------------
