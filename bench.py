@@ -220,11 +220,12 @@ def build_gpu_workload(seed, rank, total_steps, torch, okv, WL):
 
 
 def step(w, i, okv, out, ws, ev=None):
+    """One decode step through the public call: append one token per sequence, then decode."""
     c = w["cache"]
-    okv.append_quantize(c, w["knew"][i], w["vnew"][i], w["seq"], w["pos"][i], w["table"], w["lens"][i])
     if ev is not None:
         okv.time_next_decode_kernel(*ev)
-    okv.decode_attention(c, w["q"][i], w["seq"], w["table"], w["lens"][i], out=out, ws=ws)
+    okv.decode_step(c, w["knew"][i], w["vnew"][i], w["seq"], w["pos"][i], w["lens"][i], w["q"][i], w["seq"],
+                    w["table"], w["lens"][i], out=out, ws=ws)
 
 
 def prefill_append_rate(torch, okv, WL, seed):
@@ -318,7 +319,8 @@ def run_reference(args):
         "impl": "reference", "metric": METRIC, "value": round(value, 5), "unit": "tok/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(per_step * 1e3, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": config_block(wl),
+        "config": dict(config_block(wl), timed_as="NumPy fp64 oracle on the host cores, wall clock per step; "
+                       "each step one (sequence, KV head) unit, scaled to the full step"),
         "cpu_baseline": {"value": round(value, 5), "unit": "tok/s", "cores": cores, "kind": "oracle",
                          "sample": (f"each step: 1 of the {oracle_units(wl)} (sequence, KV head) units, "
                                     f"scaled x{oracle_units(wl)}")},
@@ -331,7 +333,7 @@ def run_reference(args):
 def config_block(wl):
     return {"workload": wl.name, "batch": wl.batch, "hq": wl.hq, "hkv": wl.hkv, "head_dim": 128,
             "context_start": wl.ctx[0], "block_tokens": 16, "window": 128, "group": 128,
-            "step": "append 1 bf16 K/V token per sequence + decode attention",
+            "step": "okv_decode_step: append 1 bf16 K/V token per sequence + decode attention",
             "l2": "not flushed: each step reads the 232 MB cache, larger than the 126 MB L2",
             "timed_as": "CUDA graph of K steps; split-K kernel time from a second graph of the same steps with events around it"}
 
@@ -427,8 +429,7 @@ def run_ours(args):
             dq.copy_(hqv[i], non_blocking=True)
             dpos.copy_(hpos[i], non_blocking=True)
             dlen.copy_(hlen[i], non_blocking=True)
-            okv.append_quantize(c, dk, dv, w["seq"], dpos, w["table"], dlen)
-            okv.decode_attention(c, dq, w["seq"], w["table"], dlen, out=out, ws=ws)
+            okv.decode_step(c, dk, dv, w["seq"], dpos, dlen, dq, w["seq"], w["table"], dlen, out=out, ws=ws)
             hout.copy_(out, non_blocking=True)
         e1.record()
         torch.cuda.synchronize()
@@ -465,7 +466,7 @@ def run_ours(args):
                          "algorithmic_bytes_per_launch": int(alg)},
             "append_prefill": append_rate,
             "e2e": e2e,
-            "gpu_launches": 4 * K,
+            "gpu_launches": 3 * K,
             "clocks": clk,
         }
         if not args.no_cpu_baseline and world == 1:

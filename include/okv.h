@@ -164,6 +164,23 @@ okv_status okv_decode_attention(const okv_cache_desc* desc, const void* q, int32
 /* Size of the device array behind okv_decode_attention_noalloc (8 MiB). */
 #define OKV_NOALLOC_SCRATCH_BYTES (8u << 20)
 
+/* One decode step in one call: append this step's new tokens, then decode.
+ * Equivalent to okv_append_quantize(desc, k, v, T, new_seq_slot, new_pos,
+ * block_table, slot_lens, 0, NULL, stream) followed by
+ * okv_decode_attention(desc, q, B, seq_slot, block_table, context_lens, out,
+ * workspace, workspace_bytes, stream), with the same arguments, layouts,
+ * ownership and errors as those two calls (K/V are bf16 here; there is no
+ * pre-rotated form).  For T < 128 the append and the query rotation share one
+ * launch, which saves a kernel's latency per step; longer runs take the
+ * append's own tensor-core launch.  T = 0 decodes only; B = 0 appends only.
+ * (The pages' append and decode steps: gen-hub.ru, "Что придумали в Together
+ * AI"; encorp.ai, "OSCAR има значение…".) */
+okv_status okv_decode_step(const okv_cache_desc* desc, const void* k, const void* v, int32_t T,
+                           const int32_t* new_seq_slot, const int32_t* new_pos, const int32_t* slot_lens,
+                           const void* q, int32_t B, const int32_t* seq_slot, const int32_t* block_table,
+                           const int32_t* context_lens, float* out, void* workspace, size_t workspace_bytes,
+                           void* stream);
+
 /* Decode attention that allocates nothing and takes no workspace.  The pages
  * have no counterpart to this call: it exists for callers that cannot
  * allocate device memory -- a plugin handed only its tensors by an engine

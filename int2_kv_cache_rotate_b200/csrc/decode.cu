@@ -3,6 +3,7 @@
 // un-rotation.
 #include <type_traits>
 
+#include "append_warp.cuh"
 #include "okv_common.cuh"
 #include "okv_internal.h"
 
@@ -102,11 +103,11 @@ __device__ __forceinline__ int working_ctas(const DecodeArgs& a, long long total
 // signed 8-bit limbs in MMA-fragment order and fp16 hi/lo halves.
 // ---------------------------------------------------------------------------
 constexpr int kPrepThreads = 256;
+static_assert(kPrepThreads == kAppThreads, "the fused step kernel runs append tiles and query rotations alike");
 
-__global__ void __launch_bounds__(kPrepThreads) qrot_kernel(DecodeArgs a) {
+__device__ __forceinline__ void qrot_cta(const DecodeArgs& a, int cta) {
   __shared__ float red[8][kD];
-  grid_dep_launch();  // the split-K kernel may start its partition and first copies now
-  const int b = blockIdx.x / a.hq, head = blockIdx.x % a.hq;
+  const int b = cta / a.hq, head = cta % a.hq;
   const int hk = head / a.g;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const float* U = a.u_k + (size_t)hk * kD * kD;
@@ -114,7 +115,7 @@ __global__ void __launch_bounds__(kPrepThreads) qrot_kernel(DecodeArgs a) {
 #pragma unroll
   for (int r = 0; r < 16; ++r) u[r] = __ldg(reinterpret_cast<const float4*>(U + (size_t)(16 * warp + r) * kD) + lane);
   const float xv = __bfloat162float(a.q[((size_t)b * a.hq + head) * kD + 16 * warp + (lane & 15)]);
-  if (blockIdx.x == 0) {
+  if (cta == 0) {
     // cost prefix: thread i sums its chunk of consecutive entries, then a
     // block-wide exclusive scan (warp shuffles, then the eight warp totals)
     __shared__ int warp_tot[kPrepThreads / 32];
@@ -201,6 +202,25 @@ __global__ void __launch_bounds__(kPrepThreads) qrot_kernel(DecodeArgs a) {
       float4 qs4 = make_float4(sigma * (kInvSqrtD * kLog2e), sum * (kInvSqrtD * kLog2e), sigma, sum);
       *reinterpret_cast<float4*>(a.qscale + bh * 4) = qs4;
     }
+  }
+}
+
+__global__ void __launch_bounds__(kPrepThreads) qrot_kernel(DecodeArgs a) {
+  grid_dep_launch();  // the split-K kernel may start its partition and first copies now
+  qrot_cta(a, blockIdx.x);
+}
+
+// One launch for the start of a decode step: CTAs [0, n_app) append the
+// step's new tokens (one 32-token tile of one (KV head, K|V) each), the rest
+// rotate the queries.  The two halves touch disjoint data.
+__global__ void __launch_bounds__(kPrepThreads) step_prep_kernel(AppendArgs aa, int T, int n_tiles, DecodeArgs a) {
+  grid_dep_launch();
+  const int n_app = n_tiles * aa.hkv * 2;
+  const int x = blockIdx.x;
+  if (x < n_app) {
+    append_tile<false>(aa, T, x % n_tiles, (x / n_tiles) % aa.hkv, x / (n_tiles * aa.hkv));
+  } else {
+    qrot_cta(a, x - n_app);
   }
 }
 
@@ -1433,9 +1453,9 @@ int decode_ctas_per_sm(int g, int hkv) {
   return 4;
 }
 
-okv_status launch_decode(const okv_cache_desc* d, const void* q, int B, const int32_t* seq_slot,
-                         const int32_t* block_table, const int32_t* context_lens, float* out,
-                         void* ws, const DecodePlan& plan, cudaStream_t s) {
+static DecodeArgs make_decode_args(const okv_cache_desc* d, const void* q, int B, const int32_t* seq_slot,
+                                   const int32_t* block_table, const int32_t* context_lens, float* out, void* ws,
+                                   const DecodePlan& plan) {
   DecodeArgs a;
   a.q = (const __nv_bfloat16*)q;
   a.seq_slot = seq_slot;
@@ -1462,11 +1482,12 @@ okv_status launch_decode(const okv_cache_desc* d, const void* q, int B, const in
   a.num_blocks = d->num_blocks;
   a.num_slots = d->num_seq_slots;
   a.mbps = d->max_blocks_per_seq;
+  return a;
+}
 
-  cudaError_t e = cudaSuccess;
-  qrot_kernel<<<B * a.hq, kPrepThreads, 0, s>>>(a);
-  okv_status st = check_launch("query rotation");
-  if (st != OKV_OK) return st;
+// split-K attention and the combine, after the queries have been rotated
+static okv_status launch_decode_tail(const DecodeArgs& a, int B, cudaStream_t s) {
+  okv_status st = OKV_OK;
   cudaEvent_t ev0, ev1;
   take_decode_events(&ev0, &ev1);
   if (ev0 != nullptr && cudaEventRecordWithFlags(ev0, s, cudaEventRecordExternal) != cudaSuccess)
@@ -1496,11 +1517,35 @@ okv_status launch_decode(const okv_cache_desc* d, const void* q, int B, const in
   if (st != OKV_OK) return st;
   if (ev1 != nullptr && cudaEventRecordWithFlags(ev1, s, cudaEventRecordExternal) != cudaSuccess)
     return fail(OKV_ERR_CUDA, "cudaEventRecord failed");
-  e = cudaFuncSetAttribute(combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kCombSmem);
+  cudaError_t e = cudaFuncSetAttribute(combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kCombSmem);
   if (e != cudaSuccess) return fail(OKV_ERR_CUDA, "combine smem attribute: %s", cudaGetErrorString(e));
   e = launch_pdl(combine_kernel, dim3(B * a.hq), dim3(kCombThreads), kCombSmem, s, early && tc, a);
   if (e != cudaSuccess) return fail(OKV_ERR_CUDA, "combine launch: %s", cudaGetErrorString(e));
   return check_launch("combine");
+}
+
+okv_status launch_decode(const okv_cache_desc* d, const void* q, int B, const int32_t* seq_slot,
+                         const int32_t* block_table, const int32_t* context_lens, float* out,
+                         void* ws, const DecodePlan& plan, cudaStream_t s) {
+  const DecodeArgs a = make_decode_args(d, q, B, seq_slot, block_table, context_lens, out, ws, plan);
+  qrot_kernel<<<B * a.hq, kPrepThreads, 0, s>>>(a);
+  const okv_status st = check_launch("query rotation");
+  if (st != OKV_OK) return st;
+  return launch_decode_tail(a, B, s);
+}
+
+okv_status launch_decode_step(const okv_cache_desc* d, const void* k, const void* v, int T, const int32_t* new_slot,
+                              const int32_t* new_pos, const int32_t* slot_lens, const void* q, int B,
+                              const int32_t* seq_slot, const int32_t* block_table, const int32_t* context_lens,
+                              float* out, void* ws, const DecodePlan& plan, cudaStream_t s) {
+  const DecodeArgs a = make_decode_args(d, q, B, seq_slot, block_table, context_lens, out, ws, plan);
+  const AppendArgs aa = make_append_args(d, k, v, new_slot, new_pos, block_table, slot_lens, nullptr);
+  const int n_tiles = (T + kAppTokens - 1) / kAppTokens;
+  const long long ctas = (long long)n_tiles * d->num_kv_heads * 2 + (long long)B * a.hq;
+  step_prep_kernel<<<(unsigned)ctas, kPrepThreads, 0, s>>>(aa, T, n_tiles, a);
+  const okv_status st = check_launch("decode step (append + query rotation)");
+  if (st != OKV_OK) return st;
+  return launch_decode_tail(a, B, s);
 }
 
 }  // namespace okv

@@ -186,6 +186,43 @@ okv_status okv_decode_attention(const okv_cache_desc* desc, const void* q, int32
                        (cudaStream_t)stream);
 }
 
+okv_status okv_decode_step(const okv_cache_desc* desc, const void* k, const void* v, int32_t T,
+                           const int32_t* new_seq_slot, const int32_t* new_pos, const int32_t* slot_lens,
+                           const void* q, int32_t B, const int32_t* seq_slot, const int32_t* block_table,
+                           const int32_t* context_lens, float* out, void* workspace, size_t workspace_bytes,
+                           void* stream) {
+  okv_status st = validate_desc(desc);
+  if (st != OKV_OK) return st;
+  if (T < 0 || B < 0) return fail(OKV_ERR_INVALID_ARG, "T and B must be >= 0");
+  if (B == 0)
+    return okv_append_quantize(desc, k, v, T, new_seq_slot, new_pos, block_table, slot_lens, 0, nullptr, stream);
+  if (T > 0) {
+    if (!k || !v || !new_seq_slot || !new_pos || !slot_lens)
+      return fail(OKV_ERR_INVALID_ARG, "k, v, new_seq_slot, new_pos and slot_lens must be non-NULL");
+    if (desc->num_blocks == 0) return fail(OKV_ERR_INVALID_ARG, "cache has no blocks");
+    if ((uintptr_t)k % 2 || (uintptr_t)v % 2) return fail(OKV_ERR_INVALID_ARG, "k and v must be 2-byte aligned");
+  }
+  if (!q || !seq_slot || !block_table || !context_lens || !out || !workspace)
+    return fail(OKV_ERR_INVALID_ARG, "q, seq_slot, block_table, context_lens, out and workspace must be non-NULL");
+  const int g = desc->num_q_heads / desc->num_kv_heads;
+  if (g != 1 && g != 2 && g != 4 && g != 8 && g != 16)
+    return fail(OKV_ERR_UNSUPPORTED, "Hq/Hkv = %d not in {1,2,4,8,16}", g);
+  if ((long long)B * desc->num_kv_heads * ((long long)desc->max_blocks_per_seq + kWinCost) >= 0x7fffffffLL)
+    return fail(OKV_ERR_INVALID_ARG, "B * Hkv * max_blocks_per_seq too large");
+  if ((uintptr_t)workspace % 256) return fail(OKV_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  const DecodePlan plan = make_decode_plan(B, desc->num_q_heads, desc->num_kv_heads);
+  if (workspace_bytes < plan.total)
+    return fail(OKV_ERR_INVALID_ARG, "workspace too small: %zu < %zu bytes", workspace_bytes, plan.total);
+  const cudaStream_t s = (cudaStream_t)stream;
+  if (T > kFusedAppendMaxTokens) {  // a prefill chunk: its own (tensor-core) launch, then the decode
+    st = launch_append(desc, k, v, T, new_seq_slot, new_pos, block_table, slot_lens, 0, nullptr, s);
+    if (st != OKV_OK) return st;
+    return launch_decode(desc, q, B, seq_slot, block_table, context_lens, out, workspace, plan, s);
+  }
+  return launch_decode_step(desc, k, v, T, new_seq_slot, new_pos, slot_lens, q, B, seq_slot, block_table,
+                            context_lens, out, workspace, plan, s);
+}
+
 okv_status okv_dequantize(const okv_cache_desc* desc, int32_t B, const int32_t* seq_slot,
                           const int32_t* block_table, const int32_t* context_lens,
                           int32_t max_ctx, int32_t which, int32_t basis, int32_t source,

@@ -71,6 +71,7 @@ _SIGNATURES = {
     "okv_version": (_I32, []),
     "okv_time_next_decode_kernel": (_I32, [_P, _P]),
     "okv_decode_attention_noalloc": (_I32, [_DESC, _P, _I32, _P, _P, _P, _P, _P]),
+    "okv_decode_step": (_I32, [_DESC, _P, _P, _I32, _P, _P, _P, _P, _I32, _P, _P, _P, _P, _P, _SZ, _P]),
 }
 
 
@@ -207,6 +208,27 @@ def decode_attention(cache: Cache, q, seq_slot, block_table, context_lens, out=N
         ws = workspace(cache, batch)
     _check(lib().okv_decode_attention(ctypes.byref(cache.desc), _ptr(q), batch, _ptr(seq_slot), _ptr(block_table),
                                       _ptr(context_lens), _ptr(out), _ptr(ws), ws.numel(), _stream(stream)))
+    return out
+
+
+def decode_step(cache: Cache, k, v, new_seq_slot, new_pos, slot_lens, q, seq_slot, block_table, context_lens,
+                out=None, ws=None, stream=None):
+    """Append this step's bf16 tokens, then decode (one call; see okv_decode_step)."""
+    import torch
+    _need(k, torch.bfloat16, "k"), _need(v, torch.bfloat16, "v"), _need(q, torch.bfloat16, "q")
+    for name, t in (("new_seq_slot", new_seq_slot), ("new_pos", new_pos), ("slot_lens", slot_lens),
+                    ("seq_slot", seq_slot), ("block_table", block_table), ("context_lens", context_lens)):
+        _need(t, torch.int32, name)
+    B = q.shape[0]
+    T = k.shape[0]
+    if out is None:
+        out = torch.empty((B, cache.hq, HEAD_DIM), dtype=torch.float32, device=q.device)
+    _need(out, torch.float32, "out")
+    if ws is None:
+        ws = workspace(cache, B)
+    _check(lib().okv_decode_step(ctypes.byref(cache.desc), _ptr(k), _ptr(v), T, _ptr(new_seq_slot), _ptr(new_pos),
+                                 _ptr(slot_lens), _ptr(q), B, _ptr(seq_slot), _ptr(block_table), _ptr(context_lens),
+                                 _ptr(out), _ptr(ws), ws.numel(), _stream(stream)))
     return out
 
 
