@@ -493,13 +493,6 @@ static_assert(kHW * 8 * kD * 4 <= kHStages * kHStageBytes, "merge buffer must fi
 static_assert(kHStages * kHStageBytes / kHW >= 9216, "window scratch per warp");
 static_assert(4096 + 8 * 64 + 8 * kD * 4 <= kWarpScratch, "window scratch must fit a warp's share of the ring");
 
-__device__ __forceinline__ float lo_half(uint32_t w) {
-  return __half2float(__ushort_as_half((unsigned short)(w & 0xffffu)));
-}
-__device__ __forceinline__ float hi_half(uint32_t w) {
-  return __half2float(__ushort_as_half((unsigned short)(w >> 16)));
-}
-
 __device__ __forceinline__ void mma_f16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
   asm volatile(
       "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
@@ -527,12 +520,6 @@ __device__ __forceinline__ float fast_ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
   return y;
-}
-
-__device__ __forceinline__ uint32_t cvt_u16_sat(float x) {
-  uint16_t r;
-  asm("cvt.rni.sat.u16.f32 %0, %1;\n" : "=h"(r) : "f"(x));
-  return r;
 }
 
 template <int G>

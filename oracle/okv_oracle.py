@@ -22,7 +22,7 @@ Precision: fp64 everywhere, except the quantiser, whose fp32 steps *are* its
 definition (so that integer codes can be compared bit for bit), and the fp16
 scale/min and fp16 recent-window storage, which are part of the cache format.
 
-Readings taken where the pages are silent (each is listed in the design doc):
+Readings taken where the pages are silent:
 
 * "covariance" of the queries is the uncentred second moment E[q q^T]
   (equal to the covariance for zero-mean queries), pooled over the G query
