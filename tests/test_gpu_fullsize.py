@@ -85,8 +85,9 @@ def _check(got, want, what):
 
 
 def test_fullsize_decode_100k_bench_step():
-    """4 x 100,000 tokens: prefill, then two benchmark steps (fused one-token
-    append per sequence, decode over the grown context)."""
+    """4 x 100,000 tokens: prefill, then two benchmark steps through
+    okv_decode_step (one-token bf16 append per sequence and decode over the
+    grown context, the call the benchmark times)."""
     okv = _okv()
     seed, cfg = 5, 2
     wl = WL.config(cfg)
@@ -111,10 +112,10 @@ def test_fullsize_decode_100k_bench_step():
                                    for h in range(hkv)]) for b in range(B)])
         pos = np.full(B, L0 + i, np.int32)
         lens = pos + 1
-        okv.append_quantize(cache, _d(knew).to(torch.bfloat16), _d(vnew).to(torch.bfloat16), seq, _d(pos), table_d,
-                            _d(lens))
         q = _queries(seed, cfg, 0, hkv, B, G, extra=50 + i)
-        out = okv.decode_attention(cache, _d(q).to(torch.bfloat16), seq, table_d, _d(lens), ws=ws)
+        # the benchmark's call: append one token per sequence, then decode
+        out = okv.decode_step(cache, _d(knew).to(torch.bfloat16), _d(vnew).to(torch.bfloat16), seq, _d(pos),
+                              _d(lens), _d(q).to(torch.bfloat16), seq, table_d, _d(lens), ws=ws)
         got = out.cpu().numpy()
         for (b, h) in sampled:
             oc = oracles[(b, h)]
