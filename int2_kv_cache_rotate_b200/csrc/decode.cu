@@ -435,10 +435,11 @@ __global__ void __launch_bounds__(kDecWarps * 32) decode_simt_kernel(DecodeArgs 
 //
 // A CTA of 8 warps streams a range of blocks of one sequence for every KV
 // head at once: every block is one contiguous run of Hkv x 1152 bytes, fetched
-// by a single bulk copy into a 5-stage CTA ring (16 block-heads per stage,
-// full/empty mbarriers; lane 0 of warp 0 keeps four stages in flight, and
-// every warp copies its share of a stage to registers and releases the stage
-// before computing on it).  Warp w serves KV head w % Hkv and, per stage, two
+// by a single bulk copy into a 6-stage CTA ring (16 block-heads per stage,
+// full/empty mbarriers; warp 0 refills two stages at a time, one lane per
+// block, so that its own arithmetic is delayed by the refill latency only on
+// every other step; every warp copies its share of a stage to registers and
+// releases the stage before computing on it).  Warp w serves KV head w % Hkv and, per stage, two
 // of its blocks.
 // Per 2-block step a warp computes:
 //   scores  S[32 tok x 4NT heads] = C_K (u8 codes) . Q (two s8 limbs) on
@@ -463,7 +464,10 @@ __global__ void __launch_bounds__(kDecWarps * 32) decode_simt_kernel(DecodeArgs 
 // fp16 hi+lo pairs), folded into the warp's state in registers.
 // ---------------------------------------------------------------------------
 constexpr int kHW = 8;                             // warps per CTA
-constexpr int kHStages = 6;                        // ring stages (5 in flight ahead of the consumers)
+constexpr int kHStages = 6;                        // ring stages
+constexpr int kIssueBatch = 2;                     // stages the producer issues at a time
+static_assert(kHStages % kIssueBatch == 0 && (kIssueBatch == 1 || kIssueBatch == 2),
+              "a batch of up to 16-block stages must start at a multiple of its size and fit one 32-block window");
 constexpr int kSlotsPerStage = 16;                 // block-heads per stage
 constexpr int kHStageBytes = kSlotsPerStage * kBlockHeadBytes;  // 18432
 constexpr int kPStride = 40;                       // u16 per head row of the P' tile
@@ -703,13 +707,12 @@ __global__ void __launch_bounds__(kHW * 32, (G <= 4) ? 2 : 1) decode_heads_kerne
     const int nst = (slot_ok && alive && p1 > p0) ? (p1 - p0 + nb - 1) / nb : 0;
     const int32_t* trow = a.block_table + (size_t)(slot_ok ? slot : 0) * a.mbps;
 
-    // Warp 0 puts stage j of this entry in the next ring position (ps = its
-    // stage, puse = how often that stage was filled before).  Block ids come
+    // Warp 0 fills the ring in batches of stages, one lane per block (lane
+    // nb * i + q takes block q of the batch's stage i).  Stage j of this entry
+    // sits at ring position it + j, slot (it + j) % kHStages.  Block ids come
     // from a two-window shared buffer that async copies fill one 32-block
     // window ahead (btq[bt_buf] holds blocks bt_base .. bt_base + 31), so no
-    // block-table load sits between a released stage and its refill.  Lane
-    // q < nb handles block q of the stage.
-    uint32_t ps = it % kHStages, puse = it / kHStages;
+    // block-table load sits between a released stage and its refill.
     int bt_base = p0, bt_buf = 0;
     auto bt_fill = [&](int wbase, int buf) {  // all lanes of warp 0
       const int pi = wbase + lane;
@@ -724,16 +727,13 @@ __global__ void __launch_bounds__(kHW * 32, (G <= 4) ? 2 : 1) decode_heads_kerne
       __syncwarp();
       bt_fill(p0 + 32, 1);
     }
-    auto issue = [&](int j) -> bool {  // all lanes of warp 0
-      const uint32_t s = ps;
-      bool ok = true;
-      if (lane == 0 && puse > 0) ok = mbar_wait_bounded(&empty[s], (puse - 1) & 1u);
-      if (!__shfl_sync(0xffffffffu, ok, 0)) return false;
-      if (++ps == (uint32_t)kHStages) {
-        ps = 0;
-        ++puse;
-      }
-      const int pj = p0 + j * nb;  // nb divides 32, so a stage never straddles two windows
+    // Stages first .. first + cnt - 1, whose blocks lie in one window.  With
+    // wait_prev, their slots' previous contents (ring positions up to that of
+    // stage first + cnt - 1 - kHStages) must first be released by every warp:
+    // each warp releases positions in order, so one wait on the latest covers
+    // the batch.  The block ids are read before that wait, so the two latencies overlap.
+    auto issue_batch = [&](int first, int cnt, bool wait_prev) -> bool {  // all lanes of warp 0
+      const int pj = p0 + first * nb;
       while (pj >= bt_base + 32) {
         bt_base += 32;
         bt_buf ^= 1;
@@ -741,27 +741,45 @@ __global__ void __launch_bounds__(kHW * 32, (G <= 4) ? 2 : 1) decode_heads_kerne
         __syncwarp();
         bt_fill(bt_base + 32, bt_buf ^ 1);  // the window just retired takes the one after next
       }
+      const int bi = lane / nb, q = lane - bi * nb;  // stage first + bi, block q
+      const bool act = lane < cnt * nb;
       const int pi = pj + lane;
-      const bool mine = lane < nb && pi < p1;
+      const bool mine = act && pi < p1;
       int bid = mine ? btq[bt_buf][pj - bt_base + lane] : -1;
       if (mine && (bid < 0 || bid >= a.num_blocks)) {
         raise_flag(a.status, OKV_DEV_BAD_BLOCK);
         bid = -1;
       }
-      if (lane < nb) ntok[s * kSlotsPerStage + lane] = bid >= 0 ? (uint8_t)min(kBlock, us.n_int2 - kBlock * pi) : 0;
-      const uint32_t nvalid = __popc(__ballot_sync(0xffffffffu, bid >= 0));
+      bool ok = true;
+      if (wait_prev && lane == 0) {
+        const uint32_t last = it + (uint32_t)(first + cnt - 1);  // >= kHStages
+        ok = mbar_wait_bounded(&empty[last % kHStages], (last / kHStages - 1u) & 1u);
+      }
+      if (!__shfl_sync(0xffffffffu, ok, 0)) return false;
+      const uint32_t s = (it + (uint32_t)(first + bi)) % kHStages;
+      const uint32_t valid = __ballot_sync(0xffffffffu, bid >= 0);
+      const uint32_t nvalid = __popc((valid >> (bi * nb)) & ((1u << nb) - 1u));  // lane bi * nb <= 31
+      if (act) ntok[s * kSlotsPerStage + q] = bid >= 0 ? (uint8_t)min(kBlock, us.n_int2 - kBlock * pi) : 0;
       __syncwarp();
       // the barrier must expect every byte before any copy can complete on it
-      if (lane == 0) mbar_arrive_expect_tx(&full[s], nvalid * copy_bytes);
+      if (act && q == 0) mbar_arrive_expect_tx(&full[s], nvalid * copy_bytes);
       __syncwarp();
       if (bid >= 0)
-        bulk_g2s_hint(ring + s * kHStageBytes + lane * copy_bytes, a.pages + (size_t)bid * copy_bytes, copy_bytes,
+        bulk_g2s_hint(ring + s * kHStageBytes + q * copy_bytes, a.pages + (size_t)bid * copy_bytes, copy_bytes,
                       &full[s], l2_evict_first_policy());  // each block is read once
       return true;
     };
+    // Prologue: every slot (the ring is idle at an entry's start).  A batch
+    // stops at a window boundary (nb divides 32).
     bool prod_ok = true;
-    if (warp == 0)
-      for (int j = 0; j < min(kHStages - 1, nst) && prod_ok; ++j) prod_ok = issue(j);
+    if (warp == 0) {
+      const int npro = min(kHStages, nst);
+      for (int first = 0; first < npro && prod_ok;) {
+        const int cnt = min(npro - first, (32 - (first * nb) % 32) / nb);
+        prod_ok = issue_batch(first, cnt, false);
+        first += cnt;
+      }
+    }
 
     if (!waited) {  // from here on the query rotation's outputs are read
       grid_dep_wait();
@@ -813,7 +831,12 @@ __global__ void __launch_bounds__(kHW * 32, (G <= 4) ? 2 : 1) decode_heads_kerne
     uint32_t cs = it % kHStages, cph = (it / kHStages) & 1u;  // consumer stage and phase parity
     for (int j = 0; j < nst; ++j) {
       if (warp == 0) {
-        if (prod_ok && j + kHStages - 1 < nst) prod_ok = issue(j + kHStages - 1);
+        // every kIssueBatch steps: the next kIssueBatch stages, into the slots
+        // of stages j - kIssueBatch .. j - 1 (kIssueBatch * nb blocks from a
+        // multiple of kIssueBatch * nb, which divides 32: inside one window)
+        const int nf = j + kHStages - kIssueBatch;
+        if (prod_ok && j >= kIssueBatch && j % kIssueBatch == 0 && nf < nst)
+          prod_ok = issue_batch(nf, min(kIssueBatch, nst - nf), true);
         if (!prod_ok) {
           if (lane == 0) raise_flag(a.status, OKV_DEV_TIMEOUT);
           alive = false;
