@@ -125,6 +125,34 @@ def test_fullsize_decode_100k_bench_step():
     assert cache.device_status() == 0
 
 
+@pytest.mark.parametrize("hq,hkv,L", [(4, 1, 400_000), (8, 2, 200_000), (16, 4, 100_000)])
+def test_long_ranges_every_kv_head_count(hq, hkv, L):
+    """With fewer KV heads a ring stage holds more blocks (16 / Hkv), so the
+    split-K producer's batches, its prologue split at block-id window
+    boundaries and its window refills take other paths than at 8 KV heads.
+    Two sequences sized so that every CTA streams about ten stages."""
+    okv = _okv()
+    seed, cfg, B = 9, 2, 2
+    G = hq // hkv
+    sampled = [(0, 0), (1, hkv - 1)]
+    uk, uv = H.rotations(seed + hkv, hkv)
+    table, nb = WL.block_table(seed + hkv, cfg, [L] * B, extra_tokens=16)
+    cache = okv.Cache(hq, hkv, nb, B, table.shape[1], uk, uv)
+    table_d = _d(table)
+    host = {(b, h, kind): WL.sample_rotated(seed + hkv, cfg, 0, h, L, kind, extra=b)
+            for (b, h) in sampled for kind in (0, 1)}
+    _fill(cache, table_d, [L] * B, [L] * B, sampled, host, _Pool(hkv, seed))
+    q = _queries(seed + hkv, cfg, 0, hkv, B, G, extra=3)
+    lens = np.full(B, L, np.int32)
+    got = okv.decode_attention(cache, _d(q).to(torch.bfloat16), _d(np.arange(B, dtype=np.int32)), table_d,
+                               _d(lens)).cpu().numpy()
+    for (b, h) in sampled:
+        oc = _oracle_head(uk, uv, h, host[(b, h, 0)], host[(b, h, 1)])
+        want = O.decode(oc, q[b:b + 1, h * G:(h + 1) * G], [0], [L], G)
+        _check(got[b:b + 1, h * G:(h + 1) * G], want, (hkv, b, h))
+    assert cache.device_status() == 0
+
+
 def test_fullsize_decode_8b_layer_32k():
     okv = _okv()
     seed, cfg = 6, 1
