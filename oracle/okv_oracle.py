@@ -41,7 +41,10 @@ Readings taken where the pages are silent:
   clamped to [0, 3], dequantised as s*c + m;
 * every token is quantised at append; the last W = 128 positions are also
   kept as fp16 rotated values and decode reads those positions from fp16;
-  no attention-sink tokens.
+* sink tokens: the first S positions of a sequence are kept the same way and
+  read from fp16.  The pages name sinks without a count; S is a cache
+  parameter, 0 (no sinks) by default.  S = 192 with W = 128 keeps 320 of
+  128K tokens 16-bit, the 0.24 % the pages quote.
 """
 from __future__ import annotations
 
@@ -262,14 +265,16 @@ class Cache:
     """Logical (unpaged) mixed-precision KV cache for one layer.
 
     Every appended token is quantised to INT2; its fp16 rotated values are
-    also stored, and decode reads the most recent W positions from those.
+    also stored, and decode reads the most recent W positions and the first
+    `sinks` positions from those.
     [EN] section "OSCAR има значение…" and [AF] "OSCAR: figyelem-tudatos…"
     (recent tokens stay 16-bit, history goes to INT2, paged-cache compatible).
     """
 
-    def __init__(self, hkv: int, u_k: np.ndarray, u_v: np.ndarray, window: int = W):
+    def __init__(self, hkv: int, u_k: np.ndarray, u_v: np.ndarray, window: int = W, sinks: int = 0):
         self.hkv = hkv
         self.window = window
+        self.sinks = sinks
         self.r = {0: np.stack([rotation(u) for u in u_k]), 1: np.stack([rotation(u) for u in u_v])}
         self.seqs = {}
 
@@ -316,16 +321,16 @@ class Cache:
         return st["codes"][pos], st["s16"][pos], st["m16"][pos], st["z16"][pos]
 
     def values(self, slot: int, kind: int, h: int, length: int) -> np.ndarray:
-        """Rotated vectors as decode sees them: positions < length - W dequantised
-        from INT2, the last min(length, W) from fp16.  fp64 [length, d]."""
+        """Rotated vectors as decode sees them: the first min(length, sinks) and
+        the last min(length, W) positions from fp16, the rest dequantised from
+        INT2.  fp64 [length, d]."""
         st = self.seqs[(slot, kind, h)]
         if not st["set"][:length].all():
             raise ValueError("decode over positions that were never appended")
-        first_fp16 = max(0, length - self.window)
-        out = np.empty((length, D))
-        out[:first_fp16] = dequantize(st["codes"][:first_fp16], st["s16"][:first_fp16],
-                                      st["m16"][:first_fp16])
-        out[first_fp16:] = st["z16"][first_fp16:length].astype(np.float64)
+        out = st["z16"][:length].astype(np.float64)
+        int2 = np.arange(length)
+        int2 = int2[(int2 >= self.sinks) & (int2 < length - self.window)]
+        out[int2] = dequantize(st["codes"][int2], st["s16"][int2], st["m16"][int2])
         return out
 
 

@@ -249,14 +249,14 @@ def test_dequantize_scalar():
 
 # --------------------------------------------------------- cache and decode
 
-def _brute_decode_one(q, r_k, r_v, ent_k, ent_v, length, window):
+def _brute_decode_one(q, r_k, r_v, ent_k, ent_v, length, window, sinks=0):
     """Loop-only decode for one query head from raw cache entries."""
     d = len(q)
     qr = [sum(q[c] * r_k[c, j] for c in range(d)) for j in range(d)]
 
     def val(ent, p):
         codes, s16, m16, z16 = ent(p)
-        if p >= length - window:
+        if p >= length - window or p < sinks:
             return [float(z16[j]) for j in range(d)]
         return [float(s16) * int(codes[j]) + float(m16) for j in range(d)]
 
@@ -275,11 +275,11 @@ def _brute_decode_one(q, r_k, r_v, ent_k, ent_v, length, window):
     return np.array([sum(o[j] * r_v[c, j] for j in range(d)) for c in range(d)])
 
 
-def _small_cache(seed, hkv, lens, window=O.W):
+def _small_cache(seed, hkv, lens, window=O.W, sinks=0):
     rng = np.random.default_rng(seed)
     uk = np.stack([WL.haar_orthogonal(rng) for _ in range(hkv)])
     uv = np.stack([WL.haar_orthogonal(rng) for _ in range(hkv)])
-    cache = O.Cache(hkv, uk, uv, window=window)
+    cache = O.Cache(hkv, uk, uv, window=window, sinks=sinks)
     for slot, length in enumerate(lens):
         k = WL.to_bf16_exact(rng.standard_normal((length, hkv, 128)).astype(np.float32) * 2)
         v = WL.to_bf16_exact(rng.standard_normal((length, hkv, 128)).astype(np.float32))
@@ -289,18 +289,49 @@ def _small_cache(seed, hkv, lens, window=O.W):
     return cache, rng
 
 
-def test_decode_matches_loop_brute_force():
-    lens = [27, 9]
-    cache, rng = _small_cache(10, 2, lens, window=8)
-    q = WL.to_bf16_exact(rng.standard_normal((2, 4, 128)).astype(np.float32))
-    got = O.decode(cache, q, [0, 1], lens, hq=4)
+@pytest.mark.parametrize("sinks", [0, 4])
+def test_decode_matches_loop_brute_force(sinks):
+    # with 4 sinks and a window of 8: length 27 has INT2 positions 4..18,
+    # length 9 has none (sink and window overlap), length 13 exactly none
+    lens = [27, 9, 13]
+    cache, rng = _small_cache(10, 2, lens, window=8, sinks=sinks)
+    q = WL.to_bf16_exact(rng.standard_normal((3, 4, 128)).astype(np.float32))
+    got = O.decode(cache, q, [0, 1, 2], lens, hq=4)
     for b, length in enumerate(lens):
         for h in range(4):
             hk = h // 2
             want = _brute_decode_one(
                 q[b, h].astype(float), cache.r[0][hk], cache.r[1][hk],
-                lambda p: cache.entry(b, 0, hk, p), lambda p: cache.entry(b, 1, hk, p), length, 8)
+                lambda p: cache.entry(b, 0, hk, p), lambda p: cache.entry(b, 1, hk, p), length, 8, sinks)
             assert np.abs(got[b, h] - want).max() < 1e-10 * max(1.0, np.abs(want).max())
+
+
+def test_sinks_change_only_the_first_positions():
+    """Sinks replace the INT2 values of the first S positions by their fp16
+    rotated values and nothing else; with S + W >= length every position is
+    fp16 and decode is textbook attention on the fp16 rotated operands."""
+    rng = np.random.default_rng(15)
+    uk = WL.haar_orthogonal(rng)[None]
+    uv = WL.haar_orthogonal(rng)[None]
+    n = 300
+    k = WL.to_bf16_exact(rng.standard_normal((n, 1, 128)).astype(np.float32))
+    v = WL.to_bf16_exact(rng.standard_normal((n, 1, 128)).astype(np.float32))
+    plain, sunk, all16 = O.Cache(1, uk, uv), O.Cache(1, uk, uv, sinks=32), O.Cache(1, uk, uv, sinks=192)
+    for c in (plain, sunk, all16):
+        c.append(0, 0, k, v)
+    for kind in (0, 1):
+        a, b = plain.values(0, kind, 0, n), sunk.values(0, kind, 0, n)
+        assert np.array_equal(a[32:], b[32:])
+        z16 = np.stack([plain.entry(0, kind, 0, p)[3] for p in range(32)]).astype(float)
+        assert np.array_equal(b[:32], z16) and not np.array_equal(a[:32], z16)
+    q = WL.to_bf16_exact(rng.standard_normal((1, 2, 128)).astype(np.float32))
+    got = O.decode(all16, q, [0], [n], hq=2)  # 192 + 128 >= 300
+    kr = (k[:, 0].astype(np.float64) @ all16.r[0][0]).astype(np.float32).astype(np.float16).astype(float)
+    vr = (v[:, 0].astype(np.float64) @ all16.r[1][0]).astype(np.float32).astype(np.float16).astype(float)
+    for h in range(2):
+        qr = q[0, h].astype(float) @ all16.r[0][0]
+        p = scipy.special.softmax(kr @ qr / math.sqrt(128))
+        assert np.abs(got[0, h] - (p @ vr) @ all16.r[1][0].T).max() < 1e-12
 
 
 def test_decode_window_only_is_textbook_attention():
@@ -383,6 +414,9 @@ def test_sizing_matches_pages():
     assert O.int2_kv_bytes_per_token(80, 8) * 131072 / 2 ** 30 == 5.625
     # about 2.28 bits with about 0.24 % of tokens kept 16-bit
     assert abs(O.effective_bits(0.0024) - 2.283) < 5e-4
+    # 192 sink tokens and the 128-token window at 128K: 0.24 % and 2.28 bits
+    frac = (192 + O.W) / 131072
+    assert round(100 * frac, 2) == 0.24 and round(O.effective_bits(frac), 2) == 2.28
 
 
 # ----------------------------------------------------------- quality order
