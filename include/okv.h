@@ -12,9 +12,12 @@
  *   - the rotated vectors are stored as 2-bit codes with a per-group scale
  *     and minimum (bigsaas.top, "Revolução no Serviço de LLMs…", section
  *     "Resultados e Métricas de Desempenho": INT2 at about 2.28 bits);
- *   - recent tokens are also kept in 16-bit, older ones only in INT2, in a
- *     paged cache (encorp.ai, "KV cache compression е инфраструктурно
- *     решение…", section "OSCAR има значение…");
+ *   - sink and recent tokens are also kept in 16-bit, older ones only in
+ *     INT2, in a paged cache (encorp.ai, "KV cache compression е
+ *     инфраструктурно решение…", section "OSCAR има значение…"; the pages
+ *     give no sink count, so it is a cache parameter, num_sink, 0 by default;
+ *     192 sinks with the 128-token window keep the ~0.24 % of a 128K context
+ *     that section quotes);
  *   - decode attention reads that cache; decode is bound by reading the cache
  *     from HBM (aiforradalom.hu intro).
  *
@@ -48,6 +51,11 @@
  * Block `blk`, head `h` starts at pages + (blk * num_kv_heads + h) * 1152.
  * Window ring: fp16 [num_seq_slots][num_kv_heads][2 (K,V)][W][d]; position p
  * of a sequence lives in row p % W; values are the rotated vector in fp16.
+ * Sink rows: fp16 [num_seq_slots][num_kv_heads][2 (K,V)][num_sink][d];
+ * position p < num_sink lives in row p.
+ * Every position is quantised to INT2; decode of a sequence of length L reads
+ * positions [0, min(S, L)) from the sink rows (S = num_sink),
+ * [max(L - W, S), L) from the window ring and [S, L - W) from INT2 blocks.
  */
 #ifndef OKV_H
 #define OKV_H
@@ -79,6 +87,7 @@ typedef enum {
 #define OKV_HEAD_DIM 128
 #define OKV_BLOCK_TOKENS 16
 #define OKV_WINDOW 128
+#define OKV_MAX_SINK 1024
 #define OKV_BLOCK_HEAD_BYTES 1152
 
 typedef struct {
@@ -91,12 +100,15 @@ typedef struct {
   int32_t num_blocks;         /* physical blocks in `pages`                 */
   int32_t num_seq_slots;      /* sequences the window ring holds            */
   int32_t max_blocks_per_seq; /* row length of every block table            */
-  int32_t reserved;
+  int32_t num_sink;           /* sink tokens kept fp16: a multiple of 16 in
+                                 [0, OKV_MAX_SINK], else OKV_ERR_UNSUPPORTED */
   void* pages;                /* device, num_blocks*Hkv*1152 B, 16-B aligned */
   void* window_ring;          /* device fp16, layout above, 16-B aligned     */
   const float* u_k;           /* device fp32 [Hkv][d][d]: U_K of each KV head */
   const float* u_v;           /* device fp32 [Hkv][d][d]: U_V of each KV head */
   uint32_t* status_word;      /* device, nullable: OKV_DEV_* flags (OR-ed)   */
+  void* sink_rows;            /* device fp16, layout above, 16-B aligned;
+                                 may be NULL when num_sink = 0             */
 } okv_cache_desc;
 
 /* Offline calibration of the rotations, on the host in fp64 (once per layer).
@@ -115,9 +127,10 @@ okv_status okv_calibrate_rotations(const float* q, int64_t nq, const float* k, c
                                    int64_t nk, int32_t hq, int32_t hkv, int32_t d, float* r_k,
                                    float* r_v, float* u_k, float* u_v);
 
-/* Bytes the caller allocates for `pages` and for `window_ring`. */
+/* Bytes the caller allocates for `pages`, `window_ring` and `sink_rows`. */
 size_t okv_pages_bytes(int32_t num_blocks, int32_t num_kv_heads);
 size_t okv_window_bytes(int32_t num_seq_slots, int32_t num_kv_heads);
+size_t okv_sink_bytes(int32_t num_seq_slots, int32_t num_kv_heads, int32_t num_sink);
 
 /* Append T tokens: rotate each K and V vector of every KV head by its R,
  * quantise it to 2-bit codes with fp16 scale and min (fp32 round-to-nearest
@@ -125,7 +138,7 @@ size_t okv_window_bytes(int32_t num_seq_slots, int32_t num_kv_heads);
  * c = 0 when s = 0; fp16 conversions saturate at +-65504), write codes and
  * (s, m) into slot pos%16 of block block_table[slot][pos/16], and, when
  * pos >= slot_lens[slot] - W, also write the fp16 rotated vector into the
- * window ring row pos % W.
+ * window ring row pos % W, and when pos < num_sink into sink row pos.
  *   k, v: device [T][Hkv][d], bf16 (or fp32 already rotated with OKV_PRE_ROTATED);
  *   seq_slot, pos: device int32 [T]; block_table: device int32
  *   [num_seq_slots][max_blocks_per_seq]; slot_lens: device int32
@@ -149,9 +162,10 @@ size_t okv_decode_workspace_bytes(const okv_cache_desc* desc, int32_t B);
  *   tokens in the cache for each sequence (the caller appends the step's own
  *   token first); out: device fp32 [B][Hq][d]; workspace: device, at least
  *   okv_decode_workspace_bytes(desc, B) bytes, 256-B aligned.
- * Query head j reads KV head j/(Hq/Hkv).  With L = context_lens[b], positions
- * [0, L-W) are read from the INT2 blocks and [max(0,L-W), L) from the fp16
- * window; q~ = q R_K, softmax(q~ x^T / sqrt(d)) over those, then o = o~ R_V^T.
+ * Query head j reads KV head j/(Hq/Hkv).  With L = context_lens[b] and
+ * S = num_sink, positions [0, min(S, L)) are read from the fp16 sink rows,
+ * [S, L-W) from the INT2 blocks and [max(S, L-W), L) from the fp16 window;
+ * q~ = q R_K, softmax(q~ x^T / sqrt(d)) over those, then o = o~ R_V^T.
  * L = 0 gives zeros.  Launches three kernels on `stream` (query rotation,
  * split-K attention, split combine with the value un-rotation).
  * Pages: aiforradalom.hu intro (decode streams the cache from HBM);
@@ -204,7 +218,7 @@ okv_status okv_decode_attention_noalloc(const okv_cache_desc* desc, const void* 
 /* Gather and dequantise the cache into dense fp32.
  *   which: 0 keys, 1 values.  basis: 0 rotated (as stored), 1 original
  *   (multiplied back by R^T).  source: 0 INT2 for every position, 1 as decode
- *   reads it (fp16 window for the last W positions).  out: device fp32
+ *   reads it (fp16 for the last W positions and the first num_sink).  out: device fp32
  *   [B][Hkv][max_ctx][d]; rows at positions >= context_lens[b] are zero.
  * INT2 values are s*c + m computed with one fused multiply-add. */
 okv_status okv_dequantize(const okv_cache_desc* desc, int32_t B, const int32_t* seq_slot,

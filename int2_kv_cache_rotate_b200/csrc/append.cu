@@ -122,8 +122,9 @@ __device__ __forceinline__ void finish_token_tc(const AppendArgs& a, int tok, bo
   if (t == 0)
     *reinterpret_cast<uint32_t*>(base + (kind ? kVsmOff : kKsmOff) + 4 * sl) =
         (uint32_t)__half_as_ushort(s16) | ((uint32_t)__half_as_ushort(m16) << 16);
-  if (p >= len - kWin) {
-    __half* row = a.ring + ((((size_t)slot * a.hkv + h) * 2 + kind) * kWin + (p % kWin)) * kD + 32 * t;
+  __half* wrow = window_row(a, slot, h, kind, p, len);
+  __half* srow = sink_row(a, slot, h, kind, p);
+  if (wrow != nullptr || srow != nullptr) {
 #pragma unroll
     for (int k = 0; k < 8; k += 2) {
       __half2 h0 = __halves2half2(fp16_sat(v[k][0]), fp16_sat(v[k][1]));
@@ -135,7 +136,8 @@ __device__ __forceinline__ void finish_token_tc(const AppendArgs& a, int tok, bo
       q4.y = *reinterpret_cast<uint32_t*>(&h1);
       q4.z = *reinterpret_cast<uint32_t*>(&h2);
       q4.w = *reinterpret_cast<uint32_t*>(&h3);
-      *reinterpret_cast<uint4*>(row + 4 * k) = q4;
+      if (wrow != nullptr) *reinterpret_cast<uint4*>(wrow + 32 * t + 4 * k) = q4;
+      if (srow != nullptr) *reinterpret_cast<uint4*>(srow + 32 * t + 4 * k) = q4;
     }
   }
   if (a.rotated_out != nullptr) {
@@ -555,8 +557,9 @@ __global__ void __launch_bounds__(kUmThreads, 1) append_umma_kernel(AppendArgs a
       }
       *reinterpret_cast<uint32_t*>(bp + (kind ? kVsmOff : kKsmOff) + 4 * sl) =
           (uint32_t)__half_as_ushort(s16) | ((uint32_t)__half_as_ushort(m16) << 16);
-      if (p >= len - kWin) {
-        __half* wr = a.ring + ((((size_t)slot * a.hkv + h) * 2 + kind) * kWin + (p % kWin)) * kD;
+      __half* wr = window_row(a, slot, h, kind, p, len);
+      __half* sr = sink_row(a, slot, h, kind, p);
+      if (wr != nullptr || sr != nullptr) {
 #pragma unroll
         for (int j = 0; j < 128; j += 8) {
           const __half2 h0 = __halves2half2(fp16_sat(v[j + 0]), fp16_sat(v[j + 1]));
@@ -568,7 +571,8 @@ __global__ void __launch_bounds__(kUmThreads, 1) append_umma_kernel(AppendArgs a
           q4.y = *reinterpret_cast<const uint32_t*>(&h1);
           q4.z = *reinterpret_cast<const uint32_t*>(&h2);
           q4.w = *reinterpret_cast<const uint32_t*>(&h3);
-          *reinterpret_cast<uint4*>(wr + j) = q4;
+          if (wr != nullptr) *reinterpret_cast<uint4*>(wr + j) = q4;
+          if (sr != nullptr) *reinterpret_cast<uint4*>(sr + j) = q4;
         }
       }
       if (a.rotated_out != nullptr) {

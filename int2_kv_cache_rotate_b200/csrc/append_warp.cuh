@@ -1,7 +1,8 @@
 // Warp-level append shared by the append kernels and the fused decode-step
 // kernel: rotate (U, Hadamard butterfly, bit-reversal remap), quantise to INT2
-// with fp16 scale/min, pack, and write the paged cache and the fp16 window,
-// for one 32-token tile of one (KV head, K|V).
+// with fp16 scale/min, pack, and write the paged cache and the fp16 rows of
+// the recent-token window and of the sink tokens, for one 32-token tile of
+// one (KV head, K|V).
 #pragma once
 
 #include "okv.h"
@@ -20,9 +21,10 @@ struct AppendArgs {
   const float* u_v;
   uint8_t* pages;
   __half* ring;
+  __half* sink;  // fp16 rows of the first nsink positions
   float* rotated_out;
   uint32_t* status;
-  int hkv, num_blocks, num_slots, mbps;
+  int hkv, num_blocks, num_slots, mbps, nsink;
 };
 
 inline AppendArgs make_append_args(const okv_cache_desc* d, const void* k, const void* v, const int32_t* seq_slot,
@@ -39,6 +41,8 @@ inline AppendArgs make_append_args(const okv_cache_desc* d, const void* k, const
   a.u_v = d->u_v;
   a.pages = (uint8_t*)d->pages;
   a.ring = (__half*)d->window_ring;
+  a.sink = (__half*)d->sink_rows;
+  a.nsink = d->num_sink;
   a.rotated_out = rotated_out;
   a.status = d->status_word;
   a.hkv = d->num_kv_heads;
@@ -46,6 +50,16 @@ inline AppendArgs make_append_args(const okv_cache_desc* d, const void* k, const
   a.num_slots = d->num_seq_slots;
   a.mbps = d->max_blocks_per_seq;
   return a;
+}
+
+// fp16 row of position p of (slot, KV head, K|V) in the recent-token ring
+// (for p >= len - kWin) and in the sink rows (for p < nsink); null where the
+// position has no such row.
+__device__ __forceinline__ __half* window_row(const AppendArgs& a, int slot, int h, int kind, int p, int len) {
+  return p >= len - kWin ? a.ring + ((((size_t)slot * a.hkv + h) * 2 + kind) * kWin + (p % kWin)) * kD : nullptr;
+}
+__device__ __forceinline__ __half* sink_row(const AppendArgs& a, int slot, int h, int kind, int p) {
+  return p < a.nsink ? a.sink + ((((size_t)slot * a.hkv + h) * 2 + kind) * a.nsink + p) * kD : nullptr;
 }
 
 constexpr int kAppThreads = 256;
@@ -88,14 +102,16 @@ __device__ __forceinline__ void finish_token(const AppendArgs& a, int t, int h, 
     base[v_code_offset(s16, r)] = (uint8_t)q.byte;
   }
   if (lane == 0) *reinterpret_cast<uint32_t*>(base + (kind ? kVsmOff : kKsmOff) + 4 * s16) = q.sm;
-  if (p >= len - kWin) {
-    __half* row = a.ring + ((((size_t)slot * a.hkv + h) * 2 + kind) * kWin + (p % kWin)) * kD + 4 * r;
+  __half* wrow = window_row(a, slot, h, kind, p, len);
+  __half* srow = sink_row(a, slot, h, kind, p);
+  if (wrow != nullptr || srow != nullptr) {
     __half2 lo = __halves2half2(fp16_sat(y[0]), fp16_sat(y[2]));
     __half2 hi = __halves2half2(fp16_sat(y[1]), fp16_sat(y[3]));
     uint2 w;
     w.x = *reinterpret_cast<uint32_t*>(&lo);
     w.y = *reinterpret_cast<uint32_t*>(&hi);
-    *reinterpret_cast<uint2*>(row) = w;
+    if (wrow != nullptr) *reinterpret_cast<uint2*>(wrow + 4 * r) = w;
+    if (srow != nullptr) *reinterpret_cast<uint2*>(srow + 4 * r) = w;
   }
 }
 

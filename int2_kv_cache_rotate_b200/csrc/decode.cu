@@ -10,34 +10,43 @@
 namespace okv {
 
 // ---------------------------------------------------------------------------
-// Work partition.  Batch entry b with L tokens costs ceil(max(L-W,0)/16)
-// blocks (every KV head of a block is one contiguous run) plus kWinCost per
-// 16-row chunk of its fp16 window.  Entries are laid end to end in "cost
-// space"; split-K CTA c takes the contiguous range [c*total/NC, (c+1)*total/NC).
-// Inside an entry, cost positions [0, n_chunks * kWinCost) stand for the
-// window chunks (chunk i belongs to the CTA holding position i * kWinCost) and
-// the rest for the blocks in order.  A (entry, CTA) pair writes partial slot
+// Work partition.  A batch entry with L tokens and S sink tokens reads
+// positions [0, min(S, L)) from the fp16 sink rows, [S, L - W) from INT2
+// blocks (table columns S/16 on) and [max(L - W, S), L) from the fp16 window
+// ring.  It costs one unit per INT2 block (every KV head of a block is one
+// contiguous run) plus kWinCost per 16-row fp16 chunk (window chunks first,
+// then sink chunks).  Entries are laid end to end in "cost space"; split-K
+// CTA c takes the contiguous range [c*total/NC, (c+1)*total/NC).  Inside an
+// entry, cost positions [0, n_chunks * kWinCost) stand for the fp16 chunks
+// (chunk i belongs to the CTA holding position i * kWinCost) and the rest for
+// the blocks in order.  A (entry, CTA) pair writes partial slot
 // c + b (all query heads): distinct for distinct pairs because CTAs and
 // entries are both contiguous.
 // ---------------------------------------------------------------------------
 struct UnitShape {
-  int len;      // tokens in the cache
-  int n_int2;   // tokens read from INT2 blocks
-  int n_pages;  // INT2 blocks touched
-  int n_win;    // tokens read from the fp16 window
-  int n_wchunk; // 16-row chunks of the window
-  int win_cost;
+  int len;        // tokens in the cache
+  int n_int2;     // tokens read from INT2 blocks: positions nsink .. nsink + n_int2 - 1
+  int n_pages;    // INT2 blocks touched (table columns nsink/16 on)
+  int win_first;  // first position read from the fp16 window ring
+  int n_win;      // tokens read from the ring: positions win_first .. len - 1
+  int n_wchunk;   // 16-row chunks of those
+  int n_sink;     // tokens read from the sink rows: positions 0 .. n_sink - 1
+  int n_schunk;   // 16-row chunks of those
+  int win_cost;   // cost of all fp16 chunks
   int cost;
 };
 
-__device__ __forceinline__ UnitShape unit_shape(int len) {
+__device__ __forceinline__ UnitShape unit_shape(int len, int nsink) {
   UnitShape s;
   s.len = len;
-  s.n_int2 = len > kWin ? len - kWin : 0;
+  s.n_int2 = max(0, len - kWin - nsink);
   s.n_pages = (s.n_int2 + kBlock - 1) / kBlock;
-  s.n_win = len < kWin ? len : kWin;
+  s.win_first = max(max(len - kWin, 0), nsink);
+  s.n_win = max(0, len - s.win_first);
   s.n_wchunk = (s.n_win + kBlock - 1) / kBlock;
-  s.win_cost = s.n_wchunk * kWinCost;
+  s.n_sink = min(len, nsink);
+  s.n_schunk = (s.n_sink + kBlock - 1) / kBlock;
+  s.win_cost = (s.n_wchunk + s.n_schunk) * kWinCost;
   s.cost = s.n_pages + s.win_cost;
   return s;
 }
@@ -77,6 +86,7 @@ struct DecodeArgs {
   const float* u_v;
   const uint8_t* pages;
   const __half* ring;
+  const __half* sink;  // fp16 rows of the first nsink positions
   float* out;
   uint32_t* status;
   float* qrot;       // [B][Hq][128]
@@ -85,7 +95,7 @@ struct DecodeArgs {
   __half* qwin;      // [B][Hq][2][128]: q~/sigma as fp16 hi, lo (natural channel order)
   int32_t* prefix;   // [B+1] cost prefix over batch entries
   float* part;       // [(NC + B)][Hq][kPartStride]
-  int batch, hq, hkv, g, nc, num_blocks, num_slots, mbps;
+  int batch, hq, hkv, g, nc, num_blocks, num_slots, mbps, nsink;
 };
 
 // split-K CTA count actually used: with fewer cost units than CTAs only the
@@ -122,7 +132,7 @@ __device__ __forceinline__ void qrot_cta(const DecodeArgs& a, int cta) {
     const int per = (a.batch + kPrepThreads - 1) / kPrepThreads;
     const int lo = threadIdx.x * per, hi = min(a.batch, lo + per);
     int own = 0;
-    for (int i = lo; i < hi; ++i) own += unit_shape(clamp_len(a.context_lens, i, a.mbps, a.status, true)).cost;
+    for (int i = lo; i < hi; ++i) own += unit_shape(clamp_len(a.context_lens, i, a.mbps, a.status, true), a.nsink).cost;
     int inc = own;
 #pragma unroll
     for (int d = 1; d < 32; d <<= 1) {
@@ -140,7 +150,7 @@ __device__ __forceinline__ void qrot_cta(const DecodeArgs& a, int cta) {
     int run = before + inc - own;
     for (int i = lo; i < hi; ++i) {
       a.prefix[i] = run;
-      run += unit_shape(clamp_len(a.context_lens, i, a.mbps, a.status, false)).cost;
+      run += unit_shape(clamp_len(a.context_lens, i, a.mbps, a.status, false), a.nsink).cost;
     }
     if (threadIdx.x == 0) a.prefix[a.batch] = total;
   }
@@ -238,7 +248,10 @@ struct WarpState {
   float m[G], l[G], o[G][4];
 };
 
-template <int G, bool kWindow>
+// kWindow: fp16 rows of positions first_row + t of krow0 / vrow0: the window
+// ring (kRing, row = position % W) or the sink rows (row = position);
+// otherwise the INT2 block at blockp.
+template <int G, bool kWindow, bool kRing = true>
 __device__ __forceinline__ void simt_chunk(const DecodeArgs& a, const float* qs /*smem [G][128]*/,
                                            const uint8_t* blockp, const __half* krow0,
                                            const __half* vrow0, int win_first_row, int ntok,
@@ -266,7 +279,7 @@ __device__ __forceinline__ void simt_chunk(const DecodeArgs& a, const float* qs 
         }
       }
     } else {
-      const int row = (win_first_row + tt) % kWin;
+      const int row = kRing ? (win_first_row + tt) % kWin : win_first_row + tt;
       const __half* kr = krow0 + (size_t)row * kD + 64 * half;
 #pragma unroll 4
       for (int c8 = 0; c8 < 8; ++c8) {
@@ -311,7 +324,7 @@ __device__ __forceinline__ void simt_chunk(const DecodeArgs& a, const float* qs 
 #pragma unroll
       for (int j = 0; j < 4; ++j) x[j] = fmaf(s, (float)((byte >> (2 * j)) & 3u), m);
     } else {
-      const int row = (win_first_row + t) % kWin;
+      const int row = kRing ? (win_first_row + t) % kWin : win_first_row + t;
       const uint2 w = *reinterpret_cast<const uint2*>(vrow0 + (size_t)row * kD + 4 * lane);
       const float2 f0 = __half22float2(*reinterpret_cast<const __half2*>(&w.x));
       const float2 f1 = __half22float2(*reinterpret_cast<const __half2*>(&w.y));
@@ -349,7 +362,7 @@ __global__ void __launch_bounds__(kDecWarps * 32) decode_simt_kernel(DecodeArgs 
     if (a.prefix[mid] <= start) lo = mid; else hi = mid - 1;
   }
   for (int b = lo; b < a.batch && a.prefix[b] < end; ++b) {
-    const UnitShape us = unit_shape(clamp_len(a.context_lens, b, a.mbps, a.status, false));
+    const UnitShape us = unit_shape(clamp_len(a.context_lens, b, a.mbps, a.status, false), a.nsink);
     if (us.cost == 0) continue;
     const int slot = a.seq_slot[b];
     const bool slot_ok = slot >= 0 && slot < a.num_slots;
@@ -372,18 +385,24 @@ __global__ void __launch_bounds__(kDecWarps * 32) decode_simt_kernel(DecodeArgs 
         {
           const __half* kbase = a.ring + (((size_t)slot * a.hkv + hk) * 2 + 0) * kWin * kD;
           const __half* vbase = a.ring + (((size_t)slot * a.hkv + hk) * 2 + 1) * kWin * kD;
-          const int first = us.len - us.n_win;
+          const __half* ksink = a.sink + (((size_t)slot * a.hkv + hk) * 2 + 0) * a.nsink * kD;
+          const __half* vsink = a.sink + (((size_t)slot * a.hkv + hk) * 2 + 1) * a.nsink * kD;
           const int ci0 = (l0 + kWinCost - 1) / kWinCost;
-          const int ci1 = min(us.n_wchunk, (l1 + kWinCost - 1) / kWinCost);
+          const int ci1 = min(us.n_wchunk + us.n_schunk, (l1 + kWinCost - 1) / kWinCost);
           for (int ci = ci0 + warp; ci < ci1; ci += kDecWarps) {
-            const int ntok = min(kBlock, us.n_win - ci * kBlock);
-            simt_chunk<G, true>(a, qs, nullptr, kbase, vbase, first + ci * kBlock, ntok, st, lane);
+            if (ci < us.n_wchunk) {  // window positions win_first + 16 ci .. at ring rows pos % W
+              const int ntok = min(kBlock, us.n_win - ci * kBlock);
+              simt_chunk<G, true>(a, qs, nullptr, kbase, vbase, us.win_first + ci * kBlock, ntok, st, lane);
+            } else {  // sink positions 16 (ci - n_wchunk) .. at sink rows pos
+              const int f = (ci - us.n_wchunk) * kBlock;
+              simt_chunk<G, true, false>(a, qs, nullptr, ksink, vsink, f, min(kBlock, us.n_sink - f), st, lane);
+            }
           }
         }
         const int p0 = max(l0, us.win_cost) - us.win_cost;
         const int p1 = l1 - us.win_cost;
         for (int pi = p0 + warp; pi < p1; pi += kDecWarps) {
-          const int blk = a.block_table[(size_t)slot * a.mbps + pi];
+          const int blk = a.block_table[(size_t)slot * a.mbps + (a.nsink >> 4) + pi];
           if (blk < 0 || blk >= a.num_blocks) {
             if (lane == 0) raise_flag(a.status, OKV_DEV_BAD_BLOCK);
             continue;
@@ -623,7 +642,7 @@ __global__ void __launch_bounds__(kHW * 32, (G <= 4) ? 2 : 1) decode_heads_kerne
     const int per = (a.batch + blockDim.x - 1) / blockDim.x;
     const int i0 = threadIdx.x * per, i1 = min(a.batch, i0 + per);
     int own = 0;
-    for (int i = i0; i < i1; ++i) own += unit_shape(clamp_len_cg(a.context_lens, i, a.mbps)).cost;
+    for (int i = i0; i < i1; ++i) own += unit_shape(clamp_len_cg(a.context_lens, i, a.mbps), a.nsink).cost;
     int inc = own;
 #pragma unroll
     for (int d = 1; d < 32; d <<= 1) {
@@ -646,7 +665,7 @@ __global__ void __launch_bounds__(kHW * 32, (G <= 4) ? 2 : 1) decode_heads_kerne
       if ((int)blockIdx.x < ncw && st0 >= before && st0 < before + own) {
         int pu = before;
         for (int i = i0; i < i1; ++i) {
-          const int cst = unit_shape(clamp_len_cg(a.context_lens, i, a.mbps)).cost;
+          const int cst = unit_shape(clamp_len_cg(a.context_lens, i, a.mbps), a.nsink).cost;
           if (st0 < pu + cst) {
             part_first[0] = i;
             part_first[1] = pu;
@@ -690,7 +709,7 @@ __global__ void __launch_bounds__(kHW * 32, (G <= 4) ? 2 : 1) decode_heads_kerne
   bool waited = false;  // grid_dep_wait() done (the query rotation's outputs are readable)
   long long pnext = part_first[1];
   for (int b = part_first[0]; b < a.batch && pnext < end; ++b) {
-    const UnitShape us = unit_shape(clamp_len_cg(a.context_lens, b, a.mbps));
+    const UnitShape us = unit_shape(clamp_len_cg(a.context_lens, b, a.mbps), a.nsink);
     const long long pu = pnext;
     pnext += us.cost;
     if (us.cost == 0) continue;
@@ -705,7 +724,8 @@ __global__ void __launch_bounds__(kHW * 32, (G <= 4) ? 2 : 1) decode_heads_kerne
     const int p0 = max(l0, us.win_cost) - us.win_cost;
     const int p1 = l1 - us.win_cost;
     const int nst = (slot_ok && alive && p1 > p0) ? (p1 - p0 + nb - 1) / nb : 0;
-    const int32_t* trow = a.block_table + (size_t)(slot_ok ? slot : 0) * a.mbps;
+    // INT2 block pi of this entry is table column nsink/16 + pi
+    const int32_t* trow = a.block_table + (size_t)(slot_ok ? slot : 0) * a.mbps + (a.nsink >> 4);
 
     // Warp 0 fills the ring in batches of stages, one lane per block (lane
     // nb * i + q takes block q of the batch's stage i).  Stage j of this entry
@@ -1014,13 +1034,15 @@ __global__ void __launch_bounds__(kHW * 32, (G <= 4) ? 2 : 1) decode_heads_kerne
     for (int nt = 0; nt < NT; ++nt) mma_flush(st, acci, nt, inv);
     __syncthreads();  // every warp is done with the ring: it becomes window scratch, then merge buffers
 
-    // ---------------- fp16 window: chunks ci = grp, grp + wph, ... of this warp's head ----------------
-    // window chunks owned by this CTA: chunk ci where l0 <= ci * kWinCost < l1
+    // ---------------- fp16 rows: chunks ci = grp, grp + wph, ... of this warp's head ----------------
+    // fp16 chunks owned by this CTA: chunk ci where l0 <= ci * kWinCost < l1.
+    // Chunk ci < n_wchunk: window positions win_first + 16 ci .. (ring rows
+    // pos % W); then sink positions 16 (ci - n_wchunk) .. (sink rows pos).
+    const UnitShape& ws = us;
     const int ci0 = (l0 + kWinCost - 1) / kWinCost;
-    const int ci1 = slot_ok ? min(us.n_wchunk, (l1 + kWinCost - 1) / kWinCost) : ci0;
+    const int ci1 = slot_ok ? min(ws.n_wchunk + ws.n_schunk, (l1 + kWinCost - 1) / kWinCost) : ci0;
     if (ci0 + grp < ci1) {
-      const __half* kr = a.ring + (((size_t)slot * hkv + head) * 2 + 0) * kWin * kD;
-      const __half* vr = a.ring + (((size_t)slot * hkv + head) * 2 + 1) * kWin * kD;
+      const size_t kv_rows = ((size_t)slot * hkv + head) * 2;  // K rows of (slot, head); V rows follow
       unsigned char* scratch = ring + warp * kWarpScratch;
       unsigned char* tile = scratch;                                   // 16 rows x 256 B, swizzled
       float* pw = reinterpret_cast<float*>(scratch + 4096);            // [HP][16]
@@ -1051,21 +1073,27 @@ __global__ void __launch_bounds__(kHW * 32, (G <= 4) ? 2 : 1) decode_heads_kerne
 #pragma unroll
           for (int i = 0; i < 4; ++i) wacc[nt][mt][i] = 0.f;
       }
-      for (int ci = ci0 + grp; ci < ci1; ci += wph) {
-        const int r0 = 16 * ci;
+      // One 16-row fp16 chunk: rows of positions c_first + i (i < c_n) of the
+      // window ring (row = position % W) or of the sink rows (row = position),
+      // K rows from kr and V rows right after them.
+      auto fp16_chunk = [&](auto ring_tag, const __half* kr, int c_first, int c_n) {
+        constexpr bool kRing = decltype(ring_tag)::value;
+        const __half* vr = kr + (size_t)(kRing ? kWin : a.nsink) * kD;
+        auto row_of = [&](int i) { return kRing ? ((c_first + i) & (kWin - 1)) : c_first + i; };
         // stage the V rows (swizzled 16-byte chunks) for the transposing loads
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
           const int q = lane + 32 * k, row = q >> 4, col = q & 15;
           uint4 x = make_uint4(0, 0, 0, 0);
-          if (r0 + row < us.n_win) x = *reinterpret_cast<const uint4*>(vr + (size_t)(r0 + row) * kD + 8 * col);
+          if (row < c_n)
+            x = *reinterpret_cast<const uint4*>(vr + (size_t)row_of(row) * kD + 8 * col);
           *reinterpret_cast<uint4*>(tile + row * 256 + ((col ^ (row & 7)) << 4)) = x;
         }
-        // scores of ring rows r0 + g and r0 + g + 8
+        // scores of chunk rows g and g + 8
         uint32_t ka[16], kb[16];
-        const bool va_ = r0 + g < us.n_win, vb_ = r0 + g + 8 < us.n_win;
-        const uint4* ra = reinterpret_cast<const uint4*>(kr + (size_t)(r0 + g) * kD + 32 * t);
-        const uint4* rb = reinterpret_cast<const uint4*>(kr + (size_t)(r0 + g + 8) * kD + 32 * t);
+        const bool va_ = g < c_n, vb_ = g + 8 < c_n;
+        const uint4* ra = reinterpret_cast<const uint4*>(kr + (size_t)row_of(g) * kD + 32 * t);
+        const uint4* rb = reinterpret_cast<const uint4*>(kr + (size_t)row_of(g + 8) * kD + 32 * t);
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const uint4 x = va_ ? ra[i] : make_uint4(0, 0, 0, 0);
@@ -1132,6 +1160,15 @@ __global__ void __launch_bounds__(kHW * 32, (G <= 4) ? 2 : 1) decode_heads_kerne
           }
         }
         __syncwarp();
+      };
+      for (int ci = ci0 + grp; ci < ci1; ci += wph) {
+        if (ci < ws.n_wchunk) {
+          fp16_chunk(std::true_type{}, a.ring + kv_rows * kWin * kD, ws.win_first + 16 * ci,
+                     min(16, ws.n_win - 16 * ci));
+        } else {
+          const int f = 16 * (ci - ws.n_wchunk);
+          fp16_chunk(std::false_type{}, a.sink + kv_rows * a.nsink * kD, f, min(16, ws.n_sink - f));
+        }
       }
       // window o' per (head, channel) through shared memory, then fold into the block state
 #pragma unroll
@@ -1290,7 +1327,7 @@ __global__ void __launch_bounds__(kCombThreads) combine_kernel(DecodeArgs a) {
     cp_async_commit();
   }
   grid_dep_wait();  // the split partials (and the cost prefix) are read from here on
-  const UnitShape sh = unit_shape(clamp_len(a.context_lens, b, a.mbps, a.status, false));
+  const UnitShape sh = unit_shape(clamp_len(a.context_lens, b, a.mbps, a.status, false), a.nsink);
   const long long total = a.prefix[a.batch];
   float* outp = a.out + ((size_t)b * a.hq + head) * kD;
   if (sh.cost == 0 || total == 0) {
@@ -1475,6 +1512,8 @@ static DecodeArgs make_decode_args(const okv_cache_desc* d, const void* q, int B
   a.u_v = d->u_v;
   a.pages = (const uint8_t*)d->pages;
   a.ring = (const __half*)d->window_ring;
+  a.sink = (const __half*)d->sink_rows;
+  a.nsink = d->num_sink;
   a.out = out;
   a.status = d->status_word;
   uint8_t* w = (uint8_t*)ws;

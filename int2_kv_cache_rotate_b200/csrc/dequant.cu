@@ -15,10 +15,11 @@ struct DequantArgs {
   const int32_t* context_lens;
   const uint8_t* pages;
   const __half* ring;
+  const __half* sink;  // fp16 rows of the first nsink positions
   const float* u;  // U of `which`
   float* out;
   uint32_t* status;
-  int hkv, num_blocks, num_slots, mbps, max_ctx, which, basis, source;
+  int hkv, num_blocks, num_slots, mbps, max_ctx, which, basis, source, nsink;
 };
 
 // grid (ceil(max_ctx/32), Hkv, B), 128 threads; warp w handles tokens w, w+4, ...
@@ -47,8 +48,11 @@ __global__ void __launch_bounds__(128) dequant_kernel(DequantArgs a) {
     float z[4] = {0.f, 0.f, 0.f, 0.f};
     bool have = false;
     if (p < len && slot_ok) {
-      if (p >= first_fp16) {
-        const __half* row = a.ring + ((((size_t)slot * a.hkv + hk) * 2 + a.which) * kWin + (p % kWin)) * kD;
+      if (p >= first_fp16 || (a.source == 1 && p < a.nsink)) {
+        const __half* row =
+            p < a.nsink && a.source == 1
+                ? a.sink + ((((size_t)slot * a.hkv + hk) * 2 + a.which) * a.nsink + p) * kD
+                : a.ring + ((((size_t)slot * a.hkv + hk) * 2 + a.which) * kWin + (p % kWin)) * kD;
         const uint2 w = *reinterpret_cast<const uint2*>(row + 4 * lane);
         const float2 f0 = __half22float2(*reinterpret_cast<const __half2*>(&w.x));
         const float2 f1 = __half22float2(*reinterpret_cast<const __half2*>(&w.y));
@@ -106,6 +110,8 @@ okv_status launch_dequant(const okv_cache_desc* d, int B, const int32_t* seq_slo
   a.context_lens = context_lens;
   a.pages = (const uint8_t*)d->pages;
   a.ring = (const __half*)d->window_ring;
+  a.sink = (const __half*)d->sink_rows;
+  a.nsink = d->num_sink;
   a.u = which ? d->u_v : d->u_k;
   a.out = out;
   a.status = d->status_word;

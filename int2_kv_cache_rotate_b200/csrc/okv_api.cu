@@ -66,6 +66,11 @@ okv_status validate_desc(const okv_cache_desc* d) {
     return fail(OKV_ERR_INVALID_ARG, "pages, window_ring, u_k and u_v must be 16-byte aligned");
   if ((long long)d->max_blocks_per_seq * kBlock > 0x3fffffffLL)
     return fail(OKV_ERR_INVALID_ARG, "max_blocks_per_seq too large");
+  if (d->num_sink < 0 || d->num_sink > OKV_MAX_SINK || d->num_sink % kBlock != 0)
+    return fail(OKV_ERR_UNSUPPORTED, "num_sink must be a multiple of %d in [0, %d] (got %d)", kBlock, OKV_MAX_SINK,
+                d->num_sink);
+  if (d->num_sink > 0 && (d->sink_rows == nullptr || !aligned(d->sink_rows, 16)))
+    return fail(OKV_ERR_INVALID_ARG, "sink_rows must be a 16-byte aligned device buffer when num_sink > 0");
   return OKV_OK;
 }
 
@@ -135,6 +140,11 @@ size_t okv_pages_bytes(int32_t num_blocks, int32_t num_kv_heads) {
 size_t okv_window_bytes(int32_t num_seq_slots, int32_t num_kv_heads) {
   if (num_seq_slots < 0 || num_kv_heads < 0) return 0;
   return (size_t)num_seq_slots * num_kv_heads * 2 * kWin * kD * sizeof(__half);
+}
+
+size_t okv_sink_bytes(int32_t num_seq_slots, int32_t num_kv_heads, int32_t num_sink) {
+  if (num_seq_slots < 0 || num_kv_heads < 0 || num_sink < 0) return 0;
+  return (size_t)num_seq_slots * num_kv_heads * 2 * num_sink * kD * sizeof(__half);
 }
 
 okv_status okv_append_quantize(const okv_cache_desc* desc, const void* k, const void* v, int32_t T,

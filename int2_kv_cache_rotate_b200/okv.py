@@ -41,12 +41,13 @@ class CacheDesc(ctypes.Structure):
         ("num_blocks", ctypes.c_int32),
         ("num_seq_slots", ctypes.c_int32),
         ("max_blocks_per_seq", ctypes.c_int32),
-        ("reserved", ctypes.c_int32),
+        ("num_sink", ctypes.c_int32),
         ("pages", ctypes.c_void_p),
         ("window_ring", ctypes.c_void_p),
         ("u_k", ctypes.c_void_p),
         ("u_v", ctypes.c_void_p),
         ("status_word", ctypes.c_void_p),
+        ("sink_rows", ctypes.c_void_p),
     ]
 
 
@@ -62,6 +63,7 @@ _SIGNATURES = {
     "okv_calibrate_rotations": (_I32, [_P, _I64, _P, _P, _I64, _I32, _I32, _I32, _P, _P, _P, _P]),
     "okv_pages_bytes": (_SZ, [_I32, _I32]),
     "okv_window_bytes": (_SZ, [_I32, _I32]),
+    "okv_sink_bytes": (_SZ, [_I32, _I32, _I32]),
     "okv_append_quantize": (_I32, [_DESC, _P, _P, _I32, _P, _P, _P, _P, _U32, _P, _P]),
     "okv_decode_workspace_bytes": (_SZ, [_DESC, _I32]),
     "okv_decode_attention": (_I32, [_DESC, _P, _I32, _P, _P, _P, _P, _P, _SZ, _P]),
@@ -150,9 +152,9 @@ class Cache:
     receives pointers."""
 
     def __init__(self, hq: int, hkv: int, num_blocks: int, num_seq_slots: int, max_blocks_per_seq: int,
-                 u_k, u_v, device="cuda"):
+                 u_k, u_v, device="cuda", num_sink: int = 0):
         import torch
-        self.hq, self.hkv = hq, hkv
+        self.hq, self.hkv, self.num_sink = hq, hkv, num_sink
         self.num_blocks, self.num_seq_slots, self.max_blocks_per_seq = num_blocks, num_seq_slots, max_blocks_per_seq
         nbytes = lib().okv_pages_bytes(num_blocks, hkv)
         self.pages = torch.zeros(max(nbytes, 16), dtype=torch.uint8, device=device)
@@ -160,9 +162,13 @@ class Cache:
         self.u_k = torch.as_tensor(np.asarray(u_k, dtype=np.float32)).to(device).contiguous()
         self.u_v = torch.as_tensor(np.asarray(u_v, dtype=np.float32)).to(device).contiguous()
         self.status = torch.zeros(4, dtype=torch.int32, device=device)
+        # first num_sink positions of every sequence, fp16 (sink tokens)
+        self.sink = torch.zeros((num_seq_slots, hkv, 2, max(num_sink, 0), HEAD_DIM), dtype=torch.float16,
+                                device=device)
         self.desc = CacheDesc(hq, hkv, HEAD_DIM, HEAD_DIM, BLOCK_TOKENS, WINDOW, num_blocks, num_seq_slots,
-                              max_blocks_per_seq, 0, self.pages.data_ptr(), self.ring.data_ptr(),
-                              self.u_k.data_ptr(), self.u_v.data_ptr(), self.status.data_ptr())
+                              max_blocks_per_seq, num_sink, self.pages.data_ptr(), self.ring.data_ptr(),
+                              self.u_k.data_ptr(), self.u_v.data_ptr(), self.status.data_ptr(),
+                              self.sink.data_ptr() if num_sink > 0 else None)
 
     def device_status(self) -> int:
         return int(self.status[0].item())
