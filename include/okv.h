@@ -72,7 +72,10 @@ typedef enum {
   OKV_ERR_INVALID_ARG = 1,  /* bad pointer, size, alignment or shape      */
   OKV_ERR_UNSUPPORTED = 2,  /* valid but not implemented (d != 128, ...)  */
   OKV_ERR_CUDA = 3,         /* a CUDA runtime call or a launch failed     */
-  OKV_ERR_NUMERIC = 4,      /* the eigensolver did not converge           */
+  OKV_ERR_NUMERIC = 4,      /* the eigensolver did not converge, or a loaded
+                               rotation is not orthogonal                 */
+  OKV_ERR_IO = 5,           /* a file could not be opened, read or written,
+                               or is not a valid rotations file           */
 } okv_status;
 
 /* bits of *status_word written by the kernels */
@@ -126,6 +129,35 @@ typedef struct {
 okv_status okv_calibrate_rotations(const float* q, int64_t nq, const float* k, const float* v,
                                    int64_t nk, int32_t hq, int32_t hkv, int32_t d, float* r_k,
                                    float* r_v, float* u_k, float* u_v);
+
+/* Rotation files: U_K and U_V of every layer and KV head of a model, so that a
+ * deployment loads precomputed rotations instead of calibrating (gen-hub.ru,
+ * "Открытый код — это серьёзно": rotations are computed offline, once per
+ * model, and shipped; aiforradalom.hu, "OSCAR: figyelem-tudatos…": a set of
+ * precomputed rotations per supported model).  The pages give no format; this
+ * one is little-endian:
+ *   32-byte header: "OKVROTS1", u32 version (1), u32 d, u32 num_layers,
+ *   u32 num_kv_heads, u32 tag_len, u32 0;
+ *   tag_len bytes of tag (free text, e.g. the model name; at most 4096);
+ *   fp32 U_K [num_layers][num_kv_heads][d][d], fp32 U_V the same;
+ *   u64 FNV-1a (64-bit) of everything before it.
+ * Host buffers throughout; no CUDA call is made.
+ * okv_save_rotations: tag may be NULL.  Errors: INVALID_ARG (NULL, empty
+ *   shape, tag too long), UNSUPPORTED (d != 128), IO (open or write failed).
+ * okv_rotations_file_shape: reads the header; each output is nullable.
+ * okv_load_rotations: the shape must match the file's; tag (nullable)
+ *   receives the tag, truncated to tag_capacity - 1 bytes and NUL-terminated;
+ *   verify != 0 also checks max |U^T U - I| <= 1e-4 for every matrix.  Errors:
+ *   INVALID_ARG (NULL, shape mismatch), UNSUPPORTED (other format version), IO
+ *   (missing, truncated, trailing bytes, bad magic or checksum), NUMERIC
+ *   (verify failed).  On IO and NUMERIC errors u_k and u_v may have been
+ *   partly written. */
+okv_status okv_save_rotations(const char* path, int32_t num_layers, int32_t num_kv_heads, int32_t d,
+                              const float* u_k, const float* u_v, const char* tag);
+okv_status okv_rotations_file_shape(const char* path, int32_t* num_layers, int32_t* num_kv_heads, int32_t* d,
+                                    int32_t* tag_len);
+okv_status okv_load_rotations(const char* path, int32_t num_layers, int32_t num_kv_heads, int32_t d, float* u_k,
+                              float* u_v, char* tag, size_t tag_capacity, int32_t verify);
 
 /* Bytes the caller allocates for `pages`, `window_ring` and `sink_rows`. */
 size_t okv_pages_bytes(int32_t num_blocks, int32_t num_kv_heads);

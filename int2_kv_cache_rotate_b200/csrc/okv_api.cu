@@ -128,6 +128,7 @@ const char* okv_status_string(okv_status s) {
     case OKV_ERR_UNSUPPORTED: return "OKV_ERR_UNSUPPORTED";
     case OKV_ERR_CUDA: return "OKV_ERR_CUDA";
     case OKV_ERR_NUMERIC: return "OKV_ERR_NUMERIC";
+    case OKV_ERR_IO: return "OKV_ERR_IO";
   }
   return "unknown okv_status";
 }

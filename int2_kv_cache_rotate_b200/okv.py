@@ -18,7 +18,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libokv.so")
 HEADER = os.path.join(os.path.dirname(_HERE), "include", "okv.h")
 
-OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_NUMERIC = range(5)
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_NUMERIC, ERR_IO = range(6)
 DEV_BAD_BLOCK, DEV_BAD_POS, DEV_BAD_SLOT, DEV_TIMEOUT = 1, 2, 4, 8
 PRE_ROTATED = 1
 HEAD_DIM, BLOCK_TOKENS, WINDOW, BLOCK_HEAD_BYTES = 128, 16, 128, 1152
@@ -74,6 +74,9 @@ _SIGNATURES = {
     "okv_time_next_decode_kernel": (_I32, [_P, _P]),
     "okv_decode_attention_noalloc": (_I32, [_DESC, _P, _I32, _P, _P, _P, _P, _P]),
     "okv_decode_step": (_I32, [_DESC, _P, _P, _I32, _P, _P, _P, _P, _I32, _P, _P, _P, _P, _P, _SZ, _P]),
+    "okv_save_rotations": (_I32, [ctypes.c_char_p, _I32, _I32, _I32, _P, _P, ctypes.c_char_p]),
+    "okv_rotations_file_shape": (_I32, [ctypes.c_char_p, _P, _P, _P, _P]),
+    "okv_load_rotations": (_I32, [ctypes.c_char_p, _I32, _I32, _I32, _P, _P, _P, _SZ, _I32]),
 }
 
 
@@ -175,6 +178,34 @@ class Cache:
 
     def clear_status(self):
         self.status.zero_()
+
+
+def save_rotations(path, u_k, u_v, tag: str = "") -> None:
+    """Write U_K and U_V (host fp32 [layers][Hkv][128][128], or [Hkv][128][128]
+    for one layer) to a rotations file."""
+    uk = np.ascontiguousarray(u_k, dtype=np.float32)
+    uv = np.ascontiguousarray(u_v, dtype=np.float32)
+    if uk.ndim == 3:
+        uk, uv = uk[None], uv[None]
+    if uk.ndim != 4 or uv.shape != uk.shape or uk.shape[2] != uk.shape[3]:
+        raise ValueError(f"u_k {uk.shape} and u_v {uv.shape} must both be [layers][Hkv][d][d]")
+    layers, hkv, d, _ = uk.shape
+    _check(lib().okv_save_rotations(os.fsencode(path), layers, hkv, d, uk.ctypes.data, uv.ctypes.data,
+                                    tag.encode("utf-8")))
+
+
+def load_rotations(path, verify: bool = True) -> dict:
+    """Read a rotations file: {"U_K", "U_V": fp32 [layers][Hkv][d][d], "tag": str}."""
+    p = os.fsencode(path)
+    layers, hkv, d, tag_len = (ctypes.c_int32() for _ in range(4))
+    _check(lib().okv_rotations_file_shape(p, ctypes.byref(layers), ctypes.byref(hkv), ctypes.byref(d),
+                                          ctypes.byref(tag_len)))
+    shape = (layers.value, hkv.value, d.value, d.value)
+    uk, uv = np.empty(shape, np.float32), np.empty(shape, np.float32)
+    tag = ctypes.create_string_buffer(tag_len.value + 1)
+    _check(lib().okv_load_rotations(p, layers.value, hkv.value, d.value, uk.ctypes.data, uv.ctypes.data, tag,
+                                    tag_len.value + 1, int(verify)))
+    return {"U_K": uk, "U_V": uv, "tag": tag.value.decode("utf-8")}
 
 
 def append_quantize(cache: Cache, k, v, seq_slot, pos, block_table, slot_lens, pre_rotated=False,

@@ -34,6 +34,8 @@ def test_status_strings_and_sizes():
     assert lib.okv_status_string(2) == b"OKV_ERR_UNSUPPORTED"
     assert lib.okv_pages_bytes(10, 8) == 10 * 8 * 1152
     assert lib.okv_window_bytes(3, 8) == 3 * 8 * 2 * 128 * 128 * 2
+    assert lib.okv_sink_bytes(3, 8, 192) == 3 * 8 * 2 * 192 * 128 * 2
+    assert lib.okv_status_string(5) == b"OKV_ERR_IO"
 
 
 def test_validation_before_launch():
@@ -51,6 +53,16 @@ def test_validation_before_launch():
     d = _desc(num_q_heads=30)
     assert lib.okv_append_quantize(ctypes.byref(d), fake, fake, 1, fake, fake, fake, fake, 0, None, None) \
         == okv.ERR_INVALID_ARG
+    # sink count: a multiple of 16 up to 1024, with a 16-byte aligned buffer
+    for ns in (8, 1040, -16):
+        d = _desc(num_sink=ns, sink_rows=1 << 16)
+        assert lib.okv_append_quantize(ctypes.byref(d), fake, fake, 1, fake, fake, fake, fake, 0, None, None) \
+            == okv.ERR_UNSUPPORTED, ns
+    for rows in (None, (1 << 16) + 8):
+        d = _desc(num_sink=32, sink_rows=rows)
+        assert lib.okv_decode_attention(ctypes.byref(d), fake, 4, fake, fake, fake, fake, fake, 1 << 30, None) \
+            == okv.ERR_INVALID_ARG
+        assert b"sink_rows" in lib.okv_last_error_string()
     # misaligned pages
     d = _desc(pages=4097)
     assert lib.okv_append_quantize(ctypes.byref(d), fake, fake, 1, fake, fake, fake, fake, 0, None, None) \
