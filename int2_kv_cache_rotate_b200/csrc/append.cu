@@ -600,7 +600,8 @@ okv_status launch_append(const okv_cache_desc* d, const void* k, const void* v, 
   const AppendArgs a = make_append_args(d, k, v, seq_slot, pos, block_table, slot_lens, rotated_out);
   const bool rows16 = (((uintptr_t)k | (uintptr_t)v) & 15u) == 0;  // the tile loads copy 16-byte chunks
   if (!(flags & OKV_PRE_ROTATED) && T >= kTcMinTokens && rows16) {
-    cudaError_t e = cudaFuncSetAttribute(append_umma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kUmSmem);
+    static std::atomic<uint32_t> attr_set{0};
+    cudaError_t e = set_smem_limit_once((const void*)append_umma_kernel, (int)kUmSmem, attr_set);
     if (e != cudaSuccess) return fail(OKV_ERR_CUDA, "append smem attribute: %s", cudaGetErrorString(e));
     const int pairs = 2 * d->num_kv_heads;
     const int tiles = (T + kUmTile - 1) / kUmTile;
@@ -610,8 +611,8 @@ okv_status launch_append(const okv_cache_desc* d, const void* k, const void* v, 
     return check_launch("append (tcgen05)");
   }
   if (!(flags & OKV_PRE_ROTATED) && T >= kTcMinTokens) {
-    // set on every call: the attribute belongs to the current device's context
-    cudaError_t e = cudaFuncSetAttribute(append_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kTcSmem);
+    static std::atomic<uint32_t> attr_set{0};
+    cudaError_t e = set_smem_limit_once((const void*)append_tc_kernel, (int)kTcSmem, attr_set);
     if (e != cudaSuccess) return fail(OKV_ERR_CUDA, "append smem attribute: %s", cudaGetErrorString(e));
     // about two CTAs per SM over all (KV head, K|V) pairs; each CTA takes whole rounds
     const int pairs = 2 * d->num_kv_heads;

@@ -1454,8 +1454,8 @@ __global__ void __launch_bounds__(kCombThreads) combine_kernel(DecodeArgs a) {
 template <int G>
 static okv_status launch_decode_simt(const DecodeArgs& a, cudaStream_t s) {
   const size_t smem = (size_t)(G * kD + kDecWarps * G * kD + kDecWarps * G * 2) * sizeof(float);
-  cudaError_t e = cudaFuncSetAttribute(decode_simt_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)smem);
+  static std::atomic<uint32_t> attr_set{0};
+  cudaError_t e = set_smem_limit_once((const void*)decode_simt_kernel<G>, (int)smem, attr_set);
   if (e != cudaSuccess) return fail(OKV_ERR_CUDA, "decode smem attribute: %s", cudaGetErrorString(e));
   decode_simt_kernel<G><<<a.nc, kDecWarps * 32, smem, s>>>(a);
   return check_launch("decode");
@@ -1483,8 +1483,8 @@ static cudaError_t launch_pdl(void (*kernel)(Args...), dim3 grid, dim3 block, si
 template <int G>
 static okv_status launch_decode_heads(const DecodeArgs& a, cudaStream_t s, bool early) {
   const size_t smem = HCfg<G>::smem_bytes();
-  cudaError_t e = cudaFuncSetAttribute(decode_heads_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)smem);
+  static std::atomic<uint32_t> attr_set{0};
+  cudaError_t e = set_smem_limit_once((const void*)decode_heads_kernel<G>, (int)smem, attr_set);
   if (e != cudaSuccess) return fail(OKV_ERR_CUDA, "decode smem attribute: %s", cudaGetErrorString(e));
   e = launch_pdl(decode_heads_kernel<G>, dim3(a.nc), dim3(kHW * 32), smem, s, early, a);
   if (e != cudaSuccess) return fail(OKV_ERR_CUDA, "decode launch: %s", cudaGetErrorString(e));
@@ -1566,7 +1566,8 @@ static okv_status launch_decode_tail(const DecodeArgs& a, int B, cudaStream_t s)
   if (st != OKV_OK) return st;
   if (ev1 != nullptr && cudaEventRecordWithFlags(ev1, s, cudaEventRecordExternal) != cudaSuccess)
     return fail(OKV_ERR_CUDA, "cudaEventRecord failed");
-  cudaError_t e = cudaFuncSetAttribute(combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kCombSmem);
+  static std::atomic<uint32_t> attr_set{0};
+  cudaError_t e = set_smem_limit_once((const void*)combine_kernel, (int)kCombSmem, attr_set);
   if (e != cudaSuccess) return fail(OKV_ERR_CUDA, "combine smem attribute: %s", cudaGetErrorString(e));
   e = launch_pdl(combine_kernel, dim3(B * a.hq), dim3(kCombThreads), kCombSmem, s, early && tc, a);
   if (e != cudaSuccess) return fail(OKV_ERR_CUDA, "combine launch: %s", cudaGetErrorString(e));

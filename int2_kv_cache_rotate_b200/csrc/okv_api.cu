@@ -39,10 +39,24 @@ okv_status check_launch(const char* what) {
 }
 
 int device_sm_count() {
+  static std::atomic<int> cached[32];  // per device ordinal; 0 = not read yet
   int dev = 0, sms = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (dev >= 0 && dev < 32 && (sms = cached[dev].load(std::memory_order_relaxed)) > 0) return sms;
   if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  if (dev >= 0 && dev < 32) cached[dev].store(sms, std::memory_order_relaxed);
   return sms;
+}
+
+cudaError_t set_smem_limit_once(const void* kernel, int bytes, std::atomic<uint32_t>& done) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const uint32_t bit = (dev >= 0 && dev < 32) ? (1u << dev) : 0u;
+  if (bit != 0u && (done.load(std::memory_order_acquire) & bit) != 0u) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && bit != 0u) done.fetch_or(bit, std::memory_order_release);
+  return e;
 }
 
 static bool aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }

@@ -1,6 +1,7 @@
 // Host-side declarations shared by the library's translation units.
 #pragma once
 
+#include <atomic>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -14,6 +15,12 @@ okv_status fail(okv_status s, const char* fmt, ...);
 okv_status check_launch(const char* what);
 okv_status validate_desc(const okv_cache_desc* d);
 int device_sm_count();
+
+// Sets a kernel's dynamic shared-memory limit once per device (bit d of
+// `done` records device d < 32; higher ordinals set it on every call).  The
+// attribute belongs to the device's context, so a context reset would need
+// it set again: the library assumes contexts live as long as the process.
+cudaError_t set_smem_limit_once(const void* kernel, int bytes, std::atomic<uint32_t>& done);
 // events set by okv_time_next_decode_kernel (consumed by the next decode launch)
 void take_decode_events(cudaEvent_t* start, cudaEvent_t* stop);
 

@@ -269,6 +269,39 @@ def decode_step(cache: Cache, k, v, new_seq_slot, new_pos, slot_lens, q, seq_slo
     return out
 
 
+class DecodeStepCall:
+    """okv_decode_step prepared once for fixed buffers: the arguments are
+    checked and marshalled here, and each call only invokes the library, for
+    serving loops that refill the same input tensors every step.  The tensors
+    must stay alive, and their shapes, for as long as the object is used."""
+
+    def __init__(self, cache: Cache, k, v, new_seq_slot, new_pos, slot_lens, q, seq_slot, block_table,
+                 context_lens, out=None, ws=None, stream=None):
+        import torch
+        _need(k, torch.bfloat16, "k"), _need(v, torch.bfloat16, "v"), _need(q, torch.bfloat16, "q")
+        for name, t in (("new_seq_slot", new_seq_slot), ("new_pos", new_pos), ("slot_lens", slot_lens),
+                        ("seq_slot", seq_slot), ("block_table", block_table), ("context_lens", context_lens)):
+            _need(t, torch.int32, name)
+        B = q.shape[0]
+        if out is None:
+            out = torch.empty((B, cache.hq, HEAD_DIM), dtype=torch.float32, device=q.device)
+        _need(out, torch.float32, "out")
+        if ws is None:
+            ws = workspace(cache, B)
+        self.out, self._keep = out, (cache, k, v, new_seq_slot, new_pos, slot_lens, q, seq_slot, block_table,
+                                      context_lens, ws)
+        self._fn = lib().okv_decode_step
+        self._args = (ctypes.byref(cache.desc), _ptr(k), _ptr(v), k.shape[0], _ptr(new_seq_slot), _ptr(new_pos),
+                      _ptr(slot_lens), _ptr(q), B, _ptr(seq_slot), _ptr(block_table), _ptr(context_lens), _ptr(out),
+                      _ptr(ws), ws.numel(), _stream(stream))
+
+    def __call__(self):
+        status = self._fn(*self._args)
+        if status != OK:
+            _check(status)
+        return self.out
+
+
 def decode_attention_noalloc(cache: Cache, q, seq_slot, block_table, context_lens, out=None, stream=None):
     """Decode attention with the library's static scratch (no workspace, no allocation in the library)."""
     import torch
