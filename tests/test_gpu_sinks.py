@@ -181,3 +181,60 @@ def test_dequantize_as_decode_reads_it_with_sinks():
                 assert np.array_equal(rot[b, h, :n], O.dequantize(st["codes"][:n], st["s16"][:n], st["m16"][:n]))
                 assert np.array_equal(seen[b, h, :n], oc.values(b, which, h, n).astype(np.float32))
                 assert np.all(seen[b, h, n:] == 0)
+
+
+@pytest.mark.parametrize("nsink", [0, 32])
+def test_prefix_shared_pages(nsink):
+    """Two sequences share the physical INT2 blocks of a common prefix (their
+    block tables point at the same blocks), as a prefix cache forks a prompt;
+    each then appends its own suffix into its own blocks.  The prefix is
+    appended once; the fork's sink rows (per-sequence fp16) are filled by
+    appending its first S tokens again, which rewrites identical codes into
+    the shared blocks.  Both decode within 2e-3 of the oracle, and the shared
+    blocks are left unchanged by the suffixes."""
+    okv = _okv()
+    seed, hq, hkv = 46, 32, 8
+    prefix, suffix = 1024, [600, 300]  # prefix: 64 whole blocks
+    G = hq // hkv
+    lens = [prefix + s for s in suffix]
+    nblk = [(n + 15) // 16 for n in lens]
+    shared = prefix // 16
+    rng = np.random.default_rng(seed)
+    perm = rng.permutation(shared + sum(n - shared for n in nblk) + 3).astype(np.int32)
+    table = np.full((2, max(nblk)), -1, np.int32)
+    table[:, :shared] = perm[:shared]
+    off = shared
+    for b, n in enumerate(nblk):
+        table[b, shared:n] = perm[off:off + n - shared]
+        off += n - shared
+    uk, uv = H.rotations(seed, hkv)
+    gc = okv.Cache(hq, hkv, len(perm), 2, table.shape[1], uk, uv, num_sink=nsink)
+    oc = O.Cache(hkv, uk.astype(np.float64), uv.astype(np.float64), sinks=nsink)
+    zp = {kind: np.stack([WL.sample_rotated(seed, 0, 0, h, prefix, kind) for h in range(hkv)], 1) for kind in (0, 1)}
+    zs = {(b, kind): np.stack([WL.sample_rotated(seed, 0, 0, h, n, kind, extra=1 + b) for h in range(hkv)], 1)
+          for b, n in enumerate(suffix) for kind in (0, 1)}
+    lens_d, table_d = _t(np.array(lens, np.int32)), _t(table)
+
+    def app(slot, p0, zk, zv):
+        n = zk.shape[0]
+        okv.append_quantize(gc, _t(zk), _t(zv), _t(np.full(n, slot, np.int32)),
+                            _t(np.arange(p0, p0 + n, dtype=np.int32)), table_d, lens_d, pre_rotated=True)
+
+    app(0, 0, zp[0], zp[1])                      # the prefix, once, through sequence 0
+    if nsink:
+        app(1, 0, zp[0][:nsink], zp[1][:nsink])  # the fork's own sink rows
+    torch.cuda.synchronize()
+    shared_before = gc.pages.view(len(perm), hkv * 1152)[torch.from_numpy(table[0, :shared]).long().cuda()].clone()
+    for b in range(2):
+        app(b, prefix, zs[(b, 0)], zs[(b, 1)])
+        oc.append(b, 0, zp[0], zp[1], pre_rotated=True)
+        oc.append(b, prefix, zs[(b, 0)], zs[(b, 1)], pre_rotated=True)
+    torch.cuda.synchronize()
+    shared_after = gc.pages.view(len(perm), hkv * 1152)[torch.from_numpy(table[0, :shared]).long().cuda()]
+    assert torch.equal(shared_before, shared_after)
+    q = np.stack([WL.sample_queries(seed, 0, 0, h, 2, G, extra=9) for h in range(hkv)], 1).reshape(2, hq, 128)
+    seq = np.arange(2, dtype=np.int32)
+    got = okv.decode_attention(gc, _t(q, torch.bfloat16), _t(seq), table_d, lens_d).cpu().numpy()
+    want = O.decode(oc, q, seq, lens, hq)
+    assert gc.device_status() == 0
+    assert H.rel_err_rows(got, want).max() <= TOL
