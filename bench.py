@@ -404,10 +404,14 @@ def run_ours(args):
         dist.barrier()
     assert w["cache"].device_status() == 0, w["cache"].device_status()
 
-    # end to end through the public calls: each step's inputs (k, v, q,
-    # positions, lengths) packed in pinned host memory, one host-to-device copy
-    # into a staging buffer whose views a prepared okv_decode_step reads, and
-    # the output read back
+    # end to end through the public calls, as a serving loop runs them: each
+    # step's inputs (k, v, q, positions, lengths) packed in pinned host memory
+    # and sent with one host-to-device copy into one of two staging buffers; a
+    # prepared okv_decode_step (replayed from a CUDA graph after its first
+    # call) reads that buffer's views; its output is read back to pinned host
+    # memory.  The copies run on a copy stream, so that step i + 1's inputs
+    # and step i's output move while the GPU computes; events keep each
+    # buffer from being reused before the step that reads it has finished.
     e2e = None
     if e2e_steps:
         parts = [w["knew"], w["vnew"], w["q"], w["pos"], w["lens"]]  # each [steps][...]
@@ -417,31 +421,71 @@ def run_ours(args):
         host = torch.zeros((total, step_bytes), dtype=torch.uint8).pin_memory()
         for j, x in enumerate(parts):
             host[:, offs[j]:offs[j] + sizes[j]] = x.cpu().contiguous().view(total, -1).view(torch.uint8)
-        dev = torch.empty(step_bytes, dtype=torch.uint8, device="cuda")
-        views = [dev[offs[j]:offs[j] + sizes[j]].view(x.dtype).view(x[0].shape) for j, x in enumerate(parts)]
-        dk, dv, dq, dpos, dlen = views
-        hout = torch.empty((B, hq, 128), dtype=torch.float32).pin_memory()
+        hout = torch.empty((2, B, hq, 128), dtype=torch.float32).pin_memory()
         c = w["cache"]
-        call = okv.DecodeStepCall(c, dk, dv, w["seq"], dpos, dlen, dq, w["seq"], w["table"], dlen, out=out, ws=ws)
+        devs, outs, calls = [], [], []
+        for slot in range(2):
+            dev = torch.empty(step_bytes, dtype=torch.uint8, device="cuda")
+            dk, dv, dq, dpos, dlen = [dev[offs[j]:offs[j] + sizes[j]].view(x.dtype).view(x[0].shape)
+                                      for j, x in enumerate(parts)]
+            o = torch.empty((B, hq, 128), dtype=torch.float32, device="cuda")
+            devs.append(dev)
+            outs.append(o)
+            calls.append(okv.DecodeStepCall(c, dk, dv, w["seq"], dpos, dlen, dq, w["seq"], w["table"], dlen,
+                                            out=o, ws=ws, graph=True))
         base = W + K
+        # first call of each (eager, then recorded): step base - 1 again, which the
+        # graphs above already appended (same token, same position: the same bytes)
+        for slot in range(2):
+            devs[slot].copy_(host[base - 1], non_blocking=True)
+            calls[slot]()
+        torch.cuda.synchronize()
+        main, copy = torch.cuda.current_stream(), torch.cuda.Stream()
+        ev = lambda: torch.cuda.Event()
+        inputs_in = [ev(), ev()]    # staging buffer filled
+        step_done = [ev(), ev()]    # the step that read the buffer (and wrote the output) has finished
+        output_out = [ev(), ev()]   # output copied to the host
         if world > 1:
             dist.barrier()
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
+        e0.record(main)
+        copy.wait_stream(main)
+
+        def upload(i):
+            slot = i % 2
+            with torch.cuda.stream(copy):
+                if i - 2 >= base:
+                    copy.wait_event(step_done[slot])  # step i - 2 no longer reads this buffer
+                devs[slot].copy_(host[i], non_blocking=True)
+                inputs_in[slot].record(copy)
+
+        upload(base)
         for i in range(base, base + e2e_steps):
-            dev.copy_(host[i], non_blocking=True)
-            call()
-            hout.copy_(out, non_blocking=True)
-        e1.record()
+            slot = i % 2
+            if i + 1 < base + e2e_steps:
+                upload(i + 1)
+            main.wait_event(inputs_in[slot])
+            if i - 2 >= base:
+                main.wait_event(output_out[slot])  # step i - 2's output has left this buffer
+            calls[slot]()
+            step_done[slot].record(main)
+            with torch.cuda.stream(copy):
+                copy.wait_event(step_done[slot])
+                hout[slot].copy_(outs[slot], non_blocking=True)
+                output_out[slot].record(copy)
+        main.wait_stream(copy)
+        e1.record(main)
         torch.cuda.synchronize()
         e_ms = job_time_ms(e0.elapsed_time(e1), world, dist, "cuda")
         e_units = job_units(B * e2e_steps, world, dist, "cuda")
         e2e = {"value": round(e_units / (e_ms * 1e-3), 2), "unit": "tok/s",
-               "h2d_bytes_per_step": int(sum(sizes)), "d2h_bytes_per_step": int(hout.numel() * 4),
+               "h2d_bytes_per_step": int(sum(sizes)), "d2h_bytes_per_step": int(hout[0].numel() * 4),
                "ms_per_step": round(e_ms / e2e_steps, 4),
-               "timed_as": "eager calls, one per step: one packed host-to-device copy, a prepared "
-                           "okv_decode_step, one device-to-host copy of the output"}
+               "timed_as": "one step at a time, as a serving loop: one packed host-to-device copy of the "
+                           "step's inputs and one device-to-host copy of its output on a copy stream "
+                           "(double-buffered, overlapping the neighbouring steps' kernels), the prepared "
+                           "okv_decode_step replayed from its CUDA graph"}
 
     append_rate = prefill_append_rate(torch, okv, WL, args.seed) if rank == 0 else None
 

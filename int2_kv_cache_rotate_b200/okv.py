@@ -273,10 +273,13 @@ class DecodeStepCall:
     """okv_decode_step prepared once for fixed buffers: the arguments are
     checked and marshalled here, and each call only invokes the library, for
     serving loops that refill the same input tensors every step.  The tensors
-    must stay alive, and their shapes, for as long as the object is used."""
+    must stay alive, and their shapes, for as long as the object is used.
+
+    graph=True: the first call runs eagerly and then records the step's three
+    launches in a CUDA graph; later calls replay it (one launch per step)."""
 
     def __init__(self, cache: Cache, k, v, new_seq_slot, new_pos, slot_lens, q, seq_slot, block_table,
-                 context_lens, out=None, ws=None, stream=None):
+                 context_lens, out=None, ws=None, stream=None, graph: bool = False):
         import torch
         _need(k, torch.bfloat16, "k"), _need(v, torch.bfloat16, "v"), _need(q, torch.bfloat16, "q")
         for name, t in (("new_seq_slot", new_seq_slot), ("new_pos", new_pos), ("slot_lens", slot_lens),
@@ -291,14 +294,33 @@ class DecodeStepCall:
         self.out, self._keep = out, (cache, k, v, new_seq_slot, new_pos, slot_lens, q, seq_slot, block_table,
                                       context_lens, ws)
         self._fn = lib().okv_decode_step
+        self._stream = stream
         self._args = (ctypes.byref(cache.desc), _ptr(k), _ptr(v), k.shape[0], _ptr(new_seq_slot), _ptr(new_pos),
                       _ptr(slot_lens), _ptr(q), B, _ptr(seq_slot), _ptr(block_table), _ptr(context_lens), _ptr(out),
-                      _ptr(ws), ws.numel(), _stream(stream))
+                      _ptr(ws), ws.numel())
+        self._want_graph, self._graph = graph, None
 
     def __call__(self):
-        status = self._fn(*self._args)
+        import torch
+        if self._graph is not None:
+            if self._stream is None:
+                self._graph.replay()
+            else:
+                with torch.cuda.stream(self._stream):
+                    self._graph.replay()
+            return self.out
+        status = self._fn(*self._args, _stream(self._stream))
         if status != OK:
             _check(status)
+        if self._want_graph:
+            # record the same call (the library allocates nothing and only launches)
+            cap = torch.cuda.Stream()
+            cap.wait_stream(torch.cuda.current_stream() if self._stream is None else self._stream)
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=cap):
+                status = self._fn(*self._args, cap.cuda_stream)
+            _check(status)
+            self._graph = g
         return self.out
 
 

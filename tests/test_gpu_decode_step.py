@@ -56,9 +56,11 @@ def test_decode_step_equals_append_then_decode(hq, hkv, n_new):
     assert caches[1].device_status() == 0
 
 
-def test_prepared_call_equals_decode_step_over_several_steps():
-    """DecodeStepCall (arguments marshalled once, inputs refilled in place)
-    leaves the same cache bytes and outputs as okv.decode_step, step by step."""
+@pytest.mark.parametrize("graph", [False, True])
+def test_prepared_call_equals_decode_step_over_several_steps(graph):
+    """DecodeStepCall (arguments marshalled once, inputs refilled in place;
+    eager, or replayed from a CUDA graph after its first call) leaves the same
+    cache bytes and outputs as okv.decode_step, step by step."""
     from int2_kv_cache_rotate_b200 import okv
     seed, hq, hkv = 52, 32, 8
     base = [900, 300, 130]
@@ -77,7 +79,7 @@ def test_prepared_call_equals_decode_step_over_several_steps():
     kd = torch.empty((B, hkv, 128), dtype=torch.bfloat16, device="cuda")
     vd, qd = torch.empty_like(kd), torch.empty((B, hq, 128), dtype=torch.bfloat16, device="cuda")
     pd, ld = torch.empty(B, dtype=torch.int32, device="cuda"), torch.empty(B, dtype=torch.int32, device="cuda")
-    call = okv.DecodeStepCall(caches[1], kd, vd, seq, pd, ld, qd, seq, table, ld)
+    call = okv.DecodeStepCall(caches[1], kd, vd, seq, pd, ld, qd, seq, table, ld, graph=graph)
     for i in range(steps):
         k = np.stack([np.stack([WL.sample_keys(seed, 0, 0, h, 1, extra=20 + 10 * i + b)[0] for h in range(hkv)])
                       for b in range(B)])
