@@ -2,7 +2,11 @@
 // to INT2 with fp16 scale/min, pack, and write the paged cache and fp16 window.
 // Decode steps (a few tokens) run the CUDA-core kernel; prefill chunks of 128
 // tokens or more run the tensor-core kernel.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include <algorithm>
+#include <mutex>
 
 #include "append_warp.cuh"
 #include "okv_common.cuh"
@@ -249,11 +253,12 @@ __global__ void __launch_bounds__(kTcWarps * 32, 2) append_tc_kernel(AppendArgs 
 // 128-token tile of k for this KV head in the same layout (two K-blocks).
 //
 // Roles (warp-specialised):
-//   warp 8      producer: zero-filling async copies of A tiles into a 3-stage
-//               ring (one copy group per tile); once a tile's group is in,
-//               every lane fences it for the async proxy and one lane issues
-//               the 24 MMAs (M = N = 128, K = 16) into TMEM buffer i & 1,
-//               committed to mma_done[i & 1];
+//   warp 8      producer: one lane loads each A tile with two TMA tensor
+//               copies (channels 0-63 and 64-127, the hardware applying the
+//               128-byte swizzle; rows past T are filled with zeros) into a
+//               3-stage ring, completing on afull[stage]; once a tile is in,
+//               it issues the 24 MMAs (M = N = 128, K = 16) into TMEM buffer
+//               i & 1, committed to mma_done[i & 1];
 //   warps 0-3   epilogue of even tiles, warps 4-7 of odd tiles: warp w reads
 //               TMEM lanes 32 (w % 4) .. +31, one token per thread, all 128
 //               columns; it frees the TMEM buffer (tmem_free) as soon as the
@@ -268,7 +273,8 @@ constexpr int kUmStages = 3;
 constexpr uint32_t kUmRegion = 16384;                 // 128 rows x 128 B
 constexpr uint32_t kUmBBytes = 6 * kUmRegion;         // 3 parts x 2 K-blocks
 constexpr uint32_t kUmABytes = 2 * kUmRegion;         // one tile, 2 K-blocks
-constexpr uint32_t kUmCtlBytes = 64;                  // barriers and the TMEM base
+constexpr uint32_t kUmCtlBytes = 64;                  // 7 barriers and the TMEM base
+static_assert(7 * 8 + 4 <= kUmCtlBytes, "control region");
 constexpr size_t kUmSmem = 1024 + kUmBBytes + kUmStages * kUmABytes + kUmCtlBytes;
 constexpr uint32_t kUmTmemCols = 256;
 // instruction descriptor: D f32, A and B bf16, both K-major, N = 128, M = 128
@@ -289,8 +295,14 @@ __device__ __forceinline__ uint64_t um_desc(uint32_t saddr) {
   return d;
 }
 
-__device__ __forceinline__ void um_cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+// TMA tiled load of a 3-D box at (x, y, z) into shared memory, completing on bar
+__device__ __forceinline__ void um_tma_load_3d(uint32_t dst, const CUtensorMap* map, int x, int y, int z,
+                                               uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], "
+      "[%5];\n" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
+      : "memory");
 }
 __device__ __forceinline__ void um_fence_proxy_async() {
   asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
@@ -331,7 +343,9 @@ __device__ __forceinline__ void um_ld32(uint32_t taddr, float* v) {
 
 __device__ __forceinline__ void um_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory"); }
 
-__global__ void __launch_bounds__(kUmThreads, 1) append_umma_kernel(AppendArgs a, int T) {
+__global__ void __launch_bounds__(kUmThreads, 1) append_umma_kernel(AppendArgs a, int T,
+                                                                     const __grid_constant__ CUtensorMap map_k,
+                                                                     const __grid_constant__ CUtensorMap map_v) {
   extern __shared__ unsigned char um_raw[];
   const uint32_t raw_u32 = smem_u32(um_raw);
   const uint32_t base = (raw_u32 + 1023u) & ~1023u;  // swizzle atoms need 1024-byte alignment
@@ -340,45 +354,43 @@ __global__ void __launch_bounds__(kUmThreads, 1) append_umma_kernel(AppendArgs a
   unsigned char* ctl = gbase + kUmBBytes + kUmStages * kUmABytes;
   uint64_t* mma_done = reinterpret_cast<uint64_t*>(ctl);  // [2], one commit
   uint64_t* tmem_free = mma_done + 2;                    // [2], 128 arrivals (an epilogue warpgroup)
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tmem_free + 2);
+  uint64_t* afull = tmem_free + 2;                       // [3], one arrival + the tile's bytes
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(afull + kUmStages);
 
   const int h = blockIdx.y, kind = blockIdx.z;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int n_tiles_all = (T + kUmTile - 1) / kUmTile;
   const int n = n_tiles_all > (int)blockIdx.x ? (n_tiles_all - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
   if (n == 0) return;  // before any TMEM allocation
-  const __nv_bfloat16* src = (const __nv_bfloat16*)(kind ? a.v : a.k);
+  const CUtensorMap* map = kind ? &map_v : &map_k;  // [T][Hkv][128] bf16, boxes of 128 tokens x 64 channels
   auto tile_of = [&](int i) { return (int)blockIdx.x + i * (int)gridDim.x; };
 
-  // producer lane: its 64 chunks of tile i into stage i % 3, as one copy group
+  // producer lane 0: tile i of this KV head into stage i % 3 (both K-blocks)
   auto load_tile = [&](int i) {
-    const int t0 = tile_of(i) * kUmTile;
-    const uint32_t abuf = sA + (uint32_t)(i % kUmStages) * kUmABytes;
-#pragma unroll 8
-    for (int k = 0; k < 64; ++k) {
-      const int id = lane + 32 * k;
-      const int r = id >> 4, j = id & 15;
-      const int tok = t0 + r;
-      const bool ok = tok < T;
-      const __nv_bfloat16* g = src + ((size_t)(ok ? tok : 0) * a.hkv + h) * kD + 8 * j;
-      um_cp_async16(abuf + (uint32_t)(j >> 3) * kUmRegion + um_swz((uint32_t)r, (uint32_t)(j & 7) * 16u), g,
-                    ok ? 16u : 0u);
-    }
-    cp_async_commit();
+    const int st = i % kUmStages;
+    const uint32_t abuf = sA + (uint32_t)st * kUmABytes;
+    mbar_arrive_expect_tx(&afull[st], kUmABytes);
+    um_tma_load_3d(abuf, map, 0, h, tile_of(i) * kUmTile, &afull[st]);
+    um_tma_load_3d(abuf + kUmRegion, map, 64, h, tile_of(i) * kUmTile, &afull[st]);
   };
+  int loaded = 0, landed = 0;  // tiles whose loads were issued / waited for (producer lane 0)
 
   if (tid == 0) {
     for (int i = 0; i < 2; ++i) {
       mbar_init(&mma_done[i], 1);
       mbar_init(&tmem_free[i], 128);
     }
+    for (int i = 0; i < kUmStages; ++i) mbar_init(&afull[i], 1);
     fence_mbar_init();
   }
   __syncthreads();
   if (warp == kUmProducer) {
     // the first tiles' loads go out while the other warps stage R
-    load_tile(0);
-    if (n > 1) load_tile(1);
+    if (lane == 0) {
+      load_tile(0);
+      if (n > 1) load_tile(1);
+      loaded = min(n, 2);
+    }
   } else {
     // R = U H P_br / sqrt(128), split in three bf16 parts, into B (row n = output channel,
     // K = input channel).  Warp w takes input channels 16w .. 16w + 15 in two batches of eight:
@@ -438,14 +450,12 @@ __global__ void __launch_bounds__(kUmThreads, 1) append_umma_kernel(AppendArgs a
 
   if (warp == kUmProducer) {
     for (int i = 0; i < n; ++i) {
-      // MMAs of tile i: its copy group is in (only tile i + 1's group can be younger), and the
-      // epilogue of tile i - 2 has drained TMEM buffer i & 1
-      if (i + 1 < n) cp_async_wait_group<1>();
-      else cp_async_wait_group<0>();
-      um_fence_proxy_async();  // this lane's copies, made visible to the async proxy
-      __syncwarp();
+      // MMAs of tile i: its loads have landed, and the epilogue of tile i - 2 has drained TMEM
+      // buffer i & 1
       if (lane == 0 && alive) {
-        const bool ok = i < 2 || mbar_wait_bounded(&tmem_free[i & 1], ((uint32_t)(i - 2) >> 1) & 1u);
+        bool ok = mbar_wait_bounded(&afull[i % kUmStages], ((uint32_t)(i / kUmStages)) & 1u);
+        if (ok) landed = i + 1;
+        ok = ok && (i < 2 || mbar_wait_bounded(&tmem_free[i & 1], ((uint32_t)(i - 2) >> 1) & 1u));
         if (ok) {
           um_fence_after();
           const uint32_t abuf = sA + (uint32_t)(i % kUmStages) * kUmABytes;
@@ -472,14 +482,20 @@ __global__ void __launch_bounds__(kUmThreads, 1) append_umma_kernel(AppendArgs a
       if (alive && i + 2 < n) {
         if (i >= 1 && !mbar_wait_bounded(&mma_done[(i - 1) & 1], ((uint32_t)(i - 1) >> 1) & 1u)) alive = false;
         alive = __all_sync(0xffffffffu, alive);
-        if (alive) load_tile(i + 2);
+        if (alive && lane == 0) {
+          load_tile(i + 2);
+          loaded = i + 3;
+        }
       }
       if (!alive) {
         if (lane == 0) raise_flag(a.status, OKV_DEV_TIMEOUT);
         break;
       }
     }
-    cp_async_wait_all();  // no copy may outlive the CTA
+    // no copy may outlive the CTA: after a failed wait, wait (bounded) for the loads in flight
+    if (lane == 0)
+      for (int i = landed; i < loaded; ++i)
+        if (!mbar_wait_bounded(&afull[i % kUmStages], ((uint32_t)(i / kUmStages)) & 1u)) break;
   } else {
     const int wg = warp >> 2, q = warp & 3;
     // destination of this thread's token in tile i, fetched one tile (of this warpgroup) ahead
@@ -593,13 +609,40 @@ __global__ void __launch_bounds__(kUmThreads, 1) append_umma_kernel(AppendArgs a
 
 }  // namespace
 
+// Tensor map of the bf16 input [T][Hkv][128] for the tcgen05 append's tile
+// loads: boxes of 128 tokens x 64 channels (128 bytes, the swizzle span) of one
+// KV head, 128-byte swizzle, zero fill past T.  The encoder comes from the
+// driver through the runtime, so the library links no driver library.
+static bool encode_tile_map(CUtensorMap* m, const void* base, int hkv, int T) {
+  static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  if (encode == nullptr) return false;
+  const cuuint64_t dims[3] = {(cuuint64_t)kD, (cuuint64_t)hkv, (cuuint64_t)T};
+  const cuuint64_t strides[2] = {(cuuint64_t)kD * 2, (cuuint64_t)hkv * kD * 2};  // bytes, dims 1 and 2
+  const cuuint32_t box[3] = {64, 1, (cuuint32_t)kUmTile};
+  const cuuint32_t elem[3] = {1, 1, 1};
+  return encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, elem,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 okv_status launch_append(const okv_cache_desc* d, const void* k, const void* v, int T,
                          const int32_t* seq_slot, const int32_t* pos, const int32_t* block_table,
                          const int32_t* slot_lens, uint32_t flags, float* rotated_out,
                          cudaStream_t s) {
   const AppendArgs a = make_append_args(d, k, v, seq_slot, pos, block_table, slot_lens, rotated_out);
-  const bool rows16 = (((uintptr_t)k | (uintptr_t)v) & 15u) == 0;  // the tile loads copy 16-byte chunks
-  if (!(flags & OKV_PRE_ROTATED) && T >= kTcMinTokens && rows16) {
+  const bool rows16 = (((uintptr_t)k | (uintptr_t)v) & 15u) == 0;  // TMA needs 16-byte aligned bases
+  CUtensorMap map_k, map_v;
+  const bool maps = !(flags & OKV_PRE_ROTATED) && T >= kTcMinTokens && rows16 &&
+                    encode_tile_map(&map_k, k, d->num_kv_heads, T) && encode_tile_map(&map_v, v, d->num_kv_heads, T);
+  if (maps) {
     static std::atomic<uint32_t> attr_set{0};
     cudaError_t e = set_smem_limit_once((const void*)append_umma_kernel, (int)kUmSmem, attr_set);
     if (e != cudaSuccess) return fail(OKV_ERR_CUDA, "append smem attribute: %s", cudaGetErrorString(e));
@@ -607,7 +650,7 @@ okv_status launch_append(const okv_cache_desc* d, const void* k, const void* v, 
     const int tiles = (T + kUmTile - 1) / kUmTile;
     const int per_pair = std::max(1, std::min(tiles, device_sm_count() / pairs));
     dim3 grid(per_pair, d->num_kv_heads, 2);
-    append_umma_kernel<<<grid, kUmThreads, kUmSmem, s>>>(a, T);
+    append_umma_kernel<<<grid, kUmThreads, kUmSmem, s>>>(a, T, map_k, map_v);
     return check_launch("append (tcgen05)");
   }
   if (!(flags & OKV_PRE_ROTATED) && T >= kTcMinTokens) {
