@@ -138,3 +138,15 @@ def test_calibration_matches_oracle(hq, hkv, n):
             _match_columns(u, ref["U_" + kind][h], ref["lam_" + kind][h])
             r = got["R_" + kind][h].astype(np.float64)
             assert np.abs(r - ref["R_" + kind][h]).max() < 2e-5
+
+
+def test_prepared_step_call_checks_its_inputs_on_the_host():
+    torch = pytest.importorskip("torch")
+    k = torch.zeros((2, 8, 128), dtype=torch.bfloat16)
+    i32 = torch.zeros(2, dtype=torch.int32)
+    q = torch.zeros((2, 32, 128), dtype=torch.bfloat16)
+    table = torch.zeros((2, 4), dtype=torch.int32)
+    with pytest.raises(ValueError, match="CUDA"):
+        okv.DecodeStepCall(None, k, k, i32, i32, i32, q, i32, table, i32)
+    with pytest.raises(TypeError, match="bfloat16"):
+        okv.DecodeStepCall(None, k.float(), k, i32, i32, i32, q, i32, table, i32)
