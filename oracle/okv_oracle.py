@@ -208,12 +208,15 @@ def fp16_saturate(x32: np.ndarray) -> np.ndarray:
     return x.astype(np.float16)
 
 
-def quantize(z32: np.ndarray):
-    """Quantise groups of 128 fp32 values to 2-bit codes with fp16 scale and min.
+def quantize(z32: np.ndarray, group: int = D):
+    """Quantise groups of fp32 values to 2-bit codes with fp16 scale and min.
 
-    z32: float32 [..., 128] (one group per row).  Returns (codes uint8 [..., 128],
-    s16 float16 [...], m16 float16 [...]).  Steps, all in IEEE fp32 with
-    round-to-nearest-even:
+    z32: float32 [..., 128].  With group = 128 (the built format: one group
+    per row) returns (codes uint8 [..., 128], s16 float16 [...], m16 float16
+    [...]); with a smaller group g (a divisor of 128: the groups for which the
+    pages' bit-reversal permutation spreads importance, [GH] "Что придумали…")
+    s16 and m16 are [..., 128 / g], one pair per g consecutive channels.
+    Steps, per group, all in IEEE fp32 with round-to-nearest-even:
       mn = min z, mx = max z; s32 = (mx - mn) / 3;
       s16 = fp16(s32), m16 = fp16(mn) (saturating); s = f32(s16), m = f32(m16);
       c = 0 if s == 0 else clamp(rint((z - m) / s), 0, 3).
@@ -222,7 +225,18 @@ def quantize(z32: np.ndarray):
     table; [GH] section "Почему INT2 раньше не работал" (four levels)."""
     z = np.asarray(z32, dtype=np.float32)
     if z.shape[-1] != D:
-        raise ValueError("group must be 128 channels")
+        raise ValueError("vectors must have 128 channels")
+    if group <= 0 or D % group != 0:
+        raise ValueError("group must divide 128")
+    if group != D:
+        c, s16, m16 = quantize_rows(z.reshape(*z.shape[:-1], D // group, group))
+        return c.reshape(z.shape), s16, m16
+    return quantize_rows(z)
+
+
+def quantize_rows(z: np.ndarray):
+    """The rule of `quantize` applied to each row (last axis) of fp32 z."""
+    z = np.asarray(z, dtype=np.float32)
     mn = z.min(axis=-1)
     mx = z.max(axis=-1)
     s32 = (mx - mn) / np.float32(3.0)
@@ -250,11 +264,14 @@ def unpack(packed: np.ndarray) -> np.ndarray:
     return out.reshape(*b.shape[:-1], b.shape[-1] * 4).astype(np.uint8)
 
 
-def dequantize(codes: np.ndarray, s16: np.ndarray, m16: np.ndarray) -> np.ndarray:
-    """x_hat = s * c + m, exact in fp64 then rounded once to fp32."""
+def dequantize(codes: np.ndarray, s16: np.ndarray, m16: np.ndarray, group: int = D) -> np.ndarray:
+    """x_hat = s * c + m, exact in fp64 then rounded once to fp32 (per group)."""
+    c = np.asarray(codes, dtype=np.float64)
+    if group != D:
+        c = c.reshape(*c.shape[:-1], D // group, group)
     s = np.asarray(s16, dtype=np.float64)[..., None]
     m = np.asarray(m16, dtype=np.float64)[..., None]
-    return (s * np.asarray(codes, dtype=np.float64) + m).astype(np.float32)
+    return (s * c + m).reshape(np.shape(codes)).astype(np.float32)
 
 
 # ----------------------------------------------------------------------------

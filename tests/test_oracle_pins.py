@@ -231,6 +231,71 @@ def test_quantizer_permutation_equivariant_and_bounded():
     assert np.all(c[rows, z.argmin(1)] == 0) and np.all(c[rows, z.argmax(1)] == 3)
 
 
+def _scalar_rule(vals):
+    """The quantiser's steps for one group, one scalar at a time (np.float32 /
+    np.float16 scalars, round-to-nearest-even): a loop-only second statement."""
+    mn, mx = min(vals), max(vals)
+    s16 = np.float16(np.clip(np.float32((mx - mn) / np.float32(3.0)), -65504, 65504))
+    m16 = np.float16(np.clip(mn, -65504, 65504))
+    s, m = np.float32(s16), np.float32(m16)
+    codes = [0 if s == 0 else int(min(3, max(0, np.rint(np.float32((v - m) / s))))) for v in vals]
+    return codes, s16, m16
+
+
+@pytest.mark.parametrize("group", [32, 64, 128])
+def test_group_quantizer_against_a_scalar_loop(group):
+    rng = np.random.default_rng(16)
+    z = (rng.standard_normal((3, 128)) * rng.uniform(0.1, 40, (3, 1))).astype(np.float32)
+    z[1, 5] = 3e4  # one outlier inside one group
+    c, s16, m16 = O.quantize(z, group)
+    assert c.shape == (3, 128) and s16.shape == ((3, 128 // group) if group < 128 else (3,))
+    for t in range(3):
+        for gi in range(128 // group):
+            want_c, want_s, want_m = _scalar_rule([np.float32(x) for x in z[t, gi * group:(gi + 1) * group]])
+            got_s = s16[t, gi] if group < 128 else s16[t]
+            got_m = m16[t, gi] if group < 128 else m16[t]
+            assert list(c[t, gi * group:(gi + 1) * group]) == want_c, (group, t, gi)
+            assert got_s.view(np.uint16) == want_s.view(np.uint16) and got_m.view(np.uint16) == want_m.view(np.uint16)
+    # dequantised per group: every value within half its own group's scale, and
+    # only the outlier's group pays for the outlier
+    x = O.dequantize(c, s16, m16, group)
+    err = np.abs(x.astype(np.float64) - z)
+    sg = np.asarray(s16, np.float64).reshape(3, -1)
+    for t in range(3):
+        for gi in range(128 // group):
+            e = err[t, gi * group:(gi + 1) * group].max()
+            assert e <= sg[t, gi] / 2 * (1 + 1e-3) + 1e-2, (group, t, gi, e, sg[t, gi])
+    if group < 128:
+        outlier_group = 5 // group
+        others = np.delete(sg[1], outlier_group)
+        assert others.max() < sg[1, outlier_group] / 50
+
+
+def test_group_lattice_round_trip_and_bitrev_matters_below_d():
+    rng = np.random.default_rng(17)
+    # values on each 32-channel group's own fp16 lattice m + k s round-trip exactly
+    s = np.float16(rng.uniform(0.01, 2, 4)).astype(np.float32)
+    m = np.float16(rng.uniform(-5, 5, 4)).astype(np.float32)
+    k = rng.integers(0, 4, (4, 32))
+    k[:, 0], k[:, 1] = 0, 3
+    z = (m[:, None] + k * s[:, None]).astype(np.float32).reshape(1, 128)
+    c, s16, m16 = O.quantize(z, 32)
+    assert np.array_equal(c.reshape(4, 32), k) and np.array_equal(O.dequantize(c, s16, m16, 32), z)
+    # with groups smaller than d the bit-reversal permutation changes which
+    # channels share a scale, so it changes the dequantised vectors (with one
+    # group per vector it cannot: test_bitrev_leaves_dequantised_vectors_unchanged_when_group_is_d)
+    u = WL.haar_orthogonal(rng)
+    x = WL.to_bf16_exact(rng.standard_normal((64, 128)).astype(np.float32) * 3)
+    br = O.bitrev_indices(128)
+    with_br, without = O.rotation(u), u @ O.hadamard(128)
+    z1 = (x.astype(np.float64) @ with_br).astype(np.float32)
+    z0 = (x.astype(np.float64) @ without).astype(np.float32)
+    x1 = O.dequantize(*O.quantize(z1, 32), 32).astype(np.float64) @ with_br.T
+    x0 = O.dequantize(*O.quantize(z0, 32), 32).astype(np.float64) @ without.T
+    assert np.abs(x1 - x0).max() > 1e-3
+    assert np.array_equal(O.quantize(z1)[0], O.quantize(z1, 128)[0])
+
+
 def test_pack_layout_and_inverse():
     codes = np.zeros(128, np.uint8)
     codes[:4] = [1, 2, 3, 0]
