@@ -41,6 +41,8 @@ Readings taken where the pages are silent:
   clamped to [0, 3], dequantised as s*c + m;
 * every token is quantised at append; the last W = 128 positions are also
   kept as fp16 rotated values and decode reads those positions from fp16;
+* groups smaller than 128 channels (32, 64) follow the same rule per group,
+  one fp16 scale and min each (the built format has one group per vector);
 * sink tokens: the first S positions of a sequence are kept the same way and
   read from fp16.  The pages name sinks without a count; S is a cache
   parameter, 0 (no sinks) by default.  S = 192 with W = 128 keeps 320 of
@@ -288,10 +290,12 @@ class Cache:
     (recent tokens stay 16-bit, history goes to INT2, paged-cache compatible).
     """
 
-    def __init__(self, hkv: int, u_k: np.ndarray, u_v: np.ndarray, window: int = W, sinks: int = 0):
+    def __init__(self, hkv: int, u_k: np.ndarray, u_v: np.ndarray, window: int = W, sinks: int = 0,
+                 group: int = D):
         self.hkv = hkv
         self.window = window
         self.sinks = sinks
+        self.group = group  # channels per quantisation group (128: one per token-head)
         self.r = {0: np.stack([rotation(u) for u in u_k]), 1: np.stack([rotation(u) for u in u_v])}
         self.seqs = {}
 
@@ -300,8 +304,9 @@ class Cache:
         st = self.seqs.get(key)
         if st is None or st["codes"].shape[0] < need:
             cap = max(need, 2 * (0 if st is None else st["codes"].shape[0]), 64)
-            new = {"codes": np.zeros((cap, D), np.uint8), "s16": np.zeros(cap, np.float16),
-                   "m16": np.zeros(cap, np.float16), "z16": np.zeros((cap, D), np.float16),
+            sm_shape = (cap,) if self.group == D else (cap, D // self.group)
+            new = {"codes": np.zeros((cap, D), np.uint8), "s16": np.zeros(sm_shape, np.float16),
+                   "m16": np.zeros(sm_shape, np.float16), "z16": np.zeros((cap, D), np.float16),
                    "set": np.zeros(cap, bool)}
             if st is not None:
                 n = st["codes"].shape[0]
@@ -326,7 +331,7 @@ class Cache:
             for h in range(self.hkv):
                 xs = np.asarray(x[:, h, :], dtype=np.float32)
                 z = xs if pre_rotated else (xs.astype(np.float64) @ self.r[kind][h]).astype(np.float32)
-                c, s16, m16 = quantize(z)
+                c, s16, m16 = quantize(z, self.group)
                 st = self._store(slot, kind, h, pos0 + n)
                 sl = slice(pos0, pos0 + n)
                 st["codes"][sl], st["s16"][sl], st["m16"][sl] = c, s16, m16
@@ -347,7 +352,7 @@ class Cache:
         out = st["z16"][:length].astype(np.float64)
         int2 = np.arange(length)
         int2 = int2[(int2 >= self.sinks) & (int2 < length - self.window)]
-        out[int2] = dequantize(st["codes"][int2], st["s16"][int2], st["m16"][int2])
+        out[int2] = dequantize(st["codes"][int2], st["s16"][int2], st["m16"][int2], self.group)
         return out
 
 

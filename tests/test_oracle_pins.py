@@ -314,7 +314,7 @@ def test_dequantize_scalar():
 
 # --------------------------------------------------------- cache and decode
 
-def _brute_decode_one(q, r_k, r_v, ent_k, ent_v, length, window, sinks=0):
+def _brute_decode_one(q, r_k, r_v, ent_k, ent_v, length, window, sinks=0, group=128):
     """Loop-only decode for one query head from raw cache entries."""
     d = len(q)
     qr = [sum(q[c] * r_k[c, j] for c in range(d)) for j in range(d)]
@@ -323,7 +323,9 @@ def _brute_decode_one(q, r_k, r_v, ent_k, ent_v, length, window, sinks=0):
         codes, s16, m16, z16 = ent(p)
         if p >= length - window or p < sinks:
             return [float(z16[j]) for j in range(d)]
-        return [float(s16) * int(codes[j]) + float(m16) for j in range(d)]
+        if group == d:
+            return [float(s16) * int(codes[j]) + float(m16) for j in range(d)]
+        return [float(s16[j // group]) * int(codes[j]) + float(m16[j // group]) for j in range(d)]
 
     logits = []
     for p in range(length):
@@ -340,11 +342,11 @@ def _brute_decode_one(q, r_k, r_v, ent_k, ent_v, length, window, sinks=0):
     return np.array([sum(o[j] * r_v[c, j] for j in range(d)) for c in range(d)])
 
 
-def _small_cache(seed, hkv, lens, window=O.W, sinks=0):
+def _small_cache(seed, hkv, lens, window=O.W, sinks=0, group=128):
     rng = np.random.default_rng(seed)
     uk = np.stack([WL.haar_orthogonal(rng) for _ in range(hkv)])
     uv = np.stack([WL.haar_orthogonal(rng) for _ in range(hkv)])
-    cache = O.Cache(hkv, uk, uv, window=window, sinks=sinks)
+    cache = O.Cache(hkv, uk, uv, window=window, sinks=sinks, group=group)
     for slot, length in enumerate(lens):
         k = WL.to_bf16_exact(rng.standard_normal((length, hkv, 128)).astype(np.float32) * 2)
         v = WL.to_bf16_exact(rng.standard_normal((length, hkv, 128)).astype(np.float32))
@@ -354,12 +356,12 @@ def _small_cache(seed, hkv, lens, window=O.W, sinks=0):
     return cache, rng
 
 
-@pytest.mark.parametrize("sinks", [0, 4])
-def test_decode_matches_loop_brute_force(sinks):
+@pytest.mark.parametrize("sinks,group", [(0, 128), (4, 128), (0, 32), (4, 64)])
+def test_decode_matches_loop_brute_force(sinks, group):
     # with 4 sinks and a window of 8: length 27 has INT2 positions 4..18,
     # length 9 has none (sink and window overlap), length 13 exactly none
     lens = [27, 9, 13]
-    cache, rng = _small_cache(10, 2, lens, window=8, sinks=sinks)
+    cache, rng = _small_cache(10, 2, lens, window=8, sinks=sinks, group=group)
     q = WL.to_bf16_exact(rng.standard_normal((3, 4, 128)).astype(np.float32))
     got = O.decode(cache, q, [0, 1, 2], lens, hq=4)
     for b, length in enumerate(lens):
@@ -367,7 +369,7 @@ def test_decode_matches_loop_brute_force(sinks):
             hk = h // 2
             want = _brute_decode_one(
                 q[b, h].astype(float), cache.r[0][hk], cache.r[1][hk],
-                lambda p: cache.entry(b, 0, hk, p), lambda p: cache.entry(b, 1, hk, p), length, 8, sinks)
+                lambda p: cache.entry(b, 0, hk, p), lambda p: cache.entry(b, 1, hk, p), length, 8, sinks, group)
             assert np.abs(got[b, h] - want).max() < 1e-10 * max(1.0, np.abs(want).max())
 
 
