@@ -185,7 +185,14 @@ okv_status okv_append_quantize(const okv_cache_desc* desc, const void* k, const 
                                const int32_t* block_table, const int32_t* slot_lens,
                                uint32_t flags, float* rotated_out, void* stream);
 
-/* Workspace bytes okv_decode_attention needs for batch B on the current device. */
+/* Workspace bytes okv_decode_attention (and okv_decode_step) needs for batch
+ * B on the current device: the rotated queries in the forms the split-K
+ * kernel reads, the cost prefix, and one fp32 partial (o', max, sum) per query
+ * head for every split-K CTA and batch entry -- so it grows with the device's
+ * SM count.  The split-K partials are the log-sum-exp pieces of the decode
+ * attention that streams the cache from HBM (aiforradalom.hu, "Az Apple, a
+ * Google és a NYU új technikái…", intro: decode is bound by reading the KV
+ * cache).  Returns 0 for an invalid descriptor or B < 0. */
 size_t okv_decode_workspace_bytes(const okv_cache_desc* desc, int32_t B);
 
 /* Decode attention for one new query per sequence.
@@ -207,7 +214,10 @@ okv_status okv_decode_attention(const okv_cache_desc* desc, const void* q, int32
                                 const int32_t* context_lens, float* out, void* workspace,
                                 size_t workspace_bytes, void* stream);
 
-/* Size of the device array behind okv_decode_attention_noalloc (8 MiB). */
+/* Size of the device array behind okv_decode_attention_noalloc (8 MiB).  A
+ * batch fits when okv_decode_workspace_bytes(desc, B) is at most this, which
+ * depends on the SM count: on a 148-SM B200, up to 58 sequences with 32 query
+ * and 8 KV heads (so a 64-sequence batch is refused), up to 29 with 64 and 8. */
 #define OKV_NOALLOC_SCRATCH_BYTES (8u << 20)
 
 /* One decode step in one call: append this step's new tokens, then decode.
@@ -247,7 +257,11 @@ okv_status okv_decode_attention_noalloc(const okv_cache_desc* desc, const void* 
                                         const int32_t* seq_slot, const int32_t* block_table,
                                         const int32_t* context_lens, float* out, void* stream);
 
-/* Gather and dequantise the cache into dense fp32.
+/* Gather and dequantise the cache into dense fp32 (the INT2 format's inverse:
+ * s*c + m with the fp16 scale and minimum of each group; bigsaas.top,
+ * "Revolução no Serviço de LLMs…", section "Resultados e Métricas de
+ * Desempenho": INT2 values at about 2.28 bits; the original basis undoes
+ * R = U H P_br, gen-hub.ru "Что придумали в Together AI").
  *   which: 0 keys, 1 values.  basis: 0 rotated (as stored), 1 original
  *   (multiplied back by R^T).  source: 0 INT2 for every position, 1 as decode
  *   reads it (fp16 for the last W positions and the first num_sink).  out: device fp32

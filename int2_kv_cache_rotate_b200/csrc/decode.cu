@@ -463,10 +463,24 @@ __global__ void __launch_bounds__(kDecWarps * 32) decode_simt_kernel(DecodeArgs 
 // Per 2-block step a warp computes:
 //   scores  S[32 tok x 4NT heads] = C_K (u8 codes) . Q (two s8 limbs) on
 //           mma.m16n8k32, then s_t * sigma * raw + m_t * sum(q~);
-//   values  O[128 ch x heads] += C_V . P', P' = round(p * s_t * 65535 / s_cap)
-//           as two u8 limbs, exact in int32, flushed to fp32 only when the
-//           running max or the scale cap moves (or every 96 steps);
-//   plus sum(p * m_t) for the value minimum term.
+//   values  O[128 ch x heads] += C_V . P', P' = round(p * s_t * lam_h) as two
+//           u8 limbs, exact in int32, flushed to fp32 only when the running
+//           max, the scale cap or a head's P' scale moves (or every 96 steps);
+//   plus sum(p * (m_t + 1.5 s_t)) for the value minimum term.
+// P' precision.  lam_h = lam0 * 2^k_h per query head.  lam0 = 65535 /
+// (4 s_cap), with s_cap twice the largest value scale seen, keeps P' < 2^16
+// by construction (p <= 4); k_h = 0 is the normal state.  A head whose
+// largest P' stays below 2^6 for 4 steps in a row -- its tokens all sit far
+// below an earlier dominant token, a sink or retrieval token with a long
+// flat tail -- is flushed and boosted: k_h is set so that the last step's
+// largest P' lands in [2^13, 2^14).  A boosted head whose P' would pass 16
+// bits is flushed and returns to k_h = 0 before anything is stored.  A run
+// of 4 low steps is rare where logits are merely spread out (single low steps
+// are not), so the boost costs nothing there.  The codes are also centred:
+// the 3/2 s_t part of each value goes with m_t into the fp32 sum above, and
+// every flush takes 3/2 inv_h sum P' back out of that sum, so the rounding
+// errors of P' meet zero-mean code offsets and do not add up over a long
+// range of tokens.
 // Fragment facts (PTX m16n8k32, 8-bit): lane (g = lane/4, t = lane%4) holds
 // A rows g and g+8 with K-columns 4t..4t+3 and 16+4t..16+4t+3; B K-rows
 // 4t..4t+3 and 16+4t..+3 of column g; D rows g, g+8, columns 2t, 2t+1.
@@ -493,7 +507,18 @@ constexpr int kPStride = 40;                       // u16 per head row of the P'
 constexpr int kWarpScratch = 9216;                 // ring bytes each warp may use as window scratch
 constexpr uint32_t kM2 = 0x03030303u;
 constexpr float kMaxSlack = 2.f;  // log2 units a score may exceed the reference max without a rescale
-constexpr float kPSlack = 4.f;    // = 2^kMaxSlack
+// P' = round(x) comes out of one FFMA: bits(x + 1.5 * 2^23) = kMagicBits + round(x)
+// for 0 <= x < 2^22, and the bits grow with x beyond that.
+constexpr float kMagic = 12582912.f;
+constexpr uint32_t kMagicBits = 0x4B400000u;
+constexpr uint32_t kPLowBits = kMagicBits + 64u;     // a head's step maximum below 2^6 is "low"
+constexpr uint32_t kPHighBits = kMagicBits + 65535u; // above 16 bits: back to k_h = 0 before storing
+constexpr int kLowRun = 4;                           // low steps in a row that boost a head
+constexpr int kBoostExp = 13;                        // a boost puts the step maximum in [2^13, 2^14)
+constexpr int kMaxBoost = 60;                        // k_h <= 60 (lam0 * 2^60 stays finite)
+constexpr float kPSlack = 4.f;                       // = 2^kMaxSlack
+
+__device__ __forceinline__ float pow2f(int k) { return __int_as_float((127 + k) << 23); }  // -126 <= k <= 127
 
 template <int G>
 struct HCfg {
@@ -585,11 +610,19 @@ __device__ __forceinline__ void tacc_store(uint32_t taddr, const float (&v)[16])
 // acci[mt] holds channel 16g + 2mt (regs 0,1 = hi, lo limb) and 16g + 2mt + 1
 // (regs 2,3); those channels come from code field f = 2(mt&1) and f + 1,
 // which the unshifted masks scaled by 4^f.
-// acci: exact int32 o' contributions since the last flush (row scale 4^f).
-// Flush: o' = (o' + acci / scale) * rescale, in tensor memory (warp-collective).
+// acci: exact int32 sums of P' c 4^f since the last flush; psum: this lane's
+// sum of P' over the same steps (wrapping modulo 2^32, which the plain sum
+// never reaches).
+// Flush: o' = (o' + inv * sum P' c) * rescale in tensor memory
+// (warp-collective), and msum -= 3/2 inv sum P', so that together they hold
+// inv * sum P' (c - 3/2) on top of the sum of p (m + 3/2 s).  The two parts
+// are each rounded to fp32 before they meet; their sum is what carries the
+// P' rounding errors, and there they see zero-mean code offsets.
 template <int G>
-__device__ __forceinline__ void mma_flush(MmaWarpState<G>& st, int (&acci)[HCfg<G>::NT][8][4], int nt, float inv,
-                                          float rescale = 1.f) {
+__device__ __forceinline__ void mma_flush(MmaWarpState<G>& st, int (&acci)[HCfg<G>::NT][8][4],
+                                          uint32_t (&psum)[HCfg<G>::NT], int nt, float inv, float rescale = 1.f) {
+  st.msum[nt] = fmaf(-1.5f * inv, (float)psum[nt], st.msum[nt]);
+  psum[nt] = 0u;
 #pragma unroll
   for (int hh = 0; hh < 2; ++hh) {  // two halves of 8 channels: fewer live registers
     float v[8];
@@ -843,7 +876,22 @@ __global__ void __launch_bounds__(kHW * 32, (G <= 4) ? 2 : 1) decode_heads_kerne
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) tacc_store(st.tacc + 16u * nt, zero);
     }
-    float s_cap = 0.f, lam = 0.f, inv = 0.f;
+    // P' scale: the warp's base lam0 (0 until a positive value scale is seen)
+    // and, per head of this lane's score column, the boost k, lam = lam0 2^k,
+    // inv = 1 / lam, the count of low steps in a row, and this lane's sum of
+    // P' since the last flush
+    float s_cap = 0.f, lam0 = 0.f;
+    float lam[NT];
+    int lrb[NT];  // (low steps in a row) << 8 | boost k
+    uint32_t psum[NT];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      lam[nt] = 0.f;
+      lrb[nt] = 0;
+      psum[nt] = 0u;
+    }
+    // 1 / lam of n-tile nt (0 before any value scale was seen)
+    auto inv_of = [&](int nt) { return (s_cap * (kPSlack / 65535.f)) * pow2f(-(lrb[nt] & 0xff)); };
     int since_flush = 0;
 
 
@@ -918,7 +966,7 @@ __global__ void __launch_bounds__(kHW * 32, (G <= 4) ? 2 : 1) decode_heads_kerne
           }
         }
         // token e of this lane: block e>>1, row g + 8*(e&1)
-        float sk[4], mk[4], sv[4], mv[4];
+        float sk[4], mk[4], sv[4], mc[4];
         bool tv[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
@@ -927,27 +975,25 @@ __global__ void __launch_bounds__(kHW * 32, (G <= 4) ? 2 : 1) decode_heads_kerne
           tv[e] = fullstep || ((g + 8 * (e & 1)) < ((e >> 1) ? n1 : n0));
           // masked slots may hold any bits (a slot whose block was not fetched
           // keeps stale shared memory): select, never multiply, them away
-          sk[e] = k2.x; mk[e] = k2.y; sv[e] = v2.x;
-          mv[e] = tv[e] ? v2.y : 0.f;
+          sk[e] = k2.x; mk[e] = k2.y;
+          sv[e] = tv[e] ? v2.x : 0.f;
+          mc[e] = tv[e] ? fmaf(1.5f, v2.x, v2.y) : 0.f;  // m + 3/2 s: the codes are centred in the flush
         }
-        float smax = fmaxf(fmaxf(tv[0] ? sv[0] : 0.f, tv[1] ? sv[1] : 0.f),
-                           fmaxf(tv[2] ? sv[2] : 0.f, tv[3] ? sv[3] : 0.f));
+        float smax = fmaxf(fmaxf(sv[0], sv[1]), fmaxf(sv[2], sv[3]));
         if (__any_sync(0xffffffffu, smax > s_cap)) {  // rare: raise the scale cap, flushing every head first
           smax = fmaxf(smax, __shfl_xor_sync(0xffffffffu, smax, 4));
           smax = fmaxf(smax, __shfl_xor_sync(0xffffffffu, smax, 8));
           smax = fmaxf(smax, __shfl_xor_sync(0xffffffffu, smax, 16));
 #pragma unroll
-          for (int nt = 0; nt < NT; ++nt) mma_flush(st, acci, nt, inv);
+          for (int nt = 0; nt < NT; ++nt) mma_flush(st, acci, psum, nt, inv_of(nt));
           since_flush = 0;
           // headroom: the cap jumps to twice the new maximum, and P' leaves room
           // for p up to 2^kMaxSlack, so later small increases cost nothing
           s_cap = 2.f * smax;
-          lam = 65535.f / (s_cap * kPSlack);
-          inv = (s_cap * kPSlack) / 65535.f;
-        }
-        float svl[4];
+          lam0 = 65535.f / (s_cap * kPSlack);
 #pragma unroll
-        for (int e = 0; e < 4; ++e) svl[e] = tv[e] ? sv[e] * lam : 0.f;
+          for (int nt = 0; nt < NT; ++nt) lam[nt] = lam0 * pow2f(lrb[nt] & 0xff);
+        }
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
           float sc[4];
@@ -970,7 +1016,7 @@ __global__ void __launch_bounds__(kHW * 32, (G <= 4) ? 2 : 1) decode_heads_kerne
             // warp-collectively); heads whose max did not move keep scale 1
             const bool need = bm > st.m[nt] + kMaxSlack;
             const float alpha = need ? fast_ex2(st.m[nt] - bm) : 1.f;  // ex2(-inf) = 0 on the first step
-            mma_flush(st, acci, nt, inv, alpha);
+            mma_flush(st, acci, psum, nt, inv_of(nt), alpha);
             if (need) {
               st.l[nt] *= alpha;
               st.msum[nt] *= alpha;
@@ -978,16 +1024,52 @@ __global__ void __launch_bounds__(kHW * 32, (G <= 4) ? 2 : 1) decode_heads_kerne
             }
           }
           const float mref = st.m[nt] == -INFINITY ? 0.f : st.m[nt];
-          uint16_t* prow = myp + (4 * nt + t) * kPStride;
+          float y[4];  // p * s
+          uint32_t u[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const float p = fast_ex2(sc[e] - mref);  // 0 for masked tokens
             st.l[nt] += p;
-            st.msum[nt] = fmaf(p, mv[e], st.msum[nt]);
-            // round(p * s * lam) <= 65535 via the 1.5 * 2^23 magic add (one FFMA, no conversion unit)
-            prow[16 * (e >> 1) + g + 8 * (e & 1)] =
-                (uint16_t)(__float_as_uint(fmaf(p, svl[e], 12582912.f)) - 0x4B400000u);
+            st.msum[nt] = fmaf(p, mc[e], st.msum[nt]);
+            y[e] = p * sv[e];
+            u[e] = __float_as_uint(fmaf(y[e], lam[nt], kMagic));  // kMagicBits + round(p s lam)
           }
+          // A head whose largest P' stays below 2^6 for kLowRun steps is
+          // boosted; a boosted head whose P' would pass 16 bits drops back to
+          // k = 0.  Either way this n-tile is flushed first.
+          const uint32_t um = max(max(u[0], u[1]), max(u[2], u[3]));
+          const uint32_t big = __ballot_sync(0xffffffffu, um >= kPLowBits);
+          // low steps in a row, the same in the head's 8 lanes
+          lrb[nt] = ((big >> t) & 0x11111111u) == 0u ? lrb[nt] + 256 : (lrb[nt] & 0xff);
+          const bool raise = (4 * nt + t < G) && lrb[nt] >= (kLowRun << 8) && (lrb[nt] & 0xff) < kMaxBoost;
+          if (__any_sync(0xffffffffu, um > kPHighBits || raise)) {
+            uint32_t uh = um;  // the head's step maximum (lanes of the same t)
+            uh = max(uh, __shfl_xor_sync(0xffffffffu, uh, 4));
+            uh = max(uh, __shfl_xor_sync(0xffffffffu, uh, 8));
+            uh = max(uh, __shfl_xor_sync(0xffffffffu, uh, 16));
+            float ym = fmaxf(fmaxf(y[0], y[1]), fmaxf(y[2], y[3]));
+            ym = fmaxf(ym, __shfl_xor_sync(0xffffffffu, ym, 4));
+            ym = fmaxf(ym, __shfl_xor_sync(0xffffffffu, ym, 8));
+            ym = fmaxf(ym, __shfl_xor_sync(0xffffffffu, ym, 16));
+            mma_flush(st, acci, psum, nt, inv_of(nt));
+            int k = lrb[nt] & 0xff;
+            if (uh > kPHighBits) {
+              k = 0;
+            } else if (raise) {
+              // 2^k with ym * lam0 * 2^k in [2^13, 2^14): k = 13 - floor(log2(ym * lam0))
+              const float y = ym * lam0;
+              const int ex = ((__float_as_int(y) >> 23) & 0xff) - 127;
+              if (y > 0.f) k = max(0, min(kMaxBoost, kBoostExp - ex));
+            }
+            lrb[nt] = (uh > kPHighBits || raise) ? k : (lrb[nt] & ~0xff) | k;
+            lam[nt] = lam0 * pow2f(k);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) u[e] = __float_as_uint(fmaf(y[e], lam[nt], kMagic));
+          }
+          uint16_t* prow = myp + (4 * nt + t) * kPStride;
+#pragma unroll
+          for (int e = 0; e < 4; ++e) prow[16 * (e >> 1) + g + 8 * (e & 1)] = (uint16_t)u[e];  // P' < 2^16
+          psum[nt] += (u[0] + u[1]) + (u[2] + u[3]) - 4u * kMagicBits;
         }
         __syncwarp();
         // ---- values: acci[mt] += C_V (masked, row scale 4^f) . P'
@@ -1014,7 +1096,7 @@ __global__ void __launch_bounds__(kHW * 32, (G <= 4) ? 2 : 1) decode_heads_kerne
         }
         if (++since_flush >= 96) {
 #pragma unroll
-          for (int nt = 0; nt < NT; ++nt) mma_flush(st, acci, nt, inv);
+          for (int nt = 0; nt < NT; ++nt) mma_flush(st, acci, psum, nt, inv_of(nt));
           since_flush = 0;
         }
       };
@@ -1031,7 +1113,7 @@ __global__ void __launch_bounds__(kHW * 32, (G <= 4) ? 2 : 1) decode_heads_kerne
     }
     it += (uint32_t)nst;
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) mma_flush(st, acci, nt, inv);
+    for (int nt = 0; nt < NT; ++nt) mma_flush(st, acci, psum, nt, inv_of(nt));
     __syncthreads();  // every warp is done with the ring: it becomes window scratch, then merge buffers
 
     // ---------------- fp16 rows: chunks ci = grp, grp + wph, ... of this warp's head ----------------

@@ -5,8 +5,6 @@ The layout reader encodes only where bytes live (documented in
 include/okv.h); it does no arithmetic of the method."""
 from __future__ import annotations
 
-import math
-
 import numpy as np
 
 from int2_kv_cache_rotate_b200 import workloads as WL
@@ -158,45 +156,3 @@ def ambiguity_bound(z64: np.ndarray, eps_rel: float) -> np.ndarray:
     row = near_mid(s32, 2 * tol[:, 0] / 3 + 1e-30) | near_mid(mn, tol[:, 0] + 1e-30)
     amb |= row[:, None]
     return amb
-
-
-def softmax_np(x):
-    x = x - x.max()
-    e = np.exp(x)
-    return e / e.sum()
-
-
-def fused_decode_bound(cache: O.Cache, amb_k, amb_v, q, seq_slots, lens, hq):
-    """Upper bound on how far the decode output may move when every ambiguous
-    code takes its other neighbour and every fp16 window value moves by one
-    fp16 step.  A K change moves a logit by at most sum_j |q~_j| dk_j / sqrt(d),
-    which moves the normalised weights by p_t (e^dlog - 1); a V change moves
-    rotated channel j by p_t dv_j.  Both are carried through R_V^T with the
-    largest absolute entry of R_V."""
-    g = hq // cache.hkv
-    bound = np.zeros((len(lens), hq))
-    step = 2.0 ** -10
-    for b, length in enumerate(lens):
-        if length == 0:
-            continue
-        slot = int(seq_slots[b])
-        first_fp16 = max(0, length - cache.window)
-        for hk in range(cache.hkv):
-            kx = cache.values(slot, 0, hk, length)
-            vx = cache.values(slot, 1, hk, length)
-            sk = cache.seqs[(slot, 0, hk)]["s16"][:length].astype(np.float64)[:, None]
-            sv = cache.seqs[(slot, 1, hk)]["s16"][:length].astype(np.float64)[:, None]
-            dk = np.where(amb_k[(slot, hk)][:length], sk, 0.0)
-            dv = np.where(amb_v[(slot, hk)][:length], sv, 0.0)
-            dk[first_fp16:] = np.abs(kx[first_fp16:]) * step
-            dv[first_fp16:] = np.abs(vx[first_fp16:]) * step
-            vmax = np.abs(vx).max()
-            rmax = np.abs(cache.r[1][hk]).max()
-            for h in range(hk * g, (hk + 1) * g):
-                qr = np.asarray(q[b, h], dtype=np.float64) @ cache.r[0][hk]
-                p = softmax_np(kx @ qr / math.sqrt(D))
-                dlog = (dk * np.abs(qr)[None, :]).sum(axis=1) / math.sqrt(D)
-                dw = (p * np.expm1(dlog)).sum()
-                dvo = (p[:, None] * dv).sum(axis=0)
-                bound[b, h] = (2 * dw * vmax * D + dvo.sum()) * rmax
-    return bound
