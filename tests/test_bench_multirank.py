@@ -40,7 +40,7 @@ def _rank_main(rank, world, port, result_q):
 
 
 class _RefArgs:
-    seed, warmup, steps, gpus = 0, 3, 2, 2
+    seed, warmup, steps, gpus, workload = 0, 3, 2, 2, 2
 
 
 def test_two_rank_time_is_max_and_units_sum():
