@@ -573,7 +573,8 @@ __device__ __forceinline__ float fast_ex2(float x) {
 template <int G>
 struct MmaWarpState {
   static constexpr int NT = HCfg<G>::NT;
-  float m[NT], l[NT], msum[NT];
+  float m[NT];
+  float2 l[NT], msum[NT];  // two partial sums each (paired fp32 arithmetic); the value is .x + .y
   uint32_t tacc;  // TMEM address of fp32 o' for channels 16g + 0..15 of head 4nt + t at column 16 nt + i
 };
 
@@ -621,7 +622,7 @@ __device__ __forceinline__ void tacc_store(uint32_t taddr, const float (&v)[16])
 template <int G>
 __device__ __forceinline__ void mma_flush(MmaWarpState<G>& st, int (&acci)[HCfg<G>::NT][8][4],
                                           uint32_t (&psum)[HCfg<G>::NT], int nt, float inv, float rescale = 1.f) {
-  st.msum[nt] = fmaf(-1.5f * inv, (float)psum[nt], st.msum[nt]);
+  st.msum[nt].x = fmaf(-1.5f * inv, (float)psum[nt], st.msum[nt].x);
   psum[nt] = 0u;
 #pragma unroll
   for (int hh = 0; hh < 2; ++hh) {  // two halves of 8 channels: fewer live registers
@@ -847,8 +848,8 @@ __global__ void __launch_bounds__(kHW * 32, (G <= 4) ? 2 : 1) decode_heads_kerne
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
       st.m[nt] = -INFINITY;
-      st.l[nt] = 0.f;
-      st.msum[nt] = 0.f;
+      st.l[nt] = make_float2(0.f, 0.f);
+      st.msum[nt] = make_float2(0.f, 0.f);
 #pragma unroll
       for (int mt = 0; mt < 8; ++mt)
 #pragma unroll
@@ -927,11 +928,11 @@ __global__ void __launch_bounds__(kHW * 32, (G <= 4) ? 2 : 1) decode_heads_kerne
         const unsigned char* s0 = ring + s * kHStageBytes + q0 * copy_bytes + head * kBlockHeadBytes;
         const unsigned char* s1 = s0 + copy_bytes;
 
-        // ---- everything this lane needs from the stage goes to registers, then
-        //      the stage is released so the producer can refill it while we compute
+        // ---- what the scores and weights need from the stage goes to
+        //      registers now; the value codes follow just before the value
+        //      MMAs, after which the stage is released for the producer
         uint2 kw[2][2];
         uint32_t smk[4], smv[4];
-        uint4 vw[2];
 #pragma unroll
         for (int bb = 0; bb < 2; ++bb) {
           const unsigned char* sb = bb ? s1 : s0;
@@ -941,10 +942,7 @@ __global__ void __launch_bounds__(kHW * 32, (G <= 4) ? 2 : 1) decode_heads_kerne
           smk[2 * bb + 1] = *reinterpret_cast<const uint32_t*>(sb + kKsmOff + 4 * (g + 8));
           smv[2 * bb] = *reinterpret_cast<const uint32_t*>(sb + kVsmOff + 4 * g);
           smv[2 * bb + 1] = *reinterpret_cast<const uint32_t*>(sb + kVsmOff + 4 * (g + 8));
-          vw[bb] = *reinterpret_cast<const uint4*>(sb + kVcOff + 16 * lane);
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[s]);
 
         // ---- scores: D[tok][col] for both blocks
         int dq[2][NT][4];
@@ -994,46 +992,63 @@ __global__ void __launch_bounds__(kHW * 32, (G <= 4) ? 2 : 1) decode_heads_kerne
 #pragma unroll
           for (int nt = 0; nt < NT; ++nt) lam[nt] = lam0 * pow2f(lrb[nt] & 0xff);
         }
+        // tokens in pairs (e = 0, 1: block 0; e = 2, 3: block 1) for the
+        // paired fp32 instructions
+        const float2 sk01 = make_float2(sk[0], sk[1]), sk23 = make_float2(sk[2], sk[3]);
+        const float2 mk01 = make_float2(mk[0], mk[1]), mk23 = make_float2(mk[2], mk[3]);
+        const float2 sv01 = make_float2(sv[0], sv[1]), sv23 = make_float2(sv[2], sv[3]);
+        const float2 mc01 = make_float2(mc[0], mc[1]), mc23 = make_float2(mc[2], mc[3]);
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
-          float sc[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int bb = e >> 1, r = 2 * (e & 1);
-            const int raw = dq[bb][nt][r] * 256 + dq[bb][nt][r + 1];
-            float x = fmaf(sk[e] * ah[nt], (float)raw, mk[e] * bh[nt]);
-            if constexpr (G < 4) x += hbias[nt];
-            sc[e] = tv[e] ? x : -INFINITY;
+          // x = s sigma' raw + m sum' (log2 units), taken relative to the
+          // running max mref straight away: x' = x - mref
+          const float mref0 = st.m[nt] == -INFINITY ? 0.f : st.m[nt];
+          const float2 ah2 = make_float2(ah[nt], ah[nt]), bh2 = make_float2(bh[nt], bh[nt]);
+          const float2 c2 = make_float2(hbias[nt] - mref0, hbias[nt] - mref0);  // hbias: -inf on padded heads
+          const float2 raw01 = make_float2((float)(dq[0][nt][0] * 256 + dq[0][nt][1]),
+                                           (float)(dq[0][nt][2] * 256 + dq[0][nt][3]));
+          const float2 raw23 = make_float2((float)(dq[1][nt][0] * 256 + dq[1][nt][1]),
+                                           (float)(dq[1][nt][2] * 256 + dq[1][nt][3]));
+          float2 x01 = __ffma2_rn(__fmul2_rn(sk01, ah2), raw01, __ffma2_rn(mk01, bh2, c2));
+          float2 x23 = __ffma2_rn(__fmul2_rn(sk23, ah2), raw23, __ffma2_rn(mk23, bh2, c2));
+          if constexpr (!fullstep) {
+            x01.x = tv[0] ? x01.x : -INFINITY;
+            x01.y = tv[1] ? x01.y : -INFINITY;
+            x23.x = tv[2] ? x23.x : -INFINITY;
+            x23.y = tv[3] ? x23.y : -INFINITY;
           }
           // The reference max moves only when a score passes it by more than
           // kMaxSlack (log2 units): p <= 2^kMaxSlack, which P' has room for.
-          float bm = fmaxf(fmaxf(sc[0], sc[1]), fmaxf(sc[2], sc[3]));
-          if (__any_sync(0xffffffffu, bm > st.m[nt] + kMaxSlack)) {
+          float bm = fmaxf(fmaxf(x01.x, x01.y), fmaxf(x23.x, x23.y));  // relative to mref0
+          if (__any_sync(0xffffffffu, bm > (st.m[nt] == -INFINITY ? -INFINITY : kMaxSlack))) {
             bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 4));
             bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 8));
             bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 16));
             // the whole warp flushes (the accumulators are read and written
             // warp-collectively); heads whose max did not move keep scale 1
-            const bool need = bm > st.m[nt] + kMaxSlack;
-            const float alpha = need ? fast_ex2(st.m[nt] - bm) : 1.f;  // ex2(-inf) = 0 on the first step
+            const float mnew = bm + mref0;
+            const bool need = mnew > st.m[nt] + kMaxSlack;
+            const float alpha = need ? fast_ex2(st.m[nt] - mnew) : 1.f;  // ex2(-inf) = 0 on the first step
             mma_flush(st, acci, psum, nt, inv_of(nt), alpha);
             if (need) {
-              st.l[nt] *= alpha;
-              st.msum[nt] *= alpha;
-              st.m[nt] = bm;
+              const float2 a2 = make_float2(alpha, alpha), d2 = make_float2(-bm, -bm);
+              st.l[nt] = __fmul2_rn(st.l[nt], a2);
+              st.msum[nt] = __fmul2_rn(st.msum[nt], a2);
+              st.m[nt] = mnew;
+              x01 = __fadd2_rn(x01, d2);  // now relative to the new max
+              x23 = __fadd2_rn(x23, d2);
             }
           }
-          const float mref = st.m[nt] == -INFINITY ? 0.f : st.m[nt];
-          float y[4];  // p * s
-          uint32_t u[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float p = fast_ex2(sc[e] - mref);  // 0 for masked tokens
-            st.l[nt] += p;
-            st.msum[nt] = fmaf(p, mc[e], st.msum[nt]);
-            y[e] = p * sv[e];
-            u[e] = __float_as_uint(fmaf(y[e], lam[nt], kMagic));  // kMagicBits + round(p s lam)
-          }
+          const float2 p01 = make_float2(fast_ex2(x01.x), fast_ex2(x01.y));  // 0 for masked tokens
+          const float2 p23 = make_float2(fast_ex2(x23.x), fast_ex2(x23.y));
+          st.l[nt] = __fadd2_rn(st.l[nt], __fadd2_rn(p01, p23));
+          st.msum[nt] = __ffma2_rn(p23, mc23, __ffma2_rn(p01, mc01, st.msum[nt]));
+          // kMagicBits + round(p s lam)
+          const float2 lam2 = make_float2(lam[nt], lam[nt]), mg2 = make_float2(kMagic, kMagic);
+          float2 u01 = __ffma2_rn(p01, __fmul2_rn(sv01, lam2), mg2);
+          float2 u23 = __ffma2_rn(p23, __fmul2_rn(sv23, lam2), mg2);
+          uint32_t u[4] = {__float_as_uint(u01.x), __float_as_uint(u01.y), __float_as_uint(u23.x),
+                           __float_as_uint(u23.y)};
           // A head whose largest P' stays below 2^6 for kLowRun steps is
           // boosted; a boosted head whose P' would pass 16 bits drops back to
           // k = 0.  Either way this n-tile is flushed first.
@@ -1047,7 +1062,8 @@ __global__ void __launch_bounds__(kHW * 32, (G <= 4) ? 2 : 1) decode_heads_kerne
             uh = max(uh, __shfl_xor_sync(0xffffffffu, uh, 4));
             uh = max(uh, __shfl_xor_sync(0xffffffffu, uh, 8));
             uh = max(uh, __shfl_xor_sync(0xffffffffu, uh, 16));
-            float ym = fmaxf(fmaxf(y[0], y[1]), fmaxf(y[2], y[3]));
+            const float2 y01 = __fmul2_rn(p01, sv01), y23 = __fmul2_rn(p23, sv23);  // p * s
+            float ym = fmaxf(fmaxf(y01.x, y01.y), fmaxf(y23.x, y23.y));
             ym = fmaxf(ym, __shfl_xor_sync(0xffffffffu, ym, 4));
             ym = fmaxf(ym, __shfl_xor_sync(0xffffffffu, ym, 8));
             ym = fmaxf(ym, __shfl_xor_sync(0xffffffffu, ym, 16));
@@ -1063,17 +1079,24 @@ __global__ void __launch_bounds__(kHW * 32, (G <= 4) ? 2 : 1) decode_heads_kerne
             }
             lrb[nt] = (uh > kPHighBits || raise) ? k : (lrb[nt] & ~0xff) | k;
             lam[nt] = lam0 * pow2f(k);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) u[e] = __float_as_uint(fmaf(y[e], lam[nt], kMagic));
+            const float2 l2 = make_float2(lam[nt], lam[nt]);
+            u01 = __ffma2_rn(y01, l2, mg2);
+            u23 = __ffma2_rn(y23, l2, mg2);
+            u[0] = __float_as_uint(u01.x);
+            u[1] = __float_as_uint(u01.y);
+            u[2] = __float_as_uint(u23.x);
+            u[3] = __float_as_uint(u23.y);
           }
           uint16_t* prow = myp + (4 * nt + t) * kPStride;
 #pragma unroll
           for (int e = 0; e < 4; ++e) prow[16 * (e >> 1) + g + 8 * (e & 1)] = (uint16_t)u[e];  // P' < 2^16
           psum[nt] += (u[0] + u[1]) + (u[2] + u[3]) - 4u * kMagicBits;
         }
-        __syncwarp();
+        const uint4 v0 = *reinterpret_cast<const uint4*>(s0 + kVcOff + 16 * lane);
+        const uint4 v1 = *reinterpret_cast<const uint4*>(s1 + kVcOff + 16 * lane);
+        __syncwarp();  // every lane has its value codes (and its P' row is written)
+        if (lane == 0) mbar_arrive(&empty[s]);
         // ---- values: acci[mt] += C_V (masked, row scale 4^f) . P'
-        const uint4 v0 = vw[0], v1 = vw[1];
         const uint32_t va[4] = {v0.x, v0.y, v0.z, v0.w};
         const uint32_t vb[4] = {v1.x, v1.y, v1.z, v1.w};
         uint32_t pb0[NT], pb1[NT];
@@ -1277,8 +1300,8 @@ __global__ void __launch_bounds__(kHW * 32, (G <= 4) ? 2 : 1) decode_heads_kerne
           const float* src = wo + hs * kD + 16 * g;
 #pragma unroll
           for (int i = 0; i < 16; ++i) v[i] = fmaf(v[i], ab, src[i] * aw);
-          st.l[nt] = fmaf(st.l[nt], ab, wl[nt] * aw);
-          st.msum[nt] *= ab;
+          st.l[nt] = make_float2(fmaf(st.l[nt].x + st.l[nt].y, ab, wl[nt] * aw), 0.f);
+          st.msum[nt] = make_float2((st.msum[nt].x + st.msum[nt].y) * ab, 0.f);
           st.m[nt] = M;
         }
         tacc_store(st.tacc + 16u * nt, v);
@@ -1290,7 +1313,7 @@ __global__ void __launch_bounds__(kHW * 32, (G <= 4) ? 2 : 1) decode_heads_kerne
     if (wph == 1) {
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
-        float l = st.l[nt], ms = st.msum[nt];
+        float l = st.l[nt].x + st.l[nt].y, ms = st.msum[nt].x + st.msum[nt].y;
 #pragma unroll
         for (int o = 4; o < 32; o <<= 1) {
           l += __shfl_xor_sync(0xffffffffu, l, o);
@@ -1314,7 +1337,7 @@ __global__ void __launch_bounds__(kHW * 32, (G <= 4) ? 2 : 1) decode_heads_kerne
       __syncthreads();  // window scratch no longer in use: the ring becomes merge buffers
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
-        float l = st.l[nt], ms = st.msum[nt];
+        float l = st.l[nt].x + st.l[nt].y, ms = st.msum[nt].x + st.msum[nt].y;
 #pragma unroll
         for (int o = 4; o < 32; o <<= 1) {
           l += __shfl_xor_sync(0xffffffffu, l, o);
@@ -1621,7 +1644,16 @@ static okv_status launch_decode_tail(const DecodeArgs& a, int B, cudaStream_t s)
   okv_status st = OKV_OK;
   cudaEvent_t ev0, ev1;
   take_decode_events(&ev0, &ev1);
-  if (ev0 != nullptr && cudaEventRecordWithFlags(ev0, s, cudaEventRecordExternal) != cudaSuccess)
+  // inside a stream capture the events become external event nodes of the
+  // graph, so that each replay records them; outside one they are recorded
+  // as usual
+  unsigned ev_flags = cudaEventRecordDefault;
+  if (ev0 != nullptr) {
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(s, &cs) != cudaSuccess) return fail(OKV_ERR_CUDA, "cudaStreamIsCapturing failed");
+    if (cs == cudaStreamCaptureStatusActive) ev_flags = cudaEventRecordExternal;
+  }
+  if (ev0 != nullptr && cudaEventRecordWithFlags(ev0, s, ev_flags) != cudaSuccess)
     return fail(OKV_ERR_CUDA, "cudaEventRecord failed");
   // Early (programmatic) launches overlap each kernel's start with its
   // predecessor; they are left out when the split-K kernel is being timed, so
@@ -1646,7 +1678,7 @@ static okv_status launch_decode_tail(const DecodeArgs& a, int B, cudaStream_t s)
     }
   }
   if (st != OKV_OK) return st;
-  if (ev1 != nullptr && cudaEventRecordWithFlags(ev1, s, cudaEventRecordExternal) != cudaSuccess)
+  if (ev1 != nullptr && cudaEventRecordWithFlags(ev1, s, ev_flags) != cudaSuccess)
     return fail(OKV_ERR_CUDA, "cudaEventRecord failed");
   static std::atomic<uint32_t> attr_set{0};
   cudaError_t e = set_smem_limit_once((const void*)combine_kernel, (int)kCombSmem, attr_set);
