@@ -391,6 +391,41 @@ def decode(cache: Cache, q: np.ndarray, seq_slots, context_lens, hq: int) -> np.
     return out
 
 
+def prefill(cache: Cache, q: np.ndarray, slot: int, context_len: int, hq: int) -> np.ndarray:
+    """Attention of a prefill chunk over the cache, causal.
+
+    The chunk's T tokens have been appended, so the sequence in `slot` has
+    `context_len` = L tokens and the chunk holds positions L - T .. L - 1.
+    q: [T, hq, d] (bf16-exact), query i at position L - T + i.  Query i of
+    head h attends to positions 0 .. L - T + i of KV head h // (hq // hkv),
+    each read as the cache holds it at length L (the first `sinks` and the
+    last W positions from fp16, the rest from INT2: `Cache.values`), with
+    q rotated by R_K and the output brought back with R_V^T, as in `decode`.
+    Returns fp64 [T, hq, d].  With T = 1 this is `decode` of that sequence.
+    [AF] "OSCAR: figyelem-tudatos…" and [GH] "Что это даёт на практике"
+    (the cache serves paged attention and prefix caching, so prefill chunks
+    attend over the compressed history); [GH] "Что придумали в Together AI"
+    (rotations of Q and of the attention output)."""
+    q = np.asarray(q)
+    T = q.shape[0]
+    g = hq // cache.hkv
+    out = np.zeros((T, hq, D))
+    if T == 0:
+        return out
+    if context_len < T:
+        raise ValueError("the chunk's tokens must already be in the cache")
+    first = context_len - T
+    for hk in range(cache.hkv):
+        kx = cache.values(slot, 0, hk, context_len)
+        vx = cache.values(slot, 1, hk, context_len)
+        for h in range(hk * g, (hk + 1) * g):
+            for i in range(T):
+                visible = first + i + 1
+                qr = np.asarray(q[i, h], dtype=np.float64) @ cache.r[0][hk]
+                out[i, h] = attend(qr, kx[:visible], vx[:visible]) @ cache.r[1][hk].T
+    return out
+
+
 # ----------------------------------------------------------------------------
 # Sizing arithmetic the pages quote
 # ----------------------------------------------------------------------------

@@ -511,3 +511,99 @@ def test_rotations_lower_weighted_logit_error():
     e_had = err(O.rotation(np.eye(128)))
     e_none = err(np.eye(128))
     assert e_oscar < e_none / 3 and e_had < e_none / 3
+
+
+# ------------------------------------------------------ chunked prefill attention
+
+def _brute_prefill_one(q, r_k, r_v, ent_k, ent_v, length, window, pos, sinks=0):
+    """Loop-only causal attention of one query at `pos` over a cache of
+    `length` tokens, each read as the cache holds it at that length."""
+    d = len(q)
+    qr = [sum(q[c] * r_k[c, j] for c in range(d)) for j in range(d)]
+
+    def val(ent, p):
+        codes, s16, m16, z16 = ent(p)
+        if p >= length - window or p < sinks:
+            return [float(z16[j]) for j in range(d)]
+        return [float(s16) * int(codes[j]) + float(m16) for j in range(d)]
+
+    logits = []
+    for p in range(pos + 1):  # the causal mask: positions 0 .. pos only
+        kv = val(ent_k, p)
+        logits.append(sum(qr[j] * kv[j] for j in range(d)) / math.sqrt(d))
+    mx = max(logits)
+    w = [math.exp(x - mx) for x in logits]
+    tot = sum(w)
+    o = [0.0] * d
+    for p in range(pos + 1):
+        vv = val(ent_v, p)
+        for j in range(d):
+            o[j] += w[p] * vv[j] / tot
+    return np.array([sum(o[j] * r_v[c, j] for j in range(d)) for c in range(d)])
+
+
+@pytest.mark.parametrize("sinks", [0, 4])
+def test_prefill_matches_loop_brute_force(sinks):
+    """A 9-token chunk at the end of a 27-token sequence, window 8: its early
+    queries see positions that are INT2 (older than the window of the whole
+    sequence) and its late ones reach into the window; GQA 2 to 1."""
+    cache, rng = _small_cache(20, 2, [27], window=8, sinks=sinks)
+    T, L = 9, 27
+    q = WL.to_bf16_exact(rng.standard_normal((T, 4, 128)).astype(np.float32))
+    got = O.prefill(cache, q, 0, L, hq=4)
+    for i in range(T):
+        for h in range(4):
+            hk = h // 2
+            want = _brute_prefill_one(q[i, h].astype(float), cache.r[0][hk], cache.r[1][hk],
+                                      lambda p: cache.entry(0, 0, hk, p), lambda p: cache.entry(0, 1, hk, p),
+                                      L, 8, L - T + i, sinks)
+            assert np.abs(got[i, h] - want).max() < 1e-10 * max(1.0, np.abs(want).max())
+
+
+def test_prefill_of_one_token_is_decode():
+    cache, rng = _small_cache(21, 2, [300, 41])
+    q = WL.to_bf16_exact(rng.standard_normal((1, 4, 128)).astype(np.float32))
+    for slot, L in enumerate((300, 41)):
+        assert np.array_equal(O.prefill(cache, q, slot, L, hq=4), O.decode(cache, q, [slot], [L], hq=4))
+
+
+def test_prefill_is_causal():
+    """Changing the last token's K and V moves only the last query's output."""
+    rng = np.random.default_rng(22)
+    uk, uv = WL.haar_orthogonal(rng)[None], WL.haar_orthogonal(rng)[None]
+    n = 200
+    k = WL.to_bf16_exact(rng.standard_normal((n, 1, 128)).astype(np.float32))
+    v = WL.to_bf16_exact(rng.standard_normal((n, 1, 128)).astype(np.float32))
+    a, b = O.Cache(1, uk, uv), O.Cache(1, uk, uv)
+    a.append(0, 0, k, v)
+    k2, v2 = k.copy(), v.copy()
+    k2[-1] *= -3.0
+    v2[-1] += 5.0
+    b.append(0, 0, k2, v2)
+    q = WL.to_bf16_exact(rng.standard_normal((16, 2, 128)).astype(np.float32))
+    oa, ob = O.prefill(a, q, 0, n, hq=2), O.prefill(b, q, 0, n, hq=2)
+    assert np.array_equal(oa[:-1], ob[:-1])
+    assert np.abs(oa[-1] - ob[-1]).max() > 1e-3
+
+
+def test_prefill_within_window_is_textbook_causal_attention():
+    """Every position in the fp16 window (L <= W): the chunk's attention is
+    masked softmax attention on the fp16 rotated operands (scipy's softmax
+    over an explicit lower-triangular mask)."""
+    rng = np.random.default_rng(23)
+    uk, uv = WL.haar_orthogonal(rng)[None], WL.haar_orthogonal(rng)[None]
+    cache = O.Cache(1, uk, uv)
+    n, T = 90, 30
+    k = WL.to_bf16_exact(rng.standard_normal((n, 1, 128)).astype(np.float32))
+    v = WL.to_bf16_exact(rng.standard_normal((n, 1, 128)).astype(np.float32))
+    cache.append(0, 0, k, v)
+    q = WL.to_bf16_exact(rng.standard_normal((T, 1, 128)).astype(np.float32))
+    got = O.prefill(cache, q, 0, n, hq=1)
+    kr = (k[:, 0].astype(np.float64) @ cache.r[0][0]).astype(np.float32).astype(np.float16).astype(float)
+    vr = (v[:, 0].astype(np.float64) @ cache.r[1][0]).astype(np.float32).astype(np.float16).astype(float)
+    qr = q[:, 0].astype(float) @ cache.r[0][0]
+    logits = qr @ kr.T / math.sqrt(128)
+    mask = np.arange(n)[None, :] <= (n - T + np.arange(T))[:, None]
+    p = scipy.special.softmax(np.where(mask, logits, -np.inf), axis=1)
+    want = (p @ vr) @ cache.r[1][0].T
+    assert np.abs(got[:, 0] - want).max() < 1e-12
