@@ -54,6 +54,8 @@ def parse():
     ap.add_argument("--workload", type=int, choices=[1, 2, 3, 4], default=2,
                     help="1: 8 x 32K (8B-class layer); 2: 4 x 100K decode (default, the headline); "
                          "3: 80 layers x 131K, G = 8; 4: 64 mixed contexts + an 8192-token prefill chunk")
+    ap.add_argument("--group", type=int, choices=[32, 64, 128], default=128,
+                    help="quantisation group (channels per fp16 scale/min); 128 is the headline format")
     ap.add_argument("--min-reps", type=int, default=50, help="timed replays of the K-step graph, at least")
     ap.add_argument("--min-timed-s", type=float, default=1.0, help="seconds of timed replays, at least")
     return ap.parse_args()
@@ -175,14 +177,20 @@ def workload_config(cfg=2):
     return WL.config(cfg)
 
 
-def algorithmic_bytes(lens, hkv):
-    """Cache bytes decode must read: 72 B per INT2 token-head (K and V codes,
-    scales, mins), 512 B per fp16 window token-head (K and V)."""
+def int2_bytes_per_token_head(group=128):
+    """K and V codes (2 x 32 B) and one fp16 (scale, min) pair per group for each (8 B per group)."""
+    return 64 + 8 * (128 // group)
+
+
+def algorithmic_bytes(lens, hkv, group=128):
+    """Cache bytes decode must read: 72 B per INT2 token-head with 128-channel
+    groups (80 B with 64, 96 B with 32), 512 B per fp16 window token-head (K and V)."""
+    per = int2_bytes_per_token_head(group)
     tot = 0
     for L in lens:
         n_int2 = max(0, L - 128)
         n_win = min(L, 128)
-        tot += hkv * (n_int2 * 72 + n_win * 512)
+        tot += hkv * (n_int2 * per + n_win * 512)
     return tot
 
 
@@ -248,7 +256,8 @@ class DecodeBatch:
     kernels_per_step = 3
     decode_launches_per_step = 1
 
-    def __init__(self, cfg, seed, rank, total_steps, torch, okv, WL):
+    def __init__(self, cfg, seed, rank, total_steps, torch, okv, WL, group=128):
+        self.group = group
         self.wl = wl = WL.config(cfg)
         self.cfg = cfg
         B, hq, hkv = wl.batch, wl.hq, wl.hkv
@@ -257,7 +266,7 @@ class DecodeBatch:
         qc, kc, vc = WL.calibration_set(seed, cfg, 0, hq, hkv, n=1024)
         rot = okv.calibrate_rotations(qc, kc, vc, hq, hkv)
         table, num_blocks = WL.block_table(seed + rank, cfg, [L0] * B, extra_tokens=total_steps + 16)
-        self.cache = okv.Cache(hq, hkv, num_blocks, B, table.shape[1], rot["U_K"], rot["U_V"])
+        self.cache = okv.Cache(hq, hkv, num_blocks, B, table.shape[1], rot["U_K"], rot["U_V"], group=group)
         self.table = torch.from_numpy(table).to(dev)
         gen, kv = _kv_source(torch, WL, seed, cfg, rank, hkv, dev)
         _prefill(torch, okv, self.cache, self.table, [L0] * B, kv, dev)
@@ -281,7 +290,7 @@ class DecodeBatch:
                         self.seq, self.table, self.lens[i], out=self.out, ws=self.ws)
 
     def decode_bytes(self, i):
-        return [algorithmic_bytes([self.L0 + i + 1] * self.B, self.hkv)]
+        return [algorithmic_bytes([self.L0 + i + 1] * self.B, self.hkv, self.group)]
 
     def e2e_parts(self):
         return [self.knew, self.vnew, self.q, self.pos, self.lens]
@@ -296,7 +305,7 @@ class DecodeBatch:
 
     def config(self):
         return {"workload": self.wl.name, "batch": self.B, "hq": self.hq, "hkv": self.hkv, "head_dim": 128,
-                "context_start": self.L0, "block_tokens": 16, "window": 128, "group": 128,
+                "context_start": self.L0, "block_tokens": 16, "window": 128, "group": self.group,
                 "step": "okv_decode_step: append 1 bf16 K/V token per sequence + decode attention",
                 "l2": (f"not flushed: each step reads the {self.decode_bytes(0)[0] / 1e6:.0f} MB cache, "
                        "larger than the 126 MB L2")}
@@ -309,7 +318,8 @@ class Layers:
     kernels_per_step = 3 * 80
     decode_launches_per_step = 80
 
-    def __init__(self, cfg, seed, rank, total_steps, torch, okv, WL):
+    def __init__(self, cfg, seed, rank, total_steps, torch, okv, WL, group=128):
+        self.group = group
         self.wl = wl = WL.config(cfg)
         self.cfg = cfg
         B, hq, hkv, L0, NL = wl.batch, wl.hq, wl.hkv, wl.ctx[0], wl.layers
@@ -322,7 +332,7 @@ class Layers:
             r = np.random.default_rng(np.random.SeedSequence([seed, cfg, layer, 31]))
             uk = np.stack([WL.haar_orthogonal(r) for _ in range(hkv)]).astype(np.float32)
             uv = np.stack([WL.haar_orthogonal(r) for _ in range(hkv)]).astype(np.float32)
-            c = okv.Cache(hq, hkv, num_blocks, B, table.shape[1], uk, uv)
+            c = okv.Cache(hq, hkv, num_blocks, B, table.shape[1], uk, uv, group=group)
             _prefill(torch, okv, c, self.table, [L0] * B, kv, dev)
             self.caches.append(c)
         torch.cuda.synchronize()
@@ -350,7 +360,7 @@ class Layers:
         self._layer_calls(okv, self.knew[i], self.vnew[i], self.q[i], self.pos[i], self.lens[i], self.out, ev)
 
     def decode_bytes(self, i):
-        return [algorithmic_bytes([self.L0 + i + 1] * self.B, self.hkv)] * self.NL
+        return [algorithmic_bytes([self.L0 + i + 1] * self.B, self.hkv, self.group)] * self.NL
 
     def e2e_parts(self):
         return [self.knew, self.vnew, self.q, self.pos, self.lens]
@@ -364,7 +374,7 @@ class Layers:
 
     def config(self):
         return {"workload": self.wl.name, "layers": self.NL, "batch": self.B, "hq": self.hq, "hkv": self.hkv,
-                "head_dim": 128, "context_start": self.L0, "block_tokens": 16, "window": 128, "group": 128,
+                "head_dim": 128, "context_start": self.L0, "block_tokens": 16, "window": 128, "group": self.group,
                 "step": "80 x okv_decode_step (one per layer): append 1 bf16 K/V token + decode attention",
                 "l2": (f"not flushed: each step reads {sum(self.decode_bytes(0)) / 1e9:.2f} GB of cache, "
                        "far more than the 126 MB L2")}
@@ -381,7 +391,8 @@ class Mixed:
     kernels_per_step = 3 + 1
     decode_launches_per_step = 1
 
-    def __init__(self, cfg, seed, rank, total_steps, torch, okv, WL):
+    def __init__(self, cfg, seed, rank, total_steps, torch, okv, WL, group=128):
+        self.group = group
         self.wl = wl = WL.config(cfg, seed=seed)
         self.cfg = cfg
         B, hq, hkv = wl.batch, wl.hq, wl.hkv
@@ -393,7 +404,7 @@ class Mixed:
         pre_len = S * self.CHUNK
         table, num_blocks = WL.block_table(seed + rank, cfg, lens0 + [pre_len - total_steps - 16],
                                            extra_tokens=total_steps + 16)
-        self.cache = okv.Cache(hq, hkv, num_blocks, B + 1, table.shape[1], rot["U_K"], rot["U_V"])
+        self.cache = okv.Cache(hq, hkv, num_blocks, B + 1, table.shape[1], rot["U_K"], rot["U_V"], group=group)
         self.table = torch.from_numpy(table).to(dev)
         gen, kv = _kv_source(torch, WL, seed, cfg, rank, hkv, dev)
         _prefill(torch, okv, self.cache, self.table, lens0, kv, dev, slot_lens=lens0 + [0])
@@ -430,7 +441,7 @@ class Mixed:
                     self.pv[i], self.ppos[i], self.out, ev)
 
     def decode_bytes(self, i):
-        return [algorithmic_bytes([L + i + 1 for L in self.lens0], self.hkv)]
+        return [algorithmic_bytes([L + i + 1 for L in self.lens0], self.hkv, self.group)]
 
     def e2e_parts(self):
         return [self.knew, self.vnew, self.q, self.pos, self.slot_lens, self.pk, self.pv, self.ppos]
@@ -445,7 +456,7 @@ class Mixed:
     def config(self):
         return {"workload": self.wl.name, "batch": self.B, "hq": self.hq, "hkv": self.hkv, "head_dim": 128,
                 "contexts": "log-uniform in [1024, 65536], seeded", "context_total": int(sum(self.lens0)),
-                "prefill_append_tokens": self.CHUNK, "block_tokens": 16, "window": 128, "group": 128,
+                "prefill_append_tokens": self.CHUNK, "block_tokens": 16, "window": 128, "group": self.group,
                 "step": ("okv_decode_step (1 bf16 token per sequence + decode) and okv_append_quantize of an "
                          "8192-token bf16 prefill chunk"),
                 "l2": (f"not flushed: each step reads {self.decode_bytes(0)[0] / 1e6:.0f} MB of cache and "
@@ -486,14 +497,49 @@ def prefill_append_rate(torch, okv, WL, seed):
             "bytes": moved}
 
 
+def prefill_attention_rate(torch, okv, WL, seed, L=32768, T=1024):
+    """Chunked-prefill attention: a T-token chunk at the end of an L-token
+    sequence (32 query / 8 KV heads) attends causally over the cache; median
+    of 10 launches.  flops counts the causal score and value products
+    (2 x 2 x 128 per visible (query head, key) pair)."""
+    hq, hkv = 32, 8
+    table, nb = WL.block_table(seed, 1, [L], extra_tokens=16)
+    r = np.random.default_rng(seed + 5)
+    uk = np.stack([WL.haar_orthogonal(r) for _ in range(hkv)]).astype(np.float32)
+    cache = okv.Cache(hq, hkv, nb, 1, table.shape[1], uk, uk)
+    dev = torch.device("cuda")
+    td = torch.from_numpy(table).to(dev)
+    gen, kv = _kv_source(torch, WL, seed, 1, 0, hkv, dev)
+    _prefill(torch, okv, cache, td, [L], kv, dev)
+    q = torch.randn((T, hq, 128), generator=gen, device=dev).to(torch.bfloat16)
+    ws = torch.empty(okv.prefill_workspace_bytes(cache, T), dtype=torch.uint8, device=dev)
+    out = torch.empty((T, hq, 128), dtype=torch.float32, device=dev)
+    for _ in range(2):
+        okv.prefill_attention(cache, q, 0, L, td, out=out, ws=ws)
+    torch.cuda.synchronize()
+    ts = []
+    for _ in range(10):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        okv.prefill_attention(cache, q, 0, L, td, out=out, ws=ws)
+        e1.record()
+        torch.cuda.synchronize()
+        ts.append(e0.elapsed_time(e1) * 1e3)
+    us = statistics.median(ts)
+    visible = sum(L - T + i + 1 for i in range(T))
+    flops = 4 * 128 * hq * visible
+    return {"context": L, "chunk_tokens": T, "hq": hq, "hkv": hkv, "us": round(us, 1),
+            "tflops": round(flops / us / 1e6, 1), "flops": flops}
+
+
 # ---------------------------------------------------------------- oracle arm
 
-def oracle_unit(seed, cfg, L, g):
+def oracle_unit(seed, cfg, L, g, group=128):
     """Oracle cache for one (sequence, KV head) unit at L tokens."""
     from int2_kv_cache_rotate_b200 import workloads as WL
     from oracle import okv_oracle as O
     r = np.random.default_rng(np.random.SeedSequence([seed, 77]))
-    cache = O.Cache(1, WL.haar_orthogonal(r)[None], WL.haar_orthogonal(r)[None])
+    cache = O.Cache(1, WL.haar_orthogonal(r)[None], WL.haar_orthogonal(r)[None], group=group)
     k = WL.sample_keys(seed, cfg, 0, 0, L, extra=0)[:, None, :]
     v = WL.sample_values(seed, cfg, 0, 0, L, extra=0)[:, None, :]
     cache.append(0, 0, k, v)
@@ -536,7 +582,7 @@ class OracleSample:
     total token-heads (over layers and KV heads).  Workload 4 adds the oracle
     append of the step's 8192-token chunk, timed on 256 tokens of one head."""
 
-    def __init__(self, cfg, seed):
+    def __init__(self, cfg, seed, group=128):
         wl = workload_config(cfg) if cfg != 4 else __import__(
             "int2_kv_cache_rotate_b200.workloads", fromlist=["config"]).config(4, seed=seed)
         self.cfg, self.wl, self.seed = cfg, wl, seed
@@ -544,7 +590,7 @@ class OracleSample:
         self.L = int(statistics.median(lens))
         self.g = wl.hq // wl.hkv
         self.scale = sum(lens) * wl.hkv * wl.layers / self.L  # token-heads of a step / the unit's tokens
-        self.unit = oracle_unit(seed, cfg, self.L, self.g)
+        self.unit = oracle_unit(seed, cfg, self.L, self.g, group)
         self.app_tokens = wl.prefill_append * wl.hkv  # token-heads appended by the prefill chunk
 
     def step_seconds(self, i):
@@ -564,9 +610,9 @@ class OracleSample:
         return txt
 
 
-def cpu_baseline(cfg, seed, steps=3):
+def cpu_baseline(cfg, seed, steps=3, group=128):
     cores = len(os.sched_getaffinity(0))
-    o = OracleSample(cfg, seed)
+    o = OracleSample(cfg, seed, group)
     ts = [o.step_seconds(i)[0] for i in range(steps)]
     step_s = statistics.median(ts)
     out = {"value": round(o.wl.batch / step_s, 6), "unit": "tok/s", "cores": cores, "kind": "oracle",
@@ -581,15 +627,16 @@ def run_reference(args):
     if rank != 0:
         return 0
     cfg = getattr(args, "workload", 2)
+    group = getattr(args, "group", 128)
     cores = len(os.sched_getaffinity(0))
-    o = OracleSample(cfg, args.seed)
+    o = OracleSample(cfg, args.seed, group)
     for i in range(args.warmup):
         o.step_seconds(i)
     res = [o.step_seconds(args.warmup + i) for i in range(args.steps)]
     per_step = sum(r[0] for r in res) / len(res)
     per_unit = sum(r[1] for r in res) / len(res)
     value = o.wl.batch / per_step
-    cfgblock = reference_config_block(o.wl, cfg)
+    cfgblock = dict(reference_config_block(o.wl, cfg), group=group)
     line = {
         "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "tok/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(per_step * 1e3, 3),
@@ -740,7 +787,7 @@ def run_ours(args):
     K, W = args.steps, args.warmup
     e2e_steps = 0 if args.no_e2e else K
     total = W + K + e2e_steps + 1
-    w = BUILDERS[args.workload](args.workload, args.seed, rank, total, torch, okv, WL)
+    w = BUILDERS[args.workload](args.workload, args.seed, rank, total, torch, okv, WL, group=args.group)
     # eager pre-warm (idempotent with graph step 0: same tokens, same positions)
     w.issue(okv, 0)
     torch.cuda.synchronize()
@@ -791,6 +838,7 @@ def run_ours(args):
 
     e2e = run_e2e(w, W + K, e2e_steps, torch, okv, world, dist) if e2e_steps else None
     append_rate = prefill_append_rate(torch, okv, WL, args.seed) if rank == 0 else None
+    prefill_rate = prefill_attention_rate(torch, okv, WL, args.seed) if rank == 0 and args.workload == 2 else None
 
     if rank == 0:
         alg = statistics.mean(statistics.mean(w.decode_bytes(W + i)) for i in range(K))
@@ -817,9 +865,12 @@ def run_ours(args):
             "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                          "frac": round(achieved / peak, 4), "peak_source": peak_src,
                          "traffic": (tr["bytes_per_launch"] if tr else None),
-                         "kernel": "split-K INT2 decode attention",
+                         "kernel": ("split-K INT2 decode attention" if args.group == 128 else
+                                    "split-K INT2 decode attention, per-group scales (CUDA-core kernel)"),
+                         "int2_bytes_per_token_head": int2_bytes_per_token_head(args.group),
                          "algorithmic_bytes_per_launch": int(alg)},
             "append_prefill": append_rate,
+            "prefill_attention": prefill_rate,
             "e2e": e2e,
             "gpu_launches": w.kernels_per_step * K * len(reps_ms),
             "clocks": clk,
@@ -830,7 +881,7 @@ def run_ours(args):
                                       "mtok_s_at_step_rate": round(Mixed.CHUNK * K / (ms * 1e3), 3),
                                       "bytes_per_step": step_app}
         if not args.no_cpu_baseline and world == 1:
-            line["cpu_baseline"] = cpu_baseline(args.workload, args.seed)
+            line["cpu_baseline"] = cpu_baseline(args.workload, args.seed, group=args.group)
         print(json.dumps(line), flush=True)
     del g_warm, g_time, g_kern
     if world > 1:

@@ -23,8 +23,13 @@
  *
  * Conventions
  *   - Row vectors: x_rot = x R.  Matrices are row-major fp32.
- *   - d (head_dim) = 128, quantisation group = 128 (one group per token-head),
- *     16 tokens per block, fp16 window W = 128 tokens.  Other values return
+ *   - d (head_dim) = 128, 16 tokens per block, fp16 window W = 128 tokens;
+ *     quantisation group g = 128 (one group per token-head), 64 or 32
+ *     channels.  The groups are runs of consecutive channels after the
+ *     rotation, so with g < 128 the bit-reversal permutation hands every
+ *     group an even share of the importance order that U and H leave (the
+ *     reason the pages give for P_br: gen-hub.ru "Что придумали в Together
+ *     AI").  Effective bits per element: 2 + 32/g.  Other values return
  *     OKV_ERR_UNSUPPORTED.
  *   - "device" pointers point to memory of the current CUDA device; "host"
  *     pointers to ordinary host memory.  The caller owns every buffer; the
@@ -39,16 +44,21 @@
  *   - okv_last_error_string() describes the last non-OK status of the
  *     calling thread.
  *
- * Physical layout of one block (16 tokens) of one KV head: 1152 bytes
+ * Physical layout of one block (16 tokens) of one KV head, with ng = 128/g
+ * groups per token: 1024 + 128 ng bytes (1152, 1280 or 1536 for g = 128, 64,
+ * 32; okv_block_head_bytes)
  *   [   0,  512) K codes, token-major: 16 rows of 32 bytes; byte b of row t
  *                holds channels 4b..4b+3 of token t at bits 0-1, 2-3, 4-5, 6-7
  *                (channel = index after the rotation, i.e. after P_br).
  *   [ 512, 1024) V codes, the same bytes regrouped: 32 chunks of 16 bytes;
  *                byte b of token t sits at 512 + ((b>>2)*4 + (t>>2))*16
  *                + (b&3)*4 + (t&3).
- *   [1024, 1088) K scale and min: token t at 1024 + 4t, fp16 scale then fp16 min.
- *   [1088, 1152) V scale and min, the same.
- * Block `blk`, head `h` starts at pages + (blk * num_kv_heads + h) * 1152.
+ *   [1024, 1024 + 64 ng) K scale and min: token t, group k (channels
+ *                k g .. k g + g - 1) at 1024 + 4 (t ng + k), fp16 scale then
+ *                fp16 min.
+ *   [1024 + 64 ng, 1024 + 128 ng) V scale and min, the same.
+ * Block `blk`, head `h` starts at pages + (blk * num_kv_heads + h) *
+ * okv_block_head_bytes(g).
  * Window ring: fp16 [num_seq_slots][num_kv_heads][2 (K,V)][W][d]; position p
  * of a sequence lives in row p % W; values are the rotated vector in fp16.
  * Sink rows: fp16 [num_seq_slots][num_kv_heads][2 (K,V)][num_sink][d];
@@ -91,13 +101,13 @@ typedef enum {
 #define OKV_BLOCK_TOKENS 16
 #define OKV_WINDOW 128
 #define OKV_MAX_SINK 1024
-#define OKV_BLOCK_HEAD_BYTES 1152
+#define OKV_BLOCK_HEAD_BYTES 1152  /* bytes of one block-head with g = 128 */
 
 typedef struct {
   int32_t num_q_heads;        /* Hq; a multiple of num_kv_heads            */
   int32_t num_kv_heads;       /* Hkv                                        */
   int32_t head_dim;           /* must be 128                                */
-  int32_t group;              /* must be 128                                */
+  int32_t group;              /* quantisation group: 128, 64 or 32 channels */
   int32_t block_tokens;       /* must be 16                                 */
   int32_t window;             /* must be 128                                */
   int32_t num_blocks;         /* physical blocks in `pages`                 */
@@ -159,8 +169,15 @@ okv_status okv_rotations_file_shape(const char* path, int32_t* num_layers, int32
 okv_status okv_load_rotations(const char* path, int32_t num_layers, int32_t num_kv_heads, int32_t d, float* u_k,
                               float* u_v, char* tag, size_t tag_capacity, int32_t verify);
 
+/* Bytes of one block-head (16 tokens of one KV head) for quantisation group
+ * `group` (1152, 1280, 1536 for 128, 64, 32), 0 for an unsupported group.
+ * The pages' INT2 format with a scale and a minimum per group (bigsaas.top,
+ * "Revolução no Serviço de LLMs…", section "Resultados e Métricas de
+ * Desempenho"). */
+size_t okv_block_head_bytes(int32_t group);
+
 /* Bytes the caller allocates for `pages`, `window_ring` and `sink_rows`. */
-size_t okv_pages_bytes(int32_t num_blocks, int32_t num_kv_heads);
+size_t okv_pages_bytes(int32_t num_blocks, int32_t num_kv_heads, int32_t group);
 size_t okv_window_bytes(int32_t num_seq_slots, int32_t num_kv_heads);
 size_t okv_sink_bytes(int32_t num_seq_slots, int32_t num_kv_heads, int32_t num_sink);
 
@@ -256,6 +273,32 @@ okv_status okv_decode_step(const okv_cache_desc* desc, const void* k, const void
 okv_status okv_decode_attention_noalloc(const okv_cache_desc* desc, const void* q, int32_t B,
                                         const int32_t* seq_slot, const int32_t* block_table,
                                         const int32_t* context_lens, float* out, void* stream);
+
+/* Chunked-prefill attention over the cache, for one sequence.  The chunk's
+ * T tokens must already be appended (okv_append_quantize), so sequence
+ * `slot` holds context_len = L tokens and the chunk is positions L - T ..
+ * L - 1.  Query i (position L - T + i) of head j attends to positions
+ * 0 .. L - T + i of KV head j/(Hq/Hkv), causally, each read as the cache
+ * holds it at length L: positions [0, min(S, L)) from the sink rows,
+ * [max(L - W, S), L) from the window ring, the rest from INT2 blocks.  As in
+ * decode, q~ = q R_K and o = softmax(q~ x^T / sqrt(d)) x_V R_V^T.
+ *   q: device bf16 [T][Hq][d]; slot, context_len: host ints (T <= L <=
+ *   max_blocks_per_seq * 16); block_table: device, as above; out: device
+ *   fp32 [T][Hq][d]; workspace: device, at least
+ *   okv_prefill_workspace_bytes(desc, T) bytes, 256-B aligned.
+ * Three launches on `stream` (query rotation, attention on the tensor cores,
+ * normalisation and value un-rotation).  Errors: INVALID_ARG (NULL, sizes,
+ * slot or context_len out of range, workspace too small); block ids outside
+ * [0, num_blocks) set OKV_DEV_BAD_BLOCK and those positions are skipped.
+ * Pages: aiforradalom.hu, "Az Apple, a Google és a NYU új technikái…",
+ * section "OSCAR: figyelem-tudatos és bevetésre kész", and gen-hub.ru
+ * "Что это даёт на практике" (the compressed cache serves paged attention
+ * and prefix caching, so a prefill chunk attends over the INT2 history);
+ * gen-hub.ru "Что придумали в Together AI" (the rotations of Q and of SV). */
+size_t okv_prefill_workspace_bytes(const okv_cache_desc* desc, int32_t T);
+okv_status okv_prefill_attention(const okv_cache_desc* desc, const void* q, int32_t T, int32_t slot,
+                                 int32_t context_len, const int32_t* block_table, float* out, void* workspace,
+                                 size_t workspace_bytes, void* stream);
 
 /* Gather and dequantise the cache into dense fp32 (the INT2 format's inverse:
  * s*c + m with the fp16 scale and minimum of each group; bigsaas.top,

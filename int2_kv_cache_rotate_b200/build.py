@@ -12,7 +12,8 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libokv.so")
-SOURCES = ["okv_api.cu", "append.cu", "decode.cu", "dequant.cu", "noalloc.cu", "calib.cpp", "rotio.cpp"]
+SOURCES = ["okv_api.cu", "append.cu", "decode.cu", "dequant.cu", "prefill.cu", "noalloc.cu", "calib.cpp",
+           "rotio.cpp"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

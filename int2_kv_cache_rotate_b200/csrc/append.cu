@@ -68,8 +68,11 @@ __device__ __forceinline__ int tc_column(int b, int f) {
 }
 
 // One token held by the four lanes of a quad: v[k][f] = rotated channel
-// 4 (8t + k) + f.  The min/max reduction runs on every lane (the quad
-// shuffles need all of them); `live` then gates validation and the stores.
+// 4 (8t + k) + f, so lane t holds channels 32t .. 32t + 31, one 32-channel
+// quarter.  With ng groups per vector a group is 4 / ng quarters, and the
+// min/max reduction runs over that many lanes of the quad.  It runs on every
+// lane (the quad shuffles need all of them); `live` then gates validation
+// and the stores.
 __device__ __forceinline__ void finish_token_tc(const AppendArgs& a, int tok, bool live, int h, int kind,
                                                 const float (&v)[8][4], int t) {
   float mn = v[0][0], mx = v[0][0];
@@ -80,10 +83,14 @@ __device__ __forceinline__ void finish_token_tc(const AppendArgs& a, int tok, bo
       mn = fminf(mn, v[k][f]);
       mx = fmaxf(mx, v[k][f]);
     }
-  mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, 1));
-  mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-  mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, 2));
-  mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+  if (a.ng < 4) {
+    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, 1));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+  }
+  if (a.ng < 2) {
+    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, 2));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+  }
   if (!live) return;
   const int slot = a.seq_slot[tok];
   const int p = a.pos[tok];
@@ -115,7 +122,7 @@ __device__ __forceinline__ void finish_token_tc(const AppendArgs& a, int tok, bo
 #pragma unroll
       for (int f = 0; f < 4; ++f) w[k >> 2] |= int2_code(__fsub_rn(v[k][f], m), th) << (8 * (k & 3) + 2 * f);
   }
-  uint8_t* base = a.pages + ((size_t)blk * a.hkv + h) * kBlockHeadBytes;
+  uint8_t* base = a.pages + ((size_t)blk * a.hkv + h) * a.bhb;
   const int sl = p & 15;
   if (kind == 0) {
     *reinterpret_cast<uint2*>(base + kKcOff + sl * 32 + 8 * t) = make_uint2(w[0], w[1]);
@@ -123,8 +130,8 @@ __device__ __forceinline__ void finish_token_tc(const AppendArgs& a, int tok, bo
 #pragma unroll
     for (int k = 0; k < 8; ++k) base[v_code_offset(sl, 8 * t + k)] = (uint8_t)(w[k >> 2] >> (8 * (k & 3)));
   }
-  if (t == 0)
-    *reinterpret_cast<uint32_t*>(base + (kind ? kVsmOff : kKsmOff) + 4 * sl) =
+  if ((t & (4 / a.ng - 1)) == 0)  // the first lane of each group
+    *reinterpret_cast<uint32_t*>(base + sm_offset(a.ng, kind, sl, t * a.ng / 4)) =
         (uint32_t)__half_as_ushort(s16) | ((uint32_t)__half_as_ushort(m16) << 16);
   __half* wrow = window_row(a, slot, h, kind, p, len);
   __half* srow = sink_row(a, slot, h, kind, p);
@@ -269,6 +276,12 @@ constexpr int kUmEpiWarps = 8;
 constexpr int kUmProducer = kUmEpiWarps;             // warp index of the producer
 constexpr int kUmThreads = 32 * (kUmEpiWarps + 1);
 constexpr int kUmTile = 128;
+// value codes of four consecutive slots written as 4-byte words after a byte
+// transpose across the quad of lanes that holds them (else one byte store each)
+#ifndef OKV_UM_QUAD_STORES
+#define OKV_UM_QUAD_STORES 1
+#endif
+constexpr bool kUmQuadStores = OKV_UM_QUAD_STORES != 0;
 constexpr int kUmStages = 3;
 constexpr uint32_t kUmRegion = 16384;                 // 128 rows x 128 B
 constexpr uint32_t kUmBBytes = 6 * kUmRegion;         // 3 parts x 2 K-blocks
@@ -343,6 +356,7 @@ __device__ __forceinline__ void um_ld32(uint32_t taddr, float* v) {
 
 __device__ __forceinline__ void um_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory"); }
 
+template <int NG>
 __global__ void __launch_bounds__(kUmThreads, 1) append_umma_kernel(AppendArgs a, int T,
                                                                      const __grid_constant__ CUtensorMap map_k,
                                                                      const __grid_constant__ CUtensorMap map_v) {
@@ -531,48 +545,94 @@ __global__ void __launch_bounds__(kUmThreads, 1) append_umma_kernel(AppendArgs a
       um_wait_ld();
       um_fence_before();
       mbar_arrive(&tmem_free[i & 1]);  // the buffer may take tile i + 2's MMAs
-      if (tok >= T) continue;
-      if (!slot_ok) {
+      // every lane stays in the loop body (the value codes below are
+      // exchanged across quads of lanes); `valid` gates the stores
+      bool valid = tok < T;
+      if (valid && !slot_ok) {
         raise_flag(a.status, OKV_DEV_BAD_SLOT);
-        continue;
-      }
-      if (!pos_ok) {
+        valid = false;
+      } else if (valid && !pos_ok) {
         raise_flag(a.status, OKV_DEV_BAD_POS);
-        continue;
-      }
-      if (blk < 0 || blk >= a.num_blocks) {
+        valid = false;
+      } else if (valid && (blk < 0 || blk >= a.num_blocks)) {
         raise_flag(a.status, OKV_DEV_BAD_BLOCK);
-        continue;
+        valid = false;
       }
-      float mn = v[0], mx = v[0];
-#pragma unroll
-      for (int j = 1; j < 128; ++j) {
-        mn = fminf(mn, v[j]);
-        mx = fmaxf(mx, v[j]);
-      }
-      const float s32 = __fdiv_rn(__fsub_rn(mx, mn), 3.0f);
-      const __half s16 = fp16_sat(s32);
-      const __half m16 = fp16_sat(mn);
-      const float sc = __half2float(s16);
-      const float m = __half2float(m16);
+      // per group (NG per vector, 128 / NG channels each): min and max, the
+      // fp16 scale and minimum, and the codes
+      constexpr int GW = kD / NG;
       uint32_t w[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};  // the 32 code bytes of the token
-      if (sc != 0.0f) {
-        const CodeThresholds th = code_thresholds(sc);
+      uint32_t smg[NG];                                    // (scale, min) bits of each group
 #pragma unroll
-        for (int j = 0; j < 128; ++j) w[j >> 4] |= int2_code(__fsub_rn(v[j], m), th) << (2 * (j & 15));
+      for (int k = 0; k < NG; ++k) {
+        float mn = v[GW * k], mx = v[GW * k];
+#pragma unroll
+        for (int j = GW * k + 1; j < GW * (k + 1); ++j) {
+          mn = fminf(mn, v[j]);
+          mx = fmaxf(mx, v[j]);
+        }
+        const float s32 = __fdiv_rn(__fsub_rn(mx, mn), 3.0f);
+        const __half s16 = fp16_sat(s32);
+        const __half m16 = fp16_sat(mn);
+        const float sc = __half2float(s16);
+        const float m = __half2float(m16);
+        smg[k] = (uint32_t)__half_as_ushort(s16) | ((uint32_t)__half_as_ushort(m16) << 16);
+        if (sc != 0.0f) {
+          const CodeThresholds th = code_thresholds(sc);
+#pragma unroll
+          for (int j = GW * k; j < GW * (k + 1); ++j) w[j >> 4] |= int2_code(__fsub_rn(v[j], m), th) << (2 * (j & 15));
+        }
       }
-      uint8_t* bp = a.pages + ((size_t)blk * a.hkv + h) * kBlockHeadBytes;
+      uint8_t* bp = a.pages + ((size_t)(valid ? blk : 0) * a.hkv + h) * a.bhb;
       const int sl = p & 15;
       if (kind == 0) {
-        uint4* kp = reinterpret_cast<uint4*>(bp + kKcOff + sl * 32);
-        kp[0] = make_uint4(w[0], w[1], w[2], w[3]);
-        kp[1] = make_uint4(w[4], w[5], w[6], w[7]);
-      } else {
+        if (valid) {
+          uint4* kp = reinterpret_cast<uint4*>(bp + kKcOff + sl * 32);
+          kp[0] = make_uint4(w[0], w[1], w[2], w[3]);
+          kp[1] = make_uint4(w[4], w[5], w[6], w[7]);
+        }
+      } else if constexpr (kUmQuadStores) {
+        // The value codes of four tokens in slots 4j .. 4j + 3 of one block
+        // share 4-byte words (byte b of those tokens, one per token).  When
+        // the four lanes of a quad hold exactly such tokens, in slot order,
+        // a 4 x 4 byte transpose across the quad turns lane i's share into
+        // the eight words of code bytes b = 4k + i; otherwise each lane
+        // writes its 32 bytes one by one.
+        const int qbase = lane & ~3, qi = lane & 3;
+        const int blk0 = __shfl_sync(0xffffffffu, blk, qbase);
+        const int grp0 = __shfl_sync(0xffffffffu, p >> 2, qbase);
+        const bool fits = valid && blk == blk0 && (p >> 2) == grp0 && (p & 3) == qi;
+        const uint32_t fit_mask = __ballot_sync(0xffffffffu, fits);
+        const bool quad_ok = ((fit_mask >> qbase) & 0xfu) == 0xfu;
+        uint32_t tw[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          // byte qi of word k from each lane of the quad
+          const uint32_t x0 = __shfl_sync(0xffffffffu, w[k], qbase + 0);
+          const uint32_t x1 = __shfl_sync(0xffffffffu, w[k], qbase + 1);
+          const uint32_t x2 = __shfl_sync(0xffffffffu, w[k], qbase + 2);
+          const uint32_t x3 = __shfl_sync(0xffffffffu, w[k], qbase + 3);
+          const uint32_t sel = (uint32_t)qi * 0x11u + 0x40u;  // result bytes 0, 1: byte qi of the first, of the second
+          const uint32_t lo = prmt(x0, x1, sel);
+          const uint32_t hi = prmt(x2, x3, sel);
+          tw[k] = prmt(lo, hi, 0x5410u);  // [x0.qi, x1.qi, x2.qi, x3.qi]
+        }
+        if (quad_ok) {
+          // word of code byte b = 4k + qi for slots 4 (sl >> 2) .. + 3
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            *reinterpret_cast<uint32_t*>(bp + kVcOff + ((k * 4 + (sl >> 2)) << 4) + (qi << 2)) = tw[k];
+        } else if (valid) {
+#pragma unroll
+          for (int bb = 0; bb < 32; ++bb) bp[v_code_offset(sl, bb)] = (uint8_t)(w[bb >> 2] >> (8 * (bb & 3)));
+        }
+      } else if (valid) {
 #pragma unroll
         for (int bb = 0; bb < 32; ++bb) bp[v_code_offset(sl, bb)] = (uint8_t)(w[bb >> 2] >> (8 * (bb & 3)));
       }
-      *reinterpret_cast<uint32_t*>(bp + (kind ? kVsmOff : kKsmOff) + 4 * sl) =
-          (uint32_t)__half_as_ushort(s16) | ((uint32_t)__half_as_ushort(m16) << 16);
+      if (!valid) continue;
+#pragma unroll
+      for (int k = 0; k < NG; ++k) *reinterpret_cast<uint32_t*>(bp + sm_offset(NG, kind, sl, k)) = smg[k];
       __half* wr = window_row(a, slot, h, kind, p, len);
       __half* sr = sink_row(a, slot, h, kind, p);
       if (wr != nullptr || sr != nullptr) {
@@ -643,14 +703,20 @@ okv_status launch_append(const okv_cache_desc* d, const void* k, const void* v, 
   const bool maps = !(flags & OKV_PRE_ROTATED) && T >= kTcMinTokens && rows16 &&
                     encode_tile_map(&map_k, k, d->num_kv_heads, T) && encode_tile_map(&map_v, v, d->num_kv_heads, T);
   if (maps) {
-    static std::atomic<uint32_t> attr_set{0};
-    cudaError_t e = set_smem_limit_once((const void*)append_umma_kernel, (int)kUmSmem, attr_set);
+    const void* kern = a.ng == 1 ? (const void*)append_umma_kernel<1>
+                       : a.ng == 2 ? (const void*)append_umma_kernel<2> : (const void*)append_umma_kernel<4>;
+    static std::atomic<uint32_t> attr_set[3];  // per instantiation: ng = 1, 2, 4 -> 0, 1, 2
+    cudaError_t e = set_smem_limit_once(kern, (int)kUmSmem, attr_set[a.ng >> 1]);
     if (e != cudaSuccess) return fail(OKV_ERR_CUDA, "append smem attribute: %s", cudaGetErrorString(e));
     const int pairs = 2 * d->num_kv_heads;
     const int tiles = (T + kUmTile - 1) / kUmTile;
     const int per_pair = std::max(1, std::min(tiles, device_sm_count() / pairs));
     dim3 grid(per_pair, d->num_kv_heads, 2);
-    append_umma_kernel<<<grid, kUmThreads, kUmSmem, s>>>(a, T, map_k, map_v);
+    switch (a.ng) {
+      case 1: append_umma_kernel<1><<<grid, kUmThreads, kUmSmem, s>>>(a, T, map_k, map_v); break;
+      case 2: append_umma_kernel<2><<<grid, kUmThreads, kUmSmem, s>>>(a, T, map_k, map_v); break;
+      default: append_umma_kernel<4><<<grid, kUmThreads, kUmSmem, s>>>(a, T, map_k, map_v); break;
+    }
     return check_launch("append (tcgen05)");
   }
   if (!(flags & OKV_PRE_ROTATED) && T >= kTcMinTokens) {

@@ -25,6 +25,8 @@ struct AppendArgs {
   float* rotated_out;
   uint32_t* status;
   int hkv, num_blocks, num_slots, mbps, nsink;
+  int ng;   // quantisation groups per vector (128 / group)
+  int bhb;  // bytes of one block-head
 };
 
 inline AppendArgs make_append_args(const okv_cache_desc* d, const void* k, const void* v, const int32_t* seq_slot,
@@ -49,6 +51,8 @@ inline AppendArgs make_append_args(const okv_cache_desc* d, const void* k, const
   a.num_blocks = d->num_blocks;
   a.num_slots = d->num_seq_slots;
   a.mbps = d->max_blocks_per_seq;
+  a.ng = kD / d->group;
+  a.bhb = block_head_bytes(a.ng);
   return a;
 }
 
@@ -93,15 +97,16 @@ __device__ __forceinline__ void finish_token(const AppendArgs& a, int t, int h, 
     float4 o = make_float4(y[0], y[2], y[1], y[3]);
     *reinterpret_cast<float4*>(a.rotated_out + (((size_t)t * 2 + kind) * a.hkv + h) * kD + 4 * r) = o;
   }
-  const Quantized q = quantize_warp(y);
-  uint8_t* base = a.pages + ((size_t)blk * a.hkv + h) * kBlockHeadBytes;
+  const Quantized q = quantize_warp(y, a.ng);
+  uint8_t* base = a.pages + ((size_t)blk * a.hkv + h) * a.bhb;
   const int s16 = p & 15;
   if (kind == 0) {
     base[kKcOff + s16 * 32 + r] = (uint8_t)q.byte;
   } else {
     base[v_code_offset(s16, r)] = (uint8_t)q.byte;
   }
-  if (lane == 0) *reinterpret_cast<uint32_t*>(base + (kind ? kVsmOff : kKsmOff) + 4 * s16) = q.sm;
+  // one lane per group (lanes 0 .. ng - 1) writes its group's scale and min
+  if (lane < a.ng) *reinterpret_cast<uint32_t*>(base + sm_offset(a.ng, kind, s16, r * a.ng / 32)) = q.sm;
   __half* wrow = window_row(a, slot, h, kind, p, len);
   __half* srow = sink_row(a, slot, h, kind, p);
   if (wrow != nullptr || srow != nullptr) {

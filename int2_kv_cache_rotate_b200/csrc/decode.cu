@@ -96,6 +96,7 @@ struct DecodeArgs {
   int32_t* prefix;   // [B+1] cost prefix over batch entries
   float* part;       // [(NC + B)][Hq][kPartStride]
   int batch, hq, hkv, g, nc, num_blocks, num_slots, mbps, nsink;
+  int ng;  // quantisation groups per vector (128 / group)
 };
 
 // split-K CTA count actually used: with fewer cost units than CTAs only the
@@ -264,12 +265,14 @@ __device__ __forceinline__ void simt_chunk(const DecodeArgs& a, const float* qs 
   if (valid) {
     if constexpr (!kWindow) {
       const uint4 w = *reinterpret_cast<const uint4*>(blockp + kKcOff + tt * 32 + 16 * half);
-      const uint32_t smk = *reinterpret_cast<const uint32_t*>(blockp + kKsmOff + 4 * tt);
-      const float s = __half2float(__ushort_as_half((unsigned short)(smk & 0xffff)));
-      const float m = __half2float(__ushort_as_half((unsigned short)(smk >> 16)));
       const uint32_t words[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
       for (int wi = 0; wi < 4; ++wi) {
+        // channels 64 half + 16 wi .. + 15: group (4 half + wi) ng / 8
+        const uint32_t smk =
+            *reinterpret_cast<const uint32_t*>(blockp + sm_offset(a.ng, 0, tt, (4 * half + wi) * a.ng / 8));
+        const float s = __half2float(__ushort_as_half((unsigned short)(smk & 0xffff)));
+        const float m = __half2float(__ushort_as_half((unsigned short)(smk >> 16)));
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
           const int c = 64 * half + 16 * wi + j;
@@ -318,7 +321,7 @@ __device__ __forceinline__ void simt_chunk(const DecodeArgs& a, const float* qs 
     float x[4];
     if constexpr (!kWindow) {
       const uint32_t byte = blockp[v_code_offset(t, lane)];
-      const uint32_t smv = *reinterpret_cast<const uint32_t*>(blockp + kVsmOff + 4 * t);
+      const uint32_t smv = *reinterpret_cast<const uint32_t*>(blockp + sm_offset(a.ng, 1, t, lane * a.ng / 32));
       const float s = __half2float(__ushort_as_half((unsigned short)(smv & 0xffff)));
       const float m = __half2float(__ushort_as_half((unsigned short)(smv >> 16)));
 #pragma unroll
@@ -407,7 +410,7 @@ __global__ void __launch_bounds__(kDecWarps * 32) decode_simt_kernel(DecodeArgs 
             if (lane == 0) raise_flag(a.status, OKV_DEV_BAD_BLOCK);
             continue;
           }
-          const uint8_t* bp = a.pages + ((size_t)blk * a.hkv + hk) * kBlockHeadBytes;
+          const uint8_t* bp = a.pages + ((size_t)blk * a.hkv + hk) * block_head_bytes(a.ng);
           const int ntok = min(kBlock, us.n_int2 - pi * kBlock);
           simt_chunk<G, false>(a, qs, bp, nullptr, nullptr, 0, ntok, st, lane);
         }
@@ -497,9 +500,10 @@ __global__ void __launch_bounds__(kDecWarps * 32) decode_simt_kernel(DecodeArgs 
 // fp16 hi+lo pairs), folded into the warp's state in registers.
 // ---------------------------------------------------------------------------
 constexpr int kHW = 8;                             // warps per CTA
-constexpr int kHStages = 6;                        // ring stages
+constexpr int kHStages = 6;                        // ring stages with two CTAs per SM (G <= 4)
+constexpr int kHStagesSolo = 10;                   // ring stages with one CTA per SM (G = 8)
 constexpr int kIssueBatch = 2;                     // stages the producer issues at a time
-static_assert(kHStages % kIssueBatch == 0 && (kIssueBatch == 1 || kIssueBatch == 2),
+static_assert(kHStages % kIssueBatch == 0 && kHStagesSolo % kIssueBatch == 0 && (kIssueBatch == 1 || kIssueBatch == 2),
               "a batch of up to 16-block stages must start at a multiple of its size and fit one 32-block window");
 constexpr int kSlotsPerStage = 16;                 // block-heads per stage
 constexpr int kHStageBytes = kSlotsPerStage * kBlockHeadBytes;  // 18432
@@ -524,15 +528,18 @@ template <int G>
 struct HCfg {
   static constexpr int NT = G <= 4 ? 1 : G / 4;  // n-tiles of 8 columns = 4 heads x 2 limbs
   static constexpr int HP = 4 * NT;              // heads incl. padding
-  static constexpr size_t ring_bytes = (size_t)kHStages * kHStageBytes;
+  // one CTA per SM for G = 8 (its registers): that CTA gets a deeper ring,
+  // so the bytes in flight per SM stay close to two CTAs' worth
+  static constexpr int NS = G <= 4 ? kHStages : kHStagesSolo;
+  static constexpr size_t ring_bytes = (size_t)NS * kHStageBytes;
   // fp32 o' accumulators live in tensor memory: thread (warp w, lane l) owns
   // TMEM lane 32 (w % 4) + l, columns 16 NT (w / 4) .. +16 NT
   static constexpr uint32_t tmem_cols = 32u * NT;
   static constexpr size_t smem_bytes() {
     return ring_bytes                            // ring (reused for window scratch and merging)
-           + (size_t)2 * kHStages * 8            // full / empty mbarriers
+           + (size_t)2 * NS * 8                  // full / empty mbarriers
            + 16                                  // TMEM base address
-           + (size_t)kHStages * kSlotsPerStage   // tokens per block slot
+           + (size_t)NS * kSlotsPerStage         // tokens per block slot
            + (size_t)kHW * HP * kPStride * 2     // P' tiles
            + (size_t)kHW * G * 2 * 4;            // merge (m, l)
   }
@@ -645,6 +652,7 @@ __device__ __forceinline__ void mma_flush(MmaWarpState<G>& st, int (&acci)[HCfg<
 template <int G>
 __global__ void __launch_bounds__(kHW * 32, (G <= 4) ? 2 : 1) decode_heads_kernel(DecodeArgs a) {
   constexpr int NT = HCfg<G>::NT, HP = HCfg<G>::HP;
+  constexpr int kHStages = HCfg<G>::NS;  // ring stages of this instantiation
   extern __shared__ __align__(16) unsigned char smem_raw[];
   __shared__ int btq[2][32];  // producer's block ids, two 32-block windows
   unsigned char* ring = smem_raw;
@@ -1596,12 +1604,12 @@ static okv_status launch_decode_heads(const DecodeArgs& a, cudaStream_t s, bool 
   return check_launch("decode");
 }
 
-bool decode_uses_tensor_cores(int g, int hkv) {
-  return (g == 1 || g == 2 || g == 4 || g == 8) && (hkv == 1 || hkv == 2 || hkv == 4 || hkv == 8);
+bool decode_uses_tensor_cores(int g, int hkv, int ng) {
+  return ng == 1 && (g == 1 || g == 2 || g == 4 || g == 8) && (hkv == 1 || hkv == 2 || hkv == 4 || hkv == 8);
 }
 
-int decode_ctas_per_sm(int g, int hkv) {
-  if (decode_uses_tensor_cores(g, hkv)) return g <= 4 ? 2 : 1;
+int decode_ctas_per_sm(int g, int hkv, int ng) {
+  if (decode_uses_tensor_cores(g, hkv, ng)) return g <= 4 ? 2 : 1;
   return 4;
 }
 
@@ -1636,6 +1644,7 @@ static DecodeArgs make_decode_args(const okv_cache_desc* d, const void* q, int B
   a.num_blocks = d->num_blocks;
   a.num_slots = d->num_seq_slots;
   a.mbps = d->max_blocks_per_seq;
+  a.ng = kD / d->group;
   return a;
 }
 
@@ -1659,7 +1668,7 @@ static okv_status launch_decode_tail(const DecodeArgs& a, int B, cudaStream_t s)
   // predecessor; they are left out when the split-K kernel is being timed, so
   // that the events bracket it alone.
   const bool early = ev0 == nullptr;
-  const bool tc = decode_uses_tensor_cores(a.g, a.hkv);
+  const bool tc = decode_uses_tensor_cores(a.g, a.hkv, a.ng);
   if (tc) {
     switch (a.g) {
       case 1: st = launch_decode_heads<1>(a, s, early); break;

@@ -20,6 +20,7 @@ struct DequantArgs {
   float* out;
   uint32_t* status;
   int hkv, num_blocks, num_slots, mbps, max_ctx, which, basis, source, nsink;
+  int ng;  // quantisation groups per vector
 };
 
 // grid (ceil(max_ctx/32), Hkv, B), 128 threads; warp w handles tokens w, w+4, ...
@@ -61,10 +62,12 @@ __global__ void __launch_bounds__(128) dequant_kernel(DequantArgs a) {
       } else {
         const int blk = a.block_table[(size_t)slot * a.mbps + (p >> 4)];
         if (blk >= 0 && blk < a.num_blocks) {
-          const uint8_t* bp = a.pages + ((size_t)blk * a.hkv + hk) * kBlockHeadBytes;
+          const uint8_t* bp = a.pages + ((size_t)blk * a.hkv + hk) * block_head_bytes(a.ng);
           const int t = p & 15;
           const uint32_t byte = a.which == 0 ? bp[kKcOff + t * 32 + lane] : bp[v_code_offset(t, lane)];
-          const uint32_t sm = *reinterpret_cast<const uint32_t*>(bp + (a.which ? kVsmOff : kKsmOff) + 4 * t);
+          // channels 4 lane .. 4 lane + 3 lie in group 4 lane / group = lane ng / 32
+          const uint32_t sm =
+              *reinterpret_cast<const uint32_t*>(bp + sm_offset(a.ng, a.which, t, lane * a.ng / 32));
           const float s = __half2float(__ushort_as_half((unsigned short)(sm & 0xffff)));
           const float m = __half2float(__ushort_as_half((unsigned short)(sm >> 16)));
 #pragma unroll
@@ -119,6 +122,7 @@ okv_status launch_dequant(const okv_cache_desc* d, int B, const int32_t* seq_slo
   a.num_blocks = d->num_blocks;
   a.num_slots = d->num_seq_slots;
   a.mbps = d->max_blocks_per_seq;
+  a.ng = kD / d->group;
   a.max_ctx = max_ctx;
   a.which = which;
   a.basis = basis;

@@ -61,7 +61,7 @@ extern "C" okv_status okv_decode_attention_noalloc(const okv_cache_desc* desc, c
     return fail(OKV_ERR_UNSUPPORTED, "Hq/Hkv = %d not in {1,2,4,8,16}", g);
   if ((long long)B * desc->num_kv_heads * ((long long)desc->max_blocks_per_seq + kWinCost) >= 0x7fffffffLL)
     return fail(OKV_ERR_INVALID_ARG, "B * Hkv * max_blocks_per_seq too large");
-  const DecodePlan plan = make_decode_plan(B, desc->num_q_heads, desc->num_kv_heads);
+  const DecodePlan plan = make_decode_plan(B, desc->num_q_heads, desc->num_kv_heads, kD / desc->group);
   if (plan.total > (size_t)OKV_NOALLOC_SCRATCH_BYTES)
     return fail(OKV_ERR_INVALID_ARG,
                 "batch too large for the built-in scratch: needs %zu bytes, the static array holds %zu "

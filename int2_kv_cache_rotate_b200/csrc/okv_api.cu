@@ -63,9 +63,10 @@ static bool aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
 
 okv_status validate_desc(const okv_cache_desc* d) {
   if (d == nullptr) return fail(OKV_ERR_INVALID_ARG, "desc is NULL");
-  if (d->head_dim != kD || d->group != kD || d->block_tokens != kBlock || d->window != kWin)
-    return fail(OKV_ERR_UNSUPPORTED, "only head_dim=128, group=128, block_tokens=16, window=128 are built "
-                "(got %d, %d, %d, %d)", d->head_dim, d->group, d->block_tokens, d->window);
+  if (d->head_dim != kD || d->block_tokens != kBlock || d->window != kWin ||
+      (d->group != 32 && d->group != 64 && d->group != 128))
+    return fail(OKV_ERR_UNSUPPORTED, "only head_dim=128, group in {32, 64, 128}, block_tokens=16, window=128 "
+                "are built (got %d, %d, %d, %d)", d->head_dim, d->group, d->block_tokens, d->window);
   if (d->num_kv_heads < 1 || d->num_q_heads < 1 || d->num_q_heads % d->num_kv_heads != 0)
     return fail(OKV_ERR_INVALID_ARG, "num_q_heads (%d) must be a positive multiple of num_kv_heads (%d)",
                 d->num_q_heads, d->num_kv_heads);
@@ -90,14 +91,14 @@ okv_status validate_desc(const okv_cache_desc* d) {
 
 static size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-DecodePlan make_decode_plan(int batch, int hq, int hkv) {
+DecodePlan make_decode_plan(int batch, int hq, int hkv, int ng) {
   DecodePlan p;
   p.batch = batch;
   p.hq = hq;
   p.hkv = hkv;
   p.g = hq / hkv;
   const int sms = device_sm_count();
-  p.num_ctas = (sms > 0 ? sms : 148) * decode_ctas_per_sm(p.g, hkv);
+  p.num_ctas = (sms > 0 ? sms : 148) * decode_ctas_per_sm(p.g, hkv, ng);
   if (p.num_ctas > 1024) p.num_ctas = 1024;  // the combine caches one weight per split
   p.num_units = batch * hkv;
   size_t off = 0;
@@ -123,7 +124,7 @@ using namespace okv;
 
 extern "C" {
 
-int32_t okv_version(void) { return 1; }
+int32_t okv_version(void) { return 2; }
 
 okv_status okv_time_next_decode_kernel(void* start_event, void* stop_event) {
   if ((start_event == nullptr) != (stop_event == nullptr))
@@ -147,9 +148,14 @@ const char* okv_status_string(okv_status s) {
   return "unknown okv_status";
 }
 
-size_t okv_pages_bytes(int32_t num_blocks, int32_t num_kv_heads) {
+size_t okv_block_head_bytes(int32_t group) {
+  if (group != 32 && group != 64 && group != 128) return 0;
+  return (size_t)block_head_bytes(kD / group);
+}
+
+size_t okv_pages_bytes(int32_t num_blocks, int32_t num_kv_heads, int32_t group) {
   if (num_blocks < 0 || num_kv_heads < 0) return 0;
-  return (size_t)num_blocks * (size_t)num_kv_heads * kBlockHeadBytes;
+  return (size_t)num_blocks * (size_t)num_kv_heads * okv_block_head_bytes(group);
 }
 
 size_t okv_window_bytes(int32_t num_seq_slots, int32_t num_kv_heads) {
@@ -183,9 +189,37 @@ okv_status okv_append_quantize(const okv_cache_desc* desc, const void* k, const 
                        (cudaStream_t)stream);
 }
 
+size_t okv_prefill_workspace_bytes(const okv_cache_desc* desc, int32_t T) {
+  if (validate_desc(desc) != OKV_OK || T < 0) return 0;
+  return prefill_workspace_bytes(T, desc->num_q_heads);
+}
+
+okv_status okv_prefill_attention(const okv_cache_desc* desc, const void* q, int32_t T, int32_t slot,
+                                 int32_t context_len, const int32_t* block_table, float* out, void* workspace,
+                                 size_t workspace_bytes, void* stream) {
+  okv_status st = validate_desc(desc);
+  if (st != OKV_OK) return st;
+  if (T < 0) return fail(OKV_ERR_INVALID_ARG, "T must be >= 0");
+  if (T == 0) return OKV_OK;
+  if (!q || !block_table || !out || !workspace)
+    return fail(OKV_ERR_INVALID_ARG, "q, block_table, out and workspace must be non-NULL");
+  if (slot < 0 || slot >= desc->num_seq_slots)
+    return fail(OKV_ERR_INVALID_ARG, "slot %d outside [0, %d)", slot, desc->num_seq_slots);
+  if (context_len < T || (long long)context_len > (long long)desc->max_blocks_per_seq * kBlock)
+    return fail(OKV_ERR_INVALID_ARG, "context_len %d must be in [T = %d, %lld]", context_len, T,
+                (long long)desc->max_blocks_per_seq * kBlock);
+  if ((long long)T * desc->num_q_heads > 0x7fffffffLL) return fail(OKV_ERR_INVALID_ARG, "T * Hq too large");
+  if ((uintptr_t)q % 2 || (uintptr_t)out % 4 || (uintptr_t)workspace % 256)
+    return fail(OKV_ERR_INVALID_ARG, "q must be 2-byte, out 4-byte and workspace 256-byte aligned");
+  const size_t need = prefill_workspace_bytes(T, desc->num_q_heads);
+  if (workspace_bytes < need)
+    return fail(OKV_ERR_INVALID_ARG, "workspace too small: %zu < %zu bytes", workspace_bytes, need);
+  return launch_prefill(desc, q, T, slot, context_len, block_table, out, workspace, (cudaStream_t)stream);
+}
+
 size_t okv_decode_workspace_bytes(const okv_cache_desc* desc, int32_t B) {
   if (validate_desc(desc) != OKV_OK || B < 0) return 0;
-  return make_decode_plan(B, desc->num_q_heads, desc->num_kv_heads).total;
+  return make_decode_plan(B, desc->num_q_heads, desc->num_kv_heads, kD / desc->group).total;
 }
 
 okv_status okv_decode_attention(const okv_cache_desc* desc, const void* q, int32_t B,
@@ -204,7 +238,7 @@ okv_status okv_decode_attention(const okv_cache_desc* desc, const void* q, int32
   if ((long long)B * desc->num_kv_heads * ((long long)desc->max_blocks_per_seq + kWinCost) >= 0x7fffffffLL)
     return fail(OKV_ERR_INVALID_ARG, "B * Hkv * max_blocks_per_seq too large");
   if ((uintptr_t)workspace % 256) return fail(OKV_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
-  const DecodePlan plan = make_decode_plan(B, desc->num_q_heads, desc->num_kv_heads);
+  const DecodePlan plan = make_decode_plan(B, desc->num_q_heads, desc->num_kv_heads, kD / desc->group);
   if (workspace_bytes < plan.total)
     return fail(OKV_ERR_INVALID_ARG, "workspace too small: %zu < %zu bytes", workspace_bytes, plan.total);
   return launch_decode(desc, q, B, seq_slot, block_table, context_lens, out, workspace, plan,
@@ -235,7 +269,7 @@ okv_status okv_decode_step(const okv_cache_desc* desc, const void* k, const void
   if ((long long)B * desc->num_kv_heads * ((long long)desc->max_blocks_per_seq + kWinCost) >= 0x7fffffffLL)
     return fail(OKV_ERR_INVALID_ARG, "B * Hkv * max_blocks_per_seq too large");
   if ((uintptr_t)workspace % 256) return fail(OKV_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
-  const DecodePlan plan = make_decode_plan(B, desc->num_q_heads, desc->num_kv_heads);
+  const DecodePlan plan = make_decode_plan(B, desc->num_q_heads, desc->num_kv_heads, kD / desc->group);
   if (workspace_bytes < plan.total)
     return fail(OKV_ERR_INVALID_ARG, "workspace too small: %zu < %zu bytes", workspace_bytes, plan.total);
   const cudaStream_t s = (cudaStream_t)stream;

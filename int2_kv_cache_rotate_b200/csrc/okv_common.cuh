@@ -10,14 +10,23 @@
 
 namespace okv {
 
-constexpr int kD = 128;           // head dimension = quantisation group
+constexpr int kD = 128;           // head dimension
 constexpr int kBlock = 16;        // tokens per block
 constexpr int kWin = 128;         // fp16 window length
-constexpr int kBlockHeadBytes = 1152;
+constexpr int kBlockHeadBytes = 1152;  // one block-head with 128-channel groups
 constexpr int kKcOff = 0;         // K codes, token-major 16 x 32 B
 constexpr int kVcOff = 512;       // V codes, 4-token-interleaved chunks
-constexpr int kKsmOff = 1024;     // K (fp16 scale, fp16 min) per token
-constexpr int kVsmOff = 1088;     // V (fp16 scale, fp16 min) per token
+constexpr int kKsmOff = 1024;     // K (fp16 scale, fp16 min) per token (128-channel groups)
+constexpr int kVsmOff = 1088;     // V (fp16 scale, fp16 min) per token (128-channel groups)
+
+// Layout with ng = 128 / group quantisation groups per token-head (1, 2 or
+// 4): the codes as above, then K (scale, min) pairs at 1024 + 4 (t ng + k)
+// for token t, group k (channels k group .. (k + 1) group - 1), then V pairs
+// at 1024 + 64 ng + 4 (t ng + k).  ng = 1 is the layout above.
+__host__ __device__ __forceinline__ int block_head_bytes(int ng) { return 1024 + 128 * ng; }
+__host__ __device__ __forceinline__ int sm_offset(int ng, int kind, int t, int k) {
+  return 1024 + 64 * ng * kind + 4 * (t * ng + k);
+}
 constexpr float kInvSqrtD = 0.088388347648318440550f;  // 1/sqrt(128)
 constexpr float kLog2e = 1.4426950408889634074f;
 
@@ -114,18 +123,25 @@ __device__ __forceinline__ uint32_t int2_code(float x, const CodeThresholds& t) 
 
 // INT2 group quantiser over the 128 values of a warp (y[a] = value at
 // pre-permutation index l + 32a, i.e. rotated channel 4*rev5(l) + rev2(a)).
-// All steps are IEEE fp32 round-to-nearest; returns this lane's packed code
-// byte (canonical byte rev5(l)) and the fp16 scale/min bits.
+// With ng groups per vector (ng = 128 / group: 1, 2 or 4), the group of
+// lane l's four channels is rev5(l) * ng / 32: the lanes that share
+// l mod ng form one group, so the min/max reductions stop at lane distance
+// ng.  All steps are IEEE fp32 round-to-nearest; returns this lane's packed
+// code byte (canonical byte rev5(l)) and its group's fp16 scale/min bits.
 struct Quantized {
   uint32_t byte;
   uint32_t sm;  // fp16 scale in bits 0-15, fp16 min in bits 16-31
 };
 
-__device__ __forceinline__ Quantized quantize_warp(const float y[4]) {
+__device__ __forceinline__ Quantized quantize_warp(const float y[4], int ng = 1) {
   float mn = fminf(fminf(y[0], y[1]), fminf(y[2], y[3]));
   float mx = fmaxf(fmaxf(y[0], y[1]), fmaxf(y[2], y[3]));
-  mn = warp_min(mn);
-  mx = warp_max(mx);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    if (o < ng) break;
+    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  }
   const float s32 = __fdiv_rn(__fsub_rn(mx, mn), 3.0f);
   const __half s16 = fp16_sat(s32);
   const __half m16 = fp16_sat(mn);

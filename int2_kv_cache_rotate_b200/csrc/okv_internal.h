@@ -42,10 +42,10 @@ constexpr int kPartStride = 132;  // o'[128], m, l, 2 spare
 constexpr int kWinCost = 8;       // cost of an entry's window in block units (all heads)
 constexpr int kFusedAppendMaxTokens = 127;  // okv_decode_step fuses appends this short with the query rotation
 // split-K kernel choice and residency (decode.cu)
-bool decode_uses_tensor_cores(int g, int hkv);
-int decode_ctas_per_sm(int g, int hkv);
+bool decode_uses_tensor_cores(int g, int hkv, int ng);
+int decode_ctas_per_sm(int g, int hkv, int ng);
 
-DecodePlan make_decode_plan(int batch, int hq, int hkv);
+DecodePlan make_decode_plan(int batch, int hq, int hkv, int ng);
 
 // launchers (return cudaGetLastError-mapped status)
 okv_status launch_append(const okv_cache_desc* d, const void* k, const void* v, int T,
@@ -59,6 +59,9 @@ okv_status launch_decode_step(const okv_cache_desc* d, const void* k, const void
                               const int32_t* new_pos, const int32_t* slot_lens, const void* q, int B,
                               const int32_t* seq_slot, const int32_t* block_table, const int32_t* context_lens,
                               float* out, void* ws, const DecodePlan& plan, cudaStream_t s);
+okv_status launch_prefill(const okv_cache_desc* d, const void* q, int T, int slot, int context_len,
+                          const int32_t* block_table, float* out, void* ws, cudaStream_t s);
+size_t prefill_workspace_bytes(int T, int hq);
 okv_status launch_dequant(const okv_cache_desc* d, int B, const int32_t* seq_slot,
                           const int32_t* block_table, const int32_t* context_lens, int max_ctx,
                           int which, int basis, int source, float* out, cudaStream_t s);

@@ -1,0 +1,513 @@
+// Chunked-prefill attention over the INT2 paged cache: the T queries of a
+// prefill chunk (already appended, positions L - T .. L - 1 of a sequence of
+// L tokens) attend causally to the sequence's cache as it is held at length
+// L -- sink rows and the last W positions from fp16, the rest from INT2.
+//
+// Three launches:
+//   1. query rotation: q~ = q R_K, split into fp16 hi + lo halves of
+//      q~ 2^-e (e per row so that the halves stay in fp16 range) and the
+//      per-group sums of q~;
+//   2. attention (this file's main kernel): a CTA of 4 warps takes 64 query
+//      rows (query token x query head of one KV head) and streams the key
+//      positions 0 .. its last row's position in 16-token chunks.  Every
+//      chunk is staged in shared memory as fp16: the 2-bit codes (0..3 are
+//      exact in fp16) of INT2 positions with their per-group scale s and
+//      minimum m, or the fp16 values of window and sink rows with s = 1 and
+//      m = 0.  Then, per group k of channels,
+//        score = s_k (q~_k . c_k) + m_k sum(q~_k)
+//      with q~ . c on mma.m16n8k16 (f16 in, f32 accumulate; q~ as hi + lo,
+//      so the products carry about 22 bits), an online softmax per row, and
+//        o' += sum_t (p_t s_{t,k}) c_t + sum_t p_t m_{t,k}
+//      with p s as hi + lo fp16 A operands in the registers the score MMA
+//      left them in (its D fragment is the next MMA's A fragment) and the
+//      codes as the B operand.  The dense contraction runs on the tensor
+//      cores; nothing is dequantised to a rounded value.
+//   3. normalise and un-rotate: o = (o' / l) R_V^T per row.
+#include "okv_common.cuh"
+#include "okv_internal.h"
+
+namespace okv {
+namespace {
+
+constexpr int kPfWarps = 4;
+constexpr int kPfRows = 16 * kPfWarps;  // query rows per CTA
+constexpr int kKStride = kD + 8;        // fp16 per staged key row (bank-conflict-free fragment loads)
+constexpr int kVStride = 16 + 8;        // fp16 per staged value column (values are staged transposed)
+
+struct PrefillArgs {
+  const __nv_bfloat16* q;  // [T][Hq][128]
+  const int32_t* block_table;
+  const uint8_t* pages;
+  const __half* ring;
+  const __half* sink;
+  const float* u_k;
+  const float* u_v;
+  uint32_t* status;
+  __half* qhi;   // [T][Hq][128]: hi half of q~ 2^-e
+  __half* qlo;   // [T][Hq][128]: lo half
+  float* qaux;   // [T][Hq][8]: sum of q~ per group (4), 2^e, spare
+  float* obuf;   // [T][Hq][132]: o' (128), l, spare
+  float* out;    // [T][Hq][128]
+  int T, hq, hkv, g, ng, bhb, slot, L, first, mbps, num_blocks, nsink;
+};
+
+constexpr int kQaux = 8;
+constexpr int kOStride = 132;
+
+// ---------------------------------------------------------------------------
+// 1. q~ = q R_K for the chunk.  One CTA per (query token, query head); warp w
+// holds rows 16w..16w+15 of U_K in registers, the partial sums meet in shared
+// memory and warp 0 runs the butterfly and the bit-reversal remap.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) prefill_qrot_kernel(PrefillArgs a) {
+  __shared__ float red[8][kD];
+  const int row = blockIdx.x;  // token * hq + head
+  const int head = row % a.hq;
+  const int hk = head / a.g;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const float* U = a.u_k + (size_t)hk * kD * kD;
+  const float xv = __bfloat162float(a.q[(size_t)row * kD + 16 * warp + (lane & 15)]);
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+  for (int r = 0; r < 16; ++r) {
+    const float4 u = __ldg(reinterpret_cast<const float4*>(U + (size_t)(16 * warp + r) * kD) + lane);
+    const float x = __shfl_sync(0xffffffffu, xv, r);
+    acc.x = fmaf(x, u.x, acc.x);
+    acc.y = fmaf(x, u.y, acc.y);
+    acc.z = fmaf(x, u.z, acc.z);
+    acc.w = fmaf(x, u.w, acc.w);
+  }
+  *reinterpret_cast<float4*>(&red[warp][4 * lane]) = acc;
+  __syncthreads();
+  if (warp != 0) return;
+  float y[4];
+#pragma unroll
+  for (int aa = 0; aa < 4; ++aa) {
+    float s = 0.f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) s += red[w][lane + 32 * aa];
+    y[aa] = s;
+  }
+  wht128_warp(y, lane);
+#pragma unroll
+  for (int aa = 0; aa < 4; ++aa) y[aa] *= kInvSqrtD;
+  // lane l holds rotated channels 4 r + {0, 2, 1, 3} (r = rev5(l)) in y[0..3]
+  const int r = rev5(lane);
+  const float zc[4] = {y[0], y[2], y[1], y[3]};
+  float amax = fmaxf(fmaxf(fabsf(y[0]), fabsf(y[1])), fmaxf(fabsf(y[2]), fabsf(y[3])));
+  amax = warp_max(amax);
+  // 2^-e with amax 2^-e in [1, 2): the hi half keeps 11 bits, the lo half the next 11
+  int e = 0;
+  if (amax > 0.f) e = ((__float_as_int(amax) >> 23) & 0xff) - 127;
+  e = max(-100, min(100, e));
+  const float down = __int_as_float((127 - e) << 23);
+  __half* hi = a.qhi + (size_t)row * kD + 4 * r;
+  __half* lo = a.qlo + (size_t)row * kD + 4 * r;
+#pragma unroll
+  for (int f = 0; f < 4; ++f) {
+    const float x = zc[f] * down;
+    const __half h = __float2half_rn(x);
+    hi[f] = h;
+    lo[f] = __float2half_rn(x - __half2float(h));
+  }
+  // per-group sums of q~: channels 4r.. lie in group r ng / 32
+  float part = (zc[0] + zc[1]) + (zc[2] + zc[3]);
+  float gs[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) gs[k] = warp_sum((k < a.ng && r * a.ng / 32 == k) ? part : 0.f);
+  if (lane == 0) {
+    float* aux = a.qaux + (size_t)row * kQaux;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) aux[k] = gs[k];
+    aux[4] = __int_as_float((127 + e) << 23);
+  }
+}
+
+__device__ __forceinline__ void mma_f16_pf(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};\n"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t pack_half2(float lo_elem, float hi_elem) {
+  const __half2 h = __floats2half2_rn(lo_elem, hi_elem);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+// hi and lo fp16 halves of a pair of floats, packed as MMA operand registers
+__device__ __forceinline__ void split_half2(float x0, float x1, uint32_t& hi, uint32_t& lo) {
+  const __half2 h = __floats2half2_rn(x0, x1);
+  const float2 f = __half22float2(h);
+  hi = *reinterpret_cast<const uint32_t*>(&h);
+  lo = pack_half2(x0 - f.x, x1 - f.y);
+}
+
+// ---------------------------------------------------------------------------
+// 2. attention.  Grid (ceil(rows / 64), Hkv); rows are (token, query head)
+// pairs of the KV head, token-major: row r = token (r / G), head (r % G).
+// Warp w owns rows 16w .. 16w + 15 of the CTA.  Fragment facts
+// (m16n8k16, f16): lane (g = lane / 4, t = lane % 4) holds A (row g, cols
+// 2t, 2t+1), (g + 8, 2t..), (g, 2t + 8..), (g + 8, 2t + 8..); B (rows 2t,
+// 2t + 1, col g), (2t + 8, 2t + 9, col g); D (row g, cols 2t, 2t + 1),
+// (g + 8, 2t, 2t + 1).
+// ---------------------------------------------------------------------------
+template <int NG>
+__global__ void __launch_bounds__(kPfWarps * 32) prefill_attn_kernel(PrefillArgs a) {
+  constexpr int KSG = 8 / NG;  // 16-channel k-steps per group
+  __shared__ __align__(16) __half kc[16 * kKStride];  // [token][channel]: codes or fp16 values
+  __shared__ __align__(16) __half vc[kD * kVStride];  // [channel][token]
+  __shared__ float ksm[16][NG][2], vsm[16][NG][2];    // (scale, min) per token and group
+  __shared__ int tpos_ok[16];                          // 1 if the chunk's token is a readable position
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int g = lane >> 2, t = lane & 3;
+  const int hk = blockIdx.y;
+  const int nrows = a.T * a.g;
+  const int row0 = blockIdx.x * kPfRows;
+  // this lane's two rows (g and g + 8 of the warp's 16)
+  int rtok[2], rrow[2];
+  bool rok[2];
+#pragma unroll
+  for (int h2 = 0; h2 < 2; ++h2) {
+    const int r = row0 + 16 * warp + g + 8 * h2;
+    rok[h2] = r < nrows;
+    const int rr = rok[h2] ? r : nrows - 1;
+    rtok[h2] = rr / a.g;
+    rrow[h2] = rtok[h2] * a.hq + hk * a.g + rr % a.g;  // global (token, query head) row
+  }
+  // query fragments: A operands of the score MMA, hi and lo halves
+  uint32_t qa_hi[8][4], qa_lo[8][4];
+  {
+    const __half* h0 = a.qhi + (size_t)rrow[0] * kD;
+    const __half* h1 = a.qhi + (size_t)rrow[1] * kD;
+    const __half* l0 = a.qlo + (size_t)rrow[0] * kD;
+    const __half* l1 = a.qlo + (size_t)rrow[1] * kD;
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks) {
+      const int c = 16 * ks + 2 * t;
+      qa_hi[ks][0] = *reinterpret_cast<const uint32_t*>(h0 + c);
+      qa_hi[ks][1] = *reinterpret_cast<const uint32_t*>(h1 + c);
+      qa_hi[ks][2] = *reinterpret_cast<const uint32_t*>(h0 + c + 8);
+      qa_hi[ks][3] = *reinterpret_cast<const uint32_t*>(h1 + c + 8);
+      qa_lo[ks][0] = *reinterpret_cast<const uint32_t*>(l0 + c);
+      qa_lo[ks][1] = *reinterpret_cast<const uint32_t*>(l1 + c);
+      qa_lo[ks][2] = *reinterpret_cast<const uint32_t*>(l0 + c + 8);
+      qa_lo[ks][3] = *reinterpret_cast<const uint32_t*>(l1 + c + 8);
+    }
+  }
+  float qsum[2][NG], qup[2];
+  int rpos[2];
+#pragma unroll
+  for (int h2 = 0; h2 < 2; ++h2) {
+    const float* aux = a.qaux + (size_t)rrow[h2] * kQaux;
+#pragma unroll
+    for (int k = 0; k < NG; ++k) qsum[h2][k] = aux[k] * (kInvSqrtD * kLog2e);
+    qup[h2] = aux[4] * (kInvSqrtD * kLog2e);  // undoes the 2^-e of the halves, in log2 units
+    rpos[h2] = a.first + rtok[h2];
+  }
+  float o[16][4];
+#pragma unroll
+  for (int n = 0; n < 16; ++n)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) o[n][j] = 0.f;
+  float mrow[2] = {-INFINITY, -INFINITY}, lrow[2] = {0.f, 0.f};
+  float msum[2][NG];
+#pragma unroll
+  for (int h2 = 0; h2 < 2; ++h2)
+#pragma unroll
+    for (int k = 0; k < NG; ++k) msum[h2][k] = 0.f;
+
+  const int last_row = min(nrows, row0 + kPfRows) - 1;
+  const int pmax = a.first + last_row / a.g;  // last position any row of this CTA sees
+  const int nchunks = pmax / 16 + 1;
+  const int tid = threadIdx.x;
+  for (int ch = 0; ch < nchunks; ++ch) {
+    __syncthreads();  // the previous chunk's tiles are no longer read
+    // ---- stage chunk ch: thread tid -> token tid / 8, channels 16 (tid % 8) .. + 15
+    {
+      const int tk = tid >> 3, part = tid & 7;
+      const int p = 16 * ch + tk;
+      int kind_src = 0;  // 0 masked, 1 INT2, 2 fp16 window, 3 fp16 sink
+      const uint8_t* bp = nullptr;
+      if (p <= pmax && p < a.L) {
+        if (p < a.nsink) {
+          kind_src = 3;
+        } else if (p >= a.L - kWin) {
+          kind_src = 2;
+        } else {
+          const int blk = a.block_table[(size_t)a.slot * a.mbps + (p >> 4)];
+          if (blk >= 0 && blk < a.num_blocks) {
+            kind_src = 1;
+            bp = a.pages + ((size_t)blk * a.hkv + hk) * a.bhb;
+          } else if (part == 0) {
+            raise_flag(a.status, OKV_DEV_BAD_BLOCK);
+          }
+        }
+      }
+      __half kv16[16], vv16[16];
+      if (kind_src == 1) {
+        const int sl = p & 15;
+        const uint32_t kw = *reinterpret_cast<const uint32_t*>(bp + kKcOff + sl * 32 + 4 * part);
+#pragma unroll
+        for (int j = 0; j < 16; ++j) kv16[j] = __int2half_rn((int)((kw >> (2 * j)) & 3u));
+#pragma unroll
+        for (int bq = 0; bq < 4; ++bq) {
+          const uint32_t vb = bp[v_code_offset(sl, 4 * part + bq)];
+#pragma unroll
+          for (int f = 0; f < 4; ++f) vv16[4 * bq + f] = __int2half_rn((int)((vb >> (2 * f)) & 3u));
+        }
+      } else if (kind_src >= 2) {
+        const size_t base = (((size_t)a.slot * a.hkv + hk) * 2) * (kind_src == 2 ? kWin : a.nsink);
+        const size_t rowk = kind_src == 2 ? (size_t)(p % kWin) : (size_t)p;
+        const size_t rows_per_kind = kind_src == 2 ? (size_t)kWin : (size_t)a.nsink;
+        const __half* srcb = kind_src == 2 ? a.ring : a.sink;
+        const uint4* kr = reinterpret_cast<const uint4*>(srcb + (base + rowk) * kD + 16 * part);
+        const uint4* vr = reinterpret_cast<const uint4*>(srcb + (base + rows_per_kind + rowk) * kD + 16 * part);
+        *reinterpret_cast<uint4*>(kv16) = kr[0];
+        *reinterpret_cast<uint4*>(kv16 + 8) = kr[1];
+        *reinterpret_cast<uint4*>(vv16) = vr[0];
+        *reinterpret_cast<uint4*>(vv16 + 8) = vr[1];
+      } else {
+#pragma unroll
+        for (int j = 0; j < 16; ++j) kv16[j] = vv16[j] = __float2half_rn(0.f);
+      }
+      *reinterpret_cast<uint4*>(kc + tk * kKStride + 16 * part) = *reinterpret_cast<const uint4*>(kv16);
+      *reinterpret_cast<uint4*>(kc + tk * kKStride + 16 * part + 8) = *reinterpret_cast<const uint4*>(kv16 + 8);
+#pragma unroll
+      for (int j = 0; j < 16; ++j) vc[(16 * part + j) * kVStride + tk] = vv16[j];
+      if (part < NG) {  // one thread per (token, group): the group's scale and minimum
+        float s_k = 1.f, m_k = 0.f, s_v = 1.f, m_v = 0.f;
+        if (kind_src == 1) {
+          const int sl = p & 15;
+          const uint32_t w0 = *reinterpret_cast<const uint32_t*>(bp + sm_offset(NG, 0, sl, part));
+          const uint32_t w1 = *reinterpret_cast<const uint32_t*>(bp + sm_offset(NG, 1, sl, part));
+          s_k = __half2float(__ushort_as_half((unsigned short)(w0 & 0xffff)));
+          m_k = __half2float(__ushort_as_half((unsigned short)(w0 >> 16)));
+          s_v = __half2float(__ushort_as_half((unsigned short)(w1 & 0xffff)));
+          m_v = __half2float(__ushort_as_half((unsigned short)(w1 >> 16)));
+        } else if (kind_src == 0) {
+          s_k = m_k = s_v = m_v = 0.f;
+        }
+        ksm[tk][part][0] = s_k;
+        ksm[tk][part][1] = m_k;
+        vsm[tk][part][0] = s_v;
+        vsm[tk][part][1] = m_v;
+      }
+      if (part == 0) tpos_ok[tk] = kind_src != 0;
+    }
+    __syncthreads();
+    // ---- scores of 16 rows x 16 tokens, per group
+    float d[NG][2][4];
+#pragma unroll
+    for (int k = 0; k < NG; ++k)
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) d[k][nt][j] = 0.f;
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks) {
+      const int k = ks / KSG;
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) {
+        const __half* kb = kc + (8 * nt + g) * kKStride + 16 * ks + 2 * t;
+        const uint32_t b0 = *reinterpret_cast<const uint32_t*>(kb);
+        const uint32_t b1 = *reinterpret_cast<const uint32_t*>(kb + 8);
+        mma_f16_pf(d[k][nt], qa_hi[ks], b0, b1);
+        mma_f16_pf(d[k][nt], qa_lo[ks], b0, b1);
+      }
+    }
+    // score (log2 units) of row h2, token 8 nt + 2 t + c: sum_k s_k raw_k 2^e + m_k sum_k
+    float sc[2][2][2];  // [h2][nt][c]
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        const int tk = 8 * nt + 2 * t + c;
+        const int p = 16 * ch + tk;
+        const bool ok = tpos_ok[tk] != 0;
+#pragma unroll
+        for (int h2 = 0; h2 < 2; ++h2) {
+          float x = 0.f;
+#pragma unroll
+          for (int k = 0; k < NG; ++k)
+            x = fmaf(ksm[tk][k][0] * qup[h2], d[k][nt][2 * h2 + c], fmaf(ksm[tk][k][1], qsum[h2][k], x));
+          sc[h2][nt][c] = (ok && rok[h2] && p <= rpos[h2]) ? x : -INFINITY;
+        }
+      }
+    // online softmax per row (the 4 lanes of a quad share a row)
+    float pr[2][2][2];
+#pragma unroll
+    for (int h2 = 0; h2 < 2; ++h2) {
+      float bm = fmaxf(fmaxf(sc[h2][0][0], sc[h2][0][1]), fmaxf(sc[h2][1][0], sc[h2][1][1]));
+      bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 1));
+      bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 2));
+      const float mnew = fmaxf(mrow[h2], bm);
+      const float mref = mnew == -INFINITY ? 0.f : mnew;
+      const float alpha = exp2f(mrow[h2] - mref);  // 0 while the row has seen nothing
+      mrow[h2] = mnew;
+      float ps = 0.f;
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          pr[h2][nt][c] = exp2f(sc[h2][nt][c] - mref);
+          ps += pr[h2][nt][c];
+        }
+      lrow[h2] = fmaf(lrow[h2], alpha, ps);
+#pragma unroll
+      for (int k = 0; k < NG; ++k) msum[h2][k] *= alpha;
+#pragma unroll
+      for (int n = 0; n < 16; ++n) {
+        o[n][2 * h2] *= alpha;
+        o[n][2 * h2 + 1] *= alpha;
+      }
+    }
+    // values: per group k, A = p s_k (hi + lo) over the 16 tokens, B = codes
+#pragma unroll
+    for (int k = 0; k < NG; ++k) {
+      uint32_t ah[4], al[4];
+      // A registers: (row g, tokens 2t, 2t+1), (g + 8, 2t..), (g, 2t + 8..), (g + 8, 2t + 8..)
+#pragma unroll
+      for (int q4 = 0; q4 < 4; ++q4) {
+        const int h2 = q4 & 1, nt = q4 >> 1;
+        const int t0 = 8 * nt + 2 * t;
+        split_half2(pr[h2][nt][0] * vsm[t0][k][0], pr[h2][nt][1] * vsm[t0 + 1][k][0], ah[q4], al[q4]);
+      }
+#pragma unroll
+      for (int h2 = 0; h2 < 2; ++h2)
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+          for (int c = 0; c < 2; ++c) msum[h2][k] = fmaf(pr[h2][nt][c], vsm[8 * nt + 2 * t + c][k][1], msum[h2][k]);
+#pragma unroll
+      for (int n = 0; n < 16; ++n) {
+        if (n * NG / 16 != k) continue;  // channels 8n .. 8n + 7 belong to group n ng / 16
+        const __half* vb = vc + (8 * n + g) * kVStride + 2 * t;
+        const uint32_t b0 = *reinterpret_cast<const uint32_t*>(vb);
+        const uint32_t b1 = *reinterpret_cast<const uint32_t*>(vb + 8);
+        mma_f16_pf(o[n], ah, b0, b1);
+        mma_f16_pf(o[n], al, b0, b1);
+      }
+    }
+  }
+  // ---- o' rows and sums to the buffer: the quad's lanes hold columns 2t, 2t + 1 of every n-tile
+#pragma unroll
+  for (int h2 = 0; h2 < 2; ++h2) {
+    float l = lrow[h2];
+    l += __shfl_xor_sync(0xffffffffu, l, 1);
+    l += __shfl_xor_sync(0xffffffffu, l, 2);
+    float ms[NG];
+#pragma unroll
+    for (int k = 0; k < NG; ++k) {
+      ms[k] = msum[h2][k];
+      ms[k] += __shfl_xor_sync(0xffffffffu, ms[k], 1);
+      ms[k] += __shfl_xor_sync(0xffffffffu, ms[k], 2);
+    }
+    if (!rok[h2]) continue;
+    float* dst = a.obuf + (size_t)rrow[h2] * kOStride;
+#pragma unroll
+    for (int n = 0; n < 16; ++n) {
+      const float add = ms[n * NG / 16];
+      *reinterpret_cast<float2*>(dst + 8 * n + 2 * t) = make_float2(o[n][2 * h2] + add, o[n][2 * h2 + 1] + add);
+    }
+    if (t == 0) dst[128] = l;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// 3. o = (o' / l) R_V^T: one warp per row (8 rows per CTA), U_V rows of the
+// row's KV head read through L1.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) prefill_unrotate_kernel(PrefillArgs a) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int row = blockIdx.x * 8 + warp;
+  if (row >= a.T * a.hq) return;
+  const int hk = (row % a.hq) / a.g;
+  const float* src = a.obuf + (size_t)row * kOStride;
+  const float l = src[128];
+  const float inv = l > 0.f ? 1.f / l : 0.f;
+  // lane l: pre-permutation channels l + 32 aa = rotated channels 4 rev5(l) + rev2(aa)
+  const int r = rev5(lane);
+  float y[4];
+#pragma unroll
+  for (int aa = 0; aa < 4; ++aa) y[aa] = src[4 * r + rev2(aa)] * inv;
+  wht128_warp(y, lane);
+  float x[4];
+#pragma unroll
+  for (int aa = 0; aa < 4; ++aa) x[aa] = y[aa] * kInvSqrtD;  // x_i for i = lane + 32 aa
+  // o_c = sum_i x_i U_V[c][i]: lane owns outputs c = lane + 32 j
+  const float* U = a.u_v + (size_t)hk * kD * kD;
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  for (int i = 0; i < kD; ++i) {
+    const float xi = __shfl_sync(0xffffffffu, x[i >> 5], i & 31);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) acc[j] = fmaf(xi, __ldg(U + (size_t)(lane + 32 * j) * kD + i), acc[j]);
+  }
+  float* dst = a.out + (size_t)row * kD;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) dst[lane + 32 * j] = acc[j];
+}
+
+}  // namespace
+
+size_t prefill_workspace_bytes(int T, int hq) {
+  const size_t rows = (size_t)T * hq;
+  size_t off = 0;
+  off += (rows * kD * sizeof(__half) + 255) / 256 * 256;  // qhi
+  off += (rows * kD * sizeof(__half) + 255) / 256 * 256;  // qlo
+  off += (rows * kQaux * sizeof(float) + 255) / 256 * 256;
+  off += (rows * kOStride * sizeof(float) + 255) / 256 * 256;
+  return off;
+}
+
+okv_status launch_prefill(const okv_cache_desc* d, const void* q, int T, int slot, int context_len,
+                          const int32_t* block_table, float* out, void* ws, cudaStream_t s) {
+  PrefillArgs a;
+  a.q = (const __nv_bfloat16*)q;
+  a.block_table = block_table;
+  a.pages = (const uint8_t*)d->pages;
+  a.ring = (const __half*)d->window_ring;
+  a.sink = (const __half*)d->sink_rows;
+  a.u_k = d->u_k;
+  a.u_v = d->u_v;
+  a.status = d->status_word;
+  const size_t rows = (size_t)T * d->num_q_heads;
+  uint8_t* w = (uint8_t*)ws;
+  size_t off = 0;
+  a.qhi = (__half*)(w + off);
+  off += (rows * kD * sizeof(__half) + 255) / 256 * 256;
+  a.qlo = (__half*)(w + off);
+  off += (rows * kD * sizeof(__half) + 255) / 256 * 256;
+  a.qaux = (float*)(w + off);
+  off += (rows * kQaux * sizeof(float) + 255) / 256 * 256;
+  a.obuf = (float*)(w + off);
+  a.out = out;
+  a.T = T;
+  a.hq = d->num_q_heads;
+  a.hkv = d->num_kv_heads;
+  a.g = a.hq / a.hkv;
+  a.ng = kD / d->group;
+  a.bhb = block_head_bytes(a.ng);
+  a.slot = slot;
+  a.L = context_len;
+  a.first = context_len - T;
+  a.mbps = d->max_blocks_per_seq;
+  a.num_blocks = d->num_blocks;
+  a.nsink = d->num_sink;
+  prefill_qrot_kernel<<<(unsigned)rows, 256, 0, s>>>(a);
+  okv_status st = check_launch("prefill query rotation");
+  if (st != OKV_OK) return st;
+  const dim3 grid((unsigned)((T * a.g + kPfRows - 1) / kPfRows), (unsigned)a.hkv);
+  switch (a.ng) {
+    case 1: prefill_attn_kernel<1><<<grid, kPfWarps * 32, 0, s>>>(a); break;
+    case 2: prefill_attn_kernel<2><<<grid, kPfWarps * 32, 0, s>>>(a); break;
+    default: prefill_attn_kernel<4><<<grid, kPfWarps * 32, 0, s>>>(a); break;
+  }
+  st = check_launch("prefill attention");
+  if (st != OKV_OK) return st;
+  prefill_unrotate_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, s>>>(a);
+  return check_launch("prefill un-rotation");
+}
+
+}  // namespace okv

@@ -61,7 +61,8 @@ _DESC = ctypes.POINTER(CacheDesc)
 
 _SIGNATURES = {
     "okv_calibrate_rotations": (_I32, [_P, _I64, _P, _P, _I64, _I32, _I32, _I32, _P, _P, _P, _P]),
-    "okv_pages_bytes": (_SZ, [_I32, _I32]),
+    "okv_pages_bytes": (_SZ, [_I32, _I32, _I32]),
+    "okv_block_head_bytes": (_SZ, [_I32]),
     "okv_window_bytes": (_SZ, [_I32, _I32]),
     "okv_sink_bytes": (_SZ, [_I32, _I32, _I32]),
     "okv_append_quantize": (_I32, [_DESC, _P, _P, _I32, _P, _P, _P, _P, _U32, _P, _P]),
@@ -73,6 +74,8 @@ _SIGNATURES = {
     "okv_version": (_I32, []),
     "okv_time_next_decode_kernel": (_I32, [_P, _P]),
     "okv_decode_attention_noalloc": (_I32, [_DESC, _P, _I32, _P, _P, _P, _P, _P]),
+    "okv_prefill_workspace_bytes": (_SZ, [_DESC, _I32]),
+    "okv_prefill_attention": (_I32, [_DESC, _P, _I32, _I32, _I32, _P, _P, _P, _SZ, _P]),
     "okv_decode_step": (_I32, [_DESC, _P, _P, _I32, _P, _P, _P, _P, _I32, _P, _P, _P, _P, _P, _SZ, _P]),
     "okv_save_rotations": (_I32, [ctypes.c_char_p, _I32, _I32, _I32, _P, _P, ctypes.c_char_p]),
     "okv_rotations_file_shape": (_I32, [ctypes.c_char_p, _P, _P, _P, _P]),
@@ -155,11 +158,12 @@ class Cache:
     receives pointers."""
 
     def __init__(self, hq: int, hkv: int, num_blocks: int, num_seq_slots: int, max_blocks_per_seq: int,
-                 u_k, u_v, device="cuda", num_sink: int = 0):
+                 u_k, u_v, device="cuda", num_sink: int = 0, group: int = HEAD_DIM):
         import torch
-        self.hq, self.hkv, self.num_sink = hq, hkv, num_sink
+        self.hq, self.hkv, self.num_sink, self.group = hq, hkv, num_sink, group
         self.num_blocks, self.num_seq_slots, self.max_blocks_per_seq = num_blocks, num_seq_slots, max_blocks_per_seq
-        nbytes = lib().okv_pages_bytes(num_blocks, hkv)
+        self.block_head_bytes = int(lib().okv_block_head_bytes(group))
+        nbytes = lib().okv_pages_bytes(num_blocks, hkv, group)
         self.pages = torch.zeros(max(nbytes, 16), dtype=torch.uint8, device=device)
         self.ring = torch.zeros((num_seq_slots, hkv, 2, WINDOW, HEAD_DIM), dtype=torch.float16, device=device)
         self.u_k = torch.as_tensor(np.asarray(u_k, dtype=np.float32)).to(device).contiguous()
@@ -168,7 +172,7 @@ class Cache:
         # first num_sink positions of every sequence, fp16 (sink tokens)
         self.sink = torch.zeros((num_seq_slots, hkv, 2, max(num_sink, 0), HEAD_DIM), dtype=torch.float16,
                                 device=device)
-        self.desc = CacheDesc(hq, hkv, HEAD_DIM, HEAD_DIM, BLOCK_TOKENS, WINDOW, num_blocks, num_seq_slots,
+        self.desc = CacheDesc(hq, hkv, HEAD_DIM, group, BLOCK_TOKENS, WINDOW, num_blocks, num_seq_slots,
                               max_blocks_per_seq, num_sink, self.pages.data_ptr(), self.ring.data_ptr(),
                               self.u_k.data_ptr(), self.u_v.data_ptr(), self.status.data_ptr(),
                               self.sink.data_ptr() if num_sink > 0 else None)
@@ -336,6 +340,27 @@ def decode_attention_noalloc(cache: Cache, q, seq_slot, block_table, context_len
     _need(out, torch.float32, "out")
     _check(lib().okv_decode_attention_noalloc(ctypes.byref(cache.desc), _ptr(q), batch, _ptr(seq_slot),
                                               _ptr(block_table), _ptr(context_lens), _ptr(out), _stream(stream)))
+    return out
+
+
+def prefill_workspace_bytes(cache: Cache, T: int) -> int:
+    return int(lib().okv_prefill_workspace_bytes(ctypes.byref(cache.desc), T))
+
+
+def prefill_attention(cache: Cache, q, slot: int, context_len: int, block_table, out=None, ws=None, stream=None):
+    """Causal attention of a prefill chunk (q: bf16 [T, Hq, 128], already appended at positions
+    context_len - T .. context_len - 1 of sequence `slot`) over the cache; returns fp32 [T, Hq, 128]."""
+    import torch
+    _need(q, torch.bfloat16, "q")
+    _need(block_table, torch.int32, "block_table")
+    T = q.shape[0]
+    if out is None:
+        out = torch.empty((T, cache.hq, HEAD_DIM), dtype=torch.float32, device=q.device)
+    _need(out, torch.float32, "out")
+    if ws is None:
+        ws = torch.empty(max(prefill_workspace_bytes(cache, T), 256), dtype=torch.uint8, device=q.device)
+    _check(lib().okv_prefill_attention(ctypes.byref(cache.desc), _ptr(q), T, int(slot), int(context_len),
+                                       _ptr(block_table), _ptr(out), _ptr(ws), ws.numel(), _stream(stream)))
     return out
 
 

@@ -47,6 +47,30 @@ def gather_codes(pages: np.ndarray, table: np.ndarray, slot: int, h: int, hkv: i
     return packed, s_bits.view(np.float16), m_bits.view(np.float16)
 
 
+def gather_codes_grouped(pages: np.ndarray, table: np.ndarray, slot: int, h: int, hkv: int, n: int, kind: int,
+                         group: int):
+    """Like gather_codes for a cache with `group`-channel quantisation groups:
+    packed code bytes [n, 32], fp16 scale and min [n, 128 / group]."""
+    ng = D // group
+    bhb = 1024 + 128 * ng
+    pos = np.arange(n)
+    blk = table[slot, pos // 16].astype(np.int64)
+    t = pos % 16
+    base = (blk * hkv + h) * bhb
+    b = np.arange(32)
+    if kind == 0:
+        off = base[:, None] + t[:, None] * 32 + b[None, :]
+    else:
+        off = base[:, None] + 512 + ((b[None, :] >> 2) * 4 + (t[:, None] >> 2)) * 16 + (b[None, :] & 3) * 4 \
+            + (t[:, None] & 3)
+    packed = pages[off]
+    k = np.arange(ng)
+    sm_off = base[:, None] + 1024 + 64 * ng * kind + 4 * (t[:, None] * ng + k[None, :])
+    s_bits = pages[sm_off].astype(np.uint16) | (pages[sm_off + 1].astype(np.uint16) << 8)
+    m_bits = pages[sm_off + 2].astype(np.uint16) | (pages[sm_off + 3].astype(np.uint16) << 8)
+    return packed, s_bits.view(np.float16), m_bits.view(np.float16)
+
+
 def special_vectors() -> np.ndarray:
     """Edge-case groups for the quantiser: constant, huge range, lattice,
     ties, subnormal scale, scale that rounds to zero, min that rounds up."""

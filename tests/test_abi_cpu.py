@@ -32,7 +32,10 @@ def test_status_strings_and_sizes():
     lib = okv.lib()
     assert lib.okv_status_string(0) == b"OKV_OK"
     assert lib.okv_status_string(2) == b"OKV_ERR_UNSUPPORTED"
-    assert lib.okv_pages_bytes(10, 8) == 10 * 8 * 1152
+    assert lib.okv_pages_bytes(10, 8, 128) == 10 * 8 * 1152
+    assert lib.okv_pages_bytes(10, 8, 64) == 10 * 8 * 1280
+    assert lib.okv_pages_bytes(10, 8, 32) == 10 * 8 * 1536
+    assert [lib.okv_block_head_bytes(g) for g in (128, 64, 32, 16, 0)] == [1152, 1280, 1536, 0, 0]
     assert lib.okv_window_bytes(3, 8) == 3 * 8 * 2 * 128 * 128 * 2
     assert lib.okv_sink_bytes(3, 8, 192) == 3 * 8 * 2 * 192 * 128 * 2
     assert lib.okv_status_string(5) == b"OKV_ERR_IO"
@@ -44,8 +47,9 @@ def test_validation_before_launch():
     # NULL descriptor
     assert lib.okv_append_quantize(None, fake, fake, 1, fake, fake, fake, fake, 0, None, None) == okv.ERR_INVALID_ARG
     # unsupported head dim / group / window
-    for field in ("head_dim", "group", "window", "block_tokens"):
-        d = _desc(**{field: 64})
+    for field, val in (("head_dim", 64), ("group", 16), ("group", 48), ("group", 256), ("window", 64),
+                       ("block_tokens", 64)):
+        d = _desc(**{field: val})
         st = lib.okv_append_quantize(ctypes.byref(d), fake, fake, 1, fake, fake, fake, fake, 0, None, None)
         assert st == okv.ERR_UNSUPPORTED, field
         assert b"128" in lib.okv_last_error_string() or b"16" in lib.okv_last_error_string()
