@@ -276,12 +276,6 @@ constexpr int kUmEpiWarps = 8;
 constexpr int kUmProducer = kUmEpiWarps;             // warp index of the producer
 constexpr int kUmThreads = 32 * (kUmEpiWarps + 1);
 constexpr int kUmTile = 128;
-// value codes of four consecutive slots written as 4-byte words after a byte
-// transpose across the quad of lanes that holds them (else one byte store each)
-#ifndef OKV_UM_QUAD_STORES
-#define OKV_UM_QUAD_STORES 1
-#endif
-constexpr bool kUmQuadStores = OKV_UM_QUAD_STORES != 0;
 constexpr int kUmStages = 3;
 constexpr uint32_t kUmRegion = 16384;                 // 128 rows x 128 B
 constexpr uint32_t kUmBBytes = 6 * kUmRegion;         // 3 parts x 2 K-blocks
@@ -545,8 +539,7 @@ __global__ void __launch_bounds__(kUmThreads, 1) append_umma_kernel(AppendArgs a
       um_wait_ld();
       um_fence_before();
       mbar_arrive(&tmem_free[i & 1]);  // the buffer may take tile i + 2's MMAs
-      // every lane stays in the loop body (the value codes below are
-      // exchanged across quads of lanes); `valid` gates the stores
+      // `valid` gates the stores (a token past T, or a bad destination)
       bool valid = tok < T;
       if (valid && !slot_ok) {
         raise_flag(a.status, OKV_DEV_BAD_SLOT);
@@ -591,42 +584,9 @@ __global__ void __launch_bounds__(kUmThreads, 1) append_umma_kernel(AppendArgs a
           kp[0] = make_uint4(w[0], w[1], w[2], w[3]);
           kp[1] = make_uint4(w[4], w[5], w[6], w[7]);
         }
-      } else if constexpr (kUmQuadStores) {
-        // The value codes of four tokens in slots 4j .. 4j + 3 of one block
-        // share 4-byte words (byte b of those tokens, one per token).  When
-        // the four lanes of a quad hold exactly such tokens, in slot order,
-        // a 4 x 4 byte transpose across the quad turns lane i's share into
-        // the eight words of code bytes b = 4k + i; otherwise each lane
-        // writes its 32 bytes one by one.
-        const int qbase = lane & ~3, qi = lane & 3;
-        const int blk0 = __shfl_sync(0xffffffffu, blk, qbase);
-        const int grp0 = __shfl_sync(0xffffffffu, p >> 2, qbase);
-        const bool fits = valid && blk == blk0 && (p >> 2) == grp0 && (p & 3) == qi;
-        const uint32_t fit_mask = __ballot_sync(0xffffffffu, fits);
-        const bool quad_ok = ((fit_mask >> qbase) & 0xfu) == 0xfu;
-        uint32_t tw[8];
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          // byte qi of word k from each lane of the quad
-          const uint32_t x0 = __shfl_sync(0xffffffffu, w[k], qbase + 0);
-          const uint32_t x1 = __shfl_sync(0xffffffffu, w[k], qbase + 1);
-          const uint32_t x2 = __shfl_sync(0xffffffffu, w[k], qbase + 2);
-          const uint32_t x3 = __shfl_sync(0xffffffffu, w[k], qbase + 3);
-          const uint32_t sel = (uint32_t)qi * 0x11u + 0x40u;  // result bytes 0, 1: byte qi of the first, of the second
-          const uint32_t lo = prmt(x0, x1, sel);
-          const uint32_t hi = prmt(x2, x3, sel);
-          tw[k] = prmt(lo, hi, 0x5410u);  // [x0.qi, x1.qi, x2.qi, x3.qi]
-        }
-        if (quad_ok) {
-          // word of code byte b = 4k + qi for slots 4 (sl >> 2) .. + 3
-#pragma unroll
-          for (int k = 0; k < 8; ++k)
-            *reinterpret_cast<uint32_t*>(bp + kVcOff + ((k * 4 + (sl >> 2)) << 4) + (qi << 2)) = tw[k];
-        } else if (valid) {
-#pragma unroll
-          for (int bb = 0; bb < 32; ++bb) bp[v_code_offset(sl, bb)] = (uint8_t)(w[bb >> 2] >> (8 * (bb & 3)));
-        }
       } else if (valid) {
+        // (four tokens' bytes share a 4-byte word here; assembling the words by
+        // a byte transpose across lane quads measured no faster than byte stores)
 #pragma unroll
         for (int bb = 0; bb < 32; ++bb) bp[v_code_offset(sl, bb)] = (uint8_t)(w[bb >> 2] >> (8 * (bb & 3)));
       }

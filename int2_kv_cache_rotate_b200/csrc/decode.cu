@@ -500,10 +500,9 @@ __global__ void __launch_bounds__(kDecWarps * 32) decode_simt_kernel(DecodeArgs 
 // fp16 hi+lo pairs), folded into the warp's state in registers.
 // ---------------------------------------------------------------------------
 constexpr int kHW = 8;                             // warps per CTA
-constexpr int kHStages = 6;                        // ring stages with two CTAs per SM (G <= 4)
-constexpr int kHStagesSolo = 10;                   // ring stages with one CTA per SM (G = 8)
+constexpr int kHStages = 6;                        // ring stages
 constexpr int kIssueBatch = 2;                     // stages the producer issues at a time
-static_assert(kHStages % kIssueBatch == 0 && kHStagesSolo % kIssueBatch == 0 && (kIssueBatch == 1 || kIssueBatch == 2),
+static_assert(kHStages % kIssueBatch == 0 && (kIssueBatch == 1 || kIssueBatch == 2),
               "a batch of up to 16-block stages must start at a multiple of its size and fit one 32-block window");
 constexpr int kSlotsPerStage = 16;                 // block-heads per stage
 constexpr int kHStageBytes = kSlotsPerStage * kBlockHeadBytes;  // 18432
@@ -528,9 +527,10 @@ template <int G>
 struct HCfg {
   static constexpr int NT = G <= 4 ? 1 : G / 4;  // n-tiles of 8 columns = 4 heads x 2 limbs
   static constexpr int HP = 4 * NT;              // heads incl. padding
-  // one CTA per SM for G = 8 (its registers): that CTA gets a deeper ring,
-  // so the bytes in flight per SM stay close to two CTAs' worth
-  static constexpr int NS = G <= 4 ? kHStages : kHStagesSolo;
+  // (a 10-stage ring for the one-CTA-per-SM G = 8 kernel, and a 4-stage one
+  // for G = 4, measured the same as 6: the kernel is bound by its per-step
+  // arithmetic, not by the bytes in flight)
+  static constexpr int NS = kHStages;
   static constexpr size_t ring_bytes = (size_t)NS * kHStageBytes;
   // fp32 o' accumulators live in tensor memory: thread (warp w, lane l) owns
   // TMEM lane 32 (w % 4) + l, columns 16 NT (w / 4) .. +16 NT

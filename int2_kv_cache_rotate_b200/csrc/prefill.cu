@@ -7,7 +7,7 @@
 //   1. query rotation: q~ = q R_K, split into fp16 hi + lo halves of
 //      q~ 2^-e (e per row so that the halves stay in fp16 range) and the
 //      per-group sums of q~;
-//   2. attention (this file's main kernel): a CTA of 4 warps takes 64 query
+//   2. attention (this file's main kernel): a CTA of 8 warps takes 128 query
 //      rows (query token x query head of one KV head) and streams the key
 //      positions 0 .. its last row's position in 16-token chunks.  Every
 //      chunk is staged in shared memory as fp16: the 2-bit codes (0..3 are
@@ -29,7 +29,7 @@
 namespace okv {
 namespace {
 
-constexpr int kPfWarps = 4;
+constexpr int kPfWarps = 8;
 constexpr int kPfRows = 16 * kPfWarps;  // query rows per CTA
 constexpr int kKStride = kD + 8;        // fp16 per staged key row (bank-conflict-free fragment loads)
 constexpr int kVStride = 16 + 8;        // fp16 per staged value column (values are staged transposed)
@@ -55,71 +55,81 @@ constexpr int kQaux = 8;
 constexpr int kOStride = 132;
 
 // ---------------------------------------------------------------------------
-// 1. q~ = q R_K for the chunk.  One CTA per (query token, query head); warp w
-// holds rows 16w..16w+15 of U_K in registers, the partial sums meet in shared
-// memory and warp 0 runs the butterfly and the bit-reversal remap.
+// 1. q~ = q R_K for the chunk.  One CTA per (query head, 16 query tokens):
+// warp w holds rows 16w..16w+15 of U_K in registers for all 16 tokens; per
+// token the eight warps' partial sums meet in shared memory and warp (token
+// mod 8) runs the butterfly and the bit-reversal remap.
 // ---------------------------------------------------------------------------
+constexpr int kQrTok = 16;
+
 __global__ void __launch_bounds__(256) prefill_qrot_kernel(PrefillArgs a) {
-  __shared__ float red[8][kD];
-  const int row = blockIdx.x;  // token * hq + head
-  const int head = row % a.hq;
+  __shared__ float red[2][8][kD];
+  const int head = blockIdx.y;
   const int hk = head / a.g;
+  const int tok0 = blockIdx.x * kQrTok;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const float* U = a.u_k + (size_t)hk * kD * kD;
-  const float xv = __bfloat162float(a.q[(size_t)row * kD + 16 * warp + (lane & 15)]);
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  float4 u[16];
 #pragma unroll
-  for (int r = 0; r < 16; ++r) {
-    const float4 u = __ldg(reinterpret_cast<const float4*>(U + (size_t)(16 * warp + r) * kD) + lane);
-    const float x = __shfl_sync(0xffffffffu, xv, r);
-    acc.x = fmaf(x, u.x, acc.x);
-    acc.y = fmaf(x, u.y, acc.y);
-    acc.z = fmaf(x, u.z, acc.z);
-    acc.w = fmaf(x, u.w, acc.w);
-  }
-  *reinterpret_cast<float4*>(&red[warp][4 * lane]) = acc;
-  __syncthreads();
-  if (warp != 0) return;
-  float y[4];
+  for (int r = 0; r < 16; ++r) u[r] = __ldg(reinterpret_cast<const float4*>(U + (size_t)(16 * warp + r) * kD) + lane);
+  for (int i = 0; i < kQrTok; ++i) {
+    const int tok = tok0 + i;
+    if (tok >= a.T) break;  // uniform across the CTA
+    const int row = tok * a.hq + head;
+    const float xv = __bfloat162float(a.q[(size_t)row * kD + 16 * warp + (lane & 15)]);
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-  for (int aa = 0; aa < 4; ++aa) {
-    float s = 0.f;
+    for (int r = 0; r < 16; ++r) {
+      const float x = __shfl_sync(0xffffffffu, xv, r);
+      acc.x = fmaf(x, u[r].x, acc.x);
+      acc.y = fmaf(x, u[r].y, acc.y);
+      acc.z = fmaf(x, u[r].z, acc.z);
+      acc.w = fmaf(x, u[r].w, acc.w);
+    }
+    *reinterpret_cast<float4*>(&red[i & 1][warp][4 * lane]) = acc;
+    __syncthreads();  // (double-buffered: the next token's sums go to the other half)
+    if (warp != (i & 7)) continue;
+    float y[4];
 #pragma unroll
-    for (int w = 0; w < 8; ++w) s += red[w][lane + 32 * aa];
-    y[aa] = s;
-  }
-  wht128_warp(y, lane);
+    for (int aa = 0; aa < 4; ++aa) {
+      float sum = 0.f;
 #pragma unroll
-  for (int aa = 0; aa < 4; ++aa) y[aa] *= kInvSqrtD;
-  // lane l holds rotated channels 4 r + {0, 2, 1, 3} (r = rev5(l)) in y[0..3]
-  const int r = rev5(lane);
-  const float zc[4] = {y[0], y[2], y[1], y[3]};
-  float amax = fmaxf(fmaxf(fabsf(y[0]), fabsf(y[1])), fmaxf(fabsf(y[2]), fabsf(y[3])));
-  amax = warp_max(amax);
-  // 2^-e with amax 2^-e in [1, 2): the hi half keeps 11 bits, the lo half the next 11
-  int e = 0;
-  if (amax > 0.f) e = ((__float_as_int(amax) >> 23) & 0xff) - 127;
-  e = max(-100, min(100, e));
-  const float down = __int_as_float((127 - e) << 23);
-  __half* hi = a.qhi + (size_t)row * kD + 4 * r;
-  __half* lo = a.qlo + (size_t)row * kD + 4 * r;
+      for (int w = 0; w < 8; ++w) sum += red[i & 1][w][lane + 32 * aa];
+      y[aa] = sum;
+    }
+    wht128_warp(y, lane);
 #pragma unroll
-  for (int f = 0; f < 4; ++f) {
-    const float x = zc[f] * down;
-    const __half h = __float2half_rn(x);
-    hi[f] = h;
-    lo[f] = __float2half_rn(x - __half2float(h));
-  }
-  // per-group sums of q~: channels 4r.. lie in group r ng / 32
-  float part = (zc[0] + zc[1]) + (zc[2] + zc[3]);
-  float gs[4];
+    for (int aa = 0; aa < 4; ++aa) y[aa] *= kInvSqrtD;
+    // lane l holds rotated channels 4 r + {0, 2, 1, 3} (r = rev5(l)) in y[0..3]
+    const int r = rev5(lane);
+    const float zc[4] = {y[0], y[2], y[1], y[3]};
+    float amax = fmaxf(fmaxf(fabsf(y[0]), fabsf(y[1])), fmaxf(fabsf(y[2]), fabsf(y[3])));
+    amax = warp_max(amax);
+    // 2^-e with amax 2^-e in [1, 2): the hi half keeps 11 bits, the lo half the next 11
+    int e = 0;
+    if (amax > 0.f) e = ((__float_as_int(amax) >> 23) & 0xff) - 127;
+    e = max(-100, min(100, e));
+    const float down = __int_as_float((127 - e) << 23);
+    __half* hi = a.qhi + (size_t)row * kD + 4 * r;
+    __half* lo = a.qlo + (size_t)row * kD + 4 * r;
 #pragma unroll
-  for (int k = 0; k < 4; ++k) gs[k] = warp_sum((k < a.ng && r * a.ng / 32 == k) ? part : 0.f);
-  if (lane == 0) {
-    float* aux = a.qaux + (size_t)row * kQaux;
+    for (int f = 0; f < 4; ++f) {
+      const float x = zc[f] * down;
+      const __half h = __float2half_rn(x);
+      hi[f] = h;
+      lo[f] = __float2half_rn(x - __half2float(h));
+    }
+    // per-group sums of q~: channels 4r.. lie in group r ng / 32
+    const float part = (zc[0] + zc[1]) + (zc[2] + zc[3]);
+    float gs[4];
 #pragma unroll
-    for (int k = 0; k < 4; ++k) aux[k] = gs[k];
-    aux[4] = __int_as_float((127 + e) << 23);
+    for (int k = 0; k < 4; ++k) gs[k] = warp_sum((k < a.ng && r * a.ng / 32 == k) ? part : 0.f);
+    if (lane == 0) {
+      float* aux = a.qaux + (size_t)row * kQaux;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) aux[k] = gs[k];
+      aux[4] = __int_as_float((127 + e) << 23);
+    }
   }
 }
 
@@ -145,7 +155,7 @@ __device__ __forceinline__ void split_half2(float x0, float x1, uint32_t& hi, ui
 }
 
 // ---------------------------------------------------------------------------
-// 2. attention.  Grid (ceil(rows / 64), Hkv); rows are (token, query head)
+// 2. attention.  Grid (ceil(rows / 128), Hkv); rows are (token, query head)
 // pairs of the KV head, token-major: row r = token (r / G), head (r % G).
 // Warp w owns rows 16w .. 16w + 15 of the CTA.  Fragment facts
 // (m16n8k16, f16): lane (g = lane / 4, t = lane % 4) holds A (row g, cols
@@ -222,81 +232,99 @@ __global__ void __launch_bounds__(kPfWarps * 32) prefill_attn_kernel(PrefillArgs
   const int pmax = a.first + last_row / a.g;  // last position any row of this CTA sees
   const int nchunks = pmax / 16 + 1;
   const int tid = threadIdx.x;
+  // Staging: thread tid -> K (tid < 128) or V, token (tid % 128) / 8, channels
+  // 16 (tid % 8) .. + 15 of a 16-token chunk.  Chunk ch is exactly block
+  // column ch of the sequence.  The global loads of chunk ch + 1 are issued
+  // before chunk ch's arithmetic and its block id one chunk earlier still, so
+  // neither latency sits between two barriers.
+  const int is_v = tid >> 7, tk = (tid & 127) >> 3, part = tid & 7;
+  auto chunk_block = [&](int ch) -> int {  // the chunk's block id when it holds INT2 positions, else -1
+    const int lo = 16 * ch, hi = min(16 * ch + 15, min(pmax, a.L - 1));
+    const bool int2 = ch < nchunks && hi >= lo && max(lo, a.nsink) <= min(hi, a.L - kWin - 1);
+    return int2 ? a.block_table[(size_t)a.slot * a.mbps + ch] : -1;
+  };
+  int f_src = 0;  // fetched chunk: 0 masked, 1 INT2, 2 fp16 window, 3 fp16 sink
+  uint4 f0 = make_uint4(0, 0, 0, 0), f1 = make_uint4(0, 0, 0, 0);
+  uint32_t f_sm = 0;
+  auto fetch = [&](int ch, int blk) {
+    const int p = 16 * ch + tk;
+    f_src = 0;
+    if (p <= pmax && p < a.L) {
+      if (p < a.nsink) {
+        f_src = 3;
+      } else if (p >= a.L - kWin) {
+        f_src = 2;
+      } else if (blk >= 0 && blk < a.num_blocks) {
+        f_src = 1;
+      } else if (part == 0 && !is_v) {
+        raise_flag(a.status, OKV_DEV_BAD_BLOCK);
+      }
+    }
+    if (f_src == 1) {
+      const uint8_t* bp = a.pages + ((size_t)blk * a.hkv + hk) * a.bhb;
+      const int sl = p & 15;
+      if (!is_v) {
+        f0.x = *reinterpret_cast<const uint32_t*>(bp + kKcOff + sl * 32 + 4 * part);
+      } else {
+        uint32_t w = 0;
+#pragma unroll
+        for (int bq = 0; bq < 4; ++bq) w |= (uint32_t)bp[v_code_offset(sl, 4 * part + bq)] << (8 * bq);
+        f0.x = w;
+      }
+      if (part < NG) f_sm = *reinterpret_cast<const uint32_t*>(bp + sm_offset(NG, is_v, sl, part));
+    } else if (f_src >= 2) {
+      const size_t rows_per_kind = f_src == 2 ? (size_t)kWin : (size_t)a.nsink;
+      const size_t base = (((size_t)a.slot * a.hkv + hk) * 2 + is_v) * rows_per_kind;
+      const size_t row = f_src == 2 ? (size_t)(p % kWin) : (size_t)p;
+      const __half* srcb = f_src == 2 ? a.ring : a.sink;
+      const uint4* xr = reinterpret_cast<const uint4*>(srcb + (base + row) * kD + 16 * part);
+      f0 = xr[0];
+      f1 = xr[1];
+    }
+  };
+  auto stage = [&]() {
+    __half x16[16];
+    if (f_src == 1) {
+#pragma unroll
+      for (int j = 0; j < 16; ++j) x16[j] = __int2half_rn((int)((f0.x >> (2 * j)) & 3u));  // K and V alike
+    } else if (f_src >= 2) {
+      *reinterpret_cast<uint4*>(x16) = f0;
+      *reinterpret_cast<uint4*>(x16 + 8) = f1;
+    } else {
+#pragma unroll
+      for (int j = 0; j < 16; ++j) x16[j] = __float2half_rn(0.f);
+    }
+    if (!is_v) {
+      *reinterpret_cast<uint4*>(kc + tk * kKStride + 16 * part) = *reinterpret_cast<const uint4*>(x16);
+      *reinterpret_cast<uint4*>(kc + tk * kKStride + 16 * part + 8) = *reinterpret_cast<const uint4*>(x16 + 8);
+    } else {
+#pragma unroll
+      for (int j = 0; j < 16; ++j) vc[(16 * part + j) * kVStride + tk] = x16[j];
+    }
+    if (part < NG) {  // one thread per (token, group, K|V): the group's scale and minimum
+      float s_g = 1.f, m_g = 0.f;  // fp16 rows: the values themselves
+      if (f_src == 1) {
+        s_g = __half2float(__ushort_as_half((unsigned short)(f_sm & 0xffff)));
+        m_g = __half2float(__ushort_as_half((unsigned short)(f_sm >> 16)));
+      } else if (f_src == 0) {
+        s_g = m_g = 0.f;
+      }
+      float(*dst)[NG][2] = is_v ? vsm : ksm;
+      dst[tk][part][0] = s_g;
+      dst[tk][part][1] = m_g;
+    }
+    if (part == 0 && !is_v) tpos_ok[tk] = f_src != 0;
+  };
+  fetch(0, chunk_block(0));
+  int blk_next = chunk_block(1);
   for (int ch = 0; ch < nchunks; ++ch) {
     __syncthreads();  // the previous chunk's tiles are no longer read
-    // ---- stage chunk ch: thread tid -> token tid / 8, channels 16 (tid % 8) .. + 15
-    {
-      const int tk = tid >> 3, part = tid & 7;
-      const int p = 16 * ch + tk;
-      int kind_src = 0;  // 0 masked, 1 INT2, 2 fp16 window, 3 fp16 sink
-      const uint8_t* bp = nullptr;
-      if (p <= pmax && p < a.L) {
-        if (p < a.nsink) {
-          kind_src = 3;
-        } else if (p >= a.L - kWin) {
-          kind_src = 2;
-        } else {
-          const int blk = a.block_table[(size_t)a.slot * a.mbps + (p >> 4)];
-          if (blk >= 0 && blk < a.num_blocks) {
-            kind_src = 1;
-            bp = a.pages + ((size_t)blk * a.hkv + hk) * a.bhb;
-          } else if (part == 0) {
-            raise_flag(a.status, OKV_DEV_BAD_BLOCK);
-          }
-        }
-      }
-      __half kv16[16], vv16[16];
-      if (kind_src == 1) {
-        const int sl = p & 15;
-        const uint32_t kw = *reinterpret_cast<const uint32_t*>(bp + kKcOff + sl * 32 + 4 * part);
-#pragma unroll
-        for (int j = 0; j < 16; ++j) kv16[j] = __int2half_rn((int)((kw >> (2 * j)) & 3u));
-#pragma unroll
-        for (int bq = 0; bq < 4; ++bq) {
-          const uint32_t vb = bp[v_code_offset(sl, 4 * part + bq)];
-#pragma unroll
-          for (int f = 0; f < 4; ++f) vv16[4 * bq + f] = __int2half_rn((int)((vb >> (2 * f)) & 3u));
-        }
-      } else if (kind_src >= 2) {
-        const size_t base = (((size_t)a.slot * a.hkv + hk) * 2) * (kind_src == 2 ? kWin : a.nsink);
-        const size_t rowk = kind_src == 2 ? (size_t)(p % kWin) : (size_t)p;
-        const size_t rows_per_kind = kind_src == 2 ? (size_t)kWin : (size_t)a.nsink;
-        const __half* srcb = kind_src == 2 ? a.ring : a.sink;
-        const uint4* kr = reinterpret_cast<const uint4*>(srcb + (base + rowk) * kD + 16 * part);
-        const uint4* vr = reinterpret_cast<const uint4*>(srcb + (base + rows_per_kind + rowk) * kD + 16 * part);
-        *reinterpret_cast<uint4*>(kv16) = kr[0];
-        *reinterpret_cast<uint4*>(kv16 + 8) = kr[1];
-        *reinterpret_cast<uint4*>(vv16) = vr[0];
-        *reinterpret_cast<uint4*>(vv16 + 8) = vr[1];
-      } else {
-#pragma unroll
-        for (int j = 0; j < 16; ++j) kv16[j] = vv16[j] = __float2half_rn(0.f);
-      }
-      *reinterpret_cast<uint4*>(kc + tk * kKStride + 16 * part) = *reinterpret_cast<const uint4*>(kv16);
-      *reinterpret_cast<uint4*>(kc + tk * kKStride + 16 * part + 8) = *reinterpret_cast<const uint4*>(kv16 + 8);
-#pragma unroll
-      for (int j = 0; j < 16; ++j) vc[(16 * part + j) * kVStride + tk] = vv16[j];
-      if (part < NG) {  // one thread per (token, group): the group's scale and minimum
-        float s_k = 1.f, m_k = 0.f, s_v = 1.f, m_v = 0.f;
-        if (kind_src == 1) {
-          const int sl = p & 15;
-          const uint32_t w0 = *reinterpret_cast<const uint32_t*>(bp + sm_offset(NG, 0, sl, part));
-          const uint32_t w1 = *reinterpret_cast<const uint32_t*>(bp + sm_offset(NG, 1, sl, part));
-          s_k = __half2float(__ushort_as_half((unsigned short)(w0 & 0xffff)));
-          m_k = __half2float(__ushort_as_half((unsigned short)(w0 >> 16)));
-          s_v = __half2float(__ushort_as_half((unsigned short)(w1 & 0xffff)));
-          m_v = __half2float(__ushort_as_half((unsigned short)(w1 >> 16)));
-        } else if (kind_src == 0) {
-          s_k = m_k = s_v = m_v = 0.f;
-        }
-        ksm[tk][part][0] = s_k;
-        ksm[tk][part][1] = m_k;
-        vsm[tk][part][0] = s_v;
-        vsm[tk][part][1] = m_v;
-      }
-      if (part == 0) tpos_ok[tk] = kind_src != 0;
-    }
+    stage();
     __syncthreads();
+    if (ch + 1 < nchunks) {
+      fetch(ch + 1, blk_next);
+      blk_next = chunk_block(ch + 2);
+    }
     // ---- scores of 16 rows x 16 tokens, per group
     float d[NG][2][4];
 #pragma unroll
@@ -416,37 +444,60 @@ __global__ void __launch_bounds__(kPfWarps * 32) prefill_attn_kernel(PrefillArgs
 }
 
 // ---------------------------------------------------------------------------
-// 3. o = (o' / l) R_V^T: one warp per row (8 rows per CTA), U_V rows of the
-// row's KV head read through L1.
+// 3. o = (o' / l) R_V^T.  One CTA per (query head, 16 query tokens): U_V of
+// the head's KV head is staged in shared memory once, then warp w takes
+// tokens w and w + 8: un-permute and butterfly in registers, and the U_V^T
+// matvec from shared memory (lane l produces outputs l + 32 j).
 // ---------------------------------------------------------------------------
+constexpr int kUrTok = 16;
+constexpr int kUStride = kD + 4;  // floats per staged U_V row
+
 __global__ void __launch_bounds__(256) prefill_unrotate_kernel(PrefillArgs a) {
+  extern __shared__ __align__(16) float us_[];  // U_V [128][132]
+  const int head = blockIdx.y;
+  const int hk = head / a.g;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int row = blockIdx.x * 8 + warp;
-  if (row >= a.T * a.hq) return;
-  const int hk = (row % a.hq) / a.g;
-  const float* src = a.obuf + (size_t)row * kOStride;
-  const float l = src[128];
-  const float inv = l > 0.f ? 1.f / l : 0.f;
-  // lane l: pre-permutation channels l + 32 aa = rotated channels 4 rev5(l) + rev2(aa)
-  const int r = rev5(lane);
-  float y[4];
-#pragma unroll
-  for (int aa = 0; aa < 4; ++aa) y[aa] = src[4 * r + rev2(aa)] * inv;
-  wht128_warp(y, lane);
-  float x[4];
-#pragma unroll
-  for (int aa = 0; aa < 4; ++aa) x[aa] = y[aa] * kInvSqrtD;  // x_i for i = lane + 32 aa
-  // o_c = sum_i x_i U_V[c][i]: lane owns outputs c = lane + 32 j
-  const float* U = a.u_v + (size_t)hk * kD * kD;
-  float acc[4] = {0.f, 0.f, 0.f, 0.f};
-  for (int i = 0; i < kD; ++i) {
-    const float xi = __shfl_sync(0xffffffffu, x[i >> 5], i & 31);
-#pragma unroll
-    for (int j = 0; j < 4; ++j) acc[j] = fmaf(xi, __ldg(U + (size_t)(lane + 32 * j) * kD + i), acc[j]);
+  {
+    const float4* U = reinterpret_cast<const float4*>(a.u_v + (size_t)hk * kD * kD);
+    for (int i = threadIdx.x; i < kD * kD / 4; i += blockDim.x) {
+      const int r = i / (kD / 4), c4 = i % (kD / 4);
+      *reinterpret_cast<float4*>(us_ + r * kUStride + 4 * c4) = __ldg(U + i);
+    }
   }
-  float* dst = a.out + (size_t)row * kD;
+  __syncthreads();
+  for (int i = warp; i < kUrTok; i += 8) {
+    const int tok = blockIdx.x * kUrTok + i;
+    if (tok >= a.T) break;
+    const int row = tok * a.hq + head;
+    const float* src = a.obuf + (size_t)row * kOStride;
+    const float l = src[128];
+    const float inv = l > 0.f ? 1.f / l : 0.f;
+    // lane l: pre-permutation channels l + 32 aa = rotated channels 4 rev5(l) + rev2(aa)
+    const int r = rev5(lane);
+    float y[4];
 #pragma unroll
-  for (int j = 0; j < 4; ++j) dst[lane + 32 * j] = acc[j];
+    for (int aa = 0; aa < 4; ++aa) y[aa] = src[4 * r + rev2(aa)] * inv;
+    wht128_warp(y, lane);
+    float x[4];
+#pragma unroll
+    for (int aa = 0; aa < 4; ++aa) x[aa] = y[aa] * kInvSqrtD;  // x_i for i = lane + 32 aa
+    // o_c = sum_i x_i U_V[c][i]: lane owns outputs c = lane + 32 j
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
+    for (int i4 = 0; i4 < kD / 4; ++i4) {
+      float xi[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) xi[q] = __shfl_sync(0xffffffffu, x[(4 * i4 + q) >> 5], (4 * i4 + q) & 31);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float4 uu = *reinterpret_cast<const float4*>(us_ + (lane + 32 * j) * kUStride + 4 * i4);
+        acc[j] = fmaf(xi[0], uu.x, fmaf(xi[1], uu.y, fmaf(xi[2], uu.z, fmaf(xi[3], uu.w, acc[j]))));
+      }
+    }
+    float* dst = a.out + (size_t)row * kD;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) dst[lane + 32 * j] = acc[j];
+  }
 }
 
 }  // namespace
@@ -495,7 +546,7 @@ okv_status launch_prefill(const okv_cache_desc* d, const void* q, int T, int slo
   a.mbps = d->max_blocks_per_seq;
   a.num_blocks = d->num_blocks;
   a.nsink = d->num_sink;
-  prefill_qrot_kernel<<<(unsigned)rows, 256, 0, s>>>(a);
+  prefill_qrot_kernel<<<dim3((unsigned)((T + kQrTok - 1) / kQrTok), (unsigned)a.hq), 256, 0, s>>>(a);
   okv_status st = check_launch("prefill query rotation");
   if (st != OKV_OK) return st;
   const dim3 grid((unsigned)((T * a.g + kPfRows - 1) / kPfRows), (unsigned)a.hkv);
@@ -506,7 +557,11 @@ okv_status launch_prefill(const okv_cache_desc* d, const void* q, int T, int slo
   }
   st = check_launch("prefill attention");
   if (st != OKV_OK) return st;
-  prefill_unrotate_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, s>>>(a);
+  const size_t usmem = (size_t)kD * kUStride * sizeof(float);
+  static std::atomic<uint32_t> attr_set{0};
+  cudaError_t e = set_smem_limit_once((const void*)prefill_unrotate_kernel, (int)usmem, attr_set);
+  if (e != cudaSuccess) return fail(OKV_ERR_CUDA, "prefill un-rotation smem attribute: %s", cudaGetErrorString(e));
+  prefill_unrotate_kernel<<<dim3((unsigned)((T + kUrTok - 1) / kUrTok), (unsigned)a.hq), 256, usmem, s>>>(a);
   return check_launch("prefill un-rotation");
 }
 
