@@ -558,12 +558,23 @@ __global__ void __launch_bounds__(kUmThreads, 1) append_umma_kernel(AppendArgs a
       uint32_t smg[NG];                                    // (scale, min) bits of each group
 #pragma unroll
       for (int k = 0; k < NG; ++k) {
-        float mn = v[GW * k], mx = v[GW * k];
+        // eight interleaved chains, then a tree: the extremes do not depend on the order
+        float mn8[8], mx8[8];
 #pragma unroll
-        for (int j = GW * k + 1; j < GW * (k + 1); ++j) {
-          mn = fminf(mn, v[j]);
-          mx = fmaxf(mx, v[j]);
+        for (int r = 0; r < 8; ++r) mn8[r] = mx8[r] = v[GW * k + r];
+#pragma unroll
+        for (int j = GW * k + 8; j < GW * (k + 1); ++j) {
+          mn8[j & 7] = fminf(mn8[j & 7], v[j]);
+          mx8[j & 7] = fmaxf(mx8[j & 7], v[j]);
         }
+#pragma unroll
+        for (int r = 4; r >= 1; r >>= 1)
+#pragma unroll
+          for (int u = 0; u < r; ++u) {
+            mn8[u] = fminf(mn8[u], mn8[u + r]);
+            mx8[u] = fmaxf(mx8[u], mx8[u + r]);
+          }
+        const float mn = mn8[0], mx = mx8[0];
         const float s32 = __fdiv_rn(__fsub_rn(mx, mn), 3.0f);
         const __half s16 = fp16_sat(s32);
         const __half m16 = fp16_sat(mn);

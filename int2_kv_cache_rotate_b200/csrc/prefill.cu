@@ -32,7 +32,15 @@ namespace {
 constexpr int kPfWarps = 8;
 constexpr int kPfRows = 16 * kPfWarps;  // query rows per CTA
 constexpr int kKStride = kD + 8;        // fp16 per staged key row (bank-conflict-free fragment loads)
-constexpr int kVStride = 16 + 8;        // fp16 per staged value column (values are staged transposed)
+// value rows are staged row-major, 16-byte chunk c of token row r at chunk
+// position c ^ (r & 7), and read with transposing matrix loads
+__device__ __forceinline__ int vchunk(int row, int c) { return row * kD + ((c ^ (row & 7)) << 3); }
+
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t (&r)[4], const void* p) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"((uint32_t)__cvta_generic_to_shared(p)));
+}
 
 struct PrefillArgs {
   const __nv_bfloat16* q;  // [T][Hq][128]
@@ -166,10 +174,11 @@ __device__ __forceinline__ void split_half2(float x0, float x1, uint32_t& hi, ui
 template <int NG>
 __global__ void __launch_bounds__(kPfWarps * 32) prefill_attn_kernel(PrefillArgs a) {
   constexpr int KSG = 8 / NG;  // 16-channel k-steps per group
-  __shared__ __align__(16) __half kc[16 * kKStride];  // [token][channel]: codes or fp16 values
-  __shared__ __align__(16) __half vc[kD * kVStride];  // [channel][token]
-  __shared__ float ksm[16][NG][2], vsm[16][NG][2];    // (scale, min) per token and group
-  __shared__ int tpos_ok[16];                          // 1 if the chunk's token is a readable position
+  // two buffers of each (chunk ch in buffer ch & 1): one barrier per chunk
+  __shared__ __align__(16) __half kc[2][16 * kKStride];  // [token][channel]: codes or fp16 values
+  __shared__ __align__(16) __half vt[2][16 * kD];        // [token][channel], chunks swizzled (vchunk)
+  __shared__ float ksm[2][16][NG][2], vsm[2][16][NG][2];  // (scale, min) per token and group
+  __shared__ int tpos_ok[2][16];                          // 1 if the chunk's token is a readable position
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int g = lane >> 2, t = lane & 3;
   const int hk = blockIdx.y;
@@ -282,7 +291,7 @@ __global__ void __launch_bounds__(kPfWarps * 32) prefill_attn_kernel(PrefillArgs
       f1 = xr[1];
     }
   };
-  auto stage = [&]() {
+  auto stage = [&](int buf) {
     __half x16[16];
     if (f_src == 1) {
 #pragma unroll
@@ -294,12 +303,18 @@ __global__ void __launch_bounds__(kPfWarps * 32) prefill_attn_kernel(PrefillArgs
 #pragma unroll
       for (int j = 0; j < 16; ++j) x16[j] = __float2half_rn(0.f);
     }
+    // parts 4..7 store their upper 8 channels first: the 8 lanes of a token
+    // then hit 8 distinct bank quads in each of the two store instructions
+    const int hi1 = (part >> 2) & 1;
+    const uint4 lo8 = *reinterpret_cast<const uint4*>(x16), hi8 = *reinterpret_cast<const uint4*>(x16 + 8);
+    const uint4 first = hi1 ? hi8 : lo8, second = hi1 ? lo8 : hi8;
     if (!is_v) {
-      *reinterpret_cast<uint4*>(kc + tk * kKStride + 16 * part) = *reinterpret_cast<const uint4*>(x16);
-      *reinterpret_cast<uint4*>(kc + tk * kKStride + 16 * part + 8) = *reinterpret_cast<const uint4*>(x16 + 8);
+      __half* row = kc[buf] + tk * kKStride + 16 * part;
+      *reinterpret_cast<uint4*>(row + 8 * hi1) = first;
+      *reinterpret_cast<uint4*>(row + 8 - 8 * hi1) = second;
     } else {
-#pragma unroll
-      for (int j = 0; j < 16; ++j) vc[(16 * part + j) * kVStride + tk] = x16[j];
+      *reinterpret_cast<uint4*>(vt[buf] + vchunk(tk, 2 * part + hi1)) = first;
+      *reinterpret_cast<uint4*>(vt[buf] + vchunk(tk, 2 * part + 1 - hi1)) = second;
     }
     if (part < NG) {  // one thread per (token, group, K|V): the group's scale and minimum
       float s_g = 1.f, m_g = 0.f;  // fp16 rows: the values themselves
@@ -309,21 +324,28 @@ __global__ void __launch_bounds__(kPfWarps * 32) prefill_attn_kernel(PrefillArgs
       } else if (f_src == 0) {
         s_g = m_g = 0.f;
       }
-      float(*dst)[NG][2] = is_v ? vsm : ksm;
+      float(*dst)[NG][2] = is_v ? vsm[buf] : ksm[buf];
       dst[tk][part][0] = s_g;
       dst[tk][part][1] = m_g;
     }
-    if (part == 0 && !is_v) tpos_ok[tk] = f_src != 0;
+    if (part == 0 && !is_v) tpos_ok[buf][tk] = f_src != 0;
   };
+  // chunk 0 staged, chunk 1 fetched, chunk 2's block id in flight
   fetch(0, chunk_block(0));
-  int blk_next = chunk_block(1);
+  stage(0);
+  int blk_next = chunk_block(2);
+  if (1 < nchunks) fetch(1, chunk_block(1));
+  __syncthreads();
   for (int ch = 0; ch < nchunks; ++ch) {
-    __syncthreads();  // the previous chunk's tiles are no longer read
-    stage();
-    __syncthreads();
+    const int buf = ch & 1;
+    // chunk ch + 1 goes to the other buffer: its last readers (chunk ch - 1)
+    // passed the barrier that ended the previous iteration
     if (ch + 1 < nchunks) {
-      fetch(ch + 1, blk_next);
-      blk_next = chunk_block(ch + 2);
+      stage(buf ^ 1);
+      if (ch + 2 < nchunks) {
+        fetch(ch + 2, blk_next);
+        blk_next = chunk_block(ch + 3);
+      }
     }
     // ---- scores of 16 rows x 16 tokens, per group
     float d[NG][2][4];
@@ -333,17 +355,28 @@ __global__ void __launch_bounds__(kPfWarps * 32) prefill_attn_kernel(PrefillArgs
       for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
         for (int j = 0; j < 4; ++j) d[k][nt][j] = 0.f;
+    // one group: the low halves accumulate apart, so four chains of mma run side by side
+    float dl[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
     for (int ks = 0; ks < 8; ++ks) {
       const int k = ks / KSG;
 #pragma unroll
       for (int nt = 0; nt < 2; ++nt) {
-        const __half* kb = kc + (8 * nt + g) * kKStride + 16 * ks + 2 * t;
+        const __half* kb = kc[buf] + (8 * nt + g) * kKStride + 16 * ks + 2 * t;
         const uint32_t b0 = *reinterpret_cast<const uint32_t*>(kb);
         const uint32_t b1 = *reinterpret_cast<const uint32_t*>(kb + 8);
         mma_f16_pf(d[k][nt], qa_hi[ks], b0, b1);
-        mma_f16_pf(d[k][nt], qa_lo[ks], b0, b1);
+        if constexpr (NG == 1)
+          mma_f16_pf(dl[nt], qa_lo[ks], b0, b1);
+        else
+          mma_f16_pf(d[k][nt], qa_lo[ks], b0, b1);
       }
+    }
+    if constexpr (NG == 1) {
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) d[0][nt][j] += dl[nt][j];
     }
     // score (log2 units) of row h2, token 8 nt + 2 t + c: sum_k s_k raw_k 2^e + m_k sum_k
     float sc[2][2][2];  // [h2][nt][c]
@@ -353,13 +386,13 @@ __global__ void __launch_bounds__(kPfWarps * 32) prefill_attn_kernel(PrefillArgs
       for (int c = 0; c < 2; ++c) {
         const int tk = 8 * nt + 2 * t + c;
         const int p = 16 * ch + tk;
-        const bool ok = tpos_ok[tk] != 0;
+        const bool ok = tpos_ok[buf][tk] != 0;
 #pragma unroll
         for (int h2 = 0; h2 < 2; ++h2) {
           float x = 0.f;
 #pragma unroll
           for (int k = 0; k < NG; ++k)
-            x = fmaf(ksm[tk][k][0] * qup[h2], d[k][nt][2 * h2 + c], fmaf(ksm[tk][k][1], qsum[h2][k], x));
+            x = fmaf(ksm[buf][tk][k][0] * qup[h2], d[k][nt][2 * h2 + c], fmaf(ksm[buf][tk][k][1], qsum[h2][k], x));
           sc[h2][nt][c] = (ok && rok[h2] && p <= rpos[h2]) ? x : -INFINITY;
         }
       }
@@ -400,24 +433,30 @@ __global__ void __launch_bounds__(kPfWarps * 32) prefill_attn_kernel(PrefillArgs
       for (int q4 = 0; q4 < 4; ++q4) {
         const int h2 = q4 & 1, nt = q4 >> 1;
         const int t0 = 8 * nt + 2 * t;
-        split_half2(pr[h2][nt][0] * vsm[t0][k][0], pr[h2][nt][1] * vsm[t0 + 1][k][0], ah[q4], al[q4]);
+        split_half2(pr[h2][nt][0] * vsm[buf][t0][k][0], pr[h2][nt][1] * vsm[buf][t0 + 1][k][0], ah[q4], al[q4]);
       }
 #pragma unroll
       for (int h2 = 0; h2 < 2; ++h2)
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-          for (int c = 0; c < 2; ++c) msum[h2][k] = fmaf(pr[h2][nt][c], vsm[8 * nt + 2 * t + c][k][1], msum[h2][k]);
+          for (int c = 0; c < 2; ++c)
+            msum[h2][k] = fmaf(pr[h2][nt][c], vsm[buf][8 * nt + 2 * t + c][k][1], msum[h2][k]);
+      // B operands of n-tiles 2p, 2p + 1 (channels 16p .. 16p + 15, one group):
+      // matrix m of the transposing load is tokens 8 (m & 1) .. + 7 of n-tile 2p + (m >> 1)
+      const int mrow = (lane & 7) + 8 * ((lane >> 3) & 1), mhi = lane >> 4;
 #pragma unroll
-      for (int n = 0; n < 16; ++n) {
-        if (n * NG / 16 != k) continue;  // channels 8n .. 8n + 7 belong to group n ng / 16
-        const __half* vb = vc + (8 * n + g) * kVStride + 2 * t;
-        const uint32_t b0 = *reinterpret_cast<const uint32_t*>(vb);
-        const uint32_t b1 = *reinterpret_cast<const uint32_t*>(vb + 8);
-        mma_f16_pf(o[n], ah, b0, b1);
-        mma_f16_pf(o[n], al, b0, b1);
+      for (int pp = 0; pp < 8; ++pp) {
+        if (pp * NG / 8 != k) continue;  // channels 16 pp .. belong to group pp ng / 8
+        uint32_t bq[4];
+        ldsm_x4_trans(bq, vt[buf] + vchunk(mrow, 2 * pp + mhi));
+        mma_f16_pf(o[2 * pp], ah, bq[0], bq[1]);
+        mma_f16_pf(o[2 * pp], al, bq[0], bq[1]);
+        mma_f16_pf(o[2 * pp + 1], ah, bq[2], bq[3]);
+        mma_f16_pf(o[2 * pp + 1], al, bq[2], bq[3]);
       }
     }
+    __syncthreads();  // chunk ch + 1 is staged; buffer ch & 1 is free
   }
   // ---- o' rows and sums to the buffer: the quad's lanes hold columns 2t, 2t + 1 of every n-tile
 #pragma unroll
