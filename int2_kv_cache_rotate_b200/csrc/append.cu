@@ -11,6 +11,7 @@
 #include "append_warp.cuh"
 #include "okv_common.cuh"
 #include "okv_internal.h"
+#include "umma.cuh"
 
 namespace okv {
 namespace {
@@ -285,22 +286,7 @@ static_assert(7 * 8 + 4 <= kUmCtlBytes, "control region");
 constexpr size_t kUmSmem = 1024 + kUmBBytes + kUmStages * kUmABytes + kUmCtlBytes;
 constexpr uint32_t kUmTmemCols = 256;
 // instruction descriptor: D f32, A and B bf16, both K-major, N = 128, M = 128
-constexpr uint32_t kUmIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((128u >> 3) << 17) | ((128u >> 4) << 24);
-
-__device__ __forceinline__ uint32_t um_swz(uint32_t row, uint32_t byte_in_row) {
-  return row * 128u + ((((byte_in_row >> 4) ^ (row & 7u)) << 4) | (byte_in_row & 15u));
-}
-
-// shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row groups 1024 B apart
-__device__ __forceinline__ uint64_t um_desc(uint32_t saddr) {
-  uint64_t d = 0;
-  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);   // start address
-  d |= (uint64_t)1u << 16;                   // leading byte offset (unused for swizzled K-major), 16 B
-  d |= (uint64_t)(1024u >> 4) << 32;         // stride byte offset
-  d |= (uint64_t)1u << 46;                   // descriptor version for tcgen05
-  d |= (uint64_t)2u << 61;                   // 128-byte swizzle
-  return d;
-}
+constexpr uint32_t kUmIdesc = um_idesc(128, true, true);
 
 // TMA tiled load of a 3-D box at (x, y, z) into shared memory, completing on bar
 __device__ __forceinline__ void um_tma_load_3d(uint32_t dst, const CUtensorMap* map, int x, int y, int z,
@@ -311,45 +297,6 @@ __device__ __forceinline__ void um_tma_load_3d(uint32_t dst, const CUtensorMap* 
       "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
       : "memory");
 }
-__device__ __forceinline__ void um_fence_proxy_async() {
-  asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
-}
-__device__ __forceinline__ void um_fence_before() {
-  asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
-}
-__device__ __forceinline__ void um_fence_after() {
-  asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
-}
-
-__device__ __forceinline__ void um_mma(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
-      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(tmem_d),
-      "l"(adesc), "l"(bdesc), "r"(kUmIdesc), "r"(accumulate)
-      : "memory");
-}
-
-__device__ __forceinline__ void um_commit(uint64_t* bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(smem_u32(bar))
-               : "memory");
-}
-
-__device__ __forceinline__ void um_ld32(uint32_t taddr, float* v) {
-  uint32_t r[32];
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
-        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
-        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-      : "r"(taddr));
-#pragma unroll
-  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
-}
-
-__device__ __forceinline__ void um_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory"); }
-
 template <int NG>
 __global__ void __launch_bounds__(kUmThreads, 1) append_umma_kernel(AppendArgs a, int T,
                                                                      const __grid_constant__ CUtensorMap map_k,
@@ -477,7 +424,7 @@ __global__ void __launch_bounds__(kUmThreads, 1) append_umma_kernel(AppendArgs a
               for (int ks = 0; ks < 4; ++ks) {
                 const uint64_t ad = um_desc(abuf + (uint32_t)kb * kUmRegion + (uint32_t)ks * 32u);
                 const uint64_t bd = um_desc(sB + (uint32_t)(2 * pt + kb) * kUmRegion + (uint32_t)ks * 32u);
-                um_mma(dcol, ad, bd, step > 0 ? 1u : 0u);
+                um_mma(dcol, ad, bd, kUmIdesc, step > 0 ? 1u : 0u);
                 ++step;
               }
           um_commit(&mma_done[i & 1]);

@@ -25,6 +25,7 @@
 //   3. normalise and un-rotate: o = (o' / l) R_V^T per row.
 #include "okv_common.cuh"
 #include "okv_internal.h"
+#include "umma.cuh"
 
 namespace okv {
 namespace {
@@ -483,6 +484,531 @@ __global__ void __launch_bounds__(kPfWarps * 32) prefill_attn_kernel(PrefillArgs
 }
 
 // ---------------------------------------------------------------------------
+// 2b. attention on the tcgen05 tensor cores (128-channel groups).  A CTA takes
+// 128 query rows of one KV head (the MMA's M) and streams the key positions
+// in chunks of 64 (four cache blocks), with warp roles:
+//   warps 0-3  softmax: thread r owns row r, which is TMEM lane r.  Per chunk
+//              it reads its 64 scores from TMEM, applies the per-token scale
+//              and minimum term and the causal limit, keeps the online softmax
+//              state in registers, and writes p s (hi + lo fp16) as the A
+//              operand of the value MMA;
+//   warps 4-7  staging: the chunk's codes (or fp16 window / sink rows) into
+//              shared memory as fp16 tiles in the MMA's K-major layout --
+//              keys as [token][channel], values transposed to
+//              [channel][token] -- and the per-token (scale, min) pairs;
+//   warp 8     TMEM allocation; lane 0 issues the MMAs:
+//              S(c) = q~hi K^T + q~lo K^T (M 128, N 64, K 128) into one of
+//              two TMEM score buffers, O += (p s)hi V + (p s)lo V (M 128,
+//              N 128, K 64) into the TMEM output.
+// Two buffers of every per-chunk tile; mbarriers hand them around:
+//   kv_full   staging -> MMA, softmax  (a chunk's tiles are in shared memory)
+//   s_full    MMA -> softmax           (S(c) is in TMEM)
+//   s_free    softmax -> MMA           (S(c) was read; its buffer may take S(c + 2))
+//   p_full    softmax -> MMA           (p s of chunk c is in shared memory)
+//   pv_done   MMA -> all               (O includes chunk c; c's tiles are free)
+// The running maximum is lazy: a row rescales O (TMEM load, scale, store)
+// only when a chunk's maximum exceeds the one in use by more than tau, so p
+// stays below 2^tau; tau <= 8 is chosen per chunk so that p s stays inside
+// fp16 for the chunk's largest value scale.  Every wait is bounded; on a
+// timeout the kernel raises OKV_DEV_TIMEOUT, waits (bounded) for the MMAs it
+// issued, frees TMEM and returns.
+// ---------------------------------------------------------------------------
+constexpr int kUpKC = 64;        // key positions per chunk
+constexpr int kUpSmxWarps = 4;   // warps 0..3
+constexpr int kUpStgWarps = 4;   // warps 4..7
+constexpr int kUpMmaWarp = 8;
+constexpr int kUpThreads = 32 * (kUpSmxWarps + kUpStgWarps + 1);
+constexpr uint32_t kUpQBytes = 4 * 16384;  // q~ hi and lo, 2 K-blocks of 128 rows x 128 B each
+constexpr uint32_t kUpKBytes = 2 * 8192;   // a chunk's keys: 2 K-blocks of 64 rows x 128 B
+constexpr uint32_t kUpVBytes = 16384;      // a chunk's values: 128 channel rows x 64 tokens
+constexpr uint32_t kUpPBytes = 2 * 16384;  // a chunk's p s: hi, lo, 128 rows x 64 tokens each
+constexpr uint32_t kUpOffK = kUpQBytes;
+constexpr uint32_t kUpOffV = kUpOffK + 2 * kUpKBytes;
+constexpr uint32_t kUpOffP = kUpOffV + 2 * kUpVBytes;
+constexpr uint32_t kUpOffMisc = kUpOffP + 2 * kUpPBytes;
+struct UpMisc {
+  float2 ksm[2][kUpKC];             // key (scale, min) per token: (1, 0) for fp16 rows, (0, 0) masked
+  float2 vsm[2][kUpKC];             // value (scale, min)
+  int kval[2][kUpKC];               // 1 where the token was staged (only read when a block id was bad)
+  float vsmax[2][kUpStgWarps];      // largest value scale, per staging warp
+  int bad[2][kUpStgWarps];          // a block id was out of range, per staging warp
+  uint64_t kv_full[2], s_full[2], s_free[2], p_full[2], pv_done[2];
+  uint32_t tmem_slot;
+};
+constexpr size_t kUpSmem = 1024 + kUpOffMisc + sizeof(UpMisc);
+constexpr uint32_t kUpTmemCols = 256;  // scores: 2 x 64 columns; O: columns 128 .. 255
+constexpr uint32_t kUpIdescS = um_idesc(64, false, false);
+constexpr uint32_t kUpIdescO = um_idesc(128, false, false);
+constexpr uint32_t kF16Bias2 = 0x64006400u;  // (1024, 1024) as fp16 pair: 1024 + c is exact for c < 1024
+
+// (1024 + lo, 1024 + hi) - 1024 for two 2-bit codes already in bits 0-1 and 16-17
+__device__ __forceinline__ uint32_t codes_to_half2(uint32_t x) {
+  const uint32_t b = (x & 0x00030003u) | kF16Bias2, bias = kF16Bias2;
+  const __half2 h = __hsub2(*reinterpret_cast<const __half2*>(&b), *reinterpret_cast<const __half2*>(&bias));
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+// Value codes are staged centred, as 2 c - 3 (exact in fp16), with half the
+// scale: s c + m = (s / 2)(2 c - 3) + (m + 1.5 s).  The value sum then holds
+// terms of both signs, and the minimum term m + 1.5 s is the centre of the
+// token's range, so neither sum is a large number cancelling another.
+// (1024 + 2 lo, 1024 + 2 hi) - 1027 for two codes at bits 1-2 and 17-18 of x.
+constexpr uint32_t kF16Centre2 = 0x64036403u;  // (1027, 1027)
+__device__ __forceinline__ uint32_t centred_to_half2(uint32_t x) {
+  const uint32_t b = (x & 0x00060006u) | kF16Bias2, bias = kF16Centre2;
+  const __half2 h = __hsub2(*reinterpret_cast<const __half2*>(&b), *reinterpret_cast<const __half2*>(&bias));
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+// codes at bits 2k, 2k + 1 (and 16 higher) moved to bits 1-2 (17-18)
+template <int k>
+__device__ __forceinline__ uint32_t codes_at_bit1(uint32_t x) {
+  if constexpr (k == 0)
+    return x << 1;
+  else
+    return x >> (2 * k - 1);
+}
+
+// 16 consecutive-channel codes of one word (channel 4 b + k at bits 8 b + 2 k)
+// as 8 fp16 pairs of adjacent channels (centred: 2 c - 3)
+template <bool kCentred>
+__device__ __forceinline__ void word_to_half2x8(uint32_t w, uint32_t (&e)[8]) {
+  const uint32_t ev = w & 0x33333333u;         // channels 4 b, 4 b + 2 at bits 0-1, 4-5 of byte b
+  const uint32_t od = (w >> 2) & 0x33333333u;  // channels 4 b + 1, 4 b + 3
+#pragma unroll
+  for (int b = 0; b < 4; ++b) {
+    const uint32_t x = __byte_perm(ev, od, (uint32_t)(b | (b << 4) | ((4 + b) << 8) | ((4 + b) << 12)));
+    if constexpr (kCentred) {
+      e[2 * b] = centred_to_half2(x << 1);
+      e[2 * b + 1] = centred_to_half2(x >> 3);
+    } else {
+      e[2 * b] = codes_to_half2(x);
+      e[2 * b + 1] = codes_to_half2(x >> 4);
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kUpThreads, 1) prefill_umma_kernel(PrefillArgs a) {
+  extern __shared__ unsigned char up_raw[];
+  const uint32_t raw_u32 = smem_u32(up_raw);
+  const uint32_t base = (raw_u32 + 1023u) & ~1023u;  // swizzle atoms need 1024-byte alignment
+  unsigned char* gb = up_raw + (base - raw_u32);
+  UpMisc& ms = *reinterpret_cast<UpMisc*>(gb + kUpOffMisc);
+  const uint32_t sQ = base, sK = base + kUpOffK, sV = base + kUpOffV, sP = base + kUpOffP;
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int hk = blockIdx.y;
+  const int nrows = a.T * a.g;
+  const int row0 = blockIdx.x * 128;
+  const int last_row = min(nrows, row0 + 128) - 1;
+  const int pmax = a.first + last_row / a.g;  // last position any row of this CTA sees
+  const int nch = pmax / kUpKC + 1;
+  const int32_t* table = a.block_table + (size_t)a.slot * a.mbps;
+
+  if (tid == 0) {
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&ms.kv_full[i], 32 * kUpStgWarps);
+      mbar_init(&ms.s_full[i], 1);
+      mbar_init(&ms.s_free[i], 32 * kUpSmxWarps);
+      mbar_init(&ms.p_full[i], 32 * kUpSmxWarps);
+      mbar_init(&ms.pv_done[i], 1);
+    }
+    fence_mbar_init();
+  }
+  if (warp == kUpMmaWarp) um_alloc(&ms.tmem_slot, kUpTmemCols);
+
+  // ---- softmax rows: q~ halves into the A tiles, per-row constants
+  int rrow = 0, rpos = 0;
+  bool rok = false;
+  float qsum = 0.f, qup = 0.f;
+  if (warp < kUpSmxWarps) {
+    const int r = row0 + tid;
+    rok = r < nrows;
+    const int rr = rok ? r : nrows - 1;
+    const int rtok = rr / a.g;
+    rrow = rtok * a.hq + hk * a.g + rr % a.g;
+    rpos = a.first + rtok;
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      const uint4* src = reinterpret_cast<const uint4*>((half ? a.qlo : a.qhi) + (size_t)rrow * kD);
+#pragma unroll
+      for (int c16 = 0; c16 < 16; ++c16) {
+        const uint4 x = src[c16];
+        const uint32_t off = (uint32_t)(2 * half + (c16 >> 3)) * 16384u + um_swz((uint32_t)tid, (uint32_t)(c16 & 7) * 16u);
+        *reinterpret_cast<uint4*>(gb + off) = x;
+      }
+    }
+    const float* aux = a.qaux + (size_t)rrow * kQaux;
+    qsum = aux[0] * (kInvSqrtD * kLog2e);
+    qup = aux[4] * (kInvSqrtD * kLog2e);
+    um_fence_proxy_async();  // generic stores, read by the MMA through the async proxy
+  }
+
+  // ---- staging: per-thread roles and the register-held fetch of one chunk
+  const int stid = tid - 32 * kUpSmxWarps, sw = stid >> 5;
+  const int ktk = 16 * sw + (lane & 15), kkb = lane >> 4;      // key token, K-block (64 channels)
+  const int vtq = lane & 15, vbq = 2 * sw + (lane >> 4);       // value token quad, channel sixteen
+  int ksrc = 0, vsrc[4] = {0, 0, 0, 0}, sbad = 0;               // 0 masked, 1 INT2, 2 fp16
+  uint4 kr[8];
+  uint4 vw = make_uint4(0, 0, 0, 0), vh[4][2];
+  uint32_t ksmw = 0;
+  // block ids of this thread's key token and value quad, looked up one chunk
+  // before their codes are fetched (the table read and the code read would
+  // otherwise be two dependent memory latencies per chunk)
+  auto lookup = [&](int c, int& kblk, int& vblk) {
+    const int pk = kUpKC * c + ktk, pv = kUpKC * c + 4 * vtq;
+    kblk = (c < nch && pk <= pmax && pk < a.L) ? table[pk >> 4] : -1;
+    vblk = (c < nch && pv <= pmax && pv < a.L) ? table[pv >> 4] : -1;
+  };
+  int kblk_n = -1, vblk_n = -1;  // block ids of the next chunk to fetch
+  // key position p: 1 INT2 (block-head base in *bp), 2 fp16 (row in *hp), 0 masked
+  auto locate = [&](int p, int blk, int kind, const uint8_t** bp, const __half** hp) -> int {
+    if (p > pmax || p >= a.L) return 0;
+    if (p < a.nsink || p >= a.L - kWin) {
+      const bool sink = p < a.nsink;
+      const size_t rows = sink ? (size_t)a.nsink : (size_t)kWin;
+      const size_t row = sink ? (size_t)p : (size_t)(p % kWin);
+      *hp = (sink ? a.sink : a.ring) + ((((size_t)a.slot * a.hkv + hk) * 2 + kind) * rows + row) * kD;
+      return 2;
+    }
+    if (blk < 0 || blk >= a.num_blocks) {
+      if (!sbad) raise_flag(a.status, OKV_DEV_BAD_BLOCK);
+      sbad = 1;
+      return 0;
+    }
+    *bp = a.pages + ((size_t)blk * a.hkv + hk) * a.bhb;
+    return 1;
+  };
+  auto fetch = [&](int c, int kblk, int vblk) {
+    const int p0 = kUpKC * c;
+    {
+      const uint8_t* bp = nullptr;
+      const __half* hp = nullptr;
+      const int p = p0 + ktk;
+      ksrc = locate(p, kblk, 0, &bp, &hp);
+      if (ksrc == 1) {
+        kr[0] = *reinterpret_cast<const uint4*>(bp + kKcOff + (p & 15) * 32 + 16 * kkb);
+        ksmw = *reinterpret_cast<const uint32_t*>(bp + sm_offset(1, kkb, p & 15, 0));
+      } else if (ksrc == 2) {
+        const uint4* x = reinterpret_cast<const uint4*>(hp + 64 * kkb);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) kr[j] = x[j];
+      }
+    }
+    {
+      const uint8_t* bp = nullptr;
+      bool any_int2 = false;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const __half* hp = nullptr;
+        const uint8_t* bpi = nullptr;
+        vsrc[i] = locate(p0 + 4 * vtq + i, vblk, 1, &bpi, &hp);
+        if (vsrc[i] == 1) {
+          bp = bpi;
+          any_int2 = true;
+        } else if (vsrc[i] == 2) {
+          const uint4* x = reinterpret_cast<const uint4*>(hp + 16 * vbq);
+          vh[i][0] = x[0];
+          vh[i][1] = x[1];
+        }
+      }
+      if (any_int2) vw = *reinterpret_cast<const uint4*>(bp + kVcOff + ((vbq * 4 + ((p0 + 4 * vtq) & 15) / 4) << 4));
+    }
+  };
+  auto stage = [&](int b) {
+    // keys: 8 chunks of 8 channels into row ktk of K-block kkb
+    const uint32_t kdst = sK + (uint32_t)b * kUpKBytes + (uint32_t)kkb * 8192u;
+    unsigned char* kg = gb + (kdst - base);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      uint32_t e[8];
+      const uint32_t w = i == 0 ? kr[0].x : i == 1 ? kr[0].y : i == 2 ? kr[0].z : kr[0].w;
+      word_to_half2x8<false>(w, e);
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const int jc = 2 * i + hh;
+        uint4 v = ksrc == 1 ? make_uint4(e[4 * hh], e[4 * hh + 1], e[4 * hh + 2], e[4 * hh + 3])
+                            : ksrc == 2 ? kr[jc] : make_uint4(0, 0, 0, 0);
+        *reinterpret_cast<uint4*>(kg + um_swz((uint32_t)ktk, (uint32_t)jc * 16u)) = v;
+      }
+    }
+    float s_ = 0.f, m_ = 0.f;
+    if (ksrc == 1) {
+      s_ = __half2float(__ushort_as_half((unsigned short)(ksmw & 0xffffu)));
+      m_ = __half2float(__ushort_as_half((unsigned short)(ksmw >> 16)));
+    } else if (ksrc == 2) {
+      s_ = 1.f;
+    }
+    if (kkb == 0) {
+      ms.ksm[b][ktk] = make_float2(s_, m_);
+      ms.kval[b][ktk] = ksrc != 0;
+    } else if (ksrc == 1) {
+      ms.vsm[b][ktk] = make_float2(0.5f * s_, fmaf(1.5f, s_, m_));  // centred codes
+      s_ *= 0.5f;
+    } else {
+      ms.vsm[b][ktk] = make_float2(s_, m_);
+    }
+    float vmx = kkb == 1 ? s_ : 0.f;
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) vmx = fmaxf(vmx, __shfl_xor_sync(0xffffffffu, vmx, o));
+    const int anybad = __any_sync(0xffffffffu, sbad != 0);
+    if (lane == 0) {
+      ms.vsmax[b][sw] = vmx;
+      ms.bad[b][sw] = anybad;
+    }
+    sbad = 0;
+    // values: channels 16 vbq + ch, token pairs (2 vtq + s): one 32-bit word per (channel, pair)
+    uint32_t pr[16][2];
+    if (vsrc[0] == 1 && vsrc[1] == 1 && vsrc[2] == 1 && vsrc[3] == 1) {
+      const uint32_t ws[4] = {vw.x, vw.y, vw.z, vw.w};  // word b': channels 4 b' .. + 3 of tokens 0..3
+#pragma unroll
+      for (int bb = 0; bb < 4; ++bb) {
+        const uint32_t x01 = __byte_perm(ws[bb], 0u, 0x0110u);  // tokens 0, 1 in bytes 0, 2
+        const uint32_t x23 = __byte_perm(ws[bb], 0u, 0x0302u);  // tokens 2, 3
+        pr[4 * bb + 0][0] = centred_to_half2(codes_at_bit1<0>(x01));
+        pr[4 * bb + 0][1] = centred_to_half2(codes_at_bit1<0>(x23));
+        pr[4 * bb + 1][0] = centred_to_half2(codes_at_bit1<1>(x01));
+        pr[4 * bb + 1][1] = centred_to_half2(codes_at_bit1<1>(x23));
+        pr[4 * bb + 2][0] = centred_to_half2(codes_at_bit1<2>(x01));
+        pr[4 * bb + 2][1] = centred_to_half2(codes_at_bit1<2>(x23));
+        pr[4 * bb + 3][0] = centred_to_half2(codes_at_bit1<3>(x01));
+        pr[4 * bb + 3][1] = centred_to_half2(codes_at_bit1<3>(x23));
+      }
+    } else {
+      uint32_t e[4][8];  // per token: fp16 pairs of adjacent channels
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        if (vsrc[i] == 1) {
+          const uint32_t sel = (uint32_t)(i | ((4 + i) << 4));
+          const uint32_t t01 = __byte_perm(vw.x, vw.y, sel), t23 = __byte_perm(vw.z, vw.w, sel);
+          word_to_half2x8<true>(__byte_perm(t01, t23, 0x5410u), e[i]);
+        } else if (vsrc[i] == 2) {
+          e[i][0] = vh[i][0].x; e[i][1] = vh[i][0].y; e[i][2] = vh[i][0].z; e[i][3] = vh[i][0].w;
+          e[i][4] = vh[i][1].x; e[i][5] = vh[i][1].y; e[i][6] = vh[i][1].z; e[i][7] = vh[i][1].w;
+        } else {
+#pragma unroll
+          for (int j = 0; j < 8; ++j) e[i][j] = 0u;
+        }
+      }
+#pragma unroll
+      for (int ch = 0; ch < 16; ++ch) {
+        const uint32_t sel = (ch & 1) ? 0x7632u : 0x5410u;
+        pr[ch][0] = __byte_perm(e[0][ch >> 1], e[1][ch >> 1], sel);
+        pr[ch][1] = __byte_perm(e[2][ch >> 1], e[3][ch >> 1], sel);
+      }
+    }
+    // lanes 16..31 write rows 16 apart from lanes 0..15 (same swizzle phase):
+    // they take the other token pair first, so each store covers 32 banks
+    const int flip = lane >> 4;
+    unsigned char* vg = gb + (sV + (uint32_t)b * kUpVBytes - base);
+#pragma unroll
+    for (int ch = 0; ch < 16; ++ch)
+#pragma unroll
+      for (int s0 = 0; s0 < 2; ++s0) {
+        const int s = s0 ^ flip;
+        const uint32_t v = flip ? pr[ch][s0 ^ 1] : pr[ch][s0];
+        *reinterpret_cast<uint32_t*>(vg + um_swz((uint32_t)(16 * vbq + ch), (uint32_t)(2 * vtq + s) * 4u)) = v;
+      }
+  };
+  if (warp >= kUpSmxWarps && warp < kUpMmaWarp) {
+    int kb0, vb0;
+    lookup(0, kb0, vb0);
+    fetch(0, kb0, vb0);
+    lookup(1, kblk_n, vblk_n);
+  }
+
+  um_fence_before();
+  __syncthreads();
+  um_fence_after();
+  const uint32_t tmem = ms.tmem_slot;
+  const uint32_t tS = tmem, tO = tmem + 128u;
+
+  if (warp < kUpSmxWarps) {
+    // ------------------------------------------------------------ softmax
+    const uint32_t lane_base = (uint32_t)(32 * warp) << 16;
+    float m_use = -INFINITY, l = 0.f, msum = 0.f;
+    bool alive = true;
+    for (int c = 0; c < nch && alive; ++c) {
+      const int b = c & 1;
+      const uint32_t ph = ((uint32_t)c >> 1) & 1u;
+      alive = mbar_wait_bounded(&ms.kv_full[b], ph) && mbar_wait_bounded(&ms.s_full[b], ph);
+      alive = __all_sync(0xffffffffu, alive);
+      if (!alive) break;
+      um_fence_after();
+      float sv[kUpKC];
+      um_ld32(tS + lane_base + (uint32_t)(b * kUpKC), sv);
+      um_ld32(tS + lane_base + (uint32_t)(b * kUpKC + 32), sv + 32);
+      um_wait_ld();
+      um_fence_before();
+      mbar_arrive(&ms.s_free[b]);
+      const int lim = min(rpos + 1, a.L) - kUpKC * c;  // tokens j < lim are causal and in the sequence
+      const bool bad = (ms.bad[b][0] | ms.bad[b][1] | ms.bad[b][2] | ms.bad[b][3]) != 0;
+      float bm = -INFINITY;
+#pragma unroll
+      for (int j = 0; j < kUpKC; ++j) {
+        const float2 ks = ms.ksm[b][j];
+        const float x = fmaf(ks.x * qup, sv[j], ks.y * qsum);
+        const bool ok = j < lim && (!bad || ms.kval[b][j] != 0);
+        sv[j] = ok ? x : -INFINITY;
+        bm = fmaxf(bm, sv[j]);
+      }
+      // tau: p < 2^tau and p s < 2^15 for the chunk's largest value scale
+      const float vmax = fmaxf(fmaxf(ms.vsmax[b][0], ms.vsmax[b][1]), fmaxf(ms.vsmax[b][2], ms.vsmax[b][3]));
+      const int ex = vmax > 0.f ? ((__float_as_int(vmax) >> 23) & 0xff) - 127 : 0;
+      const float tau = (float)max(0, min(8, 14 - ex));
+      const bool need = bm > m_use + tau;
+      if (__any_sync(0xffffffffu, need)) {
+        const float alpha = need ? exp2f(m_use - bm) : 1.f;  // 0 while the row has seen nothing
+        if (c > 0) {
+          // O must hold chunk c - 1 before it is scaled
+          alive = mbar_wait_bounded(&ms.pv_done[(c - 1) & 1], ((uint32_t)(c - 1) >> 1) & 1u);
+          alive = __all_sync(0xffffffffu, alive);
+          if (!alive) break;
+          um_fence_after();
+#pragma unroll 1
+          for (int q = 0; q < 4; ++q) {
+            float ov[32];
+            um_ld32(tO + lane_base + 32u * q, ov);
+            um_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) ov[i] *= alpha;
+            um_st32(tO + lane_base + 32u * q, ov);
+          }
+          um_wait_st();
+        }
+        l *= alpha;
+        msum *= alpha;
+        if (need) m_use = bm;
+      }
+      const float mref = m_use == -INFINITY ? 0.f : m_use;
+      // p s into the A tiles of chunk c, once the value MMA of chunk c - 2 has read them
+      if (c >= 2) {
+        alive = mbar_wait_bounded(&ms.pv_done[b], ((uint32_t)(c - 2) >> 1) & 1u);
+        alive = __all_sync(0xffffffffu, alive);
+        if (!alive) break;
+      }
+      unsigned char* pg = gb + (sP + (uint32_t)b * kUpPBytes - base);
+#pragma unroll
+      for (int j8 = 0; j8 < kUpKC / 8; ++j8) {
+        uint32_t hi[4], lo[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int j = 8 * j8 + 2 * u;
+          const float p0 = exp2f(sv[j] - mref), p1 = exp2f(sv[j + 1] - mref);
+          const float4 vs = *reinterpret_cast<const float4*>(&ms.vsm[b][j]);  // (s, m) of j and j + 1
+          l += p0 + p1;
+          msum = fmaf(p0, vs.y, fmaf(p1, vs.w, msum));
+          split_half2(p0 * vs.x, p1 * vs.z, hi[u], lo[u]);
+        }
+        const uint32_t off = um_swz((uint32_t)tid, (uint32_t)j8 * 16u);
+        *reinterpret_cast<uint4*>(pg + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+        *reinterpret_cast<uint4*>(pg + 16384u + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+      }
+      um_fence_proxy_async();
+      um_fence_before();
+      mbar_arrive(&ms.p_full[b]);
+    }
+    if (alive) {
+      alive = mbar_wait_bounded(&ms.pv_done[(nch - 1) & 1], ((uint32_t)(nch - 1) >> 1) & 1u);
+      alive = __all_sync(0xffffffffu, alive);
+    }
+    if (alive) {
+      um_fence_after();
+      float* dst = a.obuf + (size_t)rrow * kOStride;
+#pragma unroll 1
+      for (int q = 0; q < 4; ++q) {
+        float ov[32];
+        um_ld32(tO + lane_base + 32u * q, ov);
+        um_wait_ld();
+        if (rok) {
+#pragma unroll
+          for (int i = 0; i < 32; i += 4)
+            *reinterpret_cast<float4*>(dst + 32 * q + i) =
+                make_float4(ov[i] + msum, ov[i + 1] + msum, ov[i + 2] + msum, ov[i + 3] + msum);
+        }
+      }
+      if (rok) dst[128] = l;
+    } else if (lane == 0) {
+      raise_flag(a.status, OKV_DEV_TIMEOUT);
+    }
+  } else if (warp < kUpMmaWarp) {
+    // ------------------------------------------------------------ staging
+    for (int c = 0; c < nch; ++c) {
+      const int b = c & 1;
+      if (c >= 2 && !mbar_wait_bounded(&ms.pv_done[b], ((uint32_t)(c - 2) >> 1) & 1u)) {
+        raise_flag(a.status, OKV_DEV_TIMEOUT);
+        break;
+      }
+      stage(b);
+      um_fence_proxy_async();
+      mbar_arrive(&ms.kv_full[b]);
+      if (c + 1 < nch) {
+        fetch(c + 1, kblk_n, vblk_n);
+        lookup(c + 2, kblk_n, vblk_n);
+      }
+    }
+  } else if (lane == 0) {
+    // ------------------------------------------------------------ MMA issue
+    // order: S(0), S(1), then per chunk c: O += P(c) V(c) as soon as the
+    // softmax of c is done, then S(c + 2) once its keys are staged (which
+    // needs the value MMA of c, the previous user of their buffer)
+    uint64_t* last_bar = nullptr;  // the latest commit: it completes after every MMA issued before it
+    uint32_t last_par = 0;
+    auto issue_s = [&](int c) -> bool {
+      const int b = c & 1;
+      if (!mbar_wait_bounded(&ms.kv_full[b], ((uint32_t)c >> 1) & 1u)) return false;
+      if (c >= 2 && !mbar_wait_bounded(&ms.s_free[b], ((uint32_t)(c - 2) >> 1) & 1u)) return false;
+      um_fence_after();
+      const uint32_t kt = sK + (uint32_t)b * kUpKBytes;
+#pragma unroll
+      for (int half = 0; half < 2; ++half)
+#pragma unroll
+        for (int kb = 0; kb < 2; ++kb)
+#pragma unroll
+          for (int ks = 0; ks < 4; ++ks) {
+            const uint64_t ad = um_desc(sQ + (uint32_t)(2 * half + kb) * 16384u + (uint32_t)ks * 32u);
+            const uint64_t bd = um_desc(kt + (uint32_t)kb * 8192u + (uint32_t)ks * 32u);
+            um_mma(tS + (uint32_t)(b * kUpKC), ad, bd, kUpIdescS, (half | kb | ks) != 0 ? 1u : 0u);
+          }
+      um_commit(&ms.s_full[b]);
+      last_bar = &ms.s_full[b];
+      last_par = ((uint32_t)c >> 1) & 1u;
+      return true;
+    };
+    auto issue_pv = [&](int c) -> bool {
+      const int b = c & 1;
+      if (!mbar_wait_bounded(&ms.p_full[b], ((uint32_t)c >> 1) & 1u)) return false;
+      um_fence_after();
+      const uint32_t pt = sP + (uint32_t)b * kUpPBytes, vt2 = sV + (uint32_t)b * kUpVBytes;
+#pragma unroll
+      for (int half = 0; half < 2; ++half)
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks) {
+          const uint64_t ad = um_desc(pt + (uint32_t)half * 16384u + (uint32_t)ks * 32u);
+          const uint64_t bd = um_desc(vt2 + (uint32_t)ks * 32u);
+          um_mma(tO, ad, bd, kUpIdescO, (c > 0 || half > 0 || ks > 0) ? 1u : 0u);
+        }
+      um_commit(&ms.pv_done[b]);
+      last_bar = &ms.pv_done[b];
+      last_par = ((uint32_t)c >> 1) & 1u;
+      return true;
+    };
+    bool alive = issue_s(0) && (nch < 2 || issue_s(1));
+    for (int c = 0; c < nch && alive; ++c) alive = issue_pv(c) && (c + 2 >= nch || issue_s(c + 2));
+    if (!alive) {
+      raise_flag(a.status, OKV_DEV_TIMEOUT);
+      // the MMAs already issued finish before TMEM is freed: the last commit covers them all
+      if (last_bar != nullptr) mbar_wait_bounded(last_bar, last_par);
+    }
+  }
+  um_fence_before();
+  __syncthreads();
+  if (warp == kUpMmaWarp) {
+    um_fence_after();
+    um_dealloc(tmem, kUpTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------------------
 // 3. o = (o' / l) R_V^T.  One CTA per (query head, 16 query tokens): U_V of
 // the head's KV head is staged in shared memory once, then warp w takes
 // tokens w and w + 8: un-permute and butterfly in registers, and the U_V^T
@@ -590,7 +1116,13 @@ okv_status launch_prefill(const okv_cache_desc* d, const void* q, int T, int slo
   if (st != OKV_OK) return st;
   const dim3 grid((unsigned)((T * a.g + kPfRows - 1) / kPfRows), (unsigned)a.hkv);
   switch (a.ng) {
-    case 1: prefill_attn_kernel<1><<<grid, kPfWarps * 32, 0, s>>>(a); break;
+    case 1: {
+      static std::atomic<uint32_t> up_attr{0};
+      cudaError_t e1 = set_smem_limit_once((const void*)prefill_umma_kernel, (int)kUpSmem, up_attr);
+      if (e1 != cudaSuccess) return fail(OKV_ERR_CUDA, "prefill attention smem attribute: %s", cudaGetErrorString(e1));
+      prefill_umma_kernel<<<grid, kUpThreads, kUpSmem, s>>>(a);
+      break;
+    }
     case 2: prefill_attn_kernel<2><<<grid, kPfWarps * 32, 0, s>>>(a); break;
     default: prefill_attn_kernel<4><<<grid, kPfWarps * 32, 0, s>>>(a); break;
   }

@@ -391,7 +391,7 @@ def decode(cache: Cache, q: np.ndarray, seq_slots, context_lens, hq: int) -> np.
     return out
 
 
-def prefill(cache: Cache, q: np.ndarray, slot: int, context_len: int, hq: int) -> np.ndarray:
+def prefill(cache: Cache, q: np.ndarray, slot: int, context_len: int, hq: int, tokens=None) -> np.ndarray:
     """Attention of a prefill chunk over the cache, causal.
 
     The chunk's T tokens have been appended, so the sequence in `slot` has
@@ -402,6 +402,8 @@ def prefill(cache: Cache, q: np.ndarray, slot: int, context_len: int, hq: int) -
     last W positions from fp16, the rest from INT2: `Cache.values`), with
     q rotated by R_K and the output brought back with R_V^T, as in `decode`.
     Returns fp64 [T, hq, d].  With T = 1 this is `decode` of that sequence.
+    `tokens` (optional) lists the chunk indices i to compute; the other rows
+    stay zero (a sample of a large chunk, the arithmetic unchanged).
     [AF] "OSCAR: figyelem-tudatos…" and [GH] "Что это даёт на практике"
     (the cache serves paged attention and prefix caching, so prefill chunks
     attend over the compressed history); [GH] "Что придумали в Together AI"
@@ -419,7 +421,7 @@ def prefill(cache: Cache, q: np.ndarray, slot: int, context_len: int, hq: int) -
         kx = cache.values(slot, 0, hk, context_len)
         vx = cache.values(slot, 1, hk, context_len)
         for h in range(hk * g, (hk + 1) * g):
-            for i in range(T):
+            for i in (range(T) if tokens is None else tokens):
                 visible = first + i + 1
                 qr = np.asarray(q[i, h], dtype=np.float64) @ cache.r[0][hk]
                 out[i, h] = attend(qr, kx[:visible], vx[:visible]) @ cache.r[1][hk].T

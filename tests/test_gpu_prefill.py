@@ -37,7 +37,7 @@ def _t(x, dtype=None):
     return t.cuda()
 
 
-def _case(seed, hq, hkv, L, T, group=128, sinks=0, checked=None, scale=1.0):
+def _case(seed, hq, hkv, L, T, group=128, sinks=0, checked=None, scale=1.0, vscale=1.0, tokens=None):
     """One sequence of L tokens (pre-rotated fill, identical on both sides);
     the last T are the chunk.  Returns (got, {hk: want}) for the checked KV heads."""
     okv = _okv()
@@ -45,7 +45,7 @@ def _case(seed, hq, hkv, L, T, group=128, sinks=0, checked=None, scale=1.0):
     uk, uv = H.rotations(seed, hkv)
     gc = okv.Cache(hq, hkv, lay.num_blocks, 1, lay.mbps, uk, uv, group=group, num_sink=sinks)
     zk = np.stack([WL.sample_rotated(seed, 0, 0, h, L, 0, scale=scale) for h in range(hkv)], 1)
-    zv = np.stack([WL.sample_rotated(seed, 0, 0, h, L, 1) for h in range(hkv)], 1)
+    zv = np.stack([WL.sample_rotated(seed, 0, 0, h, L, 1, scale=vscale) for h in range(hkv)], 1)
     slots, pos = lay.flat()
     okv.append_quantize(gc, _t(zk), _t(zv), _t(slots), _t(pos), _t(lay.table), _t(np.array([L], np.int32)),
                         pre_rotated=True)
@@ -58,7 +58,10 @@ def _case(seed, hq, hkv, L, T, group=128, sinks=0, checked=None, scale=1.0):
         oc = O.Cache(1, uk[hk:hk + 1].astype(np.float64), uv[hk:hk + 1].astype(np.float64), group=group,
                      sinks=sinks)
         oc.append(0, 0, zk[:, hk:hk + 1], zv[:, hk:hk + 1], pre_rotated=True)
-        want[hk] = O.prefill(oc, q[:, hk * G:(hk + 1) * G], 0, L, G)
+        want[hk] = O.prefill(oc, q[:, hk * G:(hk + 1) * G], 0, L, G, tokens=tokens)
+    if tokens is not None:
+        got = got[list(tokens)]
+        want = {hk: w[list(tokens)] for hk, w in want.items()}
     return got, want, G
 
 
@@ -95,6 +98,29 @@ def test_prefill_with_sinks():
 def test_prefill_large_logits():
     """Rotated keys in the hundreds: peaked softmax rows."""
     got, want, G = _case(54, 8, 2, 1200, 64, scale=30.0)
+    _check(got, want, G)
+
+
+@pytest.mark.parametrize("vscale", [300.0, 8000.0])
+def test_prefill_large_value_scales(vscale):
+    """Value scales near the top of fp16: the weight the value MMA takes
+    (p times the value scale, fp16 hi + lo) must stay in range, so the
+    tensor-core kernel re-bases its running maximum more often."""
+    got, want, G = _case(57, 8, 2, 1500, 100, vscale=vscale)
+    _check(got, want, G)
+
+
+def test_prefill_many_ctas():
+    """8,192-token context, 256-token chunk at the 32 / 8 head shape: eight
+    128-row tiles per KV head, 128 key chunks each."""
+    got, want, G = _case(58, 32, 8, 8192, 256, checked=[0, 7])
+    _check(got, want, G)
+
+
+def test_prefill_benchmark_shape_sampled():
+    """The prefill benchmark's shape: a 1,024-token chunk ending a 32,768-token
+    sequence, 32 query / 8 KV heads; sampled chunk tokens of two KV heads."""
+    got, want, G = _case(59, 32, 8, 32768, 1024, checked=[0, 5], tokens=[0, 1, 255, 640, 1022, 1023])
     _check(got, want, G)
 
 

@@ -558,6 +558,10 @@ def test_prefill_matches_loop_brute_force(sinks):
                                       lambda p: cache.entry(0, 0, hk, p), lambda p: cache.entry(0, 1, hk, p),
                                       L, 8, L - T + i, sinks)
             assert np.abs(got[i, h] - want).max() < 1e-10 * max(1.0, np.abs(want).max())
+    # a sample of the chunk's tokens: the same rows, the rest zero
+    part = O.prefill(cache, q, 0, L, hq=4, tokens=[0, 4, 8])
+    assert np.array_equal(part[[0, 4, 8]], got[[0, 4, 8]])
+    assert not part[[1, 2, 3, 5, 6, 7]].any()
 
 
 def test_prefill_of_one_token_is_decode():
