@@ -487,25 +487,30 @@ __global__ void __launch_bounds__(kPfWarps * 32) prefill_attn_kernel(PrefillArgs
 // 2b. attention on the tcgen05 tensor cores (128-channel groups).  A CTA takes
 // 128 query rows of one KV head (the MMA's M) and streams the key positions
 // in chunks of 64 (four cache blocks), with warp roles:
-//   warps 0-3  softmax: thread r owns row r, which is TMEM lane r.  Per chunk
-//              it reads its 64 scores from TMEM, applies the per-token scale
-//              and minimum term and the causal limit, keeps the online softmax
-//              state in registers, and writes p s (hi + lo fp16) as the A
-//              operand of the value MMA;
-//   warps 4-7  staging: the chunk's codes (or fp16 window / sink rows) into
+//   warps 0-7  softmax: warp w serves rows 32 (w % 4) .. + 31 (TMEM lanes,
+//              one row per thread) and score columns 32 (w / 4) .. + 31 of
+//              the chunk.  Per chunk a thread reads its 32 scores from TMEM,
+//              applies the per-token scale and minimum term and the causal
+//              limit, meets its partner (the other half of the row) for the
+//              row maximum, keeps the online softmax state in registers, and
+//              writes p s (hi + lo fp16) as the A operand of the value MMA;
+//   warps 8-11 staging: the chunk's codes (or fp16 window / sink rows) into
 //              shared memory as fp16 tiles in the MMA's K-major layout --
 //              keys as [token][channel], values transposed to
 //              [channel][token] -- and the per-token (scale, min) pairs;
-//   warp 8     TMEM allocation; lane 0 issues the MMAs:
+//   warp 12    TMEM allocation; lane 0 issues the MMAs:
 //              S(c) = q~hi K^T + q~lo K^T (M 128, N 64, K 128) into one of
 //              two TMEM score buffers, O += (p s)hi V + (p s)lo V (M 128,
 //              N 128, K 64) into the TMEM output.
 // Two buffers of every per-chunk tile; mbarriers hand them around:
-//   kv_full   staging -> MMA, softmax  (a chunk's tiles are in shared memory)
+//   k_full    staging -> MMA, softmax  (a chunk's key tile and key scales are in place)
+//   v_full    staging -> MMA, softmax  (its value tile and value scales)
 //   s_full    MMA -> softmax           (S(c) is in TMEM)
-//   s_free    softmax -> MMA           (S(c) was read; its buffer may take S(c + 2))
+//   s_free    softmax -> MMA, staging  (S(c) and the key scales were read: the score
+//                                       buffer and the key tile may take chunk c + 2)
 //   p_full    softmax -> MMA           (p s of chunk c is in shared memory)
-//   pv_done   MMA -> all               (O includes chunk c; c's tiles are free)
+//   pv_done   MMA -> all               (O includes chunk c; its value tile and p s are free)
+//   mx        softmax partners         (both halves of the rows posted their maximum)
 // The running maximum is lazy: a row rescales O (TMEM load, scale, store)
 // only when a chunk's maximum exceeds the one in use by more than tau, so p
 // stays below 2^tau; tau <= 8 is chosen per chunk so that p s stays inside
@@ -514,9 +519,9 @@ __global__ void __launch_bounds__(kPfWarps * 32) prefill_attn_kernel(PrefillArgs
 // issued, frees TMEM and returns.
 // ---------------------------------------------------------------------------
 constexpr int kUpKC = 64;        // key positions per chunk
-constexpr int kUpSmxWarps = 4;   // warps 0..3
-constexpr int kUpStgWarps = 4;   // warps 4..7
-constexpr int kUpMmaWarp = 8;
+constexpr int kUpSmxWarps = 8;   // warps 0..7
+constexpr int kUpStgWarps = 4;   // warps 8..11
+constexpr int kUpMmaWarp = 12;
 constexpr int kUpThreads = 32 * (kUpSmxWarps + kUpStgWarps + 1);
 constexpr uint32_t kUpQBytes = 4 * 16384;  // q~ hi and lo, 2 K-blocks of 128 rows x 128 B each
 constexpr uint32_t kUpKBytes = 2 * 8192;   // a chunk's keys: 2 K-blocks of 64 rows x 128 B
@@ -532,7 +537,9 @@ struct UpMisc {
   int kval[2][kUpKC];               // 1 where the token was staged (only read when a block id was bad)
   float vsmax[2][kUpStgWarps];      // largest value scale, per staging warp
   int bad[2][kUpStgWarps];          // a block id was out of range, per staging warp
-  uint64_t kv_full[2], s_full[2], s_free[2], p_full[2], pv_done[2];
+  float red[2][2][128];             // per chunk parity, column half, row: the half-row maximum
+  float2 fin[2][128];               // per column half, row: (l, sum p m) at the end
+  uint64_t k_full[2], v_full[2], s_full[2], s_free[2], p_full[2], pv_done[2], mx[4][2];
   uint32_t tmem_slot;
 };
 constexpr size_t kUpSmem = 1024 + kUpOffMisc + sizeof(UpMisc);
@@ -587,6 +594,13 @@ __device__ __forceinline__ void word_to_half2x8(uint32_t w, uint32_t (&e)[8]) {
   }
 }
 
+// 2^x by the SFU's approximate exponent (PTX ex2.approx.ftz.f32); -inf gives +0
+__device__ __forceinline__ float ex2_ftz(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 __global__ void __launch_bounds__(kUpThreads, 1) prefill_umma_kernel(PrefillArgs a) {
   extern __shared__ unsigned char up_raw[];
   const uint32_t raw_u32 = smem_u32(up_raw);
@@ -606,11 +620,13 @@ __global__ void __launch_bounds__(kUpThreads, 1) prefill_umma_kernel(PrefillArgs
 
   if (tid == 0) {
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&ms.kv_full[i], 32 * kUpStgWarps);
+      mbar_init(&ms.k_full[i], 32 * kUpStgWarps);
+      mbar_init(&ms.v_full[i], 32 * kUpStgWarps);
       mbar_init(&ms.s_full[i], 1);
       mbar_init(&ms.s_free[i], 32 * kUpSmxWarps);
       mbar_init(&ms.p_full[i], 32 * kUpSmxWarps);
       mbar_init(&ms.pv_done[i], 1);
+      for (int q = 0; q < 4; ++q) mbar_init(&ms.mx[q][i], 64);
     }
     fence_mbar_init();
   }
@@ -620,20 +636,22 @@ __global__ void __launch_bounds__(kUpThreads, 1) prefill_umma_kernel(PrefillArgs
   int rrow = 0, rpos = 0;
   bool rok = false;
   float qsum = 0.f, qup = 0.f;
+  const int quarter = warp & 3, hcol = (warp >> 2) & 1;  // softmax: lane quarter, column half
+  const int rowc = 32 * quarter + lane;                    // softmax: row in the tile (TMEM lane)
   if (warp < kUpSmxWarps) {
-    const int r = row0 + tid;
+    const int r = row0 + rowc;
     rok = r < nrows;
     const int rr = rok ? r : nrows - 1;
     const int rtok = rr / a.g;
     rrow = rtok * a.hq + hk * a.g + rr % a.g;
     rpos = a.first + rtok;
-#pragma unroll
-    for (int half = 0; half < 2; ++half) {
-      const uint4* src = reinterpret_cast<const uint4*>((half ? a.qlo : a.qhi) + (size_t)rrow * kD);
+    {  // column half 0 stages the row's hi half of q~, half 1 the lo half
+      const uint4* src = reinterpret_cast<const uint4*>((hcol ? a.qlo : a.qhi) + (size_t)rrow * kD);
 #pragma unroll
       for (int c16 = 0; c16 < 16; ++c16) {
         const uint4 x = src[c16];
-        const uint32_t off = (uint32_t)(2 * half + (c16 >> 3)) * 16384u + um_swz((uint32_t)tid, (uint32_t)(c16 & 7) * 16u);
+        const uint32_t off =
+            (uint32_t)(2 * hcol + (c16 >> 3)) * 16384u + um_swz((uint32_t)rowc, (uint32_t)(c16 & 7) * 16u);
         *reinterpret_cast<uint4*>(gb + off) = x;
       }
     }
@@ -648,8 +666,9 @@ __global__ void __launch_bounds__(kUpThreads, 1) prefill_umma_kernel(PrefillArgs
   const int ktk = 16 * sw + (lane & 15), kkb = lane >> 4;      // key token, K-block (64 channels)
   const int vtq = lane & 15, vbq = 2 * sw + (lane >> 4);       // value token quad, channel sixteen
   int ksrc = 0, vsrc[4] = {0, 0, 0, 0}, sbad = 0;               // 0 masked, 1 INT2, 2 fp16
-  uint4 kr[8];
-  uint4 vw = make_uint4(0, 0, 0, 0), vh[4][2];
+  uint4 kr0 = make_uint4(0, 0, 0, 0);  // INT2 key codes of the fetched token (64 channels)
+  uint4 vw = make_uint4(0, 0, 0, 0);   // INT2 value codes of the fetched quad (16 channels x 4 tokens)
+  int fetched_p0 = 0;                  // first position of the fetched chunk
   uint32_t ksmw = 0;
   // block ids of this thread's key token and value quad, looked up one chunk
   // before their codes are fetched (the table read and the code read would
@@ -660,16 +679,17 @@ __global__ void __launch_bounds__(kUpThreads, 1) prefill_umma_kernel(PrefillArgs
     vblk = (c < nch && pv <= pmax && pv < a.L) ? table[pv >> 4] : -1;
   };
   int kblk_n = -1, vblk_n = -1;  // block ids of the next chunk to fetch
-  // key position p: 1 INT2 (block-head base in *bp), 2 fp16 (row in *hp), 0 masked
-  auto locate = [&](int p, int blk, int kind, const uint8_t** bp, const __half** hp) -> int {
+  // the fp16 row (sink or window ring) of position p
+  auto fp16_row = [&](int p, int kind) -> const __half* {
+    const bool sink = p < a.nsink;
+    const size_t rows = sink ? (size_t)a.nsink : (size_t)kWin;
+    const size_t row = sink ? (size_t)p : (size_t)(p % kWin);
+    return (sink ? a.sink : a.ring) + ((((size_t)a.slot * a.hkv + hk) * 2 + kind) * rows + row) * kD;
+  };
+  // key position p: 1 INT2 (block-head base in *bp), 2 fp16 (read at staging), 0 masked
+  auto locate = [&](int p, int blk, const uint8_t** bp) -> int {
     if (p > pmax || p >= a.L) return 0;
-    if (p < a.nsink || p >= a.L - kWin) {
-      const bool sink = p < a.nsink;
-      const size_t rows = sink ? (size_t)a.nsink : (size_t)kWin;
-      const size_t row = sink ? (size_t)p : (size_t)(p % kWin);
-      *hp = (sink ? a.sink : a.ring) + ((((size_t)a.slot * a.hkv + hk) * 2 + kind) * rows + row) * kD;
-      return 2;
-    }
+    if (p < a.nsink || p >= a.L - kWin) return 2;
     if (blk < 0 || blk >= a.num_blocks) {
       if (!sbad) raise_flag(a.status, OKV_DEV_BAD_BLOCK);
       sbad = 1;
@@ -680,18 +700,35 @@ __global__ void __launch_bounds__(kUpThreads, 1) prefill_umma_kernel(PrefillArgs
   };
   auto fetch = [&](int c, int kblk, int vblk) {
     const int p0 = kUpKC * c;
+    fetched_p0 = p0;
+    // a chunk wholly between the sink rows and the fp16 window, and below every
+    // row's position, is INT2 throughout (the common case): no per-token sorting
+    if (p0 >= a.nsink && p0 + kUpKC - 1 < a.L - kWin && p0 + kUpKC - 1 <= pmax) {
+      const bool kok = kblk >= 0 && kblk < a.num_blocks, vok = vblk >= 0 && vblk < a.num_blocks;
+      if (!(kok && vok)) {
+        if (!sbad) raise_flag(a.status, OKV_DEV_BAD_BLOCK);
+        sbad = 1;
+      }
+      ksrc = kok ? 1 : 0;
+      if (kok) {
+        const uint8_t* bp = a.pages + ((size_t)kblk * a.hkv + hk) * a.bhb;
+        kr0 = *reinterpret_cast<const uint4*>(bp + kKcOff + (ktk & 15) * 32 + 16 * kkb);
+        ksmw = *reinterpret_cast<const uint32_t*>(bp + sm_offset(1, kkb, ktk & 15, 0));
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i) vsrc[i] = vok ? 1 : 0;
+      if (vok)
+        vw = *reinterpret_cast<const uint4*>(a.pages + ((size_t)vblk * a.hkv + hk) * a.bhb + kVcOff +
+                                             ((vbq * 4 + (vtq & 3)) << 4));
+      return;
+    }
     {
       const uint8_t* bp = nullptr;
-      const __half* hp = nullptr;
       const int p = p0 + ktk;
-      ksrc = locate(p, kblk, 0, &bp, &hp);
+      ksrc = locate(p, kblk, &bp);
       if (ksrc == 1) {
-        kr[0] = *reinterpret_cast<const uint4*>(bp + kKcOff + (p & 15) * 32 + 16 * kkb);
+        kr0 = *reinterpret_cast<const uint4*>(bp + kKcOff + (p & 15) * 32 + 16 * kkb);
         ksmw = *reinterpret_cast<const uint32_t*>(bp + sm_offset(1, kkb, p & 15, 0));
-      } else if (ksrc == 2) {
-        const uint4* x = reinterpret_cast<const uint4*>(hp + 64 * kkb);
-#pragma unroll
-        for (int j = 0; j < 8; ++j) kr[j] = x[j];
       }
     }
     {
@@ -699,71 +736,87 @@ __global__ void __launch_bounds__(kUpThreads, 1) prefill_umma_kernel(PrefillArgs
       bool any_int2 = false;
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        const __half* hp = nullptr;
         const uint8_t* bpi = nullptr;
-        vsrc[i] = locate(p0 + 4 * vtq + i, vblk, 1, &bpi, &hp);
+        vsrc[i] = locate(p0 + 4 * vtq + i, vblk, &bpi);
         if (vsrc[i] == 1) {
           bp = bpi;
           any_int2 = true;
-        } else if (vsrc[i] == 2) {
-          const uint4* x = reinterpret_cast<const uint4*>(hp + 16 * vbq);
-          vh[i][0] = x[0];
-          vh[i][1] = x[1];
         }
       }
-      if (any_int2) vw = *reinterpret_cast<const uint4*>(bp + kVcOff + ((vbq * 4 + ((p0 + 4 * vtq) & 15) / 4) << 4));
+      if (any_int2) vw = *reinterpret_cast<const uint4*>(bp + kVcOff + ((vbq * 4 + (vtq & 3)) << 4));
     }
   };
-  auto stage = [&](int b) {
-    // keys: 8 chunks of 8 channels into row ktk of K-block kkb
-    const uint32_t kdst = sK + (uint32_t)b * kUpKBytes + (uint32_t)kkb * 8192u;
-    unsigned char* kg = gb + (kdst - base);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      uint32_t e[8];
-      const uint32_t w = i == 0 ? kr[0].x : i == 1 ? kr[0].y : i == 2 ? kr[0].z : kr[0].w;
-      word_to_half2x8<false>(w, e);
-#pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        const int jc = 2 * i + hh;
-        uint4 v = ksrc == 1 ? make_uint4(e[4 * hh], e[4 * hh + 1], e[4 * hh + 2], e[4 * hh + 3])
-                            : ksrc == 2 ? kr[jc] : make_uint4(0, 0, 0, 0);
-        *reinterpret_cast<uint4*>(kg + um_swz((uint32_t)ktk, (uint32_t)jc * 16u)) = v;
-      }
-    }
-    float s_ = 0.f, m_ = 0.f;
+  // (scale, min) of the fetched token: key scales for kkb 0, value scales for kkb 1
+  auto token_sm = [&](float& s_, float& m_) {
+    s_ = m_ = 0.f;
     if (ksrc == 1) {
       s_ = __half2float(__ushort_as_half((unsigned short)(ksmw & 0xffffu)));
       m_ = __half2float(__ushort_as_half((unsigned short)(ksmw >> 16)));
     } else if (ksrc == 2) {
       s_ = 1.f;
     }
+  };
+  auto stage_k = [&](int b) {
+    // keys: 8 chunks of 8 channels into row ktk of K-block kkb
+    const uint32_t kdst = sK + (uint32_t)b * kUpKBytes + (uint32_t)kkb * 8192u;
+    unsigned char* kg = gb + (kdst - base);
+    if (ksrc == 1) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        uint32_t e[8];
+        const uint32_t w = i == 0 ? kr0.x : i == 1 ? kr0.y : i == 2 ? kr0.z : kr0.w;
+        word_to_half2x8<false>(w, e);
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh)
+          *reinterpret_cast<uint4*>(kg + um_swz((uint32_t)ktk, (uint32_t)(2 * i + hh) * 16u)) =
+              make_uint4(e[4 * hh], e[4 * hh + 1], e[4 * hh + 2], e[4 * hh + 3]);
+      }
+    } else {
+      const uint4* x = ksrc == 2 ? reinterpret_cast<const uint4*>(fp16_row(fetched_p0 + ktk, 0) + 64 * kkb) : nullptr;
+#pragma unroll
+      for (int jc = 0; jc < 8; ++jc)
+        *reinterpret_cast<uint4*>(kg + um_swz((uint32_t)ktk, (uint32_t)jc * 16u)) =
+            ksrc == 2 ? x[jc] : make_uint4(0, 0, 0, 0);
+    }
     if (kkb == 0) {
+      float s_, m_;
+      token_sm(s_, m_);
       ms.ksm[b][ktk] = make_float2(s_, m_);
       ms.kval[b][ktk] = ksrc != 0;
-    } else if (ksrc == 1) {
-      ms.vsm[b][ktk] = make_float2(0.5f * s_, fmaf(1.5f, s_, m_));  // centred codes
-      s_ *= 0.5f;
-    } else {
-      ms.vsm[b][ktk] = make_float2(s_, m_);
     }
-    float vmx = kkb == 1 ? s_ : 0.f;
+    const int anybad = __any_sync(0xffffffffu, sbad != 0);
+    if (lane == 0) ms.bad[b][sw] = anybad;
+    sbad = 0;
+  };
+  const int flip = lane >> 4;
+  // lanes 16..31 write rows 16 apart from lanes 0..15 (same swizzle phase):
+  // they hold and store the other token pair first, so each store covers 32 banks
+  const uint32_t sel_a = flip ? 0x0302u : 0x0110u, sel_b = flip ? 0x0110u : 0x0302u;
+  auto stage_v = [&](int b) {
+    float vmx = 0.f;
+    if (kkb == 1) {
+      float s_, m_;
+      token_sm(s_, m_);
+      if (ksrc == 1) {
+        ms.vsm[b][ktk] = make_float2(0.5f * s_, fmaf(1.5f, s_, m_));  // centred codes
+        vmx = 0.5f * s_;
+      } else {
+        ms.vsm[b][ktk] = make_float2(s_, m_);
+        vmx = s_;
+      }
+    }
 #pragma unroll
     for (int o = 16; o >= 1; o >>= 1) vmx = fmaxf(vmx, __shfl_xor_sync(0xffffffffu, vmx, o));
-    const int anybad = __any_sync(0xffffffffu, sbad != 0);
-    if (lane == 0) {
-      ms.vsmax[b][sw] = vmx;
-      ms.bad[b][sw] = anybad;
-    }
-    sbad = 0;
-    // values: channels 16 vbq + ch, token pairs (2 vtq + s): one 32-bit word per (channel, pair)
+    if (lane == 0) ms.vsmax[b][sw] = vmx;
+    // values: channels 16 vbq + ch, token pairs (2 vtq + s): one 32-bit word per
+    // (channel, pair); pr[ch][s0] is the pair stored at position s0 ^ flip
     uint32_t pr[16][2];
     if (vsrc[0] == 1 && vsrc[1] == 1 && vsrc[2] == 1 && vsrc[3] == 1) {
       const uint32_t ws[4] = {vw.x, vw.y, vw.z, vw.w};  // word b': channels 4 b' .. + 3 of tokens 0..3
 #pragma unroll
       for (int bb = 0; bb < 4; ++bb) {
-        const uint32_t x01 = __byte_perm(ws[bb], 0u, 0x0110u);  // tokens 0, 1 in bytes 0, 2
-        const uint32_t x23 = __byte_perm(ws[bb], 0u, 0x0302u);  // tokens 2, 3
+        const uint32_t x01 = __byte_perm(ws[bb], 0u, sel_a);  // the pair's two tokens in bytes 0, 2
+        const uint32_t x23 = __byte_perm(ws[bb], 0u, sel_b);
         pr[4 * bb + 0][0] = centred_to_half2(codes_at_bit1<0>(x01));
         pr[4 * bb + 0][1] = centred_to_half2(codes_at_bit1<0>(x23));
         pr[4 * bb + 1][0] = centred_to_half2(codes_at_bit1<1>(x01));
@@ -782,8 +835,10 @@ __global__ void __launch_bounds__(kUpThreads, 1) prefill_umma_kernel(PrefillArgs
           const uint32_t t01 = __byte_perm(vw.x, vw.y, sel), t23 = __byte_perm(vw.z, vw.w, sel);
           word_to_half2x8<true>(__byte_perm(t01, t23, 0x5410u), e[i]);
         } else if (vsrc[i] == 2) {
-          e[i][0] = vh[i][0].x; e[i][1] = vh[i][0].y; e[i][2] = vh[i][0].z; e[i][3] = vh[i][0].w;
-          e[i][4] = vh[i][1].x; e[i][5] = vh[i][1].y; e[i][6] = vh[i][1].z; e[i][7] = vh[i][1].w;
+          const uint4* x = reinterpret_cast<const uint4*>(fp16_row(fetched_p0 + 4 * vtq + i, 1) + 16 * vbq);
+          const uint4 x0 = x[0], x1 = x[1];
+          e[i][0] = x0.x; e[i][1] = x0.y; e[i][2] = x0.z; e[i][3] = x0.w;
+          e[i][4] = x1.x; e[i][5] = x1.y; e[i][6] = x1.z; e[i][7] = x1.w;
         } else {
 #pragma unroll
           for (int j = 0; j < 8; ++j) e[i][j] = 0u;
@@ -792,27 +847,24 @@ __global__ void __launch_bounds__(kUpThreads, 1) prefill_umma_kernel(PrefillArgs
 #pragma unroll
       for (int ch = 0; ch < 16; ++ch) {
         const uint32_t sel = (ch & 1) ? 0x7632u : 0x5410u;
-        pr[ch][0] = __byte_perm(e[0][ch >> 1], e[1][ch >> 1], sel);
-        pr[ch][1] = __byte_perm(e[2][ch >> 1], e[3][ch >> 1], sel);
+        const uint32_t t01 = __byte_perm(e[0][ch >> 1], e[1][ch >> 1], sel);
+        const uint32_t t23 = __byte_perm(e[2][ch >> 1], e[3][ch >> 1], sel);
+        pr[ch][0] = flip ? t23 : t01;
+        pr[ch][1] = flip ? t01 : t23;
       }
     }
-    // lanes 16..31 write rows 16 apart from lanes 0..15 (same swizzle phase):
-    // they take the other token pair first, so each store covers 32 banks
-    const int flip = lane >> 4;
     unsigned char* vg = gb + (sV + (uint32_t)b * kUpVBytes - base);
 #pragma unroll
     for (int ch = 0; ch < 16; ++ch)
 #pragma unroll
-      for (int s0 = 0; s0 < 2; ++s0) {
-        const int s = s0 ^ flip;
-        const uint32_t v = flip ? pr[ch][s0 ^ 1] : pr[ch][s0];
-        *reinterpret_cast<uint32_t*>(vg + um_swz((uint32_t)(16 * vbq + ch), (uint32_t)(2 * vtq + s) * 4u)) = v;
-      }
+      for (int s0 = 0; s0 < 2; ++s0)
+        *reinterpret_cast<uint32_t*>(vg + um_swz((uint32_t)(16 * vbq + ch), (uint32_t)(2 * vtq + (s0 ^ flip)) * 4u)) =
+            pr[ch][s0];
   };
   if (warp >= kUpSmxWarps && warp < kUpMmaWarp) {
     int kb0, vb0;
     lookup(0, kb0, vb0);
-    fetch(0, kb0, vb0);
+    fetch(0, kb0, vb0);  // (fetch reads sbad, which starts clear)
     lookup(1, kblk_n, vblk_n);
   }
 
@@ -824,62 +876,93 @@ __global__ void __launch_bounds__(kUpThreads, 1) prefill_umma_kernel(PrefillArgs
 
   if (warp < kUpSmxWarps) {
     // ------------------------------------------------------------ softmax
-    const uint32_t lane_base = (uint32_t)(32 * warp) << 16;
-    float m_use = -INFINITY, l = 0.f, msum = 0.f;
+    const uint32_t lane_base = (uint32_t)(32 * quarter) << 16;
+    float m_use = -INFINITY;
+    float2 l2 = make_float2(0.f, 0.f), msum2 = make_float2(0.f, 0.f);  // two partial sums each
+    const float2 qup2 = make_float2(qup, qup), qsum2 = make_float2(qsum, qsum);
     bool alive = true;
     for (int c = 0; c < nch && alive; ++c) {
       const int b = c & 1;
       const uint32_t ph = ((uint32_t)c >> 1) & 1u;
-      alive = mbar_wait_bounded(&ms.kv_full[b], ph) && mbar_wait_bounded(&ms.s_full[b], ph);
+      alive = mbar_wait_bounded(&ms.k_full[b], ph) && mbar_wait_bounded(&ms.s_full[b], ph);
       alive = __all_sync(0xffffffffu, alive);
       if (!alive) break;
       um_fence_after();
-      float sv[kUpKC];
-      um_ld32(tS + lane_base + (uint32_t)(b * kUpKC), sv);
-      um_ld32(tS + lane_base + (uint32_t)(b * kUpKC + 32), sv + 32);
+      float sv[32];
+      um_ld32(tS + lane_base + (uint32_t)(b * kUpKC + 32 * hcol), sv);
       um_wait_ld();
       um_fence_before();
-      mbar_arrive(&ms.s_free[b]);
-      const int lim = min(rpos + 1, a.L) - kUpKC * c;  // tokens j < lim are causal and in the sequence
+      // scores in log2 units: s (q~ . c) 2^e / sqrt(d) + m sum(q~) / sqrt(d); columns j < lim are
+      // causal and inside the sequence
+      const int lim = min(rpos + 1, a.L) - kUpKC * c - 32 * hcol;
       const bool bad = (ms.bad[b][0] | ms.bad[b][1] | ms.bad[b][2] | ms.bad[b][3]) != 0;
+      const float4* k4p = reinterpret_cast<const float4*>(&ms.ksm[b][32 * hcol]);
       float bm = -INFINITY;
+      if (lim >= 32 && !bad) {
 #pragma unroll
-      for (int j = 0; j < kUpKC; ++j) {
-        const float2 ks = ms.ksm[b][j];
-        const float x = fmaf(ks.x * qup, sv[j], ks.y * qsum);
-        const bool ok = j < lim && (!bad || ms.kval[b][j] != 0);
-        sv[j] = ok ? x : -INFINITY;
-        bm = fmaxf(bm, sv[j]);
+        for (int j2 = 0; j2 < 16; ++j2) {
+          const float4 k4 = k4p[j2];  // (s, m) of columns 2 j2, 2 j2 + 1
+          const float2 x = __ffma2_rn(__fmul2_rn(make_float2(k4.x, k4.z), qup2), make_float2(sv[2 * j2], sv[2 * j2 + 1]),
+                                      __fmul2_rn(make_float2(k4.y, k4.w), qsum2));
+          sv[2 * j2] = x.x;
+          sv[2 * j2 + 1] = x.y;
+          bm = fmaxf(bm, fmaxf(x.x, x.y));
+        }
+      } else {
+        const int* kv = &ms.kval[b][32 * hcol];
+#pragma unroll
+        for (int j2 = 0; j2 < 16; ++j2) {
+          const float4 k4 = k4p[j2];
+          const float2 x = __ffma2_rn(__fmul2_rn(make_float2(k4.x, k4.z), qup2), make_float2(sv[2 * j2], sv[2 * j2 + 1]),
+                                      __fmul2_rn(make_float2(k4.y, k4.w), qsum2));
+          const bool ok0 = 2 * j2 < lim && (!bad || kv[2 * j2] != 0);
+          const bool ok1 = 2 * j2 + 1 < lim && (!bad || kv[2 * j2 + 1] != 0);
+          sv[2 * j2] = ok0 ? x.x : -INFINITY;
+          sv[2 * j2 + 1] = ok1 ? x.y : -INFINITY;
+          bm = fmaxf(bm, fmaxf(sv[2 * j2], sv[2 * j2 + 1]));
+        }
       }
+      mbar_arrive(&ms.s_free[b]);  // scores and key scales read
+      ms.red[b][hcol][rowc] = bm;
+      mbar_arrive(&ms.mx[quarter][b]);
       // tau: p < 2^tau and p s < 2^15 for the chunk's largest value scale
+      alive = mbar_wait_bounded(&ms.v_full[b], ph);
+      alive = __all_sync(0xffffffffu, alive);
+      if (!alive) break;
       const float vmax = fmaxf(fmaxf(ms.vsmax[b][0], ms.vsmax[b][1]), fmaxf(ms.vsmax[b][2], ms.vsmax[b][3]));
       const int ex = vmax > 0.f ? ((__float_as_int(vmax) >> 23) & 0xff) - 127 : 0;
       const float tau = (float)max(0, min(8, 14 - ex));
+      alive = mbar_wait_bounded(&ms.mx[quarter][b], ph);
+      alive = __all_sync(0xffffffffu, alive);
+      if (!alive) break;
+      bm = fmaxf(bm, ms.red[b][hcol ^ 1][rowc]);  // the row's maximum (both halves decide alike)
       const bool need = bm > m_use + tau;
       if (__any_sync(0xffffffffu, need)) {
-        const float alpha = need ? exp2f(m_use - bm) : 1.f;  // 0 while the row has seen nothing
+        const float alpha = need ? ex2_ftz(m_use - bm) : 1.f;  // 0 while the row has seen nothing
         if (c > 0) {
-          // O must hold chunk c - 1 before it is scaled
+          // O must hold chunk c - 1 before it is scaled; this thread scales columns 64 hcol .. + 63
           alive = mbar_wait_bounded(&ms.pv_done[(c - 1) & 1], ((uint32_t)(c - 1) >> 1) & 1u);
           alive = __all_sync(0xffffffffu, alive);
           if (!alive) break;
           um_fence_after();
 #pragma unroll 1
-          for (int q = 0; q < 4; ++q) {
+          for (int q = 0; q < 2; ++q) {
             float ov[32];
-            um_ld32(tO + lane_base + 32u * q, ov);
+            const uint32_t ta = tO + lane_base + (uint32_t)(64 * hcol + 32 * q);
+            um_ld32(ta, ov);
             um_wait_ld();
 #pragma unroll
             for (int i = 0; i < 32; ++i) ov[i] *= alpha;
-            um_st32(tO + lane_base + 32u * q, ov);
+            um_st32(ta, ov);
           }
           um_wait_st();
         }
-        l *= alpha;
-        msum *= alpha;
+        l2 = __fmul2_rn(l2, make_float2(alpha, alpha));
+        msum2 = __fmul2_rn(msum2, make_float2(alpha, alpha));
         if (need) m_use = bm;
       }
       const float mref = m_use == -INFINITY ? 0.f : m_use;
+      const float2 nm2 = make_float2(-mref, -mref);
       // p s into the A tiles of chunk c, once the value MMA of chunk c - 2 has read them
       if (c >= 2) {
         alive = mbar_wait_bounded(&ms.pv_done[b], ((uint32_t)(c - 2) >> 1) & 1u);
@@ -887,19 +970,27 @@ __global__ void __launch_bounds__(kUpThreads, 1) prefill_umma_kernel(PrefillArgs
         if (!alive) break;
       }
       unsigned char* pg = gb + (sP + (uint32_t)b * kUpPBytes - base);
+      const float4* v4p = reinterpret_cast<const float4*>(&ms.vsm[b][32 * hcol]);
 #pragma unroll
-      for (int j8 = 0; j8 < kUpKC / 8; ++j8) {
+      for (int j8 = 0; j8 < 4; ++j8) {
         uint32_t hi[4], lo[4];
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
-          const int j = 8 * j8 + 2 * u;
-          const float p0 = exp2f(sv[j] - mref), p1 = exp2f(sv[j + 1] - mref);
-          const float4 vs = *reinterpret_cast<const float4*>(&ms.vsm[b][j]);  // (s, m) of j and j + 1
-          l += p0 + p1;
-          msum = fmaf(p0, vs.y, fmaf(p1, vs.w, msum));
-          split_half2(p0 * vs.x, p1 * vs.z, hi[u], lo[u]);
+          const int j2 = 4 * j8 + u;
+          const float2 d = __fadd2_rn(make_float2(sv[2 * j2], sv[2 * j2 + 1]), nm2);
+          const float2 pp = make_float2(ex2_ftz(d.x), ex2_ftz(d.y));
+          const float4 vs = v4p[j2];  // (s, m) of columns 2 j2, 2 j2 + 1
+          l2 = __fadd2_rn(l2, pp);
+          msum2 = __ffma2_rn(pp, make_float2(vs.y, vs.w), msum2);
+          const float2 w = __fmul2_rn(pp, make_float2(vs.x, vs.z));
+          // hi: w with its low 13 mantissa bits cleared (exact in fp16 from 2^-14 up); lo: the rest
+          const float2 wh = make_float2(__uint_as_float(__float_as_uint(w.x) & 0xFFFFE000u),
+                                        __uint_as_float(__float_as_uint(w.y) & 0xFFFFE000u));
+          const float2 wl = __fadd2_rn(w, make_float2(-wh.x, -wh.y));
+          hi[u] = pack_half2(wh.x, wh.y);
+          lo[u] = pack_half2(wl.x, wl.y);
         }
-        const uint32_t off = um_swz((uint32_t)tid, (uint32_t)j8 * 16u);
+        const uint32_t off = um_swz((uint32_t)rowc, (uint32_t)(4 * hcol + j8) * 16u);
         *reinterpret_cast<uint4*>(pg + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
         *reinterpret_cast<uint4*>(pg + 16384u + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
       }
@@ -911,13 +1002,24 @@ __global__ void __launch_bounds__(kUpThreads, 1) prefill_umma_kernel(PrefillArgs
       alive = mbar_wait_bounded(&ms.pv_done[(nch - 1) & 1], ((uint32_t)(nch - 1) >> 1) & 1u);
       alive = __all_sync(0xffffffffu, alive);
     }
+    float l = 0.f, msum = 0.f;
+    if (alive) {
+      // the two halves' sums meet: one more round of the partners' barrier
+      ms.fin[hcol][rowc] = make_float2(l2.x + l2.y, msum2.x + msum2.y);
+      mbar_arrive(&ms.mx[quarter][nch & 1]);
+      alive = mbar_wait_bounded(&ms.mx[quarter][nch & 1], ((uint32_t)nch >> 1) & 1u);
+      alive = __all_sync(0xffffffffu, alive);
+      const float2 f0 = ms.fin[0][rowc], f1 = ms.fin[1][rowc];
+      l = f0.x + f1.x;
+      msum = f0.y + f1.y;
+    }
     if (alive) {
       um_fence_after();
-      float* dst = a.obuf + (size_t)rrow * kOStride;
+      float* dst = a.obuf + (size_t)rrow * kOStride + 64 * hcol;
 #pragma unroll 1
-      for (int q = 0; q < 4; ++q) {
+      for (int q = 0; q < 2; ++q) {
         float ov[32];
-        um_ld32(tO + lane_base + 32u * q, ov);
+        um_ld32(tO + lane_base + (uint32_t)(64 * hcol + 32 * q), ov);
         um_wait_ld();
         if (rok) {
 #pragma unroll
@@ -926,7 +1028,7 @@ __global__ void __launch_bounds__(kUpThreads, 1) prefill_umma_kernel(PrefillArgs
                 make_float4(ov[i] + msum, ov[i + 1] + msum, ov[i + 2] + msum, ov[i + 3] + msum);
         }
       }
-      if (rok) dst[128] = l;
+      if (rok && hcol == 0) a.obuf[(size_t)rrow * kOStride + 128] = l;
     } else if (lane == 0) {
       raise_flag(a.status, OKV_DEV_TIMEOUT);
     }
@@ -934,13 +1036,22 @@ __global__ void __launch_bounds__(kUpThreads, 1) prefill_umma_kernel(PrefillArgs
     // ------------------------------------------------------------ staging
     for (int c = 0; c < nch; ++c) {
       const int b = c & 1;
+      // keys once the score MMA and the softmax of chunk c - 2 are past them
+      if (c >= 2 && !mbar_wait_bounded(&ms.s_free[b], ((uint32_t)(c - 2) >> 1) & 1u)) {
+        raise_flag(a.status, OKV_DEV_TIMEOUT);
+        break;
+      }
+      stage_k(b);
+      um_fence_proxy_async();
+      mbar_arrive(&ms.k_full[b]);
+      // values once the value MMA of chunk c - 2 is done
       if (c >= 2 && !mbar_wait_bounded(&ms.pv_done[b], ((uint32_t)(c - 2) >> 1) & 1u)) {
         raise_flag(a.status, OKV_DEV_TIMEOUT);
         break;
       }
-      stage(b);
+      stage_v(b);
       um_fence_proxy_async();
-      mbar_arrive(&ms.kv_full[b]);
+      mbar_arrive(&ms.v_full[b]);
       if (c + 1 < nch) {
         fetch(c + 1, kblk_n, vblk_n);
         lookup(c + 2, kblk_n, vblk_n);
@@ -955,7 +1066,7 @@ __global__ void __launch_bounds__(kUpThreads, 1) prefill_umma_kernel(PrefillArgs
     uint32_t last_par = 0;
     auto issue_s = [&](int c) -> bool {
       const int b = c & 1;
-      if (!mbar_wait_bounded(&ms.kv_full[b], ((uint32_t)c >> 1) & 1u)) return false;
+      if (!mbar_wait_bounded(&ms.k_full[b], ((uint32_t)c >> 1) & 1u)) return false;
       if (c >= 2 && !mbar_wait_bounded(&ms.s_free[b], ((uint32_t)(c - 2) >> 1) & 1u)) return false;
       um_fence_after();
       const uint32_t kt = sK + (uint32_t)b * kUpKBytes;
@@ -977,6 +1088,7 @@ __global__ void __launch_bounds__(kUpThreads, 1) prefill_umma_kernel(PrefillArgs
     auto issue_pv = [&](int c) -> bool {
       const int b = c & 1;
       if (!mbar_wait_bounded(&ms.p_full[b], ((uint32_t)c >> 1) & 1u)) return false;
+      if (!mbar_wait_bounded(&ms.v_full[b], ((uint32_t)c >> 1) & 1u)) return false;
       um_fence_after();
       const uint32_t pt = sP + (uint32_t)b * kUpPBytes, vt2 = sV + (uint32_t)b * kUpVBytes;
 #pragma unroll
