@@ -1,6 +1,10 @@
 """Build ``libokv.so`` in-tree with nvcc for sm_100a (no JIT cache, no torch extension).
 
-Usage: ``python -m int2_kv_cache_rotate_b200.build [--verbose-ptxas]``.
+Usage: ``python -m int2_kv_cache_rotate_b200.build [--verbose-ptxas] [--short-wait]``.
+``--short-wait`` builds the test library ``libokv_shortwait.so`` instead: every
+bounded wait of the kernels gives up after 64 cycles (the waits of the timeout
+paths for work already issued keep their full limit), so that a test can run
+the timeout paths.
 """
 from __future__ import annotations
 
@@ -12,6 +16,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libokv.so")
+SHORT_WAIT_LIB = os.path.join(HERE, "libokv_shortwait.so")
 SOURCES = ["okv_api.cu", "append.cu", "decode.cu", "dequant.cu", "prefill.cu", "noalloc.cu", "calib.cpp",
            "rotio.cpp"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
@@ -24,9 +29,10 @@ def nvcc() -> str:
     return "nvcc"
 
 
-def build(verbose_ptxas: bool = False, out: str = LIB) -> str:
+def build(verbose_ptxas: bool = False, out: str = LIB, short_wait: bool = False) -> str:
     srcs = [os.path.join(CSRC, s) for s in SOURCES]
-    cmd = [nvcc(), *ARCH, "-O3", "-lineinfo", "-std=c++17", "-shared",
+    defs = ["-DOKV_WAIT_LIMIT_LOG2=6"] if short_wait else []
+    cmd = [nvcc(), *ARCH, "-O3", "-lineinfo", "-std=c++17", "-shared", *defs,
            "-Xcompiler", "-fPIC,-fopenmp,-O3", "-I", os.path.join(ROOT, "include"), "-I", CSRC,
            "-o", out, *srcs, "-lgomp"]
     if verbose_ptxas:
@@ -40,4 +46,7 @@ def build(verbose_ptxas: bool = False, out: str = LIB) -> str:
 
 
 if __name__ == "__main__":
-    print(build(verbose_ptxas="--verbose-ptxas" in sys.argv))
+    if "--short-wait" in sys.argv:
+        print(build(verbose_ptxas="--verbose-ptxas" in sys.argv, out=SHORT_WAIT_LIB, short_wait=True))
+    else:
+        print(build(verbose_ptxas="--verbose-ptxas" in sys.argv))

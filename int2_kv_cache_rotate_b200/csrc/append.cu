@@ -329,6 +329,7 @@ __global__ void __launch_bounds__(kUmThreads, 1) append_umma_kernel(AppendArgs a
     um_tma_load_3d(abuf + kUmRegion, map, 64, h, tile_of(i) * kUmTile, &afull[st]);
   };
   int loaded = 0, landed = 0;  // tiles whose loads were issued / waited for (producer lane 0)
+  int committed = 0;            // tiles whose MMAs were committed (producer lane 0)
 
   if (tid == 0) {
     for (int i = 0; i < 2; ++i) {
@@ -428,6 +429,7 @@ __global__ void __launch_bounds__(kUmThreads, 1) append_umma_kernel(AppendArgs a
                 ++step;
               }
           um_commit(&mma_done[i & 1]);
+          committed = i + 1;
         } else {
           alive = false;
         }
@@ -447,10 +449,15 @@ __global__ void __launch_bounds__(kUmThreads, 1) append_umma_kernel(AppendArgs a
         break;
       }
     }
-    // no copy may outlive the CTA: after a failed wait, wait (bounded) for the loads in flight
-    if (lane == 0)
+    // no copy may outlive the CTA and no MMA may write TMEM after it is freed:
+    // after a failed wait, wait (bounded) for the loads in flight and for the
+    // last commit (it completes after every MMA issued before it)
+    if (lane == 0) {
       for (int i = landed; i < loaded; ++i)
-        if (!mbar_wait_bounded(&afull[i % kUmStages], ((uint32_t)(i / kUmStages)) & 1u)) break;
+        if (!mbar_drain_bounded(&afull[i % kUmStages], ((uint32_t)(i / kUmStages)) & 1u)) break;
+      if (committed > 0)  // (the epilogue may have given up on a tile this thread completed)
+        mbar_drain_bounded(&mma_done[(committed - 1) & 1], ((uint32_t)(committed - 1) >> 1) & 1u);
+    }
   } else {
     const int wg = warp >> 2, q = warp & 3;
     // destination of this thread's token in tile i, fetched one tile (of this warpgroup) ahead

@@ -776,6 +776,7 @@ __global__ void __launch_bounds__(kHW * 32, (G <= 4) ? 2 : 1) decode_heads_kerne
     // window ahead (btq[bt_buf] holds blocks bt_base .. bt_base + 31), so no
     // block-table load sits between a released stage and its refill.
     int bt_base = p0, bt_buf = 0;
+    int issued = 0;  // stages of this entry whose copies went out (warp 0)
     auto bt_fill = [&](int wbase, int buf) {  // all lanes of warp 0
       const int pi = wbase + lane;
       if (pi < p1) cp_async4(&btq[buf][lane], trow + pi);
@@ -829,6 +830,7 @@ __global__ void __launch_bounds__(kHW * 32, (G <= 4) ? 2 : 1) decode_heads_kerne
       if (bid >= 0)
         bulk_g2s_hint(ring + s * kHStageBytes + q * copy_bytes, a.pages + (size_t)bid * copy_bytes, copy_bytes,
                       &full[s], l2_evict_first_policy());  // each block is read once
+      issued = max(issued, first + cnt);
       return true;
     };
     // Prologue: every slot (the ring is idle at an entry's start).  A batch
@@ -1141,6 +1143,15 @@ __global__ void __launch_bounds__(kHW * 32, (G <= 4) ? 2 : 1) decode_heads_kerne
       }
       __syncwarp();
       ++done;
+    }
+    if (!alive && warp == 0 && lane == 0) {
+      // after a timeout: the copies of stages issued but not consumed land
+      // before the ring is reused or the CTA exits.  A stage kHStages before
+      // the last issued one completed before its slot was refilled.
+      for (int j = max(0, issued - kHStages); j < issued; ++j) {
+        const uint32_t pos = it + (uint32_t)j;
+        if (!mbar_drain_bounded(&full[pos % kHStages], (pos / kHStages) & 1u)) break;
+      }
     }
     it += (uint32_t)nst;
 #pragma unroll

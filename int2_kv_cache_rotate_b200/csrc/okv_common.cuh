@@ -251,14 +251,48 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Bounded wait: gives up after ~2^31 SM cycles (about a second) and returns false.
-__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity) {
+// Bounded wait: gives up after 2^OKV_WAIT_LIMIT_LOG2 SM cycles (2^31 by
+// default, about a second) and returns false.  A test build sets a limit of
+// a few dozen cycles, so that waits run out while the work they wait for is
+// still in flight and the timeout paths run.
+#ifndef OKV_WAIT_LIMIT_LOG2
+#define OKV_WAIT_LIMIT_LOG2 31
+#endif
+__device__ __forceinline__ bool mbar_wait_cycles(uint64_t* bar, uint32_t parity, long long limit) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   while (!mbar_try_wait(bar, parity)) {
-    if (clock64() - t0 > (1ll << 31)) return false;
+    if (clock64() - t0 > limit) return false;
   }
   return true;
+}
+// non-blocking test of a phase (try_wait may itself suspend the thread until
+// the phase completes, so a short limit needs polling)
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity) {
+#if OKV_WAIT_LIMIT_LOG2 < 31
+  const long long t0 = clock64();
+  while (!mbar_test_wait(bar, parity)) {
+    if (clock64() - t0 > (1ll << OKV_WAIT_LIMIT_LOG2)) return false;
+  }
+  return true;
+#else
+  return mbar_wait_cycles(bar, parity, 1ll << 31);
+#endif
+}
+// The wait of a timeout path for work this CTA already issued (bulk copies,
+// MMAs), which completes on its own: always the full ~2^31-cycle limit, so
+// that nothing lands in shared memory or TMEM after the CTA has moved on.
+__device__ __forceinline__ bool mbar_drain_bounded(uint64_t* bar, uint32_t parity) {
+  return mbar_wait_cycles(bar, parity, 1ll << 31);
 }
 
 // D[16x8] += A[16x32] (u8, row-major) * B[32x8] (s8 or u8, column-major), s32 accumulate.

@@ -1106,11 +1106,10 @@ __global__ void __launch_bounds__(kUpThreads, 1) prefill_umma_kernel(PrefillArgs
     };
     bool alive = issue_s(0) && (nch < 2 || issue_s(1));
     for (int c = 0; c < nch && alive; ++c) alive = issue_pv(c) && (c + 2 >= nch || issue_s(c + 2));
-    if (!alive) {
-      raise_flag(a.status, OKV_DEV_TIMEOUT);
-      // the MMAs already issued finish before TMEM is freed: the last commit covers them all
-      if (last_bar != nullptr) mbar_wait_bounded(last_bar, last_par);
-    }
+    if (!alive) raise_flag(a.status, OKV_DEV_TIMEOUT);
+    // the MMAs already issued finish before TMEM is freed (the softmax warps may
+    // have given up on them): the last commit covers them all
+    if (last_bar != nullptr) mbar_drain_bounded(last_bar, last_par);
   }
   um_fence_before();
   __syncthreads();

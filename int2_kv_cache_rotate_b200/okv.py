@@ -15,7 +15,9 @@ import re
 import numpy as np
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libokv.so")
+# OKV_LIBRARY names another in-tree build of the same library (the short-wait
+# test build); by default the binding loads libokv.so
+LIB_PATH = os.environ.get("OKV_LIBRARY") or os.path.join(_HERE, "libokv.so")
 HEADER = os.path.join(os.path.dirname(_HERE), "include", "okv.h")
 
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_NUMERIC, ERR_IO = range(6)
