@@ -64,80 +64,130 @@ constexpr int kQaux = 8;
 constexpr int kOStride = 132;
 
 // ---------------------------------------------------------------------------
-// 1. q~ = q R_K for the chunk.  One CTA per (query head, 16 query tokens):
-// warp w holds rows 16w..16w+15 of U_K in registers for all 16 tokens; per
-// token the eight warps' partial sums meet in shared memory and warp (token
-// mod 8) runs the butterfly and the bit-reversal remap.
+// 1. q~ = q R_K for the chunk, and 3. o = (o' / l) R_V^T: one CTA per 64 rows
+// (token, query head) of one KV head.  The CTA stages the head's U (permuted
+// so that lane l's four columns l + 32 c are one 16-byte load) and the 64
+// input rows in shared memory; each warp takes 8 rows at once, so that every
+// U load feeds 8 rows, on the paired fp32 FMA.  The butterfly and the
+// bit-reversal remap run per row in registers.
 // ---------------------------------------------------------------------------
-constexpr int kQrTok = 16;
+constexpr int kRtRows = 64;
+constexpr size_t kRtSmem = (size_t)(kD * kD + kRtRows * kD) * sizeof(float);
+
+// global row of row rk (0 .. T G - 1) of KV head hk: token rk / G, query head hk G + rk % G
+__device__ __forceinline__ int rt_row(const PrefillArgs& a, int hk, int rk) {
+  return (rk / a.g) * a.hq + hk * a.g + rk % a.g;
+}
+
+// acc[rr] = x[rr] . U for 8 rows held in xs (fp32 rows of kD), U permuted in up
+__device__ __forceinline__ void rt_matvec8(const float* xs, const float* up, int lane, float2 (&acc)[8][2]) {
+#pragma unroll
+  for (int rr = 0; rr < 8; ++rr) acc[rr][0] = acc[rr][1] = make_float2(0.f, 0.f);
+#pragma unroll 1
+  for (int i = 0; i < kD; i += 4) {
+    float4 x4[8];
+#pragma unroll
+    for (int rr = 0; rr < 8; ++rr) x4[rr] = *reinterpret_cast<const float4*>(xs + rr * kD + i);
+#pragma unroll
+    for (int ii = 0; ii < 4; ++ii) {
+      const float4 u = *reinterpret_cast<const float4*>(up + (i + ii) * kD + 4 * lane);
+      const float2 u01 = make_float2(u.x, u.y), u23 = make_float2(u.z, u.w);
+#pragma unroll
+      for (int rr = 0; rr < 8; ++rr) {
+        const float xv = ii == 0 ? x4[rr].x : ii == 1 ? x4[rr].y : ii == 2 ? x4[rr].z : x4[rr].w;
+        const float2 x2 = make_float2(xv, xv);
+        acc[rr][0] = __ffma2_rn(x2, u01, acc[rr][0]);
+        acc[rr][1] = __ffma2_rn(x2, u23, acc[rr][1]);
+      }
+    }
+  }
+}
 
 __global__ void __launch_bounds__(256) prefill_qrot_kernel(PrefillArgs a) {
-  __shared__ float red[2][8][kD];
-  const int head = blockIdx.y;
-  const int hk = head / a.g;
-  const int tok0 = blockIdx.x * kQrTok;
+  extern __shared__ __align__(16) float rt_[];
+  float* up = rt_;             // up[i][4 l + c] = U_K[i][l + 32 c]
+  float* xs = rt_ + kD * kD;   // the tile's query rows, fp32
+  const int hk = blockIdx.y;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const float* U = a.u_k + (size_t)hk * kD * kD;
-  float4 u[16];
+  const int nrows = a.T * a.g;
+  const int r0 = blockIdx.x * kRtRows;
+  {
+    // lane l gathers U_K[i][l + 32 c] (coalesced across the warp) and stores one 16-byte chunk
+    // (the loads of 8 rows go out before their stores: one L2 latency per 8 rows)
+    const float* U = a.u_k + (size_t)hk * kD * kD;
+    const int l = threadIdx.x & 31, i0 = threadIdx.x >> 5;  // rows i0, i0 + 8, ...
+#pragma unroll 1
+    for (int ib = 0; ib < kD; ib += 64) {
+      float4 v[8];
 #pragma unroll
-  for (int r = 0; r < 16; ++r) u[r] = __ldg(reinterpret_cast<const float4*>(U + (size_t)(16 * warp + r) * kD) + lane);
-  for (int i = 0; i < kQrTok; ++i) {
-    const int tok = tok0 + i;
-    if (tok >= a.T) break;  // uniform across the CTA
-    const int row = tok * a.hq + head;
-    const float xv = __bfloat162float(a.q[(size_t)row * kD + 16 * warp + (lane & 15)]);
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int k = 0; k < 8; ++k) {
+        const float* ur = U + (size_t)(ib + i0 + 8 * k) * kD + l;
+        v[k] = make_float4(__ldg(ur), __ldg(ur + 32), __ldg(ur + 64), __ldg(ur + 96));
+      }
 #pragma unroll
-    for (int r = 0; r < 16; ++r) {
-      const float x = __shfl_sync(0xffffffffu, xv, r);
-      acc.x = fmaf(x, u[r].x, acc.x);
-      acc.y = fmaf(x, u[r].y, acc.y);
-      acc.z = fmaf(x, u[r].z, acc.z);
-      acc.w = fmaf(x, u[r].w, acc.w);
+      for (int k = 0; k < 8; ++k) *reinterpret_cast<float4*>(up + (ib + i0 + 8 * k) * kD + 4 * l) = v[k];
     }
-    *reinterpret_cast<float4*>(&red[i & 1][warp][4 * lane]) = acc;
-    __syncthreads();  // (double-buffered: the next token's sums go to the other half)
-    if (warp != (i & 7)) continue;
-    float y[4];
+    uint4 qv[kRtRows * kD / 8 / 256];  // this thread's 8-element pieces of the tile's rows
 #pragma unroll
-    for (int aa = 0; aa < 4; ++aa) {
-      float sum = 0.f;
-#pragma unroll
-      for (int w = 0; w < 8; ++w) sum += red[i & 1][w][lane + 32 * aa];
-      y[aa] = sum;
+    for (int k = 0; k < kRtRows * kD / 8 / 256; ++k) {
+      const int idx = threadIdx.x + 256 * k, r = idx >> 4, c8 = (idx & 15) * 8;
+      qv[k] = *reinterpret_cast<const uint4*>(a.q + (size_t)rt_row(a, hk, min(r0 + r, nrows - 1)) * kD + c8);
     }
-    wht128_warp(y, lane);
 #pragma unroll
-    for (int aa = 0; aa < 4; ++aa) y[aa] *= kInvSqrtD;
-    // lane l holds rotated channels 4 r + {0, 2, 1, 3} (r = rev5(l)) in y[0..3]
-    const int r = rev5(lane);
-    const float zc[4] = {y[0], y[2], y[1], y[3]};
-    float amax = fmaxf(fmaxf(fabsf(y[0]), fabsf(y[1])), fmaxf(fabsf(y[2]), fabsf(y[3])));
-    amax = warp_max(amax);
-    // 2^-e with amax 2^-e in [1, 2): the hi half keeps 11 bits, the lo half the next 11
-    int e = 0;
-    if (amax > 0.f) e = ((__float_as_int(amax) >> 23) & 0xff) - 127;
-    e = max(-100, min(100, e));
-    const float down = __int_as_float((127 - e) << 23);
-    __half* hi = a.qhi + (size_t)row * kD + 4 * r;
-    __half* lo = a.qlo + (size_t)row * kD + 4 * r;
-#pragma unroll
-    for (int f = 0; f < 4; ++f) {
-      const float x = zc[f] * down;
-      const __half h = __float2half_rn(x);
-      hi[f] = h;
-      lo[f] = __float2half_rn(x - __half2float(h));
+    for (int k = 0; k < kRtRows * kD / 8 / 256; ++k) {
+      const int idx = threadIdx.x + 256 * k, r = idx >> 4, c8 = (idx & 15) * 8;
+      const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&qv[k]);
+      const float2 f0 = __bfloat1622float2(b2[0]), f1 = __bfloat1622float2(b2[1]);
+      const float2 f2 = __bfloat1622float2(b2[2]), f3 = __bfloat1622float2(b2[3]);
+      *reinterpret_cast<float4*>(xs + r * kD + c8) = make_float4(f0.x, f0.y, f1.x, f1.y);
+      *reinterpret_cast<float4*>(xs + r * kD + c8 + 4) = make_float4(f2.x, f2.y, f3.x, f3.y);
     }
-    // per-group sums of q~: channels 4r.. lie in group r ng / 32
-    const float part = (zc[0] + zc[1]) + (zc[2] + zc[3]);
-    float gs[4];
+  }
+  __syncthreads();
+  {
+    const int rb = 8 * warp;
+    float2 acc[8][2];
+    rt_matvec8(xs + rb * kD, up, lane, acc);
 #pragma unroll
-    for (int k = 0; k < 4; ++k) gs[k] = warp_sum((k < a.ng && r * a.ng / 32 == k) ? part : 0.f);
-    if (lane == 0) {
+    for (int rr = 0; rr < 8; ++rr) {
+      const int rk = r0 + rb + rr;
+      if (rk >= nrows) continue;  // uniform across the warp
+      const int row = rt_row(a, hk, rk);
+      // lane l holds x[l + 32 c] in acc[rr][c / 2].(c % 2)
+      float y[4] = {acc[rr][0].x, acc[rr][0].y, acc[rr][1].x, acc[rr][1].y};
+      wht128_warp(y, lane);
+#pragma unroll
+      for (int aa = 0; aa < 4; ++aa) y[aa] *= kInvSqrtD;
+      // lane l holds rotated channels 4 r + {0, 2, 1, 3} (r = rev5(l)) in y[0..3]
+      const int r = rev5(lane);
+      const float zc[4] = {y[0], y[2], y[1], y[3]};
+      float amax = fmaxf(fmaxf(fabsf(y[0]), fabsf(y[1])), fmaxf(fabsf(y[2]), fabsf(y[3])));
+      amax = warp_max(amax);
+      // 2^-e with amax 2^-e in [1, 2): the hi half keeps 11 bits, the lo half the next 11
+      int e = 0;
+      if (amax > 0.f) e = ((__float_as_int(amax) >> 23) & 0xff) - 127;
+      e = max(-100, min(100, e));
+      const float down = __int_as_float((127 - e) << 23);
+      uint32_t hw[2], lw[2];
+#pragma unroll
+      for (int f = 0; f < 4; f += 2) {
+        const float x0 = zc[f] * down, x1 = zc[f + 1] * down;
+        const __half2 h = __floats2half2_rn(x0, x1);
+        const float2 hb = __half22float2(h);
+        const __half2 l2 = __floats2half2_rn(x0 - hb.x, x1 - hb.y);
+        hw[f >> 1] = *reinterpret_cast<const uint32_t*>(&h);
+        lw[f >> 1] = *reinterpret_cast<const uint32_t*>(&l2);
+      }
+      *reinterpret_cast<uint2*>(a.qhi + (size_t)row * kD + 4 * r) = make_uint2(hw[0], hw[1]);
+      *reinterpret_cast<uint2*>(a.qlo + (size_t)row * kD + 4 * r) = make_uint2(lw[0], lw[1]);
+      // per-group sums of q~: channels 4r.. lie in group r ng / 32
+      const float part = (zc[0] + zc[1]) + (zc[2] + zc[3]);
       float* aux = a.qaux + (size_t)row * kQaux;
-#pragma unroll
-      for (int k = 0; k < 4; ++k) aux[k] = gs[k];
-      aux[4] = __int_as_float((127 + e) << 23);
+      for (int k = 0; k < a.ng; ++k) {  // (uniform: a.ng is 1, 2 or 4)
+        const float gk = warp_sum(r * a.ng / 32 == k ? part : 0.f);
+        if (lane == 0) aux[k] = gk;
+      }
+      if (lane == 0) aux[4] = __int_as_float((127 + e) << 23);
     }
   }
 }
@@ -1119,60 +1169,74 @@ __global__ void __launch_bounds__(kUpThreads, 1) prefill_umma_kernel(PrefillArgs
   }
 }
 
-// ---------------------------------------------------------------------------
-// 3. o = (o' / l) R_V^T.  One CTA per (query head, 16 query tokens): U_V of
-// the head's KV head is staged in shared memory once, then warp w takes
-// tokens w and w + 8: un-permute and butterfly in registers, and the U_V^T
-// matvec from shared memory (lane l produces outputs l + 32 j).
-// ---------------------------------------------------------------------------
-constexpr int kUrTok = 16;
-constexpr int kUStride = kD + 4;  // floats per staged U_V row
-
+// 3. o = (o' / l) R_V^T (see 1. for the tiling): un-permute, 1 / l and the
+// butterfly per row in registers, the row to shared memory, then o = x U_V^T
+// with U_V^T permuted: ut[i][4 l + j] = U_V[l + 32 j][i].
 __global__ void __launch_bounds__(256) prefill_unrotate_kernel(PrefillArgs a) {
-  extern __shared__ __align__(16) float us_[];  // U_V [128][132]
-  const int head = blockIdx.y;
-  const int hk = head / a.g;
+  extern __shared__ __align__(16) float rt_[];
+  float* ut = rt_;
+  float* xs = rt_ + kD * kD;
+  const int hk = blockIdx.y;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int nrows = a.T * a.g;
+  const int r0 = blockIdx.x * kRtRows;
   {
-    const float4* U = reinterpret_cast<const float4*>(a.u_v + (size_t)hk * kD * kD);
-    for (int i = threadIdx.x; i < kD * kD / 4; i += blockDim.x) {
-      const int r = i / (kD / 4), c4 = i % (kD / 4);
-      *reinterpret_cast<float4*>(us_ + r * kUStride + 4 * c4) = __ldg(U + i);
+    // lane l reads 16 bytes of rows l + 32 j (columns i0 .. i0 + 3) and stores
+    // the four 16-byte chunks ut[i0 + k][4 l .. 4 l + 3]: conflict-free
+    const float* U = a.u_v + (size_t)hk * kD * kD;
+    float4 uu[4][4];  // all four of this thread's pieces are loaded before any is stored
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int t = threadIdx.x + 256 * k, l = t & 31, i0 = 4 * (t >> 5);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) uu[k][j] = __ldg(reinterpret_cast<const float4*>(U + (size_t)(l + 32 * j) * kD + i0));
+    }
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int t = threadIdx.x + 256 * k, l = t & 31, i0 = 4 * (t >> 5);
+      const float4* u = uu[k];
+      *reinterpret_cast<float4*>(ut + (i0 + 0) * kD + 4 * l) = make_float4(u[0].x, u[1].x, u[2].x, u[3].x);
+      *reinterpret_cast<float4*>(ut + (i0 + 1) * kD + 4 * l) = make_float4(u[0].y, u[1].y, u[2].y, u[3].y);
+      *reinterpret_cast<float4*>(ut + (i0 + 2) * kD + 4 * l) = make_float4(u[0].z, u[1].z, u[2].z, u[3].z);
+      *reinterpret_cast<float4*>(ut + (i0 + 3) * kD + 4 * l) = make_float4(u[0].w, u[1].w, u[2].w, u[3].w);
     }
   }
-  __syncthreads();
-  for (int i = warp; i < kUrTok; i += 8) {
-    const int tok = blockIdx.x * kUrTok + i;
-    if (tok >= a.T) break;
-    const int row = tok * a.hq + head;
-    const float* src = a.obuf + (size_t)row * kOStride;
-    const float l = src[128];
-    const float inv = l > 0.f ? 1.f / l : 0.f;
+  // this warp's 8 rows: x = H-butterfly of the un-permuted o' / l, into xs.
+  // All 8 rows' loads go out before the first butterfly.
+  const int r = rev5(lane);
+  float4 o4[8];
+  float lr[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const float* src = a.obuf + (size_t)rt_row(a, hk, min(r0 + 8 * warp + k, nrows - 1)) * kOStride;
+    o4[k] = *reinterpret_cast<const float4*>(src + 4 * r);  // rotated channels 4 r .. 4 r + 3
+    lr[k] = src[128];
+  }
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const float inv = lr[k] > 0.f ? 1.f / lr[k] : 0.f;
     // lane l: pre-permutation channels l + 32 aa = rotated channels 4 rev5(l) + rev2(aa)
-    const int r = rev5(lane);
-    float y[4];
-#pragma unroll
-    for (int aa = 0; aa < 4; ++aa) y[aa] = src[4 * r + rev2(aa)] * inv;
+    float y[4] = {o4[k].x * inv, o4[k].z * inv, o4[k].y * inv, o4[k].w * inv};
     wht128_warp(y, lane);
-    float x[4];
 #pragma unroll
-    for (int aa = 0; aa < 4; ++aa) x[aa] = y[aa] * kInvSqrtD;  // x_i for i = lane + 32 aa
-    // o_c = sum_i x_i U_V[c][i]: lane owns outputs c = lane + 32 j
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 4
-    for (int i4 = 0; i4 < kD / 4; ++i4) {
-      float xi[4];
+    for (int aa = 0; aa < 4; ++aa) xs[(8 * warp + k) * kD + lane + 32 * aa] = y[aa] * kInvSqrtD;
+  }
+  __syncthreads();  // U_V^T staged (this warp's rows need only __syncwarp, U needs the CTA)
+  {
+    const int rb = 8 * warp;
+    float2 acc[8][2];
+    rt_matvec8(xs + rb * kD, ut, lane, acc);
 #pragma unroll
-      for (int q = 0; q < 4; ++q) xi[q] = __shfl_sync(0xffffffffu, x[(4 * i4 + q) >> 5], (4 * i4 + q) & 31);
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const float4 uu = *reinterpret_cast<const float4*>(us_ + (lane + 32 * j) * kUStride + 4 * i4);
-        acc[j] = fmaf(xi[0], uu.x, fmaf(xi[1], uu.y, fmaf(xi[2], uu.z, fmaf(xi[3], uu.w, acc[j]))));
+    for (int rr = 0; rr < 8; ++rr) {
+      const int rk = r0 + rb + rr;
+      if (rk < nrows) {
+        float* dst = a.out + (size_t)rt_row(a, hk, rk) * kD;
+        dst[lane] = acc[rr][0].x;
+        dst[lane + 32] = acc[rr][0].y;
+        dst[lane + 64] = acc[rr][1].x;
+        dst[lane + 96] = acc[rr][1].y;
       }
     }
-    float* dst = a.out + (size_t)row * kD;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) dst[lane + 32 * j] = acc[j];
   }
 }
 
@@ -1222,7 +1286,12 @@ okv_status launch_prefill(const okv_cache_desc* d, const void* q, int T, int slo
   a.mbps = d->max_blocks_per_seq;
   a.num_blocks = d->num_blocks;
   a.nsink = d->num_sink;
-  prefill_qrot_kernel<<<dim3((unsigned)((T + kQrTok - 1) / kQrTok), (unsigned)a.hq), 256, 0, s>>>(a);
+  static std::atomic<uint32_t> qr_attr{0}, ur_attr{0};
+  cudaError_t e0 = set_smem_limit_once((const void*)prefill_qrot_kernel, (int)kRtSmem, qr_attr);
+  if (e0 == cudaSuccess) e0 = set_smem_limit_once((const void*)prefill_unrotate_kernel, (int)kRtSmem, ur_attr);
+  if (e0 != cudaSuccess) return fail(OKV_ERR_CUDA, "prefill rotation smem attribute: %s", cudaGetErrorString(e0));
+  const dim3 rt_grid((unsigned)((T * a.g + kRtRows - 1) / kRtRows), (unsigned)a.hkv);
+  prefill_qrot_kernel<<<rt_grid, 256, kRtSmem, s>>>(a);
   okv_status st = check_launch("prefill query rotation");
   if (st != OKV_OK) return st;
   const dim3 grid((unsigned)((T * a.g + kPfRows - 1) / kPfRows), (unsigned)a.hkv);
@@ -1239,11 +1308,7 @@ okv_status launch_prefill(const okv_cache_desc* d, const void* q, int T, int slo
   }
   st = check_launch("prefill attention");
   if (st != OKV_OK) return st;
-  const size_t usmem = (size_t)kD * kUStride * sizeof(float);
-  static std::atomic<uint32_t> attr_set{0};
-  cudaError_t e = set_smem_limit_once((const void*)prefill_unrotate_kernel, (int)usmem, attr_set);
-  if (e != cudaSuccess) return fail(OKV_ERR_CUDA, "prefill un-rotation smem attribute: %s", cudaGetErrorString(e));
-  prefill_unrotate_kernel<<<dim3((unsigned)((T + kUrTok - 1) / kUrTok), (unsigned)a.hq), 256, usmem, s>>>(a);
+  prefill_unrotate_kernel<<<rt_grid, 256, kRtSmem, s>>>(a);
   return check_launch("prefill un-rotation");
 }
 
