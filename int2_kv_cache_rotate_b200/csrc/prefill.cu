@@ -715,11 +715,17 @@ __global__ void __launch_bounds__(kUpThreads, 1) prefill_umma_kernel(PrefillArgs
   const int stid = tid - 32 * kUpSmxWarps, sw = stid >> 5;
   const int ktk = 16 * sw + (lane & 15), kkb = lane >> 4;      // key token, K-block (64 channels)
   const int vtq = lane & 15, vbq = 2 * sw + (lane >> 4);       // value token quad, channel sixteen
-  int ksrc = 0, vsrc[4] = {0, 0, 0, 0}, sbad = 0;               // 0 masked, 1 INT2, 2 fp16
-  uint4 kr0 = make_uint4(0, 0, 0, 0);  // INT2 key codes of the fetched token (64 channels)
-  uint4 vw = make_uint4(0, 0, 0, 0);   // INT2 value codes of the fetched quad (16 channels x 4 tokens)
-  int fetched_p0 = 0;                  // first position of the fetched chunk
-  uint32_t ksmw = 0;
+  // What a staging thread fetched of one chunk, held in registers until it is
+  // staged; two of them alternate, so that a chunk's loads are in flight two
+  // chunks before its tiles are written.
+  struct Fetched {
+    int ksrc, vsrc[4], sbad;  // sources: 0 masked, 1 INT2, 2 fp16; sbad: a block id was out of range
+    int p0;                   // first position of the chunk
+    uint4 kr0;                // INT2 key codes of the token (64 channels)
+    uint4 vw;                 // INT2 value codes of the quad (16 channels x 4 tokens)
+    uint32_t ksmw;            // the token's (scale, min): key scales for kkb 0, value scales for kkb 1
+  };
+  Fetched fa, fb;
   // block ids of this thread's key token and value quad, looked up one chunk
   // before their codes are fetched (the table read and the code read would
   // otherwise be two dependent memory latencies per chunk)
@@ -737,48 +743,49 @@ __global__ void __launch_bounds__(kUpThreads, 1) prefill_umma_kernel(PrefillArgs
     return (sink ? a.sink : a.ring) + ((((size_t)a.slot * a.hkv + hk) * 2 + kind) * rows + row) * kD;
   };
   // key position p: 1 INT2 (block-head base in *bp), 2 fp16 (read at staging), 0 masked
-  auto locate = [&](int p, int blk, const uint8_t** bp) -> int {
+  auto locate = [&](Fetched& f, int p, int blk, const uint8_t** bp) -> int {
     if (p > pmax || p >= a.L) return 0;
     if (p < a.nsink || p >= a.L - kWin) return 2;
     if (blk < 0 || blk >= a.num_blocks) {
-      if (!sbad) raise_flag(a.status, OKV_DEV_BAD_BLOCK);
-      sbad = 1;
+      if (!f.sbad) raise_flag(a.status, OKV_DEV_BAD_BLOCK);
+      f.sbad = 1;
       return 0;
     }
     *bp = a.pages + ((size_t)blk * a.hkv + hk) * a.bhb;
     return 1;
   };
-  auto fetch = [&](int c, int kblk, int vblk) {
+  auto fetch = [&](Fetched& f, int c, int kblk, int vblk) {
     const int p0 = kUpKC * c;
-    fetched_p0 = p0;
+    f.p0 = p0;
+    f.sbad = 0;
     // a chunk wholly between the sink rows and the fp16 window, and below every
     // row's position, is INT2 throughout (the common case): no per-token sorting
     if (p0 >= a.nsink && p0 + kUpKC - 1 < a.L - kWin && p0 + kUpKC - 1 <= pmax) {
       const bool kok = kblk >= 0 && kblk < a.num_blocks, vok = vblk >= 0 && vblk < a.num_blocks;
       if (!(kok && vok)) {
-        if (!sbad) raise_flag(a.status, OKV_DEV_BAD_BLOCK);
-        sbad = 1;
+        raise_flag(a.status, OKV_DEV_BAD_BLOCK);
+        f.sbad = 1;
       }
-      ksrc = kok ? 1 : 0;
+      f.ksrc = kok ? 1 : 0;
       if (kok) {
         const uint8_t* bp = a.pages + ((size_t)kblk * a.hkv + hk) * a.bhb;
-        kr0 = *reinterpret_cast<const uint4*>(bp + kKcOff + (ktk & 15) * 32 + 16 * kkb);
-        ksmw = *reinterpret_cast<const uint32_t*>(bp + sm_offset(1, kkb, ktk & 15, 0));
+        f.kr0 = *reinterpret_cast<const uint4*>(bp + kKcOff + (ktk & 15) * 32 + 16 * kkb);
+        f.ksmw = *reinterpret_cast<const uint32_t*>(bp + sm_offset(1, kkb, ktk & 15, 0));
       }
 #pragma unroll
-      for (int i = 0; i < 4; ++i) vsrc[i] = vok ? 1 : 0;
+      for (int i = 0; i < 4; ++i) f.vsrc[i] = vok ? 1 : 0;
       if (vok)
-        vw = *reinterpret_cast<const uint4*>(a.pages + ((size_t)vblk * a.hkv + hk) * a.bhb + kVcOff +
-                                             ((vbq * 4 + (vtq & 3)) << 4));
+        f.vw = *reinterpret_cast<const uint4*>(a.pages + ((size_t)vblk * a.hkv + hk) * a.bhb + kVcOff +
+                                               ((vbq * 4 + (vtq & 3)) << 4));
       return;
     }
     {
       const uint8_t* bp = nullptr;
       const int p = p0 + ktk;
-      ksrc = locate(p, kblk, &bp);
-      if (ksrc == 1) {
-        kr0 = *reinterpret_cast<const uint4*>(bp + kKcOff + (p & 15) * 32 + 16 * kkb);
-        ksmw = *reinterpret_cast<const uint32_t*>(bp + sm_offset(1, kkb, p & 15, 0));
+      f.ksrc = locate(f, p, kblk, &bp);
+      if (f.ksrc == 1) {
+        f.kr0 = *reinterpret_cast<const uint4*>(bp + kKcOff + (p & 15) * 32 + 16 * kkb);
+        f.ksmw = *reinterpret_cast<const uint32_t*>(bp + sm_offset(1, kkb, p & 15, 0));
       }
     }
     {
@@ -787,34 +794,34 @@ __global__ void __launch_bounds__(kUpThreads, 1) prefill_umma_kernel(PrefillArgs
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const uint8_t* bpi = nullptr;
-        vsrc[i] = locate(p0 + 4 * vtq + i, vblk, &bpi);
-        if (vsrc[i] == 1) {
+        f.vsrc[i] = locate(f, p0 + 4 * vtq + i, vblk, &bpi);
+        if (f.vsrc[i] == 1) {
           bp = bpi;
           any_int2 = true;
         }
       }
-      if (any_int2) vw = *reinterpret_cast<const uint4*>(bp + kVcOff + ((vbq * 4 + (vtq & 3)) << 4));
+      if (any_int2) f.vw = *reinterpret_cast<const uint4*>(bp + kVcOff + ((vbq * 4 + (vtq & 3)) << 4));
     }
   };
   // (scale, min) of the fetched token: key scales for kkb 0, value scales for kkb 1
-  auto token_sm = [&](float& s_, float& m_) {
+  auto token_sm = [&](const Fetched& f, float& s_, float& m_) {
     s_ = m_ = 0.f;
-    if (ksrc == 1) {
-      s_ = __half2float(__ushort_as_half((unsigned short)(ksmw & 0xffffu)));
-      m_ = __half2float(__ushort_as_half((unsigned short)(ksmw >> 16)));
-    } else if (ksrc == 2) {
+    if (f.ksrc == 1) {
+      s_ = __half2float(__ushort_as_half((unsigned short)(f.ksmw & 0xffffu)));
+      m_ = __half2float(__ushort_as_half((unsigned short)(f.ksmw >> 16)));
+    } else if (f.ksrc == 2) {
       s_ = 1.f;
     }
   };
-  auto stage_k = [&](int b) {
+  auto stage_k = [&](const Fetched& f, int b) {
     // keys: 8 chunks of 8 channels into row ktk of K-block kkb
     const uint32_t kdst = sK + (uint32_t)b * kUpKBytes + (uint32_t)kkb * 8192u;
     unsigned char* kg = gb + (kdst - base);
-    if (ksrc == 1) {
+    if (f.ksrc == 1) {
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         uint32_t e[8];
-        const uint32_t w = i == 0 ? kr0.x : i == 1 ? kr0.y : i == 2 ? kr0.z : kr0.w;
+        const uint32_t w = i == 0 ? f.kr0.x : i == 1 ? f.kr0.y : i == 2 ? f.kr0.z : f.kr0.w;
         word_to_half2x8<false>(w, e);
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh)
@@ -822,32 +829,31 @@ __global__ void __launch_bounds__(kUpThreads, 1) prefill_umma_kernel(PrefillArgs
               make_uint4(e[4 * hh], e[4 * hh + 1], e[4 * hh + 2], e[4 * hh + 3]);
       }
     } else {
-      const uint4* x = ksrc == 2 ? reinterpret_cast<const uint4*>(fp16_row(fetched_p0 + ktk, 0) + 64 * kkb) : nullptr;
+      const uint4* x = f.ksrc == 2 ? reinterpret_cast<const uint4*>(fp16_row(f.p0 + ktk, 0) + 64 * kkb) : nullptr;
 #pragma unroll
       for (int jc = 0; jc < 8; ++jc)
         *reinterpret_cast<uint4*>(kg + um_swz((uint32_t)ktk, (uint32_t)jc * 16u)) =
-            ksrc == 2 ? x[jc] : make_uint4(0, 0, 0, 0);
+            f.ksrc == 2 ? x[jc] : make_uint4(0, 0, 0, 0);
     }
     if (kkb == 0) {
       float s_, m_;
-      token_sm(s_, m_);
+      token_sm(f, s_, m_);
       ms.ksm[b][ktk] = make_float2(s_, m_);
-      ms.kval[b][ktk] = ksrc != 0;
+      ms.kval[b][ktk] = f.ksrc != 0;
     }
-    const int anybad = __any_sync(0xffffffffu, sbad != 0);
+    const int anybad = __any_sync(0xffffffffu, f.sbad != 0);
     if (lane == 0) ms.bad[b][sw] = anybad;
-    sbad = 0;
   };
   const int flip = lane >> 4;
   // lanes 16..31 write rows 16 apart from lanes 0..15 (same swizzle phase):
   // they hold and store the other token pair first, so each store covers 32 banks
   const uint32_t sel_a = flip ? 0x0302u : 0x0110u, sel_b = flip ? 0x0110u : 0x0302u;
-  auto stage_v = [&](int b) {
+  auto stage_v = [&](const Fetched& f, int b) {
     float vmx = 0.f;
     if (kkb == 1) {
       float s_, m_;
-      token_sm(s_, m_);
-      if (ksrc == 1) {
+      token_sm(f, s_, m_);
+      if (f.ksrc == 1) {
         ms.vsm[b][ktk] = make_float2(0.5f * s_, fmaf(1.5f, s_, m_));  // centred codes
         vmx = 0.5f * s_;
       } else {
@@ -861,8 +867,8 @@ __global__ void __launch_bounds__(kUpThreads, 1) prefill_umma_kernel(PrefillArgs
     // values: channels 16 vbq + ch, token pairs (2 vtq + s): one 32-bit word per
     // (channel, pair); pr[ch][s0] is the pair stored at position s0 ^ flip
     uint32_t pr[16][2];
-    if (vsrc[0] == 1 && vsrc[1] == 1 && vsrc[2] == 1 && vsrc[3] == 1) {
-      const uint32_t ws[4] = {vw.x, vw.y, vw.z, vw.w};  // word b': channels 4 b' .. + 3 of tokens 0..3
+    if (f.vsrc[0] == 1 && f.vsrc[1] == 1 && f.vsrc[2] == 1 && f.vsrc[3] == 1) {
+      const uint32_t ws[4] = {f.vw.x, f.vw.y, f.vw.z, f.vw.w};  // word b': channels 4 b' .. + 3 of tokens 0..3
 #pragma unroll
       for (int bb = 0; bb < 4; ++bb) {
         const uint32_t x01 = __byte_perm(ws[bb], 0u, sel_a);  // the pair's two tokens in bytes 0, 2
@@ -880,12 +886,12 @@ __global__ void __launch_bounds__(kUpThreads, 1) prefill_umma_kernel(PrefillArgs
       uint32_t e[4][8];  // per token: fp16 pairs of adjacent channels
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        if (vsrc[i] == 1) {
+        if (f.vsrc[i] == 1) {
           const uint32_t sel = (uint32_t)(i | ((4 + i) << 4));
-          const uint32_t t01 = __byte_perm(vw.x, vw.y, sel), t23 = __byte_perm(vw.z, vw.w, sel);
+          const uint32_t t01 = __byte_perm(f.vw.x, f.vw.y, sel), t23 = __byte_perm(f.vw.z, f.vw.w, sel);
           word_to_half2x8<true>(__byte_perm(t01, t23, 0x5410u), e[i]);
-        } else if (vsrc[i] == 2) {
-          const uint4* x = reinterpret_cast<const uint4*>(fp16_row(fetched_p0 + 4 * vtq + i, 1) + 16 * vbq);
+        } else if (f.vsrc[i] == 2) {
+          const uint4* x = reinterpret_cast<const uint4*>(fp16_row(f.p0 + 4 * vtq + i, 1) + 16 * vbq);
           const uint4 x0 = x[0], x1 = x[1];
           e[i][0] = x0.x; e[i][1] = x0.y; e[i][2] = x0.z; e[i][3] = x0.w;
           e[i][4] = x1.x; e[i][5] = x1.y; e[i][6] = x1.z; e[i][7] = x1.w;
@@ -914,8 +920,10 @@ __global__ void __launch_bounds__(kUpThreads, 1) prefill_umma_kernel(PrefillArgs
   if (warp >= kUpSmxWarps && warp < kUpMmaWarp) {
     int kb0, vb0;
     lookup(0, kb0, vb0);
-    fetch(0, kb0, vb0);  // (fetch reads sbad, which starts clear)
-    lookup(1, kblk_n, vblk_n);
+    fetch(fa, 0, kb0, vb0);
+    lookup(1, kb0, vb0);
+    if (1 < nch) fetch(fb, 1, kb0, vb0);
+    lookup(2, kblk_n, vblk_n);
   }
 
   um_fence_before();
@@ -1084,34 +1092,37 @@ __global__ void __launch_bounds__(kUpThreads, 1) prefill_umma_kernel(PrefillArgs
     }
   } else if (warp < kUpMmaWarp) {
     // ------------------------------------------------------------ staging
-    for (int c = 0; c < nch; ++c) {
+    // chunk c from fetch slot f, then chunk c + 2's loads into the same slot
+    auto run_chunk = [&](Fetched& f, int c) -> bool {
       const int b = c & 1;
       // keys once the score MMA and the softmax of chunk c - 2 are past them
-      if (c >= 2 && !mbar_wait_bounded(&ms.s_free[b], ((uint32_t)(c - 2) >> 1) & 1u)) {
-        raise_flag(a.status, OKV_DEV_TIMEOUT);
-        break;
-      }
-      stage_k(b);
+      if (c >= 2 && !mbar_wait_bounded(&ms.s_free[b], ((uint32_t)(c - 2) >> 1) & 1u)) return false;
+      stage_k(f, b);
       um_fence_proxy_async();
       mbar_arrive(&ms.k_full[b]);
       // values once the value MMA of chunk c - 2 is done
-      if (c >= 2 && !mbar_wait_bounded(&ms.pv_done[b], ((uint32_t)(c - 2) >> 1) & 1u)) {
-        raise_flag(a.status, OKV_DEV_TIMEOUT);
-        break;
-      }
-      stage_v(b);
+      if (c >= 2 && !mbar_wait_bounded(&ms.pv_done[b], ((uint32_t)(c - 2) >> 1) & 1u)) return false;
+      stage_v(f, b);
       um_fence_proxy_async();
       mbar_arrive(&ms.v_full[b]);
-      if (c + 1 < nch) {
-        fetch(c + 1, kblk_n, vblk_n);
-        lookup(c + 2, kblk_n, vblk_n);
+      if (c + 2 < nch) {
+        fetch(f, c + 2, kblk_n, vblk_n);
+        lookup(c + 3, kblk_n, vblk_n);
+      }
+      return true;
+    };
+    for (int c = 0; c < nch; c += 2) {
+      if (!run_chunk(fa, c) || (c + 1 < nch && !run_chunk(fb, c + 1))) {
+        raise_flag(a.status, OKV_DEV_TIMEOUT);
+        break;
       }
     }
   } else if (lane == 0) {
     // ------------------------------------------------------------ MMA issue
     // order: S(0), S(1), then per chunk c: O += P(c) V(c) as soon as the
-    // softmax of c is done, then S(c + 2) once its keys are staged (which
-    // needs the value MMA of c, the previous user of their buffer)
+    // softmax of c is done, then S(c + 2) once its keys are staged.  (Issuing
+    // S(c + 2) first measured slower: its wait on the keys then delays the
+    // value MMA, which the staging of the next values waits for.)
     uint64_t* last_bar = nullptr;  // the latest commit: it completes after every MMA issued before it
     uint32_t last_par = 0;
     auto issue_s = [&](int c) -> bool {
