@@ -543,7 +543,8 @@ __global__ void __launch_bounds__(kPfWarps * 32) prefill_attn_kernel(PrefillArgs
 //              applies the per-token scale and minimum term and the causal
 //              limit, meets its partner (the other half of the row) for the
 //              row maximum, keeps the online softmax state in registers, and
-//              writes p s (hi + lo fp16) as the A operand of the value MMA;
+//              writes p s (hi + lo fp16) into the chunk's score columns in
+//              TMEM, where the value MMA reads it as its A operand;
 //   warps 8-11 staging: the chunk's codes (or fp16 window / sink rows) into
 //              shared memory as fp16 tiles in the MMA's K-major layout --
 //              keys as [token][channel], values transposed to
@@ -552,6 +553,9 @@ __global__ void __launch_bounds__(kPfWarps * 32) prefill_attn_kernel(PrefillArgs
 //              S(c) = q~hi K^T + q~lo K^T (M 128, N 64, K 128) into one of
 //              two TMEM score buffers, O += (p s)hi V + (p s)lo V (M 128,
 //              N 128, K 64) into the TMEM output.
+// Both MMAs take their A operand from TMEM (q~ is staged there once; p s
+// replaces the scores it came from), so shared memory holds only the key and
+// value tiles and the MMAs read nothing else from it.
 // Two buffers of every per-chunk tile; mbarriers hand them around:
 //   k_full    staging -> MMA, softmax  (a chunk's key tile and key scales are in place)
 //   v_full    staging -> MMA, softmax  (its value tile and value scales)
@@ -573,14 +577,11 @@ constexpr int kUpSmxWarps = 8;   // warps 0..7
 constexpr int kUpStgWarps = 4;   // warps 8..11
 constexpr int kUpMmaWarp = 12;
 constexpr int kUpThreads = 32 * (kUpSmxWarps + kUpStgWarps + 1);
-constexpr uint32_t kUpQBytes = 4 * 16384;  // q~ hi and lo, 2 K-blocks of 128 rows x 128 B each
 constexpr uint32_t kUpKBytes = 2 * 8192;   // a chunk's keys: 2 K-blocks of 64 rows x 128 B
 constexpr uint32_t kUpVBytes = 16384;      // a chunk's values: 128 channel rows x 64 tokens
-constexpr uint32_t kUpPBytes = 2 * 16384;  // a chunk's p s: hi, lo, 128 rows x 64 tokens each
-constexpr uint32_t kUpOffK = kUpQBytes;
+constexpr uint32_t kUpOffK = 0;
 constexpr uint32_t kUpOffV = kUpOffK + 2 * kUpKBytes;
-constexpr uint32_t kUpOffP = kUpOffV + 2 * kUpVBytes;
-constexpr uint32_t kUpOffMisc = kUpOffP + 2 * kUpPBytes;
+constexpr uint32_t kUpOffMisc = kUpOffV + 2 * kUpVBytes;
 struct UpMisc {
   float2 ksm[2][kUpKC];             // key (scale, min) per token: (1, 0) for fp16 rows, (0, 0) masked
   float2 vsm[2][kUpKC];             // value (scale, min)
@@ -593,7 +594,10 @@ struct UpMisc {
   uint32_t tmem_slot;
 };
 constexpr size_t kUpSmem = 1024 + kUpOffMisc + sizeof(UpMisc);
-constexpr uint32_t kUpTmemCols = 256;  // scores: 2 x 64 columns; O: columns 128 .. 255
+// TMEM columns: scores (then p s: hi in the first 32, lo in the last 32) 2 x 64
+// from 0; O 128 from 128; q~ hi 64 from 256, q~ lo 64 from 320
+constexpr uint32_t kUpTmemCols = 512;
+constexpr uint32_t kUpColO = 128, kUpColQ = 256;
 constexpr uint32_t kUpIdescS = um_idesc(64, false, false);
 constexpr uint32_t kUpIdescO = um_idesc(128, false, false);
 constexpr uint32_t kF16Bias2 = 0x64006400u;  // (1024, 1024) as fp16 pair: 1024 + c is exact for c < 1024
@@ -657,7 +661,7 @@ __global__ void __launch_bounds__(kUpThreads, 1) prefill_umma_kernel(PrefillArgs
   const uint32_t base = (raw_u32 + 1023u) & ~1023u;  // swizzle atoms need 1024-byte alignment
   unsigned char* gb = up_raw + (base - raw_u32);
   UpMisc& ms = *reinterpret_cast<UpMisc*>(gb + kUpOffMisc);
-  const uint32_t sQ = base, sK = base + kUpOffK, sV = base + kUpOffV, sP = base + kUpOffP;
+  const uint32_t sK = base + kUpOffK, sV = base + kUpOffV;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int hk = blockIdx.y;
@@ -686,6 +690,7 @@ __global__ void __launch_bounds__(kUpThreads, 1) prefill_umma_kernel(PrefillArgs
   int rrow = 0, rpos = 0;
   bool rok = false;
   float qsum = 0.f, qup = 0.f;
+  uint32_t qrow[64];  // this thread's half of its q~ row (fp16 pairs), until it is in TMEM
   const int quarter = warp & 3, hcol = (warp >> 2) & 1;  // softmax: lane quarter, column half
   const int rowc = 32 * quarter + lane;                    // softmax: row in the tile (TMEM lane)
   if (warp < kUpSmxWarps) {
@@ -695,20 +700,20 @@ __global__ void __launch_bounds__(kUpThreads, 1) prefill_umma_kernel(PrefillArgs
     const int rtok = rr / a.g;
     rrow = rtok * a.hq + hk * a.g + rr % a.g;
     rpos = a.first + rtok;
-    {  // column half 0 stages the row's hi half of q~, half 1 the lo half
+    {  // column half 0 takes the row's hi half of q~, half 1 the lo half (to TMEM below)
       const uint4* src = reinterpret_cast<const uint4*>((hcol ? a.qlo : a.qhi) + (size_t)rrow * kD);
 #pragma unroll
       for (int c16 = 0; c16 < 16; ++c16) {
         const uint4 x = src[c16];
-        const uint32_t off =
-            (uint32_t)(2 * hcol + (c16 >> 3)) * 16384u + um_swz((uint32_t)rowc, (uint32_t)(c16 & 7) * 16u);
-        *reinterpret_cast<uint4*>(gb + off) = x;
+        qrow[4 * c16] = x.x;
+        qrow[4 * c16 + 1] = x.y;
+        qrow[4 * c16 + 2] = x.z;
+        qrow[4 * c16 + 3] = x.w;
       }
     }
     const float* aux = a.qaux + (size_t)rrow * kQaux;
     qsum = aux[0] * (kInvSqrtD * kLog2e);
     qup = aux[4] * (kInvSqrtD * kLog2e);
-    um_fence_proxy_async();  // generic stores, read by the MMA through the async proxy
   }
 
   // ---- staging: per-thread roles and the register-held fetch of one chunk
@@ -930,7 +935,18 @@ __global__ void __launch_bounds__(kUpThreads, 1) prefill_umma_kernel(PrefillArgs
   __syncthreads();
   um_fence_after();
   const uint32_t tmem = ms.tmem_slot;
-  const uint32_t tS = tmem, tO = tmem + 128u;
+  const uint32_t tS = tmem, tO = tmem + kUpColO, tQ = tmem + kUpColQ;
+  if (warp < kUpSmxWarps) {  // q~ of this warp's 32 rows: half hcol into columns 64 hcol ..
+    const uint32_t ta = tQ + ((uint32_t)(32 * quarter) << 16) + 64u * (uint32_t)hcol;
+    um_st16(ta, qrow);
+    um_st16(ta + 16u, qrow + 16);
+    um_st16(ta + 32u, qrow + 32);
+    um_st16(ta + 48u, qrow + 48);
+    um_wait_st();
+  }
+  um_fence_before();
+  __syncthreads();  // q~ is in TMEM before the first score MMA
+  um_fence_after();
 
   if (warp < kUpSmxWarps) {
     // ------------------------------------------------------------ softmax
@@ -1021,17 +1037,16 @@ __global__ void __launch_bounds__(kUpThreads, 1) prefill_umma_kernel(PrefillArgs
       }
       const float mref = m_use == -INFINITY ? 0.f : m_use;
       const float2 nm2 = make_float2(-mref, -mref);
-      // p s into the A tiles of chunk c, once the value MMA of chunk c - 2 has read them
-      if (c >= 2) {
-        alive = mbar_wait_bounded(&ms.pv_done[b], ((uint32_t)(c - 2) >> 1) & 1u);
-        alive = __all_sync(0xffffffffu, alive);
-        if (!alive) break;
-      }
-      unsigned char* pg = gb + (sP + (uint32_t)b * kUpPBytes - base);
+      // p s over the scores of chunk c in TMEM: columns 16 hcol .. (hi) and
+      // 32 + 16 hcol .. (lo) of the chunk's buffer.  The lo columns held the
+      // partner's scores, which it read before it posted its maximum; the
+      // value MMA of chunk c - 2, the last reader of this buffer's p s,
+      // finished before S(c) was written into it.
+      um_fence_after();
       const float4* v4p = reinterpret_cast<const float4*>(&ms.vsm[b][32 * hcol]);
+      uint32_t hi[16], lo[16];
 #pragma unroll
       for (int j8 = 0; j8 < 4; ++j8) {
-        uint32_t hi[4], lo[4];
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
           const int j2 = 4 * j8 + u;
@@ -1045,14 +1060,14 @@ __global__ void __launch_bounds__(kUpThreads, 1) prefill_umma_kernel(PrefillArgs
           const float2 wh = make_float2(__uint_as_float(__float_as_uint(w.x) & 0xFFFFE000u),
                                         __uint_as_float(__float_as_uint(w.y) & 0xFFFFE000u));
           const float2 wl = __fadd2_rn(w, make_float2(-wh.x, -wh.y));
-          hi[u] = pack_half2(wh.x, wh.y);
-          lo[u] = pack_half2(wl.x, wl.y);
+          hi[j2] = pack_half2(wh.x, wh.y);
+          lo[j2] = pack_half2(wl.x, wl.y);
         }
-        const uint32_t off = um_swz((uint32_t)rowc, (uint32_t)(4 * hcol + j8) * 16u);
-        *reinterpret_cast<uint4*>(pg + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-        *reinterpret_cast<uint4*>(pg + 16384u + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
       }
-      um_fence_proxy_async();
+      const uint32_t tp = tS + lane_base + (uint32_t)(b * kUpKC + 16 * hcol);
+      um_st16(tp, hi);
+      um_st16(tp + 32u, lo);
+      um_wait_st();
       um_fence_before();
       mbar_arrive(&ms.p_full[b]);
     }
@@ -1137,9 +1152,10 @@ __global__ void __launch_bounds__(kUpThreads, 1) prefill_umma_kernel(PrefillArgs
         for (int kb = 0; kb < 2; ++kb)
 #pragma unroll
           for (int ks = 0; ks < 4; ++ks) {
-            const uint64_t ad = um_desc(sQ + (uint32_t)(2 * half + kb) * 16384u + (uint32_t)ks * 32u);
+            // q~ channels 64 kb + 16 ks .. + 15: TMEM columns 8 (4 kb + ks) of its half
+            const uint32_t ta = tQ + 64u * (uint32_t)half + 8u * (uint32_t)(4 * kb + ks);
             const uint64_t bd = um_desc(kt + (uint32_t)kb * 8192u + (uint32_t)ks * 32u);
-            um_mma(tS + (uint32_t)(b * kUpKC), ad, bd, kUpIdescS, (half | kb | ks) != 0 ? 1u : 0u);
+            um_mma_ts(tS + (uint32_t)(b * kUpKC), ta, bd, kUpIdescS, (half | kb | ks) != 0 ? 1u : 0u);
           }
       um_commit(&ms.s_full[b]);
       last_bar = &ms.s_full[b];
@@ -1151,14 +1167,15 @@ __global__ void __launch_bounds__(kUpThreads, 1) prefill_umma_kernel(PrefillArgs
       if (!mbar_wait_bounded(&ms.p_full[b], ((uint32_t)c >> 1) & 1u)) return false;
       if (!mbar_wait_bounded(&ms.v_full[b], ((uint32_t)c >> 1) & 1u)) return false;
       um_fence_after();
-      const uint32_t pt = sP + (uint32_t)b * kUpPBytes, vt2 = sV + (uint32_t)b * kUpVBytes;
+      const uint32_t vt2 = sV + (uint32_t)b * kUpVBytes;
 #pragma unroll
       for (int half = 0; half < 2; ++half)
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks) {
-          const uint64_t ad = um_desc(pt + (uint32_t)half * 16384u + (uint32_t)ks * 32u);
+          // tokens 16 ks .. + 15 of p s (hi or lo): TMEM columns 32 half + 8 ks of the chunk's buffer
+          const uint32_t ta = tS + (uint32_t)(b * kUpKC) + 32u * (uint32_t)half + 8u * (uint32_t)ks;
           const uint64_t bd = um_desc(vt2 + (uint32_t)ks * 32u);
-          um_mma(tO, ad, bd, kUpIdescO, (c > 0 || half > 0 || ks > 0) ? 1u : 0u);
+          um_mma_ts(tO, ta, bd, kUpIdescO, (c > 0 || half > 0 || ks > 0) ? 1u : 0u);
         }
       um_commit(&ms.pv_done[b]);
       last_bar = &ms.pv_done[b];
