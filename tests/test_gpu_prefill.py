@@ -156,3 +156,45 @@ def test_prefill_rejects_bad_arguments():
     small = torch.empty(256, dtype=torch.uint8, device="cuda")
     with pytest.raises(okv.OkvError):
         okv.prefill_attention(gc, q, 0, 100, tb, ws=small)
+
+
+def test_prefill_bad_block_is_flagged_and_skipped():
+    """A block id outside the pool in the middle of the INT2 history: the
+    kernel raises OKV_DEV_BAD_BLOCK and attends as if those 16 positions were
+    absent (the oracle's attention over the remaining positions)."""
+    okv = _okv()
+    seed, hq, hkv, L, T = 60, 8, 2, 2000, 100
+    lay = H.Layout(seed, [L])
+    uk, uv = H.rotations(seed, hkv)
+    gc = okv.Cache(hq, hkv, lay.num_blocks, 1, lay.mbps, uk, uv)
+    zk = np.stack([WL.sample_rotated(seed, 0, 0, h, L, 0) for h in range(hkv)], 1)
+    zv = np.stack([WL.sample_rotated(seed, 0, 0, h, L, 1) for h in range(hkv)], 1)
+    slots, pos = lay.flat()
+    okv.append_quantize(gc, _t(zk), _t(zv), _t(slots), _t(pos), _t(lay.table), _t(np.array([L], np.int32)),
+                        pre_rotated=True)
+    torch.cuda.synchronize()
+    assert gc.device_status() == 0
+    table = lay.table.copy()
+    bad = 10                                   # positions 160 .. 175, INT2 for every row of the chunk
+    table[0, bad] = lay.num_blocks + 3
+    G = hq // hkv
+    q = np.stack([WL.sample_queries(seed, 0, 0, h, T, G, extra=9) for h in range(hkv)], 1).reshape(T, hq, 128)
+    got = okv.prefill_attention(gc, _t(q, torch.bfloat16), 0, L, _t(table)).cpu().numpy()
+    assert gc.device_status() & okv.DEV_BAD_BLOCK
+    assert np.all(np.isfinite(got))
+    first = L - T
+    keep = np.ones(L, bool)
+    keep[16 * bad:16 * bad + 16] = False
+    for hk in range(hkv):
+        oc = O.Cache(1, uk[hk:hk + 1].astype(np.float64), uv[hk:hk + 1].astype(np.float64))
+        oc.append(0, 0, zk[:, hk:hk + 1], zv[:, hk:hk + 1], pre_rotated=True)
+        kx, vx = oc.values(0, 0, 0, L), oc.values(0, 1, 0, L)
+        for i in (0, 50, T - 1):
+            vis = np.zeros(L, bool)
+            vis[:first + i + 1] = True
+            sel = vis & keep
+            for h in range(hk * G, (hk + 1) * G):
+                qr = q[i, h].astype(np.float64) @ oc.r[0][0]
+                want = O.attend(qr, kx[sel], vx[sel]) @ oc.r[1][0].T
+                err = np.abs(got[i, h] - want).max() / np.abs(want).max()
+                assert err <= TOL, (hk, i, h, err)
