@@ -522,7 +522,7 @@ def prefill_append_rate(torch, okv, WL, seed):
             "timing": "median of 50 launches, L2 flushed before each"}
 
 
-def prefill_attention_rate(torch, okv, WL, seed, L=32768, T=1024):
+def prefill_attention_rate(torch, okv, WL, seed, L=32768, T=1024, group=128):
     """Chunked-prefill attention: a T-token chunk at the end of an L-token
     sequence (32 query / 8 KV heads) attends causally over the cache; median
     of 50 calls (query rotation, attention, un-rotation), L2 flushed before
@@ -533,7 +533,7 @@ def prefill_attention_rate(torch, okv, WL, seed, L=32768, T=1024):
     table, nb = WL.block_table(seed, 1, [L], extra_tokens=16)
     r = np.random.default_rng(seed + 5)
     uk = np.stack([WL.haar_orthogonal(r) for _ in range(hkv)]).astype(np.float32)
-    cache = okv.Cache(hq, hkv, nb, 1, table.shape[1], uk, uk)
+    cache = okv.Cache(hq, hkv, nb, 1, table.shape[1], uk, uk, group=group)
     dev = torch.device("cuda")
     td = torch.from_numpy(table).to(dev)
     gen, kv = _kv_source(torch, WL, seed, 1, 0, hkv, dev)
@@ -549,7 +549,8 @@ def prefill_attention_rate(torch, okv, WL, seed, L=32768, T=1024):
     flops = 4 * 128 * hq * visible
     peak, src = measured_peak_bf16()
     tflops = flops / us / 1e6
-    return {"context": L, "chunk_tokens": T, "hq": hq, "hkv": hkv, "us": round(us, 1),
+    return {"context": L, "chunk_tokens": T, "hq": hq, "hkv": hkv, "group": group,
+            "kernel": "tcgen05" if group == 128 else "mma.sync (per-group scales)", "us": round(us, 1),
             "tflops": round(tflops, 1), "flops": flops,
             "roofline": {"bound": "tensor", "achieved": round(tflops, 1), "peak": peak, "unit": "TFLOP/s",
                          "frac": round(tflops / peak, 4), "peak_source": src,
@@ -864,7 +865,8 @@ def run_ours(args):
 
     e2e = run_e2e(w, W + K, e2e_steps, torch, okv, world, dist) if e2e_steps else None
     append_rate = prefill_append_rate(torch, okv, WL, args.seed) if rank == 0 else None
-    prefill_rate = prefill_attention_rate(torch, okv, WL, args.seed) if rank == 0 and args.workload == 2 else None
+    prefill_rate = (prefill_attention_rate(torch, okv, WL, args.seed, group=args.group)
+                    if rank == 0 and args.workload == 2 else None)
 
     if rank == 0:
         alg = statistics.mean(statistics.mean(w.decode_bytes(W + i)) for i in range(K))
