@@ -534,7 +534,9 @@ __global__ void __launch_bounds__(kPfWarps * 32) prefill_attn_kernel(PrefillArgs
 }
 
 // ---------------------------------------------------------------------------
-// 2b. attention on the tcgen05 tensor cores (128-channel groups).  A CTA takes
+// 2b. attention on the tcgen05 tensor cores (128- and 64-channel groups, NG =
+// 1 or 2 groups per vector; a group is one 64-channel K-block or both, and its
+// scores, p s and value MMA are kept apart).  A CTA takes
 // 128 query rows of one KV head (the MMA's M) and streams the key positions
 // in chunks of 64 (four cache blocks), with warp roles:
 //   warps 0-7  softmax: warp w serves rows 32 (w % 4) .. + 31 (TMEM lanes,
@@ -583,23 +585,25 @@ constexpr uint32_t kUpOffK = 0;
 constexpr uint32_t kUpOffV = kUpOffK + 2 * kUpKBytes;
 constexpr uint32_t kUpOffMisc = kUpOffV + 2 * kUpVBytes;
 struct UpMisc {
-  float2 ksm[2][kUpKC];             // key (scale, min) per token: (1, 0) for fp16 rows, (0, 0) masked
-  float2 vsm[2][kUpKC];             // value (scale, min)
+  float2 ksm[2][2 * kUpKC];         // key (scale, min) of token j, group k at j NG + k: (1, 0) fp16 rows, (0, 0) masked
+  float2 vsm[2][2 * kUpKC];         // value (scale, min), the same way
   int kval[2][kUpKC];               // 1 where the token was staged (only read when a block id was bad)
   float vsmax[2][kUpStgWarps];      // largest value scale, per staging warp
   int bad[2][kUpStgWarps];          // a block id was out of range, per staging warp
   float red[2][2][128];             // per chunk parity, column half, row: the half-row maximum
-  float2 fin[2][128];               // per column half, row: (l, sum p m) at the end
+  float4 fin[2][128];               // per column half, row: (l, sum p m of group 0, of group 1) at the end
   uint64_t k_full[2], v_full[2], s_full[2], s_free[2], p_full[2], pv_done[2], mx[4][2];
   uint32_t tmem_slot;
 };
 constexpr size_t kUpSmem = 1024 + kUpOffMisc + sizeof(UpMisc);
-// TMEM columns: scores (then p s: hi in the first 32, lo in the last 32) 2 x 64
-// from 0; O 128 from 128; q~ hi 64 from 256, q~ lo 64 from 320
+// TMEM columns: scores 2 x 64 NG from 0 (group k's 64 columns at 64 k; p s
+// of a group then replaces its scores: per column half h of the row, hi at
+// 32 h + 0..15 and lo at 32 h + 16..31 of the group's columns); O 128 from
+// 128 NG; q~ hi 64 and lo 64 after O
 constexpr uint32_t kUpTmemCols = 512;
-constexpr uint32_t kUpColO = 128, kUpColQ = 256;
 constexpr uint32_t kUpIdescS = um_idesc(64, false, false);
 constexpr uint32_t kUpIdescO = um_idesc(128, false, false);
+constexpr uint32_t kUpIdescO64 = um_idesc(64, false, false);
 constexpr uint32_t kF16Bias2 = 0x64006400u;  // (1024, 1024) as fp16 pair: 1024 + c is exact for c < 1024
 
 // (1024 + lo, 1024 + hi) - 1024 for two 2-bit codes already in bits 0-1 and 16-17
@@ -655,7 +659,11 @@ __device__ __forceinline__ float ex2_ftz(float x) {
   return y;
 }
 
+template <int NG>
 __global__ void __launch_bounds__(kUpThreads, 1) prefill_umma_kernel(PrefillArgs a) {
+  static_assert(NG == 1 || NG == 2, "one or two 64-channel groups per vector");
+  constexpr int kSW = 64 * NG;  // score columns per buffer
+  constexpr uint32_t kUpColO = 2 * kSW, kUpColQ = 2 * kSW + 128;
   extern __shared__ unsigned char up_raw[];
   const uint32_t raw_u32 = smem_u32(up_raw);
   const uint32_t base = (raw_u32 + 1023u) & ~1023u;  // swizzle atoms need 1024-byte alignment
@@ -728,7 +736,7 @@ __global__ void __launch_bounds__(kUpThreads, 1) prefill_umma_kernel(PrefillArgs
     int p0;                   // first position of the chunk
     uint4 kr0;                // INT2 key codes of the token (64 channels)
     uint4 vw;                 // INT2 value codes of the quad (16 channels x 4 tokens)
-    uint32_t ksmw;            // the token's (scale, min): key scales for kkb 0, value scales for kkb 1
+    uint32_t ksmw[NG];        // the token's (scale, min) per group: key scales for kkb 0, value scales for kkb 1
   };
   Fetched fa, fb;
   // block ids of this thread's key token and value quad, looked up one chunk
@@ -775,7 +783,9 @@ __global__ void __launch_bounds__(kUpThreads, 1) prefill_umma_kernel(PrefillArgs
       if (kok) {
         const uint8_t* bp = a.pages + ((size_t)kblk * a.hkv + hk) * a.bhb;
         f.kr0 = *reinterpret_cast<const uint4*>(bp + kKcOff + (ktk & 15) * 32 + 16 * kkb);
-        f.ksmw = *reinterpret_cast<const uint32_t*>(bp + sm_offset(1, kkb, ktk & 15, 0));
+#pragma unroll
+        for (int k = 0; k < NG; ++k)
+          f.ksmw[k] = *reinterpret_cast<const uint32_t*>(bp + sm_offset(NG, kkb, ktk & 15, k));
       }
 #pragma unroll
       for (int i = 0; i < 4; ++i) f.vsrc[i] = vok ? 1 : 0;
@@ -790,7 +800,9 @@ __global__ void __launch_bounds__(kUpThreads, 1) prefill_umma_kernel(PrefillArgs
       f.ksrc = locate(f, p, kblk, &bp);
       if (f.ksrc == 1) {
         f.kr0 = *reinterpret_cast<const uint4*>(bp + kKcOff + (p & 15) * 32 + 16 * kkb);
-        f.ksmw = *reinterpret_cast<const uint32_t*>(bp + sm_offset(1, kkb, p & 15, 0));
+#pragma unroll
+        for (int k = 0; k < NG; ++k)
+          f.ksmw[k] = *reinterpret_cast<const uint32_t*>(bp + sm_offset(NG, kkb, p & 15, k));
       }
     }
     {
@@ -809,11 +821,11 @@ __global__ void __launch_bounds__(kUpThreads, 1) prefill_umma_kernel(PrefillArgs
     }
   };
   // (scale, min) of the fetched token: key scales for kkb 0, value scales for kkb 1
-  auto token_sm = [&](const Fetched& f, float& s_, float& m_) {
+  auto token_sm = [&](const Fetched& f, int k, float& s_, float& m_) {
     s_ = m_ = 0.f;
     if (f.ksrc == 1) {
-      s_ = __half2float(__ushort_as_half((unsigned short)(f.ksmw & 0xffffu)));
-      m_ = __half2float(__ushort_as_half((unsigned short)(f.ksmw >> 16)));
+      s_ = __half2float(__ushort_as_half((unsigned short)(f.ksmw[k] & 0xffffu)));
+      m_ = __half2float(__ushort_as_half((unsigned short)(f.ksmw[k] >> 16)));
     } else if (f.ksrc == 2) {
       s_ = 1.f;
     }
@@ -841,9 +853,12 @@ __global__ void __launch_bounds__(kUpThreads, 1) prefill_umma_kernel(PrefillArgs
             f.ksrc == 2 ? x[jc] : make_uint4(0, 0, 0, 0);
     }
     if (kkb == 0) {
-      float s_, m_;
-      token_sm(f, s_, m_);
-      ms.ksm[b][ktk] = make_float2(s_, m_);
+#pragma unroll
+      for (int k = 0; k < NG; ++k) {
+        float s_, m_;
+        token_sm(f, k, s_, m_);
+        ms.ksm[b][ktk * NG + k] = make_float2(s_, m_);
+      }
       ms.kval[b][ktk] = f.ksrc != 0;
     }
     const int anybad = __any_sync(0xffffffffu, f.sbad != 0);
@@ -856,14 +871,17 @@ __global__ void __launch_bounds__(kUpThreads, 1) prefill_umma_kernel(PrefillArgs
   auto stage_v = [&](const Fetched& f, int b) {
     float vmx = 0.f;
     if (kkb == 1) {
-      float s_, m_;
-      token_sm(f, s_, m_);
-      if (f.ksrc == 1) {
-        ms.vsm[b][ktk] = make_float2(0.5f * s_, fmaf(1.5f, s_, m_));  // centred codes
-        vmx = 0.5f * s_;
-      } else {
-        ms.vsm[b][ktk] = make_float2(s_, m_);
-        vmx = s_;
+#pragma unroll
+      for (int k = 0; k < NG; ++k) {
+        float s_, m_;
+        token_sm(f, k, s_, m_);
+        if (f.ksrc == 1) {
+          ms.vsm[b][ktk * NG + k] = make_float2(0.5f * s_, fmaf(1.5f, s_, m_));  // centred codes
+          vmx = fmaxf(vmx, 0.5f * s_);
+        } else {
+          ms.vsm[b][ktk * NG + k] = make_float2(s_, m_);
+          vmx = fmaxf(vmx, s_);
+        }
       }
     }
 #pragma unroll
@@ -952,8 +970,13 @@ __global__ void __launch_bounds__(kUpThreads, 1) prefill_umma_kernel(PrefillArgs
     // ------------------------------------------------------------ softmax
     const uint32_t lane_base = (uint32_t)(32 * quarter) << 16;
     float m_use = -INFINITY;
-    float2 l2 = make_float2(0.f, 0.f), msum2 = make_float2(0.f, 0.f);  // two partial sums each
+    float2 l2 = make_float2(0.f, 0.f), msum2[NG];  // two partial sums each (paired arithmetic)
+#pragma unroll
+    for (int k = 0; k < NG; ++k) msum2[k] = make_float2(0.f, 0.f);
     const float2 qup2 = make_float2(qup, qup), qsum2 = make_float2(qsum, qsum);
+    float qsum_g[NG];  // per-group sums of q~ (log2 units)
+#pragma unroll
+    for (int k = 0; k < NG; ++k) qsum_g[k] = a.qaux[(size_t)rrow * kQaux + k] * (kInvSqrtD * kLog2e);
     bool alive = true;
     for (int c = 0; c < nch && alive; ++c) {
       const int b = c & 1;
@@ -963,7 +986,20 @@ __global__ void __launch_bounds__(kUpThreads, 1) prefill_umma_kernel(PrefillArgs
       if (!alive) break;
       um_fence_after();
       float sv[32];
-      um_ld32(tS + lane_base + (uint32_t)(b * kUpKC + 32 * hcol), sv);
+      um_ld32(tS + lane_base + (uint32_t)(b * kSW + 32 * hcol), sv);
+      if constexpr (NG == 2) {
+        // x = s0 (q~0 . c0) + m0 sum q~0 + s1 (q~1 . c1) + m1 sum q~1: group 1's raw scores
+        // and both groups' (scale, min) fold in here; the common code below then sees s = 1, m = 0
+        float sv1[32];
+        um_ld32(tS + lane_base + (uint32_t)(b * kSW + 64 + 32 * hcol), sv1);
+        um_wait_ld();
+        const float4* kk = reinterpret_cast<const float4*>(&ms.ksm[b][2 * 32 * hcol]);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const float4 k4 = kk[j];  // (s, m) of groups 0 and 1 of token j
+          sv[j] = fmaf(k4.x * qup, sv[j], fmaf(k4.y, qsum_g[0], fmaf(k4.z * qup, sv1[j], k4.w * qsum_g[1])));
+        }
+      }
       um_wait_ld();
       um_fence_before();
       // scores in log2 units: s (q~ . c) 2^e / sqrt(d) + m sum(q~) / sqrt(d); columns j < lim are
@@ -972,7 +1008,15 @@ __global__ void __launch_bounds__(kUpThreads, 1) prefill_umma_kernel(PrefillArgs
       const bool bad = (ms.bad[b][0] | ms.bad[b][1] | ms.bad[b][2] | ms.bad[b][3]) != 0;
       const float4* k4p = reinterpret_cast<const float4*>(&ms.ksm[b][32 * hcol]);
       float bm = -INFINITY;
-      if (lim >= 32 && !bad) {
+      if constexpr (NG == 2) {
+        const int* kv = &ms.kval[b][32 * hcol];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const bool ok = j < lim && (!bad || kv[j] != 0);
+          sv[j] = ok ? sv[j] : -INFINITY;
+          bm = fmaxf(bm, sv[j]);
+        }
+      } else if (lim >= 32 && !bad) {
 #pragma unroll
         for (int j2 = 0; j2 < 16; ++j2) {
           const float4 k4 = k4p[j2];  // (s, m) of columns 2 j2, 2 j2 + 1
@@ -1032,7 +1076,8 @@ __global__ void __launch_bounds__(kUpThreads, 1) prefill_umma_kernel(PrefillArgs
           um_wait_st();
         }
         l2 = __fmul2_rn(l2, make_float2(alpha, alpha));
-        msum2 = __fmul2_rn(msum2, make_float2(alpha, alpha));
+#pragma unroll
+        for (int k = 0; k < NG; ++k) msum2[k] = __fmul2_rn(msum2[k], make_float2(alpha, alpha));
         if (need) m_use = bm;
       }
       const float mref = m_use == -INFINITY ? 0.f : m_use;
@@ -1043,19 +1088,18 @@ __global__ void __launch_bounds__(kUpThreads, 1) prefill_umma_kernel(PrefillArgs
       // value MMA of chunk c - 2, the last reader of this buffer's p s,
       // finished before S(c) was written into it.
       um_fence_after();
-      const float4* v4p = reinterpret_cast<const float4*>(&ms.vsm[b][32 * hcol]);
-      uint32_t hi[16], lo[16];
 #pragma unroll
-      for (int j8 = 0; j8 < 4; ++j8) {
+      for (int k = 0; k < NG; ++k) {
+        // group k: p s_k over this thread's 32 scores of group k (p is recomputed per group)
+        uint32_t hi[16], lo[16];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int j2 = 4 * j8 + u;
+        for (int j2 = 0; j2 < 16; ++j2) {
           const float2 d = __fadd2_rn(make_float2(sv[2 * j2], sv[2 * j2 + 1]), nm2);
           const float2 pp = make_float2(ex2_ftz(d.x), ex2_ftz(d.y));
-          const float4 vs = v4p[j2];  // (s, m) of columns 2 j2, 2 j2 + 1
-          l2 = __fadd2_rn(l2, pp);
-          msum2 = __ffma2_rn(pp, make_float2(vs.y, vs.w), msum2);
-          const float2 w = __fmul2_rn(pp, make_float2(vs.x, vs.z));
+          const float2 v0 = ms.vsm[b][(32 * hcol + 2 * j2) * NG + k], v1 = ms.vsm[b][(32 * hcol + 2 * j2 + 1) * NG + k];
+          if (k == 0) l2 = __fadd2_rn(l2, pp);
+          msum2[k] = __ffma2_rn(pp, make_float2(v0.y, v1.y), msum2[k]);
+          const float2 w = __fmul2_rn(pp, make_float2(v0.x, v1.x));
           // hi: w with its low 13 mantissa bits cleared (exact in fp16 from 2^-14 up); lo: the rest
           const float2 wh = make_float2(__uint_as_float(__float_as_uint(w.x) & 0xFFFFE000u),
                                         __uint_as_float(__float_as_uint(w.y) & 0xFFFFE000u));
@@ -1063,10 +1107,14 @@ __global__ void __launch_bounds__(kUpThreads, 1) prefill_umma_kernel(PrefillArgs
           hi[j2] = pack_half2(wh.x, wh.y);
           lo[j2] = pack_half2(wl.x, wl.y);
         }
+        // NG = 1: hi at 16 hcol, lo at 32 + 16 hcol (the lo columns held the partner's
+        // scores, read before it posted its maximum); NG = 2: over this thread's own
+        // 32 score columns of group k
+        const uint32_t tp = tS + lane_base + (uint32_t)(b * kSW) +
+                            (NG == 1 ? 16u * (uint32_t)hcol : 64u * (uint32_t)k + 32u * (uint32_t)hcol);
+        um_st16(tp, hi);
+        um_st16(tp + (NG == 1 ? 32u : 16u), lo);
       }
-      const uint32_t tp = tS + lane_base + (uint32_t)(b * kUpKC + 16 * hcol);
-      um_st16(tp, hi);
-      um_st16(tp + 32u, lo);
       um_wait_st();
       um_fence_before();
       mbar_arrive(&ms.p_full[b]);
@@ -1078,13 +1126,15 @@ __global__ void __launch_bounds__(kUpThreads, 1) prefill_umma_kernel(PrefillArgs
     float l = 0.f, msum = 0.f;
     if (alive) {
       // the two halves' sums meet: one more round of the partners' barrier
-      ms.fin[hcol][rowc] = make_float2(l2.x + l2.y, msum2.x + msum2.y);
+      ms.fin[hcol][rowc] = make_float4(l2.x + l2.y, msum2[0].x + msum2[0].y,
+                                       NG == 2 ? msum2[NG - 1].x + msum2[NG - 1].y : 0.f, 0.f);
       mbar_arrive(&ms.mx[quarter][nch & 1]);
       alive = mbar_wait_bounded(&ms.mx[quarter][nch & 1], ((uint32_t)nch >> 1) & 1u);
       alive = __all_sync(0xffffffffu, alive);
-      const float2 f0 = ms.fin[0][rowc], f1 = ms.fin[1][rowc];
+      const float4 f0 = ms.fin[0][rowc], f1 = ms.fin[1][rowc];
       l = f0.x + f1.x;
-      msum = f0.y + f1.y;
+      // this thread writes channels 64 hcol ..: group hcol when NG = 2
+      msum = (NG == 2 && hcol == 1) ? f0.z + f1.z : f0.y + f1.y;
     }
     if (alive) {
       um_fence_after();
@@ -1155,7 +1205,9 @@ __global__ void __launch_bounds__(kUpThreads, 1) prefill_umma_kernel(PrefillArgs
             // q~ channels 64 kb + 16 ks .. + 15: TMEM columns 8 (4 kb + ks) of its half
             const uint32_t ta = tQ + 64u * (uint32_t)half + 8u * (uint32_t)(4 * kb + ks);
             const uint64_t bd = um_desc(kt + (uint32_t)kb * 8192u + (uint32_t)ks * 32u);
-            um_mma_ts(tS + (uint32_t)(b * kUpKC), ta, bd, kUpIdescS, (half | kb | ks) != 0 ? 1u : 0u);
+            // NG = 2: K-block kb is group kb, into its own 64 columns
+            um_mma_ts(tS + (uint32_t)(b * kSW) + (NG == 2 ? 64u * (uint32_t)kb : 0u), ta, bd, kUpIdescS,
+                      (half | ks | (NG == 2 ? 0 : kb)) != 0 ? 1u : 0u);
           }
       um_commit(&ms.s_full[b]);
       last_bar = &ms.s_full[b];
@@ -1168,15 +1220,31 @@ __global__ void __launch_bounds__(kUpThreads, 1) prefill_umma_kernel(PrefillArgs
       if (!mbar_wait_bounded(&ms.v_full[b], ((uint32_t)c >> 1) & 1u)) return false;
       um_fence_after();
       const uint32_t vt2 = sV + (uint32_t)b * kUpVBytes;
+      if constexpr (NG == 1) {
 #pragma unroll
-      for (int half = 0; half < 2; ++half)
+        for (int half = 0; half < 2; ++half)
 #pragma unroll
-        for (int ks = 0; ks < 4; ++ks) {
-          // tokens 16 ks .. + 15 of p s (hi or lo): TMEM columns 32 half + 8 ks of the chunk's buffer
-          const uint32_t ta = tS + (uint32_t)(b * kUpKC) + 32u * (uint32_t)half + 8u * (uint32_t)ks;
-          const uint64_t bd = um_desc(vt2 + (uint32_t)ks * 32u);
-          um_mma_ts(tO, ta, bd, kUpIdescO, (c > 0 || half > 0 || ks > 0) ? 1u : 0u);
-        }
+          for (int ks = 0; ks < 4; ++ks) {
+            // tokens 16 ks .. + 15 of p s (hi or lo): TMEM columns 32 half + 8 ks of the chunk's buffer
+            const uint32_t ta = tS + (uint32_t)(b * kSW) + 32u * (uint32_t)half + 8u * (uint32_t)ks;
+            const uint64_t bd = um_desc(vt2 + (uint32_t)ks * 32u);
+            um_mma_ts(tO, ta, bd, kUpIdescO, (c > 0 || half > 0 || ks > 0) ? 1u : 0u);
+          }
+      } else {
+#pragma unroll
+        for (int k = 0; k < 2; ++k)
+#pragma unroll
+          for (int half = 0; half < 2; ++half)
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks) {
+              // group k, tokens 16 ks ..: p s written by column half ks / 2 at 32 (ks / 2) +
+              // 16 half + 8 (ks % 2) of the group's columns; values: channel rows 64 k ..
+              const uint32_t ta = tS + (uint32_t)(b * kSW) + 64u * (uint32_t)k + 32u * (uint32_t)(ks >> 1) +
+                                  16u * (uint32_t)half + 8u * (uint32_t)(ks & 1);
+              const uint64_t bd = um_desc(vt2 + (uint32_t)k * 8192u + (uint32_t)ks * 32u);
+              um_mma_ts(tO + 64u * (uint32_t)k, ta, bd, kUpIdescO64, (c > 0 || half > 0 || ks > 0) ? 1u : 0u);
+            }
+      }
       um_commit(&ms.pv_done[b]);
       last_bar = &ms.pv_done[b];
       last_par = ((uint32_t)c >> 1) & 1u;
@@ -1326,12 +1394,18 @@ okv_status launch_prefill(const okv_cache_desc* d, const void* q, int T, int slo
   switch (a.ng) {
     case 1: {
       static std::atomic<uint32_t> up_attr{0};
-      cudaError_t e1 = set_smem_limit_once((const void*)prefill_umma_kernel, (int)kUpSmem, up_attr);
+      cudaError_t e1 = set_smem_limit_once((const void*)prefill_umma_kernel<1>, (int)kUpSmem, up_attr);
       if (e1 != cudaSuccess) return fail(OKV_ERR_CUDA, "prefill attention smem attribute: %s", cudaGetErrorString(e1));
-      prefill_umma_kernel<<<grid, kUpThreads, kUpSmem, s>>>(a);
+      prefill_umma_kernel<1><<<grid, kUpThreads, kUpSmem, s>>>(a);
       break;
     }
-    case 2: prefill_attn_kernel<2><<<grid, kPfWarps * 32, 0, s>>>(a); break;
+    case 2: {
+      static std::atomic<uint32_t> up2_attr{0};
+      cudaError_t e1 = set_smem_limit_once((const void*)prefill_umma_kernel<2>, (int)kUpSmem, up2_attr);
+      if (e1 != cudaSuccess) return fail(OKV_ERR_CUDA, "prefill attention smem attribute: %s", cudaGetErrorString(e1));
+      prefill_umma_kernel<2><<<grid, kUpThreads, kUpSmem, s>>>(a);
+      break;
+    }
     default: prefill_attn_kernel<4><<<grid, kPfWarps * 32, 0, s>>>(a); break;
   }
   st = check_launch("prefill attention");
