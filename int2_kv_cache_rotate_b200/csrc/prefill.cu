@@ -1190,12 +1190,17 @@ __global__ void __launch_bounds__(kUpThreads, 1) prefill_umma_kernel(PrefillArgs
     // value MMA, which the staging of the next values waits for.)
     uint64_t* last_bar = nullptr;  // the latest commit: it completes after every MMA issued before it
     uint32_t last_par = 0;
+    // Descriptors: a tile's base descriptor plus (byte offset >> 4) in the start
+    // address field (shared addresses stay below 2^18, so the field never
+    // carries), which keeps this thread's per-MMA work to an add and the MMA.
+    const uint64_t dK0 = um_desc(sK), dK1 = um_desc(sK + kUpKBytes);
+    const uint64_t dV0 = um_desc(sV), dV1 = um_desc(sV + kUpVBytes);
     auto issue_s = [&](int c) -> bool {
       const int b = c & 1;
       if (!mbar_wait_bounded(&ms.k_full[b], ((uint32_t)c >> 1) & 1u)) return false;
       if (c >= 2 && !mbar_wait_bounded(&ms.s_free[b], ((uint32_t)(c - 2) >> 1) & 1u)) return false;
       um_fence_after();
-      const uint32_t kt = sK + (uint32_t)b * kUpKBytes;
+      const uint64_t kd = b ? dK1 : dK0;
 #pragma unroll
       for (int half = 0; half < 2; ++half)
 #pragma unroll
@@ -1204,7 +1209,7 @@ __global__ void __launch_bounds__(kUpThreads, 1) prefill_umma_kernel(PrefillArgs
           for (int ks = 0; ks < 4; ++ks) {
             // q~ channels 64 kb + 16 ks .. + 15: TMEM columns 8 (4 kb + ks) of its half
             const uint32_t ta = tQ + 64u * (uint32_t)half + 8u * (uint32_t)(4 * kb + ks);
-            const uint64_t bd = um_desc(kt + (uint32_t)kb * 8192u + (uint32_t)ks * 32u);
+            const uint64_t bd = kd + (uint64_t)((kb * 8192 + ks * 32) >> 4);
             // NG = 2: K-block kb is group kb, into its own 64 columns
             um_mma_ts(tS + (uint32_t)(b * kSW) + (NG == 2 ? 64u * (uint32_t)kb : 0u), ta, bd, kUpIdescS,
                       (half | ks | (NG == 2 ? 0 : kb)) != 0 ? 1u : 0u);
@@ -1219,7 +1224,7 @@ __global__ void __launch_bounds__(kUpThreads, 1) prefill_umma_kernel(PrefillArgs
       if (!mbar_wait_bounded(&ms.p_full[b], ((uint32_t)c >> 1) & 1u)) return false;
       if (!mbar_wait_bounded(&ms.v_full[b], ((uint32_t)c >> 1) & 1u)) return false;
       um_fence_after();
-      const uint32_t vt2 = sV + (uint32_t)b * kUpVBytes;
+      const uint64_t vd = b ? dV1 : dV0;
       if constexpr (NG == 1) {
 #pragma unroll
         for (int half = 0; half < 2; ++half)
@@ -1227,7 +1232,7 @@ __global__ void __launch_bounds__(kUpThreads, 1) prefill_umma_kernel(PrefillArgs
           for (int ks = 0; ks < 4; ++ks) {
             // tokens 16 ks .. + 15 of p s (hi or lo): TMEM columns 32 half + 8 ks of the chunk's buffer
             const uint32_t ta = tS + (uint32_t)(b * kSW) + 32u * (uint32_t)half + 8u * (uint32_t)ks;
-            const uint64_t bd = um_desc(vt2 + (uint32_t)ks * 32u);
+            const uint64_t bd = vd + (uint64_t)((ks * 32) >> 4);
             um_mma_ts(tO, ta, bd, kUpIdescO, (c > 0 || half > 0 || ks > 0) ? 1u : 0u);
           }
       } else {
@@ -1241,7 +1246,7 @@ __global__ void __launch_bounds__(kUpThreads, 1) prefill_umma_kernel(PrefillArgs
               // 16 half + 8 (ks % 2) of the group's columns; values: channel rows 64 k ..
               const uint32_t ta = tS + (uint32_t)(b * kSW) + 64u * (uint32_t)k + 32u * (uint32_t)(ks >> 1) +
                                   16u * (uint32_t)half + 8u * (uint32_t)(ks & 1);
-              const uint64_t bd = um_desc(vt2 + (uint32_t)k * 8192u + (uint32_t)ks * 32u);
+              const uint64_t bd = vd + (uint64_t)((k * 8192 + ks * 32) >> 4);
               um_mma_ts(tO + 64u * (uint32_t)k, ta, bd, kUpIdescO64, (c > 0 || half > 0 || ks > 0) ? 1u : 0u);
             }
       }
