@@ -91,7 +91,8 @@ struct DecodeArgs {
   uint32_t* status;
   float* qrot;       // [B][Hq][128]
   int8_t* qlimb;     // [B][Hq][2][128]
-  float* qscale;     // [B][Hq][4]: score scale, min-term scale, sigma, sum
+  float* qscale;     // [B][Hq][kQsStride]: score scale, min-term scale, sigma, sum, then the
+                     // min-term scale of each quantisation group (groups < 128 channels)
   __half* qwin;      // [B][Hq][2][128]: q~/sigma as fp16 hi, lo (natural channel order)
   int32_t* prefix;   // [B+1] cost prefix over batch entries
   float* part;       // [(NC + B)][Hq][kPartStride]
@@ -185,12 +186,22 @@ __device__ __forceinline__ void qrot_cta(const DecodeArgs& a, int cta) {
     *reinterpret_cast<float4*>(a.qrot + bh * kD + 4 * r) = make_float4(y[0], y[2], y[1], y[3]);
     // Integer limbs for the tensor-core score tiles: Q = rint(q~/sigma) in
     // [-32000, 32000] = 256*hi + lo with hi, lo signed 8-bit.  Bytes are stored
-    // in MMA-fragment order: channel c = 32t + 16h + 4i + s goes to position
-    // 32t + 8s + 4h + i, so a lane of quad t reads its 32 bytes in one go.
+    // in MMA-fragment order, so that a lane of quad t reads its 32 bytes in one
+    // go; the order follows the K-columns each score MMA gives a lane (code
+    // byte b = c / 4 holds channel c in field f = c % 4):
+    //   ng = 1: one MMA per field f; quad t holds bytes 8t .. 8t + 7:
+    //           c = 32t + 16h + 4i + f goes to 32t + 8f + 4h + i;
+    //   ng = 2: one MMA per (group k, field pair p); quad t holds bytes
+    //           16k + 4t .. + 3 in fields 2p (K-columns 4t..) and 2p + 1
+    //           (16 + 4t..): c = 4 (16k + 4t + i) + 2p + h goes to
+    //           32t + 16k + 8p + 4h + i;
+    //   ng = 4: one MMA per group k; quad t holds field t of the group's
+    //           bytes 8k .. 8k + 7: c = 4 (8k + j) + t goes to 32t + 8k + j.
     const float zc[4] = {y[0], y[2], y[1], y[3]};  // rotated channels 4r + e
     float amax = fmaxf(fmaxf(fabsf(y[0]), fabsf(y[1])), fmaxf(fabsf(y[2]), fabsf(y[3])));
     amax = warp_max(amax);
-    const float sum = warp_sum((y[0] + y[1]) + (y[2] + y[3]));
+    const float own = (y[0] + y[1]) + (y[2] + y[3]);
+    const float sum = warp_sum(own);
     const float sigma = amax > 0.f ? amax / 32000.f : 1.f;
     const float inv = amax > 0.f ? 32000.f / amax : 0.f;
     int8_t* lim = a.qlimb + bh * 2 * kD;
@@ -202,16 +213,30 @@ __device__ __forceinline__ void qrot_cta(const DecodeArgs& a, int cta) {
       const int q = max(-32000, min(32000, __float2int_rn(x)));
       const int hi = ((q + 32896) >> 8) - 128;
       const int lo = q - 256 * hi;
-      const int pos = (c >> 5) * 32 + (c & 3) * 8 + ((c >> 4) & 1) * 4 + ((c >> 2) & 3);
+      const int cb = c >> 2, f = c & 3;
+      const int pos = a.ng == 1   ? (c >> 5) * 32 + f * 8 + ((c >> 4) & 1) * 4 + ((c >> 2) & 3)
+                      : a.ng == 2 ? ((cb >> 2) & 3) * 32 + (cb >> 4) * 16 + (f >> 1) * 8 + (f & 1) * 4 + (cb & 3)
+                                  : f * 32 + cb;
       lim[pos] = (int8_t)hi;
       lim[kD + pos] = (int8_t)lo;
       const __half hx = __float2half_rn(x);
       qw[c] = hx;
       qw[kD + c] = __float2half_rn(x - __half2float(hx));
     }
+    // per-group sums of q~ (a lane's four channels 4r .. 4r + 3 share a group)
+    float gsum[4] = {0.f, 0.f, 0.f, 0.f};
+    if (a.ng > 1) {
+      const int my = (4 * r) / (kD / a.ng);
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        if (k < a.ng) gsum[k] = warp_sum(k == my ? own : 0.f);
+    }
     if (lane == 0) {
       float4 qs4 = make_float4(sigma * (kInvSqrtD * kLog2e), sum * (kInvSqrtD * kLog2e), sigma, sum);
-      *reinterpret_cast<float4*>(a.qscale + bh * 4) = qs4;
+      *reinterpret_cast<float4*>(a.qscale + bh * kQsStride) = qs4;
+      *reinterpret_cast<float4*>(a.qscale + bh * kQsStride + 4) =
+          make_float4(gsum[0] * (kInvSqrtD * kLog2e), gsum[1] * (kInvSqrtD * kLog2e), gsum[2] * (kInvSqrtD * kLog2e),
+                      gsum[3] * (kInvSqrtD * kLog2e));
     }
   }
 }
@@ -505,7 +530,6 @@ constexpr int kIssueBatch = 2;                     // stages the producer issues
 static_assert(kHStages % kIssueBatch == 0 && (kIssueBatch == 1 || kIssueBatch == 2),
               "a batch of up to 16-block stages must start at a multiple of its size and fit one 32-block window");
 constexpr int kSlotsPerStage = 16;                 // block-heads per stage
-constexpr int kHStageBytes = kSlotsPerStage * kBlockHeadBytes;  // 18432
 constexpr int kPStride = 40;                       // u16 per head row of the P' tile
 constexpr int kWarpScratch = 9216;                 // ring bytes each warp may use as window scratch
 constexpr uint32_t kM2 = 0x03030303u;
@@ -523,15 +547,20 @@ constexpr float kPSlack = 4.f;                       // = 2^kMaxSlack
 
 __device__ __forceinline__ float pow2f(int k) { return __int_as_float((127 + k) << 23); }  // -126 <= k <= 127
 
-template <int G>
+// G query heads per KV head; NGQ quantisation groups per vector (1, or 2 / 4
+// for 64- / 32-channel groups, with G <= 4)
+template <int G, int NGQ>
 struct HCfg {
   static constexpr int NT = G <= 4 ? 1 : G / 4;  // n-tiles of 8 columns = 4 heads x 2 limbs
   static constexpr int HP = 4 * NT;              // heads incl. padding
+  static constexpr int BHB = 1024 + 128 * NGQ;   // bytes per block-head
+  static constexpr int stage_bytes = kSlotsPerStage * BHB;
   // (a 10-stage ring for the one-CTA-per-SM G = 8 kernel, and a 4-stage one
   // for G = 4, measured the same as 6: the kernel is bound by its per-step
-  // arithmetic, not by the bytes in flight)
-  static constexpr int NS = kHStages;
-  static constexpr size_t ring_bytes = (size_t)NS * kHStageBytes;
+  // arithmetic, not by the bytes in flight.  The grouped layouts' larger
+  // stages take 4, so that two CTAs still share an SM.)
+  static constexpr int NS = NGQ == 1 ? kHStages : 4;
+  static constexpr size_t ring_bytes = (size_t)NS * stage_bytes;
   // fp32 o' accumulators live in tensor memory: thread (warp w, lane l) owns
   // TMEM lane 32 (w % 4) + l, columns 16 NT (w / 4) .. +16 NT
   static constexpr uint32_t tmem_cols = 32u * NT;
@@ -540,12 +569,18 @@ struct HCfg {
            + (size_t)2 * NS * 8                  // full / empty mbarriers
            + 16                                  // TMEM base address
            + (size_t)NS * kSlotsPerStage         // tokens per block slot
-           + (size_t)kHW * HP * kPStride * 2     // P' tiles
+           + (size_t)kHW * NGQ * HP * kPStride * 2  // P' tiles (one per quantisation group)
            + (size_t)kHW * G * 2 * 4;            // merge (m, l)
   }
 };
-static_assert(kHW * 8 * kD * 4 <= kHStages * kHStageBytes, "merge buffer must fit the ring");
-static_assert(kHStages * kHStageBytes / kHW >= 9216, "window scratch per warp");
+static_assert(kHW * 8 * kD * 4 <= HCfg<4, 1>::ring_bytes && kHW * 8 * kD * 4 <= HCfg<4, 2>::ring_bytes &&
+                  kHW * 8 * kD * 4 <= HCfg<4, 4>::ring_bytes,
+              "merge buffer must fit the ring");
+static_assert(HCfg<4, 1>::ring_bytes / kHW >= kWarpScratch && HCfg<4, 2>::ring_bytes / kHW >= kWarpScratch &&
+                  HCfg<4, 4>::ring_bytes / kHW >= kWarpScratch,
+              "window scratch per warp");
+static_assert(HCfg<4, 2>::NS % kIssueBatch == 0 && HCfg<4, 4>::NS % kIssueBatch == 0,
+              "producer batches start at multiples of their size");
 static_assert(4096 + 8 * 64 + 8 * kD * 4 <= kWarpScratch, "window scratch must fit a warp's share of the ring");
 
 __device__ __forceinline__ void mma_f16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
@@ -577,11 +612,11 @@ __device__ __forceinline__ float fast_ex2(float x) {
   return y;
 }
 
-template <int G>
+template <int G, int NGQ>
 struct MmaWarpState {
-  static constexpr int NT = HCfg<G>::NT;
+  static constexpr int NT = HCfg<G, NGQ>::NT;
   float m[NT];
-  float2 l[NT], msum[NT];  // two partial sums each (paired fp32 arithmetic); the value is .x + .y
+  float2 l[NT], msum[NT][NGQ];  // two partial sums each (paired fp32 arithmetic); the value is .x + .y
   uint32_t tacc;  // TMEM address of fp32 o' for channels 16g + 0..15 of head 4nt + t at column 16 nt + i
 };
 
@@ -615,22 +650,43 @@ __device__ __forceinline__ void tacc_store(uint32_t taddr, const float (&v)[16])
   tacc_store8(taddr + 8u, v + 8);
 }
 
-// acci[mt] holds channel 16g + 2mt (regs 0,1 = hi, lo limb) and 16g + 2mt + 1
-// (regs 2,3); those channels come from code field f = 2(mt&1) and f + 1,
-// which the unshifted masks scaled by 4^f.
+// acci[mt] holds two output channels of the lane's head (regs 0,1 = hi, lo
+// limb of the first, regs 2,3 of the second), which come from code fields
+// f = 2(mt&1) and f + 1, so that the unshifted masks scaled them by 4^f.  They
+// land in TMEM columns 2mt and 2mt + 1 of the lane: column i holds channel
+// chan_base(g, i / 4) + i % 4.  With one group per vector, m-tile mt covers
+// channels 16g + 2mt, + 1 of every lane group g; with smaller groups the lanes
+// load their value codes so that every m-tile lies in one quantisation group
+// (group mt / (8 / NGQ)), whose P' it multiplies.
 // acci: exact int32 sums of P' c 4^f since the last flush; psum: this lane's
-// sum of P' over the same steps (wrapping modulo 2^32, which the plain sum
-// never reaches).
+// sum of P' per group over the same steps (wrapping modulo 2^32, which the
+// plain sum never reaches).
 // Flush: o' = (o' + inv * sum P' c) * rescale in tensor memory
 // (warp-collective), and msum -= 3/2 inv sum P', so that together they hold
 // inv * sum P' (c - 3/2) on top of the sum of p (m + 3/2 s).  The two parts
 // are each rounded to fp32 before they meet; their sum is what carries the
 // P' rounding errors, and there they see zero-mean code offsets.
-template <int G>
-__device__ __forceinline__ void mma_flush(MmaWarpState<G>& st, int (&acci)[HCfg<G>::NT][8][4],
-                                          uint32_t (&psum)[HCfg<G>::NT], int nt, float inv, float rescale = 1.f) {
-  st.msum[nt].x = fmaf(-1.5f * inv, (float)psum[nt], st.msum[nt].x);
-  psum[nt] = 0u;
+template <int NGQ>
+__device__ __forceinline__ int chan_base(int g, int q) {
+  if constexpr (NGQ == 1) return 16 * g + 4 * q;
+  else if constexpr (NGQ == 2) return 64 * (q >> 1) + 16 * (g & 3) + 4 * (g >> 2) + 8 * (q & 1);
+  else return 32 * q + 16 * (g & 1) + 4 * (g >> 1);
+}
+// quantisation group of the lane's four-channel run q (TMEM columns 4q .. 4q + 3)
+template <int NGQ>
+__host__ __device__ constexpr int run_group(int q) {
+  return NGQ == 1 ? 0 : (NGQ == 2 ? q >> 1 : q);
+}
+
+template <int G, int NGQ>
+__device__ __forceinline__ void mma_flush(MmaWarpState<G, NGQ>& st, int (&acci)[HCfg<G, NGQ>::NT][8][4],
+                                          uint32_t (&psum)[HCfg<G, NGQ>::NT][NGQ], int nt, float inv,
+                                          float rescale = 1.f) {
+#pragma unroll
+  for (int k = 0; k < NGQ; ++k) {
+    st.msum[nt][k].x = fmaf(-1.5f * inv, (float)psum[nt][k], st.msum[nt][k].x);
+    psum[nt][k] = 0u;
+  }
 #pragma unroll
   for (int hh = 0; hh < 2; ++hh) {  // two halves of 8 channels: fewer live registers
     float v[8];
@@ -649,19 +705,22 @@ __device__ __forceinline__ void mma_flush(MmaWarpState<G>& st, int (&acci)[HCfg<
   }
 }
 
-template <int G>
+template <int G, int NGQ>
 __global__ void __launch_bounds__(kHW * 32, (G <= 4) ? 2 : 1) decode_heads_kernel(DecodeArgs a) {
-  constexpr int NT = HCfg<G>::NT, HP = HCfg<G>::HP;
-  constexpr int kHStages = HCfg<G>::NS;  // ring stages of this instantiation
+  using Cfg = HCfg<G, NGQ>;
+  static_assert(NGQ == 1 || G <= 4, "grouped layouts take G <= 4 (one n-tile)");
+  constexpr int NT = Cfg::NT, HP = Cfg::HP;
+  constexpr int kHStages = Cfg::NS;  // ring stages of this instantiation
+  constexpr int kStageBytes = Cfg::stage_bytes, BHB = Cfg::BHB;
   extern __shared__ __align__(16) unsigned char smem_raw[];
   __shared__ int btq[2][32];  // producer's block ids, two 32-block windows
   unsigned char* ring = smem_raw;
-  uint64_t* full = reinterpret_cast<uint64_t*>(ring + HCfg<G>::ring_bytes);
+  uint64_t* full = reinterpret_cast<uint64_t*>(ring + Cfg::ring_bytes);
   uint64_t* empty = full + kHStages;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(empty + kHStages);          // TMEM base (16 B)
   uint8_t* ntok = reinterpret_cast<uint8_t*>(tmem_slot + 4);                    // [S][16]
-  uint16_t* pst = reinterpret_cast<uint16_t*>(ntok + kHStages * kSlotsPerStage);  // [8][HP][40]
-  float* ml = reinterpret_cast<float*>(pst + kHW * HP * kPStride);              // [8][G][2]
+  uint16_t* pst = reinterpret_cast<uint16_t*>(ntok + kHStages * kSlotsPerStage);  // [8][NGQ][HP][40]
+  float* ml = reinterpret_cast<float*>(pst + kHW * NGQ * HP * kPStride);        // [8][G][2]
   float* mo = reinterpret_cast<float*>(ring);  // [8][G][128], only while the ring is idle
 
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -670,7 +729,7 @@ __global__ void __launch_bounds__(kHW * 32, (G <= 4) ? 2 : 1) decode_heads_kerne
   const int wph = kHW / hkv;             // warps per KV head
   const int head = warp % hkv, grp = warp / hkv;
   const int nb = 2 * wph;                // blocks per stage
-  const uint32_t copy_bytes = (uint32_t)hkv * kBlockHeadBytes;
+  const uint32_t copy_bytes = (uint32_t)hkv * BHB;
   grid_dep_launch();  // the combine kernel may take SMs as split-K CTAs finish
 
   // The work partition, computed here from the context lengths with loads that
@@ -737,14 +796,14 @@ __global__ void __launch_bounds__(kHW * 32, (G <= 4) ? 2 : 1) decode_heads_kerne
   }
   if (warp == 0) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(smem_u32(tmem_slot)),
-                 "r"(HCfg<G>::tmem_cols)
+                 "r"(Cfg::tmem_cols)
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::: "memory");
   }
   asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
   __syncthreads();
   asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
-  uint16_t* myp = pst + warp * HP * kPStride;
+  uint16_t* myp = pst + warp * NGQ * HP * kPStride;  // P' tile of group k at myp + k HP kPStride
   uint32_t it = 0;    // CTA ring position (continues across batch entries)
   bool alive = true;  // cleared if a wait never completes
 
@@ -828,7 +887,7 @@ __global__ void __launch_bounds__(kHW * 32, (G <= 4) ? 2 : 1) decode_heads_kerne
       if (act && q == 0) mbar_arrive_expect_tx(&full[s], nvalid * copy_bytes);
       __syncwarp();
       if (bid >= 0)
-        bulk_g2s_hint(ring + s * kHStageBytes + q * copy_bytes, a.pages + (size_t)bid * copy_bytes, copy_bytes,
+        bulk_g2s_hint(ring + s * kStageBytes + q * copy_bytes, a.pages + (size_t)bid * copy_bytes, copy_bytes,
                       &full[s], l2_evict_first_policy());  // each block is read once
       issued = max(issued, first + cnt);
       return true;
@@ -850,16 +909,17 @@ __global__ void __launch_bounds__(kHW * 32, (G <= 4) ? 2 : 1) decode_heads_kerne
       waited = true;
     }
     // ---------------- per-warp state for (b, head), loaded while the first stages are in flight ----------------
-    MmaWarpState<G> st;
+    MmaWarpState<G, NGQ> st;
     int acci[NT][8][4];
     st.tacc = *tmem_slot + ((uint32_t)(32 * (warp & 3)) << 16) + (uint32_t)(16 * NT * (warp >> 2));
     uint32_t qb[NT][8];
-    float ah[NT], bh[NT], hbias[NT];
+    float ah[NT], bh[NT][NGQ], hbias[NT];  // bh: min-term scale of each quantisation group
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
       st.m[nt] = -INFINITY;
       st.l[nt] = make_float2(0.f, 0.f);
-      st.msum[nt] = make_float2(0.f, 0.f);
+#pragma unroll
+      for (int k = 0; k < NGQ; ++k) st.msum[nt][k] = make_float2(0.f, 0.f);
 #pragma unroll
       for (int mt = 0; mt < 8; ++mt)
 #pragma unroll
@@ -876,8 +936,9 @@ __global__ void __launch_bounds__(kHW * 32, (G <= 4) ? 2 : 1) decode_heads_kerne
       }
       const int hs = 4 * nt + t;  // head of this lane's score columns
       const bool ok = hs < G;
-      ah[nt] = ok ? a.qscale[(bh0 + hs) * 4 + 0] : 0.f;
-      bh[nt] = ok ? a.qscale[(bh0 + hs) * 4 + 1] : 0.f;
+      ah[nt] = ok ? a.qscale[(bh0 + hs) * kQsStride + 0] : 0.f;
+#pragma unroll
+      for (int k = 0; k < NGQ; ++k) bh[nt][k] = ok ? a.qscale[(bh0 + hs) * kQsStride + (NGQ == 1 ? 1 : 4 + k)] : 0.f;
       hbias[nt] = ok ? 0.f : -INFINITY;
     }
     {
@@ -894,12 +955,13 @@ __global__ void __launch_bounds__(kHW * 32, (G <= 4) ? 2 : 1) decode_heads_kerne
     float s_cap = 0.f, lam0 = 0.f;
     float lam[NT];
     int lrb[NT];  // (low steps in a row) << 8 | boost k
-    uint32_t psum[NT];
+    uint32_t psum[NT][NGQ];
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
       lam[nt] = 0.f;
       lrb[nt] = 0;
-      psum[nt] = 0u;
+#pragma unroll
+      for (int k = 0; k < NGQ; ++k) psum[nt][k] = 0u;
     }
     // 1 / lam of n-tile nt (0 before any value scale was seen)
     auto inv_of = [&](int nt) { return (s_cap * (kPSlack / 65535.f)) * pow2f(-(lrb[nt] & 0xff)); };
@@ -935,7 +997,7 @@ __global__ void __launch_bounds__(kHW * 32, (G <= 4) ? 2 : 1) decode_heads_kerne
       const int n0 = ntok[s * kSlotsPerStage + q0], n1 = ntok[s * kSlotsPerStage + q0 + 1];
       auto step = [&](auto full_tag) {
         constexpr bool fullstep = decltype(full_tag)::value;
-        const unsigned char* s0 = ring + s * kHStageBytes + q0 * copy_bytes + head * kBlockHeadBytes;
+        const unsigned char* s0 = ring + s * kStageBytes + q0 * copy_bytes + head * BHB;
         const unsigned char* s1 = s0 + copy_bytes;
 
         // ---- what the scores and weights need from the stage goes to
@@ -1013,7 +1075,7 @@ __global__ void __launch_bounds__(kHW * 32, (G <= 4) ? 2 : 1) decode_heads_kerne
           // x = s sigma' raw + m sum' (log2 units), taken relative to the
           // running max mref straight away: x' = x - mref
           const float mref0 = st.m[nt] == -INFINITY ? 0.f : st.m[nt];
-          const float2 ah2 = make_float2(ah[nt], ah[nt]), bh2 = make_float2(bh[nt], bh[nt]);
+          const float2 ah2 = make_float2(ah[nt], ah[nt]), bh2 = make_float2(bh[nt][0], bh[nt][0]);
           const float2 c2 = make_float2(hbias[nt] - mref0, hbias[nt] - mref0);  // hbias: -inf on padded heads
           const float2 raw01 = make_float2((float)(dq[0][nt][0] * 256 + dq[0][nt][1]),
                                            (float)(dq[0][nt][2] * 256 + dq[0][nt][3]));
@@ -1043,7 +1105,7 @@ __global__ void __launch_bounds__(kHW * 32, (G <= 4) ? 2 : 1) decode_heads_kerne
             if (need) {
               const float2 a2 = make_float2(alpha, alpha), d2 = make_float2(-bm, -bm);
               st.l[nt] = __fmul2_rn(st.l[nt], a2);
-              st.msum[nt] = __fmul2_rn(st.msum[nt], a2);
+              st.msum[nt][0] = __fmul2_rn(st.msum[nt][0], a2);
               st.m[nt] = mnew;
               x01 = __fadd2_rn(x01, d2);  // now relative to the new max
               x23 = __fadd2_rn(x23, d2);
@@ -1052,7 +1114,7 @@ __global__ void __launch_bounds__(kHW * 32, (G <= 4) ? 2 : 1) decode_heads_kerne
           const float2 p01 = make_float2(fast_ex2(x01.x), fast_ex2(x01.y));  // 0 for masked tokens
           const float2 p23 = make_float2(fast_ex2(x23.x), fast_ex2(x23.y));
           st.l[nt] = __fadd2_rn(st.l[nt], __fadd2_rn(p01, p23));
-          st.msum[nt] = __ffma2_rn(p23, mc23, __ffma2_rn(p01, mc01, st.msum[nt]));
+          st.msum[nt][0] = __ffma2_rn(p23, mc23, __ffma2_rn(p01, mc01, st.msum[nt][0]));
           // kMagicBits + round(p s lam)
           const float2 lam2 = make_float2(lam[nt], lam[nt]), mg2 = make_float2(kMagic, kMagic);
           float2 u01 = __ffma2_rn(p01, __fmul2_rn(sv01, lam2), mg2);
@@ -1100,7 +1162,7 @@ __global__ void __launch_bounds__(kHW * 32, (G <= 4) ? 2 : 1) decode_heads_kerne
           uint16_t* prow = myp + (4 * nt + t) * kPStride;
 #pragma unroll
           for (int e = 0; e < 4; ++e) prow[16 * (e >> 1) + g + 8 * (e & 1)] = (uint16_t)u[e];  // P' < 2^16
-          psum[nt] += (u[0] + u[1]) + (u[2] + u[3]) - 4u * kMagicBits;
+          psum[nt][0] += (u[0] + u[1]) + (u[2] + u[3]) - 4u * kMagicBits;
         }
         const uint4 v0 = *reinterpret_cast<const uint4*>(s0 + kVcOff + 16 * lane);
         const uint4 v1 = *reinterpret_cast<const uint4*>(s1 + kVcOff + 16 * lane);
@@ -1133,10 +1195,260 @@ __global__ void __launch_bounds__(kHW * 32, (G <= 4) ? 2 : 1) decode_heads_kerne
           since_flush = 0;
         }
       };
+      // Grouped layouts (NGQ = 2 or 4 groups of 128 / NGQ channels; G <= 4,
+      // one n-tile).  Scores: one MMA per (block, group, field pair) for 64-
+      // channel groups, per (block, group) for 32-channel groups, each over
+      // code bytes of one group only (the query limbs are stored in the
+      // matching order), so that every group's raw dot product comes out
+      // apart and takes its own (s, m).  Values: every m-tile lies in one
+      // group and multiplies that group's P' = round(p s_tk lam).
+      auto step_grouped = [&](auto full_tag) {
+        constexpr bool fullstep = decltype(full_tag)::value;
+        const unsigned char* s0 = ring + s * kStageBytes + q0 * copy_bytes + head * BHB;
+        const unsigned char* s1 = s0 + copy_bytes;
+        // token e of this lane: block e>>1, row g + 8*(e&1)
+        bool tv[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) tv[e] = fullstep || ((g + 8 * (e & 1)) < ((e >> 1) ? n1 : n0));
+        // (scale, min) pairs of every group: K at 1024 + 4 (row NGQ + k), V at
+        // 1024 + 64 NGQ + 4 (row NGQ + k).  The V pairs are read again where
+        // they are used (fewer live registers).  Masked slots may hold any
+        // bits (a slot whose block was not fetched keeps stale shared
+        // memory): their value scales and minima read as 0.
+        auto vpair = [&](int e, int k) -> uint32_t {
+          const unsigned char* sb = (e >> 1) ? s1 : s0;
+          const uint32_t x = *reinterpret_cast<const uint32_t*>(sb + 1024 + 64 * NGQ + 4 * ((g + 8 * (e & 1)) * NGQ + k));
+          return tv[e] ? x : 0u;
+        };
+        __half2 hm = __float2half2_rn(0.f);  // the step's largest value scale (low halves; scales are >= 0)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const unsigned char* sb = (e >> 1) ? s1 : s0;
+          const int row = g + 8 * (e & 1);
+          uint32_t xv[NGQ];
+          if constexpr (NGQ == 2) {
+            const uint2 v2 = *reinterpret_cast<const uint2*>(sb + 1024 + 128 + 8 * row);
+            xv[0] = v2.x; xv[1] = v2.y;
+          } else {
+            const uint4 v4 = *reinterpret_cast<const uint4*>(sb + 1024 + 256 + 16 * row);
+            xv[0] = v4.x; xv[1] = v4.y; xv[2] = v4.z; xv[3] = v4.w;
+          }
+#pragma unroll
+          for (int k = 0; k < NGQ; ++k) {
+            const uint32_t x = tv[e] ? xv[k] : 0u;
+            hm = __hmax2(hm, *reinterpret_cast<const __half2*>(&x));
+          }
+        }
+        float smax = __low2float(hm);
+        if (__any_sync(0xffffffffu, smax > s_cap)) {  // rare: raise the scale cap, flushing first
+          smax = fmaxf(smax, __shfl_xor_sync(0xffffffffu, smax, 4));
+          smax = fmaxf(smax, __shfl_xor_sync(0xffffffffu, smax, 8));
+          smax = fmaxf(smax, __shfl_xor_sync(0xffffffffu, smax, 16));
+          mma_flush(st, acci, psum, 0, inv_of(0));
+          since_flush = 0;
+          s_cap = 2.f * smax;
+          lam0 = 65535.f / (s_cap * kPSlack);
+          lam[0] = lam0 * pow2f(lrb[0] & 0xff);
+        }
+        // ---- scores, group by group: x = sum_k (s_tk sigma' raw_k + m_tk sum'_k), relative to mref
+        const float mref0 = st.m[0] == -INFINITY ? 0.f : st.m[0];
+        const float2 ah2 = make_float2(ah[0], ah[0]);
+        float2 x01 = make_float2(hbias[0] - mref0, hbias[0] - mref0), x23 = x01;  // hbias: -inf on padded heads
+#pragma unroll
+        for (int k = 0; k < NGQ; ++k) {
+          int dq[2][4];
+#pragma unroll
+          for (int bb = 0; bb < 2; ++bb) {
+            const unsigned char* kc = (bb ? s1 : s0) + kKcOff;
+            if constexpr (NGQ == 2) {
+              // bytes 16k + 4t .. + 3 of rows g and g + 8: field 2p at K-columns
+              // 4t.., field 2p + 1 at 16 + 4t..
+              const uint32_t wa = *reinterpret_cast<const uint32_t*>(kc + 32 * g + 16 * k + 4 * t);
+              const uint32_t wb = *reinterpret_cast<const uint32_t*>(kc + 32 * (g + 8) + 16 * k + 4 * t);
+#pragma unroll
+              for (int p = 0; p < 2; ++p) {
+                const uint32_t af[4] = {(wa >> (4 * p)) & kM2, (wb >> (4 * p)) & kM2, (wa >> (4 * p + 2)) & kM2,
+                                        (wb >> (4 * p + 2)) & kM2};
+                if (p == 0) mma_u8s8_z(dq[bb], af, qb[0][4 * k], qb[0][4 * k + 1]);
+                else mma_u8s8(dq[bb], af, qb[0][4 * k + 2], qb[0][4 * k + 3]);
+              }
+            } else {
+              // field t of bytes 8k .. 8k + 3 (K-columns 4t..) and 8k + 4 .. (16 + 4t..)
+              const uint2 wa = *reinterpret_cast<const uint2*>(kc + 32 * g + 8 * k);
+              const uint2 wb = *reinterpret_cast<const uint2*>(kc + 32 * (g + 8) + 8 * k);
+              const int sh = 2 * t;
+              const uint32_t af[4] = {(wa.x >> sh) & kM2, (wb.x >> sh) & kM2, (wa.y >> sh) & kM2, (wb.y >> sh) & kM2};
+              mma_u8s8_z(dq[bb], af, qb[0][2 * k], qb[0][2 * k + 1]);
+            }
+          }
+          float2 kf[4];  // K (scale, min) of group k for the lane's four tokens
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            kf[e] = __half22float2(*reinterpret_cast<const __half2*>(
+                ((e >> 1) ? s1 : s0) + 1024 + 4 * ((g + 8 * (e & 1)) * NGQ + k)));
+          const float2 raw01 = make_float2((float)(dq[0][0] * 256 + dq[0][1]), (float)(dq[0][2] * 256 + dq[0][3]));
+          const float2 raw23 = make_float2((float)(dq[1][0] * 256 + dq[1][1]), (float)(dq[1][2] * 256 + dq[1][3]));
+          const float2 bh2 = make_float2(bh[0][k], bh[0][k]);
+          x01 = __ffma2_rn(__fmul2_rn(make_float2(kf[0].x, kf[1].x), ah2), raw01,
+                           __ffma2_rn(make_float2(kf[0].y, kf[1].y), bh2, x01));
+          x23 = __ffma2_rn(__fmul2_rn(make_float2(kf[2].x, kf[3].x), ah2), raw23,
+                           __ffma2_rn(make_float2(kf[2].y, kf[3].y), bh2, x23));
+        }
+        if constexpr (!fullstep) {
+          x01.x = tv[0] ? x01.x : -INFINITY;
+          x01.y = tv[1] ? x01.y : -INFINITY;
+          x23.x = tv[2] ? x23.x : -INFINITY;
+          x23.y = tv[3] ? x23.y : -INFINITY;
+        }
+        // the reference max moves only when a score passes it by more than kMaxSlack
+        float bm = fmaxf(fmaxf(x01.x, x01.y), fmaxf(x23.x, x23.y));
+        if (__any_sync(0xffffffffu, bm > (st.m[0] == -INFINITY ? -INFINITY : kMaxSlack))) {
+          bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 4));
+          bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 8));
+          bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 16));
+          const float mnew = bm + mref0;
+          const bool need = mnew > st.m[0] + kMaxSlack;
+          const float alpha = need ? fast_ex2(st.m[0] - mnew) : 1.f;
+          mma_flush(st, acci, psum, 0, inv_of(0), alpha);
+          if (need) {
+            const float2 a2 = make_float2(alpha, alpha), d2 = make_float2(-bm, -bm);
+            st.l[0] = __fmul2_rn(st.l[0], a2);
+#pragma unroll
+            for (int k = 0; k < NGQ; ++k) st.msum[0][k] = __fmul2_rn(st.msum[0][k], a2);
+            st.m[0] = mnew;
+            x01 = __fadd2_rn(x01, d2);
+            x23 = __fadd2_rn(x23, d2);
+          }
+        }
+        const float2 p01 = make_float2(fast_ex2(x01.x), fast_ex2(x01.y));  // 0 for masked tokens
+        const float2 p23 = make_float2(fast_ex2(x23.x), fast_ex2(x23.y));
+        st.l[0] = __fadd2_rn(st.l[0], __fadd2_rn(p01, p23));
+        // ---- P' of every group (kMagicBits + round(p s lam)), the min terms, the step's sums of P'
+        const float2 mg2 = make_float2(kMagic, kMagic);
+        uint32_t um = 0u, ustep[NGQ];
+        auto store_p = [&](int k, const uint32_t (&u)[4]) {
+          uint16_t* prow = myp + (k * HP + t) * kPStride;
+#pragma unroll
+          for (int e = 0; e < 4; ++e) prow[16 * (e >> 1) + g + 8 * (e & 1)] = (uint16_t)u[e];  // P' < 2^16
+          ustep[k] = (u[0] + u[1]) + (u[2] + u[3]) - 4u * kMagicBits;
+        };
+        {
+          const float2 lam2 = make_float2(lam[0], lam[0]);
+#pragma unroll
+          for (int k = 0; k < NGQ; ++k) {
+            float2 vf[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const uint32_t x = vpair(e, k);
+              vf[e] = __half22float2(*reinterpret_cast<const __half2*>(&x));
+            }
+            const float2 sv01 = make_float2(vf[0].x, vf[1].x), sv23 = make_float2(vf[2].x, vf[3].x);
+            // m + 3/2 s: the codes are centred in the flush (0 for masked tokens)
+            const float2 mc01 = make_float2(fmaf(1.5f, vf[0].x, vf[0].y), fmaf(1.5f, vf[1].x, vf[1].y));
+            const float2 mc23 = make_float2(fmaf(1.5f, vf[2].x, vf[2].y), fmaf(1.5f, vf[3].x, vf[3].y));
+            st.msum[0][k] = __ffma2_rn(p23, mc23, __ffma2_rn(p01, mc01, st.msum[0][k]));
+            const float2 u01 = __ffma2_rn(p01, __fmul2_rn(sv01, lam2), mg2);
+            const float2 u23 = __ffma2_rn(p23, __fmul2_rn(sv23, lam2), mg2);
+            const uint32_t u[4] = {__float_as_uint(u01.x), __float_as_uint(u01.y), __float_as_uint(u23.x),
+                                   __float_as_uint(u23.y)};
+            um = max(um, max(max(u[0], u[1]), max(u[2], u[3])));
+            store_p(k, u);
+          }
+        }
+        // the boost rule of the 128-channel path, on the head's largest P' over its groups
+        const uint32_t big = __ballot_sync(0xffffffffu, um >= kPLowBits);
+        lrb[0] = ((big >> t) & 0x11111111u) == 0u ? lrb[0] + 256 : (lrb[0] & 0xff);
+        const bool raise = (t < G) && lrb[0] >= (kLowRun << 8) && (lrb[0] & 0xff) < kMaxBoost;
+        if (__any_sync(0xffffffffu, um > kPHighBits || raise)) {
+          uint32_t uh = um;  // the head's step maximum (lanes of the same t)
+          uh = max(uh, __shfl_xor_sync(0xffffffffu, uh, 4));
+          uh = max(uh, __shfl_xor_sync(0xffffffffu, uh, 8));
+          uh = max(uh, __shfl_xor_sync(0xffffffffu, uh, 16));
+          float ym = 0.f;  // the head's largest p s over its groups
+#pragma unroll
+          for (int k = 0; k < NGQ; ++k)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float pe = (e >> 1) ? ((e & 1) ? p23.y : p23.x) : ((e & 1) ? p01.y : p01.x);
+              const uint32_t x = vpair(e, k);
+              ym = fmaxf(ym, pe * __low2float(*reinterpret_cast<const __half2*>(&x)));
+            }
+          ym = fmaxf(ym, __shfl_xor_sync(0xffffffffu, ym, 4));
+          ym = fmaxf(ym, __shfl_xor_sync(0xffffffffu, ym, 8));
+          ym = fmaxf(ym, __shfl_xor_sync(0xffffffffu, ym, 16));
+          mma_flush(st, acci, psum, 0, inv_of(0));  // psum holds the earlier steps only
+          int kb = lrb[0] & 0xff;
+          if (uh > kPHighBits) {
+            kb = 0;
+          } else if (raise) {
+            const float y = ym * lam0;
+            const int ex = ((__float_as_int(y) >> 23) & 0xff) - 127;
+            if (y > 0.f) kb = max(0, min(kMaxBoost, kBoostExp - ex));
+          }
+          lrb[0] = (uh > kPHighBits || raise) ? kb : (lrb[0] & ~0xff) | kb;
+          lam[0] = lam0 * pow2f(kb);
+          const float2 l2 = make_float2(lam[0], lam[0]);
+#pragma unroll
+          for (int k = 0; k < NGQ; ++k) {
+            float sv[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const uint32_t x = vpair(e, k);
+              sv[e] = __low2float(*reinterpret_cast<const __half2*>(&x));
+            }
+            const float2 u01 = __ffma2_rn(__fmul2_rn(p01, make_float2(sv[0], sv[1])), l2, mg2);
+            const float2 u23 = __ffma2_rn(__fmul2_rn(p23, make_float2(sv[2], sv[3])), l2, mg2);
+            const uint32_t u[4] = {__float_as_uint(u01.x), __float_as_uint(u01.y), __float_as_uint(u23.x),
+                                   __float_as_uint(u23.y)};
+            store_p(k, u);
+          }
+        }
+#pragma unroll
+        for (int k = 0; k < NGQ; ++k) psum[0][k] += ustep[k];
+        // value code words of this lane, in m-tile order: m-tile mt takes word
+        // mt >> 1, fields 2 (mt & 1) and + 1.  Word (chunk c, token quad t, j)
+        // sits at kVcOff + 16 (4c + t) + 4j; NGQ = 2: m-tile 4k + l reads chunk
+        // 4k + (g & 3), word (g >> 2) + 2 (l >> 1); NGQ = 4: m-tile 2k + l reads
+        // chunk 2k + (g & 1), word g >> 1.
+        uint32_t va[4], vb[4];
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+          const int c = NGQ == 2 ? 4 * (w >> 1) + (g & 3) : 2 * w + (g & 1);
+          const int jj = NGQ == 2 ? (g >> 2) + 2 * (w & 1) : g >> 1;
+          const int off = kVcOff + 16 * (4 * c + t) + 4 * jj;
+          va[w] = *reinterpret_cast<const uint32_t*>(s0 + off);
+          vb[w] = *reinterpret_cast<const uint32_t*>(s1 + off);
+        }
+        __syncwarp();  // every lane has its value codes (and its P' rows are written)
+        if (lane == 0) mbar_arrive(&empty[s]);
+        uint32_t pb0[NGQ], pb1[NGQ];
+        const uint32_t sel = (g & 1) ? 0x6420u : 0x7531u;  // odd column: low byte (lo limb)
+#pragma unroll
+        for (int k = 0; k < NGQ; ++k) {
+          const uint16_t* prow = myp + (k * HP + (g >> 1)) * kPStride;
+          const uint2 x0 = *reinterpret_cast<const uint2*>(prow + 4 * t);
+          const uint2 x1 = *reinterpret_cast<const uint2*>(prow + 16 + 4 * t);
+          pb0[k] = prmt(x0.x, x0.y, sel);
+          pb1[k] = prmt(x1.x, x1.y, sel);
+        }
+#pragma unroll
+        for (int mt = 0; mt < 8; ++mt) {
+          const int jw = mt >> 1, k = mt / (8 / NGQ);
+          const uint32_t m0 = kM2 << (4 * (mt & 1)), m1 = m0 << 2;
+          const uint32_t af[4] = {va[jw] & m0, va[jw] & m1, vb[jw] & m0, vb[jw] & m1};
+          mma_u8u8(acci[0][mt], af, pb0[k], pb1[k]);
+        }
+        if (++since_flush >= 96) {
+          mma_flush(st, acci, psum, 0, inv_of(0));
+          since_flush = 0;
+        }
+      };
       if (n0 == kBlock && n1 == kBlock) {
-        step(std::true_type{});
+        if constexpr (NGQ == 1) step(std::true_type{});
+        else step_grouped(std::true_type{});
       } else if (n0 + n1 > 0) {
-        step(std::false_type{});
+        if constexpr (NGQ == 1) step(std::false_type{});
+        else step_grouped(std::false_type{});
       } else {
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[s]);
@@ -1189,7 +1501,7 @@ __global__ void __launch_bounds__(kHW * 32, (G <= 4) ? 2 : 1) decode_heads_kerne
           for (int i = 0; i < 16; ++i) qh[nt][i] = 0u;
         }
         const int hs = 4 * nt + t;
-        wsc[nt] = hs < G ? a.qscale[(bh0 + hs) * 4 + 2] * (kInvSqrtD * kLog2e) : 0.f;
+        wsc[nt] = hs < G ? a.qscale[(bh0 + hs) * kQsStride + 2] * (kInvSqrtD * kLog2e) : 0.f;
         wm[nt] = -INFINITY;
         wl[nt] = 0.f;
 #pragma unroll
@@ -1316,11 +1628,13 @@ __global__ void __launch_bounds__(kHW * 32, (G <= 4) ? 2 : 1) decode_heads_kerne
           const float M = fmaxf(st.m[nt], wm[nt]);
           const float mref = M == -INFINITY ? 0.f : M;
           const float ab = fast_ex2(st.m[nt] - mref), aw = fast_ex2(wm[nt] - mref);
-          const float* src = wo + hs * kD + 16 * g;
+          const float* src = wo + hs * kD;
 #pragma unroll
-          for (int i = 0; i < 16; ++i) v[i] = fmaf(v[i], ab, src[i] * aw);
+          for (int i = 0; i < 16; ++i) v[i] = fmaf(v[i], ab, src[chan_base<NGQ>(g, i >> 2) + (i & 3)] * aw);
           st.l[nt] = make_float2(fmaf(st.l[nt].x + st.l[nt].y, ab, wl[nt] * aw), 0.f);
-          st.msum[nt] = make_float2((st.msum[nt].x + st.msum[nt].y) * ab, 0.f);
+#pragma unroll
+          for (int k = 0; k < NGQ; ++k)
+            st.msum[nt][k] = make_float2((st.msum[nt][k].x + st.msum[nt][k].y) * ab, 0.f);
           st.m[nt] = M;
         }
         tacc_store(st.tacc + 16u * nt, v);
@@ -1332,20 +1646,26 @@ __global__ void __launch_bounds__(kHW * 32, (G <= 4) ? 2 : 1) decode_heads_kerne
     if (wph == 1) {
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
-        float l = st.l[nt].x + st.l[nt].y, ms = st.msum[nt].x + st.msum[nt].y;
+        float l = st.l[nt].x + st.l[nt].y, ms[NGQ];
+#pragma unroll
+        for (int k = 0; k < NGQ; ++k) ms[k] = st.msum[nt][k].x + st.msum[nt][k].y;
 #pragma unroll
         for (int o = 4; o < 32; o <<= 1) {
           l += __shfl_xor_sync(0xffffffffu, l, o);
-          ms += __shfl_xor_sync(0xffffffffu, ms, o);
+#pragma unroll
+          for (int k = 0; k < NGQ; ++k) ms[k] += __shfl_xor_sync(0xffffffffu, ms[k], o);
         }
         const int hs = 4 * nt + t;
         float v[16];
         tacc_load(st.tacc + 16u * nt, v);
         if (hs < G) {
-          float* dst = part_b + (size_t)hs * kPartStride + 16 * g;
+          float* dst = part_b + (size_t)hs * kPartStride;
 #pragma unroll
-          for (int i = 0; i < 16; i += 4)
-            *reinterpret_cast<float4*>(dst + i) = make_float4(v[i] + ms, v[i + 1] + ms, v[i + 2] + ms, v[i + 3] + ms);
+          for (int q = 0; q < 4; ++q) {
+            const float m_ = ms[run_group<NGQ>(q)];
+            *reinterpret_cast<float4*>(dst + chan_base<NGQ>(g, q)) =
+                make_float4(v[4 * q] + m_, v[4 * q + 1] + m_, v[4 * q + 2] + m_, v[4 * q + 3] + m_);
+          }
           if (g == 0) {
             part_b[(size_t)hs * kPartStride + 128] = st.m[nt];
             part_b[(size_t)hs * kPartStride + 129] = l;
@@ -1356,19 +1676,22 @@ __global__ void __launch_bounds__(kHW * 32, (G <= 4) ? 2 : 1) decode_heads_kerne
       __syncthreads();  // window scratch no longer in use: the ring becomes merge buffers
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
-        float l = st.l[nt].x + st.l[nt].y, ms = st.msum[nt].x + st.msum[nt].y;
+        float l = st.l[nt].x + st.l[nt].y, ms[NGQ];
+#pragma unroll
+        for (int k = 0; k < NGQ; ++k) ms[k] = st.msum[nt][k].x + st.msum[nt][k].y;
 #pragma unroll
         for (int o = 4; o < 32; o <<= 1) {
           l += __shfl_xor_sync(0xffffffffu, l, o);
-          ms += __shfl_xor_sync(0xffffffffu, ms, o);
+#pragma unroll
+          for (int k = 0; k < NGQ; ++k) ms[k] += __shfl_xor_sync(0xffffffffu, ms[k], o);
         }
         const int hs = 4 * nt + t;
         float v[16];
         tacc_load(st.tacc + 16u * nt, v);
         if (hs < G) {
-          float* dst = mo + ((size_t)warp * G + hs) * kD + 16 * g;
+          float* dst = mo + ((size_t)warp * G + hs) * kD;
 #pragma unroll
-          for (int i = 0; i < 16; ++i) dst[i] = v[i] + ms;
+          for (int i = 0; i < 16; ++i) dst[chan_base<NGQ>(g, i >> 2) + (i & 3)] = v[i] + ms[run_group<NGQ>(i >> 2)];
           if (g == 0) {
             ml[(warp * G + hs) * 2 + 0] = st.m[nt];
             ml[(warp * G + hs) * 2 + 1] = l;
@@ -1407,7 +1730,7 @@ __global__ void __launch_bounds__(kHW * 32, (G <= 4) ? 2 : 1) decode_heads_kerne
   __syncthreads();
   if (warp == 0) {
     asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(*tmem_slot), "r"(HCfg<G>::tmem_cols)
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(*tmem_slot), "r"(Cfg::tmem_cols)
                  : "memory");
   }
 }
@@ -1604,19 +1927,21 @@ static cudaError_t launch_pdl(void (*kernel)(Args...), dim3 grid, dim3 block, si
   return cudaLaunchKernelEx(&cfg, kernel, args...);
 }
 
-template <int G>
+template <int G, int NGQ = 1>
 static okv_status launch_decode_heads(const DecodeArgs& a, cudaStream_t s, bool early) {
-  const size_t smem = HCfg<G>::smem_bytes();
+  const size_t smem = HCfg<G, NGQ>::smem_bytes();
   static std::atomic<uint32_t> attr_set{0};
-  cudaError_t e = set_smem_limit_once((const void*)decode_heads_kernel<G>, (int)smem, attr_set);
+  cudaError_t e = set_smem_limit_once((const void*)decode_heads_kernel<G, NGQ>, (int)smem, attr_set);
   if (e != cudaSuccess) return fail(OKV_ERR_CUDA, "decode smem attribute: %s", cudaGetErrorString(e));
-  e = launch_pdl(decode_heads_kernel<G>, dim3(a.nc), dim3(kHW * 32), smem, s, early, a);
+  e = launch_pdl(decode_heads_kernel<G, NGQ>, dim3(a.nc), dim3(kHW * 32), smem, s, early, a);
   if (e != cudaSuccess) return fail(OKV_ERR_CUDA, "decode launch: %s", cudaGetErrorString(e));
   return check_launch("decode");
 }
 
 bool decode_uses_tensor_cores(int g, int hkv, int ng) {
-  return ng == 1 && (g == 1 || g == 2 || g == 4 || g == 8) && (hkv == 1 || hkv == 2 || hkv == 4 || hkv == 8);
+  const bool hkv_ok = hkv == 1 || hkv == 2 || hkv == 4 || hkv == 8;
+  if (ng == 1) return hkv_ok && (g == 1 || g == 2 || g == 4 || g == 8);
+  return hkv_ok && (ng == 2 || ng == 4) && (g == 1 || g == 2 || g == 4);
 }
 
 int decode_ctas_per_sm(int g, int hkv, int ng) {
@@ -1680,7 +2005,19 @@ static okv_status launch_decode_tail(const DecodeArgs& a, int B, cudaStream_t s)
   // that the events bracket it alone.
   const bool early = ev0 == nullptr;
   const bool tc = decode_uses_tensor_cores(a.g, a.hkv, a.ng);
-  if (tc) {
+  if (tc && a.ng == 2) {
+    switch (a.g) {
+      case 1: st = launch_decode_heads<1, 2>(a, s, early); break;
+      case 2: st = launch_decode_heads<2, 2>(a, s, early); break;
+      default: st = launch_decode_heads<4, 2>(a, s, early); break;
+    }
+  } else if (tc && a.ng == 4) {
+    switch (a.g) {
+      case 1: st = launch_decode_heads<1, 4>(a, s, early); break;
+      case 2: st = launch_decode_heads<2, 4>(a, s, early); break;
+      default: st = launch_decode_heads<4, 4>(a, s, early); break;
+    }
+  } else if (tc) {
     switch (a.g) {
       case 1: st = launch_decode_heads<1>(a, s, early); break;
       case 2: st = launch_decode_heads<2>(a, s, early); break;

@@ -107,7 +107,7 @@ DecodePlan make_decode_plan(int batch, int hq, int hkv, int ng) {
   p.qlimb_off = off;
   off = align_up(off + (size_t)batch * hq * 2 * kD, 256);
   p.qscale_off = off;
-  off = align_up(off + (size_t)batch * hq * 4 * sizeof(float), 256);
+  off = align_up(off + (size_t)batch * hq * kQsStride * sizeof(float), 256);
   p.qwin_off = off;
   off = align_up(off + (size_t)batch * hq * 2 * kD * 2, 256);
   p.prefix_off = off;

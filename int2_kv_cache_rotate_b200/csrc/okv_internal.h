@@ -32,13 +32,14 @@ struct DecodePlan {
   int num_units = 0;        // batch * hkv
   size_t qrot_off = 0;      // fp32 [B][Hq][128] rotated queries
   size_t qlimb_off = 0;     // int8 [B][Hq][2][128] query limbs (MMA order)
-  size_t qscale_off = 0;    // fp32 [B][Hq][4] (score scale, min term, sigma, sum)
+  size_t qscale_off = 0;    // fp32 [B][Hq][kQsStride] (score scale, min term, sigma, sum, group min terms)
   size_t qwin_off = 0;      // fp16 [B][Hq][2][128] scaled query hi/lo halves (window MMA)
   size_t prefix_off = 0;    // int32 [B+1] cost prefix over batch entries
   size_t part_off = 0;      // fp32 [(num_ctas + batch)][Hq][kPartStride]
   size_t total = 0;
 };
 constexpr int kPartStride = 132;  // o'[128], m, l, 2 spare
+constexpr int kQsStride = 8;      // floats per query head in the query-scale workspace
 constexpr int kWinCost = 8;       // cost of an entry's window in block units (all heads)
 constexpr int kFusedAppendMaxTokens = 127;  // okv_decode_step fuses appends this short with the query rotation
 // split-K kernel choice and residency (decode.cu)

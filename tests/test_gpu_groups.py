@@ -15,8 +15,17 @@ oracle's per-group quantiser and decode, on the same seeded inputs:
 * gather/dequantise bit-exact;
 * decode within 2e-3 on the tiny single-layer workload (4 query heads on 1
   KV head, 2048 tokens) and at the decode benchmark's head shape (32 / 8) at
-  100,000 tokens.
+  100,000 tokens;
+* the tensor-core split-K kernel's grouped layouts (per-group score MMAs and
+  value m-tiles) at every head grouping it takes (G = 1, 2, 4 on 8, 2 or 1 KV
+  heads, so that one warp or several serve a head), with and without sinks,
+  over lengths that end inside a block, at a block edge, inside and past the
+  fp16 window;
+* a peaked case: one INT2 key 10 nats above a flat 30,000-token context, at
+  the start and in the middle of a split, so that the per-group P' of the
+  tail behind it keeps its precision.
 """
+import math
 import numpy as np
 import pytest
 
@@ -208,3 +217,83 @@ def test_grouped_decode_100k_bench_heads(group):
         want = O.decode(oc, q[b:b + 1, h * G:(h + 1) * G], [0], [L], G)
         assert H.rel_err_rows(got[b:b + 1, h * G:(h + 1) * G], want).max() <= TOL, (b, h)
     assert cache.device_status() == 0
+
+
+def _fill_groups_sinks(seed, hq, hkv, lens, group, nsink, plant=None):
+    """GPU and oracle caches (group, sinks) from the same fp32 rotated vectors;
+    plant(b, h, zk) may edit the rotated keys first."""
+    okv = _okv()
+    lay = H.Layout(seed, lens)
+    uk, uv = H.rotations(seed, hkv)
+    gc = okv.Cache(hq, hkv, lay.num_blocks, len(lens), lay.mbps, uk, uv, num_sink=nsink, group=group)
+    oc = O.Cache(hkv, uk.astype(np.float64), uv.astype(np.float64), sinks=nsink, group=group)
+    zs = {kind: [np.stack([WL.sample_rotated(seed, 0, 0, h, n, kind, extra=b) for h in range(hkv)], axis=1)
+                 for b, n in enumerate(lens)] for kind in (0, 1)}
+    if plant is not None:
+        for b in range(len(lens)):
+            for h in range(hkv):
+                plant(b, h, zs[0][b][:, h], uk)
+    for b, n in enumerate(lens):
+        if n:
+            oc.append(b, 0, zs[0][b], zs[1][b], pre_rotated=True)
+    slots, pos = lay.flat()
+    okv.append_quantize(gc, _t(np.concatenate(zs[0])), _t(np.concatenate(zs[1])), _t(slots), _t(pos),
+                        _t(lay.table), _t(np.array(lens, np.int32)), pre_rotated=True)
+    torch.cuda.synchronize()
+    return gc, oc, lay
+
+
+@pytest.mark.parametrize("group", GROUPS)
+@pytest.mark.parametrize("hq,hkv,nsink,lens", [
+    (32, 8, 0, [1, 15, 16, 17, 100, 128, 129, 143, 300, 2000, 5003]),
+    (16, 8, 16, [1, 16, 17, 144, 145, 400, 3000]),       # G = 2
+    (8, 8, 32, [31, 33, 160, 161, 1000, 4100]),          # G = 1
+    (8, 2, 0, [0, 47, 129, 900, 6000]),                  # G = 4, 4 warps per KV head (merged)
+    (4, 1, 48, [49, 176, 177, 2500]),                    # G = 4, 8 warps per KV head
+])
+def test_grouped_decode_tensor_core_shapes(group, hq, hkv, nsink, lens):
+    okv = _okv()
+    seed = 70 + nsink + hq
+    gc, oc, lay = _fill_groups_sinks(seed, hq, hkv, lens, group, nsink)
+    q = np.stack([WL.sample_queries(seed, 0, 0, h, len(lens), hq // hkv, extra=9) for h in range(hkv)], 1)
+    q = q.reshape(len(lens), hq, 128)
+    seq = np.arange(len(lens), dtype=np.int32)
+    got = okv.decode_attention(gc, _t(q, torch.bfloat16), _t(seq), _t(lay.table),
+                               _t(np.array(lens, np.int32))).cpu().numpy()
+    assert gc.device_status() == 0
+    live = [i for i, n in enumerate(lens) if n > 0]
+    want = O.decode(oc, q[live], seq[live], [lens[i] for i in live], hq)
+    err = H.rel_err_rows(got[live], want)
+    assert err.max() <= TOL, (err.max(), np.unravel_index(err.argmax(), err.shape))
+
+
+@pytest.mark.parametrize("group", GROUPS)
+@pytest.mark.parametrize("where", [5, 17_011])
+def test_grouped_decode_peaked_tail(group, where):
+    """One INT2 key per (sequence, KV head), aligned with the first query head
+    of the group, 10 nats above an otherwise flat context of 30,000 tokens."""
+    okv = _okv()
+    seed, hq, hkv, L, gap = 90 + where % 7, 32, 8, 30_000, 10.0
+    G = hq // hkv
+    lens = [L, L]
+    q = np.stack([WL.sample_queries(seed, 0, 0, h, 2, G, extra=11) for h in range(hkv)], 1).reshape(2, hq, 128)
+
+    def plant(b, h, zk, uk):
+        q_rot = q[b, h * G].astype(np.float64) @ O.rotation(uk[h].astype(np.float64))
+        direction = q_rot / np.linalg.norm(q_rot)
+        alpha = gap * math.sqrt(128) / np.linalg.norm(q_rot)
+        for _ in range(6):
+            row = (alpha * direction).astype(np.float32)
+            c, s_, m_ = O.quantize(row[None], group)
+            logit = O.dequantize(c, s_, m_, group)[0].astype(np.float64) @ q_rot / math.sqrt(128)
+            alpha *= gap / logit
+        zk[where] = row
+
+    gc, oc, lay = _fill_groups_sinks(seed, hq, hkv, lens, group, 0, plant=plant)
+    seq = np.arange(2, dtype=np.int32)
+    got = okv.decode_attention(gc, _t(q, torch.bfloat16), _t(seq), _t(lay.table),
+                               _t(np.array(lens, np.int32))).cpu().numpy()
+    assert gc.device_status() == 0
+    want = O.decode(oc, q, seq, lens, hq)
+    err = H.rel_err_rows(got, want)
+    assert err.max() <= TOL, (err.max(), np.unravel_index(err.argmax(), err.shape))
