@@ -122,6 +122,12 @@ typedef struct {
   uint32_t* status_word;      /* device, nullable: OKV_DEV_* flags (OR-ed)   */
   void* sink_rows;            /* device fp16, layout above, 16-B aligned;
                                  may be NULL when num_sink = 0             */
+  void* r_image;              /* device, okv_r_image_bytes(Hkv) B, 16-B aligned,
+                                 nullable: the prefill append's staged R of
+                                 every (KV head, K|V), written by
+                                 okv_build_r_image for the current u_k, u_v
+                                 (rebuild it after changing them).  NULL: each
+                                 prefill append stages R itself.           */
 } okv_cache_desc;
 
 /* Offline calibration of the rotations, on the host in fp64 (once per layer).
@@ -175,6 +181,19 @@ okv_status okv_load_rotations(const char* path, int32_t num_layers, int32_t num_
  * "Revolução no Serviço de LLMs…", section "Resultados e Métricas de
  * Desempenho"). */
 size_t okv_block_head_bytes(int32_t group);
+
+/* Bytes of the optional staged-rotation buffer `r_image`: for every KV head,
+ * K and V, R = U H P_br / sqrt(d) split into three bf16 parts (their sum is R
+ * to about 2^-24 relative), 96 KB in the operand layout of the tcgen05 append. */
+size_t okv_r_image_bytes(int32_t num_kv_heads);
+
+/* Fill desc->r_image from desc->u_k and desc->u_v (one CTA per (KV head,
+ * K|V), asynchronous on `stream`).  The prefill append then copies its R
+ * instead of staging it from U at the start of every CTA.  Returns
+ * OKV_ERR_INVALID_ARG when r_image is NULL or misaligned.  Pages: gen-hub.ru,
+ * "Что придумали в Together AI" (R = U, then H, then P_br, precomputed once
+ * per layer: aiforradalom.hu, "OSCAR: figyelem-tudatos és bevetésre kész"). */
+okv_status okv_build_r_image(const okv_cache_desc* desc, void* stream);
 
 /* Bytes the caller allocates for `pages`, `window_ring` and `sink_rows`. */
 size_t okv_pages_bytes(int32_t num_blocks, int32_t num_kv_heads, int32_t group);

@@ -281,12 +281,68 @@ constexpr int kUmStages = 3;
 constexpr uint32_t kUmRegion = 16384;                 // 128 rows x 128 B
 constexpr uint32_t kUmBBytes = 6 * kUmRegion;         // 3 parts x 2 K-blocks
 constexpr uint32_t kUmABytes = 2 * kUmRegion;         // one tile, 2 K-blocks
-constexpr uint32_t kUmCtlBytes = 64;                  // 7 barriers and the TMEM base
-static_assert(7 * 8 + 4 <= kUmCtlBytes, "control region");
+constexpr uint32_t kUmCtlBytes = 80;                  // 8 barriers and the TMEM base
+static_assert(8 * 8 + 4 <= kUmCtlBytes, "control region");
 constexpr size_t kUmSmem = 1024 + kUmBBytes + kUmStages * kUmABytes + kUmCtlBytes;
 constexpr uint32_t kUmTmemCols = 256;
 // instruction descriptor: D f32, A and B bf16, both K-major, N = 128, M = 128
 constexpr uint32_t kUmIdesc = um_idesc(128, true, true);
+
+// R = U H P_br / sqrt(128) of one (KV head, K|V), split in three bf16 parts,
+// written into `img` in the B-operand image above (part pt, K-block kb at
+// (2 pt + kb) 16 KB; element (n, c) in row n, 16-byte chunk ((c % 64) / 8) ^
+// (n % 8)).  The swizzle is computed from the row index, so the image is the
+// same wherever it lies; copied to a 1024-byte aligned shared address it is
+// what the MMA descriptors expect.  Warp w of 8 takes input channels 16w ..
+// 16w + 15 in two batches of eight: after the butterflies a lane holds its
+// four output channels for all eight input channels, which is one 16-byte
+// chunk of each of those four B rows.
+__device__ __forceinline__ void stage_r_parts(const float* U, unsigned char* img, int warp, int lane) {
+  const int b = rev5(lane);
+#pragma unroll 1
+  for (int c0 = 16 * warp; c0 < 16 * warp + 16; c0 += 8) {
+    float y[8][4];
+#pragma unroll
+    for (int r = 0; r < 8; ++r)
+#pragma unroll
+      for (int aa = 0; aa < 4; ++aa) y[r][aa] = __ldg(U + (size_t)(c0 + r) * kD + lane + 32 * aa);
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+      wht128_warp(y[r], lane);
+#pragma unroll
+      for (int aa = 0; aa < 4; ++aa) y[r][aa] *= kInvSqrtD;
+    }
+    const uint32_t kb = (uint32_t)c0 >> 6, cb = ((uint32_t)c0 & 63u) * 2u;
+#pragma unroll
+    for (int aa = 0; aa < 4; ++aa) {
+      const uint32_t nn = (uint32_t)(4 * b + rev2(aa));  // rotated channel of these values
+      uint32_t pk[3][4];
+#pragma unroll
+      for (int r = 0; r < 8; r += 2) {
+        float u0 = y[r][aa], u1 = y[r + 1][aa];
+#pragma unroll
+        for (int pt = 0; pt < 3; ++pt) {
+          const __nv_bfloat162 pp = __floats2bfloat162_rn(u0, u1);
+          pk[pt][r >> 1] = *reinterpret_cast<const uint32_t*>(&pp);
+          u0 -= __low2float(pp);
+          u1 -= __high2float(pp);
+        }
+      }
+      const uint32_t off = kb * kUmRegion + um_swz(nn, cb);
+#pragma unroll
+      for (int pt = 0; pt < 3; ++pt)
+        *reinterpret_cast<uint4*>(img + (uint32_t)pt * 2 * kUmRegion + off) =
+            make_uint4(pk[pt][0], pk[pt][1], pk[pt][2], pk[pt][3]);
+    }
+  }
+}
+
+// one CTA of 8 warps per (KV head, K|V): the staged R into the cache's image buffer
+__global__ void __launch_bounds__(256) r_image_kernel(const float* u_k, const float* u_v, uint8_t* r_image) {
+  const int h = blockIdx.x, kind = blockIdx.y;
+  const float* U = (kind ? u_v : u_k) + (size_t)h * kD * kD;
+  stage_r_parts(U, r_image + ((size_t)h * 2 + kind) * kUmBBytes, threadIdx.x >> 5, threadIdx.x & 31);
+}
 
 // TMA tiled load of a 3-D box at (x, y, z) into shared memory, completing on bar
 __device__ __forceinline__ void um_tma_load_3d(uint32_t dst, const CUtensorMap* map, int x, int y, int z,
@@ -310,7 +366,8 @@ __global__ void __launch_bounds__(kUmThreads, 1) append_umma_kernel(AppendArgs a
   uint64_t* mma_done = reinterpret_cast<uint64_t*>(ctl);  // [2], one commit
   uint64_t* tmem_free = mma_done + 2;                    // [2], 128 arrivals (an epilogue warpgroup)
   uint64_t* afull = tmem_free + 2;                       // [3], one arrival + the tile's bytes
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(afull + kUmStages);
+  uint64_t* rfull = afull + kUmStages;                   // the staged R copied from the cache's image
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(rfull + 1);
 
   const int h = blockIdx.y, kind = blockIdx.z;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -330,6 +387,8 @@ __global__ void __launch_bounds__(kUmThreads, 1) append_umma_kernel(AppendArgs a
   };
   int loaded = 0, landed = 0;  // tiles whose loads were issued / waited for (producer lane 0)
   int committed = 0;            // tiles whose MMAs were committed (producer lane 0)
+  const bool r_copy = a.r_image != nullptr;  // R comes from the image, else the epilogue warps stage it
+  bool r_landed = false;                      // (producer lane 0)
 
   if (tid == 0) {
     for (int i = 0; i < 2; ++i) {
@@ -337,59 +396,24 @@ __global__ void __launch_bounds__(kUmThreads, 1) append_umma_kernel(AppendArgs a
       mbar_init(&tmem_free[i], 128);
     }
     for (int i = 0; i < kUmStages; ++i) mbar_init(&afull[i], 1);
+    mbar_init(rfull, 1);
     fence_mbar_init();
   }
   __syncthreads();
   if (warp == kUmProducer) {
-    // the first tiles' loads go out while the other warps stage R
+    // the first tiles' loads go out while the other warps stage R (or with the copy of R)
     if (lane == 0) {
+      if (r_copy) {
+        mbar_arrive_expect_tx(rfull, kUmBBytes);
+        bulk_g2s(gbase, a.r_image + ((size_t)h * 2 + kind) * kUmBBytes, kUmBBytes, rfull);
+      }
       load_tile(0);
       if (n > 1) load_tile(1);
       loaded = min(n, 2);
     }
-  } else {
-    // R = U H P_br / sqrt(128), split in three bf16 parts, into B (row n = output channel,
-    // K = input channel).  Warp w takes input channels 16w .. 16w + 15 in two batches of eight:
-    // after the butterflies a lane holds its four output channels for all eight input
-    // channels, which is one 16-byte chunk of each of those four B rows.
-    const float* U = (kind ? a.u_v : a.u_k) + (size_t)h * kD * kD;
-    const int b = rev5(lane);
-#pragma unroll 1
-    for (int c0 = 16 * warp; c0 < 16 * warp + 16; c0 += 8) {
-      float y[8][4];
-#pragma unroll
-      for (int r = 0; r < 8; ++r)
-#pragma unroll
-        for (int aa = 0; aa < 4; ++aa) y[r][aa] = __ldg(U + (size_t)(c0 + r) * kD + lane + 32 * aa);
-#pragma unroll
-      for (int r = 0; r < 8; ++r) {
-        wht128_warp(y[r], lane);
-#pragma unroll
-        for (int aa = 0; aa < 4; ++aa) y[r][aa] *= kInvSqrtD;
-      }
-      const uint32_t kb = (uint32_t)c0 >> 6, cb = ((uint32_t)c0 & 63u) * 2u;
-#pragma unroll
-      for (int aa = 0; aa < 4; ++aa) {
-        const uint32_t nn = (uint32_t)(4 * b + rev2(aa));  // rotated channel of these values
-        uint32_t pk[3][4];
-#pragma unroll
-        for (int r = 0; r < 8; r += 2) {
-          float u0 = y[r][aa], u1 = y[r + 1][aa];
-#pragma unroll
-          for (int pt = 0; pt < 3; ++pt) {
-            const __nv_bfloat162 pp = __floats2bfloat162_rn(u0, u1);
-            pk[pt][r >> 1] = *reinterpret_cast<const uint32_t*>(&pp);
-            u0 -= __low2float(pp);
-            u1 -= __high2float(pp);
-          }
-        }
-        const uint32_t off = kb * kUmRegion + um_swz(nn, cb);
-#pragma unroll
-        for (int pt = 0; pt < 3; ++pt)
-          *reinterpret_cast<uint4*>(gbase + (uint32_t)pt * 2 * kUmRegion + off) =
-              make_uint4(pk[pt][0], pk[pt][1], pk[pt][2], pk[pt][3]);
-      }
-    }
+  } else if (!r_copy) {
+    // R into B (row n = output channel, K = input channel), staged from U here
+    stage_r_parts((kind ? a.u_v : a.u_k) + (size_t)h * kD * kD, gbase, warp, lane);
     um_fence_proxy_async();  // R was written by ordinary stores; the MMA reads it through the async proxy
   }
   if (warp == 0) {
@@ -409,7 +433,12 @@ __global__ void __launch_bounds__(kUmThreads, 1) append_umma_kernel(AppendArgs a
       // MMAs of tile i: its loads have landed, and the epilogue of tile i - 2 has drained TMEM
       // buffer i & 1
       if (lane == 0 && alive) {
-        bool ok = mbar_wait_bounded(&afull[i % kUmStages], ((uint32_t)(i / kUmStages)) & 1u);
+        bool ok = true;
+        if (i == 0 && r_copy) {
+          ok = mbar_wait_bounded(rfull, 0u);
+          r_landed = ok;
+        }
+        ok = ok && mbar_wait_bounded(&afull[i % kUmStages], ((uint32_t)(i / kUmStages)) & 1u);
         if (ok) landed = i + 1;
         ok = ok && (i < 2 || mbar_wait_bounded(&tmem_free[i & 1], ((uint32_t)(i - 2) >> 1) & 1u));
         if (ok) {
@@ -453,6 +482,7 @@ __global__ void __launch_bounds__(kUmThreads, 1) append_umma_kernel(AppendArgs a
     // after a failed wait, wait (bounded) for the loads in flight and for the
     // last commit (it completes after every MMA issued before it)
     if (lane == 0) {
+      if (r_copy && !r_landed) mbar_drain_bounded(rfull, 0u);
       for (int i = landed; i < loaded; ++i)
         if (!mbar_drain_bounded(&afull[i % kUmStages], ((uint32_t)(i / kUmStages)) & 1u)) break;
       if (committed > 0)  // (the epilogue may have given up on a tile this thread completed)
@@ -616,6 +646,12 @@ static bool encode_tile_map(CUtensorMap* m, const void* base, int hkv, int T) {
   return encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, elem,
                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+okv_status launch_r_image(const okv_cache_desc* d, cudaStream_t s) {
+  static_assert(kRImageBytesPerHead == kUmBBytes, "the image holds one B operand per (KV head, K|V)");
+  r_image_kernel<<<dim3(d->num_kv_heads, 2), 256, 0, s>>>(d->u_k, d->u_v, (uint8_t*)d->r_image);
+  return check_launch("staged-rotation image");
 }
 
 okv_status launch_append(const okv_cache_desc* d, const void* k, const void* v, int T,

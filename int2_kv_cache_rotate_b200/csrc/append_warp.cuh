@@ -27,6 +27,7 @@ struct AppendArgs {
   int hkv, num_blocks, num_slots, mbps, nsink;
   int ng;   // quantisation groups per vector (128 / group)
   int bhb;  // bytes of one block-head
+  const uint8_t* r_image;  // staged R of every (KV head, K|V) for the tcgen05 append, or null
 };
 
 inline AppendArgs make_append_args(const okv_cache_desc* d, const void* k, const void* v, const int32_t* seq_slot,
@@ -53,6 +54,7 @@ inline AppendArgs make_append_args(const okv_cache_desc* d, const void* k, const
   a.mbps = d->max_blocks_per_seq;
   a.ng = kD / d->group;
   a.bhb = block_head_bytes(a.ng);
+  a.r_image = (const uint8_t*)d->r_image;
   return a;
 }
 

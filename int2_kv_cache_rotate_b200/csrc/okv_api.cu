@@ -77,6 +77,7 @@ okv_status validate_desc(const okv_cache_desc* d) {
   if (d->pages == nullptr && d->num_blocks > 0) return fail(OKV_ERR_INVALID_ARG, "pages is NULL");
   if (d->window_ring == nullptr) return fail(OKV_ERR_INVALID_ARG, "window_ring is NULL");
   if (d->u_k == nullptr || d->u_v == nullptr) return fail(OKV_ERR_INVALID_ARG, "u_k/u_v is NULL");
+  if (!aligned(d->r_image, 16)) return fail(OKV_ERR_INVALID_ARG, "r_image must be 16-byte aligned (or NULL)");
   if (!aligned(d->pages, 16) || !aligned(d->window_ring, 16) || !aligned(d->u_k, 16) || !aligned(d->u_v, 16))
     return fail(OKV_ERR_INVALID_ARG, "pages, window_ring, u_k and u_v must be 16-byte aligned");
   if ((long long)d->max_blocks_per_seq * kBlock > 0x3fffffffLL)
@@ -124,7 +125,7 @@ using namespace okv;
 
 extern "C" {
 
-int32_t okv_version(void) { return 2; }
+int32_t okv_version(void) { return 3; }
 
 okv_status okv_time_next_decode_kernel(void* start_event, void* stop_event) {
   if ((start_event == nullptr) != (stop_event == nullptr))
@@ -156,6 +157,18 @@ size_t okv_block_head_bytes(int32_t group) {
 size_t okv_pages_bytes(int32_t num_blocks, int32_t num_kv_heads, int32_t group) {
   if (num_blocks < 0 || num_kv_heads < 0) return 0;
   return (size_t)num_blocks * (size_t)num_kv_heads * okv_block_head_bytes(group);
+}
+
+size_t okv_r_image_bytes(int32_t num_kv_heads) {
+  if (num_kv_heads < 0) return 0;
+  return (size_t)num_kv_heads * 2 * kRImageBytesPerHead;
+}
+
+okv_status okv_build_r_image(const okv_cache_desc* desc, void* stream) {
+  okv_status st = validate_desc(desc);
+  if (st != OKV_OK) return st;
+  if (desc->r_image == nullptr) return fail(OKV_ERR_INVALID_ARG, "r_image is NULL");
+  return launch_r_image(desc, (cudaStream_t)stream);
 }
 
 size_t okv_window_bytes(int32_t num_seq_slots, int32_t num_kv_heads) {

@@ -48,7 +48,12 @@ int decode_ctas_per_sm(int g, int hkv, int ng);
 
 DecodePlan make_decode_plan(int batch, int hq, int hkv, int ng);
 
+// bytes of one (KV head, K|V) staged R in the cache's image buffer: three bf16
+// parts x 128 x 128
+constexpr size_t kRImageBytesPerHead = 3 * 128 * 128 * 2;
+
 // launchers (return cudaGetLastError-mapped status)
+okv_status launch_r_image(const okv_cache_desc* d, cudaStream_t s);
 okv_status launch_append(const okv_cache_desc* d, const void* k, const void* v, int T,
                          const int32_t* seq_slot, const int32_t* pos, const int32_t* block_table,
                          const int32_t* slot_lens, uint32_t flags, float* rotated_out,

@@ -50,6 +50,7 @@ class CacheDesc(ctypes.Structure):
         ("u_v", ctypes.c_void_p),
         ("status_word", ctypes.c_void_p),
         ("sink_rows", ctypes.c_void_p),
+        ("r_image", ctypes.c_void_p),
     ]
 
 
@@ -67,6 +68,8 @@ _SIGNATURES = {
     "okv_block_head_bytes": (_SZ, [_I32]),
     "okv_window_bytes": (_SZ, [_I32, _I32]),
     "okv_sink_bytes": (_SZ, [_I32, _I32, _I32]),
+    "okv_r_image_bytes": (_SZ, [_I32]),
+    "okv_build_r_image": (_I32, [_DESC, _P]),
     "okv_append_quantize": (_I32, [_DESC, _P, _P, _I32, _P, _P, _P, _P, _U32, _P, _P]),
     "okv_decode_workspace_bytes": (_SZ, [_DESC, _I32]),
     "okv_decode_attention": (_I32, [_DESC, _P, _I32, _P, _P, _P, _P, _P, _SZ, _P]),
@@ -160,7 +163,7 @@ class Cache:
     receives pointers."""
 
     def __init__(self, hq: int, hkv: int, num_blocks: int, num_seq_slots: int, max_blocks_per_seq: int,
-                 u_k, u_v, device="cuda", num_sink: int = 0, group: int = HEAD_DIM):
+                 u_k, u_v, device="cuda", num_sink: int = 0, group: int = HEAD_DIM, stage_r: bool = True):
         import torch
         self.hq, self.hkv, self.num_sink, self.group = hq, hkv, num_sink, group
         self.num_blocks, self.num_seq_slots, self.max_blocks_per_seq = num_blocks, num_seq_slots, max_blocks_per_seq
@@ -174,10 +177,20 @@ class Cache:
         # first num_sink positions of every sequence, fp16 (sink tokens)
         self.sink = torch.zeros((num_seq_slots, hkv, 2, max(num_sink, 0), HEAD_DIM), dtype=torch.float16,
                                 device=device)
+        # the prefill append's staged R of every (KV head, K|V), built once from U
+        self.r_image = torch.empty(max(int(lib().okv_r_image_bytes(hkv)), 16), dtype=torch.uint8, device=device) \
+            if stage_r else None
         self.desc = CacheDesc(hq, hkv, HEAD_DIM, group, BLOCK_TOKENS, WINDOW, num_blocks, num_seq_slots,
                               max_blocks_per_seq, num_sink, self.pages.data_ptr(), self.ring.data_ptr(),
                               self.u_k.data_ptr(), self.u_v.data_ptr(), self.status.data_ptr(),
-                              self.sink.data_ptr() if num_sink > 0 else None)
+                              self.sink.data_ptr() if num_sink > 0 else None,
+                              self.r_image.data_ptr() if stage_r else None)
+        if stage_r:
+            self.rebuild_r_image()
+
+    def rebuild_r_image(self, stream=None):
+        """Stage R from u_k, u_v into the image buffer again (after changing them)."""
+        _check(lib().okv_build_r_image(ctypes.byref(self.desc), _stream(stream)))
 
     def device_status(self) -> int:
         return int(self.status[0].item())

@@ -325,3 +325,45 @@ def test_decode_partial_last_block_with_live_tail():
     # the window ring rows holding whatever was appended last
     for b in range(len(fill)):
         assert oc.seqs[(b, 0, 0)]["set"][:dec[b]].all()
+
+
+@pytest.mark.parametrize("group", [128, 32])
+def test_staged_rotation_image_matches_in_kernel_staging(group):
+    """The tcgen05 append copying R from the cache's staged image writes the
+    same bytes (codes, scales, window rows) and the same rotated fp32 values
+    as the append staging R from U itself; after U changes, rebuilding the
+    image matches a fresh cache."""
+    okv = _okv()
+    seed, hq, hkv, n = 57, 32, 8, 1000
+    lay = H.Layout(seed, [n])
+    uk, uv = H.rotations(seed, hkv)
+    g = torch.Generator(device="cuda").manual_seed(seed)
+    k = torch.randn((n, hkv, 128), generator=g, device="cuda").to(torch.bfloat16)
+    v = torch.randn((n, hkv, 128), generator=g, device="cuda").to(torch.bfloat16)
+    slots, pos = lay.flat()
+    args = (_t(slots), _t(pos), _t(lay.table), _t(np.array([n], np.int32)))
+
+    def run(c):
+        rot = torch.empty((n, 2, hkv, 128), dtype=torch.float32, device="cuda")
+        okv.append_quantize(c, k, v, *args, rotated_out=rot)
+        torch.cuda.synchronize()
+        assert c.device_status() == 0
+        return c.pages.clone(), c.ring.clone(), rot
+
+    mk = lambda u1, u2, stage: okv.Cache(hq, hkv, lay.num_blocks, 1, lay.mbps, u1, u2, group=group, stage_r=stage)
+    with_image, without = run(mk(uk, uv, True)), run(mk(uk, uv, False))
+    for a, b in zip(with_image, without):
+        assert torch.equal(a, b)
+    # the rotation itself against the fp64 oracle
+    want = np.einsum("thc,hcd->thd", k.float().cpu().numpy().astype(np.float64),
+                     np.stack([O.rotation(uk[h].astype(np.float64)) for h in range(hkv)]))
+    got = with_image[2][:, 0].cpu().numpy()
+    assert np.abs(got - want).max() <= 1e-5 * np.abs(want).max()
+    # new rotations: rebuild the image of an existing cache
+    uk2, uv2 = H.rotations(seed + 1, hkv)
+    c = mk(uk, uv, True)
+    c.u_k.copy_(torch.from_numpy(uk2))
+    c.u_v.copy_(torch.from_numpy(uv2))
+    c.rebuild_r_image()
+    for a, b in zip(run(c), run(mk(uk2, uv2, True))):
+        assert torch.equal(a, b)
