@@ -252,8 +252,8 @@ okv_status okv_decode_attention(const okv_cache_desc* desc, const void* q, int32
 
 /* Size of the device array behind okv_decode_attention_noalloc (8 MiB).  A
  * batch fits when okv_decode_workspace_bytes(desc, B) is at most this, which
- * depends on the SM count: on a 148-SM B200, up to 58 sequences with 32 query
- * and 8 KV heads (so a 64-sequence batch is refused), up to 29 with 64 and 8. */
+ * depends on the SM count: on a 148-SM B200, up to 57 sequences with 32 query
+ * and 8 KV heads (so a 64-sequence batch is refused), up to 28 with 64 and 8. */
 #define OKV_NOALLOC_SCRATCH_BYTES (8u << 20)
 
 /* One decode step in one call: append this step's new tokens, then decode.
