@@ -7,21 +7,21 @@
 //   1. query rotation: q~ = q R_K, split into fp16 hi + lo halves of
 //      q~ 2^-e (e per row so that the halves stay in fp16 range) and the
 //      per-group sums of q~;
-//   2. attention (this file's main kernel): a CTA of 8 warps takes 128 query
+//   2. attention on the tcgen05 tensor cores (`prefill_umma_kernel<NG>`, NG
+//      = 128 / group quantisation groups per vector): a CTA takes 128 query
 //      rows (query token x query head of one KV head) and streams the key
-//      positions 0 .. its last row's position in 16-token chunks.  Every
+//      positions 0 .. its last row's position in 64-token chunks.  Every
 //      chunk is staged in shared memory as fp16: the 2-bit codes (0..3 are
 //      exact in fp16) of INT2 positions with their per-group scale s and
 //      minimum m, or the fp16 values of window and sink rows with s = 1 and
 //      m = 0.  Then, per group k of channels,
 //        score = s_k (q~_k . c_k) + m_k sum(q~_k)
-//      with q~ . c on mma.m16n8k16 (f16 in, f32 accumulate; q~ as hi + lo,
-//      so the products carry about 22 bits), an online softmax per row, and
+//      with q~ . c on the tensor cores (q~ as hi + lo, so the products carry
+//      about 22 bits), an online softmax per row, and
 //        o' += sum_t (p_t s_{t,k}) c_t + sum_t p_t m_{t,k}
-//      with p s as hi + lo fp16 A operands in the registers the score MMA
-//      left them in (its D fragment is the next MMA's A fragment) and the
-//      codes as the B operand.  The dense contraction runs on the tensor
-//      cores; nothing is dequantised to a rounded value.
+//      with p s as hi + lo fp16 operands and the codes as the other.  The
+//      dense contraction runs on the tensor cores; nothing is dequantised to
+//      a rounded value;
 //   3. normalise and un-rotate: o = (o' / l) R_V^T per row.
 #include "okv_common.cuh"
 #include "okv_internal.h"
@@ -30,18 +30,7 @@
 namespace okv {
 namespace {
 
-constexpr int kPfWarps = 8;
-constexpr int kPfRows = 16 * kPfWarps;  // query rows per CTA
-constexpr int kKStride = kD + 8;        // fp16 per staged key row (bank-conflict-free fragment loads)
-// value rows are staged row-major, 16-byte chunk c of token row r at chunk
-// position c ^ (r & 7), and read with transposing matrix loads
-__device__ __forceinline__ int vchunk(int row, int c) { return row * kD + ((c ^ (row & 7)) << 3); }
-
-__device__ __forceinline__ void ldsm_x4_trans(uint32_t (&r)[4], const void* p) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "r"((uint32_t)__cvta_generic_to_shared(p)));
-}
+constexpr int kPfRows = 128;  // query rows per attention CTA (the MMA's M)
 
 struct PrefillArgs {
   const __nv_bfloat16* q;  // [T][Hq][128]
@@ -192,351 +181,15 @@ __global__ void __launch_bounds__(256) prefill_qrot_kernel(PrefillArgs a) {
   }
 }
 
-__device__ __forceinline__ void mma_f16_pf(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-      "{%0,%1,%2,%3};\n"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-
 __device__ __forceinline__ uint32_t pack_half2(float lo_elem, float hi_elem) {
   const __half2 h = __floats2half2_rn(lo_elem, hi_elem);
   return *reinterpret_cast<const uint32_t*>(&h);
 }
 
-// hi and lo fp16 halves of a pair of floats, packed as MMA operand registers
-__device__ __forceinline__ void split_half2(float x0, float x1, uint32_t& hi, uint32_t& lo) {
-  const __half2 h = __floats2half2_rn(x0, x1);
-  const float2 f = __half22float2(h);
-  hi = *reinterpret_cast<const uint32_t*>(&h);
-  lo = pack_half2(x0 - f.x, x1 - f.y);
-}
-
 // ---------------------------------------------------------------------------
-// 2. attention.  Grid (ceil(rows / 128), Hkv); rows are (token, query head)
-// pairs of the KV head, token-major: row r = token (r / G), head (r % G).
-// Warp w owns rows 16w .. 16w + 15 of the CTA.  Fragment facts
-// (m16n8k16, f16): lane (g = lane / 4, t = lane % 4) holds A (row g, cols
-// 2t, 2t+1), (g + 8, 2t..), (g, 2t + 8..), (g + 8, 2t + 8..); B (rows 2t,
-// 2t + 1, col g), (2t + 8, 2t + 9, col g); D (row g, cols 2t, 2t + 1),
-// (g + 8, 2t, 2t + 1).
-// ---------------------------------------------------------------------------
-template <int NG>
-__global__ void __launch_bounds__(kPfWarps * 32) prefill_attn_kernel(PrefillArgs a) {
-  constexpr int KSG = 8 / NG;  // 16-channel k-steps per group
-  // two buffers of each (chunk ch in buffer ch & 1): one barrier per chunk
-  __shared__ __align__(16) __half kc[2][16 * kKStride];  // [token][channel]: codes or fp16 values
-  __shared__ __align__(16) __half vt[2][16 * kD];        // [token][channel], chunks swizzled (vchunk)
-  __shared__ float ksm[2][16][NG][2], vsm[2][16][NG][2];  // (scale, min) per token and group
-  __shared__ int tpos_ok[2][16];                          // 1 if the chunk's token is a readable position
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int g = lane >> 2, t = lane & 3;
-  const int hk = blockIdx.y;
-  const int nrows = a.T * a.g;
-  const int row0 = blockIdx.x * kPfRows;
-  // this lane's two rows (g and g + 8 of the warp's 16)
-  int rtok[2], rrow[2];
-  bool rok[2];
-#pragma unroll
-  for (int h2 = 0; h2 < 2; ++h2) {
-    const int r = row0 + 16 * warp + g + 8 * h2;
-    rok[h2] = r < nrows;
-    const int rr = rok[h2] ? r : nrows - 1;
-    rtok[h2] = rr / a.g;
-    rrow[h2] = rtok[h2] * a.hq + hk * a.g + rr % a.g;  // global (token, query head) row
-  }
-  // query fragments: A operands of the score MMA, hi and lo halves
-  uint32_t qa_hi[8][4], qa_lo[8][4];
-  {
-    const __half* h0 = a.qhi + (size_t)rrow[0] * kD;
-    const __half* h1 = a.qhi + (size_t)rrow[1] * kD;
-    const __half* l0 = a.qlo + (size_t)rrow[0] * kD;
-    const __half* l1 = a.qlo + (size_t)rrow[1] * kD;
-#pragma unroll
-    for (int ks = 0; ks < 8; ++ks) {
-      const int c = 16 * ks + 2 * t;
-      qa_hi[ks][0] = *reinterpret_cast<const uint32_t*>(h0 + c);
-      qa_hi[ks][1] = *reinterpret_cast<const uint32_t*>(h1 + c);
-      qa_hi[ks][2] = *reinterpret_cast<const uint32_t*>(h0 + c + 8);
-      qa_hi[ks][3] = *reinterpret_cast<const uint32_t*>(h1 + c + 8);
-      qa_lo[ks][0] = *reinterpret_cast<const uint32_t*>(l0 + c);
-      qa_lo[ks][1] = *reinterpret_cast<const uint32_t*>(l1 + c);
-      qa_lo[ks][2] = *reinterpret_cast<const uint32_t*>(l0 + c + 8);
-      qa_lo[ks][3] = *reinterpret_cast<const uint32_t*>(l1 + c + 8);
-    }
-  }
-  float qsum[2][NG], qup[2];
-  int rpos[2];
-#pragma unroll
-  for (int h2 = 0; h2 < 2; ++h2) {
-    const float* aux = a.qaux + (size_t)rrow[h2] * kQaux;
-#pragma unroll
-    for (int k = 0; k < NG; ++k) qsum[h2][k] = aux[k] * (kInvSqrtD * kLog2e);
-    qup[h2] = aux[4] * (kInvSqrtD * kLog2e);  // undoes the 2^-e of the halves, in log2 units
-    rpos[h2] = a.first + rtok[h2];
-  }
-  float o[16][4];
-#pragma unroll
-  for (int n = 0; n < 16; ++n)
-#pragma unroll
-    for (int j = 0; j < 4; ++j) o[n][j] = 0.f;
-  float mrow[2] = {-INFINITY, -INFINITY}, lrow[2] = {0.f, 0.f};
-  float msum[2][NG];
-#pragma unroll
-  for (int h2 = 0; h2 < 2; ++h2)
-#pragma unroll
-    for (int k = 0; k < NG; ++k) msum[h2][k] = 0.f;
-
-  const int last_row = min(nrows, row0 + kPfRows) - 1;
-  const int pmax = a.first + last_row / a.g;  // last position any row of this CTA sees
-  const int nchunks = pmax / 16 + 1;
-  const int tid = threadIdx.x;
-  // Staging: thread tid -> K (tid < 128) or V, token (tid % 128) / 8, channels
-  // 16 (tid % 8) .. + 15 of a 16-token chunk.  Chunk ch is exactly block
-  // column ch of the sequence.  The global loads of chunk ch + 1 are issued
-  // before chunk ch's arithmetic and its block id one chunk earlier still, so
-  // neither latency sits between two barriers.
-  const int is_v = tid >> 7, tk = (tid & 127) >> 3, part = tid & 7;
-  auto chunk_block = [&](int ch) -> int {  // the chunk's block id when it holds INT2 positions, else -1
-    const int lo = 16 * ch, hi = min(16 * ch + 15, min(pmax, a.L - 1));
-    const bool int2 = ch < nchunks && hi >= lo && max(lo, a.nsink) <= min(hi, a.L - kWin - 1);
-    return int2 ? a.block_table[(size_t)a.slot * a.mbps + ch] : -1;
-  };
-  int f_src = 0;  // fetched chunk: 0 masked, 1 INT2, 2 fp16 window, 3 fp16 sink
-  uint4 f0 = make_uint4(0, 0, 0, 0), f1 = make_uint4(0, 0, 0, 0);
-  uint32_t f_sm = 0;
-  auto fetch = [&](int ch, int blk) {
-    const int p = 16 * ch + tk;
-    f_src = 0;
-    if (p <= pmax && p < a.L) {
-      if (p < a.nsink) {
-        f_src = 3;
-      } else if (p >= a.L - kWin) {
-        f_src = 2;
-      } else if (blk >= 0 && blk < a.num_blocks) {
-        f_src = 1;
-      } else if (part == 0 && !is_v) {
-        raise_flag(a.status, OKV_DEV_BAD_BLOCK);
-      }
-    }
-    if (f_src == 1) {
-      const uint8_t* bp = a.pages + ((size_t)blk * a.hkv + hk) * a.bhb;
-      const int sl = p & 15;
-      if (!is_v) {
-        f0.x = *reinterpret_cast<const uint32_t*>(bp + kKcOff + sl * 32 + 4 * part);
-      } else {
-        uint32_t w = 0;
-#pragma unroll
-        for (int bq = 0; bq < 4; ++bq) w |= (uint32_t)bp[v_code_offset(sl, 4 * part + bq)] << (8 * bq);
-        f0.x = w;
-      }
-      if (part < NG) f_sm = *reinterpret_cast<const uint32_t*>(bp + sm_offset(NG, is_v, sl, part));
-    } else if (f_src >= 2) {
-      const size_t rows_per_kind = f_src == 2 ? (size_t)kWin : (size_t)a.nsink;
-      const size_t base = (((size_t)a.slot * a.hkv + hk) * 2 + is_v) * rows_per_kind;
-      const size_t row = f_src == 2 ? (size_t)(p % kWin) : (size_t)p;
-      const __half* srcb = f_src == 2 ? a.ring : a.sink;
-      const uint4* xr = reinterpret_cast<const uint4*>(srcb + (base + row) * kD + 16 * part);
-      f0 = xr[0];
-      f1 = xr[1];
-    }
-  };
-  auto stage = [&](int buf) {
-    __half x16[16];
-    if (f_src == 1) {
-#pragma unroll
-      for (int j = 0; j < 16; ++j) x16[j] = __int2half_rn((int)((f0.x >> (2 * j)) & 3u));  // K and V alike
-    } else if (f_src >= 2) {
-      *reinterpret_cast<uint4*>(x16) = f0;
-      *reinterpret_cast<uint4*>(x16 + 8) = f1;
-    } else {
-#pragma unroll
-      for (int j = 0; j < 16; ++j) x16[j] = __float2half_rn(0.f);
-    }
-    // parts 4..7 store their upper 8 channels first: the 8 lanes of a token
-    // then hit 8 distinct bank quads in each of the two store instructions
-    const int hi1 = (part >> 2) & 1;
-    const uint4 lo8 = *reinterpret_cast<const uint4*>(x16), hi8 = *reinterpret_cast<const uint4*>(x16 + 8);
-    const uint4 first = hi1 ? hi8 : lo8, second = hi1 ? lo8 : hi8;
-    if (!is_v) {
-      __half* row = kc[buf] + tk * kKStride + 16 * part;
-      *reinterpret_cast<uint4*>(row + 8 * hi1) = first;
-      *reinterpret_cast<uint4*>(row + 8 - 8 * hi1) = second;
-    } else {
-      *reinterpret_cast<uint4*>(vt[buf] + vchunk(tk, 2 * part + hi1)) = first;
-      *reinterpret_cast<uint4*>(vt[buf] + vchunk(tk, 2 * part + 1 - hi1)) = second;
-    }
-    if (part < NG) {  // one thread per (token, group, K|V): the group's scale and minimum
-      float s_g = 1.f, m_g = 0.f;  // fp16 rows: the values themselves
-      if (f_src == 1) {
-        s_g = __half2float(__ushort_as_half((unsigned short)(f_sm & 0xffff)));
-        m_g = __half2float(__ushort_as_half((unsigned short)(f_sm >> 16)));
-      } else if (f_src == 0) {
-        s_g = m_g = 0.f;
-      }
-      float(*dst)[NG][2] = is_v ? vsm[buf] : ksm[buf];
-      dst[tk][part][0] = s_g;
-      dst[tk][part][1] = m_g;
-    }
-    if (part == 0 && !is_v) tpos_ok[buf][tk] = f_src != 0;
-  };
-  // chunk 0 staged, chunk 1 fetched, chunk 2's block id in flight
-  fetch(0, chunk_block(0));
-  stage(0);
-  int blk_next = chunk_block(2);
-  if (1 < nchunks) fetch(1, chunk_block(1));
-  __syncthreads();
-  for (int ch = 0; ch < nchunks; ++ch) {
-    const int buf = ch & 1;
-    // chunk ch + 1 goes to the other buffer: its last readers (chunk ch - 1)
-    // passed the barrier that ended the previous iteration
-    if (ch + 1 < nchunks) {
-      stage(buf ^ 1);
-      if (ch + 2 < nchunks) {
-        fetch(ch + 2, blk_next);
-        blk_next = chunk_block(ch + 3);
-      }
-    }
-    // ---- scores of 16 rows x 16 tokens, per group
-    float d[NG][2][4];
-#pragma unroll
-    for (int k = 0; k < NG; ++k)
-#pragma unroll
-      for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) d[k][nt][j] = 0.f;
-    // one group: the low halves accumulate apart, so four chains of mma run side by side
-    float dl[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-#pragma unroll
-    for (int ks = 0; ks < 8; ++ks) {
-      const int k = ks / KSG;
-#pragma unroll
-      for (int nt = 0; nt < 2; ++nt) {
-        const __half* kb = kc[buf] + (8 * nt + g) * kKStride + 16 * ks + 2 * t;
-        const uint32_t b0 = *reinterpret_cast<const uint32_t*>(kb);
-        const uint32_t b1 = *reinterpret_cast<const uint32_t*>(kb + 8);
-        mma_f16_pf(d[k][nt], qa_hi[ks], b0, b1);
-        if constexpr (NG == 1)
-          mma_f16_pf(dl[nt], qa_lo[ks], b0, b1);
-        else
-          mma_f16_pf(d[k][nt], qa_lo[ks], b0, b1);
-      }
-    }
-    if constexpr (NG == 1) {
-#pragma unroll
-      for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) d[0][nt][j] += dl[nt][j];
-    }
-    // score (log2 units) of row h2, token 8 nt + 2 t + c: sum_k s_k raw_k 2^e + m_k sum_k
-    float sc[2][2][2];  // [h2][nt][c]
-#pragma unroll
-    for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        const int tk = 8 * nt + 2 * t + c;
-        const int p = 16 * ch + tk;
-        const bool ok = tpos_ok[buf][tk] != 0;
-#pragma unroll
-        for (int h2 = 0; h2 < 2; ++h2) {
-          float x = 0.f;
-#pragma unroll
-          for (int k = 0; k < NG; ++k)
-            x = fmaf(ksm[buf][tk][k][0] * qup[h2], d[k][nt][2 * h2 + c], fmaf(ksm[buf][tk][k][1], qsum[h2][k], x));
-          sc[h2][nt][c] = (ok && rok[h2] && p <= rpos[h2]) ? x : -INFINITY;
-        }
-      }
-    // online softmax per row (the 4 lanes of a quad share a row)
-    float pr[2][2][2];
-#pragma unroll
-    for (int h2 = 0; h2 < 2; ++h2) {
-      float bm = fmaxf(fmaxf(sc[h2][0][0], sc[h2][0][1]), fmaxf(sc[h2][1][0], sc[h2][1][1]));
-      bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 1));
-      bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 2));
-      const float mnew = fmaxf(mrow[h2], bm);
-      const float mref = mnew == -INFINITY ? 0.f : mnew;
-      const float alpha = exp2f(mrow[h2] - mref);  // 0 while the row has seen nothing
-      mrow[h2] = mnew;
-      float ps = 0.f;
-#pragma unroll
-      for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          pr[h2][nt][c] = exp2f(sc[h2][nt][c] - mref);
-          ps += pr[h2][nt][c];
-        }
-      lrow[h2] = fmaf(lrow[h2], alpha, ps);
-#pragma unroll
-      for (int k = 0; k < NG; ++k) msum[h2][k] *= alpha;
-#pragma unroll
-      for (int n = 0; n < 16; ++n) {
-        o[n][2 * h2] *= alpha;
-        o[n][2 * h2 + 1] *= alpha;
-      }
-    }
-    // values: per group k, A = p s_k (hi + lo) over the 16 tokens, B = codes
-#pragma unroll
-    for (int k = 0; k < NG; ++k) {
-      uint32_t ah[4], al[4];
-      // A registers: (row g, tokens 2t, 2t+1), (g + 8, 2t..), (g, 2t + 8..), (g + 8, 2t + 8..)
-#pragma unroll
-      for (int q4 = 0; q4 < 4; ++q4) {
-        const int h2 = q4 & 1, nt = q4 >> 1;
-        const int t0 = 8 * nt + 2 * t;
-        split_half2(pr[h2][nt][0] * vsm[buf][t0][k][0], pr[h2][nt][1] * vsm[buf][t0 + 1][k][0], ah[q4], al[q4]);
-      }
-#pragma unroll
-      for (int h2 = 0; h2 < 2; ++h2)
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-          for (int c = 0; c < 2; ++c)
-            msum[h2][k] = fmaf(pr[h2][nt][c], vsm[buf][8 * nt + 2 * t + c][k][1], msum[h2][k]);
-      // B operands of n-tiles 2p, 2p + 1 (channels 16p .. 16p + 15, one group):
-      // matrix m of the transposing load is tokens 8 (m & 1) .. + 7 of n-tile 2p + (m >> 1)
-      const int mrow = (lane & 7) + 8 * ((lane >> 3) & 1), mhi = lane >> 4;
-#pragma unroll
-      for (int pp = 0; pp < 8; ++pp) {
-        if (pp * NG / 8 != k) continue;  // channels 16 pp .. belong to group pp ng / 8
-        uint32_t bq[4];
-        ldsm_x4_trans(bq, vt[buf] + vchunk(mrow, 2 * pp + mhi));
-        mma_f16_pf(o[2 * pp], ah, bq[0], bq[1]);
-        mma_f16_pf(o[2 * pp], al, bq[0], bq[1]);
-        mma_f16_pf(o[2 * pp + 1], ah, bq[2], bq[3]);
-        mma_f16_pf(o[2 * pp + 1], al, bq[2], bq[3]);
-      }
-    }
-    __syncthreads();  // chunk ch + 1 is staged; buffer ch & 1 is free
-  }
-  // ---- o' rows and sums to the buffer: the quad's lanes hold columns 2t, 2t + 1 of every n-tile
-#pragma unroll
-  for (int h2 = 0; h2 < 2; ++h2) {
-    float l = lrow[h2];
-    l += __shfl_xor_sync(0xffffffffu, l, 1);
-    l += __shfl_xor_sync(0xffffffffu, l, 2);
-    float ms[NG];
-#pragma unroll
-    for (int k = 0; k < NG; ++k) {
-      ms[k] = msum[h2][k];
-      ms[k] += __shfl_xor_sync(0xffffffffu, ms[k], 1);
-      ms[k] += __shfl_xor_sync(0xffffffffu, ms[k], 2);
-    }
-    if (!rok[h2]) continue;
-    float* dst = a.obuf + (size_t)rrow[h2] * kOStride;
-#pragma unroll
-    for (int n = 0; n < 16; ++n) {
-      const float add = ms[n * NG / 16];
-      *reinterpret_cast<float2*>(dst + 8 * n + 2 * t) = make_float2(o[n][2 * h2] + add, o[n][2 * h2 + 1] + add);
-    }
-    if (t == 0) dst[128] = l;
-  }
-}
-
-// ---------------------------------------------------------------------------
-// 2b. attention on the tcgen05 tensor cores (128- and 64-channel groups, NG =
-// 1 or 2 groups per vector; a group is one 64-channel K-block or both, and its
-// scores, p s and value MMA are kept apart).  A CTA takes
+// 2. attention on the tcgen05 tensor cores (NG = 1, 2 or 4 groups per
+// vector; a group is both 64-channel K-blocks, one of them or half of one,
+// and its scores, p s and value MMA are kept apart).  A CTA takes
 // 128 query rows of one KV head (the MMA's M) and streams the key positions
 // in chunks of 64 (four cache blocks), with warp roles:
 //   warps 0-7  softmax: warp w serves rows 32 (w % 4) .. + 31 (TMEM lanes,
@@ -552,9 +205,10 @@ __global__ void __launch_bounds__(kPfWarps * 32) prefill_attn_kernel(PrefillArgs
 //              keys as [token][channel], values transposed to
 //              [channel][token] -- and the per-token (scale, min) pairs;
 //   warp 12    TMEM allocation; lane 0 issues the MMAs:
-//              S(c) = q~hi K^T + q~lo K^T (M 128, N 64, K 128) into one of
-//              two TMEM score buffers, O += (p s)hi V + (p s)lo V (M 128,
-//              N 128, K 64) into the TMEM output.
+//              S(c) = q~hi K^T + q~lo K^T (M 128, N 64 per group, K 128
+//              over the groups) into one of two TMEM score buffers (one with
+//              four groups), O += (p s)hi V + (p s)lo V (M 128, N 128 / NG
+//              per group, K 64) into the TMEM output.
 // Both MMAs take their A operand from TMEM (q~ is staged there once; p s
 // replaces the scores it came from), so shared memory holds only the key and
 // value tiles and the MMAs read nothing else from it.
@@ -585,13 +239,13 @@ constexpr uint32_t kUpOffK = 0;
 constexpr uint32_t kUpOffV = kUpOffK + 2 * kUpKBytes;
 constexpr uint32_t kUpOffMisc = kUpOffV + 2 * kUpVBytes;
 struct UpMisc {
-  float2 ksm[2][2 * kUpKC];         // key (scale, min) of token j, group k at j NG + k: (1, 0) fp16 rows, (0, 0) masked
-  float2 vsm[2][2 * kUpKC];         // value (scale, min), the same way
+  float2 ksm[2][4 * kUpKC];         // key (scale, min) of token j, group k at j NG + k: (1, 0) fp16 rows, (0, 0) masked
+  float2 vsm[2][4 * kUpKC];         // value (scale, min), the same way
   int kval[2][kUpKC];               // 1 where the token was staged (only read when a block id was bad)
   float vsmax[2][kUpStgWarps];      // largest value scale, per staging warp
   int bad[2][kUpStgWarps];          // a block id was out of range, per staging warp
   float red[2][2][128];             // per chunk parity, column half, row: the half-row maximum
-  float4 fin[2][128];               // per column half, row: (l, sum p m of group 0, of group 1) at the end
+  float4 fin[2][128];               // per column half, row: l and the sums p m the partner needs, at the end
   uint64_t k_full[2], v_full[2], s_full[2], s_free[2], p_full[2], pv_done[2], mx[4][2];
   uint32_t tmem_slot;
 };
@@ -599,11 +253,14 @@ constexpr size_t kUpSmem = 1024 + kUpOffMisc + sizeof(UpMisc);
 // TMEM columns: scores 2 x 64 NG from 0 (group k's 64 columns at 64 k; p s
 // of a group then replaces its scores: per column half h of the row, hi at
 // 32 h + 0..15 and lo at 32 h + 16..31 of the group's columns); O 128 from
-// 128 NG; q~ hi 64 and lo 64 after O
+// 128 NG; q~ hi 64 and lo 64 after O.  With four groups (32-channel groups)
+// two score buffers would fill TMEM: one buffer of 256 columns, O at 256, q~
+// at 384, and the score MMAs of chunk c + 1 wait for the value MMAs of c.
 constexpr uint32_t kUpTmemCols = 512;
 constexpr uint32_t kUpIdescS = um_idesc(64, false, false);
 constexpr uint32_t kUpIdescO = um_idesc(128, false, false);
 constexpr uint32_t kUpIdescO64 = um_idesc(64, false, false);
+constexpr uint32_t kUpIdescO32 = um_idesc(32, false, false);
 constexpr uint32_t kF16Bias2 = 0x64006400u;  // (1024, 1024) as fp16 pair: 1024 + c is exact for c < 1024
 
 // (1024 + lo, 1024 + hi) - 1024 for two 2-bit codes already in bits 0-1 and 16-17
@@ -661,9 +318,12 @@ __device__ __forceinline__ float ex2_ftz(float x) {
 
 template <int NG>
 __global__ void __launch_bounds__(kUpThreads, 1) prefill_umma_kernel(PrefillArgs a) {
-  static_assert(NG == 1 || NG == 2, "one or two 64-channel groups per vector");
-  constexpr int kSW = 64 * NG;  // score columns per buffer
-  constexpr uint32_t kUpColO = 2 * kSW, kUpColQ = 2 * kSW + 128;
+  static_assert(NG == 1 || NG == 2 || NG == 4, "one, two or four quantisation groups per vector");
+  constexpr int kSW = 64 * NG;                  // score columns per buffer
+  constexpr int kSBufs = NG == 4 ? 1 : 2;       // score buffers (TMEM holds one of four groups' width)
+  constexpr uint32_t kUpColO = kSBufs * kSW, kUpColQ = kSBufs * kSW + 128;
+  static_assert(kUpColQ + 128 <= kUpTmemCols, "TMEM columns");
+  auto sbuf = [](int b) -> uint32_t { return kSBufs == 1 ? 0u : (uint32_t)(b * kSW); };
   extern __shared__ unsigned char up_raw[];
   const uint32_t raw_u32 = smem_u32(up_raw);
   const uint32_t base = (raw_u32 + 1023u) & ~1023u;  // swizzle atoms need 1024-byte alignment
@@ -986,12 +646,35 @@ __global__ void __launch_bounds__(kUpThreads, 1) prefill_umma_kernel(PrefillArgs
       if (!alive) break;
       um_fence_after();
       float sv[32];
-      um_ld32(tS + lane_base + (uint32_t)(b * kSW + 32 * hcol), sv);
-      if constexpr (NG == 2) {
+      um_ld32(tS + lane_base + sbuf(b) + (uint32_t)(32 * hcol), sv);
+      if constexpr (NG == 4) {
+        // x = sum over the four groups of s_k (q~_k . c_k) 2^e + m_k sum q~_k, one group's raw
+        // scores at a time
+        um_wait_ld();
+        const float4* kk = reinterpret_cast<const float4*>(&ms.ksm[b][4 * 32 * hcol]);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const float4 k4 = kk[2 * j];  // (s, m) of groups 0 and 1 of token j
+          sv[j] = fmaf(k4.x * qup, sv[j], k4.y * qsum_g[0]);
+        }
+#pragma unroll 1
+        for (int k = 1; k < 4; ++k) {
+          float svk[32];
+          um_ld32(tS + lane_base + sbuf(b) + (uint32_t)(64 * k + 32 * hcol), svk);
+          um_wait_ld();
+          const float2* k2 = &ms.ksm[b][4 * 32 * hcol + k];
+          const float qg = k == 1 ? qsum_g[1] : k == 2 ? qsum_g[2] : qsum_g[3];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const float2 sm = k2[4 * j];
+            sv[j] = fmaf(sm.x * qup, svk[j], fmaf(sm.y, qg, sv[j]));
+          }
+        }
+      } else if constexpr (NG == 2) {
         // x = s0 (q~0 . c0) + m0 sum q~0 + s1 (q~1 . c1) + m1 sum q~1: group 1's raw scores
         // and both groups' (scale, min) fold in here; the common code below then sees s = 1, m = 0
         float sv1[32];
-        um_ld32(tS + lane_base + (uint32_t)(b * kSW + 64 + 32 * hcol), sv1);
+        um_ld32(tS + lane_base + sbuf(b) + (uint32_t)(64 + 32 * hcol), sv1);
         um_wait_ld();
         const float4* kk = reinterpret_cast<const float4*>(&ms.ksm[b][2 * 32 * hcol]);
 #pragma unroll
@@ -1008,7 +691,7 @@ __global__ void __launch_bounds__(kUpThreads, 1) prefill_umma_kernel(PrefillArgs
       const bool bad = (ms.bad[b][0] | ms.bad[b][1] | ms.bad[b][2] | ms.bad[b][3]) != 0;
       const float4* k4p = reinterpret_cast<const float4*>(&ms.ksm[b][32 * hcol]);
       float bm = -INFINITY;
-      if constexpr (NG == 2) {
+      if constexpr (NG >= 2) {
         const int* kv = &ms.kval[b][32 * hcol];
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
@@ -1085,8 +768,8 @@ __global__ void __launch_bounds__(kUpThreads, 1) prefill_umma_kernel(PrefillArgs
       // p s over the scores of chunk c in TMEM: columns 16 hcol .. (hi) and
       // 32 + 16 hcol .. (lo) of the chunk's buffer.  The lo columns held the
       // partner's scores, which it read before it posted its maximum; the
-      // value MMA of chunk c - 2, the last reader of this buffer's p s,
-      // finished before S(c) was written into it.
+      // value MMA of chunk c - 2 (c - 1 with one buffer), the last reader of
+      // this buffer's p s, finished before S(c) was written into it.
       um_fence_after();
 #pragma unroll
       for (int k = 0; k < NG; ++k) {
@@ -1110,7 +793,7 @@ __global__ void __launch_bounds__(kUpThreads, 1) prefill_umma_kernel(PrefillArgs
         // NG = 1: hi at 16 hcol, lo at 32 + 16 hcol (the lo columns held the partner's
         // scores, read before it posted its maximum); NG = 2: over this thread's own
         // 32 score columns of group k
-        const uint32_t tp = tS + lane_base + (uint32_t)(b * kSW) +
+        const uint32_t tp = tS + lane_base + sbuf(b) +
                             (NG == 1 ? 16u * (uint32_t)hcol : 64u * (uint32_t)k + 32u * (uint32_t)hcol);
         um_st16(tp, hi);
         um_st16(tp + (NG == 1 ? 32u : 16u), lo);
@@ -1123,18 +806,32 @@ __global__ void __launch_bounds__(kUpThreads, 1) prefill_umma_kernel(PrefillArgs
       alive = mbar_wait_bounded(&ms.pv_done[(nch - 1) & 1], ((uint32_t)(nch - 1) >> 1) & 1u);
       alive = __all_sync(0xffffffffu, alive);
     }
-    float l = 0.f, msum = 0.f;
+    float l = 0.f, msum = 0.f, msum_b = 0.f;  // msum_b: channels 64 hcol + 32 .. with four groups
     if (alive) {
       // the two halves' sums meet: one more round of the partners' barrier
-      ms.fin[hcol][rowc] = make_float4(l2.x + l2.y, msum2[0].x + msum2[0].y,
-                                       NG == 2 ? msum2[NG - 1].x + msum2[NG - 1].y : 0.f, 0.f);
+      if constexpr (NG == 4) {
+        // the partner writes channels 64 (1 - hcol) ..: groups 2 (1 - hcol) and + 1
+        const float2 a0 = hcol ? msum2[0] : msum2[2], a1 = hcol ? msum2[1] : msum2[3];
+        ms.fin[hcol][rowc] = make_float4(l2.x + l2.y, a0.x + a0.y, a1.x + a1.y, 0.f);
+      } else {
+        ms.fin[hcol][rowc] = make_float4(l2.x + l2.y, msum2[0].x + msum2[0].y,
+                                         NG == 2 ? msum2[NG - 1].x + msum2[NG - 1].y : 0.f, 0.f);
+      }
       mbar_arrive(&ms.mx[quarter][nch & 1]);
       alive = mbar_wait_bounded(&ms.mx[quarter][nch & 1], ((uint32_t)nch >> 1) & 1u);
       alive = __all_sync(0xffffffffu, alive);
       const float4 f0 = ms.fin[0][rowc], f1 = ms.fin[1][rowc];
       l = f0.x + f1.x;
-      // this thread writes channels 64 hcol ..: group hcol when NG = 2
-      msum = (NG == 2 && hcol == 1) ? f0.z + f1.z : f0.y + f1.y;
+      if constexpr (NG == 4) {
+        const float4 fp = hcol ? f0 : f1;  // the partner's post
+        const float2 o0 = hcol ? msum2[2] : msum2[0], o1 = hcol ? msum2[3] : msum2[1];
+        msum = (o0.x + o0.y) + fp.y;
+        msum_b = (o1.x + o1.y) + fp.z;
+      } else {
+        // this thread writes channels 64 hcol ..: group hcol when NG = 2
+        msum = (NG == 2 && hcol == 1) ? f0.z + f1.z : f0.y + f1.y;
+        msum_b = msum;
+      }
     }
     if (alive) {
       um_fence_after();
@@ -1145,10 +842,11 @@ __global__ void __launch_bounds__(kUpThreads, 1) prefill_umma_kernel(PrefillArgs
         um_ld32(tO + lane_base + (uint32_t)(64 * hcol + 32 * q), ov);
         um_wait_ld();
         if (rok) {
+          const float mq = q ? msum_b : msum;
 #pragma unroll
           for (int i = 0; i < 32; i += 4)
             *reinterpret_cast<float4*>(dst + 32 * q + i) =
-                make_float4(ov[i] + msum, ov[i + 1] + msum, ov[i + 2] + msum, ov[i + 3] + msum);
+                make_float4(ov[i] + mq, ov[i + 1] + mq, ov[i + 2] + mq, ov[i + 3] + mq);
         }
       }
       if (rok && hcol == 0) a.obuf[(size_t)rrow * kOStride + 128] = l;
@@ -1199,6 +897,12 @@ __global__ void __launch_bounds__(kUpThreads, 1) prefill_umma_kernel(PrefillArgs
       const int b = c & 1;
       if (!mbar_wait_bounded(&ms.k_full[b], ((uint32_t)c >> 1) & 1u)) return false;
       if (c >= 2 && !mbar_wait_bounded(&ms.s_free[b], ((uint32_t)(c - 2) >> 1) & 1u)) return false;
+      // one score buffer: the value MMAs of c - 1 read their p s from it
+      // (waiting for their completion here measured faster than relying on
+      // the issue order of this thread's MMAs)
+      if (kSBufs == 1 && c >= 1 &&
+          !mbar_wait_bounded(&ms.pv_done[(c - 1) & 1], ((uint32_t)(c - 1) >> 1) & 1u))
+        return false;
       um_fence_after();
       const uint64_t kd = b ? dK1 : dK0;
 #pragma unroll
@@ -1210,9 +914,11 @@ __global__ void __launch_bounds__(kUpThreads, 1) prefill_umma_kernel(PrefillArgs
             // q~ channels 64 kb + 16 ks .. + 15: TMEM columns 8 (4 kb + ks) of its half
             const uint32_t ta = tQ + 64u * (uint32_t)half + 8u * (uint32_t)(4 * kb + ks);
             const uint64_t bd = kd + (uint64_t)((kb * 8192 + ks * 32) >> 4);
-            // NG = 2: K-block kb is group kb, into its own 64 columns
-            um_mma_ts(tS + (uint32_t)(b * kSW) + (NG == 2 ? 64u * (uint32_t)kb : 0u), ta, bd, kUpIdescS,
-                      (half | ks | (NG == 2 ? 0 : kb)) != 0 ? 1u : 0u);
+            // NG = 2: K-block kb is group kb, into its own 64 columns; NG = 4: channels
+            // 32 g .. of group g = 2 kb + ks / 2
+            const uint32_t gcol = NG == 2 ? 64u * (uint32_t)kb : NG == 4 ? 64u * (uint32_t)(2 * kb + (ks >> 1)) : 0u;
+            const int first = NG == 2 ? (half | ks) : NG == 4 ? (half | (ks & 1)) : (half | ks | kb);
+            um_mma_ts(tS + sbuf(b) + gcol, ta, bd, kUpIdescS, first != 0 ? 1u : 0u);
           }
       um_commit(&ms.s_full[b]);
       last_bar = &ms.s_full[b];
@@ -1231,10 +937,24 @@ __global__ void __launch_bounds__(kUpThreads, 1) prefill_umma_kernel(PrefillArgs
 #pragma unroll
           for (int ks = 0; ks < 4; ++ks) {
             // tokens 16 ks .. + 15 of p s (hi or lo): TMEM columns 32 half + 8 ks of the chunk's buffer
-            const uint32_t ta = tS + (uint32_t)(b * kSW) + 32u * (uint32_t)half + 8u * (uint32_t)ks;
+            const uint32_t ta = tS + sbuf(b) + 32u * (uint32_t)half + 8u * (uint32_t)ks;
             const uint64_t bd = vd + (uint64_t)((ks * 32) >> 4);
             um_mma_ts(tO, ta, bd, kUpIdescO, (c > 0 || half > 0 || ks > 0) ? 1u : 0u);
           }
+      } else if constexpr (NG == 4) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+#pragma unroll
+          for (int half = 0; half < 2; ++half)
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks) {
+              // group k (channel rows 32 k .., output columns 32 k ..), tokens 16 ks ..: p s as
+              // for two groups, in the group's 64 score columns
+              const uint32_t ta = tS + 64u * (uint32_t)k + 32u * (uint32_t)(ks >> 1) + 16u * (uint32_t)half +
+                                  8u * (uint32_t)(ks & 1);
+              const uint64_t bd = vd + (uint64_t)((k * 4096 + ks * 32) >> 4);
+              um_mma_ts(tO + 32u * (uint32_t)k, ta, bd, kUpIdescO32, (c > 0 || half > 0 || ks > 0) ? 1u : 0u);
+            }
       } else {
 #pragma unroll
         for (int k = 0; k < 2; ++k)
@@ -1244,7 +964,7 @@ __global__ void __launch_bounds__(kUpThreads, 1) prefill_umma_kernel(PrefillArgs
             for (int ks = 0; ks < 4; ++ks) {
               // group k, tokens 16 ks ..: p s written by column half ks / 2 at 32 (ks / 2) +
               // 16 half + 8 (ks % 2) of the group's columns; values: channel rows 64 k ..
-              const uint32_t ta = tS + (uint32_t)(b * kSW) + 64u * (uint32_t)k + 32u * (uint32_t)(ks >> 1) +
+              const uint32_t ta = tS + sbuf(b) + 64u * (uint32_t)k + 32u * (uint32_t)(ks >> 1) +
                                   16u * (uint32_t)half + 8u * (uint32_t)(ks & 1);
               const uint64_t bd = vd + (uint64_t)((k * 8192 + ks * 32) >> 4);
               um_mma_ts(tO + 64u * (uint32_t)k, ta, bd, kUpIdescO64, (c > 0 || half > 0 || ks > 0) ? 1u : 0u);
@@ -1255,8 +975,13 @@ __global__ void __launch_bounds__(kUpThreads, 1) prefill_umma_kernel(PrefillArgs
       last_par = ((uint32_t)c >> 1) & 1u;
       return true;
     };
-    bool alive = issue_s(0) && (nch < 2 || issue_s(1));
-    for (int c = 0; c < nch && alive; ++c) alive = issue_pv(c) && (c + 2 >= nch || issue_s(c + 2));
+    bool alive = issue_s(0);
+    if constexpr (kSBufs == 2) {
+      alive = alive && (nch < 2 || issue_s(1));
+      for (int c = 0; c < nch && alive; ++c) alive = issue_pv(c) && (c + 2 >= nch || issue_s(c + 2));
+    } else {
+      for (int c = 0; c < nch && alive; ++c) alive = issue_pv(c) && (c + 1 >= nch || issue_s(c + 1));
+    }
     if (!alive) raise_flag(a.status, OKV_DEV_TIMEOUT);
     // the MMAs already issued finish before TMEM is freed (the softmax warps may
     // have given up on them): the last commit covers them all
@@ -1411,7 +1136,13 @@ okv_status launch_prefill(const okv_cache_desc* d, const void* q, int T, int slo
       prefill_umma_kernel<2><<<grid, kUpThreads, kUpSmem, s>>>(a);
       break;
     }
-    default: prefill_attn_kernel<4><<<grid, kPfWarps * 32, 0, s>>>(a); break;
+    default: {
+      static std::atomic<uint32_t> up4_attr{0};
+      cudaError_t e1 = set_smem_limit_once((const void*)prefill_umma_kernel<4>, (int)kUpSmem, up4_attr);
+      if (e1 != cudaSuccess) return fail(OKV_ERR_CUDA, "prefill attention smem attribute: %s", cudaGetErrorString(e1));
+      prefill_umma_kernel<4><<<grid, kUpThreads, kUpSmem, s>>>(a);
+      break;
+    }
   }
   st = check_launch("prefill attention");
   if (st != OKV_OK) return st;

@@ -90,6 +90,27 @@ def test_prefill_grouped(group):
     _check(got, want, G)
 
 
+@pytest.mark.parametrize("group", [64, 32])
+@pytest.mark.parametrize("hq,hkv,L,T,sinks,scale,vscale", [
+    (8, 8, 700, 130, 32, 1.0, 1.0),       # G = 1, sinks, a ragged last tile
+    (64, 8, 1300, 40, 0, 1.0, 1.0),       # G = 8
+    (8, 2, 1200, 64, 0, 30.0, 1.0),       # peaked rows
+    (8, 2, 1500, 100, 0, 1.0, 8000.0),    # value scales near the top of fp16
+    (16, 4, 90, 90, 0, 1.0, 1.0),         # shorter than the window: all fp16
+])
+def test_prefill_grouped_shapes(group, hq, hkv, L, T, sinks, scale, vscale):
+    got, want, G = _case(60 + hq + T, hq, hkv, L, T, group=group, sinks=sinks, scale=scale, vscale=vscale,
+                         checked=[0, hkv - 1])
+    _check(got, want, G)
+
+
+def test_prefill_grouped_benchmark_shape_sampled():
+    """32-channel groups at the prefill benchmark's shape (1,024 tokens ending
+    32,768, 32 / 8 heads), sampled chunk tokens."""
+    got, want, G = _case(61, 32, 8, 32768, 1024, group=32, checked=[3], tokens=[0, 511, 1023])
+    _check(got, want, G)
+
+
 def test_prefill_with_sinks():
     got, want, G = _case(53, 8, 2, 1000, 150, sinks=192)
     _check(got, want, G)
