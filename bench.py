@@ -550,7 +550,7 @@ def prefill_attention_rate(torch, okv, WL, seed, L=32768, T=1024, group=128):
     peak, src = measured_peak_bf16()
     tflops = flops / us / 1e6
     return {"context": L, "chunk_tokens": T, "hq": hq, "hkv": hkv, "group": group,
-            "kernel": "tcgen05" if group in (128, 64) else "mma.sync (per-group scales)", "us": round(us, 1),
+            "kernel": "tcgen05", "us": round(us, 1),
             "tflops": round(tflops, 1), "flops": flops,
             "roofline": {"bound": "tensor", "achieved": round(tflops, 1), "peak": peak, "unit": "TFLOP/s",
                          "frac": round(tflops / peak, 4), "peak_source": src,
