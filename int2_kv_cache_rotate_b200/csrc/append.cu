@@ -121,7 +121,7 @@ __device__ __forceinline__ void finish_token_tc(const AppendArgs& a, int tok, bo
 #pragma unroll
     for (int k = 0; k < 8; ++k)
 #pragma unroll
-      for (int f = 0; f < 4; ++f) w[k >> 2] |= int2_code(__fsub_rn(v[k][f], m), th) << (8 * (k & 3) + 2 * f);
+      for (int f = 0; f < 4; ++f) w[k >> 2] -= int2_code_neg(__fsub_rn(v[k][f], m), th) << (8 * (k & 3) + 2 * f);
   }
   uint8_t* base = a.pages + ((size_t)blk * a.hkv + h) * a.bhb;
   const int sl = p & 15;
@@ -568,7 +568,8 @@ __global__ void __launch_bounds__(kUmThreads, 1) append_umma_kernel(AppendArgs a
         if (sc != 0.0f) {
           const CodeThresholds th = code_thresholds(sc);
 #pragma unroll
-          for (int j = GW * k; j < GW * (k + 1); ++j) w[j >> 4] |= int2_code(__fsub_rn(v[j], m), th) << (2 * (j & 15));
+          for (int j = GW * k; j < GW * (k + 1); ++j)
+            w[j >> 4] -= int2_code_neg(__fsub_rn(v[j], m), th) << (2 * (j & 15));  // += code << 2 (j % 16)
         }
       }
       uint8_t* bp = a.pages + ((size_t)(valid ? blk : 0) * a.hkv + h) * a.bhb;

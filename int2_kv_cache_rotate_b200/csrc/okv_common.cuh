@@ -116,9 +116,17 @@ __device__ __forceinline__ CodeThresholds code_thresholds(float s) {
   return t;
 }
 
-// code of x = fl(z - m); only for s > 0 (s = 0 gives code 0 by definition)
-__device__ __forceinline__ uint32_t int2_code(float x, const CodeThresholds& t) {
-  return (uint32_t)(x > t.h1) + (uint32_t)(x >= t.h2) + (uint32_t)(x > t.h3);
+// The code of x = fl(z - m) (only for s > 0; s = 0 gives code 0 by
+// definition) is [x > s/2] + [x >= 3s/2] + [x > 5s/2].  This returns -code
+// (mod 2^32) as the sum of the three decisions as all-ones / zero masks (PTX
+// `set` writes 0xffffffff for true), so that w - (int2_code_neg(x, t) << k)
+// adds code << k to w.
+__device__ __forceinline__ uint32_t int2_code_neg(float x, const CodeThresholds& t) {
+  uint32_t a, b, c;
+  asm("set.gt.u32.f32 %0, %1, %2;" : "=r"(a) : "f"(x), "f"(t.h1));
+  asm("set.ge.u32.f32 %0, %1, %2;" : "=r"(b) : "f"(x), "f"(t.h2));
+  asm("set.gt.u32.f32 %0, %1, %2;" : "=r"(c) : "f"(x), "f"(t.h3));
+  return a + b + c;
 }
 
 // INT2 group quantiser over the 128 values of a warp (y[a] = value at
@@ -151,7 +159,7 @@ __device__ __forceinline__ Quantized quantize_warp(const float y[4], int ng = 1)
   if (s != 0.0f) {
     const CodeThresholds th = code_thresholds(s);
 #pragma unroll
-    for (int a = 0; a < 4; ++a) byte |= int2_code(__fsub_rn(y[a], m), th) << (2 * rev2(a));
+    for (int a = 0; a < 4; ++a) byte -= int2_code_neg(__fsub_rn(y[a], m), th) << (2 * rev2(a));
   }
   Quantized q;
   q.byte = byte;
