@@ -100,6 +100,17 @@ def test_validation_before_launch():
     # dequantize argument checks
     assert lib.okv_dequantize(ctypes.byref(d), 1, fake, fake, fake, 16, 2, 0, 0, fake, None) == okv.ERR_INVALID_ARG
     assert lib.okv_dequantize(ctypes.byref(d), 1, fake, fake, fake, 0, 0, 0, 0, fake, None) == okv.OK
+    # staged rotation image: size, a buffer to build into, 16-byte alignment
+    assert lib.okv_r_image_bytes(8) == 8 * 2 * 3 * 128 * 128 * 2
+    assert lib.okv_r_image_bytes(-1) == 0
+    assert lib.okv_build_r_image(ctypes.byref(d), None) == okv.ERR_INVALID_ARG
+    assert b"r_image" in lib.okv_last_error_string()
+    d4 = _desc()
+    d4.r_image = (1 << 22) + 8
+    assert lib.okv_build_r_image(ctypes.byref(d4), None) == okv.ERR_INVALID_ARG
+    assert lib.okv_append_quantize(ctypes.byref(d4), fake, fake, 1, fake, fake, fake, fake, 0, None, None) \
+        == okv.ERR_INVALID_ARG
+    assert b"r_image" in lib.okv_last_error_string()
 
 
 def test_calibrate_validation():
