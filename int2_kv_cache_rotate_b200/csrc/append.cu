@@ -1,7 +1,8 @@
 // Append kernels: rotate (U, Hadamard butterfly, bit-reversal remap), quantise
 // to INT2 with fp16 scale/min, pack, and write the paged cache and fp16 window.
 // Decode steps (a few tokens) run the CUDA-core kernel; prefill chunks of 128
-// tokens or more run the tensor-core kernel.
+// tokens or more run the tensor-core kernel, which takes R either from the
+// cache's staged image (okv_build_r_image) or stages it from U per CTA.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -43,7 +44,7 @@ __global__ void __launch_bounds__(kAppThreads) append_kernel(AppendArgs a, int T
 // are padded to 136 elements so the eight rows of a matrix fall in distinct
 // bank groups.
 // ---------------------------------------------------------------------------
-constexpr int kTcMinTokens = 128;  // below this the CUDA-core kernel wins (R staging dominates)
+constexpr int kTcMinTokens = 128;  // below this the CUDA-core kernel wins (R staging or its copy dominates)
 constexpr int kTcWarps = 8;
 constexpr int kTcRound = 16 * kTcWarps;  // tokens per CTA round
 constexpr int kRStride = 136;            // bf16 per staged row of R
