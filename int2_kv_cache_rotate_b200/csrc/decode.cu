@@ -98,6 +98,7 @@ struct DecodeArgs {
   float* part;       // [(NC + B)][Hq][kPartStride]
   int batch, hq, hkv, g, nc, num_blocks, num_slots, mbps, nsink;
   int ng;  // quantisation groups per vector (128 / group)
+  int hsplit;  // split-K CTAs per cost range: each serves G / hsplit query heads of every KV head
 };
 
 // split-K CTA count actually used: with fewer cost units than CTAs only the
@@ -705,7 +706,7 @@ __device__ __forceinline__ void mma_flush(MmaWarpState<G, NGQ>& st, int (&acci)[
   }
 }
 
-template <int G, int NGQ>
+template <int G, int NGQ, int HS = 1>
 __global__ void __launch_bounds__(kHW * 32, (G <= 4) ? 2 : 1) decode_heads_kernel(DecodeArgs a) {
   using Cfg = HCfg<G, NGQ>;
   static_assert(NGQ == 1 || G <= 4, "grouped layouts take G <= 4 (one n-tile)");
@@ -731,6 +732,13 @@ __global__ void __launch_bounds__(kHW * 32, (G <= 4) ? 2 : 1) decode_heads_kerne
   const int nb = 2 * wph;                // blocks per stage
   const uint32_t copy_bytes = (uint32_t)hkv * BHB;
   grid_dep_launch();  // the combine kernel may take SMs as split-K CTAs finish
+  // With HS > 1 the grid holds HS CTAs per cost range: CTA range + a.nc hh
+  // serves query heads G hh .. G hh + G - 1 of every KV head (G here is the
+  // query heads one CTA takes; a KV head has G HS).  The CTAs of a range
+  // stream the same blocks, the later ones mostly from L2.  (Built for the
+  // grouped layouts at G = 8; one group per vector takes G = 8 in one CTA.)
+  // first query head this CTA serves of KV head h (recomputed where used: fewer live registers)
+  auto qhead0 = [&](int h) { return HS == 1 ? h * G : h * G * HS + G * ((int)blockIdx.x / a.nc); };
 
   // The work partition, computed here from the context lengths with loads that
   // bypass L1, so that this kernel can start (and put its first copies in
@@ -762,8 +770,9 @@ __global__ void __launch_bounds__(kHW * 32, (G <= 4) ? 2 : 1) decode_heads_kerne
     before += inc - own;
     if (total > 0) {
       const int ncw = (int)min((long long)a.nc, (long long)total);
-      const long long st0 = (long long)blockIdx.x * total / ncw;
-      if ((int)blockIdx.x < ncw && st0 >= before && st0 < before + own) {
+      const int cr = HS == 1 ? (int)blockIdx.x : (int)blockIdx.x % a.nc;  // cost range
+      const long long st0 = (long long)cr * total / ncw;
+      if (cr < ncw && st0 >= before && st0 < before + own) {
         int pu = before;
         for (int i = i0; i < i1; ++i) {
           const int cst = unit_shape(clamp_len_cg(a.context_lens, i, a.mbps), a.nsink).cost;
@@ -779,7 +788,9 @@ __global__ void __launch_bounds__(kHW * 32, (G <= 4) ? 2 : 1) decode_heads_kerne
     __syncthreads();
   }
   const int nc = (int)min((long long)a.nc, (long long)total);
-  const int c = blockIdx.x;
+  // cost range of this CTA (recomputed where used, like qhead0)
+  auto crange = [&]() -> int { return HS == 1 ? (int)blockIdx.x : (int)blockIdx.x % a.nc; };
+  const int c = crange();
   if (total == 0 || c >= nc) {
     grid_dep_wait();  // no CTA finishes before the query rotation has
     return;
@@ -817,7 +828,7 @@ __global__ void __launch_bounds__(kHW * 32, (G <= 4) ? 2 : 1) decode_heads_kerne
     const int slot = __ldcg(a.seq_slot + b);
     const bool slot_ok = slot >= 0 && slot < a.num_slots;
     const int l0 = (int)(max(start, pu) - pu), l1 = (int)(min(end, pu + us.cost) - pu);
-    const size_t bh0 = (size_t)b * a.hq + (size_t)head * G;  // first query head of this warp's KV head
+    const size_t bh0 = (size_t)b * a.hq + (size_t)qhead0(head);  // first query head served
     __syncthreads();  // the previous entry's window scratch / merge buffers (on the ring) are free again
     if (!slot_ok && threadIdx.x == 0) raise_flag(a.status, OKV_DEV_BAD_SLOT);
 
@@ -888,7 +899,8 @@ __global__ void __launch_bounds__(kHW * 32, (G <= 4) ? 2 : 1) decode_heads_kerne
       __syncwarp();
       if (bid >= 0)
         bulk_g2s_hint(ring + s * kStageBytes + q * copy_bytes, a.pages + (size_t)bid * copy_bytes, copy_bytes,
-                      &full[s], l2_evict_first_policy());  // each block is read once
+                      &full[s], HS > 1 ? l2_evict_normal_policy() : l2_evict_first_policy());
+        // (each block is read once, or once per CTA of its range)
       issued = max(issued, first + cnt);
       return true;
     };
@@ -1413,9 +1425,9 @@ __global__ void __launch_bounds__(kHW * 32, (G <= 4) ? 2 : 1) decode_heads_kerne
         uint32_t va[4], vb[4];
 #pragma unroll
         for (int w = 0; w < 4; ++w) {
-          const int c = NGQ == 2 ? 4 * (w >> 1) + (g & 3) : 2 * w + (g & 1);
+          const int ch = NGQ == 2 ? 4 * (w >> 1) + (g & 3) : 2 * w + (g & 1);  // chunk row
           const int jj = NGQ == 2 ? (g >> 2) + 2 * (w & 1) : g >> 1;
-          const int off = kVcOff + 16 * (4 * c + t) + 4 * jj;
+          const int off = kVcOff + 16 * (4 * ch + t) + 4 * jj;
           va[w] = *reinterpret_cast<const uint32_t*>(s0 + off);
           vb[w] = *reinterpret_cast<const uint32_t*>(s1 + off);
         }
@@ -1642,7 +1654,7 @@ __global__ void __launch_bounds__(kHW * 32, (G <= 4) ? 2 : 1) decode_heads_kerne
     }
 
     // ---------------- partial for (c, b): one warp per KV head, or merged across its warps ----------------
-    float* part_b = a.part + ((size_t)(c + b) * a.hq + (size_t)head * G) * kPartStride;
+    float* part_b = a.part + ((size_t)(crange() + b) * a.hq + (size_t)qhead0(head)) * kPartStride;
     if (wph == 1) {
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
@@ -1715,7 +1727,7 @@ __global__ void __launch_bounds__(kHW * 32, (G <= 4) ? 2 : 1) decode_heads_kerne
             l = fmaf(ml[(w * G + gg) * 2 + 1], sc, l);
           }
         }
-        float* dst = a.part + ((size_t)(c + b) * a.hq + (size_t)hh * G + gg) * kPartStride;
+        float* dst = a.part + ((size_t)(crange() + b) * a.hq + (size_t)qhead0(hh) + gg) * kPartStride;
         dst[ch] = o;
         if (ch == 0) {
           dst[128] = mx;
@@ -1927,13 +1939,15 @@ static cudaError_t launch_pdl(void (*kernel)(Args...), dim3 grid, dim3 block, si
   return cudaLaunchKernelEx(&cfg, kernel, args...);
 }
 
-template <int G, int NGQ = 1>
+template <int G, int NGQ = 1, int HS = 1>
 static okv_status launch_decode_heads(const DecodeArgs& a, cudaStream_t s, bool early) {
+  if (a.hsplit != HS || HS * G != a.g)
+    return fail(OKV_ERR_UNSUPPORTED, "split-K head split %d x %d != %d", a.hsplit, G, a.g);
   const size_t smem = HCfg<G, NGQ>::smem_bytes();
   static std::atomic<uint32_t> attr_set{0};
-  cudaError_t e = set_smem_limit_once((const void*)decode_heads_kernel<G, NGQ>, (int)smem, attr_set);
+  cudaError_t e = set_smem_limit_once((const void*)decode_heads_kernel<G, NGQ, HS>, (int)smem, attr_set);
   if (e != cudaSuccess) return fail(OKV_ERR_CUDA, "decode smem attribute: %s", cudaGetErrorString(e));
-  e = launch_pdl(decode_heads_kernel<G, NGQ>, dim3(a.nc), dim3(kHW * 32), smem, s, early, a);
+  e = launch_pdl(decode_heads_kernel<G, NGQ, HS>, dim3(a.nc * HS), dim3(kHW * 32), smem, s, early, a);
   if (e != cudaSuccess) return fail(OKV_ERR_CUDA, "decode launch: %s", cudaGetErrorString(e));
   return check_launch("decode");
 }
@@ -1941,7 +1955,7 @@ static okv_status launch_decode_heads(const DecodeArgs& a, cudaStream_t s, bool 
 bool decode_uses_tensor_cores(int g, int hkv, int ng) {
   const bool hkv_ok = hkv == 1 || hkv == 2 || hkv == 4 || hkv == 8;
   if (ng == 1) return hkv_ok && (g == 1 || g == 2 || g == 4 || g == 8);
-  return hkv_ok && (ng == 2 || ng == 4) && (g == 1 || g == 2 || g == 4);
+  return hkv_ok && (ng == 2 || ng == 4) && (g == 1 || g == 2 || g == 4 || g == 8);
 }
 
 int decode_ctas_per_sm(int g, int hkv, int ng) {
@@ -1981,6 +1995,8 @@ static DecodeArgs make_decode_args(const okv_cache_desc* d, const void* q, int B
   a.num_slots = d->num_seq_slots;
   a.mbps = d->max_blocks_per_seq;
   a.ng = kD / d->group;
+  // grouped layouts at G = 8: two CTAs per cost range, four query heads each
+  a.hsplit = (a.ng > 1 && a.g == 8) ? 2 : 1;
   return a;
 }
 
@@ -2009,13 +2025,15 @@ static okv_status launch_decode_tail(const DecodeArgs& a, int B, cudaStream_t s)
     switch (a.g) {
       case 1: st = launch_decode_heads<1, 2>(a, s, early); break;
       case 2: st = launch_decode_heads<2, 2>(a, s, early); break;
-      default: st = launch_decode_heads<4, 2>(a, s, early); break;
+      case 4: st = launch_decode_heads<4, 2>(a, s, early); break;
+      default: st = launch_decode_heads<4, 2, 2>(a, s, early); break;  // G = 8 as two halves
     }
   } else if (tc && a.ng == 4) {
     switch (a.g) {
       case 1: st = launch_decode_heads<1, 4>(a, s, early); break;
       case 2: st = launch_decode_heads<2, 4>(a, s, early); break;
-      default: st = launch_decode_heads<4, 4>(a, s, early); break;
+      case 4: st = launch_decode_heads<4, 4>(a, s, early); break;
+      default: st = launch_decode_heads<4, 4, 2>(a, s, early); break;  // G = 8 as two halves
     }
   } else if (tc) {
     switch (a.g) {
