@@ -1954,13 +1954,18 @@ static okv_status launch_decode_heads(const DecodeArgs& a, cudaStream_t s, bool 
 
 bool decode_uses_tensor_cores(int g, int hkv, int ng) {
   const bool hkv_ok = hkv == 1 || hkv == 2 || hkv == 4 || hkv == 8;
-  if (ng == 1) return hkv_ok && (g == 1 || g == 2 || g == 4 || g == 8);
-  return hkv_ok && (ng == 2 || ng == 4) && (g == 1 || g == 2 || g == 4 || g == 8);
+  return hkv_ok && (ng == 1 || ng == 2 || ng == 4) && (g == 1 || g == 2 || g == 4 || g == 8 || g == 16);
 }
 
-int decode_ctas_per_sm(int g, int hkv, int ng) {
-  if (decode_uses_tensor_cores(g, hkv, ng)) return g <= 4 ? 2 : 1;
-  return 4;
+// split-K cost ranges for a device of `sms` SMs: two CTAs per SM for the
+// tensor-core kernel (one at G = 8 with one group per vector, whose CTA holds
+// both n-tiles), with a range split over two (G = 8 grouped) or four (G = 16)
+// CTAs of four query heads; four CTAs per SM for the CUDA-core kernel
+int decode_ranges(int sms, int g, int hkv, int ng) {
+  if (!decode_uses_tensor_cores(g, hkv, ng)) return 4 * sms;
+  if (g <= 4) return 2 * sms;
+  if (g == 8) return sms;
+  return sms / 2;  // g = 16
 }
 
 static DecodeArgs make_decode_args(const okv_cache_desc* d, const void* q, int B, const int32_t* seq_slot,
@@ -1995,8 +2000,9 @@ static DecodeArgs make_decode_args(const okv_cache_desc* d, const void* q, int B
   a.num_slots = d->num_seq_slots;
   a.mbps = d->max_blocks_per_seq;
   a.ng = kD / d->group;
-  // grouped layouts at G = 8: two CTAs per cost range, four query heads each
-  a.hsplit = (a.ng > 1 && a.g == 8) ? 2 : 1;
+  // grouped layouts at G = 8, and every layout at G = 16: two or four CTAs per
+  // cost range, four query heads each
+  a.hsplit = a.g == 16 ? 4 : (a.ng > 1 && a.g == 8) ? 2 : 1;
   return a;
 }
 
@@ -2026,21 +2032,24 @@ static okv_status launch_decode_tail(const DecodeArgs& a, int B, cudaStream_t s)
       case 1: st = launch_decode_heads<1, 2>(a, s, early); break;
       case 2: st = launch_decode_heads<2, 2>(a, s, early); break;
       case 4: st = launch_decode_heads<4, 2>(a, s, early); break;
-      default: st = launch_decode_heads<4, 2, 2>(a, s, early); break;  // G = 8 as two halves
+      case 8: st = launch_decode_heads<4, 2, 2>(a, s, early); break;  // G = 8 as two halves
+      default: st = launch_decode_heads<4, 2, 4>(a, s, early); break;  // G = 16 as four quarters
     }
   } else if (tc && a.ng == 4) {
     switch (a.g) {
       case 1: st = launch_decode_heads<1, 4>(a, s, early); break;
       case 2: st = launch_decode_heads<2, 4>(a, s, early); break;
       case 4: st = launch_decode_heads<4, 4>(a, s, early); break;
-      default: st = launch_decode_heads<4, 4, 2>(a, s, early); break;  // G = 8 as two halves
+      case 8: st = launch_decode_heads<4, 4, 2>(a, s, early); break;  // G = 8 as two halves
+      default: st = launch_decode_heads<4, 4, 4>(a, s, early); break;  // G = 16 as four quarters
     }
   } else if (tc) {
     switch (a.g) {
       case 1: st = launch_decode_heads<1>(a, s, early); break;
       case 2: st = launch_decode_heads<2>(a, s, early); break;
       case 4: st = launch_decode_heads<4>(a, s, early); break;
-      default: st = launch_decode_heads<8>(a, s, early); break;
+      case 8: st = launch_decode_heads<8>(a, s, early); break;
+      default: st = launch_decode_heads<4, 1, 4>(a, s, early); break;  // G = 16 as four quarters
     }
   } else {
     switch (a.g) {

@@ -99,7 +99,7 @@ DecodePlan make_decode_plan(int batch, int hq, int hkv, int ng) {
   p.hkv = hkv;
   p.g = hq / hkv;
   const int sms = device_sm_count();
-  p.num_ctas = (sms > 0 ? sms : 148) * decode_ctas_per_sm(p.g, hkv, ng);
+  p.num_ctas = decode_ranges(sms > 0 ? sms : 148, p.g, hkv, ng);
   if (p.num_ctas > 1024) p.num_ctas = 1024;  // the combine caches one weight per split
   p.num_units = batch * hkv;
   size_t off = 0;

@@ -44,7 +44,7 @@ constexpr int kWinCost = 8;       // cost of an entry's window in block units (a
 constexpr int kFusedAppendMaxTokens = 127;  // okv_decode_step fuses appends this short with the query rotation
 // split-K kernel choice and residency (decode.cu)
 bool decode_uses_tensor_cores(int g, int hkv, int ng);
-int decode_ctas_per_sm(int g, int hkv, int ng);
+int decode_ranges(int sms, int g, int hkv, int ng);
 
 DecodePlan make_decode_plan(int batch, int hq, int hkv, int ng);
 

@@ -18,8 +18,8 @@ oracle's per-group quantiser and decode, on the same seeded inputs:
   100,000 tokens;
 * the tensor-core split-K kernel's grouped layouts (per-group score MMAs and
   value m-tiles) at every head grouping it takes (G = 1, 2, 4 on 8, 2 or 1 KV
-  heads, so that one warp or several serve a head; G = 8 as two CTAs per
-  range of four query heads each), with and without sinks,
+  heads, so that one warp or several serve a head; G = 8 and 16 as two and
+  four CTAs per range of four query heads each), with and without sinks,
   over lengths that end inside a block, at a block edge, inside and past the
   fp16 window;
 * a peaked case: one INT2 key 10 nats above a flat 30,000-token context, at
@@ -253,6 +253,7 @@ def _fill_groups_sinks(seed, hq, hkv, lens, group, nsink, plant=None):
     (4, 1, 48, [49, 176, 177, 2500]),                    # G = 4, 8 warps per KV head
     (64, 8, 0, [1, 17, 129, 300, 4000]),                 # G = 8: two CTAs per range, four heads each
     (16, 2, 16, [16, 33, 145, 2000]),                    # G = 8 on 2 KV heads (merged), sinks
+    (32, 2, 0, [5, 129, 1500]),                          # G = 16: four CTAs per range
 ])
 def test_grouped_decode_tensor_core_shapes(group, hq, hkv, nsink, lens):
     okv = _okv()
