@@ -40,7 +40,7 @@ struct DecodePlan {
 };
 constexpr int kPartStride = 132;  // o'[128], m, l, 2 spare
 constexpr int kQsStride = 8;      // floats per query head in the query-scale workspace
-constexpr int kWinCost = 8;       // cost of an entry's window in block units (all heads)
+constexpr int kWinCost = 4;       // cost of one 16-row fp16 chunk in block units (all heads)
 constexpr int kFusedAppendMaxTokens = 127;  // okv_decode_step fuses appends this short with the query rotation
 // split-K kernel choice and residency (decode.cu)
 bool decode_uses_tensor_cores(int g, int hkv, int ng);
