@@ -1920,24 +1920,6 @@ static okv_status launch_decode_simt(const DecodeArgs& a, cudaStream_t s) {
   return check_launch("decode");
 }
 
-// Launch with programmatic stream serialisation when `early` is set: the
-// kernel may begin while its predecessor on the stream is still running (it
-// calls grid_dep_wait() before reading the predecessor's outputs).
-template <typename... Args>
-static cudaError_t launch_pdl(void (*kernel)(Args...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
-                              bool early, Args... args) {
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = grid;
-  cfg.blockDim = block;
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = early ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, kernel, args...);
-}
 
 template <int G, int NGQ = 1, int HS = 1>
 static okv_status launch_decode_heads(const DecodeArgs& a, cudaStream_t s, bool early) {

@@ -21,6 +21,24 @@ int device_sm_count();
 // attribute belongs to the device's context, so a context reset would need
 // it set again: the library assumes contexts live as long as the process.
 cudaError_t set_smem_limit_once(const void* kernel, int bytes, std::atomic<uint32_t>& done);
+// Launch with programmatic stream serialisation when `early` is set: the
+// kernel may begin while its predecessor on the stream is still running (it
+// calls grid_dep_wait() before reading the predecessor's outputs).
+template <typename... Args>
+static cudaError_t launch_pdl(void (*kernel)(Args...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                              bool early, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = early ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
 // events set by okv_time_next_decode_kernel (consumed by the next decode launch)
 void take_decode_events(cudaEvent_t* start, cudaEvent_t* stop);
 

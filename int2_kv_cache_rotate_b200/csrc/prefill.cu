@@ -361,6 +361,7 @@ __global__ void __launch_bounds__(kUpThreads, 1) prefill_umma_kernel(PrefillArgs
   uint32_t qrow[64];  // this thread's half of its q~ row (fp16 pairs), until it is in TMEM
   const int quarter = warp & 3, hcol = (warp >> 2) & 1;  // softmax: lane quarter, column half
   const int rowc = 32 * quarter + lane;                    // softmax: row in the tile (TMEM lane)
+  grid_dep_launch();  // the un-rotation may start staging U_V
   if (warp < kUpSmxWarps) {
     const int r = row0 + rowc;
     rok = r < nrows;
@@ -1027,6 +1028,7 @@ __global__ void __launch_bounds__(256) prefill_unrotate_kernel(PrefillArgs a) {
       *reinterpret_cast<float4*>(ut + (i0 + 3) * kD + 4 * l) = make_float4(u[0].w, u[1].w, u[2].w, u[3].w);
     }
   }
+  grid_dep_wait();  // the attention's outputs are read from here on
   // this warp's 8 rows: x = H-butterfly of the un-permuted o' / l, into xs.
   // All 8 rows' loads go out before the first butterfly.
   const int r = rev5(lane);
@@ -1146,7 +1148,12 @@ okv_status launch_prefill(const okv_cache_desc* d, const void* q, int T, int slo
   }
   st = check_launch("prefill attention");
   if (st != OKV_OK) return st;
-  prefill_unrotate_kernel<<<rt_grid, 256, kRtSmem, s>>>(a);
+  // The un-rotation may start (programmatic launch) while the attention's last
+  // CTAs run: it stages U_V, then waits for the attention's outputs.  Starting
+  // the attention early behind the query rotation in the same way measured
+  // slower with 64-channel groups (3.31 against 3.10 ms) and is not done.
+  const cudaError_t e3 = launch_pdl(prefill_unrotate_kernel, rt_grid, dim3(256), kRtSmem, s, true, a);
+  if (e3 != cudaSuccess) return fail(OKV_ERR_CUDA, "prefill un-rotation launch: %s", cudaGetErrorString(e3));
   return check_launch("prefill un-rotation");
 }
 
