@@ -894,8 +894,7 @@ def run_ours(args):
                          "frac": round(achieved / peak, 4), "peak_source": peak_src,
                          "traffic": (tr["bytes_per_launch"] if tr else None),
                          "kernel": ("split-K INT2 decode attention" if args.group == 128 else
-                                    "split-K INT2 decode attention, per-group scales" +
-                                    (" (CUDA-core kernel)" if w.wl.hq // w.wl.hkv > 8 else "")),
+                                    "split-K INT2 decode attention, per-group scales"),
                          "int2_bytes_per_token_head": int2_bytes_per_token_head(args.group),
                          "algorithmic_bytes_per_launch": int(alg)},
             "append_prefill": append_rate,
